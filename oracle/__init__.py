@@ -1,0 +1,237 @@
+"""CPU oracle for the CSA / HCA hot path (fp64, plain definitions).
+
+TEST INFRASTRUCTURE ONLY: the test suite, the smoke check and the benchmark's
+CPU-baseline leg are the only callers. The CUDA library never imports this
+module and this module never imports the CUDA library; the two share no code.
+
+The arithmetic lives in ``csa_oracle.c`` (plain C, fp64, OpenMP over
+independent outputs). This file only builds that library with gcc and moves
+numpy arrays in and out. Every function returns float64 arrays (int32 for
+indices); bf16 storage rounding is explicit (:func:`bf16_round`).
+
+Which page passage each function follows is stated beside it in
+``csa_oracle.c``; the readings taken where the pages are silent are listed at
+the top of that file.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "csa_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_D = ctypes.POINTER(ctypes.c_double)
+_I32 = ctypes.POINTER(ctypes.c_int32)
+
+
+def build(force: bool = False) -> str:
+    """Compile ``csa_oracle.c`` into ``_build/liboracle.so`` (gcc, -O2, OpenMP).
+
+    No fast-math: the oracle needs IEEE exp/log and the written summation order.
+    """
+    os.makedirs(_BUILD, exist_ok=True)
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-std=c11", "-Wall", "-shared", "-fPIC",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(_LIB_OVERRIDE or build())
+            i64, i32, dbl = ctypes.c_int64, ctypes.c_int, ctypes.c_double
+            lib.orc_bf16_round.restype = dbl
+            lib.orc_bf16_round.argtypes = [dbl]
+            lib.orc_bf16_round_array.argtypes = [_D, i64, _D]
+            lib.orc_project.argtypes = [_D, _D, i64, i64, i64, _D]
+            lib.orc_csa_compress.argtypes = [_D, _D, _D, i64, i32, i32, _D, _D]
+            lib.orc_hca_compress.argtypes = [_D, _D, i64, i32, i32, _D, _D]
+            lib.orc_index_scores.argtypes = [_D, _D, _D, _I32, _I32, i32, i32, i32, i64, i32, _D]
+            lib.orc_topk.argtypes = [_D, _I32, i32, i64, i32, _I32]
+            lib.orc_sparse_mqa.argtypes = [_D, _D, _I32, _I32, i32, i32, i32, i64, i32, dbl, _D, _D, _D]
+            lib.orc_dense_mqa.argtypes = [_D, _D, _I32, _I32, i32, i32, i32, i64, i32, dbl, _D, _D, _D]
+            lib.orc_num_threads.restype = i32
+            _lib = lib
+    return _lib
+
+
+# Test hook: the mutation tests load a build of a deliberately broken copy
+# of csa_oracle.c through this variable.
+_LIB_OVERRIDE = os.environ.get("CSA_ORACLE_LIB") or None
+
+
+def _f64(a) -> np.ndarray:
+    """Any array-like (numpy or a CPU torch tensor, bf16 included) -> C-contiguous float64."""
+    if hasattr(a, "detach"):  # torch tensor: go through float32, which holds bf16 exactly
+        a = a.detach().cpu()
+        if str(a.dtype) in ("torch.bfloat16", "torch.float16"):
+            a = a.float()
+        a = a.numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _i32(a) -> np.ndarray:
+    if hasattr(a, "detach"):
+        a = a.detach().cpu().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+def _p(a: np.ndarray | None):
+    if a is None:
+        return None
+    if a.dtype == np.float64:
+        return a.ctypes.data_as(_D)
+    return a.ctypes.data_as(_I32)
+
+
+def num_threads() -> int:
+    return int(_load().orc_num_threads())
+
+
+def bf16_round(x) -> np.ndarray:
+    """Nearest bf16 value (ties to even) of each element, returned as float64."""
+    x = _f64(x)
+    y = np.empty_like(x)
+    _load().orc_bf16_round_array(_p(x), x.size, _p(y))
+    return y
+
+
+def project(X, W) -> np.ndarray:
+    """P = X @ W^T with X [n, d] and W [M, d] (one row per output feature)."""
+    X, W = _f64(X), _f64(W)
+    n, d = X.shape
+    M = W.shape[0]
+    assert W.shape[1] == d
+    P = np.empty((n, M))
+    _load().orc_project(_p(X), _p(W), n, d, M, _p(P))
+    return P
+
+
+def csa_compress(proj, bias, m: int, left=None, return_weights: bool = False):
+    """Overlapping CSA compression. proj [n, 4c] = Ca|Cb|Za|Zb, bias [2m, c],
+    left [m, 4c] or None (sequence start). Returns out [n/m, c] (and the softmax
+    weights [n/m, 2m, c] when asked)."""
+    proj, bias = _f64(proj), _f64(bias)
+    n, c4 = proj.shape
+    c = c4 // 4
+    assert c4 == 4 * c and n % m == 0 and bias.shape == (2 * m, c)
+    lp = None
+    if left is not None:
+        lp = _f64(left)
+        assert lp.shape == (m, 4 * c)
+    out = np.empty((n // m, c))
+    w = np.empty((n // m, 2 * m, c)) if return_weights else None
+    _load().orc_csa_compress(_p(proj), _p(lp), _p(bias), n, c, m, _p(out), _p(w))
+    return (out, w) if return_weights else out
+
+
+def hca_compress(proj, bias, mp: int, return_weights: bool = False):
+    """Non-overlapping HCA compression. proj [n, 2c] = C|Z, bias [mp, c]."""
+    proj, bias = _f64(proj), _f64(bias)
+    n, c2 = proj.shape
+    c = c2 // 2
+    assert c2 == 2 * c and n % mp == 0 and bias.shape == (mp, c)
+    out = np.empty((n // mp, c))
+    w = np.empty((n // mp, mp, c)) if return_weights else None
+    _load().orc_hca_compress(_p(proj), _p(bias), n, c, mp, _p(out), _p(w))
+    return (out, w) if return_weights else out
+
+
+def index_scores(qI, w, K, pos, m: int, seq=None) -> np.ndarray:
+    """Indexer scores [nq, Nmax]; -inf where the entry is not visible.
+    qI [nq, HI, cI], w [nq, HI], K [B, Nmax, cI] (or [Nmax, cI]), pos [nq]."""
+    qI, w, K = _f64(qI), _f64(w), _f64(K)
+    if K.ndim == 2:
+        K = K[None]
+    nq, HI, cI = qI.shape
+    B, Nmax, _ = K.shape
+    pos = _i32(pos)
+    seq = _i32(np.zeros(nq) if seq is None else seq)
+    assert int(seq.max(initial=0)) < B
+    S = np.empty((nq, Nmax))
+    _load().orc_index_scores(_p(qI), _p(w), _p(K), _p(pos), _p(seq), nq, HI, cI, Nmax, m, _p(S))
+    return S
+
+
+def topk(scores, valid, k: int) -> np.ndarray:
+    """Top-k column indices per row among the first valid[t] columns, ordered
+    (score desc, index asc), padded with -1."""
+    S = _f64(scores)
+    nq, ncols = S.shape
+    valid = _i32(valid)
+    idx = np.empty((nq, k), dtype=np.int32)
+    _load().orc_topk(_p(S), _p(valid), nq, ncols, k, _p(idx))
+    return idx
+
+
+def sparse_mqa(q, KV, idx, scale: float, sink=None, seq=None):
+    """Shared-KV MQA over the selected entries. q [nq, H, c], KV [B, Nmax, c]
+    (or [Nmax, c]), idx [nq, k] (-1 = no entry). Returns (out [nq, H, c], lse [nq, H])."""
+    q, KV = _f64(q), _f64(KV)
+    if KV.ndim == 2:
+        KV = KV[None]
+    nq, H, c = q.shape
+    B, Nmax, _ = KV.shape
+    idx = _i32(idx)
+    k = idx.shape[1]
+    seq = _i32(np.zeros(nq) if seq is None else seq)
+    sk = None if sink is None else _f64(sink)
+    out = np.empty((nq, H, c))
+    lse = np.empty((nq, H))
+    _load().orc_sparse_mqa(_p(q), _p(KV), _p(idx), _p(seq), nq, H, c, Nmax, k, float(scale),
+                           _p(sk), _p(out), _p(lse))
+    return out, lse
+
+
+def dense_mqa(q, KV, pos, mp: int, scale: float, sink=None, seq=None):
+    """Shared-KV MQA over every visible entry s < floor(pos/mp)."""
+    q, KV = _f64(q), _f64(KV)
+    if KV.ndim == 2:
+        KV = KV[None]
+    nq, H, c = q.shape
+    B, Nmax, _ = KV.shape
+    pos = _i32(pos)
+    seq = _i32(np.zeros(nq) if seq is None else seq)
+    sk = None if sink is None else _f64(sink)
+    out = np.empty((nq, H, c))
+    lse = np.empty((nq, H))
+    _load().orc_dense_mqa(_p(q), _p(KV), _p(pos), _p(seq), nq, H, c, Nmax, mp, float(scale),
+                          _p(sk), _p(out), _p(lse))
+    return out, lse
+
+
+# ---------------------------------------------------------------------------
+# Chained steps (each one a composition of the definitions above, in the
+# order the method applies them)
+# ---------------------------------------------------------------------------
+
+def csa_compress_from_hidden(X, W, bias, m: int, X_left=None) -> np.ndarray:
+    """Projections then overlapping compression; W [4c, d] packs the a-KV,
+    b-KV, a-weight and b-weight maps (one row per output feature)."""
+    proj = project(X, W)
+    left = None if X_left is None else project(X_left, W)
+    return csa_compress(proj, bias, m, left=left)
+
+
+def hca_compress_from_hidden(X, W, bias, mp: int) -> np.ndarray:
+    return hca_compress(project(X, W), bias, mp)
+
+
+def index_topk(qI, w, K, pos, m: int, k: int, seq=None):
+    """Indexer scores, then top-k over the visible entries. Returns (idx, scores)."""
+    S = index_scores(qI, w, K, pos, m, seq=seq)
+    valid = np.minimum(_i32(pos) // m, S.shape[1]).astype(np.int32)
+    return topk(S, valid, k), S

@@ -1,0 +1,61 @@
+"""Each plausible mistake in the oracle must fail at least one pin.
+
+A mutation is planted in a temporary copy of oracle/csa_oracle.c (CPU only),
+built with gcc, loaded in place of the real oracle, and the pin suite is run
+against it; the test passes when some pin fails. The real oracle is restored
+afterwards.
+"""
+import os
+import shutil
+import subprocess
+import tempfile
+
+import pytest
+
+import oracle
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "csa_oracle.c")
+
+# (name, exact text in csa_oracle.c, replacement)
+MUTATIONS = [
+    ("b-window from block i instead of i-1", "int64_t tb = m * (i - 1) + r;", "int64_t tb = m * i + r;"),
+    ("bias rows of the b-window swapped with the a-window",
+     "bias[(m + r) * c + j]; /* Z^b + B^b */", "bias[r * c + j]; /* Z^b + B^b */"),
+    ("Z^a used for the b-window logits", "rb[3 * c + j] + bias", "rb[2 * c + j] + bias"),
+    ("C^a used for the b-window values", "acc += s * rb[1 * c + j];", "acc += s * rb[0 * c + j];"),
+    ("block 0 b-window zero-padded instead of absent",
+     "int has_b = (tb >= 0) || (left != NULL);", "int has_b = 1; if (tb < 0 && !left) { present[m + r] = 1; logit[m + r] = bias[(m + r) * c + j]; continue; }"),
+    ("HCA bias ignored", "+ bias[r * c + j];   /* Z + B' */", ";   /* Z + B' */"),
+    ("HCA values taken from Z", "acc += s * proj[(i * mp + r) * 2 * c + j];",
+     "acc += s * proj[(i * mp + r) * 2 * c + c + j];"),
+    ("HCA window shifted by one token", "logit[r] = proj[(i * mp + r) * 2 * c + c + j]",
+     "logit[r] = proj[((i * mp + r + 1) % n) * 2 * c + c + j]"),
+    ("indexer without ReLU", "(dot > 0.0 ? dot : 0.0)", "dot"),
+    ("indexer sees its own block", "if (s >= vis) {", "if (s > vis) {"),
+    ("indexer weight of head 0 for all heads", "acc += w[(int64_t)t * HI + h] *", "acc += w[(int64_t)t * HI] *"),
+    ("top-k ties to the higher index", "return a < b;", "return a > b;"),
+    ("top-k ascending", "return row[a] > row[b];", "return row[a] < row[b];"),
+    ("MQA without scale", "z[i] = scale * dot;", "z[i] = dot;"),
+    ("sink added to the numerator set twice", "if (sink) den += exp(sink[h] - mx);",
+     "if (sink) den += 2.0 * exp(sink[h] - mx);"),
+    ("dense MQA sees its own block", "int64_t vis = pos[t] / mp;", "int64_t vis = pos[t] / mp + 1;"),
+    ("bf16 rounding truncates", "double r = ldexp(round_half_even(ldexp(a, -q)), q);",
+     "double r = ldexp(floor(ldexp(a, -q)), q);"),
+    ("projection uses W transposed index", "X[t * d + k] * W[o * d + k]", "X[t * d + k] * W[k * M + o]"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_pins_catch_mutation(name, old, new, tmp_path):
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not unique/present: {old!r}"
+    mutated = tmp_path / "mut.c"
+    mutated.write_text(src.replace(old, new))
+    lib = tmp_path / "libmut.so"
+    subprocess.check_call(["gcc", "-O1", "-fopenmp", "-std=c11", "-shared", "-fPIC", "-o", str(lib),
+                           str(mutated), "-lm"])
+    pins = os.path.join(os.path.dirname(__file__), "test_oracle_pins.py")
+    env = dict(os.environ, CSA_ORACLE_LIB=str(lib))
+    r = subprocess.run(["python", "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider", pins],
+                       env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"no pin failed for mutation '{name}'\n{r.stdout[-2000:]}"

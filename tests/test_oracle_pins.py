@@ -1,0 +1,434 @@
+"""Pins for the CPU oracle: checks against facts fixed by the pages and by
+mathematics, never against the oracle itself or the CUDA path.
+
+Kinds of pin used here:
+  * hand-worked examples in tests/golden/ (values chosen so every softmax
+    weight is a simple fraction, derivation written in the fixture);
+  * closed forms (uniform weights give the window mean, m'=1 gives identity);
+  * invariants (weights sum to 1, causality, chunked composition);
+  * reductions to a library routine (numpy matmul, torch's attention);
+  * brute force over every k-subset for top-k.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _num(v):
+    """Parse the fixture notation: numbers, 'ln3', 'ln3+0.5', '6/7', '-inf'."""
+    if v is None:
+        return None
+    if isinstance(v, (int, float)):
+        return float(v)
+    s = v.strip()
+    if s == "-inf":
+        return -math.inf
+    if "/" in s:
+        a, b = s.split("/")
+        return float(a) / float(b)
+    total = 0.0
+    for sign, term in _terms(s):
+        total += sign * (math.log(float(term[2:])) if term.startswith("ln") else float(term))
+    return total
+
+
+def _terms(s):
+    out, sign, cur = [], 1.0, ""
+    for ch in s:
+        if ch in "+-" and cur:
+            out.append((sign, cur))
+            sign, cur = (1.0 if ch == "+" else -1.0), ""
+        elif ch == "-" and not cur:
+            sign = -sign
+        else:
+            cur += ch
+    out.append((sign, cur))
+    return out
+
+
+def _load(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+rng = np.random.default_rng(12345)
+
+
+# --------------------------------------------------------------------------
+# bf16 storage rounding
+# --------------------------------------------------------------------------
+
+def test_bf16_round_matches_torch_on_fp32_values():
+    x = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32),
+        (rng.standard_normal(2000) * 1e-39).astype(np.float32),  # fp32 subnormals
+        (rng.standard_normal(2000) * 1e38).astype(np.float32),
+        np.array([0.0, -0.0, 1.0, -1.0, 3.3895314e38, 3.4e38], dtype=np.float32),
+    ])
+    # exact ties: 1 + 2^-8 lies halfway between 1 and 1 + 2^-7 -> even (1.0)
+    ties = np.array([1 + 2**-8, 1 + 3 * 2**-8, -(1 + 2**-8), 2**-130 + 2**-134], dtype=np.float32)
+    x = np.concatenate([x, ties])
+    want = torch.from_numpy(x).to(torch.bfloat16).float().numpy().astype(np.float64)
+    got = oracle.bf16_round(x.astype(np.float64))
+    np.testing.assert_array_equal(got, want)
+
+
+def test_bf16_round_ties_to_even_by_hand():
+    assert oracle.bf16_round(np.array([1 + 2**-8]))[0] == 1.0
+    assert oracle.bf16_round(np.array([1 + 3 * 2**-8]))[0] == 1 + 2**-6
+    assert oracle.bf16_round(np.array([1 + 2**-8 + 2**-20]))[0] == 1 + 2**-7
+
+
+# --------------------------------------------------------------------------
+# a1 projections
+# --------------------------------------------------------------------------
+
+def test_project_matches_numpy_matmul():
+    X = rng.standard_normal((37, 53))
+    W = rng.standard_normal((19, 53))
+    np.testing.assert_allclose(oracle.project(X, W), X @ W.T, rtol=1e-13, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# a2 CSA compressor
+# --------------------------------------------------------------------------
+
+def _csa_fixture():
+    g = _load("csa_compress_m2.json")
+    cols = [[_num(v) for v in g[k]] for k in ("Ca", "Cb", "Za", "Zb")]
+    proj = np.array(cols).T  # [n, 4] with c = 1
+    bias = np.array([[_num(v) for v in r] for r in g["bias"]])
+    return g, proj, bias
+
+
+def test_csa_compress_handworked():
+    g, proj, bias = _csa_fixture()
+    out = oracle.csa_compress(proj, bias, g["m"])
+    np.testing.assert_allclose(out[:, 0], g["expected"], rtol=0, atol=1e-12)
+
+
+def test_csa_compress_handworked_with_left_context():
+    g, proj, bias = _csa_fixture()
+    m = g["m"]
+    out = oracle.csa_compress(proj[m:], bias, m, left=proj[:m])
+    np.testing.assert_allclose(out[:, 0], g["expected_second_block_alone_with_left_context"],
+                               rtol=0, atol=1e-12)
+
+
+def test_csa_uniform_weights_give_window_mean():
+    # Z = const and B = 0 make every softmax weight equal; with Ca = Cb = C the
+    # compressed entry is the plain mean of C over the window: 2m tokens, or
+    # m tokens for block 0 (no b-window at the start of a sequence).
+    m, c, n = 4, 6, 40
+    C = rng.standard_normal((n, c))
+    Z = np.full((n, c), 0.37)
+    proj = np.concatenate([C, C, Z, Z], axis=1)
+    out = oracle.csa_compress(proj, np.zeros((2 * m, c)), m)
+    want = np.stack([C[0:m].mean(0)] + [C[m * (i - 1): m * (i + 1)].mean(0) for i in range(1, n // m)])
+    np.testing.assert_allclose(out, want, rtol=1e-13, atol=1e-13)
+
+
+def test_csa_weights_sum_to_one_and_block0_has_no_b_window():
+    m, c, n = 4, 16, 64
+    proj = rng.standard_normal((n, 4 * c)) * 3
+    bias = rng.standard_normal((2 * m, c))
+    out, w = oracle.csa_compress(proj, bias, m, return_weights=True)
+    np.testing.assert_allclose(w.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+    assert np.all(w[0, m:, :] == 0.0)
+    assert np.all(w[1:, m:, :] > 0.0)
+    # with a left context the first block does have a b-window
+    _, w2 = oracle.csa_compress(proj[m:], bias, m, left=proj[:m], return_weights=True)
+    assert np.all(w2[0, m:, :] > 0.0)
+
+
+def test_csa_with_b_logits_at_minus_inf_is_non_overlapping():
+    # Z^b -> -inf removes the b-window: each entry is then the softmax(Za + Ba)
+    # average of its own m tokens, which is the HCA form with m' = m.
+    m, c, n = 4, 8, 32
+    Ca, Cb, Za = (rng.standard_normal((n, c)) for _ in range(3))
+    Zb = np.full((n, c), -1e300)
+    bias = rng.standard_normal((2 * m, c))
+    out = oracle.csa_compress(np.concatenate([Ca, Cb, Za, Zb], 1), bias, m)
+    want = np.empty((n // m, c))
+    for i in range(n // m):
+        lg = Za[m * i: m * i + m] + bias[:m]
+        e = np.exp(lg - lg.max(0))
+        want[i] = (e / e.sum(0) * Ca[m * i: m * i + m]).sum(0)
+    np.testing.assert_allclose(out, want, rtol=1e-12, atol=1e-13)
+    hca = oracle.hca_compress(np.concatenate([Ca, Za], 1), bias[:m], m)
+    np.testing.assert_allclose(out, hca, rtol=1e-12, atol=1e-13)
+
+
+def test_csa_chunked_composition():
+    # compress(0..n) == compress(0..a) ++ compress(a..n with the m rows before a)
+    m, c, n = 4, 8, 96
+    proj = rng.standard_normal((n, 4 * c))
+    bias = rng.standard_normal((2 * m, c))
+    full = oracle.csa_compress(proj, bias, m)
+    for a in (4, 28, 60, 92):
+        head = oracle.csa_compress(proj[:a], bias, m)
+        tail = oracle.csa_compress(proj[a:], bias, m, left=proj[a - m: a])
+        np.testing.assert_array_equal(np.concatenate([head, tail]), full)
+
+
+def test_csa_from_hidden_is_projection_then_compression():
+    m, c, d, n = 4, 4, 24, 16
+    X = rng.standard_normal((n, d))
+    W = rng.standard_normal((4 * c, d))
+    bias = rng.standard_normal((2 * m, c))
+    got = oracle.csa_compress_from_hidden(X, W, bias, m)
+    np.testing.assert_allclose(got, oracle.csa_compress(X @ W.T, bias, m), rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# a3 HCA compressor
+# --------------------------------------------------------------------------
+
+def test_hca_compress_handworked():
+    g = _load("hca_compress_mp2.json")
+    C = np.array([[_num(v) for v in r] for r in g["C"]])
+    Z = np.array([[_num(v) for v in r] for r in g["Z"]])
+    bias = np.array(g["bias"], dtype=float)
+    out = oracle.hca_compress(np.concatenate([C, Z], 1), bias, g["mp"])
+    np.testing.assert_allclose(out, np.array(g["expected"]), rtol=0, atol=1e-12)
+
+
+def test_hca_mp1_is_identity():
+    n, c = 20, 7
+    C = rng.standard_normal((n, c))
+    Z = rng.standard_normal((n, c))
+    out = oracle.hca_compress(np.concatenate([C, Z], 1), np.zeros((1, c)), 1)
+    np.testing.assert_array_equal(out, C)
+
+
+def test_hca_uniform_weights_give_block_mean_and_weights_sum_to_one():
+    mp, c, n = 128, 4, 512
+    C = rng.standard_normal((n, c))
+    out = oracle.hca_compress(np.concatenate([C, np.zeros((n, c))], 1), np.zeros((mp, c)), mp)
+    np.testing.assert_allclose(out, C.reshape(n // mp, mp, c).mean(1), rtol=1e-12, atol=1e-13)
+    proj = rng.standard_normal((n, 2 * c)) * 4
+    _, w = oracle.hca_compress(proj, rng.standard_normal((mp, c)), mp, return_weights=True)
+    np.testing.assert_allclose(w.sum(1), 1.0, atol=1e-12)
+
+
+def test_entry_counts_match_the_pages():
+    g = _load("entry_counts.json")
+    n = g["tokens"]
+    # the oracle emits n/m entries per sequence; use a proportionally small run
+    # to confirm the count rule, then apply it at the pages' size
+    assert oracle.csa_compress(np.zeros((64, 4)), np.zeros((8, 1)), 4).shape[0] == 64 // 4
+    assert oracle.hca_compress(np.zeros((256, 2)), np.zeros((128, 1)), 128).shape[0] == 256 // 128
+    assert n // g["m"] == g["expected_csa_entries"]
+    assert abs(n / g["mp"] - g["expected_hca_entries_approx"]) <= g["hca_tolerance_fraction"] * n / g["mp"]
+
+
+# --------------------------------------------------------------------------
+# a4 indexer + a5 top-k
+# --------------------------------------------------------------------------
+
+def _indexer_fixture():
+    g = _load("indexer_topk.json")
+    K = np.array(g["K"], dtype=float)
+    npos = len(g["pos"])
+    q = np.broadcast_to(np.array(g["q"], dtype=float), (npos, 2, 2)).copy()
+    w = np.broadcast_to(np.array(g["w"], dtype=float), (npos, 2)).copy()
+    return g, K, q, w
+
+
+def test_indexer_handworked():
+    g, K, q, w = _indexer_fixture()
+    S = oracle.index_scores(q, w, K, g["pos"], g["m"])
+    want = np.array([[_num(v) for v in r] for r in g["expected_scores"]])
+    np.testing.assert_array_equal(S, want)
+
+
+def test_topk_handworked():
+    g, K, q, w = _indexer_fixture()
+    idx, _ = oracle.index_topk(q, w, K, g["pos"], g["m"], g["k"])
+    np.testing.assert_array_equal(idx, np.array(g["expected_topk"]))
+
+
+def test_indexer_single_head_unit_weight_is_relu_dot():
+    nq, cI, N, m = 9, 32, 50, 4
+    q = rng.standard_normal((nq, 1, cI))
+    K = rng.standard_normal((N, cI))
+    pos = np.full(nq, N * m)
+    S = oracle.index_scores(q, np.ones((nq, 1)), K, pos, m)
+    np.testing.assert_allclose(S, np.maximum(q[:, 0, :] @ K.T, 0.0), rtol=1e-13, atol=1e-13)
+
+
+def test_indexer_is_linear_in_head_weights():
+    nq, H, cI, N, m = 5, 4, 16, 40, 4
+    q = rng.standard_normal((nq, H, cI))
+    K = rng.standard_normal((N, cI))
+    pos = np.full(nq, N * m)
+    w = rng.random((nq, H))
+    total = oracle.index_scores(q, w, K, pos, m)
+    parts = sum(oracle.index_scores(q, np.eye(H)[h][None].repeat(nq, 0), K, pos, m) * w[:, h:h + 1]
+                for h in range(H))
+    np.testing.assert_allclose(total, parts, rtol=1e-12, atol=1e-12)
+
+
+def test_indexer_causality():
+    # a query at position p must not depend on any entry s >= floor(p/m)
+    nq, H, cI, N, m = 12, 3, 8, 32, 4
+    q = rng.standard_normal((nq, H, cI))
+    w = rng.random((nq, H))
+    K = rng.standard_normal((N, cI))
+    pos = rng.integers(0, N * m, nq)
+    S1 = oracle.index_scores(q, w, K, pos, m)
+    for t in range(nq):
+        v = pos[t] // m
+        assert np.all(np.isinf(S1[t, v:])) and np.all(np.isfinite(S1[t, :v]))
+        K2 = K.copy()
+        K2[v:] = rng.standard_normal((N - v, cI)) * 100
+        S2 = oracle.index_scores(q[t:t + 1], w[t:t + 1], K2, pos[t:t + 1], m)
+        np.testing.assert_array_equal(S2[0], S1[t])
+    idx, _ = oracle.index_topk(q, w, K, pos, m, k=40)
+    for t in range(nq):
+        sel = idx[t][idx[t] >= 0]
+        assert np.all(sel < pos[t] // m)
+        assert len(sel) == min(40, pos[t] // m)
+
+
+def _brute_topk(row, v, k):
+    kk = min(k, v)
+    best, best_key = (), None
+    for sub in itertools.combinations(range(v), kk):
+        key = (sum(row[list(sub)]) if sub else 0.0, tuple(-s for s in sub))
+        if best_key is None or key > best_key:
+            best, best_key = sub, key
+    ordered = sorted(best, key=lambda s: (-row[s], s))
+    return ordered + [-1] * (k - kk)
+
+
+def test_topk_brute_force_with_ties():
+    # integer scores from a small range force many ties; the brute force takes
+    # the max-sum k-subset and, among equal sums, the lexicographically smallest
+    # index set, then orders it (score desc, index asc)
+    for trial in range(300):
+        V = int(rng.integers(0, 11))
+        ncols = V + int(rng.integers(0, 3))
+        k = int(rng.integers(1, 5))
+        row = rng.integers(-3, 4, ncols).astype(float)
+        got = oracle.topk(row[None], [V], k)[0]
+        assert list(got) == _brute_topk(row, V, k), (row, V, k)
+
+
+def test_topk_matches_library_sort():
+    S = rng.standard_normal((20, 3000))
+    valid = rng.integers(0, 3001, 20)
+    k = 512
+    idx = oracle.topk(S, valid, k)
+    for t in range(20):
+        v = valid[t]
+        order = np.lexsort((np.arange(v), -S[t, :v]))[:k]
+        want = np.full(k, -1)
+        want[: len(order)] = order
+        np.testing.assert_array_equal(idx[t], want)
+
+
+# --------------------------------------------------------------------------
+# a6 / a7 shared-KV MQA
+# --------------------------------------------------------------------------
+
+def test_mqa_handworked_with_sink():
+    g = _load("mqa_sink.json")
+    KV = np.array(g["KV"], dtype=float)
+    q = np.array([[[_num(v) for v in g["q"]]]])
+    for case in g["cases"]:
+        sink = None if case["sink"] is None else np.array([_num(case["sink"])])
+        out, lse = oracle.sparse_mqa(q, KV, np.array([case["idx"]]), 1.0, sink=sink)
+        np.testing.assert_allclose(out[0, 0], [_num(v) for v in case["out"]], rtol=0, atol=1e-14)
+        want_lse = _num(case["lse"])
+        if math.isinf(want_lse):
+            assert lse[0, 0] == want_lse
+        else:
+            assert abs(lse[0, 0] - want_lse) < 1e-14
+
+
+def test_mqa_single_entry_returns_that_entry():
+    H, c, N = 4, 32, 10
+    q = rng.standard_normal((3, H, c))
+    KV = rng.standard_normal((N, c))
+    idx = np.array([[7, -1, -1], [-1, 2, -1], [-1, -1, 0]])
+    out, _ = oracle.sparse_mqa(q, KV, idx, 0.125)
+    for t, s in enumerate((7, 2, 0)):
+        np.testing.assert_array_equal(out[t], np.broadcast_to(KV[s], (H, c)))
+
+
+def test_mqa_matches_torch_attention():
+    # shared-KV MQA over a set of entries is standard attention with one KV
+    # head and a boolean mask; torch's scaled_dot_product_attention in fp64
+    nq, H, c, N = 6, 4, 16, 30
+    q = rng.standard_normal((nq, H, c))
+    KV = rng.standard_normal((N, c))
+    idx = np.stack([rng.permutation(N)[:8] for _ in range(nq)]).astype(np.int32)
+    idx[0, 3:] = -1
+    scale = 1.0 / math.sqrt(c)
+    out, lse = oracle.sparse_mqa(q, KV, idx, scale)
+    mask = np.zeros((nq, N), dtype=bool)
+    for t in range(nq):
+        mask[t, idx[t][idx[t] >= 0]] = True
+    qt = torch.from_numpy(q).transpose(0, 1)[:, :, None, :]          # [H, nq, 1, c]
+    kt = torch.from_numpy(KV)[None, None].expand(H, nq, N, c)         # [H, nq, N, c]
+    mt = torch.from_numpy(mask)[None, :, None, :].expand(H, nq, 1, N)
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, kt, attn_mask=mt, scale=scale)
+    np.testing.assert_allclose(out, ref[:, :, 0, :].transpose(0, 1).numpy(), rtol=1e-12, atol=1e-12)
+    logits = torch.einsum("thc,nc->thn", torch.from_numpy(q), torch.from_numpy(KV)) * scale
+    logits = logits.masked_fill(~torch.from_numpy(mask)[:, None, :], -math.inf)
+    np.testing.assert_allclose(lse, torch.logsumexp(logits, -1).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_sparse_with_k_at_least_visible_equals_dense():
+    # with top-k >= the visible count CSA's selection keeps every visible entry,
+    # and sparse MQA equals dense MQA over all of them
+    nq, HI, cI, H, c, N, m = 8, 4, 16, 4, 32, 40, 4
+    qI = rng.standard_normal((nq, HI, cI))
+    w = rng.random((nq, HI))
+    K = rng.standard_normal((N, cI))
+    KV = rng.standard_normal((N, c))
+    q = rng.standard_normal((nq, H, c))
+    pos = rng.integers(0, N * m, nq)
+    idx, _ = oracle.index_topk(qI, w, K, pos, m, k=N)
+    sp, lse_s = oracle.sparse_mqa(q, KV, idx, 0.2)
+    de, lse_d = oracle.dense_mqa(q, KV, pos, m, 0.2)
+    np.testing.assert_allclose(sp, de, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse_s, lse_d, rtol=1e-12, atol=1e-12)
+
+
+def test_sink_scales_output_below_one():
+    # with a sink the attention weights sum to D / (D + e^{z'}) < 1:
+    # out_sink = out * e^{lse} / (e^{lse} + e^{z'}),  lse_sink = log(e^{lse} + e^{z'})
+    nq, H, c, N = 4, 3, 16, 12
+    q = rng.standard_normal((nq, H, c))
+    KV = rng.standard_normal((N, c))
+    idx = np.tile(np.arange(N, dtype=np.int32), (nq, 1))
+    sink = rng.standard_normal(H)
+    o0, l0 = oracle.sparse_mqa(q, KV, idx, 0.3)
+    o1, l1 = oracle.sparse_mqa(q, KV, idx, 0.3, sink=sink)
+    frac = np.exp(l0) / (np.exp(l0) + np.exp(sink)[None])
+    assert np.all(frac < 1.0)
+    np.testing.assert_allclose(o1, o0 * frac[..., None], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(l1, np.logaddexp(l0, sink[None]), rtol=1e-12, atol=1e-12)
+
+
+def test_dense_mqa_causality_and_empty():
+    H, c, N, mp = 2, 8, 6, 128
+    q = rng.standard_normal((3, H, c))
+    KV = rng.standard_normal((N, c))
+    pos = np.array([0, 127, 128 * 3 + 5])
+    out, lse = oracle.dense_mqa(q, KV, pos, mp, 0.5)
+    assert np.all(out[0] == 0) and np.all(np.isneginf(lse[0]))
+    assert np.all(out[1] == 0) and np.all(np.isneginf(lse[1]))
+    want, _ = oracle.sparse_mqa(q[2:], KV, np.array([[0, 1, 2]]), 0.5)
+    np.testing.assert_allclose(out[2], want[0], rtol=1e-13, atol=1e-14)
