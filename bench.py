@@ -1,0 +1,629 @@
+#!/usr/bin/env python
+"""Throughput benchmark of the CSA / HCA hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Default workload: CSA decode shaped like V4-Flash (64 concurrent queries, each
+against its own compressed cache of a 64K..128K-token context: up to 32768
+entries of dim 512, indexer keys 64 heads x 128, top-k 512, 64 query heads).
+A step is one pass of the decode hot path over the batch: lightning indexer,
+top-k, sparse shared-KV MQA (the csa_decode entry point). Caches and queries
+are resident in HBM before timing; the L2 is flushed (256 MiB write) before
+every timed step, outside the timed events; each step is timed with CUDA
+events on the stream the library launches on.
+
+Other workloads (--workload): pro_decode, hca_decode, hca_compress, prefill.
+
+Multi-GPU (under torchrun): every rank runs its own independent batch
+(decode queries are independent: no collective on the data path), the step
+time is the max over ranks, value = all ranks' queries / that time.
+
+--impl reference times the CPU oracle (fp64, the host's cores) on a bounded
+sample of the same workload.
+
+Prints ONE JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import datetime
+import hashlib
+import io
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "CSA/HCA decode queries/s at 128K–1M ctx and prefill tok/s; % of HBM/TC roofline"
+PROFILES = os.path.join(ROOT, "profiles")
+CSRC = os.path.join(ROOT, "compressed_sparse_attention_14_b200", "csrc")
+
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ----------------------------------------------------------------------------
+# process group / ranks
+# ----------------------------------------------------------------------------
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        if torch.cuda.is_available():
+            dist.barrier(device_ids=[torch.cuda.current_device()])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_done(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for r in csv.reader(f):
+                if len(r) >= 9:
+                    rows.append([x.strip() for x in r])
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = sorted(float(r[1]) for r in rows if r[1].replace(".", "").isdigit())
+        mx = max((float(r[2]) for r in rows if r[2].replace(".", "").isdigit()), default=None)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def source_sha(files) -> str:
+    h = hashlib.sha256()
+    for f in sorted(files):
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str, files) -> float | None:
+    """DRAM bytes per launch from a committed ncu summary, if the kernel's
+    sources are unchanged since the capture; None otherwise."""
+    p = os.path.join(PROFILES, "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(f"{kernel}@{workload}")
+    if not e or e.get("source_sha") != source_sha(files):
+        return None
+    return float(e["dram_bytes_per_launch"])
+
+
+def cpu_oracle_threads() -> int:
+    import oracle
+    return oracle.num_threads()
+
+
+class Timer:
+    """Per-step CUDA-event timing on the current stream with an L2 flush
+    before every step (outside the events)."""
+
+    def __init__(self):
+        self.flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        self.ms = []
+
+    def step(self, fn):
+        self.flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        self.ms.append((a, b))
+
+    def total_ms(self) -> float:
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in self.ms)
+
+
+# ----------------------------------------------------------------------------
+# workloads (ours)
+# ----------------------------------------------------------------------------
+
+def decode_workload(shape, rank):
+    import compressed_sparse_attention_14_b200 as csa
+    s = shape
+    inp = synth.decode_inputs(dataclass_seed(s, rank), device="cuda")
+    B = s.batch
+    mode = csa.CSA_BF16
+    out = torch.empty_like(inp["q"])
+    lse = torch.empty((B, s.heads), dtype=torch.float32, device="cuda")
+    ws = torch.empty(csa.csa_decode_workspace_size(B, s.n_max, s.heads, s.c, s.idx_heads, s.idx_dim, s.k, mode),
+                     dtype=torch.uint8, device="cuda")
+
+    def step():
+        csa.csa_decode(inp["qI"], inp["w"], inp["idx_cache"], inp["q"], inp["kv_cache"], inp["ctx_len"], s.m, s.k,
+                       out=out, lse=lse, ws=ws)
+
+    ctx = inp["ctx_len"].double()
+    vis = torch.floor(ctx / s.m)
+    v_sum = float(vis.sum())
+    # algorithmic bytes: indexer keys of the visible entries, q^I and w; the
+    # selected KV rows; q and out (bf16)
+    idx_bytes = v_sum * s.idx_dim * 2 + B * (s.idx_heads * s.idx_dim * 2 + s.idx_heads * 4)
+    step_bytes = idx_bytes + B * (s.k * s.c * 2 + 2 * s.heads * s.c * 2)
+    # the indexer kernel also writes one fp32 score per visible entry
+    idx_kernel_bytes = idx_bytes + v_sum * 4
+
+    pinned = {k: inp[k].cpu().pin_memory() for k in ("q", "qI", "w", "ctx_len")}
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dev_in = {k: torch.empty_like(inp[k]) for k in pinned}
+
+    def e2e_step():
+        for k, v in pinned.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        csa.csa_decode(dev_in["qI"], dev_in["w"], inp["idx_cache"], dev_in["q"], inp["kv_cache"], dev_in["ctx_len"],
+                       s.m, s.k, out=out, lse=lse, ws=ws)
+        out_h.copy_(out, non_blocking=True)
+
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = out_h.numel() * out_h.element_size()
+    return dict(step=step, e2e_step=e2e_step, units=B, unit="queries/s", h2d=h2d, d2h=d2h,
+                dominant="index_scores_ffma", dominant_bytes=idx_kernel_bytes, dominant_bound="hbm",
+                dominant_files=("indexer.cu", "common.cuh"), step_bytes=step_bytes,
+                config=dict(workload=s.name, batch=B, ctx_len=f"U[{s.ctx_lo},{s.ctx_hi}]", m=s.m,
+                            entries_max=s.n_max, head_dim=s.c, heads=s.heads, index_heads=s.idx_heads,
+                            index_dim=s.idx_dim, topk=s.k, visible_entries_total=int(v_sum),
+                            l2="flushed before every timed step (256 MiB write)"),
+                inputs=inp)
+
+
+def dataclass_seed(s, rank):
+    import dataclasses
+    return dataclasses.replace(s, seed=s.seed + 1000 * rank) if rank else s
+
+
+def hca_decode_workload(rank):
+    import compressed_sparse_attention_14_b200 as csa
+    s = dataclass_seed(synth.HCA, rank)
+    inp = synth.hca_decode_inputs(s, device="cuda")
+    B = s.batch
+    out = torch.empty_like(inp["q"])
+    lse = torch.empty((B, s.heads), dtype=torch.float32, device="cuda")
+    ws = torch.empty(csa.workspace_size("hca_decode", B, s.n_max, s.heads, s.c, csa.CSA_BF16), dtype=torch.uint8,
+                     device="cuda")
+
+    def step():
+        csa.hca_decode(inp["q"], inp["kv_cache"], inp["ctx_len"], s.mp, out=out, lse=lse, ws=ws)
+
+    pinned = {k: inp[k].cpu().pin_memory() for k in ("q", "ctx_len")}
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dev_in = {k: torch.empty_like(inp[k]) for k in pinned}
+
+    def e2e_step():
+        for k, v in pinned.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        csa.hca_decode(dev_in["q"], inp["kv_cache"], dev_in["ctx_len"], s.mp, out=out, lse=lse, ws=ws)
+        out_h.copy_(out, non_blocking=True)
+
+    kv_bytes = B * s.n_max * s.c * 2.0
+    step_bytes = kv_bytes + 2 * B * s.heads * s.c * 2
+    return dict(step=step, e2e_step=e2e_step, units=B, unit="queries/s",
+                h2d=sum(v.numel() * v.element_size() for v in pinned.values()),
+                d2h=out_h.numel() * out_h.element_size(),
+                dominant="mqa_partial_ffma", dominant_bytes=kv_bytes + B * s.heads * s.c * 2,
+                dominant_bound="hbm", dominant_files=("mqa.cu", "common.cuh"), step_bytes=step_bytes,
+                config=dict(workload=s.name.split("_plus")[0], batch=B, ctx_len=s.ctx, mp=s.mp, entries=s.n_max,
+                            head_dim=s.c, heads=s.heads, l2="flushed before every timed step (256 MiB write)"))
+
+
+def hca_compress_workload(rank):
+    import compressed_sparse_attention_14_b200 as csa
+    s = dataclass_seed(synth.HCA, rank)
+    inp = synth.hca_compress_inputs(s, device="cuda")
+    n, d = inp["x"].shape
+    out = torch.empty((n // s.mp, s.c), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(csa.workspace_size("hca_compress_from_hidden", n, d, s.c, s.mp, csa.CSA_BF16),
+                     dtype=torch.uint8, device="cuda")
+
+    def step():
+        csa.hca_compress_from_hidden(inp["x"], inp["W"], inp["bias"], s.mp, out=out, ws=ws)
+
+    x_h = inp["x"].cpu().pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    x_d = torch.empty_like(inp["x"])
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        csa.hca_compress_from_hidden(x_d, inp["W"], inp["bias"], s.mp, out=out, ws=ws)
+        out_h.copy_(out, non_blocking=True)
+
+    flops = 2.0 * n * d * 2 * s.c
+    return dict(step=step, e2e_step=e2e_step, units=n, unit="tokens/s", h2d=x_h.numel() * 2,
+                d2h=out_h.numel() * 2, dominant="project_ffma", dominant_flops=flops, dominant_bound="tensor",
+                dominant_files=("gemm.cu", "common.cuh"), step_bytes=n * d * 2.0,
+                config=dict(workload=f"hca_compress_chunk{n}_d{d}", tokens=n, d=d, mp=s.mp, head_dim=s.c,
+                            l2="inputs larger than L2 and flushed before every timed step"))
+
+
+def prefill_workload(rank):
+    import compressed_sparse_attention_14_b200 as csa
+    s = dataclass_seed(synth.PREFILL, rank)
+    inp = synth.prefill_inputs(s, device="cuda")
+    n = inp["n"]
+    Nmax = inp["kv_cache"].shape[0]
+    out = torch.empty_like(inp["q"])
+    ws = torch.empty(csa.workspace_size("csa_prefill", n, Nmax, s.d, s.m, s.c, s.idx_dim, s.heads, s.idx_heads,
+                                        s.k, csa.CSA_BF16), dtype=torch.uint8, device="cuda")
+
+    def step():
+        csa.csa_prefill(inp["x"], inp["x_left"], inp["W_kv"], inp["B_kv"], inp["W_idx"], inp["B_idx"], inp["start"],
+                        inp["kv_cache"], inp["idx_cache"], inp["qI"], inp["w"], inp["q"], s.k, m=s.m, out=out, ws=ws)
+
+    pos = torch.arange(inp["start"], inp["start"] + n, dtype=torch.float64)
+    pairs = float(torch.floor(pos / s.m).sum())
+    idx_flops = 2.0 * pairs * s.idx_heads * s.idx_dim
+    names = ("x", "qI", "w", "q")
+    pinned = {k: inp[k].cpu().pin_memory() for k in names}
+    dev_in = {k: torch.empty_like(inp[k]) for k in names}
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def e2e_step():
+        for k, v in pinned.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        csa.csa_prefill(dev_in["x"], inp["x_left"], inp["W_kv"], inp["B_kv"], inp["W_idx"], inp["B_idx"],
+                        inp["start"], inp["kv_cache"], inp["idx_cache"], dev_in["qI"], dev_in["w"], dev_in["q"], s.k,
+                        m=s.m, out=out, ws=ws)
+        out_h.copy_(out, non_blocking=True)
+
+    return dict(step=step, e2e_step=e2e_step, units=n, unit="tokens/s",
+                h2d=sum(v.numel() * v.element_size() for v in pinned.values()), d2h=out_h.numel() * 2,
+                dominant="index_scores_ffma", dominant_flops=idx_flops, dominant_bound="tensor",
+                dominant_files=("indexer.cu", "common.cuh"), step_bytes=None,
+                config=dict(workload=s.name, tokens=n, start=inp["start"], d=s.d, m=s.m, head_dim=s.c,
+                            heads=s.heads, index_heads=s.idx_heads, index_dim=s.idx_dim, topk=s.k,
+                            causal_pairs=int(pairs), l2="inputs larger than L2"))
+
+
+WORKLOADS = {
+    "flash_decode": lambda r: decode_workload(synth.FLASH_DECODE, r),
+    "pro_decode": lambda r: decode_workload(synth.PRO_DECODE, r),
+    "hca_decode": hca_decode_workload,
+    "hca_compress": hca_compress_workload,
+    "prefill": prefill_workload,
+}
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle timing (the reference arm and the cpu_baseline object)
+# ----------------------------------------------------------------------------
+
+def oracle_decode_sample(shape, n_queries: int, seed_rank: int = 0):
+    """Time the oracle (indexer + top-k + sparse MQA, fp64) on the first
+    n_queries of the decode batch. Returns (seconds, queries)."""
+    import oracle
+    s = dataclass_seed(shape, seed_rank)
+    inp = synth.decode_inputs(s, device="cpu", batch=n_queries)
+    t0 = time.perf_counter()
+    idx, _ = oracle.index_topk(inp["qI"], inp["w"], inp["idx_cache"], inp["ctx_len"], s.m, s.k,
+                               seq=torch.arange(n_queries))
+    oracle.sparse_mqa(inp["q"], inp["kv_cache"], idx, 1 / math.sqrt(s.c), seq=torch.arange(n_queries))
+    return time.perf_counter() - t0, n_queries
+
+
+def oracle_hca_sample(n_queries: int):
+    import oracle
+    s = synth.HCA
+    inp = synth.hca_decode_inputs(s, batch=n_queries)
+    t0 = time.perf_counter()
+    oracle.dense_mqa(inp["q"], inp["kv_cache"], inp["ctx_len"], s.mp, 1 / math.sqrt(s.c), seq=torch.arange(n_queries))
+    return time.perf_counter() - t0, n_queries
+
+
+def oracle_hca_compress_sample(n_blocks: int):
+    import oracle
+    s = synth.HCA
+    inp = synth.hca_compress_inputs(s, chunk=n_blocks * s.mp)
+    t0 = time.perf_counter()
+    oracle.hca_compress(oracle.project_loops(inp["x"], inp["W"]), inp["bias"], s.mp)
+    return time.perf_counter() - t0, n_blocks * s.mp
+
+
+def oracle_prefill_sample(n_tokens: int):
+    """Indexer + top-k + MQA of the last n_tokens of the chunk against a cache
+    of the chunk's full size (the dominant per-token work; the projection and
+    compression of those tokens' blocks are included)."""
+    import oracle
+    s = synth.PREFILL
+    m = s.m
+    Nmax = (s.start + s.n) // m
+    kv = synth.normal((Nmax, s.c), s.seed, "oracle_kv", dtype=torch.bfloat16)
+    ik = synth.normal((Nmax, s.idx_dim), s.seed, "oracle_ik", dtype=torch.bfloat16)
+    q = synth.normal((n_tokens, s.heads, s.c), s.seed, "q")
+    qI = synth.normal((n_tokens, s.idx_heads, s.idx_dim), s.seed, "qI")
+    w = synth.head_weights(n_tokens, s.idx_heads, s.seed)
+    x = synth.normal((n_tokens, s.d), s.seed, "x")
+    Wkv = synth.normal((4 * s.c, s.d), s.seed, "W_kv", std=1 / math.sqrt(s.d))
+    Bkv = synth.normal((2 * m, s.c), s.seed, "B_kv", dtype=torch.float32)
+    pos = torch.arange(s.start + s.n - n_tokens, s.start + s.n, dtype=torch.int32)
+    t0 = time.perf_counter()
+    oracle.csa_compress(oracle.project_loops(x, Wkv), Bkv, m)
+    idx, _ = oracle.index_topk(qI, w, ik, pos, m, s.k)
+    oracle.sparse_mqa(q, kv, idx, 1 / math.sqrt(s.c))
+    return time.perf_counter() - t0, n_tokens
+
+
+def oracle_measure(workload: str, budget_s: float = 15.0):
+    """Grow the sample until it takes about budget_s seconds; return
+    (units per second, description, units)."""
+    threads = cpu_oracle_threads()
+    if workload in ("flash_decode", "pro_decode"):
+        shape = synth.FLASH_DECODE if workload == "flash_decode" else synth.PRO_DECODE
+        n = max(1, threads // 2)
+        while True:
+            sec, units = oracle_decode_sample(shape, min(n, shape.batch))
+            if sec >= budget_s / 3 or n >= shape.batch:
+                break
+            n *= 2
+        desc = f"first {units} of the {shape.batch} decode queries (indexer + top-k + sparse MQA, fp64)"
+    elif workload == "hca_decode":
+        n = max(1, threads // 4)
+        while True:
+            sec, units = oracle_hca_sample(min(n, synth.HCA.batch))
+            if sec >= budget_s / 3 or n >= synth.HCA.batch:
+                break
+            n *= 2
+        desc = f"first {units} of the {synth.HCA.batch} HCA decode queries (dense MQA, fp64)"
+    elif workload == "hca_compress":
+        n = 2
+        while True:
+            sec, units = oracle_hca_compress_sample(n)
+            if sec >= budget_s / 3 or n >= 1024:
+                break
+            n *= 2
+        desc = f"{units} tokens ({units // synth.HCA.mp} blocks) of the compressor chunk (projection + compression, fp64)"
+    else:
+        n = max(1, threads // 2)
+        while True:
+            sec, units = oracle_prefill_sample(n)
+            if sec >= budget_s / 3 or n >= 4096:
+                break
+            n *= 2
+        desc = (f"last {units} tokens of the prefill chunk (projection + compression of their blocks, indexer over "
+                f"~65K entries, top-k, sparse MQA; fp64)")
+    return units / sec, desc, units, sec
+
+
+# ----------------------------------------------------------------------------
+# main
+# ----------------------------------------------------------------------------
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        dist_done(world)
+        return
+    threads = cpu_oracle_threads()
+    per_step, desc, units, _ = oracle_measure(args.workload, budget_s=6.0)
+    # each step: a sample of about the size measured above
+    times = []
+    for i in range(args.warmup + args.steps):
+        if args.workload in ("flash_decode", "pro_decode"):
+            shape = synth.FLASH_DECODE if args.workload == "flash_decode" else synth.PRO_DECODE
+            sec, u = oracle_decode_sample(shape, units)
+        elif args.workload == "hca_decode":
+            sec, u = oracle_hca_sample(units)
+        elif args.workload == "hca_compress":
+            sec, u = oracle_hca_compress_sample(units // synth.HCA.mp)
+        else:
+            sec, u = oracle_prefill_sample(units)
+        if i >= args.warmup:
+            times.append(sec)
+    total = sum(times)
+    value = units * len(times) / total
+    wl = WORKLOADS_CONFIG_NAME.get(args.workload, args.workload)
+    unit = "tokens/s" if args.workload in ("hca_compress", "prefill") else "queries/s"
+    line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference", "config": {"workload": wl, "sample_per_step": desc},
+            "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    dist_done(world)
+
+
+WORKLOADS_CONFIG_NAME = {
+    "flash_decode": synth.FLASH_DECODE.name,
+    "pro_decode": synth.PRO_DECODE.name,
+    "hca_decode": synth.HCA.name.split("_plus")[0],
+    "hca_compress": "hca_compress_chunk131072_d4096",
+    "prefill": synth.PREFILL.name,
+}
+
+
+def run_ours(args, rank, world, local):
+    import compressed_sparse_attention_14_b200 as csa
+    wl = WORKLOADS[args.workload](rank)
+    step, e2e_step = wl["step"], wl["e2e_step"]
+
+    # warm-up
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    timer = Timer()
+    vis = [v.strip() for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    clocks = ClockSampler(vis[local] if local < len(vis) else local)
+    csa.trace_enable(True)
+    l0 = csa.launch_count()
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    t_wall0 = time.perf_counter()
+    for _ in range(args.steps):
+        timer.step(step)
+    torch.cuda.synchronize()
+    barrier(world)
+    t_wall = time.perf_counter() - t_wall0
+    launches = csa.launch_count() - l0
+    ms_total = timer.total_ms()
+    trace = csa.trace_read()
+    csa.trace_enable(False)
+    clk = clocks.stop()
+    ms_total_max = max_over_ranks(ms_total, world)
+    ms_step = ms_total_max / args.steps
+
+    # end to end: host buffers in, host result out, through the public call
+    e2e_timer = Timer()
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    for _ in range(args.steps):
+        e2e_timer.step(e2e_step)
+    e2e_ms = max_over_ranks(e2e_timer.total_ms(), world) / args.steps
+
+    units = wl["units"]
+    value = world * units / (ms_step / 1e3)
+    peaks = measured_peaks()
+    dom = wl["dominant"]
+    dom_ms, dom_n = trace.get(dom, (float("nan"), 0))
+    dom_avg_s = dom_ms / max(dom_n, 1) / 1e3
+    if wl["dominant_bound"] == "hbm":
+        per_launch = wl["dominant_bytes"] * args.steps / max(dom_n, 1)
+        achieved = per_launch / dom_avg_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"] + " hbm_gbs"}
+    else:
+        per_launch = wl["dominant_flops"] * args.steps / max(dom_n, 1)
+        achieved = per_launch / dom_avg_s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "peak_source": peaks["source"] + " bf16_tflops"}
+    roof["kernel"] = dom
+    roof["launches_per_step"] = dom_n / args.steps
+    roof["traffic"] = ncu_traffic(dom, args.workload, wl["dominant_files"])
+
+    line = {"metric": METRIC, "value": value, "unit": wl["unit"], "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": wl["config"],
+            "roofline": roof,
+            "kernels_ms_per_step": {k: v[0] / args.steps for k, v in sorted(trace.items())},
+            "e2e": {"value": world * units / (e2e_ms / 1e3), "unit": wl["unit"], "h2d_bytes_per_step": wl["h2d"],
+                    "d2h_bytes_per_step": wl["d2h"]},
+            "gpu_launches": launches, "clocks": clk, "wall_s_timed": t_wall}
+    if wl.get("step_bytes"):
+        sb = wl["step_bytes"] / (ms_step / 1e3) / 1e9
+        line["step_roofline"] = {"bound": "hbm", "achieved": sb, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                 "frac": sb / peaks["hbm_gbs"]}
+    del wl
+    torch.cuda.empty_cache()
+    if rank == 0 and not args.no_cpu_baseline:
+        cps, desc, _, _ = oracle_measure(args.workload)
+        line["cpu_baseline"] = {"value": cps, "unit": line["unit"], "cores": cpu_oracle_threads(),
+                                "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    dist_done(world)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="flash_decode", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
+    args = ap.parse_args()
+    rank, world, local = dist_init()
+    if world != args.gpus and rank == 0:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,332 @@
+"""Python binding of libcsa, the B200 (sm_100a) CUDA library for the
+DeepSeek-V4 compressed attention hot path (CSA and HCA).
+
+Argument marshalling only: every function below checks tensor devices,
+dtypes and shapes, allocates outputs and the workspace with torch, and calls
+the C entry point of the same name (include/csa.h) on the current CUDA
+stream. All arithmetic runs in the library's kernels. There is no CPU path:
+importing this package without the built library raises.
+
+dtype: bf16 tensors run the CSA_BF16 mode, fp32 tensors the CSA_FP32 mode
+(biases, head weights `w`, sinks, scores and lse are fp32 in both).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsa.so")
+
+CSA_OK, CSA_ERR_INVALID_ARG, CSA_ERR_UNSUPPORTED, CSA_ERR_WORKSPACE, CSA_ERR_CUDA, CSA_ERR_TIMEOUT = range(6)
+CSA_BF16, CSA_FP32 = 0, 1
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with "
+                      "`python compressed_sparse_attention_14_b200/build.py` (nvcc, sm_100a)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+_F = ctypes.c_float
+
+# name -> (restype, argtypes)
+_SIGS = {
+    "csa_last_error": (ctypes.c_char_p, []),
+    "csa_abi_version": (_I, []),
+    "csa_launch_count": (ctypes.c_uint64, []),
+    "csa_trace_enable": (None, [_I]),
+    "csa_trace_read": (_I, [_I, _P, _P, _P, _P]),
+    "csa_poll_status": (_I, [_P, _I]),
+    "csa_project": (_I, [_P, _P, _I64, _I, _I, _P, _I, _P]),
+    "csa_compress": (_I, [_P, _P, _P, _I64, _I, _I, _P, _I, _P]),
+    "hca_compress": (_I, [_P, _P, _I64, _I, _I, _P, _I, _P]),
+    "csa_compress_from_hidden_workspace_size": (_SZ, [_I64, _I, _I, _I, _I]),
+    "csa_compress_from_hidden": (_I, [_P, _P, _P, _P, _I64, _I, _I, _I, _P, _P, _SZ, _I, _P]),
+    "hca_compress_from_hidden_workspace_size": (_SZ, [_I64, _I, _I, _I, _I]),
+    "hca_compress_from_hidden": (_I, [_P, _P, _P, _I64, _I, _I, _I, _P, _P, _SZ, _I, _P]),
+    "csa_index_scores": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _P, _I, _P]),
+    "csa_topk_workspace_size": (_SZ, [_I, _I64, _I]),
+    "csa_topk_from_scores": (_I, [_P, _I64, _P, _I, _I, _I64, _I, _P, _P, _P, _SZ, _P]),
+    "csa_index_topk_workspace_size": (_SZ, [_I, _I64, _I, _I]),
+    "csa_index_topk": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I, _P, _P, _P, _SZ, _I, _P]),
+    "csa_sparse_mqa_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "csa_sparse_mqa": (_I, [_P, _P, _P, _P, _I, _I, _I, _I64, _I, _F, _P, _P, _P, _P, _SZ, _I, _P]),
+    "hca_dense_mqa_workspace_size": (_SZ, [_I, _I, _I, _I64, _I]),
+    "hca_dense_mqa": (_I, [_P, _P, _P, _P, _I, _I, _I, _I64, _I, _F, _P, _P, _P, _P, _SZ, _I, _P]),
+    "csa_decode_workspace_size": (_SZ, [_I, _I64, _I, _I, _I, _I, _I, _I]),
+    "csa_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I64, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P,
+                        _P, _SZ, _I, _P]),
+    "hca_decode_workspace_size": (_SZ, [_I, _I64, _I, _I, _I]),
+    "hca_decode": (_I, [_P, _P, _P, _I, _I64, _I, _I, _I, _F, _P, _P, _P, _P, _SZ, _I, _P]),
+    "csa_prefill_workspace_size": (_SZ, [_I64, _I64, _I, _I, _I, _I, _I, _I, _I, _I]),
+    "csa_prefill": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I, _I, _I, _I, _P, _P, _I64, _P, _P, _P,
+                         _I, _I, _I, _F, _P, _P, _P, _P, _P, _SZ, _I, _P]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+EXPORTED = tuple(_SIGS)
+
+
+class CsaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"libcsa error {code}: {msg}")
+        self.code = code
+
+
+def _check(rc: int) -> None:
+    if rc != CSA_OK:
+        raise CsaError(rc, _lib.csa_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libcsa takes CUDA tensors only")
+    if not t.is_contiguous():
+        raise ValueError("libcsa takes contiguous tensors only")
+    return t.data_ptr()
+
+
+def _stream():
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _mode(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return CSA_BF16
+    if t.dtype == torch.float32:
+        return CSA_FP32
+    raise ValueError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _ws(nbytes: int, device, ws: Optional[torch.Tensor] = None) -> Optional[torch.Tensor]:
+    if nbytes == 0:
+        return None
+    if ws is not None and ws.numel() * ws.element_size() >= nbytes:
+        return ws
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def _nbytes(t: Optional[torch.Tensor]) -> int:
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+def abi_version() -> int:
+    return _lib.csa_abi_version()
+
+
+def launch_count() -> int:
+    """Kernels this library has launched so far in this process."""
+    return int(_lib.csa_launch_count())
+
+
+def trace_enable(on: bool = True) -> None:
+    """Start (or stop) per-kernel event timing; discards earlier records."""
+    _lib.csa_trace_enable(int(on))
+
+
+def trace_read(max_kernels: int = 64) -> dict:
+    """{kernel name: (total device ms, launches)} for the records so far."""
+    names = ctypes.create_string_buffer(64 * max_kernels)
+    ms = (ctypes.c_double * max_kernels)()
+    cnt = (ctypes.c_int * max_kernels)()
+    n = ctypes.c_int(0)
+    _check(_lib.csa_trace_read(max_kernels, ctypes.addressof(names), ctypes.addressof(ms), ctypes.addressof(cnt),
+                               ctypes.addressof(n)))
+    out = {}
+    for i in range(n.value):
+        nm = names.raw[64 * i: 64 * i + 64].split(b"\0", 1)[0].decode()
+        out[nm] = (ms[i], cnt[i])
+    return out
+
+
+def poll_status(reset: bool = True) -> None:
+    _check(_lib.csa_poll_status(_stream(), int(reset)))
+
+
+def workspace_size(name: str, *args) -> int:
+    return int(getattr(_lib, name + "_workspace_size")(*args))
+
+
+# ---------------------------------------------------------------- a1
+def csa_project(x: torch.Tensor, W: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    n, d = x.shape
+    M = W.shape[0]
+    out = torch.empty((n, M), dtype=torch.float32, device=x.device) if out is None else out
+    _check(_lib.csa_project(_ptr(x), _ptr(W), n, d, M, _ptr(out), _mode(x), _stream()))
+    return out
+
+
+# ---------------------------------------------------------------- a2 / a3
+def csa_compress(proj, bias, m: int, left=None, out=None):
+    n, c4 = proj.shape
+    c = c4 // 4
+    out = torch.empty((n // m, c), dtype=proj.dtype, device=proj.device) if out is None else out
+    _check(_lib.csa_compress(_ptr(proj), _ptr(left), _ptr(bias), n, c, m, _ptr(out), _mode(proj), _stream()))
+    return out
+
+
+def hca_compress(proj, bias, mp: int, out=None):
+    n, c2 = proj.shape
+    c = c2 // 2
+    out = torch.empty((n // mp, c), dtype=proj.dtype, device=proj.device) if out is None else out
+    _check(_lib.hca_compress(_ptr(proj), _ptr(bias), n, c, mp, _ptr(out), _mode(proj), _stream()))
+    return out
+
+
+def csa_compress_from_hidden(x, W, bias, m: int, x_left=None, out=None, ws=None):
+    n, d = x.shape
+    c = W.shape[0] // 4
+    mode = _mode(x)
+    out = torch.empty((n // m, c), dtype=x.dtype, device=x.device) if out is None else out
+    nb = _lib.csa_compress_from_hidden_workspace_size(n, d, c, m, mode)
+    ws = _ws(nb, x.device, ws)
+    _check(_lib.csa_compress_from_hidden(_ptr(x), _ptr(x_left), _ptr(W), _ptr(bias), n, d, c, m, _ptr(out),
+                                         _ptr(ws), _nbytes(ws), mode, _stream()))
+    return out
+
+
+def hca_compress_from_hidden(x, W, bias, mp: int, out=None, ws=None):
+    n, d = x.shape
+    c = W.shape[0] // 2
+    mode = _mode(x)
+    out = torch.empty((n // mp, c), dtype=x.dtype, device=x.device) if out is None else out
+    nb = _lib.hca_compress_from_hidden_workspace_size(n, d, c, mp, mode)
+    ws = _ws(nb, x.device, ws)
+    _check(_lib.hca_compress_from_hidden(_ptr(x), _ptr(W), _ptr(bias), n, d, c, mp, _ptr(out), _ptr(ws),
+                                         _nbytes(ws), mode, _stream()))
+    return out
+
+
+# ---------------------------------------------------------------- a4 / a5
+def _kv3(K):
+    return K if K.dim() == 3 else K.unsqueeze(0)
+
+
+def csa_index_scores(qI, w, K, pos, m: int, seq_of_q=None):
+    nq, HI, cI = qI.shape
+    K = _kv3(K)
+    Nmax = K.shape[1]
+    scores = torch.empty((nq, Nmax), dtype=torch.float32, device=qI.device)
+    _check(_lib.csa_index_scores(_ptr(qI), _ptr(w), _ptr(K), _ptr(pos), _ptr(seq_of_q), nq, HI, cI, Nmax, m,
+                                 _ptr(scores), _mode(qI), _stream()))
+    return scores
+
+
+def csa_topk_from_scores(scores, k: int, valid=None, valid_div: int = 1, ws=None):
+    nq, ncols = scores.shape
+    idx = torch.empty((nq, k), dtype=torch.int32, device=scores.device)
+    top = torch.empty((nq, k), dtype=torch.float32, device=scores.device)
+    ws = _ws(_lib.csa_topk_workspace_size(nq, ncols, k), scores.device, ws)
+    _check(_lib.csa_topk_from_scores(_ptr(scores), ncols, _ptr(valid), valid_div, nq, ncols, k, _ptr(idx),
+                                     _ptr(top), _ptr(ws), _nbytes(ws), _stream()))
+    return idx, top
+
+
+def csa_index_topk(qI, w, K, pos, m: int, k: int, seq_of_q=None, ws=None):
+    nq, HI, cI = qI.shape
+    K = _kv3(K)
+    Nmax = K.shape[1]
+    mode = _mode(qI)
+    idx = torch.empty((nq, k), dtype=torch.int32, device=qI.device)
+    top = torch.empty((nq, k), dtype=torch.float32, device=qI.device)
+    ws = _ws(_lib.csa_index_topk_workspace_size(nq, Nmax, k, mode), qI.device, ws)
+    _check(_lib.csa_index_topk(_ptr(qI), _ptr(w), _ptr(K), _ptr(pos), _ptr(seq_of_q), nq, HI, cI, Nmax, m, k,
+                               _ptr(idx), _ptr(top), _ptr(ws), _nbytes(ws), mode, _stream()))
+    return idx, top
+
+
+# ---------------------------------------------------------------- a6 / a7
+def csa_sparse_mqa(q, KV, idx, scale: float = 0.0, sink=None, seq_of_q=None, out=None, ws=None):
+    nq, H, c = q.shape
+    KV = _kv3(KV)
+    Nmax = KV.shape[1]
+    k = idx.shape[1]
+    mode = _mode(q)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((nq, H), dtype=torch.float32, device=q.device)
+    ws = _ws(_lib.csa_sparse_mqa_workspace_size(nq, H, c, k, mode), q.device, ws)
+    _check(_lib.csa_sparse_mqa(_ptr(q), _ptr(KV), _ptr(idx), _ptr(seq_of_q), nq, H, c, Nmax, k, scale,
+                               _ptr(sink), _ptr(out), _ptr(lse), _ptr(ws), _nbytes(ws), mode, _stream()))
+    return out, lse
+
+
+def hca_dense_mqa(q, KV, pos, mp: int, scale: float = 0.0, sink=None, seq_of_q=None, out=None, ws=None):
+    nq, H, c = q.shape
+    KV = _kv3(KV)
+    Nmax = KV.shape[1]
+    mode = _mode(q)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((nq, H), dtype=torch.float32, device=q.device)
+    ws = _ws(_lib.hca_dense_mqa_workspace_size(nq, H, c, Nmax, mode), q.device, ws)
+    _check(_lib.hca_dense_mqa(_ptr(q), _ptr(KV), _ptr(pos), _ptr(seq_of_q), nq, H, c, Nmax, mp, scale,
+                              _ptr(sink), _ptr(out), _ptr(lse), _ptr(ws), _nbytes(ws), mode, _stream()))
+    return out, lse
+
+
+# ---------------------------------------------------------------- fused
+def csa_decode_workspace_size(B, Nmax, H, c, HI, cI, k, mode) -> int:
+    return int(_lib.csa_decode_workspace_size(B, Nmax, H, c, HI, cI, k, mode))
+
+
+def csa_decode(qI, w, idx_cache, q, kv_cache, ctx_len, m: int, k: int, scale: float = 0.0, sink=None,
+               out=None, lse=None, topk_idx=None, ws=None, return_topk: bool = False):
+    B, HI, cI = qI.shape
+    _, H, c = q.shape
+    Nmax = kv_cache.shape[1]
+    mode = _mode(q)
+    out = torch.empty_like(q) if out is None else out
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    if return_topk and topk_idx is None:
+        topk_idx = torch.empty((B, k), dtype=torch.int32, device=q.device)
+    ws = _ws(csa_decode_workspace_size(B, Nmax, H, c, HI, cI, k, mode), q.device, ws)
+    _check(_lib.csa_decode(_ptr(qI), _ptr(w), _ptr(idx_cache), _ptr(q), _ptr(kv_cache), _ptr(ctx_len), B, Nmax,
+                           m, H, c, HI, cI, k, scale, _ptr(sink), _ptr(out), _ptr(lse), _ptr(topk_idx),
+                           _ptr(ws), _nbytes(ws), mode, _stream()))
+    return (out, lse, topk_idx) if return_topk else (out, lse)
+
+
+def hca_decode(q, kv_cache, ctx_len, mp: int, scale: float = 0.0, sink=None, out=None, lse=None, ws=None):
+    B, H, c = q.shape
+    Nmax = kv_cache.shape[1]
+    mode = _mode(q)
+    out = torch.empty_like(q) if out is None else out
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    ws = _ws(_lib.hca_decode_workspace_size(B, Nmax, H, c, mode), q.device, ws)
+    _check(_lib.hca_decode(_ptr(q), _ptr(kv_cache), _ptr(ctx_len), B, Nmax, mp, H, c, scale, _ptr(sink),
+                           _ptr(out), _ptr(lse), _ptr(ws), _nbytes(ws), mode, _stream()))
+    return out, lse
+
+
+def csa_prefill(x, x_left, W_kv, B_kv, W_idx, B_idx, start: int, kv_cache, idx_cache, qI, w, q, k: int,
+                m: int = 4, scale: float = 0.0, sink=None, out=None, ws=None, return_topk: bool = False):
+    n, d = x.shape
+    c = W_kv.shape[0] // 4
+    cI = W_idx.shape[0] // 4
+    _, H, _ = q.shape
+    _, HI, _ = qI.shape
+    Nmax = kv_cache.shape[0]
+    mode = _mode(x)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((n, H), dtype=torch.float32, device=x.device)
+    topk_idx = torch.empty((n, k), dtype=torch.int32, device=x.device) if return_topk else None
+    nb = _lib.csa_prefill_workspace_size(n, Nmax, d, m, c, cI, H, HI, k, mode)
+    ws = _ws(nb, x.device, ws)
+    _check(_lib.csa_prefill(_ptr(x), _ptr(x_left), _ptr(W_kv), _ptr(B_kv), _ptr(W_idx), _ptr(B_idx), start, n, d,
+                            m, c, cI, _ptr(kv_cache), _ptr(idx_cache), Nmax, _ptr(qI), _ptr(w), _ptr(q), H, HI, k,
+                            scale, _ptr(sink), _ptr(out), _ptr(lse), _ptr(topk_idx), _ptr(ws), _nbytes(ws), mode,
+                            _stream()))
+    return (out, lse, topk_idx) if return_topk else (out, lse)

@@ -1,0 +1,544 @@
+// C ABI of libcsa: argument checks, workspace planning and launch order for
+// every entry point declared in include/csa.h. All checks run on the host
+// before the first launch; nothing here allocates device memory.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+#include <string>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace csa {
+
+__device__ int g_status_word = 0;
+
+
+static thread_local std::string g_err;
+
+static int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+static int cuda_status(cudaError_t e, const char* where) {
+    if (e == cudaSuccess) return CSA_OK;
+    return fail(CSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+#define CSA_TRY(expr)                          \
+    do {                                       \
+        int _rc = (expr);                      \
+        if (_rc != CSA_OK) return _rc;         \
+    } while (0)
+
+#define CSA_CUDA(expr, where)                                  \
+    do {                                                       \
+        cudaError_t _e = (expr);                               \
+        if (_e != cudaSuccess) return cuda_status(_e, where);  \
+    } while (0)
+
+static int check_ptr(const void* p, const char* name, bool required = true) {
+    if (!p) return required ? fail(CSA_ERR_INVALID_ARG, "%s is NULL", name) : CSA_OK;
+    if (((uintptr_t)p) & 15u) return fail(CSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+    return CSA_OK;
+}
+
+static int check_dtype(int dtype, ElemType* t) {
+    if (dtype == CSA_BF16) { *t = ElemType::BF16; return CSA_OK; }
+    if (dtype == CSA_FP32) { *t = ElemType::F32; return CSA_OK; }
+    return fail(CSA_ERR_INVALID_ARG, "dtype %d is neither CSA_BF16 nor CSA_FP32", dtype);
+}
+
+static int check_ws(void* ws, size_t have, size_t need) {
+    if (need == 0) return CSA_OK;
+    if (!ws) return fail(CSA_ERR_WORKSPACE, "workspace is NULL but %zu bytes are needed", need);
+    if (((uintptr_t)ws) & 255u) return fail(CSA_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+    if (have < need) return fail(CSA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", have, need);
+    return CSA_OK;
+}
+
+static float default_scale(float scale, int c) { return scale == 0.f ? 1.f / sqrtf((float)c) : scale; }
+
+// Carves consecutive 256-byte aligned regions out of a workspace.
+struct Carve {
+    char* base;
+    size_t off = 0;
+    explicit Carve(void* b) : base((char*)b) {}
+    void* take(size_t bytes) {
+        void* p = base ? base + off : nullptr;
+        off += align256(bytes);
+        return p;
+    }
+};
+
+static int check_attn_shape(int H, int c) {
+    if (H < 1 || H > CSA_MAX_HEADS) return fail(CSA_ERR_UNSUPPORTED, "H=%d outside [1, %d]", H, CSA_MAX_HEADS);
+    if (c < 32 || c > CSA_MAX_HEAD_DIM || c % 32)
+        return fail(CSA_ERR_UNSUPPORTED, "head dim c=%d must be a multiple of 32 in [32, %d]", c, CSA_MAX_HEAD_DIM);
+    return CSA_OK;
+}
+
+static int check_index_shape(int HI, int cI) {
+    if (HI < 1 || HI > CSA_MAX_INDEX_HEADS)
+        return fail(CSA_ERR_UNSUPPORTED, "HI=%d outside [1, %d]", HI, CSA_MAX_INDEX_HEADS);
+    if (cI < 8 || cI > CSA_MAX_INDEX_DIM || cI % 8)
+        return fail(CSA_ERR_UNSUPPORTED, "index dim cI=%d must be a multiple of 8 in [8, %d]", cI, CSA_MAX_INDEX_DIM);
+    return CSA_OK;
+}
+
+static int check_k(int k) {
+    if (k < 1 || k > CSA_MAX_TOPK) return fail(CSA_ERR_UNSUPPORTED, "k=%d outside [1, %d]", k, CSA_MAX_TOPK);
+    return CSA_OK;
+}
+
+// ---- plans shared by the size queries and the calls ------------------------
+
+static size_t index_topk_bytes(int nq, int64_t Nmax, int k) {
+    return align256((size_t)nq * (size_t)Nmax * sizeof(float)) + topk_workspace_bytes(nq, Nmax, k);
+}
+
+static int64_t prefill_query_chunk(int64_t n, int64_t Nmax) {
+    // bound the fp32 score block of one query chunk to 1 GiB
+    int64_t qc = ((int64_t)1 << 28) / (Nmax > 0 ? Nmax : 1);
+    if (qc < 1) qc = 1;
+    if (qc > n) qc = n;
+    return qc;
+}
+
+}  // namespace csa
+
+using namespace csa;
+
+extern "C" {
+
+const char* csa_last_error(void) { return g_err.c_str(); }
+int csa_abi_version(void) { return CSA_ABI_VERSION; }
+uint64_t csa_launch_count(void) { return launch_count(); }
+
+void csa_trace_enable(int on) { trace_enable(on); }
+
+int csa_trace_read(int max_kernels, char* names, double* total_ms, int* counts, int* n_kernels) {
+    if (max_kernels < 0 || (max_kernels > 0 && (!names || !total_ms || !counts)) || !n_kernels)
+        return fail(CSA_ERR_INVALID_ARG, "csa_trace_read: bad buffers");
+    int e = trace_read(max_kernels, names, total_ms, counts, n_kernels);
+    if (e) return cuda_status((cudaError_t)e, "csa_trace_read");
+    return CSA_OK;
+}
+
+int csa_poll_status(void* stream, int reset) {
+    cudaStream_t st = (cudaStream_t)stream;
+    int v = 0;
+    CSA_CUDA(cudaStreamSynchronize(st), "csa_poll_status sync");
+    CSA_CUDA(cudaMemcpyFromSymbol(&v, g_status_word, sizeof(int)), "csa_poll_status read");
+    if (reset) {
+        int z = 0;
+        CSA_CUDA(cudaMemcpyToSymbol(g_status_word, &z, sizeof(int)), "csa_poll_status reset");
+    }
+    if (v != 0) return fail(v, "a kernel reported device error %d", v);
+    return CSA_OK;
+}
+
+// ---------------------------------------------------------------- a1
+int csa_project(const void* x, const void* W, int64_t n, int d, int M, float* out, int dtype,
+                void* stream) {
+    ElemType t;
+    CSA_TRY(check_dtype(dtype, &t));
+    if (n < 0 || d < 8 || d % 8 || M < 8 || M % 8)
+        return fail(CSA_ERR_INVALID_ARG, "csa_project: need n>=0, d and M multiples of 8 (n=%lld d=%d M=%d)",
+                    (long long)n, d, M);
+    if (n == 0) return CSA_OK;
+    CSA_TRY(check_ptr(x, "x"));
+    CSA_TRY(check_ptr(W, "W"));
+    CSA_TRY(check_ptr(out, "out"));
+    CSA_CUDA(project(x, W, n, d, M, out, t, (cudaStream_t)stream), "csa_project");
+    return CSA_OK;
+}
+
+// ---------------------------------------------------------------- a2 / a3
+static int check_compress(int64_t n, int c, int m, int mmax, const char* who) {
+    if (m < 1 || m > mmax) return fail(CSA_ERR_INVALID_ARG, "%s: compression rate %d outside [1, %d]", who, m, mmax);
+    if (n < 0 || n % m) return fail(CSA_ERR_INVALID_ARG, "%s: n=%lld is not a multiple of %d", who, (long long)n, m);
+    if (c < 8 || c % 8) return fail(CSA_ERR_INVALID_ARG, "%s: c=%d must be a positive multiple of 8", who, c);
+    return CSA_OK;
+}
+
+int csa_compress(const void* proj, const void* left, const float* bias, int64_t n, int c, int m,
+                 void* out, int dtype, void* stream) {
+    ElemType t;
+    CSA_TRY(check_dtype(dtype, &t));
+    CSA_TRY(check_compress(n, c, m, 64, "csa_compress"));
+    if (n == 0) return CSA_OK;
+    CSA_TRY(check_ptr(proj, "proj"));
+    CSA_TRY(check_ptr(left, "left", false));
+    CSA_TRY(check_ptr(bias, "bias"));
+    CSA_TRY(check_ptr(out, "out"));
+    CSA_CUDA(compress_csa(proj, left, bias, n, c, m, out, t, t, (cudaStream_t)stream), "csa_compress");
+    return CSA_OK;
+}
+
+int hca_compress(const void* proj, const float* bias, int64_t n, int c, int mp, void* out,
+                 int dtype, void* stream) {
+    ElemType t;
+    CSA_TRY(check_dtype(dtype, &t));
+    CSA_TRY(check_compress(n, c, mp, 1024, "hca_compress"));
+    if (n == 0) return CSA_OK;
+    CSA_TRY(check_ptr(proj, "proj"));
+    CSA_TRY(check_ptr(bias, "bias"));
+    CSA_TRY(check_ptr(out, "out"));
+    CSA_CUDA(compress_hca(proj, bias, n, c, mp, out, t, t, (cudaStream_t)stream), "hca_compress");
+    return CSA_OK;
+}
+
+size_t csa_compress_from_hidden_workspace_size(int64_t n, int d, int c, int m, int dtype) {
+    (void)d; (void)dtype;
+    if (n < 0 || c < 0 || m < 1) return 0;
+    return align256((size_t)n * 4 * c * sizeof(float)) + align256((size_t)m * 4 * c * sizeof(float));
+}
+
+int csa_compress_from_hidden(const void* x, const void* x_left, const void* W, const float* bias,
+                             int64_t n, int d, int c, int m, void* out, void* ws, size_t ws_bytes,
+                             int dtype, void* stream) {
+    ElemType t;
+    CSA_TRY(check_dtype(dtype, &t));
+    CSA_TRY(check_compress(n, c, m, 64, "csa_compress_from_hidden"));
+    if (d < 8 || d % 8) return fail(CSA_ERR_INVALID_ARG, "d=%d must be a positive multiple of 8", d);
+    if (n == 0) return CSA_OK;
+    CSA_TRY(check_ptr(x, "x"));
+    CSA_TRY(check_ptr(x_left, "x_left", false));
+    CSA_TRY(check_ptr(W, "W"));
+    CSA_TRY(check_ptr(bias, "bias"));
+    CSA_TRY(check_ptr(out, "out"));
+    CSA_TRY(check_ws(ws, ws_bytes, csa_compress_from_hidden_workspace_size(n, d, c, m, dtype)));
+    cudaStream_t st = (cudaStream_t)stream;
+    Carve cv(ws);
+    float* proj = (float*)cv.take((size_t)n * 4 * c * sizeof(float));
+    float* lproj = (float*)cv.take((size_t)m * 4 * c * sizeof(float));
+    CSA_CUDA(project(x, W, n, d, 4 * c, proj, t, st), "csa_compress_from_hidden: projection");
+    if (x_left) CSA_CUDA(project(x_left, W, m, d, 4 * c, lproj, t, st), "csa_compress_from_hidden: left projection");
+    CSA_CUDA(compress_csa(proj, x_left ? lproj : nullptr, bias, n, c, m, out, ElemType::F32, t, st),
+             "csa_compress_from_hidden: compress");
+    return CSA_OK;
+}
+
+size_t hca_compress_from_hidden_workspace_size(int64_t n, int d, int c, int mp, int dtype) {
+    (void)d; (void)mp; (void)dtype;
+    if (n < 0 || c < 0) return 0;
+    return align256((size_t)n * 2 * c * sizeof(float));
+}
+
+int hca_compress_from_hidden(const void* x, const void* W, const float* bias, int64_t n, int d,
+                             int c, int mp, void* out, void* ws, size_t ws_bytes, int dtype,
+                             void* stream) {
+    ElemType t;
+    CSA_TRY(check_dtype(dtype, &t));
+    CSA_TRY(check_compress(n, c, mp, 1024, "hca_compress_from_hidden"));
+    if (d < 8 || d % 8) return fail(CSA_ERR_INVALID_ARG, "d=%d must be a positive multiple of 8", d);
+    if (n == 0) return CSA_OK;
+    CSA_TRY(check_ptr(x, "x"));
+    CSA_TRY(check_ptr(W, "W"));
+    CSA_TRY(check_ptr(bias, "bias"));
+    CSA_TRY(check_ptr(out, "out"));
+    CSA_TRY(check_ws(ws, ws_bytes, hca_compress_from_hidden_workspace_size(n, d, c, mp, dtype)));
+    cudaStream_t st = (cudaStream_t)stream;
+    float* proj = (float*)ws;
+    CSA_CUDA(project(x, W, n, d, 2 * c, proj, t, st), "hca_compress_from_hidden: projection");
+    CSA_CUDA(compress_hca(proj, bias, n, c, mp, out, ElemType::F32, t, st), "hca_compress_from_hidden: compress");
+    return CSA_OK;
+}
+
+// ---------------------------------------------------------------- a4 / a5
+int csa_index_scores(const void* qI, const float* w, const void* K, const int32_t* pos,
+                     const int32_t* seq_of_q, int nq, int HI, int cI, int64_t Nmax, int m,
+                     float* scores, int dtype, void* stream) {
+    ElemType t;
+    CSA_TRY(check_dtype(dtype, &t));
+    CSA_TRY(check_index_shape(HI, cI));
+    if (nq < 0 || Nmax < 0 || m < 1) return fail(CSA_ERR_INVALID_ARG, "bad nq/Nmax/m");
+    if (Nmax > INT32_MAX) return fail(CSA_ERR_UNSUPPORTED, "Nmax beyond int32 entry indices");
+    if (nq == 0 || Nmax == 0) return CSA_OK;
+    CSA_TRY(check_ptr(qI, "qI"));
+    CSA_TRY(check_ptr(w, "w"));
+    CSA_TRY(check_ptr(K, "K"));
+    CSA_TRY(check_ptr(pos, "pos"));
+    CSA_TRY(check_ptr(seq_of_q, "seq_of_q", false));
+    CSA_TRY(check_ptr(scores, "scores"));
+    QuerySpec qs{seq_of_q, pos, 0, 0};
+    CSA_CUDA(index_scores(qI, w, K, qs, nq, HI, cI, Nmax, m, scores, Nmax, t, (cudaStream_t)stream),
+             "csa_index_scores");
+    return CSA_OK;
+}
+
+size_t csa_topk_workspace_size(int nq, int64_t ncols, int k) {
+    if (nq < 0 || ncols < 0 || k < 1) return 0;
+    return topk_workspace_bytes(nq, ncols, k);
+}
+
+int csa_topk_from_scores(const float* scores, int64_t ld, const int32_t* valid, int valid_div,
+                         int nq, int64_t ncols, int k, int32_t* idx, float* top_scores, void* ws,
+                         size_t ws_bytes, void* stream) {
+    CSA_TRY(check_k(k));
+    if (nq < 0 || ncols < 0 || ld < ncols || valid_div < 1)
+        return fail(CSA_ERR_INVALID_ARG, "csa_topk_from_scores: bad nq/ncols/ld/valid_div");
+    if (ncols > INT32_MAX) return fail(CSA_ERR_UNSUPPORTED, "ncols beyond int32 indices");
+    if (nq == 0) return CSA_OK;
+    if (ncols > 0) CSA_TRY(check_ptr(scores, "scores"));
+    CSA_TRY(check_ptr(valid, "valid", false));
+    CSA_TRY(check_ptr(idx, "idx"));
+    CSA_TRY(check_ptr(top_scores, "top_scores", false));
+    CSA_TRY(check_ws(ws, ws_bytes, topk_workspace_bytes(nq, ncols, k)));
+    CSA_CUDA(topk_select(scores, ld, valid, valid_div, nq, ncols, k, idx, top_scores, ws,
+                         (cudaStream_t)stream), "csa_topk_from_scores");
+    return CSA_OK;
+}
+
+size_t csa_index_topk_workspace_size(int nq, int64_t Nmax, int k, int dtype) {
+    (void)dtype;
+    if (nq < 0 || Nmax < 0 || k < 1) return 0;
+    return index_topk_bytes(nq, Nmax, k);
+}
+
+int csa_index_topk(const void* qI, const float* w, const void* K, const int32_t* pos,
+                   const int32_t* seq_of_q, int nq, int HI, int cI, int64_t Nmax, int m, int k,
+                   int32_t* idx, float* top_scores, void* ws, size_t ws_bytes, int dtype,
+                   void* stream) {
+    ElemType t;
+    CSA_TRY(check_dtype(dtype, &t));
+    CSA_TRY(check_index_shape(HI, cI));
+    CSA_TRY(check_k(k));
+    if (nq < 0 || Nmax < 0 || m < 1) return fail(CSA_ERR_INVALID_ARG, "bad nq/Nmax/m");
+    if (Nmax > INT32_MAX) return fail(CSA_ERR_UNSUPPORTED, "Nmax beyond int32 entry indices");
+    if (nq == 0) return CSA_OK;
+    CSA_TRY(check_ptr(qI, "qI"));
+    CSA_TRY(check_ptr(w, "w"));
+    CSA_TRY(check_ptr(K, "K", Nmax > 0));
+    CSA_TRY(check_ptr(pos, "pos"));
+    CSA_TRY(check_ptr(seq_of_q, "seq_of_q", false));
+    CSA_TRY(check_ptr(idx, "idx"));
+    CSA_TRY(check_ptr(top_scores, "top_scores", false));
+    CSA_TRY(check_ws(ws, ws_bytes, index_topk_bytes(nq, Nmax, k)));
+    cudaStream_t st = (cudaStream_t)stream;
+    Carve cv(ws);
+    float* sc = (float*)cv.take((size_t)nq * Nmax * sizeof(float));
+    void* tws = cv.take(topk_workspace_bytes(nq, Nmax, k));
+    QuerySpec qs{seq_of_q, pos, 0, 0};
+    CSA_CUDA(index_scores(qI, w, K, qs, nq, HI, cI, Nmax, m, sc, Nmax, t, st), "csa_index_topk: scores");
+    CSA_CUDA(topk_select(sc, Nmax, pos, m, nq, Nmax, k, idx, top_scores, tws, st), "csa_index_topk: top-k");
+    return CSA_OK;
+}
+
+// ---------------------------------------------------------------- a6 / a7
+size_t csa_sparse_mqa_workspace_size(int nq, int H, int c, int k, int dtype) {
+    ElemType t = dtype == CSA_FP32 ? ElemType::F32 : ElemType::BF16;
+    if (nq < 0 || H < 1 || c < 1 || k < 1) return 0;
+    return mqa_workspace_bytes(nq, H, c, k, t);
+}
+
+int csa_sparse_mqa(const void* q, const void* KV, const int32_t* idx, const int32_t* seq_of_q,
+                   int nq, int H, int c, int64_t Nmax, int k, float scale, const float* sink,
+                   void* out, float* lse, void* ws, size_t ws_bytes, int dtype, void* stream) {
+    ElemType t;
+    CSA_TRY(check_dtype(dtype, &t));
+    CSA_TRY(check_attn_shape(H, c));
+    CSA_TRY(check_k(k));
+    if (nq < 0 || Nmax < 0) return fail(CSA_ERR_INVALID_ARG, "bad nq/Nmax");
+    if (nq == 0) return CSA_OK;
+    CSA_TRY(check_ptr(q, "q"));
+    CSA_TRY(check_ptr(KV, "KV", Nmax > 0));
+    CSA_TRY(check_ptr(idx, "idx"));
+    CSA_TRY(check_ptr(seq_of_q, "seq_of_q", false));
+    CSA_TRY(check_ptr(sink, "sink", false));
+    CSA_TRY(check_ptr(out, "out"));
+    CSA_TRY(check_ptr(lse, "lse", false));
+    CSA_TRY(check_ws(ws, ws_bytes, mqa_workspace_bytes(nq, H, c, k, t)));
+    QuerySpec qs{seq_of_q, nullptr, 0, 0};
+    CSA_CUDA(mqa(q, KV, idx, k, qs, 1, nq, H, c, Nmax, default_scale(scale, c), sink, out, lse, ws, t,
+                 (cudaStream_t)stream), "csa_sparse_mqa");
+    return CSA_OK;
+}
+
+size_t hca_dense_mqa_workspace_size(int nq, int H, int c, int64_t Nmax, int dtype) {
+    ElemType t = dtype == CSA_FP32 ? ElemType::F32 : ElemType::BF16;
+    if (nq < 0 || H < 1 || c < 1 || Nmax < 0) return 0;
+    return mqa_workspace_bytes(nq, H, c, Nmax, t);
+}
+
+int hca_dense_mqa(const void* q, const void* KV, const int32_t* pos, const int32_t* seq_of_q,
+                  int nq, int H, int c, int64_t Nmax, int mp, float scale, const float* sink,
+                  void* out, float* lse, void* ws, size_t ws_bytes, int dtype, void* stream) {
+    ElemType t;
+    CSA_TRY(check_dtype(dtype, &t));
+    CSA_TRY(check_attn_shape(H, c));
+    if (nq < 0 || Nmax < 0 || mp < 1) return fail(CSA_ERR_INVALID_ARG, "bad nq/Nmax/mp");
+    if (Nmax > INT32_MAX) return fail(CSA_ERR_UNSUPPORTED, "Nmax beyond int32 entry indices");
+    if (nq == 0) return CSA_OK;
+    CSA_TRY(check_ptr(q, "q"));
+    CSA_TRY(check_ptr(KV, "KV", Nmax > 0));
+    CSA_TRY(check_ptr(pos, "pos"));
+    CSA_TRY(check_ptr(seq_of_q, "seq_of_q", false));
+    CSA_TRY(check_ptr(sink, "sink", false));
+    CSA_TRY(check_ptr(out, "out"));
+    CSA_TRY(check_ptr(lse, "lse", false));
+    CSA_TRY(check_ws(ws, ws_bytes, mqa_workspace_bytes(nq, H, c, Nmax, t)));
+    QuerySpec qs{seq_of_q, pos, 0, 0};
+    CSA_CUDA(mqa(q, KV, nullptr, 0, qs, mp, nq, H, c, Nmax, default_scale(scale, c), sink, out, lse, ws,
+                 t, (cudaStream_t)stream), "hca_dense_mqa");
+    return CSA_OK;
+}
+
+// ---------------------------------------------------------------- fused
+size_t csa_decode_workspace_size(int B, int64_t Nmax, int H, int c, int HI, int cI, int k, int dtype) {
+    (void)HI; (void)cI;
+    ElemType t = dtype == CSA_FP32 ? ElemType::F32 : ElemType::BF16;
+    if (B < 0 || Nmax < 0 || k < 1 || H < 1 || c < 1) return 0;
+    return index_topk_bytes(B, Nmax, k) + align256((size_t)B * k * sizeof(int32_t)) +
+           mqa_workspace_bytes(B, H, c, k, t);
+}
+
+int csa_decode(const void* qI, const float* w, const void* idx_cache, const void* q,
+               const void* kv_cache, const int32_t* ctx_len, int B, int64_t Nmax, int m, int H,
+               int c, int HI, int cI, int k, float scale, const float* sink, void* out, float* lse,
+               int32_t* topk_idx, void* ws, size_t ws_bytes, int dtype, void* stream) {
+    ElemType t;
+    CSA_TRY(check_dtype(dtype, &t));
+    CSA_TRY(check_index_shape(HI, cI));
+    CSA_TRY(check_attn_shape(H, c));
+    CSA_TRY(check_k(k));
+    if (B < 0 || Nmax < 0 || m < 1) return fail(CSA_ERR_INVALID_ARG, "bad B/Nmax/m");
+    if (Nmax > INT32_MAX) return fail(CSA_ERR_UNSUPPORTED, "Nmax beyond int32 entry indices");
+    if (B == 0) return CSA_OK;
+    CSA_TRY(check_ptr(qI, "qI"));
+    CSA_TRY(check_ptr(w, "w"));
+    CSA_TRY(check_ptr(idx_cache, "idx_cache", Nmax > 0));
+    CSA_TRY(check_ptr(q, "q"));
+    CSA_TRY(check_ptr(kv_cache, "kv_cache", Nmax > 0));
+    CSA_TRY(check_ptr(ctx_len, "ctx_len"));
+    CSA_TRY(check_ptr(sink, "sink", false));
+    CSA_TRY(check_ptr(out, "out"));
+    CSA_TRY(check_ptr(lse, "lse", false));
+    CSA_TRY(check_ptr(topk_idx, "topk_idx", false));
+    CSA_TRY(check_ws(ws, ws_bytes, csa_decode_workspace_size(B, Nmax, H, c, HI, cI, k, dtype)));
+    cudaStream_t st = (cudaStream_t)stream;
+    Carve cv(ws);
+    float* sc = (float*)cv.take((size_t)B * Nmax * sizeof(float));
+    void* tws = cv.take(topk_workspace_bytes(B, Nmax, k));
+    int32_t* sel = (int32_t*)cv.take((size_t)B * k * sizeof(int32_t));
+    void* mws = cv.take(mqa_workspace_bytes(B, H, c, k, t));
+    if (topk_idx) sel = topk_idx;
+    QuerySpec qs{nullptr, ctx_len, 0, 0};
+    CSA_CUDA(index_scores(qI, w, idx_cache, qs, B, HI, cI, Nmax, m, sc, Nmax, t, st), "csa_decode: indexer");
+    CSA_CUDA(topk_select(sc, Nmax, ctx_len, m, B, Nmax, k, sel, nullptr, tws, st), "csa_decode: top-k");
+    CSA_CUDA(mqa(q, kv_cache, sel, k, qs, 1, B, H, c, Nmax, default_scale(scale, c), sink, out, lse, mws, t, st),
+             "csa_decode: mqa");
+    return CSA_OK;
+}
+
+size_t hca_decode_workspace_size(int B, int64_t Nmax, int H, int c, int dtype) {
+    return hca_dense_mqa_workspace_size(B, H, c, Nmax, dtype);
+}
+
+int hca_decode(const void* q, const void* kv_cache, const int32_t* ctx_len, int B, int64_t Nmax,
+               int mp, int H, int c, float scale, const float* sink, void* out, float* lse,
+               void* ws, size_t ws_bytes, int dtype, void* stream) {
+    return hca_dense_mqa(q, kv_cache, ctx_len, nullptr, B, H, c, Nmax, mp, scale, sink, out, lse, ws,
+                         ws_bytes, dtype, stream);
+}
+
+size_t csa_prefill_workspace_size(int64_t n, int64_t Nmax, int d, int m, int c, int cI, int H,
+                                  int HI, int k, int dtype) {
+    (void)d; (void)HI;
+    ElemType t = dtype == CSA_FP32 ? ElemType::F32 : ElemType::BF16;
+    if (n < 0 || Nmax < 0 || m < 1 || c < 1 || cI < 1 || k < 1) return 0;
+    const int cw = c > cI ? c : cI;
+    int64_t qc = prefill_query_chunk(n, Nmax);
+    size_t b = align256((size_t)n * 4 * cw * sizeof(float)) + align256((size_t)m * 4 * cw * sizeof(float));
+    b += index_topk_bytes((int)qc, Nmax, k) + align256((size_t)qc * k * sizeof(int32_t));
+    b += mqa_workspace_bytes((int)qc, H, c, k, t);
+    return b;
+}
+
+int csa_prefill(const void* x, const void* x_left, const void* W_kv, const float* B_kv,
+                const void* W_idx, const float* B_idx, int64_t start, int64_t n, int d, int m,
+                int c, int cI, void* kv_cache, void* idx_cache, int64_t Nmax, const void* qI,
+                const float* w, const void* q, int H, int HI, int k, float scale,
+                const float* sink, void* out, float* lse, int32_t* topk_idx, void* ws,
+                size_t ws_bytes, int dtype, void* stream) {
+    ElemType t;
+    CSA_TRY(check_dtype(dtype, &t));
+    CSA_TRY(check_index_shape(HI, cI));
+    CSA_TRY(check_attn_shape(H, c));
+    CSA_TRY(check_k(k));
+    CSA_TRY(check_compress(n, c, m, 64, "csa_prefill"));
+    if (d < 8 || d % 8) return fail(CSA_ERR_INVALID_ARG, "d=%d must be a positive multiple of 8", d);
+    if (start < 0 || start % m) return fail(CSA_ERR_INVALID_ARG, "start=%lld is not a non-negative multiple of m", (long long)start);
+    if (start > 0 && !x_left) return fail(CSA_ERR_INVALID_ARG, "x_left is required when start > 0");
+    if ((start + n) / m > Nmax) return fail(CSA_ERR_INVALID_ARG, "caches hold %lld entries, %lld needed",
+                                            (long long)Nmax, (long long)((start + n) / m));
+    if (Nmax > INT32_MAX || start + n > INT32_MAX) return fail(CSA_ERR_UNSUPPORTED, "positions beyond int32");
+    if (n == 0) return CSA_OK;
+    CSA_TRY(check_ptr(x, "x"));
+    CSA_TRY(check_ptr(x_left, "x_left", false));
+    CSA_TRY(check_ptr(W_kv, "W_kv"));
+    CSA_TRY(check_ptr(B_kv, "B_kv"));
+    CSA_TRY(check_ptr(W_idx, "W_idx"));
+    CSA_TRY(check_ptr(B_idx, "B_idx"));
+    CSA_TRY(check_ptr(kv_cache, "kv_cache"));
+    CSA_TRY(check_ptr(idx_cache, "idx_cache"));
+    CSA_TRY(check_ptr(qI, "qI"));
+    CSA_TRY(check_ptr(w, "w"));
+    CSA_TRY(check_ptr(q, "q"));
+    CSA_TRY(check_ptr(sink, "sink", false));
+    CSA_TRY(check_ptr(out, "out"));
+    CSA_TRY(check_ptr(lse, "lse", false));
+    CSA_TRY(check_ptr(topk_idx, "topk_idx", false));
+    CSA_TRY(check_ws(ws, ws_bytes, csa_prefill_workspace_size(n, Nmax, d, m, c, cI, H, HI, k, dtype)));
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t es = elem_size(t);
+    const int cw = c > cI ? c : cI;
+    const int64_t qc = prefill_query_chunk(n, Nmax);
+    Carve cv(ws);
+    float* proj = (float*)cv.take((size_t)n * 4 * cw * sizeof(float));
+    float* lproj = (float*)cv.take((size_t)m * 4 * cw * sizeof(float));
+    float* sc = (float*)cv.take((size_t)qc * Nmax * sizeof(float));
+    void* tws = cv.take(topk_workspace_bytes((int)qc, Nmax, k));
+    int32_t* sel_ws = (int32_t*)cv.take((size_t)qc * k * sizeof(int32_t));
+    void* mws = cv.take(mqa_workspace_bytes((int)qc, H, c, k, t));
+
+    // 1-2. compress the chunk into both caches (entries start/m ..)
+    const int64_t e0 = start / m;
+    struct { const void* W; const float* B; int cc; void* cache; } streams[2] = {
+        {W_kv, B_kv, c, kv_cache}, {W_idx, B_idx, cI, idx_cache}};
+    for (auto& s : streams) {
+        CSA_CUDA(project(x, s.W, n, d, 4 * s.cc, proj, t, st), "csa_prefill: projection");
+        if (start > 0) CSA_CUDA(project(x_left, s.W, m, d, 4 * s.cc, lproj, t, st), "csa_prefill: left projection");
+        CSA_CUDA(compress_csa(proj, start > 0 ? lproj : nullptr, s.B, n, s.cc, m,
+                              (char*)s.cache + (size_t)e0 * s.cc * es, ElemType::F32, t, st),
+                 "csa_prefill: compress");
+    }
+    // 3. indexer -> top-k -> sparse MQA per query chunk
+    const float sc_scale = default_scale(scale, c);
+    for (int64_t q0 = 0; q0 < n; q0 += qc) {
+        const int nqc = (int)((n - q0) < qc ? (n - q0) : qc);
+        QuerySpec qs{nullptr, nullptr, start + q0, 1};
+        int32_t* sel = topk_idx ? topk_idx + q0 * k : sel_ws;
+        CSA_CUDA(index_scores((const char*)qI + (size_t)q0 * HI * cI * es, w + q0 * HI, idx_cache, qs, nqc, HI,
+                              cI, Nmax, m, sc, Nmax, t, st), "csa_prefill: indexer");
+        // visible count of query t is floor((start + q0 + t) / m); pass it through a
+        // position-based valid rule: the top-k kernel reads valid[] = positions
+        CSA_CUDA(topk_select_positions(sc, Nmax, start + q0, m, nqc, Nmax, k, sel, tws, st), "csa_prefill: top-k");
+        CSA_CUDA(mqa((const char*)q + (size_t)q0 * H * c * es, kv_cache, sel, k, qs, 1, nqc, H, c, Nmax,
+                     sc_scale, sink, (char*)out + (size_t)q0 * H * c * es, lse ? lse + q0 * H : nullptr, mws,
+                     t, st), "csa_prefill: mqa");
+    }
+    return CSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,90 @@
+// Shared device helpers for libcsa (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace csa {
+
+using bf16 = __nv_bfloat16;
+
+// Kernels that give up on a bounded wait record an error code in the
+// library's device status word (passed to them as a pointer; first writer
+// wins) instead of trapping; csa_poll_status() reads it back.
+__device__ __forceinline__ void report_device_error(int* status, int code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+// ---- element conversion -------------------------------------------------
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(bf16 v) { return __bfloat162float(v); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ bf16 from_f32<bf16>(float v) { return __float2bfloat16_rn(v); }
+
+// Load 8 consecutive elements (16-byte aligned for bf16, 32-byte for fp32)
+// as fp32.
+__device__ __forceinline__ void load8(const bf16* p, float (&v)[8]) {
+    uint4 u = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 f = __bfloat1622float2(h[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+    float4 a = *reinterpret_cast<const float4*>(p);
+    float4 b = *reinterpret_cast<const float4*>(p + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+__device__ __forceinline__ void store8(bf16* p, const float (&v)[8]) {
+    uint4 u;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    *reinterpret_cast<uint4*>(p) = u;
+}
+__device__ __forceinline__ void store8(float* p, const float (&v)[8]) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4*>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// Query -> sequence and query -> position lookups shared by the attention
+// kernels. seq: explicit array, else identity (decode: query b reads
+// sequence b), else all queries on sequence 0 (prefill of one sequence).
+struct QueryMap {
+    const int32_t* seq;    // nullable
+    const int32_t* pos;    // nullable: then pos = pos_base + t
+    int64_t pos_base;
+    int single_seq;        // 1: every query reads sequence 0
+    __device__ __forceinline__ int seq_of(int t) const {
+        return seq ? seq[t] : (single_seq ? 0 : t);
+    }
+    __device__ __forceinline__ int64_t pos_of(int t) const {
+        return pos ? (int64_t)pos[t] : pos_base + t;
+    }
+};
+
+__device__ __forceinline__ int64_t visible_entries(int64_t pos, int m, int64_t nmax) {
+    int64_t v = pos < 0 ? 0 : pos / m;
+    return v < nmax ? v : nmax;
+}
+
+}  // namespace csa

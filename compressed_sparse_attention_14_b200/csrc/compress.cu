@@ -1,0 +1,158 @@
+// CSA / HCA token compressors on projected inputs.
+//
+// CSA [Notes §1.1, equation C^Comp_i]: entry i mixes the a-stream of its own
+// m tokens and the b-stream of the previous block's m tokens with ONE
+// softmax per channel over the 2m logits Z + B (positional bias).
+// HCA [Notes §1.2, comparison table]: one non-overlapping window of m' tokens.
+//
+// ([Notes] = "DeepSeek-V4: 迈向高效百万级上下文智能", study notes on the DeepSeek-V4
+// report, notes.kuangjux.top.)
+//
+// HBM-bound elementwise work: one thread owns (entry, 8 channels), reads each
+// projected row of its window with 16-byte vector loads (consecutive threads
+// take consecutive channel groups, so a warp reads 512 contiguous bytes of
+// bf16), runs the windowed softmax online in registers and writes 8 output
+// channels with one vector store. Every projected element is read once.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace csa {
+
+struct OnlineSoftmax8 {
+    float mx[8], den[8], acc[8];
+    __device__ __forceinline__ void init() {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) { mx[u] = -INFINITY; den[u] = 0.f; acc[u] = 0.f; }
+    }
+    __device__ __forceinline__ void push(const float (&logit)[8], const float (&val)[8]) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            float nm = fmaxf(mx[u], logit[u]);
+            float keep = expf(mx[u] - nm);   // 0 for the first push (mx = -inf)
+            float p = expf(logit[u] - nm);
+            den[u] = den[u] * keep + p;
+            acc[u] = acc[u] * keep + p * val[u];
+            mx[u] = nm;
+        }
+    }
+};
+
+template <typename TIn, typename TOut>
+__global__ void __launch_bounds__(256) csa_compress_kernel(const TIn* __restrict__ proj,
+                                                           const TIn* __restrict__ left,
+                                                           const float* __restrict__ bias,
+                                                           int64_t nb, int c, int m,
+                                                           TOut* __restrict__ out) {
+    const int groups = c / 8;
+    int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= nb * groups) return;
+    const int64_t i = gid / groups;
+    const int j = (int)(gid % groups) * 8;
+    const int64_t ld = 4 * (int64_t)c;
+
+    OnlineSoftmax8 sm;
+    sm.init();
+    float z[8], b[8], v[8];
+    // a-window: tokens m*i .. m*i+m-1, C^a and Z^a, bias rows 0..m-1
+    for (int r = 0; r < m; ++r) {
+        const TIn* row = proj + (m * i + r) * ld;
+        load8(row + 2 * c + j, z);
+        load8(bias + (int64_t)r * c + j, b);
+        load8(row + j, v);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) z[u] += b[u];
+        sm.push(z, v);
+    }
+    // b-window: tokens m*(i-1) .. m*i-1, C^b and Z^b, bias rows m..2m-1;
+    // absent for block 0 at the start of a sequence
+    if (i > 0 || left != nullptr) {
+        for (int r = 0; r < m; ++r) {
+            const TIn* row = (i > 0) ? proj + (m * (i - 1) + r) * ld : left + (int64_t)r * ld;
+            load8(row + 3 * c + j, z);
+            load8(bias + (int64_t)(m + r) * c + j, b);
+            load8(row + c + j, v);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) z[u] += b[u];
+            sm.push(z, v);
+        }
+    }
+    float o[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) o[u] = sm.acc[u] / sm.den[u];
+    if constexpr (sizeof(TOut) == 2) store8(reinterpret_cast<bf16*>(out + i * c + j), o);
+    else store8(reinterpret_cast<float*>(out + i * c + j), o);
+}
+
+template <typename TIn, typename TOut>
+__global__ void __launch_bounds__(256) hca_compress_kernel(const TIn* __restrict__ proj,
+                                                           const float* __restrict__ bias,
+                                                           int64_t nb, int c, int mp,
+                                                           TOut* __restrict__ out) {
+    const int groups = c / 8;
+    int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= nb * groups) return;
+    const int64_t i = gid / groups;
+    const int j = (int)(gid % groups) * 8;
+    const int64_t ld = 2 * (int64_t)c;
+
+    OnlineSoftmax8 sm;
+    sm.init();
+    float z[8], b[8], v[8];
+#pragma unroll 4
+    for (int r = 0; r < mp; ++r) {
+        const TIn* row = proj + (mp * i + r) * ld;
+        load8(row + c + j, z);
+        load8(bias + (int64_t)r * c + j, b);
+        load8(row + j, v);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) z[u] += b[u];
+        sm.push(z, v);
+    }
+    float o[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) o[u] = sm.acc[u] / sm.den[u];
+    if constexpr (sizeof(TOut) == 2) store8(reinterpret_cast<bf16*>(out + i * c + j), o);
+    else store8(reinterpret_cast<float*>(out + i * c + j), o);
+}
+
+template <typename TIn, typename TOut>
+cudaError_t launch_csa_compress(const void* proj, const void* left, const float* bias, int64_t n,
+                                int c, int m, void* out, cudaStream_t st) {
+    int64_t nb = n / m;
+    int64_t threads = nb * (c / 8);
+    if (threads == 0) return cudaSuccess;
+    CSA_LAUNCH(st, "csa_compress", csa_compress_kernel<TIn, TOut><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
+        (const TIn*)proj, (const TIn*)left, bias, nb, c, m, (TOut*)out));
+    return cudaGetLastError();
+}
+
+template <typename TIn, typename TOut>
+cudaError_t launch_hca_compress(const void* proj, const float* bias, int64_t n, int c, int mp,
+                                void* out, cudaStream_t st) {
+    int64_t nb = n / mp;
+    int64_t threads = nb * (c / 8);
+    if (threads == 0) return cudaSuccess;
+    CSA_LAUNCH(st, "hca_compress", hca_compress_kernel<TIn, TOut><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
+        (const TIn*)proj, bias, nb, c, mp, (TOut*)out));
+    return cudaGetLastError();
+}
+
+cudaError_t compress_csa(const void* proj, const void* left, const float* bias, int64_t n, int c,
+                         int m, void* out, ElemType in_t, ElemType out_t, cudaStream_t st) {
+    if (in_t == ElemType::BF16 && out_t == ElemType::BF16)
+        return launch_csa_compress<bf16, bf16>(proj, left, bias, n, c, m, out, st);
+    if (in_t == ElemType::F32 && out_t == ElemType::BF16)
+        return launch_csa_compress<float, bf16>(proj, left, bias, n, c, m, out, st);
+    return launch_csa_compress<float, float>(proj, left, bias, n, c, m, out, st);
+}
+
+cudaError_t compress_hca(const void* proj, const float* bias, int64_t n, int c, int mp, void* out,
+                         ElemType in_t, ElemType out_t, cudaStream_t st) {
+    if (in_t == ElemType::BF16 && out_t == ElemType::BF16)
+        return launch_hca_compress<bf16, bf16>(proj, bias, n, c, mp, out, st);
+    if (in_t == ElemType::F32 && out_t == ElemType::BF16)
+        return launch_hca_compress<float, bf16>(proj, bias, n, c, mp, out, st);
+    return launch_hca_compress<float, float>(proj, bias, n, c, mp, out, st);
+}
+
+}  // namespace csa

@@ -1,0 +1,70 @@
+// Internal launchers of libcsa (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/csa.h"
+
+namespace csa {
+
+enum class ElemType { BF16 = 0, F32 = 1 };
+
+// trace.cu: launch accounting and optional per-kernel event timing. Every
+// kernel launch goes through CSA_LAUNCH(stream, "name", kernel<<<...>>>(...)).
+int trace_begin(cudaStream_t st);
+void trace_end(int token, cudaStream_t st, const char* name);
+uint64_t launch_count();
+void trace_enable(int on);
+int trace_read(int max_kernels, char* names, double* total_ms, int* counts, int* n_out);
+
+#define CSA_LAUNCH(st, name, ...)                  \
+    do {                                           \
+        int _csa_tok = ::csa::trace_begin(st);     \
+        __VA_ARGS__;                               \
+        ::csa::trace_end(_csa_tok, st, name);      \
+    } while (0)
+
+inline size_t elem_size(ElemType t) { return t == ElemType::BF16 ? 2 : 4; }
+inline size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+// Query -> (sequence, position) description passed to attention launchers.
+struct QuerySpec {
+    const int32_t* seq;   // nullable
+    const int32_t* pos;   // nullable: then pos = pos_base + t
+    int64_t pos_base;
+    int single_seq;
+};
+
+// compress.cu
+cudaError_t compress_csa(const void* proj, const void* left, const float* bias, int64_t n, int c,
+                         int m, void* out, ElemType in_t, ElemType out_t, cudaStream_t st);
+cudaError_t compress_hca(const void* proj, const float* bias, int64_t n, int c, int mp, void* out,
+                         ElemType in_t, ElemType out_t, cudaStream_t st);
+
+// gemm.cu: out[n, M] (fp32) = x[n, d] . W[M, d]^T
+cudaError_t project(const void* x, const void* W, int64_t n, int d, int M, float* out, ElemType t,
+                    cudaStream_t st);
+
+// indexer.cu: scores[t, 0..Nmax) with ld = ld_scores; -inf past the visible range
+cudaError_t index_scores(const void* qI, const float* w, const void* K, QuerySpec qs, int nq,
+                         int HI, int cI, int64_t Nmax, int m, float* scores, int64_t ld_scores,
+                         ElemType t, cudaStream_t st);
+
+// topk.cu
+size_t topk_workspace_bytes(int nq, int64_t ncols, int k);
+cudaError_t topk_select(const float* scores, int64_t ld, const int32_t* valid, int valid_div,
+                        int nq, int64_t ncols, int k, int32_t* idx, float* top_scores, void* ws,
+                        cudaStream_t st);
+// as topk_select with the candidate count of row t = (pos_base + t) / m
+cudaError_t topk_select_positions(const float* scores, int64_t ld, int64_t pos_base, int m, int nq,
+                                  int64_t ncols, int k, int32_t* idx, void* ws, cudaStream_t st);
+
+// mqa.cu: sparse (idx != nullptr) or dense (entries s < pos/mp) shared-KV MQA
+size_t mqa_workspace_bytes(int nq, int H, int c, int64_t max_entries, ElemType t);
+cudaError_t mqa(const void* q, const void* KV, const int32_t* idx, int k, QuerySpec qs, int mp,
+                int nq, int H, int c, int64_t Nmax, float scale, const float* sink, void* out,
+                float* lse, void* ws, ElemType t, cudaStream_t st);
+
+}  // namespace csa

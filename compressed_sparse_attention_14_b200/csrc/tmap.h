@@ -1,0 +1,18 @@
+// Host-side TMA tensor-map encoding for libcsa. cuTensorMapEncodeTiled is
+// reached through the runtime's driver entry point, so the library does not
+// link libcuda directly.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace csa {
+
+// Row-major bf16 matrix [rows, cols] (cols contiguous, row pitch `pitch_elems`)
+// viewed as 2D tiles of box_rows x box_cols (box_cols * 2 <= 128 bytes) with
+// 128-byte swizzle. Returns false if the driver rejects the map.
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t pitch_elems,
+                       uint32_t box_rows, uint32_t box_cols);
+
+}  // namespace csa

@@ -1,0 +1,248 @@
+/*
+ * csa.h — C ABI of libcsa: the DeepSeek-V4 compressed attention hot path
+ * (CSA: overlapping token compressor, lightning indexer, top-k selection and
+ * shared-KV MQA over the selected entries; HCA: non-overlapping heavy
+ * compression and dense shared-KV MQA) for NVIDIA B200 (sm_100a).
+ *
+ * Sources, cited by page title and section:
+ *   [Notes] "DeepSeek-V4: 迈向高效百万级上下文智能" — study notes on the
+ *           DeepSeek-V4 report (notes.kuangjux.top): §1.1 CSA (compressor and
+ *           indexer equations), §1.2 HCA (comparison table), §1.3 (sink
+ *           equation), model configuration table.
+ *   [Walk]  mlpod.com walk-through of "DeepSeek-V4: Towards Highly Efficient
+ *           Million-Token Context Intelligence": §2.3.1 CSA, §2.3.2 HCA and
+ *           MQA, §2.3.3 attention details (causality, sink).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Every pointer argument is a DEVICE pointer owned by the caller, unless
+ *    stated otherwise, 16-byte aligned. The library never allocates device
+ *    memory; calls that need scratch take a caller-provided workspace `ws`
+ *    of at least the size returned by the matching *_workspace_size query.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream) and does not synchronize.
+ *  - Arrays are dense and row-major with the shapes given in brackets.
+ *  - dtype selects the storage type of activations, weights, caches and
+ *    outputs: CSA_BF16 (bfloat16; fp32 accumulation) or CSA_FP32 (fp32 in
+ *    and out, fp32 arithmetic). Biases, indexer head weights `w`, sink
+ *    logits, scores and lse are always fp32; indices are int32.
+ *  - Return value: CSA_OK, or an error code with a message readable through
+ *    csa_last_error() on the calling thread. Argument errors are found on the
+ *    host before anything is launched, so nothing is written on error.
+ *  - Positions are 0-based token positions. A query at position p sees
+ *    compressed entry s iff s < floor(p / m) (m' for HCA): it sees only
+ *    blocks that end at or before it [Walk §2.3.3 item 3; Walk §2.3.1].
+ */
+#ifndef CSA_H_
+#define CSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CSA_ABI_VERSION 1
+
+enum csa_status {
+    CSA_OK = 0,
+    CSA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size or shape   */
+    CSA_ERR_UNSUPPORTED = 2,  /* shape outside what the kernels implement     */
+    CSA_ERR_WORKSPACE = 3,    /* ws missing or smaller than the query's size  */
+    CSA_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed         */
+    CSA_ERR_TIMEOUT = 5       /* a device-side wait hit its bound             */
+};
+
+enum csa_dtype { CSA_BF16 = 0, CSA_FP32 = 1 };
+
+/* Limits of this build (checked; larger values give CSA_ERR_UNSUPPORTED). */
+#define CSA_MAX_TOPK 2048
+#define CSA_MAX_HEADS 128
+#define CSA_MAX_HEAD_DIM 512
+#define CSA_MAX_INDEX_HEADS 64
+#define CSA_MAX_INDEX_DIM 256
+
+/* Message of the last failing call on this thread ("" if none). The string
+ * is owned by the library and valid until the next call on this thread. */
+const char* csa_last_error(void);
+int csa_abi_version(void);
+
+/* Number of kernels this library has launched in this process (all devices,
+ * all threads). Lets a caller count the launches inside a timed region. */
+uint64_t csa_launch_count(void);
+
+/* Per-kernel device timing (tracing). While enabled, every kernel launch is
+ * bracketed by CUDA events recorded on the launching stream. Enabling (or
+ * disabling) discards the records gathered so far. */
+void csa_trace_enable(int on);
+/* Waits for the recorded events and aggregates them per kernel name:
+ * names [max_kernels][64] (NUL-terminated), total_ms [max_kernels] (sum of
+ * device times), counts [max_kernels] (launches); *n_kernels receives the
+ * number of distinct kernels written. Host pointers. */
+int csa_trace_read(int max_kernels, char* names, double* total_ms, int* counts, int* n_kernels);
+
+/* Device-side status word: the first CSA_ERR_TIMEOUT (or other device error)
+ * raised by a kernel since the last reset. Synchronizes `stream`. Returns
+ * CSA_OK when no kernel reported an error; resets the word when `reset`. */
+int csa_poll_status(void* stream, int reset);
+
+/* ------------------------------------------------------------------------
+ * a1. Projection [Walk §2.3.1 "KV compression": the KV streams and their
+ * compression weights are learnable linear maps of the hidden state H].
+ *   out[t][o] = sum_k x[t][k] * W[o][k]
+ * x [n, d], W [M, d] (one row per output feature, i.e. nn.Linear layout),
+ * out [n, M] always fp32. n >= 0, d % 8 == 0, M % 8 == 0.
+ * ------------------------------------------------------------------------ */
+int csa_project(const void* x, const void* W, int64_t n, int d, int M, float* out, int dtype,
+                void* stream);
+
+/* ------------------------------------------------------------------------
+ * a2. CSA overlapping compressor [Notes §1.1, equation C^Comp_i and the
+ * sentence after it]. Per block i and channel j, ONE softmax over the 2m
+ * logits Z^a[mi+r][j] + B[r][j] and Z^b[m(i-1)+r][j] + B[m+r][j] (r < m),
+ * then out[i][j] = sum S^a C^a[mi+r][j] + sum S^b C^b[m(i-1)+r][j].
+ *   proj [n, 4c]: each row C^a | C^b | Z^a | Z^b (dtype)
+ *   left [m, 4c]: the m projected rows just before this chunk, or NULL at
+ *                 the start of a sequence (block 0 then has no b-window)
+ *   bias [2m, c] fp32: rows 0..m-1 pair with the a-window, m..2m-1 with b
+ *   out  [n/m, c] (dtype), written in full.
+ * n % m == 0, c % 8 == 0, 1 <= m <= 64.
+ * ------------------------------------------------------------------------ */
+int csa_compress(const void* proj, const void* left, const float* bias, int64_t n, int c, int m,
+                 void* out, int dtype, void* stream);
+
+/* a3. HCA compressor [Notes §1.2 and its comparison table; Walk §2.3.2]:
+ * per block i of mp tokens, one softmax per channel over Z[i*mp+r][j] +
+ * B'[r][j], out[i][j] = sum_r S_r C[i*mp+r][j]; no overlap.
+ *   proj [n, 2c]: rows C | Z (dtype); bias [mp, c] fp32; out [n/mp, c].
+ * n % mp == 0, c % 8 == 0, 1 <= mp <= 1024. */
+int hca_compress(const void* proj, const float* bias, int64_t n, int c, int mp, void* out,
+                 int dtype, void* stream);
+
+/* a1+a2 fused: projection of the hidden states then CSA compression.
+ *   x [n, d], x_left [m, d] or NULL (sequence start), W [4c, d] packing the
+ *   a-KV, b-KV, a-weight and b-weight maps (rows 0..c-1, c..2c-1, ...),
+ *   bias [2m, c], out [n/m, c]. */
+size_t csa_compress_from_hidden_workspace_size(int64_t n, int d, int c, int m, int dtype);
+int csa_compress_from_hidden(const void* x, const void* x_left, const void* W, const float* bias,
+                             int64_t n, int d, int c, int m, void* out, void* ws, size_t ws_bytes,
+                             int dtype, void* stream);
+
+/* a1+a3 fused: x [n, d], W [2c, d] (C map rows then Z map rows), bias
+ * [mp, c], out [n/mp, c]. */
+size_t hca_compress_from_hidden_workspace_size(int64_t n, int d, int c, int mp, int dtype);
+int hca_compress_from_hidden(const void* x, const void* W, const float* bias, int64_t n, int d,
+                             int c, int mp, void* out, void* ws, size_t ws_bytes, int dtype,
+                             void* stream);
+
+/* ------------------------------------------------------------------------
+ * a4. Lightning indexer [Notes §1.1, equation I_{t,s}; Walk §2.3.1]:
+ *   scores[t][s] = sum_h w[t][h] * ReLU(qI[t][h] . K[seq_t][s]),
+ *   for s < floor(pos[t] / m); columns s >= that are set to -inf.
+ *   qI [nq, HI, cI] (dtype), w [nq, HI] fp32, K [B, Nmax, cI] (dtype),
+ *   pos [nq] int32, seq_of_q [nq] int32 or NULL (query t reads sequence t),
+ *   scores [nq, Nmax] fp32.
+ * cI % 8 == 0, cI <= CSA_MAX_INDEX_DIM, HI <= CSA_MAX_INDEX_HEADS.
+ * ------------------------------------------------------------------------ */
+int csa_index_scores(const void* qI, const float* w, const void* K, const int32_t* pos,
+                     const int32_t* seq_of_q, int nq, int HI, int cI, int64_t Nmax, int m,
+                     float* scores, int dtype, void* stream);
+
+/* a5. Top-k selection [Walk §2.3.1: the k highest-scoring compressed blocks
+ * are kept; Notes model table: k = 512 / 1024]. Row t's candidates are
+ * columns 0 .. min(valid[t] / valid_div, ncols) - 1 of scores (row stride
+ * ld floats). Output idx [nq, k]: the min(k, candidates) best, ordered by
+ * (score descending, column ascending), padded with -1; top_scores [nq, k]
+ * (NULL allowed) gets their scores, -inf in padded slots. Deterministic and
+ * bit-exact: equal scores are resolved by the lower column. -0.0 == +0.0.
+ * 1 <= k <= CSA_MAX_TOPK. */
+size_t csa_topk_workspace_size(int nq, int64_t ncols, int k);
+int csa_topk_from_scores(const float* scores, int64_t ld, const int32_t* valid, int valid_div,
+                         int nq, int64_t ncols, int k, int32_t* idx, float* top_scores, void* ws,
+                         size_t ws_bytes, void* stream);
+
+/* a4+a5: indexer then top-k over the visible entries of each query. */
+size_t csa_index_topk_workspace_size(int nq, int64_t Nmax, int k, int dtype);
+int csa_index_topk(const void* qI, const float* w, const void* K, const int32_t* pos,
+                   const int32_t* seq_of_q, int nq, int HI, int cI, int64_t Nmax, int m, int k,
+                   int32_t* idx, float* top_scores, void* ws, size_t ws_bytes, int dtype,
+                   void* stream);
+
+/* ------------------------------------------------------------------------
+ * a6. Sparse shared-KV MQA [Notes §1.1 last paragraph: every compressed
+ * entry is both key and value, all query heads share it; Walk §2.3.2; sink
+ * from Notes §1.3 equation s_{h,i,j}]:
+ *   z_s = scale * q[t][h] . KV[seq_t][s] for s in idx[t][0..k) (-1 = none),
+ *   out[t][h] = sum_s exp(z_s) KV[s] / (sum_s exp(z_s) + exp(sink[h])),
+ *   lse[t][h] = log of that denominator (-inf for an empty set, no sink).
+ *   q [nq, H, c] (dtype), KV [B, Nmax, c] (dtype), idx [nq, k] int32,
+ *   seq_of_q [nq] or NULL (identity), sink [H] fp32 or NULL (no sink term),
+ *   out [nq, H, c] (dtype), lse [nq, H] fp32 or NULL.
+ *   scale == 0 selects 1/sqrt(c).
+ * c % 8 == 0, c <= CSA_MAX_HEAD_DIM, H <= CSA_MAX_HEADS, k <= CSA_MAX_TOPK.
+ * ------------------------------------------------------------------------ */
+size_t csa_sparse_mqa_workspace_size(int nq, int H, int c, int k, int dtype);
+int csa_sparse_mqa(const void* q, const void* KV, const int32_t* idx, const int32_t* seq_of_q,
+                   int nq, int H, int c, int64_t Nmax, int k, float scale, const float* sink,
+                   void* out, float* lse, void* ws, size_t ws_bytes, int dtype, void* stream);
+
+/* a7. Dense shared-KV MQA over every visible HCA entry [Walk §2.3.2: after
+ * heavy compression full attention is affordable; Notes §1.2 table]: as a6
+ * with the entry set s < floor(pos[t] / mp). */
+size_t hca_dense_mqa_workspace_size(int nq, int H, int c, int64_t Nmax, int dtype);
+int hca_dense_mqa(const void* q, const void* KV, const int32_t* pos, const int32_t* seq_of_q,
+                  int nq, int H, int c, int64_t Nmax, int mp, float scale, const float* sink,
+                  void* out, float* lse, void* ws, size_t ws_bytes, int dtype, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Fused steps.
+ *
+ * csa_decode: one decode query per sequence b against its cached entries:
+ * indexer (a4) over idx_cache[b][0 .. floor(ctx_len[b]/m)), top-k (a5),
+ * sparse MQA (a6) over kv_cache[b]. The query position is ctx_len[b].
+ *   qI [B, HI, cI], w [B, HI], idx_cache [B, Nmax, cI], q [B, H, c],
+ *   kv_cache [B, Nmax, c], ctx_len [B] int32 (device), out [B, H, c],
+ *   lse [B, H] or NULL, topk_idx [B, k] or NULL (selected entries).
+ * ------------------------------------------------------------------------ */
+size_t csa_decode_workspace_size(int B, int64_t Nmax, int H, int c, int HI, int cI, int k,
+                                 int dtype);
+int csa_decode(const void* qI, const float* w, const void* idx_cache, const void* q,
+               const void* kv_cache, const int32_t* ctx_len, int B, int64_t Nmax, int m, int H,
+               int c, int HI, int cI, int k, float scale, const float* sink, void* out, float* lse,
+               int32_t* topk_idx, void* ws, size_t ws_bytes, int dtype, void* stream);
+
+/* hca_decode: dense MQA (a7) of query b over kv_cache[b][0 .. floor(ctx_len[b]/mp)). */
+size_t hca_decode_workspace_size(int B, int64_t Nmax, int H, int c, int dtype);
+int hca_decode(const void* q, const void* kv_cache, const int32_t* ctx_len, int B, int64_t Nmax,
+               int mp, int H, int c, float scale, const float* sink, void* out, float* lse,
+               void* ws, size_t ws_bytes, int dtype, void* stream);
+
+/* csa_prefill: one chunk of n new tokens of ONE sequence at positions
+ * start .. start+n-1 (start % m == 0, n % m == 0):
+ *   1. compress the chunk's KV entries (a1+a2 with W_kv [4c, d], B_kv
+ *      [2m, c]) into kv_cache rows start/m .. (start+n)/m - 1;
+ *   2. the same for the indexer keys (W_idx [4cI, d], B_idx [2m, cI]) into
+ *      idx_cache;
+ *   3. for each new token t: indexer over the visible entries, top-k, and
+ *      sparse MQA over kv_cache.
+ *   x [n, d], x_left [m, d] (the m hidden rows before the chunk; NULL when
+ *   start == 0), kv_cache [Nmax, c] and idx_cache [Nmax, cI] with
+ *   Nmax >= (start+n)/m (rows before start/m already filled by earlier
+ *   chunks), qI [n, HI, cI], w [n, HI], q [n, H, c], out [n, H, c],
+ *   lse [n, H] or NULL, topk_idx [n, k] or NULL.
+ * ------------------------------------------------------------------------ */
+size_t csa_prefill_workspace_size(int64_t n, int64_t Nmax, int d, int m, int c, int cI, int H,
+                                  int HI, int k, int dtype);
+int csa_prefill(const void* x, const void* x_left, const void* W_kv, const float* B_kv,
+                const void* W_idx, const float* B_idx, int64_t start, int64_t n, int d, int m,
+                int c, int cI, void* kv_cache, void* idx_cache, int64_t Nmax, const void* qI,
+                const float* w, const void* q, int H, int HI, int k, float scale,
+                const float* sink, void* out, float* lse, int32_t* topk_idx, void* ws,
+                size_t ws_bytes, int dtype, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_H_ */

@@ -110,7 +110,18 @@ def bf16_round(x) -> np.ndarray:
 
 
 def project(X, W) -> np.ndarray:
-    """P = X @ W^T with X [n, d] and W [M, d] (one row per output feature)."""
+    """P = X @ W^T with X [n, d] and W [M, d] (one row per output feature).
+
+    A plain fp64 matrix product (numpy's, used as a library primitive so that
+    full-size projections finish on the host); project_loops() is the same
+    definition written as loops in C."""
+    X, W = _f64(X), _f64(W)
+    assert X.shape[1] == W.shape[1]
+    return X @ W.T
+
+
+def project_loops(X, W) -> np.ndarray:
+    """P = X @ W^T as the plain triple loop of csa_oracle.c."""
     X, W = _f64(X), _f64(W)
     n, d = X.shape
     M = W.shape[0]

@@ -1,0 +1,105 @@
+"""Host-side checks of the C ABI (no GPU needed, no kernel is launched):
+the library loads, exports every function include/csa.h declares, rejects
+bad arguments before touching the device, and sizes its workspaces."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import compressed_sparse_attention_14_b200 as csa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "csa.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b((?:csa|hca)_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declarations_are_exported():
+    names = _declared()
+    assert len(names) >= 20
+    lib = ctypes.CDLL(csa.LIB_PATH)
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+    assert sorted(csa.EXPORTED) == names
+
+
+def test_abi_version():
+    assert csa.abi_version() == 1
+
+
+def _lib():
+    return csa._lib
+
+
+def test_invalid_arguments_are_rejected_on_the_host():
+    L = _lib()
+    fake = 0x10000  # 16-byte aligned, never dereferenced: checks fail first
+    # n not a multiple of m
+    assert L.csa_compress(fake, None, fake, 6, 8, 4, fake, csa.CSA_BF16, None) == csa.CSA_ERR_INVALID_ARG
+    assert b"multiple" in L.csa_last_error()
+    # c not a multiple of 8
+    assert L.csa_compress(fake, None, fake, 8, 12, 4, fake, csa.CSA_BF16, None) == csa.CSA_ERR_INVALID_ARG
+    # null required pointer
+    assert L.csa_compress(None, None, fake, 8, 8, 4, fake, csa.CSA_BF16, None) == csa.CSA_ERR_INVALID_ARG
+    assert b"NULL" in L.csa_last_error()
+    # misaligned pointer
+    assert L.hca_compress(fake + 4, fake, 128, 8, 128, fake, csa.CSA_BF16, None) == csa.CSA_ERR_INVALID_ARG
+    assert b"aligned" in L.csa_last_error()
+    # bad dtype
+    assert L.hca_compress(fake, fake, 128, 8, 128, fake, 7, None) == csa.CSA_ERR_INVALID_ARG
+    # k out of range
+    assert L.csa_topk_from_scores(fake, 16, None, 1, 1, 16, 0, fake, None, None, 0, None) == csa.CSA_ERR_UNSUPPORTED
+    assert L.csa_topk_from_scores(fake, 16, None, 1, 1, 16, 4096, fake, None, None, 0, None) == csa.CSA_ERR_UNSUPPORTED
+    # attention shapes beyond the kernels
+    assert L.csa_sparse_mqa(fake, fake, fake, None, 1, 256, 128, 8, 4, 0.0, None, fake, None, None, 0,
+                            csa.CSA_BF16, None) == csa.CSA_ERR_UNSUPPORTED
+    assert L.csa_sparse_mqa(fake, fake, fake, None, 1, 8, 1024, 8, 4, 0.0, None, fake, None, None, 0,
+                            csa.CSA_BF16, None) == csa.CSA_ERR_UNSUPPORTED
+    # missing / short workspace
+    need = L.csa_decode_workspace_size(2, 1024, 8, 128, 4, 64, 16, csa.CSA_BF16)
+    assert need > 0
+    rc = L.csa_decode(fake, fake, fake, fake, fake, fake, 2, 1024, 4, 8, 128, 4, 64, 16, 0.0, None, fake, None,
+                      None, None, 0, csa.CSA_BF16, None)
+    assert rc == csa.CSA_ERR_WORKSPACE
+    rc = L.csa_decode(fake, fake, fake, fake, fake, fake, 2, 1024, 4, 8, 128, 4, 64, 16, 0.0, None, fake, None,
+                      None, fake * 16, need - 1, csa.CSA_BF16, None)
+    assert rc == csa.CSA_ERR_WORKSPACE
+    # prefill: start not a multiple of m, cache too small, missing left rows
+    args = dict(n=8, Nmax=4, start=4)
+    rc = L.csa_prefill(fake, fake, fake, fake, fake, fake, 2, 8, 64, 4, 32, 32, fake, fake, 16, fake, fake, fake,
+                       8, 4, 4, 0.0, None, fake, None, None, None, 0, csa.CSA_BF16, None)
+    assert rc == csa.CSA_ERR_INVALID_ARG
+    rc = L.csa_prefill(fake, fake, fake, fake, fake, fake, 4, 8, 64, 4, 32, 32, fake, fake, 2, fake, fake, fake,
+                       8, 4, 4, 0.0, None, fake, None, None, None, 0, csa.CSA_BF16, None)
+    assert rc == csa.CSA_ERR_INVALID_ARG
+    rc = L.csa_prefill(fake, None, fake, fake, fake, fake, 4, 8, 64, 4, 32, 32, fake, fake, 16, fake, fake, fake,
+                       8, 4, 4, 0.0, None, fake, None, None, None, 0, csa.CSA_BF16, None)
+    assert rc == csa.CSA_ERR_INVALID_ARG
+    del args
+
+
+def test_empty_inputs_are_no_ops():
+    L = _lib()
+    assert L.csa_compress(None, None, None, 0, 8, 4, None, csa.CSA_BF16, None) == csa.CSA_OK
+    assert L.csa_topk_from_scores(None, 0, None, 1, 0, 0, 8, None, None, None, 0, None) == csa.CSA_OK
+    assert L.csa_decode(None, None, None, None, None, None, 0, 16, 4, 8, 128, 4, 64, 16, 0.0, None, None, None,
+                        None, None, 0, csa.CSA_BF16, None) == csa.CSA_OK
+
+
+def test_workspace_sizes():
+    L = _lib()
+    # one-level top-k needs no workspace; multi-level needs two candidate buffers
+    assert L.csa_topk_workspace_size(64, 16384, 512) == 0
+    two = L.csa_topk_workspace_size(32, 262144, 1024)
+    assert two >= 2 * 32 * 16 * 1024 * 8
+    assert L.csa_decode_workspace_size(64, 32768, 64, 512, 64, 128, 512, csa.CSA_BF16) >= 64 * 32768 * 4
+    small = L.csa_prefill_workspace_size(1024, 256, 512, 4, 128, 64, 8, 4, 16, csa.CSA_BF16)
+    assert small >= 1024 * 4 * 128 * 4
+    # the prefill score block is bounded (query chunking) at long context
+    big = L.csa_prefill_workspace_size(65536, 65536, 4096, 4, 512, 128, 64, 64, 512, csa.CSA_BF16)
+    assert big < 8 * (1 << 30)

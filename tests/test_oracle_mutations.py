@@ -41,7 +41,8 @@ MUTATIONS = [
     ("dense MQA sees its own block", "int64_t vis = pos[t] / mp;", "int64_t vis = pos[t] / mp + 1;"),
     ("bf16 rounding truncates", "double r = ldexp(round_half_even(ldexp(a, -q)), q);",
      "double r = ldexp(floor(ldexp(a, -q)), q);"),
-    ("projection uses W transposed index", "X[t * d + k] * W[o * d + k]", "X[t * d + k] * W[k * M + o]"),
+    ("projection loops use a transposed W index", "X[t * d + k] * W[o * d + k]",
+     "X[t * d + k] * W[(k * M + o) % (M * d)]"),
 ]
 
 

@@ -92,10 +92,13 @@ def test_bf16_round_ties_to_even_by_hand():
 # a1 projections
 # --------------------------------------------------------------------------
 
-def test_project_matches_numpy_matmul():
+def test_project_loops_match_library_matmul():
     X = rng.standard_normal((37, 53))
     W = rng.standard_normal((19, 53))
-    np.testing.assert_allclose(oracle.project(X, W), X @ W.T, rtol=1e-13, atol=1e-12)
+    np.testing.assert_allclose(oracle.project_loops(X, W), X @ W.T, rtol=1e-13, atol=1e-12)
+    np.testing.assert_allclose(oracle.project(X, W), oracle.project_loops(X, W), rtol=1e-13, atol=1e-12)
+    # by hand: [1, 2] . [3, 4] = 11, [1, 2] . [-1, 0.5] = 0
+    np.testing.assert_array_equal(oracle.project_loops([[1.0, 2.0]], [[3.0, 4.0], [-1.0, 0.5]]), [[11.0, 0.0]])
 
 
 # --------------------------------------------------------------------------
