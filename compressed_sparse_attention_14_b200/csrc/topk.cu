@@ -61,6 +61,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_select_kernel(TopkLevel L) 
     __shared__ uint64_t s_prefix;
     __shared__ uint32_t s_remaining;
     __shared__ int s_done;
+    __shared__ uint32_t s_n, s_tie;
 
     const int row = blockIdx.y;
     const int seg = blockIdx.x;
@@ -79,20 +80,25 @@ __global__ void __launch_bounds__(kTopkThreads) topk_select_kernel(TopkLevel L) 
     }
     const int64_t beg = (int64_t)seg * L.seg_len;
     int64_t n64 = n_row - beg;
-    const int n = n64 <= 0 ? 0 : (n64 > L.seg_len ? L.seg_len : (int)n64);
+    const int n_in = n64 <= 0 ? 0 : (n64 > L.seg_len ? L.seg_len : (int)n64);
 
-    for (int i = tid; i < n; i += kTopkThreads) {
-        uint64_t x;
-        if (kRaw) {
-            float s = L.scores[(int64_t)row * L.ld + beg + i];
-            x = ((uint64_t)orderable(s) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)(beg + i));
-        } else {
-            x = L.cand[(int64_t)row * L.cand_ld + beg + i];
-        }
-        s_elems[i] = x;
-    }
-    if (tid == 0) { s_prefix = 0; s_remaining = (uint32_t)k; s_done = 0; s_cnt = 0; }
+    if (tid == 0) { s_prefix = 0; s_remaining = (uint32_t)k; s_done = 0; s_cnt = 0; s_n = 0; s_tie = 0; }
     __syncthreads();
+    if (kRaw) {
+        for (int i = tid; i < n_in; i += kTopkThreads) {
+            float s = L.scores[(int64_t)row * L.ld + beg + i];
+            s_elems[i] = ((uint64_t)orderable(s) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)(beg + i));
+        }
+    } else {
+        // candidate rows carry empty slots (0); keep only real candidates, so
+        // every composite in shared memory is distinct
+        for (int i = tid; i < n_in; i += kTopkThreads) {
+            uint64_t x = L.cand[(int64_t)row * L.cand_ld + beg + i];
+            if (x != 0ull) s_elems[atomicAdd(&s_n, 1u)] = x;
+        }
+    }
+    __syncthreads();
+    const int n = kRaw ? n_in : (int)s_n;
 
     // ---- radix select: threshold T such that exactly min(k, n) elements are >= T
     uint64_t thr = 0;
@@ -147,12 +153,24 @@ __global__ void __launch_bounds__(kTopkThreads) topk_select_kernel(TopkLevel L) 
     }
     const int kk = n < k ? n : k;
 
-    // ---- collect the winners (order arbitrary)
+    // ---- collect the winners (order arbitrary): everything above the
+    // threshold, then copies of the threshold value up to exactly kk (the
+    // composites are distinct, so at most one element equals thr; the second
+    // pass keeps the count exact regardless)
     for (int i = tid; i < n; i += kTopkThreads) {
         uint64_t x = s_elems[i];
-        if (x >= thr) {
+        if (x > thr) {
             uint32_t slot = atomicAdd(&s_cnt, 1u);
             if (slot < (uint32_t)CSA_MAX_TOPK) s_sel[slot] = x;
+        }
+    }
+    __syncthreads();
+    const uint32_t n_gt = s_cnt;
+    for (int i = tid; i < n; i += kTopkThreads) {
+        uint64_t x = s_elems[i];
+        if (x == thr) {
+            uint32_t t = atomicAdd(&s_tie, 1u);
+            if (n_gt + t < (uint32_t)kk) s_sel[n_gt + t] = x;
         }
     }
     __syncthreads();
