@@ -54,6 +54,7 @@ _SIGS = {
     "csa_index_scores": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _P, _I, _P]),
     "csa_topk_workspace_size": (_SZ, [_I, _I64, _I]),
     "csa_topk_from_scores": (_I, [_P, _I64, _P, _I, _I, _I64, _I, _P, _P, _P, _SZ, _P]),
+    "csa_topk_from_scores_noalloc": (_I, [_P, _I64, _P, _I, _I, _I64, _I, _P, _P, _P]),
     "csa_index_topk_workspace_size": (_SZ, [_I, _I64, _I, _I]),
     "csa_index_topk": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I, _P, _P, _P, _SZ, _I, _P]),
     "csa_sparse_mqa_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
@@ -232,6 +233,19 @@ def csa_topk_from_scores(scores, k: int, valid=None, valid_div: int = 1, ws=None
     _check(_lib.csa_topk_from_scores(_ptr(scores), ncols, _ptr(valid), valid_div, nq, ncols, k, _ptr(idx),
                                      _ptr(top), _ptr(ws), _nbytes(ws), _stream()))
     return idx, top
+
+
+def csa_topk_from_scores_noalloc(scores, k: int, valid=None, valid_div: int = 1, idx=None, top_scores=None):
+    """csa_topk_from_scores without a workspace (for callers that cannot
+    allocate device memory when they select): the library's fixed 8 MiB
+    device array holds the intermediate candidates. Pass preallocated idx /
+    top_scores to make the call itself allocation-free."""
+    nq, ncols = scores.shape
+    if idx is None:
+        idx = torch.empty((nq, k), dtype=torch.int32, device=scores.device)
+    _check(_lib.csa_topk_from_scores_noalloc(_ptr(scores), ncols, _ptr(valid), valid_div, nq, ncols, k, _ptr(idx),
+                                             _ptr(top_scores), _stream()))
+    return idx, top_scores
 
 
 def csa_index_topk(qI, w, K, pos, m: int, k: int, seq_of_q=None, ws=None):

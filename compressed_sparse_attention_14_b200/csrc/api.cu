@@ -29,6 +29,16 @@ static int fail(int code, const char* fmt, ...) {
     return code;
 }
 
+int set_last_error(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
 static int cuda_status(cudaError_t e, const char* where) {
     if (e == cudaSuccess) return CSA_OK;
     return fail(CSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));

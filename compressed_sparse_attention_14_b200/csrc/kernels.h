@@ -37,6 +37,10 @@ struct QuerySpec {
     int single_seq;
 };
 
+// api.cu: record the thread's last error message (csa_last_error) and
+// return `code`.
+int set_last_error(int code, const char* fmt, ...);
+
 // compress.cu
 cudaError_t compress_csa(const void* proj, const void* left, const float* bias, int64_t n, int c,
                          int m, void* out, ElemType in_t, ElemType out_t, cudaStream_t st);

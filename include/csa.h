@@ -162,6 +162,23 @@ int csa_topk_from_scores(const float* scores, int64_t ld, const int32_t* valid, 
                          int nq, int64_t ncols, int k, int32_t* idx, float* top_scores, void* ws,
                          size_t ws_bytes, void* stream);
 
+/* a5 without a workspace, for callers that cannot allocate device memory at
+ * the point of the call (a plug-in whose host framework owns every device
+ * allocation and gives it no workspace, a serving loop that forbids
+ * allocation after start-up). The pages have no counterpart: this is a
+ * library convenience. Same arguments and exactly the same result as
+ * csa_topk_from_scores, minus ws/ws_bytes. The multi-level candidate buffers
+ * live in a fixed 8 MiB array in the library's device memory (held on every
+ * GPU that loads the library until the process exits): a selection needing
+ * more scratch than that (csa_topk_workspace_size > 8 MiB) is rejected with
+ * CSA_ERR_UNSUPPORTED. All calls share the array: calls that may run at the
+ * same time on the GPU race on it and must be serialized by the caller. The
+ * first call on each device (with that device current) looks up the
+ * array's address; make it before any stream capture begins. No cudaMalloc,
+ * cudaFree or other allocating call is made. */
+int csa_topk_from_scores_noalloc(const float* scores, int64_t ld, const int32_t* valid, int valid_div, int nq,
+                                 int64_t ncols, int k, int32_t* idx, float* top_scores, void* stream);
+
 /* a4+a5: indexer then top-k over the visible entries of each query. */
 size_t csa_index_topk_workspace_size(int nq, int64_t Nmax, int k, int dtype);
 int csa_index_topk(const void* qI, const float* w, const void* K, const int32_t* pos,
