@@ -51,16 +51,16 @@ _SIGS = {
     "csa_compress_from_hidden": (_I, [_P, _P, _P, _P, _I64, _I, _I, _I, _P, _P, _SZ, _I, _P]),
     "hca_compress_from_hidden_workspace_size": (_SZ, [_I64, _I, _I, _I, _I]),
     "hca_compress_from_hidden": (_I, [_P, _P, _P, _I64, _I, _I, _I, _P, _P, _SZ, _I, _P]),
-    "csa_index_scores": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _P, _I, _P]),
+    "csa_index_scores": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I64, _I, _P, _I, _P]),
     "csa_topk_workspace_size": (_SZ, [_I, _I64, _I]),
     "csa_topk_from_scores": (_I, [_P, _I64, _P, _I, _I, _I64, _I, _P, _P, _P, _SZ, _P]),
     "csa_topk_from_scores_noalloc": (_I, [_P, _I64, _P, _I, _I, _I64, _I, _P, _P, _P]),
     "csa_index_topk_workspace_size": (_SZ, [_I, _I64, _I, _I]),
-    "csa_index_topk": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I, _P, _P, _P, _SZ, _I, _P]),
+    "csa_index_topk": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I64, _I, _I, _P, _P, _P, _SZ, _I, _P]),
     "csa_sparse_mqa_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
-    "csa_sparse_mqa": (_I, [_P, _P, _P, _P, _I, _I, _I, _I64, _I, _F, _P, _P, _P, _P, _SZ, _I, _P]),
+    "csa_sparse_mqa": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I64, _I, _F, _P, _P, _P, _P, _SZ, _I, _P]),
     "hca_dense_mqa_workspace_size": (_SZ, [_I, _I, _I, _I64, _I]),
-    "hca_dense_mqa": (_I, [_P, _P, _P, _P, _I, _I, _I, _I64, _I, _F, _P, _P, _P, _P, _SZ, _I, _P]),
+    "hca_dense_mqa": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I64, _I, _F, _P, _P, _P, _P, _SZ, _I, _P]),
     "csa_decode_workspace_size": (_SZ, [_I, _I64, _I, _I, _I, _I, _I, _I]),
     "csa_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I64, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P,
                         _P, _SZ, _I, _P]),
@@ -220,8 +220,8 @@ def csa_index_scores(qI, w, K, pos, m: int, seq_of_q=None):
     K = _kv3(K)
     Nmax = K.shape[1]
     scores = torch.empty((nq, Nmax), dtype=torch.float32, device=qI.device)
-    _check(_lib.csa_index_scores(_ptr(qI), _ptr(w), _ptr(K), _ptr(pos), _ptr(seq_of_q), nq, HI, cI, Nmax, m,
-                                 _ptr(scores), _mode(qI), _stream()))
+    _check(_lib.csa_index_scores(_ptr(qI), _ptr(w), _ptr(K), _ptr(pos), _ptr(seq_of_q), nq, K.shape[0], HI, cI,
+                                 Nmax, m, _ptr(scores), _mode(qI), _stream()))
     return scores
 
 
@@ -256,7 +256,8 @@ def csa_index_topk(qI, w, K, pos, m: int, k: int, seq_of_q=None, ws=None):
     idx = torch.empty((nq, k), dtype=torch.int32, device=qI.device)
     top = torch.empty((nq, k), dtype=torch.float32, device=qI.device)
     ws = _ws(_lib.csa_index_topk_workspace_size(nq, Nmax, k, mode), qI.device, ws)
-    _check(_lib.csa_index_topk(_ptr(qI), _ptr(w), _ptr(K), _ptr(pos), _ptr(seq_of_q), nq, HI, cI, Nmax, m, k,
+    _check(_lib.csa_index_topk(_ptr(qI), _ptr(w), _ptr(K), _ptr(pos), _ptr(seq_of_q), nq, K.shape[0], HI, cI,
+                               Nmax, m, k,
                                _ptr(idx), _ptr(top), _ptr(ws), _nbytes(ws), mode, _stream()))
     return idx, top
 
@@ -271,7 +272,7 @@ def csa_sparse_mqa(q, KV, idx, scale: float = 0.0, sink=None, seq_of_q=None, out
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty((nq, H), dtype=torch.float32, device=q.device)
     ws = _ws(_lib.csa_sparse_mqa_workspace_size(nq, H, c, k, mode), q.device, ws)
-    _check(_lib.csa_sparse_mqa(_ptr(q), _ptr(KV), _ptr(idx), _ptr(seq_of_q), nq, H, c, Nmax, k, scale,
+    _check(_lib.csa_sparse_mqa(_ptr(q), _ptr(KV), _ptr(idx), _ptr(seq_of_q), nq, KV.shape[0], H, c, Nmax, k, scale,
                                _ptr(sink), _ptr(out), _ptr(lse), _ptr(ws), _nbytes(ws), mode, _stream()))
     return out, lse
 
@@ -284,7 +285,7 @@ def hca_dense_mqa(q, KV, pos, mp: int, scale: float = 0.0, sink=None, seq_of_q=N
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty((nq, H), dtype=torch.float32, device=q.device)
     ws = _ws(_lib.hca_dense_mqa_workspace_size(nq, H, c, Nmax, mode), q.device, ws)
-    _check(_lib.hca_dense_mqa(_ptr(q), _ptr(KV), _ptr(pos), _ptr(seq_of_q), nq, H, c, Nmax, mp, scale,
+    _check(_lib.hca_dense_mqa(_ptr(q), _ptr(KV), _ptr(pos), _ptr(seq_of_q), nq, KV.shape[0], H, c, Nmax, mp, scale,
                               _ptr(sink), _ptr(out), _ptr(lse), _ptr(ws), _nbytes(ws), mode, _stream()))
     return out, lse
 

@@ -16,6 +16,18 @@ namespace csa {
 
 __device__ int g_status_word = 0;
 
+int* device_status() {
+    static int* addr[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+        addr[dev] = (int*)p;
+    }
+    return addr[dev];
+}
+
 
 static thread_local std::string g_err;
 
@@ -110,16 +122,41 @@ static int check_k(int k) {
     return CSA_OK;
 }
 
+// Indexer of the mode: tcgen05 kernel for bf16, FFMA kernel for fp32.
+static cudaError_t run_indexer(const void* qI, const float* w, const void* K, QuerySpec qs, int nq, int n_seq,
+                               int HI, int cI, int64_t Nmax, int m, float* scores, int64_t ld, int group,
+                               bool fill_invisible, ElemType t, cudaStream_t st) {
+    if (t == ElemType::BF16)
+        return index_scores_tc(qI, w, K, qs, nq, n_seq, HI, cI, Nmax, m, scores, ld, group, fill_invisible,
+                               device_status(), st);
+    return index_scores(qI, w, K, qs, nq, HI, cI, Nmax, m, scores, ld, t, st);
+}
+
+static int check_index_mode(int HI, int cI, ElemType t) {
+    if (t == ElemType::BF16 && !index_tc_supported(HI, cI, 1))
+        return fail(CSA_ERR_UNSUPPORTED, "bf16 indexer needs cI a multiple of 64 (<= 256) and HI <= 256 (cI=%d HI=%d)",
+                    cI, HI);
+    return CSA_OK;
+}
+
+static int check_rows(int nq, const char* who) {
+    if (nq > 65535) return fail(CSA_ERR_UNSUPPORTED, "%s: at most 65535 queries per call (got %d)", who, nq);
+    return CSA_OK;
+}
+
 // ---- plans shared by the size queries and the calls ------------------------
 
 static size_t index_topk_bytes(int nq, int64_t Nmax, int k) {
     return align256((size_t)nq * (size_t)Nmax * sizeof(float)) + topk_workspace_bytes(nq, Nmax, k);
 }
 
-static int64_t prefill_query_chunk(int64_t n, int64_t Nmax) {
-    // bound the fp32 score block of one query chunk to 1 GiB
+static int64_t prefill_query_chunk(int64_t n, int64_t Nmax, int m) {
+    // bound the fp32 score block of one query chunk to 1 GiB; whole
+    // compressed blocks (multiples of m tokens) and at most 65535 queries
     int64_t qc = ((int64_t)1 << 28) / (Nmax > 0 ? Nmax : 1);
-    if (qc < 1) qc = 1;
+    if (qc > 65535) qc = 65535;
+    qc -= qc % m;
+    if (qc < m) qc = m;
     if (qc > n) qc = n;
     return qc;
 }
@@ -267,12 +304,15 @@ int hca_compress_from_hidden(const void* x, const void* W, const float* bias, in
 
 // ---------------------------------------------------------------- a4 / a5
 int csa_index_scores(const void* qI, const float* w, const void* K, const int32_t* pos,
-                     const int32_t* seq_of_q, int nq, int HI, int cI, int64_t Nmax, int m,
+                     const int32_t* seq_of_q, int nq, int n_seq, int HI, int cI, int64_t Nmax, int m,
                      float* scores, int dtype, void* stream) {
     ElemType t;
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_index_shape(HI, cI));
-    if (nq < 0 || Nmax < 0 || m < 1) return fail(CSA_ERR_INVALID_ARG, "bad nq/Nmax/m");
+    CSA_TRY(check_index_mode(HI, cI, t));
+    CSA_TRY(check_rows(nq, "csa_index_scores"));
+    if (nq < 0 || Nmax < 0 || m < 1 || n_seq < 1) return fail(CSA_ERR_INVALID_ARG, "bad nq/n_seq/Nmax/m");
+    if (!seq_of_q && n_seq < nq) return fail(CSA_ERR_INVALID_ARG, "seq_of_q is NULL (query t reads sequence t) but n_seq < nq");
     if (Nmax > INT32_MAX) return fail(CSA_ERR_UNSUPPORTED, "Nmax beyond int32 entry indices");
     if (nq == 0 || Nmax == 0) return CSA_OK;
     CSA_TRY(check_ptr(qI, "qI"));
@@ -282,7 +322,7 @@ int csa_index_scores(const void* qI, const float* w, const void* K, const int32_
     CSA_TRY(check_ptr(seq_of_q, "seq_of_q", false));
     CSA_TRY(check_ptr(scores, "scores"));
     QuerySpec qs{seq_of_q, pos, 0, 0};
-    CSA_CUDA(index_scores(qI, w, K, qs, nq, HI, cI, Nmax, m, scores, Nmax, t, (cudaStream_t)stream),
+    CSA_CUDA(run_indexer(qI, w, K, qs, nq, n_seq, HI, cI, Nmax, m, scores, Nmax, 1, true, t, (cudaStream_t)stream),
              "csa_index_scores");
     return CSA_OK;
 }
@@ -299,6 +339,7 @@ int csa_topk_from_scores(const float* scores, int64_t ld, const int32_t* valid, 
     if (nq < 0 || ncols < 0 || ld < ncols || valid_div < 1)
         return fail(CSA_ERR_INVALID_ARG, "csa_topk_from_scores: bad nq/ncols/ld/valid_div");
     if (ncols > INT32_MAX) return fail(CSA_ERR_UNSUPPORTED, "ncols beyond int32 indices");
+    CSA_TRY(check_rows(nq, "csa_topk_from_scores"));
     if (nq == 0) return CSA_OK;
     if (ncols > 0) CSA_TRY(check_ptr(scores, "scores"));
     CSA_TRY(check_ptr(valid, "valid", false));
@@ -317,14 +358,17 @@ size_t csa_index_topk_workspace_size(int nq, int64_t Nmax, int k, int dtype) {
 }
 
 int csa_index_topk(const void* qI, const float* w, const void* K, const int32_t* pos,
-                   const int32_t* seq_of_q, int nq, int HI, int cI, int64_t Nmax, int m, int k,
+                   const int32_t* seq_of_q, int nq, int n_seq, int HI, int cI, int64_t Nmax, int m, int k,
                    int32_t* idx, float* top_scores, void* ws, size_t ws_bytes, int dtype,
                    void* stream) {
     ElemType t;
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_index_shape(HI, cI));
+    CSA_TRY(check_index_mode(HI, cI, t));
     CSA_TRY(check_k(k));
-    if (nq < 0 || Nmax < 0 || m < 1) return fail(CSA_ERR_INVALID_ARG, "bad nq/Nmax/m");
+    CSA_TRY(check_rows(nq, "csa_index_topk"));
+    if (nq < 0 || Nmax < 0 || m < 1 || n_seq < 1) return fail(CSA_ERR_INVALID_ARG, "bad nq/n_seq/Nmax/m");
+    if (!seq_of_q && n_seq < nq) return fail(CSA_ERR_INVALID_ARG, "seq_of_q is NULL (query t reads sequence t) but n_seq < nq");
     if (Nmax > INT32_MAX) return fail(CSA_ERR_UNSUPPORTED, "Nmax beyond int32 entry indices");
     if (nq == 0) return CSA_OK;
     CSA_TRY(check_ptr(qI, "qI"));
@@ -340,7 +384,7 @@ int csa_index_topk(const void* qI, const float* w, const void* K, const int32_t*
     float* sc = (float*)cv.take((size_t)nq * Nmax * sizeof(float));
     void* tws = cv.take(topk_workspace_bytes(nq, Nmax, k));
     QuerySpec qs{seq_of_q, pos, 0, 0};
-    CSA_CUDA(index_scores(qI, w, K, qs, nq, HI, cI, Nmax, m, sc, Nmax, t, st), "csa_index_topk: scores");
+    CSA_CUDA(run_indexer(qI, w, K, qs, nq, n_seq, HI, cI, Nmax, m, sc, Nmax, 1, false, t, st), "csa_index_topk: scores");
     CSA_CUDA(topk_select(sc, Nmax, pos, m, nq, Nmax, k, idx, top_scores, tws, st), "csa_index_topk: top-k");
     return CSA_OK;
 }
@@ -353,13 +397,15 @@ size_t csa_sparse_mqa_workspace_size(int nq, int H, int c, int k, int dtype) {
 }
 
 int csa_sparse_mqa(const void* q, const void* KV, const int32_t* idx, const int32_t* seq_of_q,
-                   int nq, int H, int c, int64_t Nmax, int k, float scale, const float* sink,
+                   int nq, int n_seq, int H, int c, int64_t Nmax, int k, float scale, const float* sink,
                    void* out, float* lse, void* ws, size_t ws_bytes, int dtype, void* stream) {
     ElemType t;
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_attn_shape(H, c));
     CSA_TRY(check_k(k));
-    if (nq < 0 || Nmax < 0) return fail(CSA_ERR_INVALID_ARG, "bad nq/Nmax");
+    CSA_TRY(check_rows(nq, "csa_sparse_mqa"));
+    if (nq < 0 || Nmax < 0 || n_seq < 1) return fail(CSA_ERR_INVALID_ARG, "bad nq/n_seq/Nmax");
+    if (!seq_of_q && n_seq < nq) return fail(CSA_ERR_INVALID_ARG, "seq_of_q is NULL (query t reads sequence t) but n_seq < nq");
     if (nq == 0) return CSA_OK;
     CSA_TRY(check_ptr(q, "q"));
     CSA_TRY(check_ptr(KV, "KV", Nmax > 0));
@@ -370,7 +416,7 @@ int csa_sparse_mqa(const void* q, const void* KV, const int32_t* idx, const int3
     CSA_TRY(check_ptr(lse, "lse", false));
     CSA_TRY(check_ws(ws, ws_bytes, mqa_workspace_bytes(nq, H, c, k, t)));
     QuerySpec qs{seq_of_q, nullptr, 0, 0};
-    CSA_CUDA(mqa(q, KV, idx, k, qs, 1, nq, H, c, Nmax, default_scale(scale, c), sink, out, lse, ws, t,
+    CSA_CUDA(mqa(q, KV, idx, k, qs, 1, nq, n_seq, H, c, Nmax, default_scale(scale, c), sink, out, lse, ws, t,
                  (cudaStream_t)stream), "csa_sparse_mqa");
     return CSA_OK;
 }
@@ -382,12 +428,14 @@ size_t hca_dense_mqa_workspace_size(int nq, int H, int c, int64_t Nmax, int dtyp
 }
 
 int hca_dense_mqa(const void* q, const void* KV, const int32_t* pos, const int32_t* seq_of_q,
-                  int nq, int H, int c, int64_t Nmax, int mp, float scale, const float* sink,
+                  int nq, int n_seq, int H, int c, int64_t Nmax, int mp, float scale, const float* sink,
                   void* out, float* lse, void* ws, size_t ws_bytes, int dtype, void* stream) {
     ElemType t;
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_attn_shape(H, c));
-    if (nq < 0 || Nmax < 0 || mp < 1) return fail(CSA_ERR_INVALID_ARG, "bad nq/Nmax/mp");
+    CSA_TRY(check_rows(nq, "hca_dense_mqa"));
+    if (nq < 0 || Nmax < 0 || mp < 1 || n_seq < 1) return fail(CSA_ERR_INVALID_ARG, "bad nq/n_seq/Nmax/mp");
+    if (!seq_of_q && n_seq < nq) return fail(CSA_ERR_INVALID_ARG, "seq_of_q is NULL (query t reads sequence t) but n_seq < nq");
     if (Nmax > INT32_MAX) return fail(CSA_ERR_UNSUPPORTED, "Nmax beyond int32 entry indices");
     if (nq == 0) return CSA_OK;
     CSA_TRY(check_ptr(q, "q"));
@@ -399,7 +447,7 @@ int hca_dense_mqa(const void* q, const void* KV, const int32_t* pos, const int32
     CSA_TRY(check_ptr(lse, "lse", false));
     CSA_TRY(check_ws(ws, ws_bytes, mqa_workspace_bytes(nq, H, c, Nmax, t)));
     QuerySpec qs{seq_of_q, pos, 0, 0};
-    CSA_CUDA(mqa(q, KV, nullptr, 0, qs, mp, nq, H, c, Nmax, default_scale(scale, c), sink, out, lse, ws,
+    CSA_CUDA(mqa(q, KV, nullptr, 0, qs, mp, nq, n_seq, H, c, Nmax, default_scale(scale, c), sink, out, lse, ws,
                  t, (cudaStream_t)stream), "hca_dense_mqa");
     return CSA_OK;
 }
@@ -420,8 +468,10 @@ int csa_decode(const void* qI, const float* w, const void* idx_cache, const void
     ElemType t;
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_index_shape(HI, cI));
+    CSA_TRY(check_index_mode(HI, cI, t));
     CSA_TRY(check_attn_shape(H, c));
     CSA_TRY(check_k(k));
+    CSA_TRY(check_rows(B, "csa_decode"));
     if (B < 0 || Nmax < 0 || m < 1) return fail(CSA_ERR_INVALID_ARG, "bad B/Nmax/m");
     if (Nmax > INT32_MAX) return fail(CSA_ERR_UNSUPPORTED, "Nmax beyond int32 entry indices");
     if (B == 0) return CSA_OK;
@@ -444,9 +494,9 @@ int csa_decode(const void* qI, const float* w, const void* idx_cache, const void
     void* mws = cv.take(mqa_workspace_bytes(B, H, c, k, t));
     if (topk_idx) sel = topk_idx;
     QuerySpec qs{nullptr, ctx_len, 0, 0};
-    CSA_CUDA(index_scores(qI, w, idx_cache, qs, B, HI, cI, Nmax, m, sc, Nmax, t, st), "csa_decode: indexer");
+    CSA_CUDA(run_indexer(qI, w, idx_cache, qs, B, B, HI, cI, Nmax, m, sc, Nmax, 1, false, t, st), "csa_decode: indexer");
     CSA_CUDA(topk_select(sc, Nmax, ctx_len, m, B, Nmax, k, sel, nullptr, tws, st), "csa_decode: top-k");
-    CSA_CUDA(mqa(q, kv_cache, sel, k, qs, 1, B, H, c, Nmax, default_scale(scale, c), sink, out, lse, mws, t, st),
+    CSA_CUDA(mqa(q, kv_cache, sel, k, qs, 1, B, B, H, c, Nmax, default_scale(scale, c), sink, out, lse, mws, t, st),
              "csa_decode: mqa");
     return CSA_OK;
 }
@@ -458,7 +508,7 @@ size_t hca_decode_workspace_size(int B, int64_t Nmax, int H, int c, int dtype) {
 int hca_decode(const void* q, const void* kv_cache, const int32_t* ctx_len, int B, int64_t Nmax,
                int mp, int H, int c, float scale, const float* sink, void* out, float* lse,
                void* ws, size_t ws_bytes, int dtype, void* stream) {
-    return hca_dense_mqa(q, kv_cache, ctx_len, nullptr, B, H, c, Nmax, mp, scale, sink, out, lse, ws,
+    return hca_dense_mqa(q, kv_cache, ctx_len, nullptr, B, B, H, c, Nmax, mp, scale, sink, out, lse, ws,
                          ws_bytes, dtype, stream);
 }
 
@@ -468,7 +518,7 @@ size_t csa_prefill_workspace_size(int64_t n, int64_t Nmax, int d, int m, int c, 
     ElemType t = dtype == CSA_FP32 ? ElemType::F32 : ElemType::BF16;
     if (n < 0 || Nmax < 0 || m < 1 || c < 1 || cI < 1 || k < 1) return 0;
     const int cw = c > cI ? c : cI;
-    int64_t qc = prefill_query_chunk(n, Nmax);
+    int64_t qc = prefill_query_chunk(n, Nmax, m);
     size_t b = align256((size_t)n * 4 * cw * sizeof(float)) + align256((size_t)m * 4 * cw * sizeof(float));
     b += index_topk_bytes((int)qc, Nmax, k) + align256((size_t)qc * k * sizeof(int32_t));
     b += mqa_workspace_bytes((int)qc, H, c, k, t);
@@ -484,6 +534,7 @@ int csa_prefill(const void* x, const void* x_left, const void* W_kv, const float
     ElemType t;
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_index_shape(HI, cI));
+    CSA_TRY(check_index_mode(HI, cI, t));
     CSA_TRY(check_attn_shape(H, c));
     CSA_TRY(check_k(k));
     CSA_TRY(check_compress(n, c, m, 64, "csa_prefill"));
@@ -513,7 +564,7 @@ int csa_prefill(const void* x, const void* x_left, const void* W_kv, const float
     cudaStream_t st = (cudaStream_t)stream;
     const size_t es = elem_size(t);
     const int cw = c > cI ? c : cI;
-    const int64_t qc = prefill_query_chunk(n, Nmax);
+    const int64_t qc = prefill_query_chunk(n, Nmax, m);
     Carve cv(ws);
     float* proj = (float*)cv.take((size_t)n * 4 * cw * sizeof(float));
     float* lproj = (float*)cv.take((size_t)m * 4 * cw * sizeof(float));
@@ -539,12 +590,15 @@ int csa_prefill(const void* x, const void* x_left, const void* W_kv, const float
         const int nqc = (int)((n - q0) < qc ? (n - q0) : qc);
         QuerySpec qs{nullptr, nullptr, start + q0, 1};
         int32_t* sel = topk_idx ? topk_idx + q0 * k : sel_ws;
-        CSA_CUDA(index_scores((const char*)qI + (size_t)q0 * HI * cI * es, w + q0 * HI, idx_cache, qs, nqc, HI,
-                              cI, Nmax, m, sc, Nmax, t, st), "csa_prefill: indexer");
+        // the m tokens of one compressed block see the same entries: score them
+        // together against each key tile when the group fits one MMA
+        const int group = (m <= 4 && index_tc_supported(HI, cI, m)) ? m : 1;
+        CSA_CUDA(run_indexer((const char*)qI + (size_t)q0 * HI * cI * es, w + q0 * HI, idx_cache, qs, nqc, 1, HI,
+                             cI, Nmax, m, sc, Nmax, group, false, t, st), "csa_prefill: indexer");
         // visible count of query t is floor((start + q0 + t) / m); pass it through a
         // position-based valid rule: the top-k kernel reads valid[] = positions
         CSA_CUDA(topk_select_positions(sc, Nmax, start + q0, m, nqc, Nmax, k, sel, tws, st), "csa_prefill: top-k");
-        CSA_CUDA(mqa((const char*)q + (size_t)q0 * H * c * es, kv_cache, sel, k, qs, 1, nqc, H, c, Nmax,
+        CSA_CUDA(mqa((const char*)q + (size_t)q0 * H * c * es, kv_cache, sel, k, qs, 1, nqc, 1, H, c, Nmax,
                      sc_scale, sink, (char*)out + (size_t)q0 * H * c * es, lse ? lse + q0 * H : nullptr, mws,
                      t, st), "csa_prefill: mqa");
     }

@@ -1,0 +1,421 @@
+// Lightning indexer on the 5th-generation tensor cores [Notes §1.1, equation
+// I_{t,s}; Walk §2.3.1] ([Notes] = "DeepSeek-V4: 迈向高效百万级上下文智能" study
+// notes; [Walk] = the mlpod.com walk-through of the DeepSeek-V4 report):
+//   I[t][s] = sum_h w[t][h] * ReLU(qI[t][h] . K[s]),  s < floor(p_t / m).
+//
+// The head contraction is a dense GEMM: for a tile of 128 keys and a group
+// of g queries that see the same entries (decode: g = 1; prefill: the m
+// tokens of one compressed block share floor(p/m), so g = m),
+//   S^T[key][(query, head)] = K_tile (128 x cI) . Q_group^T (cI x g*HI)
+// runs as tcgen05.mma with M = 128 keys, N = g*HI (padded to a multiple of
+// 16), K = cI, operands in shared memory with 128-byte swizzle, fp32
+// accumulator in tensor memory. Each TMEM lane then holds one key's g*HI
+// dot products, so the epilogue thread owning that lane reduces
+// sum_h w_h * max(x_h, 0) with no cross-thread traffic.
+//
+// Persistent CTAs, one per SM. The (group, key tile) work list is cut into
+// equal contiguous ranges, one per CTA (the visible length of each group is
+// read on the device). Warp roles:
+//   warp 0     TMA producer: the group's Q rows once per group, then the key
+//              tiles through a ring of `stages` shared-memory buffers;
+//   warp 1     allocates TMEM; one lane issues the MMAs of each tile into one
+//              of two accumulator buffers and commits their completion;
+//   warps 2-5  epilogue: tcgen05.ld of the accumulator, ReLU/weight/head
+//              reduction, coalesced fp32 score stores.
+// Every wait is bounded; a timeout records CSA_ERR_TIMEOUT in the status
+// word, stops all roles, drains the copies in flight and frees TMEM.
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+#include "tmap.h"
+
+namespace csa {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kKeys = 128;
+constexpr uint32_t kWaitLimit = 1u << 24;
+
+struct IdxArgs {
+    QueryMap qm;
+    int nq, n_seq;
+    int group;          // queries sharing one key stream
+    int HI, cI;
+    int npad;           // MMA N
+    int kblocks;        // cI / 64
+    int stages;
+    int64_t Nmax;
+    int m;
+    const float* w;     // [nq][HI]
+    float* scores;      // [nq][ld]
+    int64_t ld;
+    int* status;
+    uint32_t stage_bytes, q_bytes, tmem_cols;
+};
+
+struct Smem {
+    uint8_t* stage0;    // stages x stage_bytes
+    uint8_t* q;         // q_bytes
+    float* w;           // 256
+    uint64_t* full;     // [stages]
+    uint64_t* empty;    // [stages]
+    uint64_t* tfull;    // [2]
+    uint64_t* tempty;   // [2]
+    uint64_t* qfull;
+    uint64_t* qempty;
+};
+
+__device__ __forceinline__ Smem carve(uint8_t* base, const IdxArgs& a) {
+    Smem s;
+    s.stage0 = base;
+    s.q = base + (size_t)a.stages * a.stage_bytes;
+    s.w = (float*)(s.q + a.q_bytes);
+    uint64_t* bars = (uint64_t*)(s.w + 256);
+    s.full = bars;
+    s.empty = bars + a.stages;
+    s.tfull = bars + 2 * a.stages;
+    s.tempty = s.tfull + 2;
+    s.qfull = s.tempty + 2;
+    s.qempty = s.qfull + 1;
+    return s;
+}
+
+__device__ __forceinline__ int group_seq(const IdxArgs& a, int g) {
+    int s = a.qm.seq_of(g * a.group);
+    return (s >= 0 && s < a.n_seq) ? s : -1;
+}
+__device__ __forceinline__ int64_t group_visible(const IdxArgs& a, int g) {
+    if (group_seq(a, g) < 0) return 0;
+    return visible_entries(a.qm.pos_of(g * a.group), a.m, a.Nmax);
+}
+__device__ __forceinline__ int64_t group_tiles(const IdxArgs& a, int g) {
+    return (group_visible(a, g) + kKeys - 1) / kKeys;
+}
+
+// Warp-cooperative: total tiles, and the (group, tile) at flat index `target`.
+__device__ int64_t total_tiles(const IdxArgs& a, int ngroups, int lane) {
+    int64_t sum = 0;
+    for (int g0 = 0; g0 < ngroups; g0 += 32) {
+        int g = g0 + lane;
+        sum += (g < ngroups) ? group_tiles(a, g) : 0;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    return sum;
+}
+__device__ void locate(const IdxArgs& a, int ngroups, int64_t target, int lane, int& g_out, int64_t& t_out) {
+    int64_t base = 0;
+    for (int g0 = 0; g0 < ngroups; g0 += 32) {
+        int g = g0 + lane;
+        int64_t c = (g < ngroups) ? group_tiles(a, g) : 0;
+        int64_t incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int64_t tot = __shfl_sync(0xffffffffu, incl, 31);
+        if (base + tot > target) {
+            unsigned mask = __ballot_sync(0xffffffffu, base + incl > target);
+            int L = __ffs(mask) - 1;
+            int64_t excl = __shfl_sync(0xffffffffu, incl - c, L);
+            g_out = g0 + L;
+            t_out = target - (base + excl);
+            return;
+        }
+        base += tot;
+    }
+    g_out = ngroups;
+    t_out = 0;
+}
+
+// Iterator over this CTA's (group, tile) range.
+struct Walk {
+    int g;
+    int64_t t, tiles_g;
+    __device__ void start(const IdxArgs& a, int g0, int64_t t0) {
+        g = g0;
+        t = t0;
+        tiles_g = (g < (a.nq + a.group - 1) / a.group) ? group_tiles(a, g) : 0;
+    }
+    __device__ void next(const IdxArgs& a, int ngroups) {
+        if (++t < tiles_g) return;
+        t = 0;
+        do {
+            ++g;
+            tiles_g = (g < ngroups) ? group_tiles(a, g) : 1;
+        } while (tiles_g == 0);
+    }
+    __device__ bool last_of_group() const { return t + 1 == tiles_g; }
+};
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                              int* status) {
+    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+        if (tc::mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 255u && *abort_flag) return false;
+    }
+    report_device_error(status, CSA_ERR_TIMEOUT);
+    *abort_flag = 1;
+    return false;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __grid_constant__ IdxArgs a,
+                                                                      const __grid_constant__ CUtensorMap tmK,
+                                                                      const __grid_constant__ CUtensorMap tmQ) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    Smem sm = carve(base, a);
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ngroups = (a.nq + a.group - 1) / a.group;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < a.stages; ++i) { tc::mbar_init(&sm.full[i], 1); tc::mbar_init(&sm.empty[i], 1); }
+        for (int i = 0; i < 2; ++i) { tc::mbar_init(&sm.tfull[i], 1); tc::mbar_init(&sm.tempty[i], 4); }
+        tc::mbar_init(sm.qfull, 1);
+        tc::mbar_init(sm.qempty, 1);
+        tc::fence_mbar_init();
+        s_abort = 0;
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(&s_tmem, a.tmem_cols);
+        tc::tmem_relinquish();
+        tc::tc_fence_before();
+    }
+    if (warp == 0 && lane == 0) {
+        tc::tma_prefetch_desc(&tmK);
+        tc::tma_prefetch_desc(&tmQ);
+    }
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = s_tmem;
+
+    // this CTA's share of the work list
+    const int64_t T = total_tiles(a, ngroups, lane);
+    const int64_t begin = T * blockIdx.x / gridDim.x;
+    const int64_t end = T * (blockIdx.x + 1) / gridDim.x;
+    const int64_t my = end - begin;
+    int g0 = ngroups;
+    int64_t t0 = 0;
+    if (my > 0) locate(a, ngroups, begin, lane, g0, t0);
+    volatile int* abort_flag = &s_abort;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0 && my > 0) {
+            Walk wk;
+            wk.start(a, g0, t0);
+            int cur = -1;
+            uint32_t switches = 0;
+            int64_t it = 0;
+            for (; it < my; ++it) {
+                if (wk.g != cur) {
+                    if (switches > 0 && !wait_or_abort(sm.qempty, (switches - 1) & 1, abort_flag, a.status)) break;
+                    tc::mbar_expect_tx(sm.qfull, a.q_bytes);
+                    for (int kb = 0; kb < a.kblocks; ++kb)
+                        tc::tma_load_2d(sm.q + (size_t)kb * a.npad * 128, &tmQ, sm.qfull, kb * 64,
+                                        wk.g * a.group * a.HI);
+                    cur = wk.g;
+                    ++switches;
+                }
+                const int s = (int)(it % a.stages);
+                if (it >= a.stages && !wait_or_abort(&sm.empty[s], ((it / a.stages) - 1) & 1, abort_flag, a.status))
+                    break;
+                tc::mbar_expect_tx(&sm.full[s], a.stage_bytes);
+                const int row = (int)((int64_t)group_seq(a, wk.g) * a.Nmax + wk.t * kKeys);
+                uint8_t* dst = sm.stage0 + (size_t)s * a.stage_bytes;
+                for (int kb = 0; kb < a.kblocks; ++kb)
+                    tc::tma_load_2d(dst + (size_t)kb * kKeys * 128, &tmK, &sm.full[s], kb * 64, row);
+                wk.next(a, ngroups);
+            }
+            // drain: the copies of the last `stages` tiles (and the last Q) must land
+            for (int64_t j = (it > a.stages ? it - a.stages : 0); j < it; ++j)
+                tc::mbar_wait(&sm.full[j % a.stages], (j / a.stages) & 1, kWaitLimit);
+            if (switches > 0) tc::mbar_wait(sm.qfull, (switches - 1) & 1, kWaitLimit);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && my > 0) {
+            Walk wk;
+            wk.start(a, g0, t0);
+            int cur = -1;
+            uint32_t switches = 0;
+            const uint32_t idesc = tc::idesc_bf16_f32(128, a.npad, 0, 0);
+            const uint32_t q_addr = tc::smem_u32(sm.q);
+            const uint32_t st_addr = tc::smem_u32(sm.stage0);
+            int64_t it = 0;
+            for (; it < my; ++it) {
+                if (wk.g != cur) {
+                    if (!wait_or_abort(sm.qfull, switches & 1, abort_flag, a.status)) break;
+                    cur = wk.g;
+                    ++switches;
+                }
+                const int s = (int)(it % a.stages);
+                const int buf = (int)(it & 1);
+                if (!wait_or_abort(&sm.full[s], (it / a.stages) & 1, abort_flag, a.status)) break;
+                if (it >= 2 && !wait_or_abort(&sm.tempty[buf], ((it >> 1) - 1) & 1, abort_flag, a.status)) break;
+                tc::tc_fence_after();
+                const uint32_t a_base = st_addr + (uint32_t)s * a.stage_bytes;
+                const uint32_t d = tmem + (uint32_t)(buf * a.npad);
+                for (int ks = 0; ks < a.kblocks * 4; ++ks) {
+                    uint64_t ad = tc::sdesc_sw128(a_base + (ks >> 2) * (kKeys * 128) + (ks & 3) * 32, 16, 1024);
+                    uint64_t bd = tc::sdesc_sw128(q_addr + (ks >> 2) * (a.npad * 128) + (ks & 3) * 32, 16, 1024);
+                    tc::umma_bf16(d, ad, bd, idesc, ks > 0 ? 1u : 0u);
+                }
+                tc::umma_commit(&sm.empty[s]);
+                tc::umma_commit(&sm.tfull[buf]);
+                if (wk.last_of_group() || it + 1 == my) tc::umma_commit(sm.qempty);
+                wk.next(a, ngroups);
+            }
+            // the last commit covers every MMA issued before it
+            if (it > 0) tc::mbar_wait(&sm.tfull[(it - 1) & 1], ((it - 1) >> 1) & 1, kWaitLimit);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int quad = warp & 3;                 // TMEM lane quadrant of this warp
+        const int row = quad * 32 + lane;          // key within the tile
+        const int ethread = threadIdx.x - 64;      // 0..127
+        Walk wk;
+        wk.start(a, g0, t0);
+        int cur = -1;
+        int64_t vis = 0;
+        for (int64_t it = 0; it < my; ++it) {
+            if (wk.g != cur) {
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                for (int c = ethread; c < a.npad; c += 128) {
+                    int gq = c / a.HI, h = c % a.HI;
+                    int tq = wk.g * a.group + gq;
+                    sm.w[c] = (gq < a.group && tq < a.nq) ? a.w[(int64_t)tq * a.HI + h] : 0.f;
+                }
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                cur = wk.g;
+                vis = group_visible(a, wk.g);
+            }
+            const int buf = (int)(it & 1);
+            if (!wait_or_abort(&sm.tfull[buf], (it >> 1) & 1, abort_flag, a.status)) break;
+            tc::tc_fence_after();
+            float sc[4] = {0.f, 0.f, 0.f, 0.f};
+            const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * a.npad);
+            for (int cc = 0; cc < a.npad; cc += 16) {
+                float v[16];
+                tc::tmem_ld16(taddr + cc, v);
+                tc::tmem_ld_wait();
+                float part = 0.f;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) part = fmaf(sm.w[cc + i], fmaxf(v[i], 0.f), part);
+                const int gq = (a.group > 1) ? cc / a.HI : 0;
+                if (gq == 0) sc[0] += part;
+                else if (gq == 1) sc[1] += part;
+                else if (gq == 2) sc[2] += part;
+                else sc[3] += part;
+            }
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&sm.tempty[buf]);
+            const int64_t key = wk.t * kKeys + row;
+            if (key < vis) {
+#pragma unroll
+                for (int gq = 0; gq < 4; ++gq) {
+                    const int tq = wk.g * a.group + gq;
+                    if (gq < a.group && tq < a.nq) a.scores[(int64_t)tq * a.ld + key] = sc[gq];
+                }
+            }
+            wk.next(a, ngroups);
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, a.tmem_cols);
+    }
+}
+
+// -inf for the columns a query cannot see (s >= floor(p/m)), so the score
+// matrix is complete; the fused paths skip it (top-k reads only visible ones).
+__global__ void fill_invisible_kernel(float* scores, int64_t ld, QueryMap qm, int nq, int n_seq, int64_t Nmax,
+                                      int m) {
+    const int t = blockIdx.x;
+    int s = qm.seq_of(t);
+    int64_t vis = (s >= 0 && s < n_seq) ? visible_entries(qm.pos_of(t), m, Nmax) : 0;
+    for (int64_t c = vis + (int64_t)blockIdx.y * blockDim.x + threadIdx.x; c < Nmax; c += (int64_t)gridDim.y * blockDim.x)
+        scores[(int64_t)t * ld + c] = -INFINITY;
+}
+
+static int num_sms() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+bool index_tc_supported(int HI, int cI, int group) {
+    if (cI % 64 != 0 || cI > 256) return false;
+    if (group < 1 || group > 4) return false;
+    if (group > 1 && HI % 16 != 0) return false;
+    int n = group * HI;
+    return n <= 256;
+}
+
+cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, QuerySpec qs, int nq, int n_seq, int HI,
+                            int cI, int64_t Nmax, int m, float* scores, int64_t ld, int group, bool fill_invisible,
+                            int* status, cudaStream_t st) {
+    if (nq == 0 || Nmax == 0) return cudaSuccess;
+    IdxArgs a{};
+    a.qm = QueryMap{qs.seq, qs.pos, qs.pos_base, qs.single_seq};
+    a.nq = nq;
+    a.n_seq = n_seq;
+    a.group = group;
+    a.HI = HI;
+    a.cI = cI;
+    int n = group * HI;
+    a.npad = n < 16 ? 16 : ((n + 15) / 16) * 16;
+    a.kblocks = cI / 64;
+    a.Nmax = Nmax;
+    a.m = m;
+    a.w = w;
+    a.scores = scores;
+    a.ld = ld;
+    a.status = status;
+    a.stage_bytes = (uint32_t)(kKeys * cI * 2);
+    a.q_bytes = (uint32_t)(a.npad * cI * 2);
+    uint32_t cols = 32;
+    while (cols < (uint32_t)(2 * a.npad)) cols <<= 1;
+    a.tmem_cols = cols;
+    const size_t fixed = 1024 + a.q_bytes + 256 * sizeof(float) + 64 * sizeof(uint64_t);
+    const size_t budget = 226 * 1024;
+    int stages = (int)((budget - fixed) / a.stage_bytes);
+    if (stages > 8) stages = 8;
+    if (stages < 2) return cudaErrorInvalidConfiguration;
+    a.stages = stages;
+    const size_t smem = fixed + (size_t)stages * a.stage_bytes;
+
+    CUtensorMap tmK, tmQ;
+    if (!make_tmap_bf16_2d(&tmK, K, (uint64_t)n_seq * Nmax, cI, cI, kKeys, 64)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_2d(&tmQ, qI, (uint64_t)nq * HI, cI, cI, a.npad, 64)) return cudaErrorInvalidValue;
+
+    cudaError_t e;
+    if (fill_invisible) {
+        QueryMap qm = a.qm;
+        CSA_LAUNCH(st, "index_fill_invisible",
+                   fill_invisible_kernel<<<dim3(nq, 8), 256, 0, st>>>(scores, ld, qm, nq, n_seq, Nmax, m));
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    e = cudaFuncSetAttribute(index_scores_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    CSA_LAUNCH(st, "index_scores_tc", index_scores_tc_kernel<<<num_sms(), kThreads, smem, st>>>(a, tmK, tmQ));
+    return cudaGetLastError();
+}
+
+}  // namespace csa

@@ -51,10 +51,20 @@ cudaError_t compress_hca(const void* proj, const float* bias, int64_t n, int c, 
 cudaError_t project(const void* x, const void* W, int64_t n, int d, int M, float* out, ElemType t,
                     cudaStream_t st);
 
-// indexer.cu: scores[t, 0..Nmax) with ld = ld_scores; -inf past the visible range
+// indexer.cu (FFMA, fp32 mode): scores[t, 0..Nmax) with ld = ld_scores;
+// -inf past the visible range
 cudaError_t index_scores(const void* qI, const float* w, const void* K, QuerySpec qs, int nq,
                          int HI, int cI, int64_t Nmax, int m, float* scores, int64_t ld_scores,
                          ElemType t, cudaStream_t st);
+// indexer_tc.cu (tcgen05, bf16): groups of `group` consecutive queries share
+// one visible range; fill_invisible writes -inf past each visible range.
+bool index_tc_supported(int HI, int cI, int group);
+cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, QuerySpec qs, int nq, int n_seq, int HI,
+                            int cI, int64_t Nmax, int m, float* scores, int64_t ld, int group, bool fill_invisible,
+                            int* status, cudaStream_t st);
+
+// api.cu: device address of the status word on the current device
+int* device_status();
 
 // topk.cu
 size_t topk_workspace_bytes(int nq, int64_t ncols, int k);
@@ -68,7 +78,7 @@ cudaError_t topk_select_positions(const float* scores, int64_t ld, int64_t pos_b
 // mqa.cu: sparse (idx != nullptr) or dense (entries s < pos/mp) shared-KV MQA
 size_t mqa_workspace_bytes(int nq, int H, int c, int64_t max_entries, ElemType t);
 cudaError_t mqa(const void* q, const void* KV, const int32_t* idx, int k, QuerySpec qs, int mp,
-                int nq, int H, int c, int64_t Nmax, float scale, const float* sink, void* out,
+                int nq, int n_seq, int H, int c, int64_t Nmax, float scale, const float* sink, void* out,
                 float* lse, void* ws, ElemType t, cudaStream_t st);
 
 }  // namespace csa

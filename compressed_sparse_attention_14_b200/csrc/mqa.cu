@@ -29,6 +29,7 @@ struct MqaPartialArgs {
     const int32_t* idx;   // nullable -> dense
     int k;
     QueryMap qm;
+    int n_seq;
     int mp;
     int H, c;
     int64_t Nmax;
@@ -56,9 +57,12 @@ __global__ void __launch_bounds__(256) mqa_partial_ffma_kernel(MqaPartialArgs a)
     const int h = h0 + warp;
 
     const T* qg = (const T*)a.q + (int64_t)t * a.H * c;
-    const T* KVb = (const T*)a.KV + (int64_t)a.qm.seq_of(t) * a.Nmax * c;
+    const int seq = a.qm.seq_of(t);
+    const bool seq_ok = seq >= 0 && seq < a.n_seq;
+    const T* KVb = (const T*)a.KV + (int64_t)(seq_ok ? seq : 0) * a.Nmax * c;
     int64_t n_ent;
-    if (a.idx) n_ent = a.k;
+    if (!seq_ok) n_ent = 0;
+    else if (a.idx) n_ent = a.k;
     else n_ent = visible_entries(a.qm.pos_of(t), a.mp, a.Nmax);
     const int64_t e_beg = (int64_t)split * a.split_len;
     int64_t e_end = e_beg + a.split_len;
@@ -193,7 +197,7 @@ size_t mqa_workspace_bytes(int nq, int H, int c, int64_t max_entries, ElemType) 
 }
 
 cudaError_t mqa(const void* q, const void* KV, const int32_t* idx, int k, QuerySpec qs, int mp,
-                int nq, int H, int c, int64_t Nmax, float scale, const float* sink, void* out,
+                int nq, int n_seq, int H, int c, int64_t Nmax, float scale, const float* sink, void* out,
                 float* lse, void* ws, ElemType t, cudaStream_t st) {
     if (nq == 0) return cudaSuccess;
     const int64_t max_entries = idx ? k : Nmax;
@@ -201,7 +205,7 @@ cudaError_t mqa(const void* q, const void* KV, const int32_t* idx, int k, QueryS
     MqaPartialArgs a{};
     a.q = q; a.KV = KV; a.idx = idx; a.k = k;
     a.qm = QueryMap{qs.seq, qs.pos, qs.pos_base, qs.single_seq};
-    a.mp = mp; a.H = H; a.c = c; a.Nmax = Nmax; a.scale = scale; a.nsplit = ns;
+    a.n_seq = n_seq; a.mp = mp; a.H = H; a.c = c; a.Nmax = Nmax; a.scale = scale; a.nsplit = ns;
     int64_t per = (max_entries + ns - 1) / ns;
     a.split_len = ((per + kMqaTile - 1) / kMqaTile) * kMqaTile;
     if (a.split_len == 0) a.split_len = kMqaTile;

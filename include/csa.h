@@ -142,11 +142,13 @@ int hca_compress_from_hidden(const void* x, const void* W, const float* bias, in
  *   for s < floor(pos[t] / m); columns s >= that are set to -inf.
  *   qI [nq, HI, cI] (dtype), w [nq, HI] fp32, K [B, Nmax, cI] (dtype),
  *   pos [nq] int32, seq_of_q [nq] int32 or NULL (query t reads sequence t),
- *   scores [nq, Nmax] fp32.
- * cI % 8 == 0, cI <= CSA_MAX_INDEX_DIM, HI <= CSA_MAX_INDEX_HEADS.
+ *   n_seq = B (sequences in K; a query whose sequence is outside [0, n_seq)
+ *   sees no entry), scores [nq, Nmax] fp32.
+ * cI % 8 == 0, cI <= CSA_MAX_INDEX_DIM, HI <= CSA_MAX_INDEX_HEADS; in bf16
+ * mode (tensor cores) cI % 64 == 0. nq <= 65535.
  * ------------------------------------------------------------------------ */
 int csa_index_scores(const void* qI, const float* w, const void* K, const int32_t* pos,
-                     const int32_t* seq_of_q, int nq, int HI, int cI, int64_t Nmax, int m,
+                     const int32_t* seq_of_q, int nq, int n_seq, int HI, int cI, int64_t Nmax, int m,
                      float* scores, int dtype, void* stream);
 
 /* a5. Top-k selection [Walk §2.3.1: the k highest-scoring compressed blocks
@@ -182,7 +184,7 @@ int csa_topk_from_scores_noalloc(const float* scores, int64_t ld, const int32_t*
 /* a4+a5: indexer then top-k over the visible entries of each query. */
 size_t csa_index_topk_workspace_size(int nq, int64_t Nmax, int k, int dtype);
 int csa_index_topk(const void* qI, const float* w, const void* K, const int32_t* pos,
-                   const int32_t* seq_of_q, int nq, int HI, int cI, int64_t Nmax, int m, int k,
+                   const int32_t* seq_of_q, int nq, int n_seq, int HI, int cI, int64_t Nmax, int m, int k,
                    int32_t* idx, float* top_scores, void* ws, size_t ws_bytes, int dtype,
                    void* stream);
 
@@ -194,14 +196,16 @@ int csa_index_topk(const void* qI, const float* w, const void* K, const int32_t*
  *   out[t][h] = sum_s exp(z_s) KV[s] / (sum_s exp(z_s) + exp(sink[h])),
  *   lse[t][h] = log of that denominator (-inf for an empty set, no sink).
  *   q [nq, H, c] (dtype), KV [B, Nmax, c] (dtype), idx [nq, k] int32,
- *   seq_of_q [nq] or NULL (identity), sink [H] fp32 or NULL (no sink term),
+ *   seq_of_q [nq] or NULL (identity), n_seq = B (sequences in KV), sink [H]
+ *   fp32 or NULL (no sink term),
  *   out [nq, H, c] (dtype), lse [nq, H] fp32 or NULL.
  *   scale == 0 selects 1/sqrt(c).
- * c % 8 == 0, c <= CSA_MAX_HEAD_DIM, H <= CSA_MAX_HEADS, k <= CSA_MAX_TOPK.
+ * c % 32 == 0, c <= CSA_MAX_HEAD_DIM, H <= CSA_MAX_HEADS, k <= CSA_MAX_TOPK,
+ * nq <= 65535.
  * ------------------------------------------------------------------------ */
 size_t csa_sparse_mqa_workspace_size(int nq, int H, int c, int k, int dtype);
 int csa_sparse_mqa(const void* q, const void* KV, const int32_t* idx, const int32_t* seq_of_q,
-                   int nq, int H, int c, int64_t Nmax, int k, float scale, const float* sink,
+                   int nq, int n_seq, int H, int c, int64_t Nmax, int k, float scale, const float* sink,
                    void* out, float* lse, void* ws, size_t ws_bytes, int dtype, void* stream);
 
 /* a7. Dense shared-KV MQA over every visible HCA entry [Walk §2.3.2: after
@@ -209,7 +213,7 @@ int csa_sparse_mqa(const void* q, const void* KV, const int32_t* idx, const int3
  * with the entry set s < floor(pos[t] / mp). */
 size_t hca_dense_mqa_workspace_size(int nq, int H, int c, int64_t Nmax, int dtype);
 int hca_dense_mqa(const void* q, const void* KV, const int32_t* pos, const int32_t* seq_of_q,
-                  int nq, int H, int c, int64_t Nmax, int mp, float scale, const float* sink,
+                  int nq, int n_seq, int H, int c, int64_t Nmax, int mp, float scale, const float* sink,
                   void* out, float* lse, void* ws, size_t ws_bytes, int dtype, void* stream);
 
 /* ------------------------------------------------------------------------

@@ -56,10 +56,18 @@ def test_invalid_arguments_are_rejected_on_the_host():
     assert L.csa_topk_from_scores(fake, 16, None, 1, 1, 16, 0, fake, None, None, 0, None) == csa.CSA_ERR_UNSUPPORTED
     assert L.csa_topk_from_scores(fake, 16, None, 1, 1, 16, 4096, fake, None, None, 0, None) == csa.CSA_ERR_UNSUPPORTED
     # attention shapes beyond the kernels
-    assert L.csa_sparse_mqa(fake, fake, fake, None, 1, 256, 128, 8, 4, 0.0, None, fake, None, None, 0,
+    assert L.csa_sparse_mqa(fake, fake, fake, None, 1, 1, 256, 128, 8, 4, 0.0, None, fake, None, None, 0,
                             csa.CSA_BF16, None) == csa.CSA_ERR_UNSUPPORTED
-    assert L.csa_sparse_mqa(fake, fake, fake, None, 1, 8, 1024, 8, 4, 0.0, None, fake, None, None, 0,
+    assert L.csa_sparse_mqa(fake, fake, fake, None, 1, 1, 8, 1024, 8, 4, 0.0, None, fake, None, None, 0,
                             csa.CSA_BF16, None) == csa.CSA_ERR_UNSUPPORTED
+    # identity query->sequence map needs one sequence per query
+    assert L.csa_sparse_mqa(fake, fake, fake, None, 4, 2, 8, 128, 8, 4, 0.0, None, fake, None, None, 0,
+                            csa.CSA_BF16, None) == csa.CSA_ERR_INVALID_ARG
+    # bf16 indexer runs on tensor cores: cI must be a multiple of 64
+    assert L.csa_index_scores(fake, fake, fake, fake, None, 2, 2, 4, 32, 16, 4, fake, csa.CSA_BF16,
+                              None) == csa.CSA_ERR_UNSUPPORTED
+    # more rows than one launch grid holds
+    assert L.csa_topk_from_scores(fake, 16, None, 1, 70000, 16, 4, fake, None, None, 0, None) == csa.CSA_ERR_UNSUPPORTED
     # missing / short workspace
     need = L.csa_decode_workspace_size(2, 1024, 8, 128, 4, 64, 16, csa.CSA_BF16)
     assert need > 0
@@ -71,13 +79,13 @@ def test_invalid_arguments_are_rejected_on_the_host():
     assert rc == csa.CSA_ERR_WORKSPACE
     # prefill: start not a multiple of m, cache too small, missing left rows
     args = dict(n=8, Nmax=4, start=4)
-    rc = L.csa_prefill(fake, fake, fake, fake, fake, fake, 2, 8, 64, 4, 32, 32, fake, fake, 16, fake, fake, fake,
+    rc = L.csa_prefill(fake, fake, fake, fake, fake, fake, 2, 8, 64, 4, 32, 64, fake, fake, 16, fake, fake, fake,
                        8, 4, 4, 0.0, None, fake, None, None, None, 0, csa.CSA_BF16, None)
     assert rc == csa.CSA_ERR_INVALID_ARG
-    rc = L.csa_prefill(fake, fake, fake, fake, fake, fake, 4, 8, 64, 4, 32, 32, fake, fake, 2, fake, fake, fake,
+    rc = L.csa_prefill(fake, fake, fake, fake, fake, fake, 4, 8, 64, 4, 32, 64, fake, fake, 2, fake, fake, fake,
                        8, 4, 4, 0.0, None, fake, None, None, None, 0, csa.CSA_BF16, None)
     assert rc == csa.CSA_ERR_INVALID_ARG
-    rc = L.csa_prefill(fake, None, fake, fake, fake, fake, 4, 8, 64, 4, 32, 32, fake, fake, 16, fake, fake, fake,
+    rc = L.csa_prefill(fake, None, fake, fake, fake, fake, 4, 8, 64, 4, 32, 64, fake, fake, 16, fake, fake, fake,
                        8, 4, 4, 0.0, None, fake, None, None, None, 0, csa.CSA_BF16, None)
     assert rc == csa.CSA_ERR_INVALID_ARG
     del args
