@@ -249,9 +249,14 @@ def decode_workload(shape, rank):
 
     h2d = sum(v.numel() * v.element_size() for v in pinned.values())
     d2h = out_h.numel() * out_h.element_size()
+    mqa_bytes = B * (s.k * s.c * 2 + 2 * s.heads * s.c * 2)
+    kernels = {
+        "index_scores_tc": dict(bound="hbm", work=idx_kernel_bytes, files=("indexer_tc.cu", "tc.cuh", "common.cuh")),
+        "mqa_tc": dict(bound="hbm", work=mqa_bytes, files=("mqa_tc.cu", "tc.cuh", "common.cuh")),
+        "topk_select": dict(bound="hbm", work=v_sum * 4 + B * s.k * 4, files=("topk.cu",)),
+    }
     return dict(step=step, e2e_step=e2e_step, units=B, unit="queries/s", h2d=h2d, d2h=d2h,
-                dominant="index_scores_ffma", dominant_bytes=idx_kernel_bytes, dominant_bound="hbm",
-                dominant_files=("indexer.cu", "common.cuh"), step_bytes=step_bytes,
+                kernels=kernels, step_bytes=step_bytes,
                 config=dict(workload=s.name, batch=B, ctx_len=f"U[{s.ctx_lo},{s.ctx_hi}]", m=s.m,
                             entries_max=s.n_max, head_dim=s.c, heads=s.heads, index_heads=s.idx_heads,
                             index_dim=s.idx_dim, topk=s.k, visible_entries_total=int(v_sum),
@@ -289,11 +294,12 @@ def hca_decode_workload(rank):
 
     kv_bytes = B * s.n_max * s.c * 2.0
     step_bytes = kv_bytes + 2 * B * s.heads * s.c * 2
+    kernels = {"mqa_tc": dict(bound="hbm", work=kv_bytes + B * s.heads * s.c * 2,
+                              files=("mqa_tc.cu", "tc.cuh", "common.cuh")),
+               "mqa_combine": dict(bound="hbm", work=2 * B * s.heads * s.c * 2, files=("mqa.cu",))}
     return dict(step=step, e2e_step=e2e_step, units=B, unit="queries/s",
                 h2d=sum(v.numel() * v.element_size() for v in pinned.values()),
-                d2h=out_h.numel() * out_h.element_size(),
-                dominant="mqa_partial_ffma", dominant_bytes=kv_bytes + B * s.heads * s.c * 2,
-                dominant_bound="hbm", dominant_files=("mqa.cu", "common.cuh"), step_bytes=step_bytes,
+                d2h=out_h.numel() * out_h.element_size(), kernels=kernels, step_bytes=step_bytes,
                 config=dict(workload=s.name.split("_plus")[0], batch=B, ctx_len=s.ctx, mp=s.mp, entries=s.n_max,
                             head_dim=s.c, heads=s.heads, l2="flushed before every timed step (256 MiB write)"))
 
@@ -320,9 +326,11 @@ def hca_compress_workload(rank):
         out_h.copy_(out, non_blocking=True)
 
     flops = 2.0 * n * d * 2 * s.c
+    kernels = {"project_ffma": dict(bound="tensor", work=flops, files=("gemm.cu", "common.cuh")),
+               "hca_compress": dict(bound="hbm", work=n * 2 * s.c * 4 + (n // s.mp) * s.c * 2,
+                                    files=("compress.cu", "common.cuh"))}
     return dict(step=step, e2e_step=e2e_step, units=n, unit="tokens/s", h2d=x_h.numel() * 2,
-                d2h=out_h.numel() * 2, dominant="project_ffma", dominant_flops=flops, dominant_bound="tensor",
-                dominant_files=("gemm.cu", "common.cuh"), step_bytes=n * d * 2.0,
+                d2h=out_h.numel() * 2, kernels=kernels, step_bytes=None,
                 config=dict(workload=f"hca_compress_chunk{n}_d{d}", tokens=n, d=d, mp=s.mp, head_dim=s.c,
                             l2="inputs larger than L2 and flushed before every timed step"))
 
@@ -357,10 +365,14 @@ def prefill_workload(rank):
                         m=s.m, out=out, ws=ws)
         out_h.copy_(out, non_blocking=True)
 
+    mqa_flops = 4.0 * n * s.heads * s.k * s.c
+    proj_flops = 2.0 * (n + s.m) * s.d * 4 * (s.c + s.idx_dim)
+    kernels = {"index_scores_tc": dict(bound="tensor", work=idx_flops, files=("indexer_tc.cu", "tc.cuh", "common.cuh")),
+               "mqa_tc": dict(bound="tensor", work=mqa_flops, files=("mqa_tc.cu", "tc.cuh", "common.cuh")),
+               "project_ffma": dict(bound="tensor", work=proj_flops, files=("gemm.cu", "common.cuh"))}
     return dict(step=step, e2e_step=e2e_step, units=n, unit="tokens/s",
                 h2d=sum(v.numel() * v.element_size() for v in pinned.values()), d2h=out_h.numel() * 2,
-                dominant="index_scores_ffma", dominant_flops=idx_flops, dominant_bound="tensor",
-                dominant_files=("indexer.cu", "common.cuh"), step_bytes=None,
+                kernels=kernels, step_bytes=None,
                 config=dict(workload=s.name, tokens=n, start=inp["start"], d=s.d, m=s.m, head_dim=s.c,
                             heads=s.heads, index_heads=s.idx_heads, index_dim=s.idx_dim, topk=s.k,
                             causal_pairs=int(pairs), l2="inputs larger than L2"))
@@ -576,28 +588,38 @@ def run_ours(args, rank, world, local):
     units = wl["units"]
     value = world * units / (ms_step / 1e3)
     peaks = measured_peaks()
-    dom = wl["dominant"]
-    dom_ms, dom_n = trace.get(dom, (float("nan"), 0))
-    dom_avg_s = dom_ms / max(dom_n, 1) / 1e3
-    if wl["dominant_bound"] == "hbm":
-        per_launch = wl["dominant_bytes"] * args.steps / max(dom_n, 1)
-        achieved = per_launch / dom_avg_s / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"] + " hbm_gbs"}
-    else:
-        per_launch = wl["dominant_flops"] * args.steps / max(dom_n, 1)
-        achieved = per_launch / dom_avg_s / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"], "peak_source": peaks["source"] + " bf16_tflops"}
-    roof["kernel"] = dom
-    roof["launches_per_step"] = dom_n / args.steps
-    roof["traffic"] = ncu_traffic(dom, args.workload, wl["dominant_files"])
+
+    def roofline_of(name):
+        info = wl["kernels"][name]
+        k_ms, k_n = trace.get(name, (float("nan"), 0))
+        avg_s = k_ms / max(k_n, 1) / 1e3
+        per_launch = info["work"] * args.steps / max(k_n, 1)   # the work is per step
+        if info["bound"] == "hbm":
+            achieved = per_launch / avg_s / 1e9
+            r = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                 "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"] + " hbm_gbs (copy, burst)"}
+        else:
+            achieved = per_launch / avg_s / 1e12
+            r = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                 "frac": achieved / peaks["bf16_tflops"], "peak_source": peaks["source"] + " bf16_tflops (burst)"}
+        r["kernel"] = name
+        r["launches_per_step"] = k_n / args.steps
+        r["ms_per_launch"] = avg_s * 1e3
+        r["traffic"] = ncu_traffic(name, args.workload, info["files"])
+        return r
+
+    timed = [n for n in wl["kernels"] if n in trace]
+    dom = max(timed, key=lambda n: trace[n][0]) if timed else next(iter(wl["kernels"]))
+    roof = roofline_of(dom)
+    others = {n: roofline_of(n) for n in timed if n != dom}
 
     line = {"metric": METRIC, "value": value, "unit": wl["unit"], "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": wl["config"],
             "roofline": roof,
             "kernels_ms_per_step": {k: v[0] / args.steps for k, v in sorted(trace.items())},
+            "other_kernels_roofline": {n: {k: r[k] for k in ("bound", "achieved", "unit", "frac")}
+                                       for n, r in others.items()},
             "e2e": {"value": world * units / (e2e_ms / 1e3), "unit": wl["unit"], "h2d_bytes_per_step": wl["h2d"],
                     "d2h_bytes_per_step": wl["d2h"]},
             "gpu_launches": launches, "clocks": clk, "wall_s_timed": t_wall}

@@ -109,6 +109,17 @@ static int check_attn_shape(int H, int c) {
     return CSA_OK;
 }
 
+static int check_attn_mode(int H, int c, ElemType t) {
+    if (t == ElemType::BF16 && !mqa_tc_supported(H, c))
+        return fail(CSA_ERR_UNSUPPORTED, "bf16 MQA needs c a multiple of 128 (c=%d)", c);
+    return CSA_OK;
+}
+
+static int check_cache_rows(int64_t n_seq, int64_t Nmax) {
+    if (n_seq * Nmax > INT32_MAX) return fail(CSA_ERR_UNSUPPORTED, "cache rows n_seq*Nmax beyond int32");
+    return CSA_OK;
+}
+
 static int check_index_shape(int HI, int cI) {
     if (HI < 1 || HI > CSA_MAX_INDEX_HEADS)
         return fail(CSA_ERR_UNSUPPORTED, "HI=%d outside [1, %d]", HI, CSA_MAX_INDEX_HEADS);
@@ -314,6 +325,7 @@ int csa_index_scores(const void* qI, const float* w, const void* K, const int32_
     if (nq < 0 || Nmax < 0 || m < 1 || n_seq < 1) return fail(CSA_ERR_INVALID_ARG, "bad nq/n_seq/Nmax/m");
     if (!seq_of_q && n_seq < nq) return fail(CSA_ERR_INVALID_ARG, "seq_of_q is NULL (query t reads sequence t) but n_seq < nq");
     if (Nmax > INT32_MAX) return fail(CSA_ERR_UNSUPPORTED, "Nmax beyond int32 entry indices");
+    CSA_TRY(check_cache_rows(n_seq, Nmax));
     if (nq == 0 || Nmax == 0) return CSA_OK;
     CSA_TRY(check_ptr(qI, "qI"));
     CSA_TRY(check_ptr(w, "w"));
@@ -402,6 +414,8 @@ int csa_sparse_mqa(const void* q, const void* KV, const int32_t* idx, const int3
     ElemType t;
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_attn_shape(H, c));
+    CSA_TRY(check_attn_mode(H, c, t));
+    CSA_TRY(check_cache_rows(n_seq, Nmax));
     CSA_TRY(check_k(k));
     CSA_TRY(check_rows(nq, "csa_sparse_mqa"));
     if (nq < 0 || Nmax < 0 || n_seq < 1) return fail(CSA_ERR_INVALID_ARG, "bad nq/n_seq/Nmax");
@@ -433,6 +447,8 @@ int hca_dense_mqa(const void* q, const void* KV, const int32_t* pos, const int32
     ElemType t;
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_attn_shape(H, c));
+    CSA_TRY(check_attn_mode(H, c, t));
+    CSA_TRY(check_cache_rows(n_seq, Nmax));
     CSA_TRY(check_rows(nq, "hca_dense_mqa"));
     if (nq < 0 || Nmax < 0 || mp < 1 || n_seq < 1) return fail(CSA_ERR_INVALID_ARG, "bad nq/n_seq/Nmax/mp");
     if (!seq_of_q && n_seq < nq) return fail(CSA_ERR_INVALID_ARG, "seq_of_q is NULL (query t reads sequence t) but n_seq < nq");
@@ -470,6 +486,8 @@ int csa_decode(const void* qI, const float* w, const void* idx_cache, const void
     CSA_TRY(check_index_shape(HI, cI));
     CSA_TRY(check_index_mode(HI, cI, t));
     CSA_TRY(check_attn_shape(H, c));
+    CSA_TRY(check_attn_mode(H, c, t));
+    CSA_TRY(check_cache_rows(B, Nmax));
     CSA_TRY(check_k(k));
     CSA_TRY(check_rows(B, "csa_decode"));
     if (B < 0 || Nmax < 0 || m < 1) return fail(CSA_ERR_INVALID_ARG, "bad B/Nmax/m");
@@ -536,6 +554,7 @@ int csa_prefill(const void* x, const void* x_left, const void* W_kv, const float
     CSA_TRY(check_index_shape(HI, cI));
     CSA_TRY(check_index_mode(HI, cI, t));
     CSA_TRY(check_attn_shape(H, c));
+    CSA_TRY(check_attn_mode(H, c, t));
     CSA_TRY(check_k(k));
     CSA_TRY(check_compress(n, c, m, 64, "csa_prefill"));
     if (d < 8 || d % 8) return fail(CSA_ERR_INVALID_ARG, "d=%d must be a positive multiple of 8", d);

@@ -64,6 +64,7 @@ struct Smem {
     uint64_t* tempty;   // [2]
     uint64_t* qfull;
     uint64_t* qempty;
+    uint64_t* fin;
 };
 
 __device__ __forceinline__ Smem carve(uint8_t* base, const IdxArgs& a) {
@@ -78,6 +79,7 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const IdxArgs& a) {
     s.tempty = s.tfull + 2;
     s.qfull = s.tempty + 2;
     s.qempty = s.qfull + 1;
+    s.fin = s.qempty + 1;
     return s;
 }
 
@@ -180,6 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
         for (int i = 0; i < 2; ++i) { tc::mbar_init(&sm.tfull[i], 1); tc::mbar_init(&sm.tempty[i], 4); }
         tc::mbar_init(sm.qfull, 1);
         tc::mbar_init(sm.qempty, 1);
+        tc::mbar_init(sm.fin, 1);
         tc::fence_mbar_init();
         s_abort = 0;
     }
@@ -273,8 +276,9 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
                 if (wk.last_of_group() || it + 1 == my) tc::umma_commit(sm.qempty);
                 wk.next(a, ngroups);
             }
-            // the last commit covers every MMA issued before it
-            if (it > 0) tc::mbar_wait(&sm.tfull[(it - 1) & 1], ((it - 1) >> 1) & 1, kWaitLimit);
+            // a last commit covers every MMA this thread issued (also on abort)
+            tc::umma_commit(sm.fin);
+            tc::mbar_wait(sm.fin, 0, kWaitLimit);
         }
     } else {
         // ------------------------------------------------------------ epilogue

@@ -75,6 +75,13 @@ cudaError_t topk_select(const float* scores, int64_t ld, const int32_t* valid, i
 cudaError_t topk_select_positions(const float* scores, int64_t ld, int64_t pos_base, int m, int nq,
                                   int64_t ncols, int k, int32_t* idx, void* ws, cudaStream_t st);
 
+// mqa_tc.cu: tensor-core shared-KV MQA (bf16); ws holds split partials when nsplit > 1
+bool mqa_tc_supported(int H, int c);
+int mqa_tc_nsplit(int nq, int H, int64_t max_entries, int num_sms);
+cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, QuerySpec qs, int mp, int nq, int n_seq,
+                   int H, int c, int64_t Nmax, float scale, const float* sink, void* out, float* lse, void* ws,
+                   int nsplit, int* status, cudaStream_t st);
+
 // mqa.cu: sparse (idx != nullptr) or dense (entries s < pos/mp) shared-KV MQA
 size_t mqa_workspace_bytes(int nq, int H, int c, int64_t max_entries, ElemType t);
 cudaError_t mqa(const void* q, const void* KV, const int32_t* idx, int k, QuerySpec qs, int mp,

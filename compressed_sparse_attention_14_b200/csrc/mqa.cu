@@ -190,8 +190,24 @@ static int mqa_nsplit(int nq, int H, int64_t max_entries) {
     return (int)want;
 }
 
-size_t mqa_workspace_bytes(int nq, int H, int c, int64_t max_entries, ElemType) {
-    int ns = mqa_nsplit(nq, H, max_entries);
+static int num_sms_cached() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    }
+    return n;
+}
+
+static int plan_nsplit(int nq, int H, int64_t max_entries, ElemType t) {
+    return t == ElemType::BF16 ? mqa_tc_nsplit(nq, H, max_entries, num_sms_cached())
+                               : mqa_nsplit(nq, H, max_entries);
+}
+
+size_t mqa_workspace_bytes(int nq, int H, int c, int64_t max_entries, ElemType t) {
+    int ns = plan_nsplit(nq, H, max_entries, t);
+    if (t == ElemType::BF16 && ns == 1) return 0;   // a single split writes the output directly
     return align256((size_t)nq * ns * H * c * sizeof(float)) +
            align256((size_t)nq * ns * H * 2 * sizeof(float));
 }
@@ -201,6 +217,17 @@ cudaError_t mqa(const void* q, const void* KV, const int32_t* idx, int k, QueryS
                 float* lse, void* ws, ElemType t, cudaStream_t st) {
     if (nq == 0) return cudaSuccess;
     const int64_t max_entries = idx ? k : Nmax;
+    if (t == ElemType::BF16) {
+        const int ns = plan_nsplit(nq, H, max_entries, t);
+        cudaError_t e = mqa_tc(q, KV, idx, k, qs, mp, nq, n_seq, H, c, Nmax, scale, sink, out, lse, ws, ns,
+                               device_status(), st);
+        if (e != cudaSuccess || ns == 1) return e;
+        float* part_o = (float*)ws;
+        float* part_ml = (float*)((char*)ws + align256((size_t)nq * ns * H * c * sizeof(float)));
+        CSA_LAUNCH(st, "mqa_combine", mqa_combine_kernel<bf16><<<dim3(H, nq), 128, 0, st>>>(
+                                          part_o, part_ml, ns, H, c, sink, (bf16*)out, lse));
+        return cudaGetLastError();
+    }
     const int ns = mqa_nsplit(nq, H, max_entries);
     MqaPartialArgs a{};
     a.q = q; a.KV = KV; a.idx = idx; a.k = k;

@@ -1,0 +1,502 @@
+// Shared-KV multi-query attention on the 5th-generation tensor cores
+// [Notes §1.1 last paragraph: each compressed entry is both key and value,
+// shared by all query heads; Walk §2.3.2; sink from Notes §1.3, equation
+// s_{h,i,j}] ([Notes] = "DeepSeek-V4: 迈向高效百万级上下文智能" study notes;
+// [Walk] = the mlpod.com walk-through of the DeepSeek-V4 report).
+//
+// One CTA serves (query t, a group of up to 64 heads, one split of t's entry
+// list) and walks the split in tiles of 128 entries. Because key and value
+// are the same row, ONE shared-memory copy of a tile (128 entries x c dims,
+// 128-byte swizzle, 64-dim blocks) feeds both products:
+//   S^T  = KV_tile . q^T       M = 128 entries, N = heads, K = c  (KV K-major)
+//   O^T += KV_tile^T . P^T     M = 128 dims,    N = heads, K = 128 (KV MN-major)
+// with S^T (double-buffered) and O^T in tensor memory. A TMEM lane of S^T
+// holds one entry's logits for every head, so the softmax threads work per
+// entry; the per-head running max is a reference value that only moves (and
+// then O^T and the partial sums are rescaled in place) when a logit exceeds
+// it by more than 2^8 — exact, since the final normalisation uses the same
+// reference, and cheap, since it rarely moves after the first tile.
+//
+// Entry sources: CSA (sparse) gathers the selected rows with TMA
+// tile::gather4 (four rows per copy); HCA (dense) loads 128 consecutive rows
+// per 64-dim block with one TMA box. The tile's 64-dim blocks are released
+// one by one as the second product finishes with them, so the next tile's
+// gather overlaps it.
+//
+// Warp roles: warp 0 loads (all lanes issue gathers), warp 1 allocates TMEM
+// and one lane issues the MMAs, warps 2-5 run the softmax and the epilogue.
+// Split-KV partials (O, max, sum) go to the workspace and are merged by
+// mqa_combine (fixed split boundaries: deterministic); a single split writes
+// the normalised output directly. Waits are bounded (CSA_ERR_TIMEOUT).
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+#include "tmap.h"
+
+namespace csa {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kE = 128;                 // entries per tile
+constexpr int kMaxDBlocks = 8;          // c <= 512
+constexpr uint32_t kWaitLimit = 1u << 24;
+constexpr float kRescaleLog2 = 8.0f;    // move the reference max past 2^8
+
+struct MqaArgs {
+    QueryMap qm;
+    int n_seq, mp;
+    const int32_t* idx;       // sparse entry lists, or nullptr (dense)
+    int k;
+    int nq, H, c;
+    int hg;                   // heads per CTA (MMA N) = 64
+    int64_t Nmax;
+    float scale_log2;
+    const float* sink;
+    int nsplit;
+    int64_t split_len;
+    bf16* out;
+    float* lse;
+    float* part_o;
+    float* part_ml;
+    int* status;
+    int dblocks, mtiles;
+    uint32_t tmem_cols, q_bytes;
+};
+
+__device__ __forceinline__ void gather4(void* dst, const void* tmap, uint64_t* bar, int x, int y0, int y1, int y2,
+                                        int y3) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(tc::smem_u32(dst)),
+        "l"(tmap), "r"(tc::smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
+        : "memory");
+}
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                              int* status) {
+    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+        if (tc::mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 255u && *abort_flag) return false;
+    }
+    report_device_error(status, CSA_ERR_TIMEOUT);
+    *abort_flag = 1;
+    return false;
+}
+
+__device__ __forceinline__ bool bar_or_128(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.or.pred p, 1, 128, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ void bar_sync_128() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+}  // namespace
+
+__global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_constant__ MqaArgs a,
+                                                             const __grid_constant__ CUtensorMap tmQ,
+                                                             const __grid_constant__ CUtensorMap tmRow,
+                                                             const __grid_constant__ CUtensorMap tmTile) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t* kv_s = base;                                        // dblocks x 16 KB
+    uint8_t* q_s = kv_s + (size_t)a.dblocks * kE * 128;          // dblocks x hg*128
+    uint8_t* p_s = q_s + a.q_bytes;                              // 128 x 128 B
+    float* mref_s = (float*)(p_s + kE * 128);                    // [64]
+    float* alpha_s = mref_s + 64;                                // [64]
+    float* red_s = alpha_s + 64;                                 // [4][64]
+    float* lsum_s = red_s + 256;                                 // [64]
+    uint64_t* bars = (uint64_t*)(lsum_s + 64);
+    uint64_t* kv_full = bars;                                    // [8]
+    uint64_t* kv_empty = bars + kMaxDBlocks;                     // [8]
+    uint64_t* s_full = bars + 2 * kMaxDBlocks;                   // [2]
+    uint64_t* s_empty = s_full + 2;                              // [2]
+    uint64_t* q_full = s_empty + 2;
+    uint64_t* p_full = q_full + 1;
+    uint64_t* o_done = p_full + 1;
+    uint64_t* fin = o_done + 1;
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.z;
+    const int h0 = blockIdx.y * a.hg;
+    const int split = blockIdx.x;
+    const int seq = a.qm.seq_of(t);
+    const bool seq_ok = seq >= 0 && seq < a.n_seq;
+    int64_t n_ent = 0;
+    if (seq_ok) n_ent = a.idx ? (int64_t)a.k : visible_entries(a.qm.pos_of(t), a.mp, a.Nmax);
+    const int64_t e_beg = (int64_t)split * a.split_len;
+    int64_t e_end = e_beg + a.split_len;
+    if (e_end > n_ent) e_end = n_ent;
+    const int ntiles = e_end > e_beg ? (int)((e_end - e_beg + kE - 1) / kE) : 0;
+    const int64_t row0 = (int64_t)(seq_ok ? seq : 0) * a.Nmax;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kMaxDBlocks; ++i) { tc::mbar_init(&kv_full[i], 1); tc::mbar_init(&kv_empty[i], 1); }
+        for (int i = 0; i < 2; ++i) { tc::mbar_init(&s_full[i], 1); tc::mbar_init(&s_empty[i], 4); }
+        tc::mbar_init(q_full, 1);
+        tc::mbar_init(p_full, 4);
+        tc::mbar_init(o_done, 1);
+        tc::mbar_init(fin, 1);
+        tc::fence_mbar_init();
+        s_abort = 0;
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(&s_tmem, a.tmem_cols);
+        tc::tmem_relinquish();
+        tc::tc_fence_before();
+    }
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    const uint32_t tmem_S = tmem;                              // 2 x hg columns
+    const uint32_t tmem_O = tmem + 2 * (uint32_t)a.hg;         // mtiles x hg columns
+    volatile int* abort_flag = &s_abort;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- loads
+        if (ntiles > 0) {
+            if (lane == 0) {
+                tc::mbar_expect_tx(q_full, a.q_bytes);
+                for (int b = 0; b < a.dblocks; ++b)
+                    tc::tma_load_2d(q_s + (size_t)b * a.hg * 128, &tmQ, q_full, b * 64, t * a.H + h0);
+            }
+            int j = 0;
+            for (; j < ntiles; ++j) {
+                bool ok = true;
+                if (lane == 0) {
+                    for (int b = 0; b < a.dblocks && ok; ++b) {
+                        if (j > 0) ok = wait_or_abort(&kv_empty[b], (j - 1) & 1, abort_flag, a.status);
+                        if (ok) tc::mbar_expect_tx(&kv_full[b], kE * 128);
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                const int64_t e0 = e_beg + (int64_t)j * kE;
+                if (a.idx) {
+                    int rows[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int64_t e = e0 + lane * 4 + u;
+                        int s = -1;
+                        if (e < e_end) s = a.idx[(int64_t)t * a.k + e];
+                        if (s < 0 || s >= a.Nmax) s = 0;   // masked in the softmax
+                        rows[u] = (int)(row0 + s);
+                    }
+                    for (int b = 0; b < a.dblocks; ++b)
+                        gather4(kv_s + (size_t)b * kE * 128 + lane * 4 * 128, &tmRow, &kv_full[b], b * 64, rows[0],
+                                rows[1], rows[2], rows[3]);
+                } else if (lane == 0) {
+                    for (int b = 0; b < a.dblocks; ++b)
+                        tc::tma_load_2d(kv_s + (size_t)b * kE * 128, &tmTile, &kv_full[b], b * 64, (int)(row0 + e0));
+                }
+            }
+            // drain: the last issued tile and q must have landed
+            if (lane == 0 && j > 0)
+                for (int b = 0; b < a.dblocks; ++b) tc::mbar_wait(&kv_full[b], (j - 1) & 1, kWaitLimit);
+            if (lane == 0) tc::mbar_wait(q_full, 0, kWaitLimit);
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA
+        if (lane == 0 && ntiles > 0) {
+            const uint32_t idesc1 = tc::idesc_bf16_f32(128, a.hg, 0, 0);
+            const uint32_t idesc2 = tc::idesc_bf16_f32(128, a.hg, 1, 1);
+            const uint32_t kv_addr = tc::smem_u32(kv_s);
+            const uint32_t q_addr = tc::smem_u32(q_s);
+            const uint32_t p_addr = tc::smem_u32(p_s);
+            bool ok = wait_or_abort(q_full, 0, abort_flag, a.status);
+            int j = 0;
+            for (; ok && j < ntiles; ++j) {
+                const int sb = j & 1;
+                if (j >= 2 && !(ok = wait_or_abort(&s_empty[sb], ((j >> 1) - 1) & 1, abort_flag, a.status))) break;
+                // S^T = KV . q^T
+                for (int b = 0; b < a.dblocks && ok; ++b) {
+                    if (!(ok = wait_or_abort(&kv_full[b], j & 1, abort_flag, a.status))) break;
+                    tc::tc_fence_after();
+                    for (int kk = 0; kk < 4; ++kk) {
+                        uint64_t ad = tc::sdesc_sw128(kv_addr + b * (kE * 128) + kk * 32, 16, 1024);
+                        uint64_t bd = tc::sdesc_sw128(q_addr + b * (a.hg * 128) + kk * 32, 16, 1024);
+                        tc::umma_bf16(tmem_S + sb * a.hg, ad, bd, idesc1, (b | kk) ? 1u : 0u);
+                    }
+                }
+                if (!ok) break;
+                tc::umma_commit(&s_full[sb]);
+                // O^T += KV^T . P^T once the softmax has written P
+                if (!(ok = wait_or_abort(p_full, j & 1, abort_flag, a.status))) break;
+                tc::tc_fence_after();
+                for (int mt = 0; mt < a.mtiles; ++mt) {
+                    for (int ke = 0; ke < kE / 16; ++ke) {
+                        uint64_t ad = tc::sdesc_sw128(kv_addr + (2 * mt) * (kE * 128) + ke * 2048, kE * 128, 1024);
+                        uint64_t bd = tc::sdesc_sw128(p_addr + ke * 2048, kE * 128, 1024);
+                        tc::umma_bf16(tmem_O + mt * a.hg, ad, bd, idesc2, (j > 0 || ke > 0) ? 1u : 0u);
+                    }
+                    tc::umma_commit(&kv_empty[2 * mt]);
+                    tc::umma_commit(&kv_empty[2 * mt + 1]);
+                }
+                tc::umma_commit(o_done);
+            }
+            // a last commit covers every MMA this thread issued (also on abort)
+            tc::umma_commit(fin);
+            tc::mbar_wait(fin, 0, kWaitLimit);
+        }
+    } else {
+        // ---------------------------------------------------------------- softmax + epilogue
+        const int quad = warp & 3;
+        const int row = quad * 32 + lane;            // entry within the tile / dim within an M tile
+        const int eth = threadIdx.x - 64;            // 0..127
+        const int hg = a.hg;
+        if (eth < 64) { mref_s[eth] = -INFINITY; lsum_s[eth] = 0.f; }
+        float lpart[64];
+#pragma unroll
+        for (int h = 0; h < 64; ++h) lpart[h] = 0.f;
+        bar_sync_128();
+        bool ok = true;
+        int j = 0;
+        for (; j < ntiles; ++j) {
+            const int sb = j & 1;
+            if (!(ok = wait_or_abort(&s_full[sb], (j >> 1) & 1, abort_flag, a.status))) break;
+            tc::tc_fence_after();
+            const int64_t e = e_beg + (int64_t)j * kE + row;
+            bool valid = e < e_end;
+            if (valid && a.idx) {
+                int s = a.idx[(int64_t)t * a.k + e];
+                valid = s >= 0 && s < a.Nmax;
+            }
+            float z[64];
+            const uint32_t taddr = tmem_S + ((uint32_t)(quad * 32) << 16) + sb * hg;
+#pragma unroll
+            for (int cc = 0; cc < 64; cc += 16) {
+                if (cc < hg) {
+                    float v[16];
+                    tc::tmem_ld16(taddr + cc, v);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) z[cc + i] = v[i];
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) z[cc + i] = -INFINITY;
+                }
+            }
+            tc::tmem_ld_wait();
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&s_empty[sb]);
+            bool need = false;
+#pragma unroll
+            for (int h = 0; h < 64; ++h) {
+                z[h] = valid ? z[h] * a.scale_log2 : -INFINITY;
+                need |= z[h] > mref_s[h] + kRescaleLog2;
+            }
+            if (bar_or_128(need)) {
+                // new reference: per-head max over the tile's 128 entries
+#pragma unroll
+                for (int h = 0; h < 64; ++h) {
+                    float mx = warp_max(z[h]);
+                    if (lane == (h & 31)) red_s[quad * 64 + h] = mx;
+                }
+                bar_sync_128();
+                if (eth < 64) {
+                    float old = mref_s[eth];
+                    float nm = fmaxf(fmaxf(fmaxf(red_s[eth], red_s[64 + eth]), fmaxf(red_s[128 + eth], red_s[192 + eth])),
+                                     old);
+                    alpha_s[eth] = (old == -INFINITY) ? 0.f : exp2f(old - nm);
+                    mref_s[eth] = nm;
+                }
+                bar_sync_128();
+#pragma unroll
+                for (int h = 0; h < 64; ++h) lpart[h] *= alpha_s[h];
+                if (j > 0) {
+                    // rescale O^T (all previous products must have landed)
+                    if (!(ok = wait_or_abort(o_done, (j - 1) & 1, abort_flag, a.status))) break;
+                    tc::tc_fence_after();
+                    for (int mt = 0; mt < a.mtiles; ++mt) {
+                        for (int cc = 0; cc < hg; cc += 16) {
+                            float v[16];
+                            const uint32_t oaddr = tmem_O + ((uint32_t)(quad * 32) << 16) + mt * hg + cc;
+                            tc::tmem_ld16(oaddr, v);
+                            tc::tmem_ld_wait();
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) v[i] *= alpha_s[cc + i];
+                            tc::tmem_st16(oaddr, v);
+                        }
+                    }
+                    tc::tmem_st_wait();
+                    tc::tc_fence_before();
+                }
+            }
+            // P = 2^(z - m), rows of 64 bf16 (128 bytes), 128-byte swizzle
+            uint32_t pk[32];
+#pragma unroll
+            for (int h = 0; h < 64; h += 2) {
+                float p0 = (z[h] == -INFINITY) ? 0.f : exp2f(z[h] - mref_s[h]);
+                float p1 = (z[h + 1] == -INFINITY) ? 0.f : exp2f(z[h + 1] - mref_s[h + 1]);
+                lpart[h] += p0;
+                lpart[h + 1] += p1;
+                __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+                pk[h >> 1] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+            // the previous tile's second product must be done reading P
+            if (j > 0 && !(ok = wait_or_abort(o_done, (j - 1) & 1, abort_flag, a.status))) break;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                uint4 v = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+                *reinterpret_cast<uint4*>(p_s + row * 128 + ((ch ^ (row & 7)) * 16)) = v;
+            }
+            tc::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(p_full);
+        }
+        // ------------------------------------------------------------ epilogue
+        if (ok && ntiles > 0) ok = wait_or_abort(o_done, (ntiles - 1) & 1, abort_flag, a.status);
+        tc::tc_fence_after();
+        // per-head sums: fixed-order reduction of the 128 per-entry partials
+        float* lred = (float*)kv_s;   // the KV tile is no longer read
+        bar_sync_128();
+#pragma unroll
+        for (int h = 0; h < 64; ++h) lred[h * 128 + eth] = lpart[h];
+        bar_sync_128();
+        if (eth < 64) {
+            float sum = 0.f;
+            for (int i = 0; i < 128; ++i) sum += lred[eth * 128 + i];
+            lsum_s[eth] = sum;
+        }
+        bar_sync_128();
+        const bool have_o = ok && ntiles > 0;
+        if (a.nsplit == 1) {
+            // normalise: denominator = sum + sink term (same reference max)
+            if (eth < 64) {
+                const int h = h0 + eth;
+                float m = mref_s[eth];
+                float L = lsum_s[eth];
+                float sk = (a.sink && h < a.H) ? a.sink[h] * 1.4426950408889634f : -INFINITY;
+                float lse;
+                if (m == -INFINITY) {              // no visible entry
+                    alpha_s[eth] = 0.f;
+                    lse = (sk == -INFINITY) ? -INFINITY : sk * 0.6931471805599453f;
+                } else {
+                    float Lt = L + ((sk == -INFINITY) ? 0.f : exp2f(sk - m));
+                    alpha_s[eth] = 1.f / Lt;
+                    lse = (m + log2f(Lt)) * 0.6931471805599453f;
+                }
+                if (a.lse && h < a.H) a.lse[(int64_t)t * a.H + h] = lse;
+            }
+            bar_sync_128();
+            for (int mt = 0; mt < a.mtiles; ++mt) {
+                const int dim = mt * 128 + row;
+                for (int cc = 0; cc < hg; cc += 16) {
+                    float v[16];
+                    if (have_o) {
+                        tc::tmem_ld16(tmem_O + ((uint32_t)(quad * 32) << 16) + mt * hg + cc, v);
+                        tc::tmem_ld_wait();
+                    }
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int h = h0 + cc + i;
+                        if (h < a.H) {
+                            float o = (have_o && mref_s[cc + i] != -INFINITY) ? v[i] * alpha_s[cc + i] : 0.f;
+                            a.out[((int64_t)t * a.H + h) * a.c + dim] = __float2bfloat16_rn(o);
+                        }
+                    }
+                }
+            }
+        } else {
+            if (eth < 64 && h0 + eth < a.H) {
+                float* pm = a.part_ml + (((int64_t)t * a.nsplit + split) * a.H + h0 + eth) * 2;
+                pm[0] = (have_o && mref_s[eth] != -INFINITY) ? mref_s[eth] * 0.6931471805599453f : -INFINITY;
+                pm[1] = have_o ? lsum_s[eth] : 0.f;
+            }
+            if (have_o) {
+                for (int mt = 0; mt < a.mtiles; ++mt) {
+                    const int dim = mt * 128 + row;
+                    for (int cc = 0; cc < hg; cc += 16) {
+                        float v[16];
+                        tc::tmem_ld16(tmem_O + ((uint32_t)(quad * 32) << 16) + mt * hg + cc, v);
+                        tc::tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int h = h0 + cc + i;
+                            if (h < a.H) a.part_o[(((int64_t)t * a.nsplit + split) * a.H + h) * a.c + dim] = v[i];
+                        }
+                    }
+                }
+            }
+        }
+        tc::tc_fence_before();
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, a.tmem_cols);
+    }
+}
+
+bool mqa_tc_supported(int H, int c) { return c % 128 == 0 && c <= 512 && H >= 1; }
+
+int mqa_tc_nsplit(int nq, int H, int64_t max_entries, int num_sms) {
+    const int hgroups = (H + 63) / 64;
+    const int64_t ctas = (int64_t)nq * hgroups;
+    int64_t ns = ctas > 0 ? num_sms / ctas : 1;
+    const int64_t tiles = (max_entries + kE - 1) / kE;
+    if (ns > tiles) ns = tiles;
+    if (ns < 1) ns = 1;
+    if (ns > 64) ns = 64;
+    return (int)ns;
+}
+
+cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, QuerySpec qs, int mp, int nq, int n_seq,
+                   int H, int c, int64_t Nmax, float scale, const float* sink, void* out, float* lse, void* ws,
+                   int nsplit, int* status, cudaStream_t st) {
+    if (nq == 0) return cudaSuccess;
+    MqaArgs a{};
+    a.qm = QueryMap{qs.seq, qs.pos, qs.pos_base, qs.single_seq};
+    a.n_seq = n_seq;
+    a.mp = mp;
+    a.idx = idx;
+    a.k = k;
+    a.nq = nq;
+    a.H = H;
+    a.c = c;
+    a.hg = 64;   // heads per CTA; smaller H pads with rows that are never written out
+    a.Nmax = Nmax;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.sink = sink;
+    a.nsplit = nsplit;
+    const int64_t max_entries = idx ? k : Nmax;
+    int64_t per = (max_entries + nsplit - 1) / nsplit;
+    a.split_len = ((per + kE - 1) / kE) * kE;
+    if (a.split_len == 0) a.split_len = kE;
+    a.out = (bf16*)out;
+    a.lse = lse;
+    a.part_o = (float*)ws;
+    a.part_ml = (float*)((char*)ws + align256((size_t)nq * nsplit * H * c * sizeof(float)));
+    a.status = status;
+    a.dblocks = c / 64;
+    a.mtiles = c / 128;
+    a.q_bytes = (uint32_t)(a.hg * c * 2);
+    uint32_t need = 2 * a.hg + a.mtiles * a.hg, cols = 32;
+    while (cols < need) cols <<= 1;
+    a.tmem_cols = cols;
+
+    CUtensorMap tmQ, tmRow, tmTile;
+    if (!make_tmap_bf16_2d(&tmQ, q, (uint64_t)nq * H, c, c, a.hg, 64)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_2d(&tmRow, KV, (uint64_t)n_seq * Nmax, c, c, 1, 64)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_2d(&tmTile, KV, (uint64_t)n_seq * Nmax, c, c, kE, 64)) return cudaErrorInvalidValue;
+
+    const size_t smem = 1024 + (size_t)a.dblocks * kE * 128 + a.q_bytes + kE * 128 + (64 * 4 + 256) * sizeof(float) +
+                        32 * sizeof(uint64_t);
+    cudaError_t e = cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(nsplit, (H + a.hg - 1) / a.hg, nq);
+    CSA_LAUNCH(st, "mqa_tc", mqa_tc_kernel<<<grid, kThreads, smem, st>>>(a, tmQ, tmRow, tmTile));
+    return cudaGetLastError();
+}
+
+}  // namespace csa

@@ -79,13 +79,13 @@ def test_invalid_arguments_are_rejected_on_the_host():
     assert rc == csa.CSA_ERR_WORKSPACE
     # prefill: start not a multiple of m, cache too small, missing left rows
     args = dict(n=8, Nmax=4, start=4)
-    rc = L.csa_prefill(fake, fake, fake, fake, fake, fake, 2, 8, 64, 4, 32, 64, fake, fake, 16, fake, fake, fake,
+    rc = L.csa_prefill(fake, fake, fake, fake, fake, fake, 2, 8, 64, 4, 128, 64, fake, fake, 16, fake, fake, fake,
                        8, 4, 4, 0.0, None, fake, None, None, None, 0, csa.CSA_BF16, None)
     assert rc == csa.CSA_ERR_INVALID_ARG
-    rc = L.csa_prefill(fake, fake, fake, fake, fake, fake, 4, 8, 64, 4, 32, 64, fake, fake, 2, fake, fake, fake,
+    rc = L.csa_prefill(fake, fake, fake, fake, fake, fake, 4, 8, 64, 4, 128, 64, fake, fake, 2, fake, fake, fake,
                        8, 4, 4, 0.0, None, fake, None, None, None, 0, csa.CSA_BF16, None)
     assert rc == csa.CSA_ERR_INVALID_ARG
-    rc = L.csa_prefill(fake, None, fake, fake, fake, fake, 4, 8, 64, 4, 32, 64, fake, fake, 16, fake, fake, fake,
+    rc = L.csa_prefill(fake, None, fake, fake, fake, fake, 4, 8, 64, 4, 128, 64, fake, fake, 16, fake, fake, fake,
                        8, 4, 4, 0.0, None, fake, None, None, None, 0, csa.CSA_BF16, None)
     assert rc == csa.CSA_ERR_INVALID_ARG
     del args
