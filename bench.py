@@ -211,9 +211,10 @@ class Timer:
 # workloads (ours)
 # ----------------------------------------------------------------------------
 
-def decode_workload(shape, rank):
+def decode_workload(shape, rank, batch=None):
+    import dataclasses
     import compressed_sparse_attention_14_b200 as csa
-    s = shape
+    s = shape if batch is None else dataclasses.replace(shape, batch=batch)
     inp = synth.decode_inputs(dataclass_seed(s, rank), device="cuda")
     B = s.batch
     mode = csa.CSA_BF16
@@ -379,11 +380,11 @@ def prefill_workload(rank):
 
 
 WORKLOADS = {
-    "flash_decode": lambda r: decode_workload(synth.FLASH_DECODE, r),
-    "pro_decode": lambda r: decode_workload(synth.PRO_DECODE, r),
-    "hca_decode": hca_decode_workload,
-    "hca_compress": hca_compress_workload,
-    "prefill": prefill_workload,
+    "flash_decode": lambda r, b=None: decode_workload(synth.FLASH_DECODE, r, b),
+    "pro_decode": lambda r, b=None: decode_workload(synth.PRO_DECODE, r, b),
+    "hca_decode": lambda r, b=None: hca_decode_workload(r),
+    "hca_compress": lambda r, b=None: hca_compress_workload(r),
+    "prefill": lambda r, b=None: prefill_workload(r),
 }
 
 
@@ -536,7 +537,7 @@ WORKLOADS_CONFIG_NAME = {
 
 def run_ours(args, rank, world, local):
     import compressed_sparse_attention_14_b200 as csa
-    wl = WORKLOADS[args.workload](rank)
+    wl = WORKLOADS[args.workload](rank, args.batch)
     step, e2e_step = wl["step"], wl["e2e_step"]
 
     # warm-up
@@ -646,6 +647,8 @@ def main():
     ap.add_argument("--workload", default="flash_decode", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="decode workloads: use only the first N queries (small profiling cases)")
     args = ap.parse_args()
     rank, world, local = dist_init()
     if world != args.gpus and rank == 0:
