@@ -19,7 +19,7 @@
 //   warp 0     TMA producer: the group's Q rows once per group, then the key
 //              tiles through a ring of `stages` shared-memory buffers;
 //   warp 1     allocates TMEM; one lane issues the MMAs of each tile into one
-//              of two accumulator buffers and commits their completion;
+//              of 2-4 accumulator buffers and commits their completion;
 //   warps 2-5  epilogue: tcgen05.ld of the accumulator, ReLU/weight/head
 //              reduction, coalesced fp32 score stores.
 // Every wait is bounded; a timeout records CSA_ERR_TIMEOUT in the status
@@ -52,6 +52,7 @@ struct IdxArgs {
     int64_t ld;
     int* status;
     uint32_t stage_bytes, q_bytes, tmem_cols;
+    int nbuf;           // TMEM accumulator buffers (2..4)
 };
 
 struct Smem {
@@ -60,8 +61,8 @@ struct Smem {
     float* w;           // 256
     uint64_t* full;     // [stages]
     uint64_t* empty;    // [stages]
-    uint64_t* tfull;    // [2]
-    uint64_t* tempty;   // [2]
+    uint64_t* tfull;    // [4]
+    uint64_t* tempty;   // [4]
     uint64_t* qfull;
     uint64_t* qempty;
     uint64_t* fin;
@@ -76,8 +77,8 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const IdxArgs& a) {
     s.full = bars;
     s.empty = bars + a.stages;
     s.tfull = bars + 2 * a.stages;
-    s.tempty = s.tfull + 2;
-    s.qfull = s.tempty + 2;
+    s.tempty = s.tfull + 4;
+    s.qfull = s.tempty + 4;
     s.qempty = s.qfull + 1;
     s.fin = s.qempty + 1;
     return s;
@@ -179,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < a.stages; ++i) { tc::mbar_init(&sm.full[i], 1); tc::mbar_init(&sm.empty[i], 1); }
-        for (int i = 0; i < 2; ++i) { tc::mbar_init(&sm.tfull[i], 1); tc::mbar_init(&sm.tempty[i], 4); }
+        for (int i = 0; i < 4; ++i) { tc::mbar_init(&sm.tfull[i], 1); tc::mbar_init(&sm.tempty[i], 4); }
         tc::mbar_init(sm.qfull, 1);
         tc::mbar_init(sm.qempty, 1);
         tc::mbar_init(sm.fin, 1);
@@ -250,8 +251,13 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
             int cur = -1;
             uint32_t switches = 0;
             const uint32_t idesc = tc::idesc_bf16_f32(128, a.npad, 0, 0);
-            const uint32_t q_addr = tc::smem_u32(sm.q);
-            const uint32_t st_addr = tc::smem_u32(sm.stage0);
+            // descriptors built once; a K step or a stage only moves the start
+            // address field (bits 0-13, in 16-byte units), so it is added in place
+            const uint64_t a_desc0 = tc::sdesc_sw128(tc::smem_u32(sm.stage0), 16, 1024);
+            const uint64_t b_desc0 = tc::sdesc_sw128(tc::smem_u32(sm.q), 16, 1024);
+            const uint32_t stage_step = a.stage_bytes >> 4;
+            const uint32_t a_kb_step = (kKeys * 128) >> 4;
+            const uint32_t b_kb_step = (uint32_t)(a.npad * 128) >> 4;
             int64_t it = 0;
             for (; it < my; ++it) {
                 if (wk.g != cur) {
@@ -260,16 +266,19 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
                     ++switches;
                 }
                 const int s = (int)(it % a.stages);
-                const int buf = (int)(it & 1);
+                const int buf = (int)(it % a.nbuf);
+                const int64_t use = it / a.nbuf;
                 if (!wait_or_abort(&sm.full[s], (it / a.stages) & 1, abort_flag, a.status)) break;
-                if (it >= 2 && !wait_or_abort(&sm.tempty[buf], ((it >> 1) - 1) & 1, abort_flag, a.status)) break;
+                if (use >= 1 && !wait_or_abort(&sm.tempty[buf], (use - 1) & 1, abort_flag, a.status)) break;
                 tc::tc_fence_after();
-                const uint32_t a_base = st_addr + (uint32_t)s * a.stage_bytes;
+                const uint64_t a_s = a_desc0 + (uint64_t)(s * stage_step);
                 const uint32_t d = tmem + (uint32_t)(buf * a.npad);
-                for (int ks = 0; ks < a.kblocks * 4; ++ks) {
-                    uint64_t ad = tc::sdesc_sw128(a_base + (ks >> 2) * (kKeys * 128) + (ks & 3) * 32, 16, 1024);
-                    uint64_t bd = tc::sdesc_sw128(q_addr + (ks >> 2) * (a.npad * 128) + (ks & 3) * 32, 16, 1024);
-                    tc::umma_bf16(d, ad, bd, idesc, ks > 0 ? 1u : 0u);
+                for (int kb = 0; kb < a.kblocks; ++kb) {
+                    const uint64_t ad = a_s + (uint64_t)(kb * a_kb_step);
+                    const uint64_t bd = b_desc0 + (uint64_t)(kb * b_kb_step);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)   // 16 bf16 = 32 bytes = 2 units per K step
+                        tc::umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) ? 1u : 0u);
                 }
                 tc::umma_commit(&sm.empty[s]);
                 tc::umma_commit(&sm.tfull[buf]);
@@ -301,23 +310,36 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
                 cur = wk.g;
                 vis = group_visible(a, wk.g);
             }
-            const int buf = (int)(it & 1);
-            if (!wait_or_abort(&sm.tfull[buf], (it >> 1) & 1, abort_flag, a.status)) break;
+            const int buf = (int)(it % a.nbuf);
+            if (!wait_or_abort(&sm.tfull[buf], (uint32_t)((it / a.nbuf) & 1), abort_flag, a.status)) break;
             tc::tc_fence_after();
             float sc[4] = {0.f, 0.f, 0.f, 0.f};
             const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * a.npad);
-            for (int cc = 0; cc < a.npad; cc += 16) {
-                float v[16];
-                tc::tmem_ld16(taddr + cc, v);
-                tc::tmem_ld_wait();
-                float part = 0.f;
+            // 64 columns per round: four loads in flight, one wait
+            for (int c0 = 0; c0 < a.npad; c0 += 64) {
+                float v[64];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) part = fmaf(sm.w[cc + i], fmaxf(v[i], 0.f), part);
-                const int gq = (a.group > 1) ? cc / a.HI : 0;
-                if (gq == 0) sc[0] += part;
-                else if (gq == 1) sc[1] += part;
-                else if (gq == 2) sc[2] += part;
-                else sc[3] += part;
+                for (int u = 0; u < 4; ++u) {
+                    if (c0 + 16 * u < a.npad) {
+                        float* vv = v + 16 * u;
+                        tc::tmem_ld16(taddr + c0 + 16 * u, *reinterpret_cast<float(*)[16]>(vv));
+                    }
+                }
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int cc = c0 + 16 * u;
+                    if (cc < a.npad) {
+                        float part = 0.f;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) part = fmaf(sm.w[cc + i], fmaxf(v[16 * u + i], 0.f), part);
+                        const int gq = (a.group > 1) ? cc / a.HI : 0;
+                        if (gq == 0) sc[0] += part;
+                        else if (gq == 1) sc[1] += part;
+                        else if (gq == 2) sc[2] += part;
+                        else sc[3] += part;
+                    }
+                }
             }
             tc::tc_fence_before();
             __syncwarp();
@@ -393,8 +415,12 @@ cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, Query
     a.status = status;
     a.stage_bytes = (uint32_t)(kKeys * cI * 2);
     a.q_bytes = (uint32_t)(a.npad * cI * 2);
+    // as many accumulator buffers (2..4) as fit 512 TMEM columns
+    a.nbuf = 512 / a.npad;
+    if (a.nbuf > 4) a.nbuf = 4;
+    if (a.nbuf < 2) a.nbuf = 2;
     uint32_t cols = 32;
-    while (cols < (uint32_t)(2 * a.npad)) cols <<= 1;
+    while (cols < (uint32_t)(a.nbuf * a.npad)) cols <<= 1;
     a.tmem_cols = cols;
     const size_t fixed = 1024 + a.q_bytes + 256 * sizeof(float) + 64 * sizeof(uint64_t);
     const size_t budget = 226 * 1024;

@@ -5,7 +5,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
-#include "../../include/csa.h"
+#include "csa.h"
 
 namespace csa {
 

@@ -147,36 +147,56 @@ __global__ void __launch_bounds__(256) mqa_partial_ffma_kernel(MqaPartialArgs a)
     }
 }
 
+// Merge of split-KV partials for one (query, head): split s holds O_s (fp32,
+// scaled by exp(-m_s)), m_s and l_s; the result is
+//   out = sum_s e^{m_s - M} O_s / (sum_s e^{m_s - M} l_s + [sink] e^{z' - M})
+// with M the largest of the m_s and the sink logit, and lse = M + log(...).
+// The split weights are computed once into shared memory; each thread then
+// combines 4 consecutive dims with 16-byte loads.
 template <typename T>
 __global__ void __launch_bounds__(128) mqa_combine_kernel(const float* __restrict__ part_o,
                                                           const float* __restrict__ part_ml,
                                                           int nsplit, int H, int c,
                                                           const float* __restrict__ sink,
                                                           T* __restrict__ out, float* __restrict__ lse) {
+    __shared__ float s_w[64];
+    __shared__ float s_inv;
     const int t = blockIdx.y, h = blockIdx.x;
     const float* ml = part_ml + ((int64_t)t * nsplit * H + h) * 2;
-    float M = sink ? sink[h] : -INFINITY;
-    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, ml[(int64_t)s * H * 2]);
-    float L = 0.f;
-    if (M != -INFINITY) {
-        for (int s = 0; s < nsplit; ++s) {
+    if (threadIdx.x < 32) {
+        float M = sink ? sink[h] : -INFINITY;
+        for (int s = threadIdx.x; s < nsplit; s += 32) M = fmaxf(M, ml[(int64_t)s * H * 2]);
+        M = warp_max(M);
+        float L = 0.f;
+        for (int s = threadIdx.x; s < nsplit; s += 32) {
             float ms = ml[(int64_t)s * H * 2];
-            if (ms != -INFINITY) L += ml[(int64_t)s * H * 2 + 1] * expf(ms - M);
+            float wgt = (ms == -INFINITY || M == -INFINITY) ? 0.f : expf(ms - M);
+            s_w[s] = wgt;
+            L += wgt * ml[(int64_t)s * H * 2 + 1];
         }
-        if (sink) L += expf(sink[h] - M);
+        L = warp_sum(L);
+        if (threadIdx.x == 0) {
+            if (sink && M != -INFINITY) L += expf(sink[h] - M);
+            s_inv = (L > 0.f) ? 1.f / L : 0.f;
+            if (lse) lse[(int64_t)t * H + h] = (L > 0.f) ? M + logf(L) : -INFINITY;
+        }
     }
-    const float inv = (L > 0.f) ? 1.f / L : 0.f;
+    __syncthreads();
+    const float inv = s_inv;
     T* o = out + ((int64_t)t * H + h) * c;
-    for (int d = threadIdx.x; d < c; d += blockDim.x) {
-        float acc = 0.f;
+    for (int d = threadIdx.x * 4; d < c; d += blockDim.x * 4) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int s = 0; s < nsplit; ++s) {
-            float ms = ml[(int64_t)s * H * 2];
-            if (ms == -INFINITY) continue;
-            acc += part_o[(((int64_t)t * nsplit + s) * H + h) * c + d] * expf(ms - M);
+            const float wgt = s_w[s];
+            if (wgt == 0.f) continue;
+            const float4 v = *reinterpret_cast<const float4*>(part_o + (((int64_t)t * nsplit + s) * H + h) * c + d);
+            acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
         }
-        o[d] = from_f32<T>(acc * inv);
+        o[d] = from_f32<T>(acc.x * inv);
+        o[d + 1] = from_f32<T>(acc.y * inv);
+        o[d + 2] = from_f32<T>(acc.z * inv);
+        o[d + 3] = from_f32<T>(acc.w * inv);
     }
-    if (lse && threadIdx.x == 0) lse[(int64_t)t * H + h] = (L > 0.f) ? M + logf(L) : -INFINITY;
 }
 
 static int mqa_nsplit(int nq, int H, int64_t max_entries) {

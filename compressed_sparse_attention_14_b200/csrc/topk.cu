@@ -108,9 +108,19 @@ __global__ void __launch_bounds__(kTopkThreads) topk_select_kernel(TopkLevel L) 
             __syncthreads();
             const uint64_t prefix = s_prefix;
             const uint64_t hi_mask = (shift == 56) ? 0ull : (~0ull << (shift + 8));
-            for (int i = tid; i < n; i += kTopkThreads) {
-                uint64_t x = s_elems[i];
-                if ((x & hi_mask) == prefix) atomicAdd(&s_hist[(x >> shift) & 255u], 1u);
+            // warp-aggregated histogram: one atomic per distinct digit per warp
+            // (the leading digits of similar scores coincide, so plain atomics
+            // would serialize on one or two bins)
+            const int lane = tid & 31;
+            for (int i0 = tid - lane; i0 < n; i0 += kTopkThreads) {
+                const int i = i0 + lane;
+                uint32_t d = 256u;
+                if (i < n) {
+                    uint64_t x = s_elems[i];
+                    if ((x & hi_mask) == prefix) d = (uint32_t)((x >> shift) & 255u);
+                }
+                const unsigned peers = __match_any_sync(0xffffffffu, d);
+                if (d < 256u && lane == __ffs(peers) - 1) atomicAdd(&s_hist[d], (uint32_t)__popc(peers));
             }
             __syncthreads();
             if (tid < 32) {
@@ -215,20 +225,29 @@ __global__ void __launch_bounds__(kTopkThreads) topk_select_kernel(TopkLevel L) 
 // Largest segment one CTA holds: 16384 composites = 128 KB of shared memory.
 constexpr int kTopkSegMax = 16384;
 
-static int topk_seg_len(int64_t n, int k) {
-    (void)k;
-    return n <= kTopkSegMax ? (int)(n > 0 ? n : 1) : kTopkSegMax;
+// Segment length of the first level: the whole row when it fits, else
+// shorter segments (down to 4k, at least 4096) while few rows would leave
+// SMs idle.
+static int topk_seg_len(int64_t n, int k, int nq) {
+    if (n <= kTopkSegMax) return (int)(n > 0 ? n : 1);
+    int seg = kTopkSegMax;
+    const int min_seg = 4 * k > 4096 ? 4 * k : 4096;
+    while (seg / 2 >= min_seg && (int64_t)nq * ((n + seg - 1) / seg) < 2 * 148) seg /= 2;
+    return seg;
 }
 
-// Number of candidate slots per row needed by level `lvl` outputs.
+// Candidate slots needed by the levels (the same plan topk_run follows).
 size_t topk_workspace_bytes(int nq, int64_t ncols, int k) {
     int64_t n = ncols;
     size_t best = 0;
+    bool first = true;
     while (n > kTopkSegMax) {
-        int64_t nseg = (n + kTopkSegMax - 1) / kTopkSegMax;
+        int64_t seg = first ? topk_seg_len(n, k, nq) : kTopkSegMax;
+        int64_t nseg = (n + seg - 1) / seg;
         n = nseg * k;
         size_t b = (size_t)nq * (size_t)n * sizeof(uint64_t);
         if (b > best) best = b;
+        first = false;
     }
     // two ping-pong buffers, 256-byte aligned
     return best ? 2 * ((best + 255) & ~(size_t)255) : 0;
@@ -248,7 +267,7 @@ static cudaError_t launch_level(const TopkLevel& L, int nq, int nseg, int seg_le
 static cudaError_t topk_run(TopkLevel L, int nq, int64_t ncols, int k, void* ws, cudaStream_t st) {
     if (nq == 0) return cudaSuccess;
     if (ncols <= kTopkSegMax) {
-        L.seg_len = topk_seg_len(ncols, k);
+        L.seg_len = topk_seg_len(ncols, k, nq);
         return launch_level<true, true>(L, nq, 1, L.seg_len, st);
     }
     size_t half = topk_workspace_bytes(nq, ncols, k) / 2;
@@ -259,18 +278,19 @@ static cudaError_t topk_run(TopkLevel L, int nq, int64_t ncols, int k, void* ws,
     cudaError_t e = cudaSuccess;
     while (true) {
         if (n <= kTopkSegMax) {
-            L.seg_len = topk_seg_len(n, k);
+            L.seg_len = (int)(n > 0 ? n : 1);
             L.cand_ld = n;
             return raw ? launch_level<true, true>(L, nq, 1, L.seg_len, st)
                        : launch_level<false, true>(L, nq, 1, L.seg_len, st);
         }
-        int nseg = (int)((n + kTopkSegMax - 1) / kTopkSegMax);
-        L.seg_len = kTopkSegMax;
+        const int seg = raw ? topk_seg_len(n, k, nq) : kTopkSegMax;
+        int nseg = (int)((n + seg - 1) / seg);
+        L.seg_len = seg;
         L.cand_ld = n;
         L.cand_out = buf[which];
         L.cand_out_ld = (int64_t)nseg * k;
-        e = raw ? launch_level<true, false>(L, nq, nseg, kTopkSegMax, st)
-                : launch_level<false, false>(L, nq, nseg, kTopkSegMax, st);
+        e = raw ? launch_level<true, false>(L, nq, nseg, seg, st)
+                : launch_level<false, false>(L, nq, nseg, seg, st);
         if (e != cudaSuccess) return e;
         L.cand = buf[which];
         n = (int64_t)nseg * k;
