@@ -331,7 +331,7 @@ def hca_compress_workload(rank):
         out_h.copy_(out, non_blocking=True)
 
     flops = 2.0 * n * d * 2 * s.c
-    kernels = {"project_ffma": dict(bound="tensor", work=flops, files=("gemm.cu", "common.cuh")),
+    kernels = {"project_tc": dict(bound="tensor", work=flops, files=("gemm_tc.cu", "tc.cuh", "common.cuh")),
                "hca_compress": dict(bound="hbm", work=n * 2 * s.c * 4 + (n // s.mp) * s.c * 2,
                                     files=("compress.cu", "common.cuh"))}
     return dict(step=step, e2e_step=e2e_step, units=n, unit="tokens/s", h2d=x_h.numel() * 2,
@@ -374,7 +374,7 @@ def prefill_workload(rank):
     proj_flops = 2.0 * (n + s.m) * s.d * 4 * (s.c + s.idx_dim)
     kernels = {"index_scores_tc": dict(bound="tensor", work=idx_flops, files=("indexer_tc.cu", "tc.cuh", "common.cuh")),
                "mqa_tc": dict(bound="tensor", work=mqa_flops, files=("mqa_tc.cu", "tc.cuh", "common.cuh")),
-               "project_ffma": dict(bound="tensor", work=proj_flops, files=("gemm.cu", "common.cuh"))}
+               "project_tc": dict(bound="tensor", work=proj_flops, files=("gemm_tc.cu", "tc.cuh", "common.cuh"))}
     return dict(step=step, e2e_step=e2e_step, units=n, unit="tokens/s",
                 h2d=sum(v.numel() * v.element_size() for v in pinned.values()), d2h=out_h.numel() * 2,
                 kernels=kernels, step_bytes=None,

@@ -3,7 +3,8 @@
 // maps of the hidden state] ([Walk] = mlpod.com walk-through of the
 // DeepSeek-V4 report):  out[t][o] = sum_k x[t][k] * W[o][k], fp32 result.
 //
-// FFMA tile kernel: 64x64 output tile per CTA, k-steps of 16 staged in
+// bf16 inputs run on the tensor cores (gemm_tc.cu); this FFMA kernel serves
+// the fp32 mode: 64x64 output tile per CTA, k-steps of 16 staged in
 // shared memory as fp32 (transposed so a warp reads consecutive rows), each
 // thread accumulates a 4x4 register block.
 #include "common.cuh"
@@ -63,6 +64,7 @@ __global__ void __launch_bounds__(256) project_ffma_kernel(const T* __restrict__
 cudaError_t project(const void* x, const void* W, int64_t n, int d, int M, float* out, ElemType t,
                     cudaStream_t st) {
     if (n == 0 || M == 0) return cudaSuccess;
+    if (t == ElemType::BF16) return project_tc(x, W, n, d, M, out, device_status(), st);
     dim3 grid((M + kBN - 1) / kBN, (unsigned)((n + kBM - 1) / kBM));
     if (t == ElemType::BF16)
         CSA_LAUNCH(st, "project_ffma", project_ffma_kernel<bf16><<<grid, 256, 0, st>>>((const bf16*)x, (const bf16*)W, n, d, M, out));

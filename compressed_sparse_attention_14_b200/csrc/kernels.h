@@ -47,9 +47,11 @@ cudaError_t compress_csa(const void* proj, const void* left, const float* bias, 
 cudaError_t compress_hca(const void* proj, const float* bias, int64_t n, int c, int mp, void* out,
                          ElemType in_t, ElemType out_t, cudaStream_t st);
 
-// gemm.cu: out[n, M] (fp32) = x[n, d] . W[M, d]^T
+// gemm.cu: out[n, M] (fp32) = x[n, d] . W[M, d]^T (bf16 -> gemm_tc.cu)
 cudaError_t project(const void* x, const void* W, int64_t n, int d, int M, float* out, ElemType t,
                     cudaStream_t st);
+cudaError_t project_tc(const void* x, const void* W, int64_t n, int d, int M, float* out, int* status,
+                       cudaStream_t st);
 
 // indexer.cu (FFMA, fp32 mode): scores[t, 0..Nmax) with ld = ld_scores;
 // -inf past the visible range
