@@ -20,8 +20,9 @@
 //              tiles through a ring of `stages` shared-memory buffers;
 //   warp 1     allocates TMEM; one lane issues the MMAs of each tile into one
 //              of 2-4 accumulator buffers and commits their completion;
-//   warps 2-5  epilogue: tcgen05.ld of the accumulator, ReLU/weight/head
-//              reduction, coalesced fp32 score stores.
+//   warps 2-9  epilogue, two sets of four warps taking alternate tiles:
+//              tcgen05.ld of the accumulator, ReLU/weight/head reduction,
+//              coalesced fp32 score stores.
 // Every wait is bounded; a timeout records CSA_ERR_TIMEOUT in the status
 // word, stops all roles, drains the copies in flight and frees TMEM.
 #include "common.cuh"
@@ -33,7 +34,7 @@ namespace csa {
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;   // producer, MMA, two epilogue sets of 4 warps
 constexpr int kKeys = 128;
 constexpr uint32_t kWaitLimit = 1u << 24;
 
@@ -58,7 +59,7 @@ struct IdxArgs {
 struct Smem {
     uint8_t* stage0;    // stages x stage_bytes
     uint8_t* q;         // q_bytes
-    float* w;           // 256
+    float* w;           // [2][256], one copy per epilogue set
     uint64_t* full;     // [stages]
     uint64_t* empty;    // [stages]
     uint64_t* tfull;    // [4]
@@ -73,7 +74,7 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const IdxArgs& a) {
     s.stage0 = base;
     s.q = base + (size_t)a.stages * a.stage_bytes;
     s.w = (float*)(s.q + a.q_bytes);
-    uint64_t* bars = (uint64_t*)(s.w + 256);
+    uint64_t* bars = (uint64_t*)(s.w + 512);
     s.full = bars;
     s.empty = bars + a.stages;
     s.tfull = bars + 2 * a.stages;
@@ -291,22 +292,29 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int quad = warp & 3;                 // TMEM lane quadrant of this warp
+        // two sets of four warps take alternate tiles; within a set, warp w
+        // reads TMEM lane quadrant w % 4
+        const int set = (warp - 2) >> 2;
+        const int quad = warp & 3;
         const int row = quad * 32 + lane;          // key within the tile
-        const int ethread = threadIdx.x - 64;      // 0..127
+        const int ethread = (warp - 2 - 4 * set) * 32 + lane;   // 0..127 within the set
+        float* wv = sm.w + set * 256;
         Walk wk;
         wk.start(a, g0, t0);
         int cur = -1;
         int64_t vis = 0;
-        for (int64_t it = 0; it < my; ++it) {
+        for (int64_t it = 0; it < my; ++it, wk.next(a, ngroups)) {
+            if ((int)(it & 1) != set) continue;
             if (wk.g != cur) {
-                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (set == 0) asm volatile("bar.sync 1, 128;" ::: "memory");
+                else asm volatile("bar.sync 2, 128;" ::: "memory");
                 for (int c = ethread; c < a.npad; c += 128) {
-                    int gq = c / a.HI, h = c % a.HI;
-                    int tq = wk.g * a.group + gq;
-                    sm.w[c] = (gq < a.group && tq < a.nq) ? a.w[(int64_t)tq * a.HI + h] : 0.f;
+                    const int gq = c / a.HI, h = c % a.HI;
+                    const int tq = wk.g * a.group + gq;
+                    wv[c] = (gq < a.group && tq < a.nq) ? a.w[(int64_t)tq * a.HI + h] : 0.f;
                 }
-                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (set == 0) asm volatile("bar.sync 1, 128;" ::: "memory");
+                else asm volatile("bar.sync 2, 128;" ::: "memory");
                 cur = wk.g;
                 vis = group_visible(a, wk.g);
             }
@@ -315,7 +323,8 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
             tc::tc_fence_after();
             float sc[4] = {0.f, 0.f, 0.f, 0.f};
             const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * a.npad);
-            // 64 columns per round: four loads in flight, one wait
+            // 64 columns per round: four loads in flight, one wait; four
+            // independent partial sums per 16 columns
             for (int c0 = 0; c0 < a.npad; c0 += 64) {
                 float v[64];
 #pragma unroll
@@ -330,9 +339,16 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
                 for (int u = 0; u < 4; ++u) {
                     const int cc = c0 + 16 * u;
                     if (cc < a.npad) {
-                        float part = 0.f;
+                        float p4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) part = fmaf(sm.w[cc + i], fmaxf(v[16 * u + i], 0.f), part);
+                        for (int i = 0; i < 16; i += 4) {
+                            const float4 w4 = *reinterpret_cast<const float4*>(wv + cc + i);
+                            p4[0] = fmaf(w4.x, fmaxf(v[16 * u + i], 0.f), p4[0]);
+                            p4[1] = fmaf(w4.y, fmaxf(v[16 * u + i + 1], 0.f), p4[1]);
+                            p4[2] = fmaf(w4.z, fmaxf(v[16 * u + i + 2], 0.f), p4[2]);
+                            p4[3] = fmaf(w4.w, fmaxf(v[16 * u + i + 3], 0.f), p4[3]);
+                        }
+                        const float part = (p4[0] + p4[1]) + (p4[2] + p4[3]);
                         const int gq = (a.group > 1) ? cc / a.HI : 0;
                         if (gq == 0) sc[0] += part;
                         else if (gq == 1) sc[1] += part;
@@ -352,7 +368,6 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
                     if (gq < a.group && tq < a.nq) a.scores[(int64_t)tq * a.ld + key] = sc[gq];
                 }
             }
-            wk.next(a, ngroups);
         }
     }
 
@@ -422,7 +437,7 @@ cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, Query
     uint32_t cols = 32;
     while (cols < (uint32_t)(a.nbuf * a.npad)) cols <<= 1;
     a.tmem_cols = cols;
-    const size_t fixed = 1024 + a.q_bytes + 256 * sizeof(float) + 64 * sizeof(uint64_t);
+    const size_t fixed = 1024 + a.q_bytes + 512 * sizeof(float) + 64 * sizeof(uint64_t);
     const size_t budget = 226 * 1024;
     int stages = (int)((budget - fixed) / a.stage_bytes);
     if (stages > 8) stages = 8;

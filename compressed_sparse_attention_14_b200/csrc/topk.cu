@@ -16,12 +16,11 @@
 // composites >= T; a bitonic network sorts them.
 //
 // Rows longer than one CTA's shared memory take two steps:
-//   1. filter (several CTAs per row): every CTA of the row sorts the same
-//      strided sample of 2048 scores and takes a threshold estimate low
-//      enough that, for any row that is not adversarial, well over k scores
-//      reach it (a rank ~1.25x the expected count plus 16); each CTA appends
-//      the composites of its slice that reach it to the row's candidate
-//      buffer;
+//   1. threshold (one CTA per row): sort a strided sample of 2048 scores and
+//      take an estimate low enough that, for any row that is not
+//      adversarial, well over k scores reach it (a rank ~1.25x the expected
+//      count plus 16); filter (several CTAs per row): each appends the
+//      composites of its slice that reach it to the row's candidate buffer;
 //   2. final (one CTA per row): when at least min(k, n) and at most the
 //      buffer's capacity of candidates arrived, the exact selection runs on
 //      them; otherwise it runs on the whole row, streamed from global memory.
@@ -220,19 +219,15 @@ __global__ void __launch_bounds__(kThreads) topk_rows_kernel(RowSpec R, int k, i
     sort_and_write(s_sel, kk, k, idx + (int64_t)row * k, top ? top + (int64_t)row * k : nullptr);
 }
 
-// Step 1 of long rows: sampled threshold, then each CTA filters one slice.
-__global__ void __launch_bounds__(kThreads) topk_filter_kernel(RowSpec R, int k, uint64_t* cand, int cap,
-                                                               uint32_t* cnt) {
+// Step 1a of long rows: one CTA per row sorts a strided sample of 2048
+// scores and keeps a threshold estimate (an orderable key) for the filter.
+__global__ void __launch_bounds__(kThreads) topk_threshold_kernel(RowSpec R, int k, uint32_t* thr_out) {
     __shared__ uint32_t s_key[kSample];
-    __shared__ uint32_t s_thr;
-    const int row = blockIdx.y;
+    const int row = blockIdx.x;
     const int tid = threadIdx.x;
     const int64_t n = R.count(row);
     if (n <= kSegMax) return;   // the final step reads such rows whole
-    const int64_t beg = (int64_t)blockIdx.x * kSlice;
-    if (beg >= n) return;
     const float* srow = R.scores + (int64_t)row * R.ld;
-    // the same strided sample in every CTA of the row
     for (int j = tid; j < kSample; j += kThreads) s_key[j] = orderable(srow[(int64_t)j * n / kSample]);
     __syncthreads();
     for (int size = 2; size <= kSample; size <<= 1) {
@@ -251,10 +246,22 @@ __global__ void __launch_bounds__(kThreads) topk_filter_kernel(RowSpec R, int k,
         // expected sample entries at or above the k-th score: k * S / n
         int64_t r = (int64_t)((1.25 * (double)k * kSample) / (double)n) + 16;
         if (r > kSample - 1) r = kSample - 1;
-        s_thr = s_key[r];
+        thr_out[row] = s_key[r];
     }
-    __syncthreads();
-    const uint32_t thr = s_thr;
+}
+
+// Step 1b: each CTA appends the composites of its slice that reach the
+// row's threshold to the row's candidate buffer.
+__global__ void __launch_bounds__(kThreads) topk_filter_kernel(RowSpec R, const uint32_t* thr_in, uint64_t* cand,
+                                                               int cap, uint32_t* cnt) {
+    const int row = blockIdx.y;
+    const int tid = threadIdx.x;
+    const int64_t n = R.count(row);
+    if (n <= kSegMax) return;
+    const int64_t beg = (int64_t)blockIdx.x * kSlice;
+    if (beg >= n) return;
+    const float* srow = R.scores + (int64_t)row * R.ld;
+    const uint32_t thr = thr_in[row];
     int64_t end = beg + kSlice;
     if (end > n) end = n;
     uint64_t* crow = cand + (int64_t)row * cap;
@@ -321,7 +328,7 @@ static int candidate_cap(int k) {
 
 size_t topk_workspace_bytes(int nq, int64_t ncols, int k) {
     if (ncols <= kSegMax) return 0;
-    return align256((size_t)nq * candidate_cap(k) * sizeof(uint64_t)) + align256((size_t)nq * sizeof(uint32_t));
+    return align256((size_t)nq * candidate_cap(k) * sizeof(uint64_t)) + align256((size_t)nq * 2 * sizeof(uint32_t));
 }
 
 static cudaError_t topk_run(const RowSpec& R, int nq, int k, int32_t* idx, float* top, void* ws, cudaStream_t st) {
@@ -338,10 +345,14 @@ static cudaError_t topk_run(const RowSpec& R, int nq, int k, int32_t* idx, float
     const int cap = candidate_cap(k);
     uint64_t* cand = (uint64_t*)ws;
     uint32_t* cnt = (uint32_t*)((char*)ws + align256((size_t)nq * cap * sizeof(uint64_t)));
+    uint32_t* thr = cnt + nq;
     e = cudaMemsetAsync(cnt, 0, (size_t)nq * sizeof(uint32_t), st);
     if (e != cudaSuccess) return e;
+    CSA_LAUNCH(st, "topk_threshold", topk_threshold_kernel<<<nq, kThreads, 0, st>>>(R, k, thr));
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
     const int slices = (int)((R.ncols + kSlice - 1) / kSlice);
-    CSA_LAUNCH(st, "topk_filter", topk_filter_kernel<<<dim3(slices, nq), kThreads, 0, st>>>(R, k, cand, cap, cnt));
+    CSA_LAUNCH(st, "topk_filter", topk_filter_kernel<<<dim3(slices, nq), kThreads, 0, st>>>(R, thr, cand, cap, cnt));
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(topk_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
