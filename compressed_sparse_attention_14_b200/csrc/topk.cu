@@ -16,11 +16,12 @@
 // composites >= T; a bitonic network sorts them.
 //
 // Rows longer than one CTA's shared memory take two steps:
-//   1. threshold (one CTA per row): sort a strided sample of 2048 scores and
-//      take an estimate low enough that, for any row that is not
-//      adversarial, well over k scores reach it (a rank ~1.25x the expected
-//      count plus 16); filter (several CTAs per row): each appends the
-//      composites of its slice that reach it to the row's candidate buffer;
+//   1. threshold (one CTA per row): from a strided sample of 1024 scores take
+//      an estimate low enough that, for any row that is not adversarial,
+//      well over k scores reach it (the sample value of rank ~1.25x the
+//      expected count plus 16); filter (several CTAs per row): each appends
+//      the composites of its slice that reach it to the row's candidate
+//      buffer;
 //   2. final (one CTA per row): when at least min(k, n) and at most the
 //      buffer's capacity of candidates arrived, the exact selection runs on
 //      them; otherwise it runs on the whole row, streamed from global memory.
@@ -43,10 +44,11 @@ __device__ __forceinline__ uint64_t composite(float s, int64_t col) {
     return ((uint64_t)orderable(s) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)col);
 }
 
-constexpr int kThreads = 1024;
+// Small CTAs: these steps are dominated by barrier latency, not arithmetic.
+constexpr int kThreads = 256;
 constexpr int kSegMax = 16384;     // composites one CTA holds (128 KB)
-constexpr int kSample = 2048;      // sample for the threshold estimate
-constexpr int kSlice = 8192;       // scores per filter CTA
+constexpr int kSample = 1024;      // sample for the threshold estimate
+constexpr int kSlice = 4096;       // scores per filter CTA
 
 // The candidate columns of each row: 0 .. count(row) - 1.
 struct RowSpec {
@@ -168,34 +170,97 @@ __device__ void collect(const Src& src, int64_t n, uint64_t thr, int kk, uint64_
     __syncthreads();
 }
 
-// Bitonic sort of sel[0..P) descending (P a power of two >= kk; the slots
-// above kk are filled with 0), then idx / score output for one row.
-__device__ void sort_and_write(uint64_t* sel, int kk, int k, int32_t* idx_row, float* score_row) {
-    const int tid = threadIdx.x;
-    int P = 1;
-    while (P < kk) P <<= 1;
-    for (int j = kk + tid; j < P; j += kThreads) sel[j] = 0ull;
-    __syncthreads();
-    for (int size = 2; size <= P; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int i = tid; i < (P >> 1); i += kThreads) {
-                const int lo = 2 * i - (i & (stride - 1));
-                const int hi = lo + stride;
-                const bool desc = (lo & size) == 0;
-                const uint64_t a = sel[lo], b = sel[hi];
-                if ((a < b) == desc) { sel[lo] = b; sel[hi] = a; }
-            }
-            __syncthreads();
+// Bitonic sort of up to 2048 64-bit keys, descending, by all threads of the
+// CTA. Element e = j * kThreads + t lives in register v[j] of thread t. A
+// compare-exchange partner at distance `stride` is in the same warp
+// (stride < 32: shuffle), in another warp (stride < kThreads: double-buffered
+// shared memory, one barrier), or in the same thread (register swap).
+constexpr int kSortMax = CSA_MAX_TOPK;
+constexpr int kPerThread = kSortMax / kThreads;
+
+template <int SJ>
+__device__ __forceinline__ void swap_in_thread(uint64_t (&v)[kPerThread], int E, int size, int t) {
+#pragma unroll
+    for (int j = 0; j < kPerThread; ++j) {
+        if ((j & SJ) == 0 && j < E) {
+            const int e = j * kThreads + t;
+            const bool desc = (e & size) == 0;
+            const uint64_t a = v[j], b = v[j ^ SJ];
+            const bool sw = (a < b) == desc;
+            v[j] = sw ? b : a;
+            v[j ^ SJ] = sw ? a : b;
         }
     }
-    for (int j = tid; j < k; j += kThreads) {
-        const uint64_t x = (j < kk) ? sel[j] : 0ull;
-        if (x == 0ull) {
-            idx_row[j] = -1;
-            if (score_row) score_row[j] = -INFINITY;
-        } else {
-            idx_row[j] = (int32_t)(0xFFFFFFFFu - (uint32_t)(x & 0xFFFFFFFFull));
-            if (score_row) score_row[j] = from_orderable((uint32_t)(x >> 32));
+}
+
+__device__ void bitonic_desc(uint64_t (&v)[kPerThread], int P, uint64_t* xbuf /* [2][kSortMax] */) {
+    const int t = threadIdx.x;
+    const int E = P / kThreads;          // P >= kThreads here
+    int pb = 0;
+    for (int size = 2; size <= P; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            if (stride >= kThreads) {
+                const int sj = stride / kThreads;
+                if (sj == 1) swap_in_thread<1>(v, E, size, t);
+                else if (sj == 2) swap_in_thread<2>(v, E, size, t);
+                else swap_in_thread<4>(v, E, size, t);
+            } else if (stride >= 32) {
+#pragma unroll
+                for (int j = 0; j < kPerThread; ++j)
+                    if (j < E) xbuf[pb * kSortMax + j * kThreads + t] = v[j];
+                __syncthreads();
+#pragma unroll
+                for (int j = 0; j < kPerThread; ++j) {
+                    if (j < E) {
+                        const int e = j * kThreads + t;
+                        const uint64_t y = xbuf[pb * kSortMax + j * kThreads + (t ^ stride)];
+                        const bool keep_max = ((e & stride) == 0) == ((e & size) == 0);
+                        v[j] = keep_max ? (v[j] > y ? v[j] : y) : (v[j] < y ? v[j] : y);
+                    }
+                }
+                pb ^= 1;
+            } else {
+#pragma unroll
+                for (int j = 0; j < kPerThread; ++j) {
+                    if (j < E) {
+                        const int e = j * kThreads + t;
+                        const uint64_t y = __shfl_xor_sync(0xffffffffu, v[j], stride);
+                        const bool keep_max = ((e & stride) == 0) == ((e & size) == 0);
+                        v[j] = keep_max ? (v[j] > y ? v[j] : y) : (v[j] < y ? v[j] : y);
+                    }
+                }
+            }
+        }
+    }
+}
+
+// Sort sel[0..kk) (the winners, arbitrary order) descending and write the
+// row's idx / scores; slots past kk get -1 / -inf.
+__device__ void sort_and_write(uint64_t* sel, int kk, int k, int32_t* idx_row, float* score_row,
+                               uint64_t* xbuf) {
+    const int tid = threadIdx.x;
+    int P = kThreads;
+    while (P < kk) P <<= 1;
+    uint64_t v[kPerThread];
+#pragma unroll
+    for (int j = 0; j < kPerThread; ++j) {
+        const int e = j * kThreads + tid;
+        v[j] = (e < kk) ? sel[e] : 0ull;
+    }
+    __syncthreads();   // sel may alias xbuf
+    bitonic_desc(v, P, xbuf);
+#pragma unroll
+    for (int j = 0; j < kPerThread; ++j) {
+        const int e = j * kThreads + tid;
+        if (e < k) {
+            const uint64_t x = (e < kk) ? v[j] : 0ull;
+            if (x == 0ull) {
+                idx_row[e] = -1;
+                if (score_row) score_row[e] = -INFINITY;
+            } else {
+                idx_row[e] = (int32_t)(0xFFFFFFFFu - (uint32_t)(x & 0xFFFFFFFFull));
+                if (score_row) score_row[e] = from_orderable((uint32_t)(x >> 32));
+            }
         }
     }
 }
@@ -205,7 +270,8 @@ __device__ void sort_and_write(uint64_t* sel, int kk, int k, int32_t* idx_row, f
 // Rows of at most kSegMax candidates: one CTA per row, the row in smem.
 __global__ void __launch_bounds__(kThreads) topk_rows_kernel(RowSpec R, int k, int32_t* idx, float* top) {
     extern __shared__ uint64_t s_elems[];
-    __shared__ uint64_t s_sel[CSA_MAX_TOPK];
+    __shared__ uint64_t s_x[2 * kSortMax];
+    uint64_t* s_sel = s_x;
     __shared__ SelShared sh;
     const int row = blockIdx.x;
     const int64_t n = R.count(row);
@@ -216,44 +282,51 @@ __global__ void __launch_bounds__(kThreads) topk_rows_kernel(RowSpec R, int k, i
     SmemSrc src{s_elems};
     const uint64_t thr = radix_threshold(src, n, k, sh);
     collect(src, n, thr, kk, s_sel, sh);
-    sort_and_write(s_sel, kk, k, idx + (int64_t)row * k, top ? top + (int64_t)row * k : nullptr);
+    sort_and_write(s_sel, kk, k, idx + (int64_t)row * k, top ? top + (int64_t)row * k : nullptr, s_x);
 }
 
-// Step 1a of long rows: one CTA per row sorts a strided sample of 2048
-// scores and keeps a threshold estimate (an orderable key) for the filter.
-__global__ void __launch_bounds__(kThreads) topk_threshold_kernel(RowSpec R, int k, uint32_t* thr_out) {
-    __shared__ uint32_t s_key[kSample];
+// Step 1a of long rows: one CTA per row takes a strided sample of 1024
+// scores, sorts it (one element per thread; shuffles inside a warp, shared
+// memory across warps) and keeps the sample value of rank r as the row's
+// threshold estimate (an orderable key).
+constexpr int kThrThreads = kSample;
+__global__ void __launch_bounds__(kThrThreads) topk_threshold_kernel(RowSpec R, int k, uint32_t* thr_out) {
+    __shared__ uint32_t s_key[2][kSample];
     const int row = blockIdx.x;
-    const int tid = threadIdx.x;
+    const int t = threadIdx.x;
     const int64_t n = R.count(row);
     if (n <= kSegMax) return;   // the final step reads such rows whole
     const float* srow = R.scores + (int64_t)row * R.ld;
-    for (int j = tid; j < kSample; j += kThreads) s_key[j] = orderable(srow[(int64_t)j * n / kSample]);
-    __syncthreads();
+    uint32_t x = orderable(srow[(int64_t)t * n / kSample]);
+    int pb = 0;
     for (int size = 2; size <= kSample; size <<= 1) {
         for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int i = tid; i < kSample / 2; i += kThreads) {
-                const int lo = 2 * i - (i & (stride - 1));
-                const int hi = lo + stride;
-                const bool desc = (lo & size) == 0;
-                const uint32_t a = s_key[lo], b = s_key[hi];
-                if ((a < b) == desc) { s_key[lo] = b; s_key[hi] = a; }
+            uint32_t y;
+            if (stride >= 32) {
+                s_key[pb][t] = x;
+                __syncthreads();
+                y = s_key[pb][t ^ stride];
+                pb ^= 1;
+            } else {
+                y = __shfl_xor_sync(0xffffffffu, x, stride);
             }
-            __syncthreads();
+            const bool keep_max = ((t & stride) == 0) == ((t & size) == 0);
+            x = keep_max ? max(x, y) : min(x, y);
         }
     }
-    if (tid == 0) {
-        // expected sample entries at or above the k-th score: k * S / n
-        int64_t r = (int64_t)((1.25 * (double)k * kSample) / (double)n) + 16;
-        if (r > kSample - 1) r = kSample - 1;
-        thr_out[row] = s_key[r];
-    }
+    // expected sample entries at or above the k-th score: k * S / n
+    int64_t r = (int64_t)((1.25 * (double)k * kSample) / (double)n) + 16;
+    if (r > kSample - 1) r = kSample - 1;
+    if (t == (int)r) thr_out[row] = x;
 }
 
-// Step 1b: each CTA appends the composites of its slice that reach the
-// row's threshold to the row's candidate buffer.
+// Step 1b: each CTA collects the composites of its slice that reach the
+// row's threshold in shared memory, reserves room in the row's candidate
+// buffer with one atomic, and copies them there.
 __global__ void __launch_bounds__(kThreads) topk_filter_kernel(RowSpec R, const uint32_t* thr_in, uint64_t* cand,
                                                                int cap, uint32_t* cnt) {
+    __shared__ uint64_t s_out[kSlice];
+    __shared__ uint32_t s_n, s_base;
     const int row = blockIdx.y;
     const int tid = threadIdx.x;
     const int64_t n = R.count(row);
@@ -264,7 +337,8 @@ __global__ void __launch_bounds__(kThreads) topk_filter_kernel(RowSpec R, const 
     const uint32_t thr = thr_in[row];
     int64_t end = beg + kSlice;
     if (end > n) end = n;
-    uint64_t* crow = cand + (int64_t)row * cap;
+    if (tid == 0) s_n = 0;
+    __syncthreads();
     const int lane = tid & 31;
     for (int64_t i0 = beg + tid - lane; i0 < end; i0 += kThreads) {
         const int64_t i = i0 + lane;
@@ -274,20 +348,26 @@ __global__ void __launch_bounds__(kThreads) topk_filter_kernel(RowSpec R, const 
         if (!m) continue;
         const int leader = __ffs(m) - 1;
         uint32_t base = 0;
-        if (lane == leader) base = atomicAdd(&cnt[row], (uint32_t)__popc(m));
+        if (lane == leader) base = atomicAdd(&s_n, (uint32_t)__popc(m));
         base = __shfl_sync(0xffffffffu, base, leader);
-        if (take) {
-            const uint32_t slot = base + __popc(m & ((1u << lane) - 1u));
-            if (slot < (uint32_t)cap) crow[slot] = composite(s, i);
-        }
+        if (take) s_out[base + __popc(m & ((1u << lane) - 1u))] = composite(s, i);
     }
+    __syncthreads();
+    const uint32_t c = s_n;
+    if (tid == 0) s_base = c ? atomicAdd(&cnt[row], c) : 0u;
+    __syncthreads();
+    const uint32_t base = s_base;
+    uint64_t* crow = cand + (int64_t)row * cap;
+    for (uint32_t j = tid; j < c; j += kThreads)
+        if (base + j < (uint32_t)cap) crow[base + j] = s_out[j];
 }
 
 // Step 2 of long rows (short rows are read whole): exact selection.
 __global__ void __launch_bounds__(kThreads) topk_final_kernel(RowSpec R, int k, const uint64_t* cand, int cap,
                                                               const uint32_t* cnt, int32_t* idx, float* top) {
     extern __shared__ uint64_t s_elems[];
-    __shared__ uint64_t s_sel[CSA_MAX_TOPK];
+    __shared__ uint64_t s_x[2 * kSortMax];
+    uint64_t* s_sel = s_x;
     __shared__ SelShared sh;
     const int row = blockIdx.x;
     const int64_t n = R.count(row);
@@ -315,7 +395,7 @@ __global__ void __launch_bounds__(kThreads) topk_final_kernel(RowSpec R, int k, 
             collect(src, n, thr, kk, s_sel, sh);
         }
     }
-    sort_and_write(s_sel, kk, k, idx + (int64_t)row * k, top ? top + (int64_t)row * k : nullptr);
+    sort_and_write(s_sel, kk, k, idx + (int64_t)row * k, top ? top + (int64_t)row * k : nullptr, s_x);
 }
 
 // ---------------------------------------------------------------- host side
@@ -348,7 +428,7 @@ static cudaError_t topk_run(const RowSpec& R, int nq, int k, int32_t* idx, float
     uint32_t* thr = cnt + nq;
     e = cudaMemsetAsync(cnt, 0, (size_t)nq * sizeof(uint32_t), st);
     if (e != cudaSuccess) return e;
-    CSA_LAUNCH(st, "topk_threshold", topk_threshold_kernel<<<nq, kThreads, 0, st>>>(R, k, thr));
+    CSA_LAUNCH(st, "topk_threshold", topk_threshold_kernel<<<nq, kThrThreads, 0, st>>>(R, k, thr));
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int slices = (int)((R.ncols + kSlice - 1) / kSlice);
