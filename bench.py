@@ -90,6 +90,12 @@ def max_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
+def job_rate(units_per_rank: float, world: int, ms_step_max: float) -> float:
+    """Whole-job throughput: every rank processes units_per_rank units per
+    step and the step takes the slowest rank's time."""
+    return world * units_per_rank / (ms_step_max / 1e3)
+
+
 def dist_done(world):
     if world > 1:
         import torch.distributed as dist
@@ -592,7 +598,7 @@ def run_ours(args, rank, world, local):
     e2e_ms = max_over_ranks(e2e_timer.total_ms(), world) / args.steps
 
     units = wl["units"]
-    value = world * units / (ms_step / 1e3)
+    value = job_rate(units, world, ms_step)
     peaks = measured_peaks()
 
     def roofline_of(name):
@@ -626,7 +632,7 @@ def run_ours(args, rank, world, local):
             "kernels_ms_per_step": {k: v[0] / args.steps for k, v in sorted(trace.items())},
             "other_kernels_roofline": {n: {k: r[k] for k in ("bound", "achieved", "unit", "frac")}
                                        for n, r in others.items()},
-            "e2e": {"value": world * units / (e2e_ms / 1e3), "unit": wl["unit"], "h2d_bytes_per_step": wl["h2d"],
+            "e2e": {"value": job_rate(units, world, e2e_ms), "unit": wl["unit"], "h2d_bytes_per_step": wl["h2d"],
                     "d2h_bytes_per_step": wl["d2h"]},
             "gpu_launches": launches, "clocks": clk, "wall_s_timed": t_wall}
     if wl.get("step_bytes"):
