@@ -17,9 +17,10 @@
 // it by more than 2^8 — exact, since the final normalisation uses the same
 // reference, and cheap, since it rarely moves after the first tile.
 //
-// Entry sources: CSA (sparse) gathers the selected rows with TMA
-// tile::gather4 (four rows per copy); HCA (dense) loads 128 consecutive rows
-// per 64-dim block with one TMA box. The tile's 64-dim blocks are released
+// Entry sources: CSA (sparse) gathers the selected rows with 16-byte
+// cp.async (the producer warp moves four rows' 128-byte block per
+// instruction); HCA (dense) loads 128 consecutive rows per 64-dim block with
+// one TMA box. The tile's 64-dim blocks are released
 // one by one as the second product finishes with them, so the next tile's
 // gather overlaps it.
 //
@@ -46,6 +47,7 @@ constexpr float kRescaleLog2 = 8.0f;    // move the reference max past 2^8
 struct MqaArgs {
     QueryMap qm;
     int n_seq, mp;
+    const void* KV;           // [n_seq * Nmax][c] bf16
     const int32_t* idx;       // sparse entry lists, or nullptr (dense)
     int k;
     int nq, H, c;
@@ -64,13 +66,23 @@ struct MqaArgs {
     uint32_t tmem_cols, q_bytes;
 };
 
-__device__ __forceinline__ void gather4(void* dst, const void* tmap, uint64_t* bar, int x, int y0, int y1, int y2,
-                                        int y3) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(tc::smem_u32(dst)),
-        "l"(tmap), "r"(tc::smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
-        : "memory");
+// 16-byte asynchronous global -> shared copy (L1 bypassed) and its groups.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until at most n (0..7) of this thread's most recent groups are pending.
+__device__ __forceinline__ void cp_async_wait_pending(int n) {
+    switch (n) {
+        case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+        case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+        case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+        case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+        case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
+        case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
+        case 6: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
+        default: asm volatile("cp.async.wait_group 7;" ::: "memory"); break;
+    }
 }
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
@@ -102,7 +114,6 @@ __device__ __forceinline__ void bar_sync_128() { asm volatile("bar.sync 1, 128;"
 
 __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_constant__ MqaArgs a,
                                                              const __grid_constant__ CUtensorMap tmQ,
-                                                             const __grid_constant__ CUtensorMap tmRow,
                                                              const __grid_constant__ CUtensorMap tmTile) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -170,33 +181,71 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
                     tc::tma_load_2d(q_s + (size_t)b * a.hg * 128, &tmQ, q_full, b * 64, t * a.H + h0);
             }
             int j = 0;
-            for (; j < ntiles; ++j) {
-                bool ok = true;
-                if (lane == 0) {
-                    for (int b = 0; b < a.dblocks && ok; ++b) {
-                        if (j > 0) ok = wait_or_abort(&kv_empty[b], (j - 1) & 1, abort_flag, a.status);
-                        if (ok) tc::mbar_expect_tx(&kv_full[b], kE * 128);
-                    }
-                }
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
-                const int64_t e0 = e_beg + (int64_t)j * kE;
-                if (a.idx) {
-                    int rows[4];
+            if (a.idx) {
+                // Sparse rows: 16-byte cp.async by the whole warp. One warp
+                // instruction moves one 64-dim block (128 B) of four rows, so
+                // every access is a full, aligned 128-byte line; the chunk
+                // lands at its 128-byte-swizzle position. (A TMA gather4 moves
+                // the same 512 B per instruction but its issue rate, not DRAM,
+                // bounded the tile load.) Block b is handed to the MMA once
+                // this warp's copies of it have completed.
+                const int chunk = lane & 7, rsub = lane >> 3;
+                const char* kv_g = (const char*)a.KV;
+                const int64_t row_bytes = (int64_t)a.c * 2;
+                for (; j < ntiles; ++j) {
+                    const int64_t e0 = e_beg + (int64_t)j * kE;
+                    int rows[kE / 4];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int64_t e = e0 + lane * 4 + u;
+                    for (int i = 0; i < kE / 4; ++i) {
+                        const int64_t e = e0 + 4 * i + rsub;
                         int s = -1;
                         if (e < e_end) s = a.idx[(int64_t)t * a.k + e];
                         if (s < 0 || s >= a.Nmax) s = 0;   // masked in the softmax
-                        rows[u] = (int)(row0 + s);
+                        rows[i] = (int)(row0 + s);
                     }
-                    for (int b = 0; b < a.dblocks; ++b)
-                        gather4(kv_s + (size_t)b * kE * 128 + lane * 4 * 128, &tmRow, &kv_full[b], b * 64, rows[0],
-                                rows[1], rows[2], rows[3]);
-                } else if (lane == 0) {
-                    for (int b = 0; b < a.dblocks; ++b)
-                        tc::tma_load_2d(kv_s + (size_t)b * kE * 128, &tmTile, &kv_full[b], b * 64, (int)(row0 + e0));
+                    bool ok = true;
+                    for (int b = 0; b < a.dblocks; ++b) {
+                        if (j > 0 && lane == 0) ok = wait_or_abort(&kv_empty[b], (j - 1) & 1, abort_flag, a.status);
+                        ok = __shfl_sync(0xffffffffu, ok, 0);
+                        if (!ok) break;
+                        uint8_t* dst = kv_s + (size_t)b * kE * 128;
+#pragma unroll
+                        for (int i = 0; i < kE / 4; ++i) {
+                            const int r = 4 * i + rsub;
+                            cp_async16(dst + r * 128 + ((chunk ^ (r & 7)) << 4),
+                                       kv_g + (int64_t)rows[i] * row_bytes + b * 128 + chunk * 16);
+                        }
+                        cp_async_commit();
+                    }
+                    // hand the blocks over in order as they complete
+                    const int issued = ok ? a.dblocks : 0;
+                    for (int b = 0; b < issued; ++b) {
+                        cp_async_wait_pending(issued - 1 - b);
+                        tc::fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) tc::mbar_arrive(&kv_full[b]);
+                    }
+                    if (!ok) {
+                        cp_async_wait_pending(0);
+                        break;
+                    }
+                }
+            } else {
+                for (; j < ntiles; ++j) {
+                    bool ok = true;
+                    if (lane == 0) {
+                        for (int b = 0; b < a.dblocks && ok; ++b) {
+                            if (j > 0) ok = wait_or_abort(&kv_empty[b], (j - 1) & 1, abort_flag, a.status);
+                            if (ok) tc::mbar_expect_tx(&kv_full[b], kE * 128);
+                        }
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                    const int64_t e0 = e_beg + (int64_t)j * kE;
+                    if (lane == 0)
+                        for (int b = 0; b < a.dblocks; ++b)
+                            tc::tma_load_2d(kv_s + (size_t)b * kE * 128, &tmTile, &kv_full[b], b * 64,
+                                            (int)(row0 + e0));
                 }
             }
             // drain: the last issued tile and q must have landed
@@ -295,11 +344,28 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
                 need |= z[h] > mref_s[h] + kRescaleLog2;
             }
             if (bar_or_128(need)) {
-                // new reference: per-head max over the tile's 128 entries
+                // new reference: per-head max over the tile's 128 entries. A
+                // butterfly reduce-scatter over the warp leaves lane l with the
+                // maxima of heads 2l and 2l+1 (62 shuffles instead of 320).
+                {
+                    float v[64];
 #pragma unroll
-                for (int h = 0; h < 64; ++h) {
-                    float mx = warp_max(z[h]);
-                    if (lane == (h & 31)) red_s[quad * 64 + h] = mx;
+                    for (int h = 0; h < 64; ++h) v[h] = z[h];
+#pragma unroll
+                    for (int r = 0; r < 5; ++r) {
+                        const int o = 16 >> r, nh = 32 >> r;
+                        const bool upper = (lane & o) != 0;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            if (i < nh) {
+                                const float send = upper ? v[i] : v[i + nh];
+                                const float keep = upper ? v[i + nh] : v[i];
+                                v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, o));
+                            }
+                        }
+                    }
+                    red_s[quad * 64 + 2 * lane] = v[0];
+                    red_s[quad * 64 + 2 * lane + 1] = v[1];
                 }
                 bar_sync_128();
                 if (eth < 64) {
@@ -357,14 +423,16 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
         if (ok && ntiles > 0) ok = wait_or_abort(o_done, (ntiles - 1) & 1, abort_flag, a.status);
         tc::tc_fence_after();
         // per-head sums: fixed-order reduction of the 128 per-entry partials
-        float* lred = (float*)kv_s;   // the KV tile is no longer read
+        // [128][65] floats (padded: no bank conflicts) over the KV tile and, for
+        // c = 128, the start of q: neither is read any more
+        float* lred = (float*)kv_s;
         bar_sync_128();
 #pragma unroll
-        for (int h = 0; h < 64; ++h) lred[h * 128 + eth] = lpart[h];
+        for (int h = 0; h < 64; ++h) lred[eth * 65 + h] = lpart[h];
         bar_sync_128();
         if (eth < 64) {
             float sum = 0.f;
-            for (int i = 0; i < 128; ++i) sum += lred[eth * 128 + i];
+            for (int i = 0; i < 128; ++i) sum += lred[i * 65 + eth];
             lsum_s[eth] = sum;
         }
         bar_sync_128();
@@ -390,19 +458,20 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
             bar_sync_128();
             for (int mt = 0; mt < a.mtiles; ++mt) {
                 const int dim = mt * 128 + row;
-                for (int cc = 0; cc < hg; cc += 16) {
-                    float v[16];
-                    if (have_o) {
-                        tc::tmem_ld16(tmem_O + ((uint32_t)(quad * 32) << 16) + mt * hg + cc, v);
-                        tc::tmem_ld_wait();
-                    }
+                float v[64];
+                if (have_o) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int h = h0 + cc + i;
-                        if (h < a.H) {
-                            float o = (have_o && mref_s[cc + i] != -INFINITY) ? v[i] * alpha_s[cc + i] : 0.f;
-                            a.out[((int64_t)t * a.H + h) * a.c + dim] = __float2bfloat16_rn(o);
-                        }
+                    for (int u = 0; u < 4; ++u)
+                        tc::tmem_ld16(tmem_O + ((uint32_t)(quad * 32) << 16) + mt * hg + 16 * u,
+                                      *reinterpret_cast<float(*)[16]>(v + 16 * u));
+                    tc::tmem_ld_wait();
+                }
+#pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    const int h = h0 + i;
+                    if (h < a.H) {
+                        float o = (have_o && mref_s[i] != -INFINITY) ? v[i] * alpha_s[i] : 0.f;
+                        a.out[((int64_t)t * a.H + h) * a.c + dim] = __float2bfloat16_rn(o);
                     }
                 }
             }
@@ -415,15 +484,16 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
             if (have_o) {
                 for (int mt = 0; mt < a.mtiles; ++mt) {
                     const int dim = mt * 128 + row;
-                    for (int cc = 0; cc < hg; cc += 16) {
-                        float v[16];
-                        tc::tmem_ld16(tmem_O + ((uint32_t)(quad * 32) << 16) + mt * hg + cc, v);
-                        tc::tmem_ld_wait();
+                    float v[64];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int h = h0 + cc + i;
-                            if (h < a.H) a.part_o[(((int64_t)t * a.nsplit + split) * a.H + h) * a.c + dim] = v[i];
-                        }
+                    for (int u = 0; u < 4; ++u)
+                        tc::tmem_ld16(tmem_O + ((uint32_t)(quad * 32) << 16) + mt * hg + 16 * u,
+                                      *reinterpret_cast<float(*)[16]>(v + 16 * u));
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) {
+                        const int h = h0 + i;
+                        if (h < a.H) a.part_o[(((int64_t)t * a.nsplit + split) * a.H + h) * a.c + dim] = v[i];
                     }
                 }
             }
@@ -459,6 +529,7 @@ cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, Que
     a.qm = QueryMap{qs.seq, qs.pos, qs.pos_base, qs.single_seq};
     a.n_seq = n_seq;
     a.mp = mp;
+    a.KV = KV;
     a.idx = idx;
     a.k = k;
     a.nq = nq;
@@ -485,9 +556,8 @@ cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, Que
     while (cols < need) cols <<= 1;
     a.tmem_cols = cols;
 
-    CUtensorMap tmQ, tmRow, tmTile;
+    CUtensorMap tmQ, tmTile;
     if (!make_tmap_bf16_2d(&tmQ, q, (uint64_t)nq * H, c, c, a.hg, 64)) return cudaErrorInvalidValue;
-    if (!make_tmap_bf16_2d(&tmRow, KV, (uint64_t)n_seq * Nmax, c, c, 1, 64)) return cudaErrorInvalidValue;
     if (!make_tmap_bf16_2d(&tmTile, KV, (uint64_t)n_seq * Nmax, c, c, kE, 64)) return cudaErrorInvalidValue;
 
     const size_t smem = 1024 + (size_t)a.dblocks * kE * 128 + a.q_bytes + kE * 128 + (64 * 4 + 256) * sizeof(float) +
@@ -495,7 +565,7 @@ cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, Que
     cudaError_t e = cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(nsplit, (H + a.hg - 1) / a.hg, nq);
-    CSA_LAUNCH(st, "mqa_tc", mqa_tc_kernel<<<grid, kThreads, smem, st>>>(a, tmQ, tmRow, tmTile));
+    CSA_LAUNCH(st, "mqa_tc", mqa_tc_kernel<<<grid, kThreads, smem, st>>>(a, tmQ, tmTile));
     return cudaGetLastError();
 }
 
