@@ -264,8 +264,8 @@ def decode_workload(shape, rank, batch=None):
     kernels = {
         "index_scores_tc": dict(bound="hbm", work=idx_kernel_bytes, files=("indexer_tc.cu", "tc.cuh", "common.cuh")),
         "mqa_tc": dict(bound="hbm", work=mqa_bytes, files=("mqa_tc.cu", "tc.cuh", "common.cuh")),
-        "topk_select": dict(bound="hbm", work=B * s.k * 4, files=("topk.cu",)),
-        "topk_filter": dict(bound="hbm", work=v_sum * 4, files=("topk.cu",)),
+        # one pass over each row's visible scores, k indices out
+        "topk_select": dict(bound="hbm", work=v_sum * 4 + B * s.k * 4, files=("topk.cu",)),
     }
     return dict(step=step, e2e_step=e2e_step, units=B, unit="queries/s", h2d=h2d, d2h=d2h,
                 kernels=kernels, step_bytes=step_bytes,

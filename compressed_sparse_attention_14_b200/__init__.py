@@ -237,9 +237,9 @@ def csa_topk_from_scores(scores, k: int, valid=None, valid_div: int = 1, ws=None
 
 def csa_topk_from_scores_noalloc(scores, k: int, valid=None, valid_div: int = 1, idx=None, top_scores=None):
     """csa_topk_from_scores without a workspace (for callers that cannot
-    allocate device memory when they select): the library's fixed 8 MiB
-    device array holds the intermediate candidates. Pass preallocated idx /
-    top_scores to make the call itself allocation-free."""
+    allocate device memory when they select): the selection keeps its
+    scratch in on-chip shared memory. Pass preallocated idx / top_scores to
+    make the call itself allocation-free."""
     nq, ncols = scores.shape
     if idx is None:
         idx = torch.empty((nq, k), dtype=torch.int32, device=scores.device)

@@ -10,23 +10,30 @@
 // +0.0). Composite keys are distinct and their descending order is exactly
 // the selection order, so the k largest composites ARE the answer.
 //
-// Exact selection (one CTA): an MSB-first radix select on the composites
-// (8-bit digits, warp-aggregated shared-memory histograms, a warp scan picks
-// the digit) finds the k-th largest composite T; the winners are all
-// composites >= T; a bitonic network sorts them.
-//
-// Rows longer than one CTA's shared memory take two steps:
-//   1. threshold (one CTA per row): from a strided sample of 1024 scores take
-//      an estimate low enough that, for any row that is not adversarial,
-//      well over k scores reach it (the sample value of rank ~1.25x the
-//      expected count plus 16); filter (several CTAs per row): each appends
-//      the composites of its slice that reach it to the row's candidate
-//      buffer;
-//   2. final (one CTA per row): when at least min(k, n) and at most the
-//      buffer's capacity of candidates arrived, the exact selection runs on
-//      them; otherwise it runs on the whole row, streamed from global memory.
-// Either way the result is exact: the k best are among the candidates
-// whenever at least k scores reach the threshold.
+// One launch, no global scratch; a row is served by one CTA, or by a cluster
+// of G CTAs (G = 2, 4, 8 when there are few long rows, so that the row's
+// pass over its scores has G SMs' worth of loads in flight):
+//   * a row of at most kCap candidates is read whole into shared memory;
+//   * a longer row is first narrowed to a candidate set: every CTA of the
+//     cluster takes the same strided sample of kSample scores and finds
+//     (radix select) the sample score of rank r = mu + 4 sqrt(mu) + 4,
+//     mu = k * kSample / n being the expected number of samples at or above
+//     the row's k-th score; CTA g keeps every score of its slice of the row
+//     at or above it (16-byte loads, warp-aggregated appends to its shared
+//     memory); CTA 0 then pulls the other CTAs' candidates over distributed
+//     shared memory. If at least min(k, n) and at most kCap scores reach the
+//     estimate, the k best are all among them; otherwise (ties, a row
+//     ordered against the strided sample) CTA 0 selects exactly on the whole
+//     row, streamed from global memory.
+//   * exact selection on the candidates: up to kSortMax of them are simply
+//     sorted (bitonic network); more go through an MSB-first radix select on
+//     the composites (8-bit digits, warp-aggregated shared-memory
+//     histograms, a warp scan picks the digit) that finds the k-th largest
+//     composite T; the winners are the composites >= T, and those are sorted.
+#include <cooperative_groups.h>
+
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -44,11 +51,24 @@ __device__ __forceinline__ uint64_t composite(float s, int64_t col) {
     return ((uint64_t)orderable(s) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)col);
 }
 
-// Small CTAs: these steps are dominated by barrier latency, not arithmetic.
-constexpr int kThreads = 256;
-constexpr int kSegMax = 16384;     // composites one CTA holds (128 KB)
-constexpr int kSample = 1024;      // sample for the threshold estimate
-constexpr int kSlice = 4096;       // scores per filter CTA
+namespace cg = cooperative_groups;
+
+constexpr int kThreads = 512;
+constexpr int kMaxCluster = 8;
+constexpr int kCap = 8192;          // candidates one CTA holds (64 KB)
+constexpr int kSample = 4096;       // sample for the threshold estimate
+constexpr int kSortMax = CSA_MAX_TOPK;
+constexpr int kPerThread = kSortMax / kThreads;
+// Dynamic shared memory: the candidates, then a scratch area that holds the
+// sample, later the winners and the sort's exchange buffer (the sort reads
+// the winners into registers before it reuses the area).
+constexpr size_t kCandBytes = (size_t)kCap * sizeof(uint64_t);
+constexpr size_t kScratchBytes = (size_t)2 * kSortMax * sizeof(uint64_t);
+static_assert(kScratchBytes >= (size_t)kSample * sizeof(uint64_t), "the sample must fit the scratch area");
+constexpr size_t kSmemBytes = kCandBytes + kScratchBytes;
+// When the launch has no more CTAs than SMs, each asks for more shared
+// memory than two CTAs can share, so that every CTA gets an SM of its own.
+constexpr size_t kSmemSpread = 160 * 1024;
 
 // The candidate columns of each row: 0 .. count(row) - 1.
 struct RowSpec {
@@ -155,7 +175,7 @@ __device__ void collect(const Src& src, int64_t n, uint64_t thr, int kk, uint64_
         const uint64_t x = src(i);
         if (x > thr) {
             const uint32_t slot = atomicAdd(&sh.cnt, 1u);
-            if (slot < (uint32_t)CSA_MAX_TOPK) sel[slot] = x;
+            if (slot < (uint32_t)kSortMax) sel[slot] = x;
         }
     }
     __syncthreads();
@@ -170,13 +190,12 @@ __device__ void collect(const Src& src, int64_t n, uint64_t thr, int kk, uint64_
     __syncthreads();
 }
 
-// Bitonic sort of up to 2048 64-bit keys, descending, by all threads of the
-// CTA. Element e = j * kThreads + t lives in register v[j] of thread t. A
+// Bitonic sort of up to kSortMax 64-bit keys, descending, by all threads of
+// the CTA. Element e = j * kThreads + t lives in register v[j] of thread t. A
 // compare-exchange partner at distance `stride` is in the same warp
 // (stride < 32: shuffle), in another warp (stride < kThreads: double-buffered
 // shared memory, one barrier), or in the same thread (register swap).
-constexpr int kSortMax = CSA_MAX_TOPK;
-constexpr int kPerThread = kSortMax / kThreads;
+static_assert(kSortMax <= 4 * kThreads, "in-thread strides above 2 * kThreads are not generated");
 
 template <int SJ>
 __device__ __forceinline__ void swap_in_thread(uint64_t (&v)[kPerThread], int E, int size, int t) {
@@ -200,10 +219,8 @@ __device__ void bitonic_desc(uint64_t (&v)[kPerThread], int P, uint64_t* xbuf /*
     for (int size = 2; size <= P; size <<= 1) {
         for (int stride = size >> 1; stride > 0; stride >>= 1) {
             if (stride >= kThreads) {
-                const int sj = stride / kThreads;
-                if (sj == 1) swap_in_thread<1>(v, E, size, t);
-                else if (sj == 2) swap_in_thread<2>(v, E, size, t);
-                else swap_in_thread<4>(v, E, size, t);
+                if (stride == kThreads) swap_in_thread<1>(v, E, size, t);
+                else swap_in_thread<2>(v, E, size, t);
             } else if (stride >= 32) {
 #pragma unroll
                 for (int j = 0; j < kPerThread; ++j)
@@ -234,20 +251,21 @@ __device__ void bitonic_desc(uint64_t (&v)[kPerThread], int P, uint64_t* xbuf /*
     }
 }
 
-// Sort sel[0..kk) (the winners, arbitrary order) descending and write the
-// row's idx / scores; slots past kk get -1 / -inf.
-__device__ void sort_and_write(uint64_t* sel, int kk, int k, int32_t* idx_row, float* score_row,
+// Sort src[0..cnt) (cnt <= kSortMax, arbitrary order) descending and write
+// the first kk = min(cnt, k) as the row's idx / scores; slots past kk get
+// -1 / -inf. src may alias xbuf.
+__device__ void sort_and_write(const uint64_t* src, int cnt, int kk, int k, int32_t* idx_row, float* score_row,
                                uint64_t* xbuf) {
     const int tid = threadIdx.x;
     int P = kThreads;
-    while (P < kk) P <<= 1;
+    while (P < cnt) P <<= 1;
     uint64_t v[kPerThread];
 #pragma unroll
     for (int j = 0; j < kPerThread; ++j) {
         const int e = j * kThreads + tid;
-        v[j] = (e < kk) ? sel[e] : 0ull;
+        v[j] = (e < cnt) ? src[e] : 0ull;
     }
-    __syncthreads();   // sel may alias xbuf
+    __syncthreads();   // src may alias xbuf
     bitonic_desc(v, P, xbuf);
 #pragma unroll
     for (int j = 0; j < kPerThread; ++j) {
@@ -265,192 +283,394 @@ __device__ void sort_and_write(uint64_t* sel, int kk, int k, int32_t* idx_row, f
     }
 }
 
-// ---------------------------------------------------------------- kernels
+// ---------------------------------------------------------------- key bins
+// Counting by value: a key (orderable score) falls into bin
+// (key - kmin) >> shift, shift chosen so that the keys span at most kBins
+// bins; bin order is value order. Exact integer arithmetic, so the smallest
+// key of bin B is kmin + (B << shift).
+constexpr int kBins = 2 * kThreads;     // two per thread in the scans
+constexpr int kBucketMax = 4096;        // candidates placed by counting (the scratch area)
+constexpr uint32_t kMaxBinLoad = 64;    // larger bins (heavy ties): bitonic path
+static_assert(kScratchBytes >= (size_t)kBucketMax * sizeof(uint64_t), "buckets must fit the scratch area");
 
-// Rows of at most kSegMax candidates: one CTA per row, the row in smem.
-__global__ void __launch_bounds__(kThreads) topk_rows_kernel(RowSpec R, int k, int32_t* idx, float* top) {
-    extern __shared__ uint64_t s_elems[];
-    __shared__ uint64_t s_x[2 * kSortMax];
-    uint64_t* s_sel = s_x;
-    __shared__ SelShared sh;
-    const int row = blockIdx.x;
-    const int64_t n = R.count(row);
-    const float* srow = R.scores + (int64_t)row * R.ld;
-    for (int64_t i = threadIdx.x; i < n; i += kThreads) s_elems[i] = composite(srow[i], i);
+struct BinShared {
+    uint32_t cnt[kBins];
+    uint32_t start[kBins];
+    uint32_t cur[kBins];
+    uint32_t red[2][kThreads / 32];
+    uint32_t B;
+    int overflow;
+};
+
+struct KeyBins {
+    uint32_t kmin;
+    int shift;
+    __device__ __forceinline__ int bin(uint32_t key) const { return (int)((key - kmin) >> shift); }
+};
+
+// Min and max over the CTA of the keys each thread passes (have = false: none).
+__device__ KeyBins key_bins(uint32_t lo, uint32_t hi, BinShared& bs) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    lo = __reduce_min_sync(0xffffffffu, lo);
+    hi = __reduce_max_sync(0xffffffffu, hi);
+    if (lane == 0) { bs.red[0][warp] = lo; bs.red[1][warp] = hi; }
     __syncthreads();
-    const int kk = (int)(n < k ? n : k);
-    SmemSrc src{s_elems};
-    const uint64_t thr = radix_threshold(src, n, k, sh);
-    collect(src, n, thr, kk, s_sel, sh);
-    sort_and_write(s_sel, kk, k, idx + (int64_t)row * k, top ? top + (int64_t)row * k : nullptr, s_x);
+    uint32_t mn = 0xffffffffu, mx = 0u;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) { mn = min(mn, bs.red[0][w]); mx = max(mx, bs.red[1][w]); }
+    KeyBins kb;
+    kb.kmin = mn;
+    const uint32_t span = mx > mn ? mx - mn : 0u;
+    const int bits = 32 - __clz(span);
+    kb.shift = bits > 10 ? bits - 10 : 0;    // (span >> shift) < 1024 = kBins
+    static_assert(kBins == 1024, "shift rule assumes 1024 bins");
+    return kb;
 }
 
-// Step 1a of long rows: one CTA per row takes a strided sample of 1024
-// scores, sorts it (one element per thread; shuffles inside a warp, shared
-// memory across warps) and keeps the sample value of rank r as the row's
-// threshold estimate (an orderable key).
-constexpr int kThrThreads = kSample;
-__global__ void __launch_bounds__(kThrThreads) topk_threshold_kernel(RowSpec R, int k, uint32_t* thr_out) {
-    __shared__ uint32_t s_key[2][kSample];
-    const int row = blockIdx.x;
-    const int t = threadIdx.x;
-    const int64_t n = R.count(row);
-    if (n <= kSegMax) return;   // the final step reads such rows whole
-    const float* srow = R.scores + (int64_t)row * R.ld;
-    uint32_t x = orderable(srow[(int64_t)t * n / kSample]);
-    int pb = 0;
-    for (int size = 2; size <= kSample; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            uint32_t y;
-            if (stride >= 32) {
-                s_key[pb][t] = x;
-                __syncthreads();
-                y = s_key[pb][t ^ stride];
-                pb ^= 1;
-            } else {
-                y = __shfl_xor_sync(0xffffffffu, x, stride);
-            }
-            const bool keep_max = ((t & stride) == 0) == ((t & size) == 0);
-            x = keep_max ? max(x, y) : min(x, y);
+// start[b] = elements in the bins above b (descending exclusive scan of
+// cnt); cur[b] = start[b]. Thread t owns bins kBins-1-2t and kBins-2-2t.
+// Also flags bins holding more than kMaxBinLoad. Ends with a barrier.
+__device__ void bins_scan_desc(BinShared& bs) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b0 = kBins - 1 - 2 * tid, b1 = b0 - 1;
+    const uint32_t c0 = bs.cnt[b0], c1 = bs.cnt[b1];
+    uint32_t incl = c0 + c1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) bs.red[0][warp] = incl;
+    if (c0 > kMaxBinLoad || c1 > kMaxBinLoad) bs.overflow = 1;
+    __syncthreads();
+    uint32_t base = 0;
+    for (int w = 0; w < warp; ++w) base += bs.red[0][w];
+    const uint32_t excl = base + incl - (c0 + c1);
+    bs.start[b0] = excl;
+    bs.start[b1] = excl + c0;
+    bs.cur[b0] = excl;
+    bs.cur[b1] = excl + c0;
+    __syncthreads();
+}
+
+__device__ __forceinline__ void bins_clear(BinShared& bs) {
+    for (int b = threadIdx.x; b < kBins; b += kThreads) bs.cnt[b] = 0;
+    if (threadIdx.x == 0) bs.overflow = 0;
+}
+
+// Threshold estimate from the row's strided sample: the smallest key of the
+// bin that holds the sample's r-th largest score, so that at least r sample
+// scores reach it.
+__device__ uint32_t sample_threshold(const float* srow, int64_t n, int r, BinShared& bs) {
+    constexpr int kPer = kSample / kThreads;
+    const int tid = threadIdx.x;
+    uint32_t key[kPer];
+    uint32_t lo = 0xffffffffu, hi = 0u;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+        const int t = u * kThreads + tid;
+        key[u] = orderable(__ldcg(srow + ((int64_t)t * n) / kSample));
+        lo = min(lo, key[u]);
+        hi = max(hi, key[u]);
+    }
+    bins_clear(bs);
+    const KeyBins kb = key_bins(lo, hi, bs);   // its barrier also orders the clear
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) atomicAdd(&bs.cnt[kb.bin(key[u])], 1u);
+    __syncthreads();
+    bins_scan_desc(bs);
+    const uint32_t ur = (uint32_t)r;
+    for (int b = tid; b < kBins; b += kThreads)
+        if (bs.start[b] < ur && bs.start[b] + bs.cnt[b] >= ur) bs.B = (uint32_t)b;
+    __syncthreads();
+    return kb.kmin + (bs.B << kb.shift);
+}
+
+// Exact top-k of e[0..n) (n <= kBucketMax, distinct composites) by counting:
+// place each key in its value bin (bins in descending order, arbitrary order
+// inside a bin), then each key's output slot is its bin's start plus the
+// number of keys of its bin above it. Writes the first k slots (padding
+// past n). Returns false, having written nothing, when some bin holds more
+// than kMaxBinLoad keys.
+__device__ bool select_by_bins(const uint64_t* e, int n, int k, int32_t* idx_row, float* score_row, uint64_t* bucket,
+                               BinShared& bs) {
+    const int tid = threadIdx.x;
+    uint32_t lo = 0xffffffffu, hi = 0u;
+    for (int i = tid; i < n; i += kThreads) {
+        const uint32_t key = (uint32_t)(e[i] >> 32);
+        lo = min(lo, key);
+        hi = max(hi, key);
+    }
+    bins_clear(bs);
+    const KeyBins kb = key_bins(lo, hi, bs);
+    for (int i = tid; i < n; i += kThreads) atomicAdd(&bs.cnt[kb.bin((uint32_t)(e[i] >> 32))], 1u);
+    __syncthreads();
+    bins_scan_desc(bs);
+    if (bs.overflow) return false;
+    for (int i = tid; i < n; i += kThreads) {
+        const uint64_t x = e[i];
+        bucket[atomicAdd(&bs.cur[kb.bin((uint32_t)(x >> 32))], 1u)] = x;
+    }
+    __syncthreads();
+    for (int p = tid; p < n; p += kThreads) {
+        const uint64_t x = bucket[p];
+        const int b = kb.bin((uint32_t)(x >> 32));
+        if ((int)bs.start[b] >= k) continue;
+        const int s0 = (int)bs.start[b], s1 = (int)bs.cur[b];
+        int rank = 0;
+        for (int q = s0; q < s1; ++q) rank += bucket[q] > x;
+        const int pos = s0 + rank;
+        if (pos < k) {
+            idx_row[pos] = (int32_t)(0xFFFFFFFFu - (uint32_t)(x & 0xFFFFFFFFull));
+            if (score_row) score_row[pos] = from_orderable((uint32_t)(x >> 32));
         }
     }
-    // expected sample entries at or above the k-th score: k * S / n
-    int64_t r = (int64_t)((1.25 * (double)k * kSample) / (double)n) + 16;
-    if (r > kSample - 1) r = kSample - 1;
-    if (t == (int)r) thr_out[row] = x;
+    for (int pos = n + tid; pos < k; pos += kThreads) {
+        idx_row[pos] = -1;
+        if (score_row) score_row[pos] = -INFINITY;
+    }
+    return true;
 }
 
-// Step 1b: each CTA collects the composites of its slice that reach the
-// row's threshold in shared memory, reserves room in the row's candidate
-// buffer with one atomic, and copies them there.
-__global__ void __launch_bounds__(kThreads) topk_filter_kernel(RowSpec R, const uint32_t* thr_in, uint64_t* cand,
-                                                               int cap, uint32_t* cnt) {
-    __shared__ uint64_t s_out[kSlice];
-    __shared__ uint32_t s_n, s_base;
-    const int row = blockIdx.y;
-    const int tid = threadIdx.x;
-    const int64_t n = R.count(row);
-    if (n <= kSegMax) return;
-    const int64_t beg = (int64_t)blockIdx.x * kSlice;
-    if (beg >= n) return;
-    const float* srow = R.scores + (int64_t)row * R.ld;
-    const uint32_t thr = thr_in[row];
-    int64_t end = beg + kSlice;
-    if (end > n) end = n;
-    if (tid == 0) s_n = 0;
-    __syncthreads();
-    const int lane = tid & 31;
-    for (int64_t i0 = beg + tid - lane; i0 < end; i0 += kThreads) {
-        const int64_t i = i0 + lane;
-        const float s = (i < end) ? srow[i] : 0.f;
-        const bool take = (i < end) && orderable(s) >= thr;
-        const unsigned m = __ballot_sync(0xffffffffu, take);
-        if (!m) continue;
+// Exact selection among n distinct composites (in shared memory, or the row
+// in global memory): by counting when they fit the buckets, else all of
+// them sorted when they fit the network, else radix select of the k-th,
+// collect the winners, sort those.
+template <class Src>
+__device__ void select_exact(const Src& src, int64_t n, int k, int32_t* idx_row, float* score_row,
+                             uint64_t* scratch, SelShared& sh, BinShared& bs) {
+    const int kk = (int)(n < k ? n : k);
+    if constexpr (std::is_same<Src, SmemSrc>::value) {
+        if (n <= kBucketMax && select_by_bins(src.e, (int)n, k, idx_row, score_row, scratch, bs)) return;
+        __syncthreads();   // the scratch area may hold buckets
+        if (n <= kSortMax) {
+            sort_and_write(src.e, (int)n, kk, k, idx_row, score_row, scratch);
+            return;
+        }
+    }
+    const uint64_t thr = radix_threshold(src, n, k, sh);
+    collect(src, n, thr, kk, scratch, sh);
+    sort_and_write(scratch, kk, kk, k, idx_row, score_row, scratch);
+}
+
+// Warp-aggregated append of s (column i) to buf when it reaches thr
+// (orderable); *cnt counts every taker, also past cap.
+__device__ __forceinline__ void append_if(float s, int64_t i, bool in, uint32_t thr, uint64_t* buf, uint32_t cap,
+                                          uint32_t* cnt) {
+    const int lane = threadIdx.x & 31;
+    const bool take = in && orderable(s) >= thr;
+    const unsigned m = __ballot_sync(0xffffffffu, take);
+    if (m) {
         const int leader = __ffs(m) - 1;
         uint32_t base = 0;
-        if (lane == leader) base = atomicAdd(&s_n, (uint32_t)__popc(m));
+        if (lane == leader) base = atomicAdd(cnt, (uint32_t)__popc(m));
         base = __shfl_sync(0xffffffffu, base, leader);
-        if (take) s_out[base + __popc(m & ((1u << lane) - 1u))] = composite(s, i);
+        const uint32_t slot = base + __popc(m & ((1u << lane) - 1u));
+        if (take && slot < cap) buf[slot] = composite(s, i);
     }
-    __syncthreads();
-    const uint32_t c = s_n;
-    if (tid == 0) s_base = c ? atomicAdd(&cnt[row], c) : 0u;
-    __syncthreads();
-    const uint32_t base = s_base;
-    uint64_t* crow = cand + (int64_t)row * cap;
-    for (uint32_t j = tid; j < c; j += kThreads)
-        if (base + j < (uint32_t)cap) crow[base + j] = s_out[j];
 }
 
-// Step 2 of long rows (short rows are read whole): exact selection.
-__global__ void __launch_bounds__(kThreads) topk_final_kernel(RowSpec R, int k, const uint64_t* cand, int cap,
-                                                              const uint32_t* cnt, int32_t* idx, float* top) {
-    extern __shared__ uint64_t s_elems[];
-    __shared__ uint64_t s_x[2 * kSortMax];
-    uint64_t* s_sel = s_x;
-    __shared__ SelShared sh;
-    const int row = blockIdx.x;
-    const int64_t n = R.count(row);
-    const int kk = (int)(n < k ? n : k);
-    const float* srow = R.scores + (int64_t)row * R.ld;
-    if (n <= kSegMax) {
-        for (int64_t i = threadIdx.x; i < n; i += kThreads) s_elems[i] = composite(srow[i], i);
-        __syncthreads();
-        SmemSrc src{s_elems};
-        const uint64_t thr = radix_threshold(src, n, k, sh);
-        collect(src, n, thr, kk, s_sel, sh);
-    } else {
-        const uint32_t c = cnt[row];
-        if (c >= (uint32_t)kk && c <= (uint32_t)cap) {
-            const uint64_t* crow = cand + (int64_t)row * cap;
-            for (int64_t i = threadIdx.x; i < (int64_t)c; i += kThreads) s_elems[i] = crow[i];
-            __syncthreads();
-            SmemSrc src{s_elems};
-            const uint64_t thr = radix_threshold(src, (int64_t)c, k, sh);
-            collect(src, (int64_t)c, thr, kk, s_sel, sh);
-        } else {
-            // the estimate missed (ties, adversarial rows): exact on the whole row
-            RowSrc src{srow};
-            const uint64_t thr = radix_threshold(src, n, k, sh);
-            collect(src, n, thr, kk, s_sel, sh);
+// Every score of srow[lo, hi) that reaches thr, appended to buf; kU 16-byte
+// loads in flight per thread.
+template <int kU>
+__device__ void filter_slice(const float* srow, int64_t lo, int64_t hi, uint32_t thr, uint64_t* buf, uint32_t cap,
+                             uint32_t* cnt) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    // scalar head up to the first 16-byte boundary, 16-byte body, scalar
+    // tail; the head and tail loads are issued first and used last
+    int64_t lo_v = lo + (int64_t)((4u - (((uint32_t)((uintptr_t)(srow + lo)) >> 2) & 3u)) & 3u);
+    if (lo_v > hi) lo_v = hi;
+    const int64_t nvec = (hi - lo_v) >> 2;
+    const int64_t hi_v = lo_v + 4 * nvec;
+    const int64_t ih = lo + tid, it = hi_v + tid;
+    const bool inh = ih < lo_v, intl = it < hi;
+    const float sh = inh ? __ldcg(srow + ih) : 0.f;
+    const float stl = intl ? __ldcg(srow + it) : 0.f;
+    const float4* v4 = reinterpret_cast<const float4*>(srow + lo_v);
+    static_assert(4 * kU <= 64, "one mask bit per value");
+    for (int64_t b0 = 0; b0 < nvec; b0 += kU * kThreads) {
+        float f[4 * kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int64_t j = b0 + u * kThreads + tid;
+            const float4 q = j < nvec ? __ldcg(v4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            f[4 * u] = q.x;
+            f[4 * u + 1] = q.y;
+            f[4 * u + 2] = q.z;
+            f[4 * u + 3] = q.w;
+        }
+        // this thread's takers, then one reservation per warp
+        uint64_t mask = 0;
+#pragma unroll
+        for (int e = 0; e < 4 * kU; ++e) {
+            const int64_t j = b0 + (e >> 2) * kThreads + tid;
+            if (j < nvec && orderable(f[e]) >= thr) mask |= 1ull << e;
+        }
+        const uint32_t mine = __popcll(mask);
+        uint32_t incl = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+        if (total == 0) continue;
+        uint32_t base = 0;
+        if (lane == 31) base = atomicAdd(cnt, total);
+        uint32_t slot = __shfl_sync(0xffffffffu, base, 31) + incl - mine;
+#pragma unroll
+        for (int e = 0; e < 4 * kU; ++e) {
+            if (mask & (1ull << e)) {
+                const int64_t i = lo_v + 4 * (b0 + (e >> 2) * kThreads + tid) + (e & 3);
+                if (slot < cap) buf[slot] = composite(f[e], i);
+                ++slot;
+            }
         }
     }
-    sort_and_write(s_sel, kk, k, idx + (int64_t)row * k, top ? top + (int64_t)row * k : nullptr, s_x);
+    append_if(sh, ih, inh, thr, buf, cap, cnt);
+    append_if(stl, it, intl, thr, buf, cap, cnt);
+}
+
+__device__ __forceinline__ void cluster_arrive_release() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+constexpr int kFilterLoads = 4;   // 16-byte filter loads in flight per thread
+
+__global__ void __launch_bounds__(kThreads, 2) topk_kernel(RowSpec R, int k, int32_t* idx, float* top) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    uint64_t* cand = reinterpret_cast<uint64_t*>(smem_raw);
+    uint64_t* scratch = reinterpret_cast<uint64_t*>(smem_raw + kCandBytes);
+    __shared__ SelShared sh;
+    __shared__ BinShared bs;
+    __shared__ uint32_t s_cnt, s_total, s_base;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int G = (int)cluster.num_blocks();
+    const int g = (int)cluster.block_rank();
+    const int row = blockIdx.x / G;
+    const int tid = threadIdx.x;
+    const int64_t n = R.count(row);
+    const float* srow = R.scores + (int64_t)row * R.ld;
+    int32_t* idx_row = idx + (int64_t)row * k;
+    float* score_row = top ? top + (int64_t)row * k : nullptr;
+    const int kk = (int)(n < k ? n : k);
+
+    if (n <= kCap) {   // the same branch for every CTA of the cluster
+        if (g != 0) return;
+        for (int64_t i = tid; i < n; i += kThreads) cand[i] = composite(srow[i], i);
+        __syncthreads();
+        select_exact(SmemSrc{cand}, n, k, idx_row, score_row, scratch, sh, bs);
+        return;
+    }
+
+    // ---- threshold from the sample (identical in every CTA of the cluster)
+    if (tid == 0) { s_cnt = 0; s_total = 0; }
+    // CTA 0's total must be zero before any CTA of the cluster adds to it:
+    // arrive here, wait just before the first addition
+    if (G > 1) cluster_arrive_release();
+    const double mu = (double)k * kSample / (double)n;
+    int r = (int)(mu + 4.0 * sqrt(mu) + 4.0);
+    if (r > kSample) r = kSample;
+    const uint32_t thr = sample_threshold(srow, n, r, bs);
+
+    // ---- this CTA's slice: keep every score that reaches it
+    const int64_t lo = n * g / G, hi = n * (g + 1) / G;
+    if (G == 1) {
+        filter_slice<kFilterLoads>(srow, lo, hi, thr, cand, kCap, &s_cnt);
+        __syncthreads();
+    } else {
+        // CTA 0 filters into its scratch area; every CTA then reserves a
+        // range of CTA 0's candidate array with one remote addition and
+        // stores its candidates there over distributed shared memory
+        uint64_t* buf = g == 0 ? scratch : cand;
+        const uint32_t cap = g == 0 ? (uint32_t)kBucketMax : (uint32_t)kCap;
+        filter_slice<kFilterLoads>(srow, lo, hi, thr, buf, cap, &s_cnt);
+        __syncthreads();
+        const uint32_t mine = s_cnt;
+        cluster_wait_acquire();
+        if (tid == 0) {
+            // a CTA that dropped candidates forces the exact fallback
+            const uint32_t add = mine <= cap ? mine : (uint32_t)kCap + 1u;
+            s_base = add ? atomicAdd(cluster.map_shared_rank(&s_total, 0), add) : 0u;
+        }
+        __syncthreads();
+        const uint32_t base = s_base;
+        uint64_t* dst = cluster.map_shared_rank(cand, 0);
+        if (mine <= cap)
+            for (uint32_t j = tid; j < mine && base + j < (uint32_t)kCap; j += kThreads) dst[base + j] = buf[j];
+        cluster.sync();   // every CTA's candidates are in CTA 0
+        if (g != 0) return;
+    }
+    const uint32_t c = G == 1 ? s_cnt : s_total;
+    if (c >= (uint32_t)kk && c <= (uint32_t)kCap)
+        select_exact(SmemSrc{cand}, (int64_t)c, k, idx_row, score_row, scratch, sh, bs);
+    else
+        select_exact(RowSrc{srow}, n, k, idx_row, score_row, scratch, sh, bs);   // the estimate missed
 }
 
 // ---------------------------------------------------------------- host side
 
-static int candidate_cap(int k) {
-    int cap = 8 * k;
-    if (cap > kSegMax) cap = kSegMax;
-    return cap;
-}
-
 size_t topk_workspace_bytes(int nq, int64_t ncols, int k) {
-    if (ncols <= kSegMax) return 0;
-    return align256((size_t)nq * candidate_cap(k) * sizeof(uint64_t)) + align256((size_t)nq * 2 * sizeof(uint32_t));
+    (void)nq;
+    (void)ncols;
+    (void)k;
+    return 0;
 }
 
-static cudaError_t topk_run(const RowSpec& R, int nq, int k, int32_t* idx, float* top, void* ws, cudaStream_t st) {
-    if (nq == 0) return cudaSuccess;
-    const size_t smem = (size_t)kSegMax * sizeof(uint64_t);
-    cudaError_t e;
-    if (R.ncols <= kSegMax) {
-        e = cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        const size_t need = (size_t)(R.ncols > 0 ? R.ncols : 1) * sizeof(uint64_t);
-        CSA_LAUNCH(st, "topk_select", topk_rows_kernel<<<nq, kThreads, need, st>>>(R, k, idx, top));
-        return cudaGetLastError();
+static int sm_count() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
     }
-    const int cap = candidate_cap(k);
-    uint64_t* cand = (uint64_t*)ws;
-    uint32_t* cnt = (uint32_t*)((char*)ws + align256((size_t)nq * cap * sizeof(uint64_t)));
-    uint32_t* thr = cnt + nq;
-    e = cudaMemsetAsync(cnt, 0, (size_t)nq * sizeof(uint32_t), st);
+    return n;
+}
+
+static cudaError_t topk_run(const RowSpec& R, int nq, int k, int32_t* idx, float* top, cudaStream_t st) {
+    if (nq == 0) return cudaSuccess;
+    // CTAs per row: enough to give long rows most of the SMs when rows are few
+    int G = 1;
+    if (R.ncols > kCap)
+        while (G < kMaxCluster && (int64_t)nq * G * 2 <= sm_count()) G <<= 1;
+    const bool spread = (int64_t)nq * G <= sm_count();
+    auto kern = topk_kernel;
+    const size_t smem = spread ? kSmemSpread : kSmemBytes;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    CSA_LAUNCH(st, "topk_threshold", topk_threshold_kernel<<<nq, kThrThreads, 0, st>>>(R, k, thr));
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    const int slices = (int)((R.ncols + kSlice - 1) / kSlice);
-    CSA_LAUNCH(st, "topk_filter", topk_filter_kernel<<<dim3(slices, nq), kThreads, 0, st>>>(R, thr, cand, cap, cnt));
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(topk_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    CSA_LAUNCH(st, "topk_select", topk_final_kernel<<<nq, kThreads, smem, st>>>(R, k, cand, cap, cnt, idx, top));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)nq * G);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)G;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t le = cudaSuccess;
+    CSA_LAUNCH(st, "topk_select", le = cudaLaunchKernelEx(&cfg, kern, R, k, idx, top));
+    if (le != cudaSuccess) return le;
     return cudaGetLastError();
 }
 
 cudaError_t topk_select(const float* scores, int64_t ld, const int32_t* valid, int valid_div, int nq, int64_t ncols,
                         int k, int32_t* idx, float* top_scores, void* ws, cudaStream_t st) {
+    (void)ws;
     RowSpec R{scores, ld, valid, valid_div, 0, 0, ncols};
-    return topk_run(R, nq, k, idx, top_scores, ws, st);
+    return topk_run(R, nq, k, idx, top_scores, st);
 }
 
 cudaError_t topk_select_positions(const float* scores, int64_t ld, int64_t pos_base, int m, int nq, int64_t ncols,
                                   int k, int32_t* idx, void* ws, cudaStream_t st) {
+    (void)ws;
     RowSpec R{scores, ld, nullptr, m, pos_base, 1, ncols};
-    return topk_run(R, nq, k, idx, nullptr, ws, st);
+    return topk_run(R, nq, k, idx, nullptr, st);
 }
 
 }  // namespace csa

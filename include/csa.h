@@ -158,7 +158,8 @@ int csa_index_scores(const void* qI, const float* w, const void* K, const int32_
  * (score descending, column ascending), padded with -1; top_scores [nq, k]
  * (NULL allowed) gets their scores, -inf in padded slots. Deterministic and
  * bit-exact: equal scores are resolved by the lower column. -0.0 == +0.0.
- * 1 <= k <= CSA_MAX_TOPK. */
+ * 1 <= k <= CSA_MAX_TOPK, nq <= 65535. csa_topk_workspace_size returns 0:
+ * the selection needs no workspace (ws may be NULL). */
 size_t csa_topk_workspace_size(int nq, int64_t ncols, int k);
 int csa_topk_from_scores(const float* scores, int64_t ld, const int32_t* valid, int valid_div,
                          int nq, int64_t ncols, int k, int32_t* idx, float* top_scores, void* ws,
@@ -169,15 +170,10 @@ int csa_topk_from_scores(const float* scores, int64_t ld, const int32_t* valid, 
  * allocation and gives it no workspace, a serving loop that forbids
  * allocation after start-up). The pages have no counterpart: this is a
  * library convenience. Same arguments and exactly the same result as
- * csa_topk_from_scores, minus ws/ws_bytes. The multi-level candidate buffers
- * live in a fixed 8 MiB array in the library's device memory (held on every
- * GPU that loads the library until the process exits): a selection needing
- * more scratch than that (csa_topk_workspace_size > 8 MiB) is rejected with
- * CSA_ERR_UNSUPPORTED. All calls share the array: calls that may run at the
- * same time on the GPU race on it and must be serialized by the caller. The
- * first call on each device (with that device current) looks up the
- * array's address; make it before any stream capture begins. No cudaMalloc,
- * cudaFree or other allocating call is made. */
+ * csa_topk_from_scores, minus ws/ws_bytes; nq <= 65535. The selection keeps
+ * all of its scratch in on-chip shared memory: no cudaMalloc, cudaFree or
+ * other allocating call is made, no device memory is held between calls, and
+ * calls on different streams share no state. */
 int csa_topk_from_scores_noalloc(const float* scores, int64_t ld, const int32_t* valid, int valid_div, int nq,
                                  int64_t ncols, int k, int32_t* idx, float* top_scores, void* stream);
 

@@ -68,6 +68,8 @@ def test_invalid_arguments_are_rejected_on_the_host():
                               None) == csa.CSA_ERR_UNSUPPORTED
     # more rows than one launch grid holds
     assert L.csa_topk_from_scores(fake, 16, None, 1, 70000, 16, 4, fake, None, None, 0, None) == csa.CSA_ERR_UNSUPPORTED
+    assert L.csa_topk_from_scores_noalloc(fake, 16, None, 1, 70000, 16, 4, fake, None, None) == csa.CSA_ERR_UNSUPPORTED
+    assert b"65535" in L.csa_last_error()
     # missing / short workspace
     need = L.csa_decode_workspace_size(2, 1024, 8, 128, 4, 64, 16, csa.CSA_BF16)
     assert need > 0
@@ -101,10 +103,9 @@ def test_empty_inputs_are_no_ops():
 
 def test_workspace_sizes():
     L = _lib()
-    # rows that fit one CTA need no workspace; longer rows need a candidate
-    # buffer of 8k composites per row plus a counter
+    # the selection keeps its scratch in shared memory at every row length
     assert L.csa_topk_workspace_size(64, 16384, 512) == 0
-    assert L.csa_topk_workspace_size(32, 262144, 1024) >= 32 * 8 * 1024 * 8 + 32 * 4
+    assert L.csa_topk_workspace_size(32, 262144, 1024) == 0
     assert L.csa_decode_workspace_size(64, 32768, 64, 512, 64, 128, 512, csa.CSA_BF16) >= 64 * 32768 * 4
     small = L.csa_prefill_workspace_size(1024, 256, 512, 4, 128, 64, 8, 4, 16, csa.CSA_BF16)
     assert small >= 1024 * 4 * 128 * 4

@@ -144,6 +144,24 @@ def test_topk_valid_div(csa):
     np.testing.assert_array_equal(host(idx), ref)
 
 
+def test_topk_rows_against_a_strided_sample(csa):
+    """Rows built so that a strided sample misjudges them: the sampled
+    positions hold the largest scores (too few candidates reach the estimate)
+    or the smallest (too many). The selection must stay exact."""
+    nq, ncols, k = 4, 50000, 512
+    g = torch.Generator().manual_seed(5)
+    S = torch.rand(nq, ncols, generator=g)
+    for S_pos in (4096, 1024):
+        pos = (torch.arange(S_pos, dtype=torch.int64) * ncols) // S_pos
+        S[0, pos] += 10.0
+        S[1, pos] -= 10.0
+    S[2, ::97] += 10.0            # a regular stride unrelated to the sample's
+    S[3] = torch.round(S[3] * 4) / 4   # heavy ties
+    idx, top = csa.csa_topk_from_scores(S.to(DEV), k)
+    ref = oracle.topk(S.double().numpy(), np.full(nq, ncols, dtype=np.int32), k)
+    np.testing.assert_array_equal(host(idx), ref)
+
+
 # ---------------------------------------------------------------- a4 + a5
 @pytest.mark.parametrize("dtype", MODES)
 def test_index_topk(csa, dtype):

@@ -2,12 +2,12 @@
 
 Some callers cannot allocate device memory when they select entries (a
 plug-in whose host framework owns all device allocations and gives it no
-workspace; a serving loop that forbids allocation after start-up). For them
-the library keeps the selection's scratch in a fixed device array. This
-checks, through the C ABI, that two calls in a row return exactly what the
-workspace-taking csa_topk_from_scores returns (top-k is integer work: the
-comparison is bit-exact), and that a selection too large for the fixed
-array is refused on the host. This file is collected last on purpose.
+workspace; a serving loop that forbids allocation after start-up). The
+selection keeps its scratch in on-chip shared memory. This checks, through
+the C ABI, that calls in a row return exactly what the workspace-taking
+csa_topk_from_scores returns (top-k is integer work: the comparison is
+bit-exact), at row lengths up to 2^20 and k up to the maximum. (Its host-side
+argument checks are in test_abi.py.) This file is collected last on purpose.
 """
 import ctypes
 
@@ -29,9 +29,10 @@ def test_noalloc_topk_equals_workspace_topk_two_calls_in_a_row():
     import compressed_sparse_attention_14_b200 as csa
     g = torch.Generator().manual_seed(2024)
     cases = [
-        # (rows, columns, k, valid divisor): multi-level selections that use the scratch
+        # (rows, columns, k, valid divisor): sampled-threshold rows, short rows
         (32, 262144, 1024, 4),
         (64, 40000, 512, 1),
+        (8, 1 << 20, 2048, 1),
     ]
     for nq, ncols, k, div in cases:
         S = torch.randn(nq, ncols, generator=g)
@@ -46,12 +47,3 @@ def test_noalloc_topk_equals_workspace_topk_two_calls_in_a_row():
         torch.cuda.synchronize()
         assert torch.equal(idx, ref_idx)
         assert torch.equal(top, ref_top)
-
-
-def test_noalloc_topk_refuses_selections_beyond_the_fixed_array():
-    import compressed_sparse_attention_14_b200 as csa
-    nq, ncols, k = 64, 1 << 20, 2048     # 64 rows x 64 segments x 2048 x 8 B: far above 8 MiB
-    fake = 0x10000
-    rc = csa._lib.csa_topk_from_scores_noalloc(fake, ncols, None, 1, nq, ncols, k, fake, None, None)
-    assert rc == csa.CSA_ERR_UNSUPPORTED
-    assert b"fixed" in csa._lib.csa_last_error()
