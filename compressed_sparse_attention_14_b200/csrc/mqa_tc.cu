@@ -26,15 +26,24 @@
 //
 // Warp roles: warp 0 loads (all lanes issue gathers), warp 1 allocates TMEM
 // and one lane issues the MMAs, warps 2-5 run the softmax and the epilogue.
-// Split-KV partials (O, max, sum) go to the workspace and are merged by
-// mqa_combine (fixed split boundaries: deterministic); a single split writes
-// the normalised output directly. Waits are bounded (CSA_ERR_TIMEOUT).
+// A single split writes the normalised output directly. Up to
+// kMaxClusterSplits splits of one query run as one thread-block cluster and
+// merge on chip: each CTA stages its unnormalised O (fp32) in the shared
+// memory its KV tile used, and after a cluster barrier CTA g combines the
+// g-th slice of the head dimension from every split's O over distributed
+// shared memory (fixed order: deterministic). More splits write partials
+// (O, max, sum) to the workspace for mqa_combine. Waits are bounded
+// (CSA_ERR_TIMEOUT).
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
 #include "tmap.h"
 
 namespace csa {
+
+namespace cg = cooperative_groups;
 
 namespace {
 
@@ -43,6 +52,9 @@ constexpr int kE = 128;                 // entries per tile
 constexpr int kMaxDBlocks = 8;          // c <= 512
 constexpr uint32_t kWaitLimit = 1u << 24;
 constexpr float kRescaleLog2 = 8.0f;    // move the reference max past 2^8
+// Splits merged in one cluster: at most 4, since clusters of one-CTA-per-SM
+// blocks larger than that fit fewer at a time than the SMs allow.
+constexpr int kMaxClusterSplits = 4;
 
 struct MqaArgs {
     QueryMap qm;
@@ -56,6 +68,7 @@ struct MqaArgs {
     float scale_log2;
     const float* sink;
     int nsplit;
+    int cluster;              // the splits of a query form one cluster
     int64_t split_len;
     bf16* out;
     float* lse;
@@ -111,6 +124,65 @@ __device__ __forceinline__ bool bar_or_128(bool v) {
 __device__ __forceinline__ void bar_sync_128() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 }  // namespace
+
+// The splits of query t (one cluster, rank = split) merge on chip: after a
+// cluster barrier, CTA `split` combines its slice of the head dimension for
+// every head from all splits' staged O (fp32, [head][dim] where the KV tile
+// was), their reference maxima and sums (log2 domain) and the sink.
+__device__ __noinline__ void cluster_merge(const MqaArgs& a, int t, int h0, int split, float* obuf, float* mref_s,
+                                       float* lsum_s) {
+    __shared__ float coef_s[kMaxClusterSplits][64];
+    cg::cluster_group cl = cg::this_cluster();
+    const int G = a.nsplit;
+    cl.sync();   // every split's obuf, reference max and sum are final
+    const int tid = threadIdx.x;
+    if (tid < 64) {
+        const int h = h0 + tid;
+        // (remote values are re-read instead of kept in indexed arrays,
+        // which would live in local memory)
+        const float sk = (a.sink && h < a.H) ? a.sink[h] * 1.4426950408889634f : -INFINITY;
+        float M = sk;
+        for (int q = 0; q < G; ++q) M = fmaxf(M, cl.map_shared_rank(mref_s, q)[tid]);
+        float L = (sk == -INFINITY) ? 0.f : exp2f(sk - M);
+        for (int q = 0; q < G; ++q) {
+            const float mq = cl.map_shared_rank(mref_s, q)[tid];
+            if (mq != -INFINITY) L += cl.map_shared_rank(lsum_s, q)[tid] * exp2f(mq - M);
+        }
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        for (int q = 0; q < G; ++q) {
+            const float mq = cl.map_shared_rank(mref_s, q)[tid];
+            coef_s[q][tid] = (mq == -INFINITY) ? 0.f : exp2f(mq - M) * inv;
+        }
+        if (split == 0 && a.lse && h < a.H)
+            a.lse[(int64_t)t * a.H + h] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+    }
+    __syncthreads();
+    // this CTA's slice of the head dimension, every head, in units of 4
+    // dims (16-byte aligned, whatever G): sum over the splits in rank order
+    const int n4 = a.c / 4;
+    const int lo4 = split * n4 / G, dn4 = (split + 1) * n4 / G - lo4;
+    for (int e = tid; e < 64 * dn4; e += kThreads) {
+        const int i = e / dn4, dim = 4 * (lo4 + e % dn4);
+        const int h = h0 + i;
+        if (h >= a.H) continue;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int q = 0; q < G; ++q) {
+            const float w = coef_s[q][i];
+            if (w == 0.f) continue;
+            const float4 v = *reinterpret_cast<const float4*>(cl.map_shared_rank(obuf, q) + i * a.c + dim);
+            acc.x = fmaf(w, v.x, acc.x);
+            acc.y = fmaf(w, v.y, acc.y);
+            acc.z = fmaf(w, v.z, acc.z);
+            acc.w = fmaf(w, v.w, acc.w);
+        }
+        __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x, acc.y), hi2 = __floats2bfloat162_rn(acc.z, acc.w);
+        uint2 pk;
+        pk.x = *reinterpret_cast<uint32_t*>(&lo2);
+        pk.y = *reinterpret_cast<uint32_t*>(&hi2);
+        *reinterpret_cast<uint2*>(a.out + ((int64_t)t * a.H + h) * a.c + dim) = pk;
+    }
+    cl.sync();   // the other CTAs' shared memory stays alive until read
+}
 
 __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_constant__ MqaArgs a,
                                                              const __grid_constant__ CUtensorMap tmQ,
@@ -437,7 +509,25 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
         }
         bar_sync_128();
         const bool have_o = ok && ntiles > 0;
-        if (a.nsplit == 1) {
+        if (a.cluster) {
+            // stage this split's O^T as obuf[head][dim] (fp32) where the KV
+            // tile was; the combine after the role branches reads it
+            float* obuf = (float*)kv_s;
+            if (eth < 64 && !have_o) { mref_s[eth] = -INFINITY; lsum_s[eth] = 0.f; }
+            if (have_o) {
+                for (int mt = 0; mt < a.mtiles; ++mt) {
+                    const int dim = mt * 128 + row;
+                    float v[64];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        tc::tmem_ld16(tmem_O + ((uint32_t)(quad * 32) << 16) + mt * hg + 16 * u,
+                                      *reinterpret_cast<float(*)[16]>(v + 16 * u));
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) obuf[i * a.c + dim] = v[i];
+                }
+            }
+        } else if (a.nsplit == 1) {
             // normalise: denominator = sum + sink term (same reference max)
             if (eth < 64) {
                 const int h = h0 + eth;
@@ -506,6 +596,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, a.tmem_cols);
     }
+    if (a.cluster) cluster_merge(a, t, h0, split, (float*)kv_s, mref_s, lsum_s);
 }
 
 bool mqa_tc_supported(int H, int c) { return c % 128 == 0 && c <= 512 && H >= 1; }
@@ -520,6 +611,8 @@ int mqa_tc_nsplit(int nq, int H, int64_t max_entries, int num_sms) {
     if (ns > 64) ns = 64;
     return (int)ns;
 }
+
+bool mqa_tc_cluster(int nsplit) { return nsplit >= 2 && nsplit <= kMaxClusterSplits; }
 
 cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, QuerySpec qs, int mp, int nq, int n_seq,
                    int H, int c, int64_t Nmax, float scale, const float* sink, void* out, float* lse, void* ws,
@@ -540,6 +633,7 @@ cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, Que
     a.scale_log2 = scale * 1.4426950408889634f;
     a.sink = sink;
     a.nsplit = nsplit;
+    a.cluster = mqa_tc_cluster(nsplit) ? 1 : 0;
     const int64_t max_entries = idx ? k : Nmax;
     int64_t per = (max_entries + nsplit - 1) / nsplit;
     a.split_len = ((per + kE - 1) / kE) * kE;
@@ -564,8 +658,21 @@ cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, Que
                         32 * sizeof(uint64_t);
     cudaError_t e = cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(nsplit, (H + a.hg - 1) / a.hg, nq);
-    CSA_LAUNCH(st, "mqa_tc", mqa_tc_kernel<<<grid, kThreads, smem, st>>>(a, tmQ, tmTile));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(nsplit, (H + a.hg - 1) / a.hg, nq);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = a.cluster ? (unsigned)nsplit : 1u;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t le = cudaSuccess;
+    CSA_LAUNCH(st, "mqa_tc", le = cudaLaunchKernelEx(&cfg, mqa_tc_kernel, a, tmQ, tmTile));
+    if (le != cudaSuccess) return le;
     return cudaGetLastError();
 }
 
