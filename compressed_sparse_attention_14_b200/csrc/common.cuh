@@ -16,6 +16,16 @@ __device__ __forceinline__ void report_device_error(int* status, int code) {
     if (status) atomicCAS(status, 0, code);
 }
 
+// ---- programmatic dependent launch
+// Kernels launched with launch_pdl() may start while the previous kernel on
+// the stream drains. pdl_wait() returns once that kernel has completed and
+// its writes are visible (at once when there is none); every CTA calls it
+// before its first global memory access, read or write. pdl_launch_next()
+// lets the next kernel on the stream begin launching once every CTA of this
+// one has called it (or exited).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_next() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---- element conversion -------------------------------------------------
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(bf16 v) { return __bfloat162float(v); }

@@ -43,6 +43,8 @@ __global__ void __launch_bounds__(256) csa_compress_kernel(const TIn* __restrict
                                                            const float* __restrict__ bias,
                                                            int64_t nb, int c, int m,
                                                            TOut* __restrict__ out) {
+    pdl_wait();
+    pdl_launch_next();
     const int groups = c / 8;
     int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (gid >= nb * groups) return;
@@ -88,6 +90,8 @@ __global__ void __launch_bounds__(256) hca_compress_kernel(const TIn* __restrict
                                                            const float* __restrict__ bias,
                                                            int64_t nb, int c, int mp,
                                                            TOut* __restrict__ out) {
+    pdl_wait();
+    pdl_launch_next();
     const int groups = c / 8;
     int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (gid >= nb * groups) return;
@@ -121,8 +125,11 @@ cudaError_t launch_csa_compress(const void* proj, const void* left, const float*
     int64_t nb = n / m;
     int64_t threads = nb * (c / 8);
     if (threads == 0) return cudaSuccess;
-    CSA_LAUNCH(st, "csa_compress", csa_compress_kernel<TIn, TOut><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
-        (const TIn*)proj, (const TIn*)left, bias, nb, c, m, (TOut*)out));
+    cudaError_t e = cudaSuccess;
+    CSA_LAUNCH(st, "csa_compress",
+               e = launch_pdl(csa_compress_kernel<TIn, TOut>, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, st,
+                              0, (const TIn*)proj, (const TIn*)left, bias, nb, c, m, (TOut*)out));
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -132,8 +139,11 @@ cudaError_t launch_hca_compress(const void* proj, const float* bias, int64_t n, 
     int64_t nb = n / mp;
     int64_t threads = nb * (c / 8);
     if (threads == 0) return cudaSuccess;
-    CSA_LAUNCH(st, "hca_compress", hca_compress_kernel<TIn, TOut><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
-        (const TIn*)proj, bias, nb, c, mp, (TOut*)out));
+    cudaError_t e = cudaSuccess;
+    CSA_LAUNCH(st, "hca_compress",
+               e = launch_pdl(hca_compress_kernel<TIn, TOut>, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, st,
+                              0, (const TIn*)proj, bias, nb, c, mp, (TOut*)out));
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -90,6 +90,8 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
     tc::tc_fence_after();
     const uint32_t tmem = s_tmem;
     volatile int* abort_flag = &s_abort;
+    pdl_wait();
+    pdl_launch_next();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -215,7 +217,8 @@ cudaError_t project_tc(const void* x, const void* W, int64_t n, int d, int M, fl
     if (e != cudaSuccess) return e;
     const int ntiles = a.tiles_m * a.tiles_n;
     const int grid = ntiles < sm_count() ? ntiles : sm_count();
-    CSA_LAUNCH(st, "project_tc", project_tc_kernel<<<grid, kThreads, smem, st>>>(a, tmX, tmW));
+    CSA_LAUNCH(st, "project_tc", e = launch_pdl(project_tc_kernel, dim3(grid), dim3(kThreads), smem, st, 0, a, tmX, tmW));
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -200,6 +200,8 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = s_tmem;
+    pdl_wait();
+    pdl_launch_next();
 
     // this CTA's share of the work list
     const int64_t T = total_tiles(a, ngroups, lane);
@@ -382,6 +384,8 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
 // matrix is complete; the fused paths skip it (top-k reads only visible ones).
 __global__ void fill_invisible_kernel(float* scores, int64_t ld, QueryMap qm, int nq, int n_seq, int64_t Nmax,
                                       int m) {
+    pdl_wait();
+    pdl_launch_next();
     const int t = blockIdx.x;
     int s = qm.seq_of(t);
     int64_t vis = (s >= 0 && s < n_seq) ? visible_entries(qm.pos_of(t), m, Nmax) : 0;
@@ -453,13 +457,16 @@ cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, Query
     if (fill_invisible) {
         QueryMap qm = a.qm;
         CSA_LAUNCH(st, "index_fill_invisible",
-                   fill_invisible_kernel<<<dim3(nq, 8), 256, 0, st>>>(scores, ld, qm, nq, n_seq, Nmax, m));
-        e = cudaGetLastError();
+                   e = launch_pdl(fill_invisible_kernel, dim3(nq, 8), dim3(256), 0, st, 0, scores, ld, qm, nq, n_seq,
+                                  Nmax, m));
+        if (e == cudaSuccess) e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     e = cudaFuncSetAttribute(index_scores_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    CSA_LAUNCH(st, "index_scores_tc", index_scores_tc_kernel<<<num_sms(), kThreads, smem, st>>>(a, tmK, tmQ));
+    CSA_LAUNCH(st, "index_scores_tc",
+               e = launch_pdl(index_scores_tc_kernel, dim3(num_sms()), dim3(kThreads), smem, st, 0, a, tmK, tmQ));
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

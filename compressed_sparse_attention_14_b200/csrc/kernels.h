@@ -26,6 +26,34 @@ int trace_read(int max_kernels, char* names, double* total_ms, int* counts, int*
         ::csa::trace_end(_csa_tok, st, name);      \
     } while (0)
 
+// Launch `kern` with programmatic dependent launch allowed (the kernel must
+// call pdl_wait() before touching global memory) and, when cluster_x > 0,
+// as clusters of cluster_x CTAs along x.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       unsigned cluster_x, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    unsigned n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (cluster_x > 0) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster_x;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 inline size_t elem_size(ElemType t) { return t == ElemType::BF16 ? 2 : 4; }
 inline size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
 

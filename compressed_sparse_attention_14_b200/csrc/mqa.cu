@@ -159,6 +159,8 @@ __global__ void __launch_bounds__(128) mqa_combine_kernel(const float* __restric
                                                           int nsplit, int H, int c,
                                                           const float* __restrict__ sink,
                                                           T* __restrict__ out, float* __restrict__ lse) {
+    pdl_wait();
+    pdl_launch_next();
     __shared__ float s_w[64];
     __shared__ float s_inv;
     const int t = blockIdx.y, h = blockIdx.x;
@@ -245,8 +247,10 @@ cudaError_t mqa(const void* q, const void* KV, const int32_t* idx, int k, QueryS
         if (e != cudaSuccess || ns == 1 || mqa_tc_cluster(ns)) return e;
         float* part_o = (float*)ws;
         float* part_ml = (float*)((char*)ws + align256((size_t)nq * ns * H * c * sizeof(float)));
-        CSA_LAUNCH(st, "mqa_combine", mqa_combine_kernel<bf16><<<dim3(H, nq), 128, 0, st>>>(
-                                          part_o, part_ml, ns, H, c, sink, (bf16*)out, lse));
+        CSA_LAUNCH(st, "mqa_combine",
+                   e = launch_pdl(mqa_combine_kernel<bf16>, dim3(H, nq), dim3(128), 0, st, 0, (const float*)part_o,
+                                  (const float*)part_ml, ns, H, c, sink, (bf16*)out, lse));
+        if (e != cudaSuccess) return e;
         return cudaGetLastError();
     }
     const int ns = mqa_nsplit(nq, H, max_entries);

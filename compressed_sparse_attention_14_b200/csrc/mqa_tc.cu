@@ -208,6 +208,8 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
 
+    pdl_wait();
+    pdl_launch_next();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = blockIdx.z;
     const int h0 = blockIdx.y * a.hg;
@@ -658,20 +660,10 @@ cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, Que
                         32 * sizeof(uint64_t);
     cudaError_t e = cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(nsplit, (H + a.hg - 1) / a.hg, nq);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = a.cluster ? (unsigned)nsplit : 1u;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     cudaError_t le = cudaSuccess;
-    CSA_LAUNCH(st, "mqa_tc", le = cudaLaunchKernelEx(&cfg, mqa_tc_kernel, a, tmQ, tmTile));
+    CSA_LAUNCH(st, "mqa_tc",
+               le = launch_pdl(mqa_tc_kernel, dim3(nsplit, (H + a.hg - 1) / a.hg, nq), dim3(kThreads), smem, st,
+                               a.cluster ? (unsigned)nsplit : 0u, a, tmQ, tmTile));
     if (le != cudaSuccess) return le;
     return cudaGetLastError();
 }

@@ -547,6 +547,8 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(RowSpec R, int k, int
     __shared__ SelShared sh;
     __shared__ BinShared bs;
     __shared__ uint32_t s_cnt, s_total, s_base;
+    pdl_wait();
+    pdl_launch_next();
     cg::cluster_group cluster = cg::this_cluster();
     const int G = (int)cluster.num_blocks();
     const int g = (int)cluster.block_rank();
@@ -641,20 +643,9 @@ static cudaError_t topk_run(const RowSpec& R, int nq, int k, int32_t* idx, float
     const size_t smem = spread ? kSmemSpread : kSmemBytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)nq * G);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)G;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     cudaError_t le = cudaSuccess;
-    CSA_LAUNCH(st, "topk_select", le = cudaLaunchKernelEx(&cfg, kern, R, k, idx, top));
+    CSA_LAUNCH(st, "topk_select",
+               le = launch_pdl(kern, dim3((unsigned)nq * G), dim3(kThreads), smem, st, (unsigned)G, R, k, idx, top));
     if (le != cudaSuccess) return le;
     return cudaGetLastError();
 }
