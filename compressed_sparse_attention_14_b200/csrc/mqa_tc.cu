@@ -76,6 +76,7 @@ struct MqaArgs {
     float* part_ml;
     int* status;
     int dblocks, mtiles;
+    int ring;                 // dense: 32 KB slots (a pair of 64-dim blocks) in the KV ring; 0 for sparse
     uint32_t tmem_cols, q_bytes;
 };
 
@@ -190,7 +191,10 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t* kv_s = base;                                        // dblocks x 16 KB
-    uint8_t* q_s = kv_s + (size_t)a.dblocks * kE * 128;          // dblocks x hg*128
+    // KV area: sparse, one tile (dblocks x 16 KB); dense, a ring of `ring`
+    // 32 KB slots
+    const size_t kv_bytes = a.ring ? (size_t)a.ring * 2 * kE * 128 : (size_t)a.dblocks * kE * 128;
+    uint8_t* q_s = kv_s + kv_bytes;                              // dblocks x hg*128
     uint8_t* p_s = q_s + a.q_bytes;                              // 128 x 128 B
     float* mref_s = (float*)(p_s + kE * 128);                    // [64]
     float* alpha_s = mref_s + 64;                                // [64]
@@ -304,26 +308,38 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
                         break;
                     }
                 }
-            } else {
-                for (; j < ntiles; ++j) {
-                    bool ok = true;
-                    if (lane == 0) {
-                        for (int b = 0; b < a.dblocks && ok; ++b) {
-                            if (j > 0) ok = wait_or_abort(&kv_empty[b], (j - 1) & 1, abort_flag, a.status);
-                            if (ok) tc::mbar_expect_tx(&kv_full[b], kE * 128);
+            } else if (lane == 0) {
+                // Dense rows stream through the ring twice per tile, pair
+                // by pair of 64-dim blocks: for the first product (S) and
+                // again, from L2, for the second (O). Order S(0), then
+                // S(j), O(j-1) for j >= 1, then O(n-1): the HBM read of
+                // tile j+1 overlaps the softmax of tile j.
+                uint32_t cnt = 0;
+                bool ok = true;
+                for (int step = 0; ok && step <= ntiles; ++step) {
+                    for (int pass = 0; ok && pass < 2; ++pass) {
+                        const int jt = pass == 0 ? step : step - 1;   // S pass of tile step, O pass of step-1
+                        if (jt < 0 || jt >= ntiles) continue;
+                        const int row = (int)(row0 + e_beg + (int64_t)jt * kE);
+                        for (int mt = 0; mt < a.mtiles; ++mt, ++cnt) {
+                            const int slot = (int)(cnt % (uint32_t)a.ring);
+                            if (cnt >= (uint32_t)a.ring &&
+                                !(ok = wait_or_abort(&kv_empty[slot], ((cnt / a.ring) - 1) & 1, abort_flag, a.status)))
+                                break;
+                            uint8_t* dst = kv_s + (size_t)slot * 2 * kE * 128;
+                            tc::mbar_expect_tx(&kv_full[slot], 2 * kE * 128);
+                            tc::tma_load_2d(dst, &tmTile, &kv_full[slot], 2 * mt * 64, row);
+                            tc::tma_load_2d(dst + kE * 128, &tmTile, &kv_full[slot], (2 * mt + 1) * 64, row);
                         }
                     }
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
-                    if (!ok) break;
-                    const int64_t e0 = e_beg + (int64_t)j * kE;
-                    if (lane == 0)
-                        for (int b = 0; b < a.dblocks; ++b)
-                            tc::tma_load_2d(kv_s + (size_t)b * kE * 128, &tmTile, &kv_full[b], b * 64,
-                                            (int)(row0 + e0));
                 }
+                // drain: the copies still in flight must land
+                for (uint32_t i = cnt > (uint32_t)a.ring ? cnt - a.ring : 0; i < cnt; ++i)
+                    tc::mbar_wait(&kv_full[i % a.ring], (i / a.ring) & 1, kWaitLimit);
+                j = 0;
             }
-            // drain: the last issued tile and q must have landed
-            if (lane == 0 && j > 0)
+            // drain (sparse): the last issued tile and q must have landed
+            if (a.idx && lane == 0 && j > 0)
                 for (int b = 0; b < a.dblocks; ++b) tc::mbar_wait(&kv_full[b], (j - 1) & 1, kWaitLimit);
             if (lane == 0) tc::mbar_wait(q_full, 0, kWaitLimit);
         }
@@ -337,6 +353,52 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
             const uint32_t p_addr = tc::smem_u32(p_s);
             bool ok = wait_or_abort(q_full, 0, abort_flag, a.status);
             int j = 0;
+            if (!a.idx) {
+                // dense: the ring order of the producer, pair by pair
+                uint32_t cnt = 0;
+                for (int step = 0; ok && step <= ntiles; ++step) {
+                    for (int pass = 0; ok && pass < 2; ++pass) {
+                        const int jt = pass == 0 ? step : step - 1;
+                        if (jt < 0 || jt >= ntiles) continue;
+                        const int sb = jt & 1;
+                        if (pass == 0) {
+                            if (jt >= 2 && !(ok = wait_or_abort(&s_empty[sb], ((jt >> 1) - 1) & 1, abort_flag,
+                                                               a.status)))
+                                break;
+                        } else {
+                            if (!(ok = wait_or_abort(p_full, jt & 1, abort_flag, a.status))) break;
+                            tc::tc_fence_after();
+                        }
+                        for (int mt = 0; mt < a.mtiles; ++mt, ++cnt) {
+                            const int slot = (int)(cnt % (uint32_t)a.ring);
+                            if (!(ok = wait_or_abort(&kv_full[slot], (cnt / a.ring) & 1, abort_flag, a.status))) break;
+                            tc::tc_fence_after();
+                            const uint32_t sa = kv_addr + (uint32_t)slot * 2 * kE * 128;
+                            if (pass == 0) {
+                                // S^T += KV[:, blocks 2mt, 2mt+1] . q[:, same]^T
+                                for (int bb = 0; bb < 2; ++bb)
+                                    for (int kk = 0; kk < 4; ++kk) {
+                                        uint64_t ad = tc::sdesc_sw128(sa + bb * (kE * 128) + kk * 32, 16, 1024);
+                                        uint64_t bd = tc::sdesc_sw128(q_addr + (2 * mt + bb) * (a.hg * 128) + kk * 32,
+                                                                      16, 1024);
+                                        tc::umma_bf16(tmem_S + sb * a.hg, ad, bd, idesc1, (mt | bb | kk) ? 1u : 0u);
+                                    }
+                            } else {
+                                // O^T[dims of mt] += KV^T . P^T
+                                for (int ke = 0; ke < kE / 16; ++ke) {
+                                    uint64_t ad = tc::sdesc_sw128(sa + ke * 2048, kE * 128, 1024);
+                                    uint64_t bd = tc::sdesc_sw128(p_addr + ke * 2048, kE * 128, 1024);
+                                    tc::umma_bf16(tmem_O + mt * a.hg, ad, bd, idesc2, (jt > 0 || ke > 0) ? 1u : 0u);
+                                }
+                            }
+                            tc::umma_commit(&kv_empty[slot]);
+                        }
+                        if (!ok) break;
+                        tc::umma_commit(pass == 0 ? &s_full[sb] : o_done);
+                    }
+                }
+                j = ntiles;   // skip the sparse loop below
+            }
             for (; ok && j < ntiles; ++j) {
                 const int sb = j & 1;
                 if (j >= 2 && !(ok = wait_or_abort(&s_empty[sb], ((j >> 1) - 1) & 1, abort_flag, a.status))) break;
@@ -656,8 +718,19 @@ cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, Que
     if (!make_tmap_bf16_2d(&tmQ, q, (uint64_t)nq * H, c, c, a.hg, 64)) return cudaErrorInvalidValue;
     if (!make_tmap_bf16_2d(&tmTile, KV, (uint64_t)n_seq * Nmax, c, c, kE, 64)) return cudaErrorInvalidValue;
 
-    const size_t smem = 1024 + (size_t)a.dblocks * kE * 128 + a.q_bytes + kE * 128 + (64 * 4 + 256) * sizeof(float) +
-                        32 * sizeof(uint64_t);
+    const size_t fixed = 1024 + a.q_bytes + kE * 128 + (64 * 4 + 256) * sizeof(float) + 32 * sizeof(uint64_t);
+    size_t kv_bytes = (size_t)a.dblocks * kE * 128;
+    if (!idx) {
+        // dense ring: as many 32 KB slots as fit (at most 8, at least the
+        // KV tile's size so the staging areas that reuse it still fit)
+        // (4 KB left for the kernel's static shared memory)
+        int ring = (int)((223 * 1024 - fixed) / (2 * kE * 128));
+        if (ring > kMaxDBlocks) ring = kMaxDBlocks;
+        if (ring < a.mtiles) ring = a.mtiles;
+        a.ring = ring;
+        kv_bytes = (size_t)ring * 2 * kE * 128;
+    }
+    const size_t smem = fixed + kv_bytes;
     cudaError_t e = cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaError_t le = cudaSuccess;

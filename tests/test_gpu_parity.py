@@ -198,6 +198,44 @@ def test_sparse_mqa(csa, dtype, H, c, k, with_sink):
     assert_close(lse, ref_l, torch.float32 if dtype == torch.float32 else dtype, "sparse_mqa lse")
 
 
+# (kind, queries, head dim, heads, k or visible entries): query counts chosen
+# so that the KV of one query is split 3 ways (merged in a thread-block
+# cluster; 3 does not divide c/4, so the merge slices are uneven), or 7 ways
+# (partials merged by the separate combine launch), with one and two head
+# groups
+SPLIT_CASES = [
+    ("sparse", 40, 512, 64, 512),
+    ("sparse", 40, 128, 64, 384),
+    ("sparse", 24, 512, 128, 512),
+    ("sparse", 20, 256, 64, 1024),
+    ("dense", 40, 512, 64, 700),
+    ("dense", 20, 128, 64, 1100),
+]
+
+
+@pytest.mark.parametrize("kind,nq,c,H,kv", SPLIT_CASES)
+def test_mqa_split_merges(csa, kind, nq, c, H, kv):
+    B, Nmax = 4, 1200
+    q_h, q = _g((nq, H, c), "qs", torch.bfloat16)
+    KV_h, KV = _g((B, Nmax, c), "KVs", torch.bfloat16)
+    seq_h = (torch.arange(nq, dtype=torch.int32) % B)
+    sink_h = synth.normal((H,), 4, "sink_s", dtype=torch.float32)
+    if kind == "sparse":
+        g = torch.Generator().manual_seed(9)
+        idx_h = torch.stack([torch.randperm(Nmax, generator=g)[:kv] for _ in range(nq)]).to(torch.int32)
+        idx_h[3, kv // 2:] = -1         # one split of this query sees nothing
+        out, lse = csa.csa_sparse_mqa(q, KV, idx_h.to(DEV), 0.0, sink=sink_h.to(DEV), seq_of_q=seq_h.to(DEV))
+        ref_o, ref_l = oracle.sparse_mqa(q_h, KV_h, idx_h, 1 / math.sqrt(c), sink=sink_h, seq=seq_h)
+    else:
+        mp = 4
+        pos_h = torch.full((nq,), kv * mp + 1, dtype=torch.int32)
+        pos_h[1] = 5 * mp               # few visible entries: most splits empty
+        out, lse = csa.hca_dense_mqa(q, KV, pos_h.to(DEV), mp, 0.0, sink=sink_h.to(DEV), seq_of_q=seq_h.to(DEV))
+        ref_o, ref_l = oracle.dense_mqa(q_h, KV_h, pos_h, mp, 1 / math.sqrt(c), sink=sink_h, seq=seq_h)
+    assert_close(out, ref_o, torch.bfloat16, f"{kind} split out")
+    assert_close(lse, ref_l, torch.bfloat16, f"{kind} split lse")
+
+
 @pytest.mark.parametrize("dtype", MODES)
 def test_dense_mqa(csa, dtype):
     nq, H, c, Nmax, mp = 4, 64, 512, 700, 128
