@@ -347,10 +347,15 @@ def hca_compress_workload(rank):
                             l2="inputs larger than L2 and flushed before every timed step"))
 
 
-def prefill_workload(rank):
+def prefill_workload(rank, tokens=None):
     import compressed_sparse_attention_14_b200 as csa
     s = dataclass_seed(synth.PREFILL, rank)
-    inp = synth.prefill_inputs(s, device="cuda")
+    if tokens is None:
+        inp = synth.prefill_inputs(s, device="cuda")
+    else:
+        # the last `tokens` tokens of the chunk: same positions and context
+        # (a small profiling case)
+        inp = synth.prefill_inputs(s, device="cuda", n=tokens, start=s.start + s.n - tokens)
     n = inp["n"]
     Nmax = inp["kv_cache"].shape[0]
     out = torch.empty_like(inp["q"])
@@ -395,7 +400,7 @@ WORKLOADS = {
     "pro_decode": lambda r, b=None: decode_workload(synth.PRO_DECODE, r, b),
     "hca_decode": lambda r, b=None: hca_decode_workload(r),
     "hca_compress": lambda r, b=None: hca_compress_workload(r),
-    "prefill": lambda r, b=None: prefill_workload(r),
+    "prefill": lambda r, b=None: prefill_workload(r, b),
 }
 
 
@@ -669,7 +674,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
     ap.add_argument("--batch", type=int, default=None,
-                    help="decode workloads: use only the first N queries (small profiling cases)")
+                    help="decode workloads: only the first N queries; prefill: only the last N tokens of the "
+                         "chunk, a multiple of m (small profiling cases)")
     args = ap.parse_args()
     rank, world, local = dist_init()
     if world != args.gpus and rank == 0:
