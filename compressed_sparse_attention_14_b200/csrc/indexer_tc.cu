@@ -154,6 +154,22 @@ struct Walk {
     __device__ bool last_of_group() const { return t + 1 == tiles_g; }
 };
 
+// Paired fp32: two values in one 64-bit register; d = a * b + c lane by
+// lane, round to nearest (sm_100 packed FMA).
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+    return d;
+}
+__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                               int* status) {
     for (uint32_t i = 0; i < kWaitLimit; ++i) {
@@ -341,15 +357,20 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
                 for (int u = 0; u < 4; ++u) {
                     const int cc = c0 + 16 * u;
                     if (cc < a.npad) {
-                        float p4[4] = {0.f, 0.f, 0.f, 0.f};
+                        // four independent partial sums, two per paired fp32
+                        // FMA (each lane rounds as a separate fmaf would)
+                        uint64_t p01 = 0, p23 = 0;
 #pragma unroll
                         for (int i = 0; i < 16; i += 4) {
                             const float4 w4 = *reinterpret_cast<const float4*>(wv + cc + i);
-                            p4[0] = fmaf(w4.x, fmaxf(v[16 * u + i], 0.f), p4[0]);
-                            p4[1] = fmaf(w4.y, fmaxf(v[16 * u + i + 1], 0.f), p4[1]);
-                            p4[2] = fmaf(w4.z, fmaxf(v[16 * u + i + 2], 0.f), p4[2]);
-                            p4[3] = fmaf(w4.w, fmaxf(v[16 * u + i + 3], 0.f), p4[3]);
+                            p01 = fma2(pack2(w4.x, w4.y),
+                                       pack2(fmaxf(v[16 * u + i], 0.f), fmaxf(v[16 * u + i + 1], 0.f)), p01);
+                            p23 = fma2(pack2(w4.z, w4.w),
+                                       pack2(fmaxf(v[16 * u + i + 2], 0.f), fmaxf(v[16 * u + i + 3], 0.f)), p23);
                         }
+                        float p4[4];
+                        unpack2(p01, p4[0], p4[1]);
+                        unpack2(p23, p4[2], p4[3]);
                         const float part = (p4[0] + p4[1]) + (p4[2] + p4[3]);
                         const int gq = (a.group > 1) ? cc / a.HI : 0;
                         if (gq == 0) sc[0] += part;
