@@ -130,18 +130,20 @@ __device__ __forceinline__ void bar_sync_128() { asm volatile("bar.sync 1, 128;"
 // cluster barrier, CTA `split` combines its slice of the head dimension for
 // every head from all splits' staged O (fp32, [head][dim] where the KV tile
 // was), their reference maxima and sums (log2 domain) and the sink.
-__device__ __noinline__ void cluster_merge(const MqaArgs& a, int t, int h0, int split, float* obuf, float* mref_s,
-                                       float* lsum_s) {
+// (The launch parameters come in by value: read through a pointer to the
+// kernel's parameter block inside this out-of-line function, every access
+// would be a slow generic load.)
+__device__ __noinline__ void cluster_merge(int G, int c, int H, const float* sink, float* lse_out, bf16* out, int t,
+                                           int h0, int split, float* obuf, float* mref_s, float* lsum_s) {
     __shared__ float coef_s[kMaxClusterSplits][64];
     cg::cluster_group cl = cg::this_cluster();
-    const int G = a.nsplit;
     cl.sync();   // every split's obuf, reference max and sum are final
     const int tid = threadIdx.x;
     if (tid < 64) {
         const int h = h0 + tid;
         // (remote values are re-read instead of kept in indexed arrays,
         // which would live in local memory)
-        const float sk = (a.sink && h < a.H) ? a.sink[h] * 1.4426950408889634f : -INFINITY;
+        const float sk = (sink && h < H) ? sink[h] * 1.4426950408889634f : -INFINITY;
         float M = sk;
         for (int q = 0; q < G; ++q) M = fmaxf(M, cl.map_shared_rank(mref_s, q)[tid]);
         float L = (sk == -INFINITY) ? 0.f : exp2f(sk - M);
@@ -154,33 +156,43 @@ __device__ __noinline__ void cluster_merge(const MqaArgs& a, int t, int h0, int 
             const float mq = cl.map_shared_rank(mref_s, q)[tid];
             coef_s[q][tid] = (mq == -INFINITY) ? 0.f : exp2f(mq - M) * inv;
         }
-        if (split == 0 && a.lse && h < a.H)
-            a.lse[(int64_t)t * a.H + h] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+        if (split == 0 && lse_out && h < H)
+            lse_out[(int64_t)t * H + h] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
     }
     __syncthreads();
     // this CTA's slice of the head dimension, every head, in units of 4
     // dims (16-byte aligned, whatever G): sum over the splits in rank order
-    const int n4 = a.c / 4;
+    const int n4 = c / 4;
     const int lo4 = split * n4 / G, dn4 = (split + 1) * n4 / G - lo4;
-    for (int e = tid; e < 64 * dn4; e += kThreads) {
-        const int i = e / dn4, dim = 4 * (lo4 + e % dn4);
+    // warp w takes heads w, w + 6, ...; its lanes walk the slice's 4-dim
+    // chunks (no division in the loop)
+    const int nh = H - h0 < 64 ? H - h0 : 64;
+    for (int i = tid >> 5; i < nh; i += kThreads / 32) {
         const int h = h0 + i;
-        if (h >= a.H) continue;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int q = 0; q < G; ++q) {
-            const float w = coef_s[q][i];
-            if (w == 0.f) continue;
-            const float4 v = *reinterpret_cast<const float4*>(cl.map_shared_rank(obuf, q) + i * a.c + dim);
-            acc.x = fmaf(w, v.x, acc.x);
-            acc.y = fmaf(w, v.y, acc.y);
-            acc.z = fmaf(w, v.z, acc.z);
-            acc.w = fmaf(w, v.w, acc.w);
+        float w[kMaxClusterSplits];
+#pragma unroll
+        for (int q = 0; q < kMaxClusterSplits; ++q) w[q] = q < G ? coef_s[q][i] : 0.f;
+        for (int j = tid & 31; j < dn4; j += 32) {
+            const int dim = 4 * (lo4 + j);
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int q = 0; q < kMaxClusterSplits; ++q) {
+                if (w[q] == 0.f) continue;   // also every q >= G
+                // this CTA's own split is read from its shared memory
+                // directly, the others' over distributed shared memory
+                const float* src = q == split ? obuf : cl.map_shared_rank(obuf, q);
+                const float4 v = *reinterpret_cast<const float4*>(src + i * c + dim);
+                acc.x = fmaf(w[q], v.x, acc.x);
+                acc.y = fmaf(w[q], v.y, acc.y);
+                acc.z = fmaf(w[q], v.z, acc.z);
+                acc.w = fmaf(w[q], v.w, acc.w);
+            }
+            __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x, acc.y), hi2 = __floats2bfloat162_rn(acc.z, acc.w);
+            uint2 pk;
+            pk.x = *reinterpret_cast<uint32_t*>(&lo2);
+            pk.y = *reinterpret_cast<uint32_t*>(&hi2);
+            *reinterpret_cast<uint2*>(out + ((int64_t)t * H + h) * c + dim) = pk;
         }
-        __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x, acc.y), hi2 = __floats2bfloat162_rn(acc.z, acc.w);
-        uint2 pk;
-        pk.x = *reinterpret_cast<uint32_t*>(&lo2);
-        pk.y = *reinterpret_cast<uint32_t*>(&hi2);
-        *reinterpret_cast<uint2*>(a.out + ((int64_t)t * a.H + h) * a.c + dim) = pk;
     }
     cl.sync();   // the other CTAs' shared memory stays alive until read
 }
@@ -660,7 +672,8 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, a.tmem_cols);
     }
-    if (a.cluster) cluster_merge(a, t, h0, split, (float*)kv_s, mref_s, lsum_s);
+    if (a.cluster)
+        cluster_merge(a.nsplit, a.c, a.H, a.sink, a.lse, a.out, t, h0, split, (float*)kv_s, mref_s, lsum_s);
 }
 
 bool mqa_tc_supported(int H, int c) { return c % 128 == 0 && c <= 512 && H >= 1; }
