@@ -141,21 +141,26 @@ __device__ __noinline__ void cluster_merge(int G, int c, int H, const float* sin
     const int tid = threadIdx.x;
     if (tid < 64) {
         const int h = h0 + tid;
-        // (remote values are re-read instead of kept in indexed arrays,
-        // which would live in local memory)
+        // every split's max and sum loaded at once (fully unrolled over the
+        // largest cluster, so the arrays stay in registers)
         const float sk = (sink && h < H) ? sink[h] * 1.4426950408889634f : -INFINITY;
+        float mq[kMaxClusterSplits], lq[kMaxClusterSplits];
+#pragma unroll
+        for (int q = 0; q < kMaxClusterSplits; ++q) {
+            mq[q] = q < G ? cl.map_shared_rank(mref_s, q)[tid] : -INFINITY;
+            lq[q] = q < G ? cl.map_shared_rank(lsum_s, q)[tid] : 0.f;
+        }
         float M = sk;
-        for (int q = 0; q < G; ++q) M = fmaxf(M, cl.map_shared_rank(mref_s, q)[tid]);
+#pragma unroll
+        for (int q = 0; q < kMaxClusterSplits; ++q) M = fmaxf(M, mq[q]);
         float L = (sk == -INFINITY) ? 0.f : exp2f(sk - M);
-        for (int q = 0; q < G; ++q) {
-            const float mq = cl.map_shared_rank(mref_s, q)[tid];
-            if (mq != -INFINITY) L += cl.map_shared_rank(lsum_s, q)[tid] * exp2f(mq - M);
-        }
+#pragma unroll
+        for (int q = 0; q < kMaxClusterSplits; ++q)
+            if (mq[q] != -INFINITY) L += lq[q] * exp2f(mq[q] - M);
         const float inv = L > 0.f ? 1.f / L : 0.f;
-        for (int q = 0; q < G; ++q) {
-            const float mq = cl.map_shared_rank(mref_s, q)[tid];
-            coef_s[q][tid] = (mq == -INFINITY) ? 0.f : exp2f(mq - M) * inv;
-        }
+#pragma unroll
+        for (int q = 0; q < kMaxClusterSplits; ++q)
+            if (q < G) coef_s[q][tid] = (mq[q] == -INFINITY) ? 0.f : exp2f(mq[q] - M) * inv;
         if (split == 0 && lse_out && h < H)
             lse_out[(int64_t)t * H + h] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
     }
@@ -172,26 +177,42 @@ __device__ __noinline__ void cluster_merge(int G, int c, int H, const float* sin
         float w[kMaxClusterSplits];
 #pragma unroll
         for (int q = 0; q < kMaxClusterSplits; ++q) w[q] = q < G ? coef_s[q][i] : 0.f;
-        for (int j = tid & 31; j < dn4; j += 32) {
-            const int dim = 4 * (lo4 + j);
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        // two 4-dim chunks per lane per round, all their loads issued
+        // before any is used
+        for (int j0 = tid & 31; j0 < dn4; j0 += 64) {
+            float4 v[kMaxClusterSplits][2];
 #pragma unroll
             for (int q = 0; q < kMaxClusterSplits; ++q) {
-                if (w[q] == 0.f) continue;   // also every q >= G
                 // this CTA's own split is read from its shared memory
                 // directly, the others' over distributed shared memory
                 const float* src = q == split ? obuf : cl.map_shared_rank(obuf, q);
-                const float4 v = *reinterpret_cast<const float4*>(src + i * c + dim);
-                acc.x = fmaf(w[q], v.x, acc.x);
-                acc.y = fmaf(w[q], v.y, acc.y);
-                acc.z = fmaf(w[q], v.z, acc.z);
-                acc.w = fmaf(w[q], v.w, acc.w);
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const int j = j0 + 32 * r;
+                    v[q][r] = (w[q] != 0.f && j < dn4)   // also every q >= G
+                                  ? *reinterpret_cast<const float4*>(src + i * c + 4 * (lo4 + j))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
             }
-            __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x, acc.y), hi2 = __floats2bfloat162_rn(acc.z, acc.w);
-            uint2 pk;
-            pk.x = *reinterpret_cast<uint32_t*>(&lo2);
-            pk.y = *reinterpret_cast<uint32_t*>(&hi2);
-            *reinterpret_cast<uint2*>(out + ((int64_t)t * H + h) * c + dim) = pk;
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int j = j0 + 32 * r;
+                if (j >= dn4) continue;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int q = 0; q < kMaxClusterSplits; ++q) {
+                    if (w[q] == 0.f) continue;   // an empty split staged no O
+                    acc.x = fmaf(w[q], v[q][r].x, acc.x);
+                    acc.y = fmaf(w[q], v[q][r].y, acc.y);
+                    acc.z = fmaf(w[q], v[q][r].z, acc.z);
+                    acc.w = fmaf(w[q], v[q][r].w, acc.w);
+                }
+                __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x, acc.y), hi2 = __floats2bfloat162_rn(acc.z, acc.w);
+                uint2 pk;
+                pk.x = *reinterpret_cast<uint32_t*>(&lo2);
+                pk.y = *reinterpret_cast<uint32_t*>(&hi2);
+                *reinterpret_cast<uint2*>(out + ((int64_t)t * H + h) * c + 4 * (lo4 + j)) = pk;
+            }
         }
     }
     cl.sync();   // the other CTAs' shared memory stays alive until read
