@@ -600,9 +600,15 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
         for (int h = 0; h < 64; ++h) lred[eth * 65 + h] = lpart[h];
         bar_sync_128();
         if (eth < 64) {
-            float sum = 0.f;
-            for (int i = 0; i < 128; ++i) sum += lred[i * 65 + eth];
-            lsum_s[eth] = sum;
+            // eight interleaved partial sums (fixed order), so the loads
+            // are not one dependent chain of 128
+            float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+            for (int i = 0; i < 128; i += 8) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) ps[u] += lred[(i + u) * 65 + eth];
+            }
+            lsum_s[eth] = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
         }
         bar_sync_128();
         const bool have_o = ok && ntiles > 0;
