@@ -54,7 +54,7 @@ def assert_scores_close(gpu_scores, ref_scores, bound):
 
 
 def score_bound(qI, w, K, pos, m, seq=None):
-    """sum_h w_h |q_h . K_s| (the scale against which score rounding is judged)."""
+    """sum_h w_h |q_h . K_s| (the scale against which score rounding is measured)."""
     qa = np.abs(oracle._f64(qI))
     # |q . K| <= |q| . |K|: a valid upper bound that avoids a second dot product pass
     return oracle.index_scores(qa, np.abs(oracle._f64(w)), np.abs(oracle._f64(K)), pos, m, seq=seq)

@@ -145,7 +145,7 @@ def test_topk_valid_div(csa):
 
 
 def test_topk_rows_against_a_strided_sample(csa):
-    """Rows built so that a strided sample misjudges them: the sampled
+    """Rows built so that a strided sample misleads the estimate: the sampled
     positions hold the largest scores (too few candidates reach the estimate)
     or the smallest (too many). The selection must stay exact."""
     nq, ncols, k = 4, 50000, 512
