@@ -480,14 +480,16 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
         int j = 0;
         for (; j < ntiles; ++j) {
             const int sb = j & 1;
-            if (!(ok = wait_or_abort(&s_full[sb], (j >> 1) & 1, abort_flag, a.status))) break;
-            tc::tc_fence_after();
+            // this row's entry (its index is read before the wait, so the
+            // load's latency hides behind it)
             const int64_t e = e_beg + (int64_t)j * kE + row;
             bool valid = e < e_end;
             if (valid && a.idx) {
                 int s = a.idx[(int64_t)t * a.k + e];
                 valid = s >= 0 && s < a.Nmax;
             }
+            if (!(ok = wait_or_abort(&s_full[sb], (j >> 1) & 1, abort_flag, a.status))) break;
+            tc::tc_fence_after();
             float z[64];
             const uint32_t taddr = tmem_S + ((uint32_t)(quad * 32) << 16) + sb * hg;
 #pragma unroll
