@@ -123,7 +123,10 @@ def _tie_scores(nq, ncols, seed):
     return S
 
 
-@pytest.mark.parametrize("ncols,k", [(100, 16), (5000, 512), (40000, 1024), (70000, 2048), (300000, 512)])
+# odd column counts: rows start off the 16-byte boundary (the row pass reads
+# an unaligned head and tail one score at a time)
+@pytest.mark.parametrize("ncols,k", [(100, 16), (5000, 512), (40000, 1024), (70000, 2048), (300000, 512),
+                                     (10001, 512), (20003, 64)])
 def test_topk_bitexact(csa, ncols, k):
     nq = 6
     S = _tie_scores(nq, ncols, ncols + k)
