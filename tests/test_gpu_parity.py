@@ -213,6 +213,9 @@ SPLIT_CASES = [
     ("sparse", 20, 256, 64, 1024),
     ("dense", 40, 512, 64, 700),
     ("dense", 20, 128, 64, 1100),
+    ("dense", 24, 512, 128, 700),      # two head groups, 3-way cluster
+    ("dense", 40, 384, 64, 900),       # three 128-dim M tiles cycling through a 4-slot ring
+    ("sparse", 40, 384, 64, 512),
 ]
 
 
