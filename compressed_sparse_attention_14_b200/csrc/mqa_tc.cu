@@ -17,12 +17,15 @@
 // it by more than 2^8 — exact, since the final normalisation uses the same
 // reference, and cheap, since it rarely moves after the first tile.
 //
-// Entry sources: CSA (sparse) gathers the selected rows with 16-byte
-// cp.async (the producer warp moves four rows' 128-byte block per
-// instruction); HCA (dense) loads 128 consecutive rows per 64-dim block with
-// one TMA box. The tile's 64-dim blocks are released
+// Entry sources. CSA (sparse): one tile buffer; the selected rows are
+// gathered with 16-byte cp.async (the producer warp moves four rows'
+// 128-byte block per instruction), and the tile's 64-dim blocks are released
 // one by one as the second product finishes with them, so the next tile's
-// gather overlaps it.
+// gather overlaps it. HCA (dense): consecutive rows stream through a ring of
+// 32 KB slots (a pair of 64-dim blocks per slot, one TMA box per block);
+// every tile passes through twice, for S and again (from L2) for O, in the
+// order S(0), S(1), O(0), S(2), O(1), ..., O(n-1), so the HBM read of tile
+// j+1 overlaps the softmax of tile j.
 //
 // Warp roles: warp 0 loads (all lanes issue gathers), warp 1 allocates TMEM
 // and one lane issues the MMAs, warps 2-5 run the softmax and the epilogue.
