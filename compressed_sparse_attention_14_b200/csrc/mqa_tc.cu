@@ -654,6 +654,11 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
                 if (a.lse && h < a.H) a.lse[(int64_t)t * a.H + h] = lse;
             }
             bar_sync_128();
+            // the normalised O goes through shared memory (the KV area,
+            // [head][dim] bf16) so that the output rows leave in 16-byte
+            // stores: a thread holds one dim of every head, and 2-byte
+            // stores at a head stride are slow
+            bf16* stage = reinterpret_cast<bf16*>(kv_s);
             for (int mt = 0; mt < a.mtiles; ++mt) {
                 const int dim = mt * 128 + row;
                 float v[64];
@@ -666,12 +671,17 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
                 }
 #pragma unroll
                 for (int i = 0; i < 64; ++i) {
-                    const int h = h0 + i;
-                    if (h < a.H) {
-                        float o = (have_o && mref_s[i] != -INFINITY) ? v[i] * alpha_s[i] : 0.f;
-                        a.out[((int64_t)t * a.H + h) * a.c + dim] = __float2bfloat16_rn(o);
-                    }
+                    const float o = (have_o && mref_s[i] != -INFINITY) ? v[i] * alpha_s[i] : 0.f;
+                    stage[i * a.c + dim] = __float2bfloat16_rn(o);
                 }
+            }
+            bar_sync_128();
+            const int nh = a.H - h0 < 64 ? a.H - h0 : 64;
+            const int cpr = a.c / 8;   // 16-byte chunks per head row
+            for (int e = eth; e < nh * cpr; e += 128) {
+                const int i = e / cpr, ch = e - i * cpr;
+                *reinterpret_cast<uint4*>(a.out + ((int64_t)t * a.H + h0 + i) * a.c + ch * 8) =
+                    *reinterpret_cast<const uint4*>(stage + i * a.c + ch * 8);
             }
         } else {
             if (eth < 64 && h0 + eth < a.H) {
