@@ -63,6 +63,8 @@ def _load():
             lib.orc_topk.argtypes = [_D, _I32, i32, i64, i32, _I32]
             lib.orc_sparse_mqa.argtypes = [_D, _D, _I32, _I32, i32, i32, i32, i64, i32, dbl, _D, _D, _D]
             lib.orc_dense_mqa.argtypes = [_D, _D, _I32, _I32, i32, i32, i32, i64, i32, dbl, _D, _D, _D]
+            lib.orc_norm_rope.argtypes = [_D, i64, i32, i32, _D, dbl, i32, dbl, _I32, i32, _D]
+            lib.orc_window_entries.argtypes = [_I32, i32, i32, i64, i64, _I32]
             lib.orc_num_threads.restype = i32
             _lib = lib
     return _lib
@@ -224,6 +226,35 @@ def dense_mqa(q, KV, pos, mp: int, scale: float, sink=None, seq=None):
     return out, lse
 
 
+def norm_rope(x, pos, gamma=None, eps: float = 1e-6, rope_dims: int = 64, base: float = 10000.0,
+              inverse: bool = False) -> np.ndarray:
+    """RMSNorm (when gamma is given) then rotary encoding of the last rope_dims
+    channels. x [..., G, c] or [G, c]: the rows of group g share position
+    pos[g] (x [nq, H, c] with pos [nq]: every head of query t at pos[t]).
+    inverse turns by -pos (the output's back-rotation)."""
+    x = _f64(x)
+    shape = x.shape
+    c = shape[-1]
+    pos = _i32(pos).reshape(-1)
+    rows = x.size // c
+    group = rows // max(pos.size, 1) if pos.size else 1
+    assert group * pos.size == rows, "rows must split evenly over the positions"
+    g = None if gamma is None else _f64(gamma)
+    y = np.empty_like(x)
+    _load().orc_norm_rope(_p(x), rows, group, c, _p(g), float(eps), int(rope_dims), float(base), _p(pos),
+                          1 if inverse else 0, _p(y))
+    return y.reshape(shape)
+
+
+def window_entries(pos, n_win: int, ring_off: int, ring_len: int) -> np.ndarray:
+    """Rows of the n_win most recent tokens (the query's own included) in the
+    window ring of each query's sequence; -1 before the sequence start."""
+    pos = _i32(pos).reshape(-1)
+    ent = np.empty((pos.size, n_win), dtype=np.int32)
+    _load().orc_window_entries(_p(pos), pos.size, n_win, ring_off, ring_len, _p(ent))
+    return ent
+
+
 # ---------------------------------------------------------------------------
 # Chained steps (each one a composition of the definitions above, in the
 # order the method applies them)
@@ -246,3 +277,27 @@ def index_topk(qI, w, K, pos, m: int, k: int, seq=None):
     S = index_scores(qI, w, K, pos, m, seq=seq)
     valid = np.minimum(_i32(pos) // m, S.shape[1]).astype(np.int32)
     return topk(S, valid, k), S
+
+
+def attend_decode(qI, w, idx_cache, q, kv_cache, ctx_len, m: int, k: int, n_win: int, ring_len: int,
+                  scale: float, q_gamma=None, eps: float = 1e-6, rope_dims: int = 64, base: float = 10000.0,
+                  sink=None, sel=None):
+    """One decode query per sequence with the complete attention output:
+    query RMSNorm + rotary at its position, indexer + top-k over the
+    compressed entries, the sliding window of the n_win latest tokens (rows
+    Nmax + (tau mod ring_len) of kv_cache [B, Nmax + ring_len, c]) joined to
+    the selection in one softmax, then the output turned back by the query's
+    position. sel, when given, replaces the oracle's own top-k (to compare an
+    attention output against a selection made elsewhere).
+    Returns (out, lse, idx, scores)."""
+    ctx = _i32(ctx_len)
+    B = ctx.size
+    Nmax = int(idx_cache.shape[1])
+    seq = np.arange(B, dtype=np.int32)
+    idx, S = index_topk(qI, w, idx_cache, ctx, m, k, seq=seq)
+    chosen = idx if sel is None else _i32(sel)
+    ent = np.concatenate([chosen, window_entries(ctx, n_win, Nmax, ring_len)], axis=1)
+    qn = norm_rope(q, ctx, gamma=q_gamma, eps=eps, rope_dims=rope_dims, base=base)
+    out, lse = sparse_mqa(qn, kv_cache, ent, scale, sink=sink, seq=seq)
+    out = norm_rope(out, ctx, gamma=None, rope_dims=rope_dims, base=base, inverse=True)
+    return out, lse, idx, S

@@ -31,7 +31,12 @@
  *   - MQA scale is given by the caller; an empty visible set gives out = 0
  *     and lse = -inf (or the sink logit when a sink is given);
  *   - bf16 rounding (nearest, ties to even) only where a value is stored as
- *     bf16: the compressed caches and the outputs.
+ *     bf16: the compressed caches and the outputs;
+ *   - RMSNorm is x / sqrt(mean(x^2) + eps) * gamma over the c channels of a
+ *     row; the rotary pairs are consecutive channels of the last R, turned by
+ *     p * base^(-2i/R); the output is turned back by the query's position;
+ *   - the sliding window of a query at position p holds tokens p-n_win+1 .. p
+ *     (itself included) and joins the selected entries in one softmax.
  */
 #include <math.h>
 #include <stdint.h>
@@ -322,6 +327,71 @@ void orc_dense_mqa(const double* q, const double* KV, const int32_t* pos, const 
         mqa_one(q + (int64_t)t * H * c, KV + (int64_t)seq[t] * Nmax * c, ent, vis, H, c, scale,
                 sink, out + (int64_t)t * H * c, lse + (int64_t)t * H);
         free(ent);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Query / KV normalisation and partial rotary encoding [Walk §2.3.3 items 1 */
+/* and 2; Notes §1.3 "Partial RoPE"]: every query head and every compressed  */
+/* KV entry is RMS-normalised over its c channels before the core attention; */
+/* the last R channels of both are then rotated by the row's position, and   */
+/* the attention output is rotated back by the query's position so that it  */
+/* carries relative rather than absolute position.                           */
+/* Readings (the pages give no formula):                                      */
+/*   norm:   y_j = x_j / sqrt(mean_j(x_j^2) + eps) * gamma_j                  */
+/*   rotary: channels (c-R+2i, c-R+2i+1), i < R/2, form a pair turned by the  */
+/*           angle p * theta_i, theta_i = base^(-2i/R), in the original       */
+/*           rotary form (a, b) -> (a cos - b sin, a sin + b cos); the        */
+/*           inverse turns by -p.                                             */
+/* Row r belongs to group r / group (the H heads of one query share its      */
+/* position); pos[g] is the position of group g. gamma == NULL skips the     */
+/* norm, R == 0 skips the rotation.                                           */
+/* ------------------------------------------------------------------------ */
+void orc_norm_rope(const double* x, int64_t rows, int group, int c, const double* gamma, double eps,
+                   int R, double base, const int32_t* pos, int inverse, double* y) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const double* xr = x + r * c;
+        double* yr = y + r * c;
+        if (gamma) {
+            double ss = 0.0;
+            for (int j = 0; j < c; ++j) ss += xr[j] * xr[j];
+            double inv = 1.0 / sqrt(ss / c + eps);
+            for (int j = 0; j < c; ++j) yr[j] = xr[j] * inv * gamma[j];
+        } else {
+            for (int j = 0; j < c; ++j) yr[j] = xr[j];
+        }
+        double p = (double)pos[r / group];
+        for (int i = 0; i < R / 2; ++i) {
+            double theta = pow(base, -2.0 * i / R);
+            double ang = (inverse ? -p : p) * theta;
+            int j = c - R + 2 * i;
+            double a = yr[j], b = yr[j + 1];
+            yr[j] = a * cos(ang) - b * sin(ang);
+            yr[j + 1] = a * sin(ang) + b * cos(ang);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Sliding-window branch [Walk §2.3.3 item 3; Notes §1.3 "sliding window     */
+/* branch", n_win = 128]: besides its selected compressed entries, the query */
+/* at position p attends to the uncompressed KV rows of the n_win most       */
+/* recent tokens, itself included (tokens p-n_win+1 .. p that exist). The    */
+/* rows live in a per-sequence window ring [Walk §5 item 2, the SWA state   */
+/* cache; Notes §2.6 Fig. 6]: token tau is row ring_off + (tau mod          */
+/* ring_len) of its sequence's cache block. ent[t][j] is the row of token   */
+/* p_t - n_win + 1 + j, or -1 before the start of the sequence. The window  */
+/* rows then join the selected entries in ONE softmax (orc_sparse_mqa over  */
+/* the concatenated list).                                                   */
+/* ------------------------------------------------------------------------ */
+void orc_window_entries(const int32_t* pos, int nq, int n_win, int64_t ring_off, int64_t ring_len,
+                        int32_t* ent) {
+    for (int t = 0; t < nq; ++t) {
+        for (int j = 0; j < n_win; ++j) {
+            int64_t tau = (int64_t)pos[t] - n_win + 1 + j;
+            ent[(int64_t)t * n_win + j] = tau < 0 ? -1 : (int32_t)(ring_off + tau % ring_len);
+        }
     }
 }
 

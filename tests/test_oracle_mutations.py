@@ -43,6 +43,18 @@ MUTATIONS = [
      "double r = ldexp(floor(ldexp(a, -q)), q);"),
     ("projection loops use a transposed W index", "X[t * d + k] * W[o * d + k]",
      "X[t * d + k] * W[(k * M + o) % (M * d)]"),
+    ("RMSNorm over the sum of squares instead of the mean", "sqrt(ss / c + eps)", "sqrt(ss + eps)"),
+    ("rotary frequencies base^(-i/R)", "pow(base, -2.0 * i / R)", "pow(base, -1.0 * i / R)"),
+    ("rotation turns the other way", "yr[j] = a * cos(ang) - b * sin(ang);", "yr[j] = a * cos(ang) + b * sin(ang);"),
+    ("rotary pairs split in halves instead of adjacent channels",
+     "int j = c - R + 2 * i;\n            double a = yr[j], b = yr[j + 1];\n"
+     "            yr[j] = a * cos(ang) - b * sin(ang);\n            yr[j + 1] = a * sin(ang) + b * cos(ang);",
+     "int j = c - R + i;\n            double a = yr[j], b = yr[j + R / 2];\n"
+     "            yr[j] = a * cos(ang) - b * sin(ang);\n            yr[j + R / 2] = a * sin(ang) + b * cos(ang);"),
+    ("output back-rotation turns forward", "double ang = (inverse ? -p : p) * theta;", "double ang = p * theta;"),
+    ("window leaves out the query's own token", "int64_t tau = (int64_t)pos[t] - n_win + 1 + j;",
+     "int64_t tau = (int64_t)pos[t] - n_win + j;"),
+    ("window ring rows shifted by one", "ring_off + tau % ring_len", "ring_off + (tau + 1) % ring_len"),
 ]
 
 

@@ -435,3 +435,175 @@ def test_dense_mqa_causality_and_empty():
     assert np.all(out[1] == 0) and np.all(np.isneginf(lse[1]))
     want, _ = oracle.sparse_mqa(q[2:], KV, np.array([[0, 1, 2]]), 0.5)
     np.testing.assert_allclose(out[2], want[0], rtol=1e-13, atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# Attention output completion: q/KV RMSNorm, partial rotary encoding with the
+# output's back-rotation, the sliding-window branch in the same softmax
+# (DeepSeek-V4 walk-through §2.3.3 items 1-3; study notes §1.3)
+# --------------------------------------------------------------------------
+
+def test_rmsnorm_closed_form():
+    # x = (3, 4, 0, 0): mean of squares 25/4, root 5/2 -> (6/5, 8/5, 0, 0)
+    x = np.array([[3.0, 4.0, 0.0, 0.0]])
+    y = oracle.norm_rope(x, [0], gamma=np.ones(4), eps=0.0, rope_dims=0)
+    np.testing.assert_allclose(y, [[1.2, 1.6, 0.0, 0.0]], rtol=0, atol=1e-15)
+    y = oracle.norm_rope(x, [0], gamma=np.array([1.0, 2.0, 3.0, 4.0]), eps=0.0, rope_dims=0)
+    np.testing.assert_allclose(y, [[1.2, 3.2, 0.0, 0.0]], rtol=0, atol=1e-15)
+    # eps = 7/4 moves the denominator to sqrt(25/4 + 7/4) = sqrt(8)
+    y = oracle.norm_rope(x, [0], gamma=np.ones(4), eps=1.75, rope_dims=0)
+    np.testing.assert_allclose(y, x / math.sqrt(8.0), rtol=0, atol=1e-15)
+
+
+def test_rmsnorm_unit_rms_and_scale_invariance():
+    x = rng.standard_normal((5, 3, 64))
+    y = oracle.norm_rope(x, np.arange(5), gamma=np.ones(64), eps=0.0, rope_dims=0)
+    np.testing.assert_allclose(np.sqrt((y ** 2).mean(-1)), 1.0, rtol=1e-14)
+    y2 = oracle.norm_rope(7.5 * x, np.arange(5), gamma=np.ones(64), eps=0.0, rope_dims=0)
+    np.testing.assert_allclose(y2, y, rtol=1e-13, atol=1e-14)
+
+
+def test_rope_closed_form_pairs_and_frequencies():
+    # c = 8, R = 4: the pairs are channels (4,5) and (6,7) with frequencies
+    # 10000^0 = 1 and 10000^(-2/4) = 0.01; at position 50 they turn by 50 and
+    # 0.5 radians. A unit vector on channel 4 goes to (cos 50, sin 50); one on
+    # channel 7 to (-sin 0.5, cos 0.5); channels 0-3 do not move.
+    x = np.zeros((1, 8))
+    x[0, 4] = 1.0
+    x[0, 7] = 1.0
+    x[0, 1] = 2.0
+    y = oracle.norm_rope(x, [50], rope_dims=4)
+    want = [0, 2.0, 0, 0, math.cos(50.0), math.sin(50.0), -math.sin(0.5), math.cos(0.5)]
+    np.testing.assert_allclose(y[0], want, rtol=0, atol=1e-13)
+
+
+def test_rope_is_complex_multiplication():
+    # the rotation of each pair is multiplication of a + ib by exp(i p theta)
+    c, R, base = 32, 16, 10000.0
+    x = rng.standard_normal((6, c))
+    pos = rng.integers(0, 1 << 20, 6)
+    y = oracle.norm_rope(x, pos, rope_dims=R, base=base)
+    z = x[:, c - R::2] + 1j * x[:, c - R + 1::2]
+    theta = base ** (-np.arange(R // 2) * 2.0 / R)
+    z = z * np.exp(1j * pos[:, None] * theta[None])
+    np.testing.assert_allclose(y[:, c - R::2], z.real, rtol=1e-9, atol=1e-9)
+    np.testing.assert_allclose(y[:, c - R + 1::2], z.imag, rtol=1e-9, atol=1e-9)
+    np.testing.assert_array_equal(y[:, :c - R], x[:, :c - R])
+
+
+def test_rope_relative_position_and_inverse():
+    c, R = 64, 64
+    q = rng.standard_normal((1, c))
+    k = rng.standard_normal((1, c))
+    for p, s in ((1000, 10), (131072, 131000), (7, 7)):
+        lhs = (oracle.norm_rope(q, [p], rope_dims=R) @ oracle.norm_rope(k, [s], rope_dims=R).T).item()
+        rhs = (oracle.norm_rope(q, [p - s], rope_dims=R) @ k.T).item()
+        assert abs(lhs - rhs) < 1e-9 * (1 + abs(rhs))
+    x = rng.standard_normal((4, 2, c))
+    pos = np.array([0, 5, 1 << 19, 1 << 20])
+    back = oracle.norm_rope(oracle.norm_rope(x, pos, rope_dims=R), pos, rope_dims=R, inverse=True)
+    np.testing.assert_allclose(back, x, rtol=1e-9, atol=1e-9)
+
+
+def test_rope_heads_of_a_query_share_its_position():
+    # rows of one query are its heads: each is normalised on its own and
+    # turned by the query's position, as a one-row call on that head gives
+    x = rng.standard_normal((3, 4, 16))
+    pos = np.array([3, 99, 12345])
+    g = rng.random(16) + 0.5
+    y = oracle.norm_rope(x, pos, gamma=g, rope_dims=8)
+    for t in range(3):
+        for h in range(4):
+            one = oracle.norm_rope(x[t, h][None], [pos[t]], gamma=g, rope_dims=8)[0]
+            np.testing.assert_array_equal(y[t, h], one)
+
+
+def _ring_after(tokens_kv, n_tokens, ring_len):
+    """Window ring of one sequence after tokens 0..n_tokens-1 were written in
+    order, token tau overwriting row tau mod ring_len."""
+    ring = np.zeros((ring_len, tokens_kv.shape[1]))
+    for tau in range(n_tokens):
+        ring[tau % ring_len] = tokens_kv[tau]
+    return ring
+
+
+@pytest.mark.parametrize("n_win,ring_len", [(8, 8), (8, 13), (1, 4)])
+def test_window_branch_is_banded_causal_attention(n_win, ring_len):
+    # With no compressed entry selected, the branch is plain causal attention
+    # restricted to the last n_win tokens (itself included), computed here by
+    # torch over the token-ordered rows with a band mask.
+    T, H, c = 30, 3, 16
+    tok = rng.standard_normal((T, c))
+    qs = rng.standard_normal((T, H, c))
+    scale = 0.25
+    band = np.tril(np.ones((T, T), dtype=bool)) & ~np.tril(np.ones((T, T), dtype=bool), -n_win)
+    qt = torch.from_numpy(qs).transpose(0, 1)[:, :, None, :]
+    kt = torch.from_numpy(tok)[None, None].expand(H, T, T, c)
+    mt = torch.from_numpy(band)[None, :, None, :].expand(H, T, 1, T)
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, kt, attn_mask=mt, scale=scale)
+    ref = ref[:, :, 0, :].transpose(0, 1).numpy()
+    Nmax = 5                                     # compressed rows before the ring
+    for p in range(T):
+        cache = np.concatenate([rng.standard_normal((Nmax, c)), _ring_after(tok, p + 1, ring_len)])
+        ent = oracle.window_entries([p], n_win, Nmax, ring_len)
+        out, _ = oracle.sparse_mqa(qs[p][None], cache, ent, scale)
+        np.testing.assert_allclose(out[0], ref[p], rtol=1e-12, atol=1e-12)
+
+
+def test_window_joins_the_selection_in_one_softmax():
+    # one softmax over selected entries + window rows equals the merge of the
+    # two partial softmaxes by their log-sum-exp (sink counted once); two
+    # separately normalised branches would not
+    H, c, N = 4, 16, 40
+    q = rng.standard_normal((3, H, c))
+    KV = rng.standard_normal((N, c))
+    sel = np.array([[1, 5, 9, -1], [0, 2, -1, -1], [3, 4, 6, 7]], dtype=np.int32)
+    win = oracle.window_entries([2, 40, 70], 6, 30, 10)
+    sink = rng.standard_normal(H)
+    o, l = oracle.sparse_mqa(q, KV, np.concatenate([sel, win], 1), 0.3, sink=sink)
+    o1, l1 = oracle.sparse_mqa(q, KV, sel, 0.3)
+    o2, l2 = oracle.sparse_mqa(q, KV, win, 0.3)
+    den = np.exp(l1) + np.exp(l2) + np.exp(sink)[None]
+    want = (np.exp(l1)[..., None] * o1 + np.exp(l2)[..., None] * o2) / den[..., None]
+    np.testing.assert_allclose(o, want, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(l, np.log(den), rtol=1e-12, atol=1e-12)
+    assert not np.allclose(o, 0.5 * (o1 + o2))
+
+
+def test_back_rotated_output_depends_only_on_relative_positions():
+    # KV rows rotated at their positions, the query rotated at p, the output
+    # turned back by p: shifting every position by the same amount changes
+    # nothing (the reason the pages give for the output's back-rotation)
+    H, c, R, N = 2, 32, 16, 12
+    v = rng.standard_normal((N, c))
+    q = rng.standard_normal((1, H, c))
+    epos = np.sort(rng.integers(0, 5000, N))
+    p = 6000
+    outs = []
+    for shift in (0, 777, 1 << 19):
+        kv = oracle.norm_rope(v, epos + shift, rope_dims=R)
+        qq = oracle.norm_rope(q, [p + shift], rope_dims=R)
+        o, _ = oracle.sparse_mqa(qq, kv, np.arange(N, dtype=np.int32)[None], 0.2)
+        outs.append(oracle.norm_rope(o, [p + shift], rope_dims=R, inverse=True))
+    np.testing.assert_allclose(outs[1], outs[0], rtol=1e-8, atol=1e-8)
+    np.testing.assert_allclose(outs[2], outs[0], rtol=1e-8, atol=1e-8)
+
+
+def test_attend_decode_reduces_to_plain_decode():
+    # no norm, no rotation, no window: the complete step is indexer -> top-k ->
+    # sparse MQA over the selection
+    B, HI, cI, H, c, m, k, N = 3, 4, 16, 2, 32, 4, 5, 20
+    qI = rng.standard_normal((B, HI, cI))
+    w = rng.random((B, HI))
+    K = rng.standard_normal((B, N, cI))
+    q = rng.standard_normal((B, H, c))
+    KVc = rng.standard_normal((B, N + 4, c))
+    ctx = np.array([9, 50, 79])
+    out, lse, idx, _ = oracle.attend_decode(qI, w, K, q, KVc, ctx, m, k, n_win=0, ring_len=4, scale=0.3,
+                                            rope_dims=0)
+    seq = np.arange(B)
+    ref_idx, _ = oracle.index_topk(qI, w, K, ctx, m, k, seq=seq)
+    ref, ref_l = oracle.sparse_mqa(q, KVc, ref_idx, 0.3, seq=seq)
+    np.testing.assert_array_equal(idx, ref_idx)
+    np.testing.assert_allclose(out, ref, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(lse, ref_l, rtol=1e-13, atol=1e-14)
