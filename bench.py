@@ -12,7 +12,10 @@ are resident in HBM before timing; the L2 is flushed (256 MiB write) before
 every timed step, outside the timed events; each step is timed with CUDA
 events on the stream the library launches on.
 
-Other workloads (--workload): pro_decode, hca_decode, hca_compress, prefill.
+Other workloads (--workload): pro_decode, hca_decode, hca_compress, prefill,
+flash_attend_decode (the Flash decode with the complete attention output:
+query RMSNorm + partial rotary, the 128-token sliding window joined to the
+selection in one softmax with a sink, the output turned back by position).
 
 Multi-GPU (under torchrun): every rank runs its own independent batch
 (decode queries are independent: no collective on the data path), the step
@@ -276,6 +279,77 @@ def decode_workload(shape, rank, batch=None):
                 inputs=inp)
 
 
+ATTEND_WINDOW = 128     # sliding-window tokens per query (V4's n_win)
+ATTEND_ROPE = 64        # rotary channels at the end of each head
+
+
+def attend_decode_workload(shape, rank, batch=None):
+    """The decode step with the complete attention output (csa_attend_decode):
+    query RMSNorm + partial rotary, indexer, top-k, the 128-token sliding
+    window joined to the selection in one softmax with a sink, and the output
+    turned back by the query position."""
+    import dataclasses
+    import compressed_sparse_attention_14_b200 as csa
+    s = shape if batch is None else dataclasses.replace(shape, batch=batch)
+    inp = synth.attend_decode_inputs(dataclass_seed(s, rank), device="cuda", n_win=ATTEND_WINDOW)
+    B, L = s.batch, inp["ring_len"]
+    mode = csa.CSA_BF16
+    out = torch.empty_like(inp["q"])
+    lse = torch.empty((B, s.heads), dtype=torch.float32, device="cuda")
+    ws = torch.empty(csa.workspace_size("csa_attend_decode", B, s.n_max, L, ATTEND_WINDOW, s.heads, s.c, s.idx_heads,
+                                        s.idx_dim, s.k, mode), dtype=torch.uint8, device="cuda")
+
+    def call(qI, w, q, ctx):
+        csa.csa_attend_decode(qI, w, inp["idx_cache"], q, inp["kv_cache"], ctx, s.m, s.k, n_win=ATTEND_WINDOW,
+                              ring_len=L, q_gamma=inp["q_gamma"], rope_dims=ATTEND_ROPE, sink=inp["sink"], out=out,
+                              lse=lse, ws=ws)
+
+    def step():
+        call(inp["qI"], inp["w"], inp["q"], inp["ctx_len"])
+
+    ctx = inp["ctx_len"].double()
+    v_sum = float(torch.floor(ctx / s.m).sum())
+    ke = s.k + ATTEND_WINDOW
+    qo = B * s.heads * s.c * 2                  # one bf16 pass over q or out
+    idx_bytes = v_sum * s.idx_dim * 2 + B * (s.idx_heads * s.idx_dim * 2 + s.idx_heads * 4)
+    # indexer, the selected and window rows, q read + normalised q written,
+    # the normalised q read by the MQA, out written, out read + written back
+    step_bytes = idx_bytes + B * ke * s.c * 2 + 2 * qo + 2 * qo + 2 * qo
+    idx_kernel_bytes = idx_bytes + v_sum * 4
+
+    pinned = {k: inp[k].cpu().pin_memory() for k in ("q", "qI", "w", "ctx_len")}
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dev_in = {k: torch.empty_like(inp[k]) for k in pinned}
+
+    def e2e_step():
+        for k, v in pinned.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        call(dev_in["qI"], dev_in["w"], dev_in["q"], dev_in["ctx_len"])
+        out_h.copy_(out, non_blocking=True)
+
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = out_h.numel() * out_h.element_size()
+    kernels = {
+        "index_scores_tc": dict(bound="hbm", work=idx_kernel_bytes, files=("indexer_tc.cu", "tc.cuh", "common.cuh")),
+        "mqa_tc": dict(bound="hbm", work=B * ke * s.c * 2 + 2 * qo, files=("mqa_tc.cu", "tc.cuh", "common.cuh")),
+        "topk_select": dict(bound="hbm", work=v_sum * 4 + B * s.k * 4, files=("topk.cu",)),
+        # two launches per step (query in, output back): each one read and one write of [B, H, c]
+        "norm_rope": dict(bound="hbm", work=2 * 2 * qo, files=("norm_rope.cu",)),
+        "window_entries": dict(bound="hbm", work=B * (s.k + ke) * 4, files=("norm_rope.cu",)),
+    }
+    return dict(step=step, e2e_step=e2e_step, units=B, unit="queries/s", h2d=h2d, d2h=d2h,
+                kernels=kernels, step_bytes=step_bytes,
+                config=dict(workload=ATTEND_NAME, batch=B, ctx_len=f"U[{s.ctx_lo},{s.ctx_hi}]", m=s.m,
+                            entries_max=s.n_max, head_dim=s.c, heads=s.heads, index_heads=s.idx_heads,
+                            index_dim=s.idx_dim, topk=s.k, window=ATTEND_WINDOW, window_ring=L,
+                            rope_dims=ATTEND_ROPE, q_rmsnorm=True, sink=True, visible_entries_total=int(v_sum),
+                            l2="flushed before every timed step (256 MiB write + 256 MiB read)"),
+                inputs=inp)
+
+
+ATTEND_NAME = synth.FLASH_DECODE.name + "_win128_rope64_qnorm_sink"
+
+
 def dataclass_seed(s, rank):
     import dataclasses
     return dataclasses.replace(s, seed=s.seed + 1000 * rank) if rank else s
@@ -401,6 +475,7 @@ WORKLOADS = {
     "hca_decode": lambda r, b=None: hca_decode_workload(r),
     "hca_compress": lambda r, b=None: hca_compress_workload(r),
     "prefill": lambda r, b=None: prefill_workload(r, b),
+    "flash_attend_decode": lambda r, b=None: attend_decode_workload(synth.FLASH_DECODE, r, b),
 }
 
 
@@ -418,6 +493,20 @@ def oracle_decode_sample(shape, n_queries: int, seed_rank: int = 0):
     idx, _ = oracle.index_topk(inp["qI"], inp["w"], inp["idx_cache"], inp["ctx_len"], s.m, s.k,
                                seq=torch.arange(n_queries))
     oracle.sparse_mqa(inp["q"], inp["kv_cache"], idx, 1 / math.sqrt(s.c), seq=torch.arange(n_queries))
+    return time.perf_counter() - t0, n_queries
+
+
+def oracle_attend_sample(shape, n_queries: int, seed_rank: int = 0):
+    """Time the oracle's complete decode step (query norm + rotary, indexer,
+    top-k, window joined in one softmax with the sink, back-rotation) on the
+    first n_queries of the batch. Returns (seconds, queries)."""
+    import oracle
+    s = dataclass_seed(shape, seed_rank)
+    inp = synth.attend_decode_inputs(s, device="cpu", batch=n_queries, n_win=ATTEND_WINDOW)
+    t0 = time.perf_counter()
+    oracle.attend_decode(inp["qI"], inp["w"], inp["idx_cache"], inp["q"], inp["kv_cache"], inp["ctx_len"], s.m, s.k,
+                         ATTEND_WINDOW, inp["ring_len"], 1 / math.sqrt(s.c), q_gamma=inp["q_gamma"],
+                         rope_dims=ATTEND_ROPE, sink=inp["sink"])
     return time.perf_counter() - t0, n_queries
 
 
@@ -476,6 +565,16 @@ def oracle_measure(workload: str, budget_s: float = 15.0):
                 break
             n *= 2
         desc = f"first {units} of the {shape.batch} decode queries (indexer + top-k + sparse MQA, fp64)"
+    elif workload == "flash_attend_decode":
+        shape = synth.FLASH_DECODE
+        n = max(1, threads // 2)
+        while True:
+            sec, units = oracle_attend_sample(shape, min(n, shape.batch))
+            if sec >= budget_s / 3 or n >= shape.batch:
+                break
+            n *= 2
+        desc = (f"first {units} of the {shape.batch} decode queries (query norm + rotary, indexer, top-k, window "
+                f"+ selection MQA with sink, back-rotation; fp64)")
     elif workload == "hca_decode":
         n = max(1, threads // 4)
         while True:
@@ -520,6 +619,8 @@ def run_reference(args, rank, world):
         if args.workload in ("flash_decode", "pro_decode"):
             shape = synth.FLASH_DECODE if args.workload == "flash_decode" else synth.PRO_DECODE
             sec, u = oracle_decode_sample(shape, units)
+        elif args.workload == "flash_attend_decode":
+            sec, u = oracle_attend_sample(synth.FLASH_DECODE, units)
         elif args.workload == "hca_decode":
             sec, u = oracle_hca_sample(units)
         elif args.workload == "hca_compress":
@@ -548,6 +649,7 @@ WORKLOADS_CONFIG_NAME = {
     "hca_decode": synth.HCA.name.split("_plus")[0],
     "hca_compress": "hca_compress_chunk131072_d4096",
     "prefill": synth.PREFILL.name,
+    "flash_attend_decode": ATTEND_NAME,
 }
 
 

@@ -69,6 +69,11 @@ _SIGS = {
     "csa_prefill_workspace_size": (_SZ, [_I64, _I64, _I, _I, _I, _I, _I, _I, _I, _I]),
     "csa_prefill": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I, _I, _I, _I, _P, _P, _I64, _P, _P, _P,
                          _I, _I, _I, _F, _P, _P, _P, _P, _P, _SZ, _I, _P]),
+    "csa_norm_rope": (_I, [_P, _P, _I64, _I, _I, _P, _F, _I, _F, _P, _I64, _I64, _I, _I, _P]),
+    "csa_window_entries": (_I, [_P, _I, _P, _I64, _I, _I, _I64, _I64, _P, _P]),
+    "csa_attend_decode_workspace_size": (_SZ, [_I, _I64, _I64, _I, _I, _I, _I, _I, _I, _I]),
+    "csa_attend_decode": (_I, [_P, _P, _P, _P, _P, _P, _I, _I64, _I64, _I, _I, _I, _I, _I, _I, _I, _F, _P, _F,
+                               _I, _F, _P, _P, _P, _P, _P, _SZ, _I, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -344,4 +349,75 @@ def csa_prefill(x, x_left, W_kv, B_kv, W_idx, B_idx, start: int, kv_cache, idx_c
                             m, c, cI, _ptr(kv_cache), _ptr(idx_cache), Nmax, _ptr(qI), _ptr(w), _ptr(q), H, HI, k,
                             scale, _ptr(sink), _ptr(out), _ptr(lse), _ptr(topk_idx), _ptr(ws), _nbytes(ws), mode,
                             _stream()))
+    return (out, lse, topk_idx) if return_topk else (out, lse)
+
+
+# ---------------------------------------------------------------- attention output completion
+def csa_norm_rope(x, pos=None, gamma=None, eps: float = 1e-6, rope_dims: int = 64, rope_base: float = 10000.0,
+                  inverse: bool = False, pos0: int = 0, pos_step: int = 1, group: Optional[int] = None, out=None):
+    """RMSNorm (when gamma is given) then rotary encoding of the last rope_dims
+    channels. x [..., c]: with pos [G] the rows split into G equal groups of
+    consecutive rows sharing pos[g] (x [nq, H, c] with pos [nq]: all heads of
+    query t at pos[t]); with pos None, group g of `group` rows (default 1)
+    sits at pos0 + g * pos_step. out may be x (in place)."""
+    c = x.shape[-1]
+    rows = x.numel() // c
+    if pos is not None:
+        G = pos.numel()
+        if G == 0 or rows % G:
+            raise ValueError(f"{rows} rows do not split into {G} position groups")
+        group = rows // G
+    elif group is None:
+        group = 1
+    out = torch.empty_like(x) if out is None else out
+    _check(_lib.csa_norm_rope(_ptr(x), _ptr(out), rows, group, c, _ptr(gamma), eps, rope_dims, rope_base, _ptr(pos),
+                              pos0, pos_step, int(inverse), _mode(x), _stream()))
+    return out
+
+
+def csa_window_entries(sel, pos, n_win: int, ring_off: int, ring_len: int, pos0: int = 0, nq: Optional[int] = None):
+    """[nq, k + n_win] entry lists: the selection sel [nq, k] (or None) followed
+    by the rows ring_off + (tau mod ring_len) of tokens p-n_win+1 .. p (-1 before
+    the sequence start); p = pos[t], or pos0 + t when pos is None."""
+    if sel is not None:
+        nq, k = sel.shape
+        dev = sel.device
+    else:
+        k = 0
+        if nq is None:
+            nq = pos.numel()
+        dev = pos.device if pos is not None else torch.device("cuda", torch.cuda.current_device())
+    ent = torch.empty((nq, k + n_win), dtype=torch.int32, device=dev)
+    _check(_lib.csa_window_entries(_ptr(sel), k, _ptr(pos), pos0, nq, n_win, ring_off, ring_len, _ptr(ent),
+                                   _stream()))
+    return ent
+
+
+def csa_attend_decode(qI, w, idx_cache, q, kv_cache, ctx_len, m: int, k: int, n_win: int = 128,
+                      ring_len: Optional[int] = None, scale: float = 0.0, q_gamma=None, eps: float = 1e-6,
+                      rope_dims: int = 64, rope_base: float = 10000.0, sink=None, out=None, lse=None,
+                      topk_idx=None, ws=None, return_topk: bool = False):
+    """Decode with the complete attention output: query RMSNorm + rotary,
+    indexer, top-k, the sliding window joined to the selection in one softmax,
+    and the output turned back by the query position. kv_cache [B, Nmax +
+    ring_len, c] (compressed rows, then the window ring); idx_cache [B, Nmax, cI]."""
+    B, HI, cI = qI.shape
+    _, H, c = q.shape
+    Nmax = idx_cache.shape[1]
+    if ring_len is None:
+        ring_len = kv_cache.shape[1] - Nmax
+    if kv_cache.shape[1] != Nmax + ring_len:
+        raise ValueError(f"kv_cache has {kv_cache.shape[1]} rows per sequence, Nmax + ring_len = {Nmax + ring_len}")
+    mode = _mode(q)
+    out = torch.empty_like(q) if out is None else out
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    if return_topk and topk_idx is None:
+        topk_idx = torch.empty((B, k), dtype=torch.int32, device=q.device)
+    nb = _lib.csa_attend_decode_workspace_size(B, Nmax, ring_len, n_win, H, c, HI, cI, k, mode)
+    ws = _ws(nb, q.device, ws)
+    _check(_lib.csa_attend_decode(_ptr(qI), _ptr(w), _ptr(idx_cache), _ptr(q), _ptr(kv_cache), _ptr(ctx_len), B,
+                                  Nmax, ring_len, n_win, m, H, c, HI, cI, k, scale, _ptr(q_gamma), eps, rope_dims,
+                                  rope_base, _ptr(sink), _ptr(out), _ptr(lse), _ptr(topk_idx), _ptr(ws), _nbytes(ws),
+                                  mode, _stream()))
     return (out, lse, topk_idx) if return_topk else (out, lse)

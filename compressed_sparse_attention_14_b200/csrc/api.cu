@@ -624,4 +624,136 @@ int csa_prefill(const void* x, const void* x_left, const void* W_kv, const float
     return CSA_OK;
 }
 
+// ---------------------------------------------------------------- attention output completion
+static int check_norm_rope(int c, int rope_dims, float rope_base, float eps) {
+    if (!norm_rope_supported(c, rope_dims))
+        return fail(CSA_ERR_UNSUPPORTED, "norm/rotary needs c a multiple of 8 in [8, %d] and rope_dims a multiple "
+                    "of 8 in [0, c] (c=%d rope_dims=%d)", CSA_MAX_HEAD_DIM, c, rope_dims);
+    if (rope_dims > 0 && !(rope_base > 0.f)) return fail(CSA_ERR_INVALID_ARG, "rope_base must be positive");
+    if (!(eps >= 0.f)) return fail(CSA_ERR_INVALID_ARG, "eps must be non-negative");
+    return CSA_OK;
+}
+
+static int check_window(int n_win, int64_t ring_off, int64_t ring_len) {
+    if (n_win < 0) return fail(CSA_ERR_INVALID_ARG, "n_win=%d is negative", n_win);
+    if (n_win > 0 && ring_len < n_win)
+        return fail(CSA_ERR_INVALID_ARG, "the window ring (%lld rows) is shorter than the window (%d)",
+                    (long long)ring_len, n_win);
+    if (ring_off < 0 || ring_off + ring_len > INT32_MAX)
+        return fail(CSA_ERR_UNSUPPORTED, "window ring rows beyond int32 entry indices");
+    return CSA_OK;
+}
+
+int csa_norm_rope(const void* x, void* y, int64_t rows, int group, int c, const float* gamma, float eps,
+                  int rope_dims, float rope_base, const int32_t* pos, int64_t pos0, int64_t pos_step, int inverse,
+                  int dtype, void* stream) {
+    ElemType t;
+    CSA_TRY(check_dtype(dtype, &t));
+    CSA_TRY(check_norm_rope(c, rope_dims, rope_base, eps));
+    if (rows < 0 || group < 1 || rows % group)
+        return fail(CSA_ERR_INVALID_ARG, "rows=%lld must be a non-negative multiple of group=%d", (long long)rows, group);
+    if ((rows + 15) / 16 > INT32_MAX) return fail(CSA_ERR_UNSUPPORTED, "rows=%lld beyond one launch", (long long)rows);
+    if (rows == 0) return CSA_OK;
+    CSA_TRY(check_ptr(x, "x"));
+    CSA_TRY(check_ptr(y, "y"));
+    CSA_TRY(check_ptr(gamma, "gamma", false));
+    CSA_TRY(check_ptr(pos, "pos", false));
+    if (x != y && (const char*)x < (const char*)y + rows * c * elem_size(t) &&
+        (const char*)y < (const char*)x + rows * c * elem_size(t))
+        return fail(CSA_ERR_INVALID_ARG, "x and y overlap without being the same array");
+    CSA_CUDA(norm_rope(x, y, rows, group, c, gamma, eps, rope_dims, (double)rope_base, pos, pos0, pos_step,
+                       inverse ? 1 : 0, t, (cudaStream_t)stream), "csa_norm_rope");
+    return CSA_OK;
+}
+
+int csa_window_entries(const int32_t* sel, int k, const int32_t* pos, int64_t pos0, int nq, int n_win,
+                       int64_t ring_off, int64_t ring_len, int32_t* ent, void* stream) {
+    CSA_TRY(check_window(n_win, ring_off, ring_len));
+    if (nq < 0 || k < 0) return fail(CSA_ERR_INVALID_ARG, "bad nq/k");
+    if ((int64_t)k + n_win > INT32_MAX / 2) return fail(CSA_ERR_UNSUPPORTED, "entry list too wide");
+    if (((int64_t)nq * ((int64_t)k + n_win) + 255) / 256 > INT32_MAX)
+        return fail(CSA_ERR_UNSUPPORTED, "entry lists beyond one launch");
+    if (nq == 0 || k + n_win == 0) return CSA_OK;
+    CSA_TRY(check_ptr(sel, "sel", k > 0));
+    CSA_TRY(check_ptr(pos, "pos", false));
+    CSA_TRY(check_ptr(ent, "ent"));
+    if (sel && sel == ent) return fail(CSA_ERR_INVALID_ARG, "ent must not be the selection array");
+    CSA_CUDA(window_entries(sel, k, pos, pos0, nq, n_win, ring_off, ring_len, ent, (cudaStream_t)stream),
+             "csa_window_entries");
+    return CSA_OK;
+}
+
+size_t csa_attend_decode_workspace_size(int B, int64_t Nmax, int64_t ring_len, int n_win, int H, int c, int HI,
+                                        int cI, int k, int dtype) {
+    (void)HI; (void)cI; (void)ring_len;
+    ElemType t = dtype == CSA_FP32 ? ElemType::F32 : ElemType::BF16;
+    if (B < 0 || Nmax < 0 || k < 1 || n_win < 0 || H < 1 || c < 1) return 0;
+    const int ke = k + n_win;
+    return index_topk_bytes(B, Nmax, k) + align256((size_t)B * k * sizeof(int32_t)) +
+           align256((size_t)B * ke * sizeof(int32_t)) + align256((size_t)B * H * c * elem_size(t)) +
+           mqa_workspace_bytes(B, H, c, ke, t);
+}
+
+int csa_attend_decode(const void* qI, const float* w, const void* idx_cache, const void* q, const void* kv_cache,
+                      const int32_t* ctx_len, int B, int64_t Nmax, int64_t ring_len, int n_win, int m, int H, int c,
+                      int HI, int cI, int k, float scale, const float* q_gamma, float eps, int rope_dims,
+                      float rope_base, const float* sink, void* out, float* lse, int32_t* topk_idx, void* ws,
+                      size_t ws_bytes, int dtype, void* stream) {
+    ElemType t;
+    CSA_TRY(check_dtype(dtype, &t));
+    CSA_TRY(check_index_shape(HI, cI));
+    CSA_TRY(check_index_mode(HI, cI, t));
+    CSA_TRY(check_attn_shape(H, c));
+    CSA_TRY(check_attn_mode(H, c, t));
+    CSA_TRY(check_norm_rope(c, rope_dims, rope_base, eps));
+    CSA_TRY(check_k(k));
+    CSA_TRY(check_rows(B, "csa_attend_decode"));
+    if (B < 0 || Nmax < 0 || m < 1 || ring_len < 0) return fail(CSA_ERR_INVALID_ARG, "bad B/Nmax/m/ring_len");
+    CSA_TRY(check_window(n_win, Nmax, ring_len));
+    if (k + n_win > CSA_MAX_TOPK)
+        return fail(CSA_ERR_UNSUPPORTED, "k + n_win = %d beyond %d entries per query", k + n_win, CSA_MAX_TOPK);
+    const int64_t rows = Nmax + ring_len;   // cache rows per sequence
+    CSA_TRY(check_cache_rows(B, rows));
+    if (B == 0) return CSA_OK;
+    CSA_TRY(check_ptr(qI, "qI"));
+    CSA_TRY(check_ptr(w, "w"));
+    CSA_TRY(check_ptr(idx_cache, "idx_cache", Nmax > 0));
+    CSA_TRY(check_ptr(q, "q"));
+    CSA_TRY(check_ptr(kv_cache, "kv_cache", rows > 0));
+    CSA_TRY(check_ptr(ctx_len, "ctx_len"));
+    CSA_TRY(check_ptr(q_gamma, "q_gamma", false));
+    CSA_TRY(check_ptr(sink, "sink", false));
+    CSA_TRY(check_ptr(out, "out"));
+    CSA_TRY(check_ptr(lse, "lse", false));
+    CSA_TRY(check_ptr(topk_idx, "topk_idx", false));
+    CSA_TRY(check_ws(ws, ws_bytes,
+                     csa_attend_decode_workspace_size(B, Nmax, ring_len, n_win, H, c, HI, cI, k, dtype)));
+    cudaStream_t st = (cudaStream_t)stream;
+    const int ke = k + n_win;
+    Carve cv(ws);
+    float* sc = (float*)cv.take((size_t)B * Nmax * sizeof(float));
+    void* tws = cv.take(topk_workspace_bytes(B, Nmax, k));
+    int32_t* sel = (int32_t*)cv.take((size_t)B * k * sizeof(int32_t));
+    int32_t* ent = (int32_t*)cv.take((size_t)B * ke * sizeof(int32_t));
+    void* qn = cv.take((size_t)B * H * c * elem_size(t));
+    void* mws = cv.take(mqa_workspace_bytes(B, H, c, ke, t));
+    if (topk_idx) sel = topk_idx;
+    const bool prep_q = q_gamma || rope_dims > 0;
+    QuerySpec qs{nullptr, ctx_len, 0, 0};
+    if (prep_q)
+        CSA_CUDA(norm_rope(q, qn, (int64_t)B * H, H, c, q_gamma, eps, rope_dims, (double)rope_base, ctx_len, 0, 0, 0,
+                           t, st), "csa_attend_decode: query norm/rotary");
+    CSA_CUDA(run_indexer(qI, w, idx_cache, qs, B, B, HI, cI, Nmax, m, sc, Nmax, 1, false, t, st),
+             "csa_attend_decode: indexer");
+    CSA_CUDA(topk_select(sc, Nmax, ctx_len, m, B, Nmax, k, sel, nullptr, tws, st), "csa_attend_decode: top-k");
+    CSA_CUDA(window_entries(sel, k, ctx_len, 0, B, n_win, Nmax, ring_len > 0 ? ring_len : 1, ent, st),
+             "csa_attend_decode: window entries");
+    CSA_CUDA(mqa(prep_q ? qn : q, kv_cache, ent, ke, qs, 1, B, B, H, c, rows, default_scale(scale, c), sink, out,
+                 lse, mws, t, st), "csa_attend_decode: mqa");
+    if (rope_dims > 0)
+        CSA_CUDA(norm_rope(out, out, (int64_t)B * H, H, c, nullptr, 0.f, rope_dims, (double)rope_base, ctx_len, 0, 0,
+                           1, t, st), "csa_attend_decode: output back-rotation");
+    return CSA_OK;
+}
+
 }  // extern "C"

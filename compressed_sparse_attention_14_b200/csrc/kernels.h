@@ -120,4 +120,17 @@ cudaError_t mqa(const void* q, const void* KV, const int32_t* idx, int k, QueryS
                 int nq, int n_seq, int H, int c, int64_t Nmax, float scale, const float* sink, void* out,
                 float* lse, void* ws, ElemType t, cudaStream_t st);
 
+// norm_rope.cu: RMSNorm (gamma != nullptr) then rotary encoding of the last R
+// channels of every row of c channels; row r takes the position of group
+// r / group: pos[g], or pos0 + g * pos_step when pos is null. y may equal x.
+bool norm_rope_supported(int c, int R);
+cudaError_t norm_rope(const void* x, void* y, int64_t rows, int group, int c, const float* gamma, float eps, int R,
+                      double base, const int32_t* pos, int64_t pos0, int64_t pos_step, int inverse, ElemType t,
+                      cudaStream_t st);
+// ent[t] = sel[t][0..k) then the window rows of tokens p_t - n_win + 1 .. p_t
+// (ring_off + tau mod ring_len; -1 before the sequence start), p_t = pos[t]
+// or pos0 + t when pos is null.
+cudaError_t window_entries(const int32_t* sel, int k, const int32_t* pos, int64_t pos0, int nq, int n_win,
+                           int64_t ring_off, int64_t ring_len, int32_t* ent, cudaStream_t st);
+
 }  // namespace csa

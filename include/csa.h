@@ -258,6 +258,66 @@ int csa_prefill(const void* x, const void* x_left, const void* W_kv, const float
                 const float* sink, void* out, float* lse, int32_t* topk_idx, void* ws,
                 size_t ws_bytes, int dtype, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Completion of the attention output around a6 [Walk §2.3.3 items 1-3;
+ * Notes §1.3 "Partial RoPE" and "sliding window branch"; the window's state
+ * cache: Walk §5 item 2, Notes §2.6 Fig. 6].
+ *
+ * csa_norm_rope: RMSNorm then partial rotary encoding, row by row. For each
+ * row of c channels:
+ *   y_j = x_j / sqrt(mean_j(x_j^2) + eps) * gamma_j       (gamma NULL: y = x)
+ * then the last R = rope_dims channels, as adjacent pairs (c-R+2i,
+ * c-R+2i+1), are turned by the angle p * rope_base^(-2i/R):
+ *   (a, b) -> (a cos - b sin, a sin + b cos)               (inverse: angle -p)
+ * Row r has the position of group r / group: pos[r / group] (device int32
+ * [rows / group]) or, with pos NULL, pos0 + (r / group) * pos_step. Queries
+ * [nq, H, c] use group = H and their positions; compressed KV entries use
+ * group = 1; the attention output is turned back with inverse = 1 and no
+ * gamma. x, y [rows, c] (dtype); y == x (in place) is allowed, other overlap
+ * is not. gamma [c] fp32 or NULL. c % 8 == 0, 8 <= c <= CSA_MAX_HEAD_DIM,
+ * rope_dims % 8 == 0, 0 <= rope_dims <= c, rows % group == 0. Angles are
+ * formed in fp64 (positions up to 2^31 keep their accuracy).
+ * ------------------------------------------------------------------------ */
+int csa_norm_rope(const void* x, void* y, int64_t rows, int group, int c, const float* gamma, float eps,
+                  int rope_dims, float rope_base, const int32_t* pos, int64_t pos0, int64_t pos_step, int inverse,
+                  int dtype, void* stream);
+
+/* csa_window_entries: entry lists that join the sliding window to the
+ * selected compressed entries, for one softmax over both (a6 with
+ * k' = k + n_win). Row t of ent [nq, k + n_win] int32 is sel[t][0..k)
+ * followed by the window rows of the n_win most recent tokens, the query's
+ * own included: slot k + j holds token tau = p_t - n_win + 1 + j at row
+ * ring_off + (tau mod ring_len) of the query's sequence, or -1 when tau < 0.
+ * p_t = pos[t] (device int32 [nq]) or, with pos NULL, pos0 + t. sel [nq, k]
+ * (NULL only when k == 0) and ent must not be the same array.
+ * n_win <= ring_len, ring_off + ring_len <= INT32_MAX. */
+int csa_window_entries(const int32_t* sel, int k, const int32_t* pos, int64_t pos0, int nq, int n_win,
+                       int64_t ring_off, int64_t ring_len, int32_t* ent, void* stream);
+
+/* csa_attend_decode: csa_decode with the complete attention output. Per
+ * sequence b (query position p = ctx_len[b]):
+ *   1. q' = csa_norm_rope(q[b]) with q_gamma, eps, rope_dims, rope_base at p
+ *      (skipped when q_gamma is NULL and rope_dims is 0);
+ *   2. indexer (a4) over idx_cache[b][0 .. floor(p/m)) and top-k (a5);
+ *   3. the entry list: the selection, then the window rows of tokens
+ *      p-n_win+1 .. p;
+ *   4. sparse MQA (a6) of q' over those entries of kv_cache[b], ONE softmax
+ *      (and the sink, if given) over selection and window together;
+ *   5. out turned back by p on the last rope_dims channels.
+ *   kv_cache [B, Nmax + ring_len, c]: rows 0..Nmax-1 hold the compressed
+ *   entries (already normalised and rotated at their positions), rows
+ *   Nmax + (tau mod ring_len) the window ring (token tau's uncompressed KV;
+ *   the caller has written the current token's row). idx_cache [B, Nmax, cI].
+ *   Other arguments as csa_decode. k + n_win <= CSA_MAX_TOPK,
+ *   n_win <= ring_len (ring_len may be 0 when n_win is 0). */
+size_t csa_attend_decode_workspace_size(int B, int64_t Nmax, int64_t ring_len, int n_win, int H, int c, int HI,
+                                        int cI, int k, int dtype);
+int csa_attend_decode(const void* qI, const float* w, const void* idx_cache, const void* q, const void* kv_cache,
+                      const int32_t* ctx_len, int B, int64_t Nmax, int64_t ring_len, int n_win, int m, int H, int c,
+                      int HI, int cI, int k, float scale, const float* q_gamma, float eps, int rope_dims,
+                      float rope_base, const float* sink, void* out, float* lse, int32_t* topk_idx, void* ws,
+                      size_t ws_bytes, int dtype, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -9,6 +9,7 @@ Distributions (one reading, applied to every workload):
   * projection weights: N(0, 1/d) (variance 1/d), bf16, stored [out, in];
   * positional biases: N(0, 0.1) (variance 0.1), fp32;
   * indexer head weights w: softmax over heads of N(0, 1) logits, fp32;
+  * RMSNorm weights: 1 + N(0, 0.01), fp32; sink logits: N(0, 1), fp32;
   * per-query context lengths: integers uniform on [lo, hi], inclusive.
 
 Generation uses torch's seeded generators on the target device. The stream
@@ -142,6 +143,24 @@ def decode_inputs(s: DecodeShape, device="cpu", batch: Optional[int] = None):
         w=head_weights(B, s.idx_heads, s.seed, device=device),
         ctx_len=ctx,
     )
+
+
+def attend_decode_inputs(s: DecodeShape, device="cpu", batch: Optional[int] = None, n_win: int = 128,
+                         ring_len: Optional[int] = None):
+    """decode_inputs plus what the complete attention output takes: each
+    sequence's KV block extended by its sliding-window ring (ring_len rows of
+    uncompressed token KV after the n_max compressed rows), the query RMSNorm
+    weight (1 + N(0, 0.01)) and per-head sink logits N(0, 1)."""
+    inp = decode_inputs(s, device, batch)
+    B = inp["q"].shape[0]
+    L = n_win if ring_len is None else ring_len
+    ring = normal((B, L, s.c), s.seed, "window_ring", device=device)
+    inp["kv_cache"] = torch.cat([inp["kv_cache"], ring], dim=1).contiguous()
+    del ring
+    inp["q_gamma"] = 1.0 + normal((s.c,), s.seed, "q_gamma", std=0.1, dtype=torch.float32, device=device)
+    inp["sink"] = normal((s.heads,), s.seed, "sink", dtype=torch.float32, device=device)
+    inp["ring_len"] = L
+    return inp
 
 
 def hca_decode_inputs(s: HcaShape, device="cpu", batch: Optional[int] = None, n_max: Optional[int] = None):

@@ -93,12 +93,60 @@ def test_invalid_arguments_are_rejected_on_the_host():
     del args
 
 
+def test_attention_completion_arguments_are_checked_on_the_host():
+    L = _lib()
+    fake = 0x10000
+    F = ctypes.c_float
+    # rotary width not a multiple of 8, wider than c, c not a multiple of 8
+    assert L.csa_norm_rope(fake, fake, 64, 1, 128, None, F(1e-6), 12, F(1e4), None, 0, 1, 0, csa.CSA_BF16,
+                           None) == csa.CSA_ERR_UNSUPPORTED
+    assert L.csa_norm_rope(fake, fake, 64, 1, 128, None, F(1e-6), 136, F(1e4), None, 0, 1, 0, csa.CSA_BF16,
+                           None) == csa.CSA_ERR_UNSUPPORTED
+    assert L.csa_norm_rope(fake, fake, 64, 1, 100, None, F(1e-6), 8, F(1e4), None, 0, 1, 0, csa.CSA_BF16,
+                           None) == csa.CSA_ERR_UNSUPPORTED
+    # rows must split into whole position groups; base positive; eps >= 0
+    assert L.csa_norm_rope(fake, fake, 65, 8, 128, None, F(1e-6), 64, F(1e4), fake, 0, 1, 0, csa.CSA_BF16,
+                           None) == csa.CSA_ERR_INVALID_ARG
+    assert L.csa_norm_rope(fake, fake, 64, 8, 128, None, F(1e-6), 64, F(0.0), fake, 0, 1, 0, csa.CSA_BF16,
+                           None) == csa.CSA_ERR_INVALID_ARG
+    assert L.csa_norm_rope(fake, fake, 64, 8, 128, None, F(-1.0), 64, F(1e4), fake, 0, 1, 0, csa.CSA_BF16,
+                           None) == csa.CSA_ERR_INVALID_ARG
+    # partial overlap of x and y (in place, y == x, is allowed)
+    assert L.csa_norm_rope(fake, fake + 256, 64, 1, 128, None, F(1e-6), 64, F(1e4), None, 0, 1, 0, csa.CSA_BF16,
+                           None) == csa.CSA_ERR_INVALID_ARG
+    assert b"overlap" in L.csa_last_error()
+    # the window must fit its ring; the list must not overwrite the selection
+    assert L.csa_window_entries(fake, 16, fake, 0, 4, 128, 1000, 64, fake * 2, None) == csa.CSA_ERR_INVALID_ARG
+    assert L.csa_window_entries(fake, 16, fake, 0, 4, 8, 1000, 64, fake, None) == csa.CSA_ERR_INVALID_ARG
+    assert L.csa_window_entries(fake, 16, fake, 0, 4, 8, (1 << 31) - 10, 64, fake * 2, None) == csa.CSA_ERR_UNSUPPORTED
+    # selection + window beyond the per-query entry limit; window longer than the ring
+    assert L.csa_attend_decode(fake, fake, fake, fake, fake, fake, 2, 1024, 128, 128, 4, 8, 128, 4, 64, 2000,
+                               F(0.0), None, F(1e-6), 64, F(1e4), None, fake, None, None, None, 0, csa.CSA_BF16,
+                               None) == csa.CSA_ERR_UNSUPPORTED
+    assert L.csa_attend_decode(fake, fake, fake, fake, fake, fake, 2, 1024, 64, 128, 4, 8, 128, 4, 64, 16,
+                               F(0.0), None, F(1e-6), 64, F(1e4), None, fake, None, None, None, 0, csa.CSA_BF16,
+                               None) == csa.CSA_ERR_INVALID_ARG
+    # missing workspace
+    need = L.csa_attend_decode_workspace_size(2, 1024, 128, 128, 8, 128, 4, 64, 16, csa.CSA_BF16)
+    assert need > L.csa_decode_workspace_size(2, 1024, 8, 128, 4, 64, 16, csa.CSA_BF16)
+    assert L.csa_attend_decode(fake, fake, fake, fake, fake, fake, 2, 1024, 128, 128, 4, 8, 128, 4, 64, 16,
+                               F(0.0), None, F(1e-6), 64, F(1e4), None, fake, None, None, None, 0, csa.CSA_BF16,
+                               None) == csa.CSA_ERR_WORKSPACE
+
+
 def test_empty_inputs_are_no_ops():
     L = _lib()
     assert L.csa_compress(None, None, None, 0, 8, 4, None, csa.CSA_BF16, None) == csa.CSA_OK
     assert L.csa_topk_from_scores(None, 0, None, 1, 0, 0, 8, None, None, None, 0, None) == csa.CSA_OK
     assert L.csa_decode(None, None, None, None, None, None, 0, 16, 4, 8, 128, 4, 64, 16, 0.0, None, None, None,
                         None, None, 0, csa.CSA_BF16, None) == csa.CSA_OK
+    F = ctypes.c_float
+    assert L.csa_norm_rope(None, None, 0, 1, 128, None, F(1e-6), 64, F(1e4), None, 0, 1, 0, csa.CSA_BF16,
+                           None) == csa.CSA_OK
+    assert L.csa_window_entries(None, 0, None, 0, 0, 128, 0, 128, None, None) == csa.CSA_OK
+    assert L.csa_attend_decode(None, None, None, None, None, None, 0, 16, 128, 128, 4, 8, 128, 4, 64, 16, F(0.0),
+                               None, F(1e-6), 64, F(1e4), None, None, None, None, None, 0, csa.CSA_BF16,
+                               None) == csa.CSA_OK
 
 
 def test_workspace_sizes():
