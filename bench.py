@@ -15,7 +15,9 @@ events on the stream the library launches on.
 Other workloads (--workload): pro_decode, hca_decode, hca_compress, prefill,
 flash_attend_decode (the Flash decode with the complete attention output:
 query RMSNorm + partial rotary, the 128-token sliding window joined to the
-selection in one softmax with a sink, the output turned back by position).
+selection in one softmax with a sink, the output turned back by position),
+flash_decode_compress (one decode step's compression of both CSA streams
+through the per-sequence state cache, from the new tokens' hidden states).
 
 Multi-GPU (under torchrun): every rank runs its own independent batch
 (decode queries are independent: no collective on the data path), the step
@@ -349,6 +351,65 @@ def attend_decode_workload(shape, rank, batch=None):
 
 ATTEND_NAME = synth.FLASH_DECODE.name + "_win128_rope64_qnorm_sink"
 
+COMPRESS_STEP_D = 4096   # V4-Flash hidden size
+
+
+def decode_compress_workload(rank, batch=None):
+    """One decode step's compression of both CSA streams (csa_decode_compress):
+    the new token of each of the Flash batch's sequences is projected from its
+    hidden state (d = 4096) into the KV and index-key streams, stored in the
+    sequence's state ring, and the sequences whose token closes a block (about
+    one in four) get their new entries. Every timed step redoes the same
+    tokens at the same positions."""
+    import dataclasses
+    import compressed_sparse_attention_14_b200 as csa
+    s = synth.FLASH_DECODE if batch is None else dataclasses.replace(synth.FLASH_DECODE, batch=batch)
+    s = dataclass_seed(s, rank)
+    inp = synth.decode_compress_inputs(s, COMPRESS_STEP_D, device="cuda")
+    B, d, m, c, cI = s.batch, COMPRESS_STEP_D, s.m, s.c, s.idx_dim
+    ws = torch.empty(csa.workspace_size("csa_decode_compress", B, c, cI), dtype=torch.uint8, device="cuda")
+
+    def call(x, pos):
+        csa.csa_decode_compress(x, inp["W_kv"], inp["B_kv"], inp["W_idx"], inp["B_idx"], pos, inp["state_kv"],
+                                inp["state_idx"], inp["kv_cache"], inp["idx_cache"], m, ws=ws)
+
+    def step():
+        call(inp["x"], inp["pos"])
+
+    closing = int(((inp["pos"] + 1) % m == 0).sum())
+    w_bytes = (4 * c + 4 * cI) * d * 2
+    proj_bytes = B * 4 * (c + cI) * 4
+    # weights, hidden states and fp32 projections (written, read back), the
+    # ring rows stored, the 2m ring rows read and one entry written per block closed
+    step_bytes = (w_bytes + B * d * 2 + 2 * proj_bytes + proj_bytes
+                  + closing * (2 * m * 4 * (c + cI) * 4 + (c + cI) * 2))
+    pinned = {k: inp[k].cpu().pin_memory() for k in ("x", "pos")}
+    dev_in = {k: torch.empty_like(inp[k]) for k in pinned}
+    flag_h = torch.empty((1,), dtype=inp["kv_cache"].dtype).pin_memory()
+
+    def e2e_step():
+        for k, v in pinned.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        call(dev_in["x"], dev_in["pos"])
+        flag_h.copy_(inp["kv_cache"].view(-1)[:1], non_blocking=True)
+
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    kernels = {
+        # two launches per step (KV: M = 4c, index keys: M = 4cI); work per step
+        "project_tc": dict(bound="hbm", work=w_bytes + 2 * B * d * 2 + proj_bytes, files=("gemm_tc.cu", "tc.cuh")),
+        "csa_compress_step": dict(bound="hbm", work=2 * proj_bytes, files=("compress.cu",)),
+    }
+    d2h = flag_h.numel() * flag_h.element_size()
+    return dict(step=step, e2e_step=e2e_step, units=B, unit="tokens/s", h2d=h2d, d2h=d2h,
+                kernels=kernels, step_bytes=step_bytes,
+                config=dict(workload=COMPRESS_STEP_NAME, batch=B, d=d, m=m, head_dim=c, index_dim=cI,
+                            positions=f"U[{s.ctx_lo},{s.ctx_hi}]", blocks_closed_per_step=closing,
+                            l2="flushed before every timed step (256 MiB write + 256 MiB read)"),
+                inputs=inp)
+
+
+COMPRESS_STEP_NAME = f"csa_decode_compress_flash_b64_d{COMPRESS_STEP_D}_m4"
+
 
 def dataclass_seed(s, rank):
     import dataclasses
@@ -476,6 +537,7 @@ WORKLOADS = {
     "hca_compress": lambda r, b=None: hca_compress_workload(r),
     "prefill": lambda r, b=None: prefill_workload(r, b),
     "flash_attend_decode": lambda r, b=None: attend_decode_workload(synth.FLASH_DECODE, r, b),
+    "flash_decode_compress": lambda r, b=None: decode_compress_workload(r, b),
 }
 
 
@@ -508,6 +570,24 @@ def oracle_attend_sample(shape, n_queries: int, seed_rank: int = 0):
                          ATTEND_WINDOW, inp["ring_len"], 1 / math.sqrt(s.c), q_gamma=inp["q_gamma"],
                          rope_dims=ATTEND_ROPE, sink=inp["sink"])
     return time.perf_counter() - t0, n_queries
+
+
+def oracle_decode_compress_sample(n_tokens: int):
+    """The oracle's decode-time compression work for n_tokens new tokens: the
+    projections of their hidden states into both streams (plain C loops) and
+    the compression of one block per m tokens. Returns (seconds, tokens)."""
+    import oracle
+    s = synth.FLASH_DECODE
+    inp = synth.decode_compress_inputs(dataclass_seed(s, 0), COMPRESS_STEP_D, device="cpu", batch=n_tokens,
+                                       caches=False)
+    n = n_tokens - n_tokens % s.m
+    t0 = time.perf_counter()
+    pk = oracle.project_loops(inp["x"], inp["W_kv"])
+    pi = oracle.project_loops(inp["x"], inp["W_idx"])
+    if n:
+        oracle.csa_compress(pk[:n], inp["B_kv"], s.m)
+        oracle.csa_compress(pi[:n], inp["B_idx"], s.m)
+    return time.perf_counter() - t0, n_tokens
 
 
 def oracle_hca_sample(n_queries: int):
@@ -575,6 +655,15 @@ def oracle_measure(workload: str, budget_s: float = 15.0):
             n *= 2
         desc = (f"first {units} of the {shape.batch} decode queries (query norm + rotary, indexer, top-k, window "
                 f"+ selection MQA with sink, back-rotation; fp64)")
+    elif workload == "flash_decode_compress":
+        n = 4
+        while True:
+            sec, units = oracle_decode_compress_sample(n)
+            if sec >= budget_s / 3 or n >= 1024:
+                break
+            n *= 2
+        desc = (f"{units} new tokens (projection of their hidden states into both CSA streams, compression of one "
+                f"block per {synth.FLASH_DECODE.m} tokens; fp64)")
     elif workload == "hca_decode":
         n = max(1, threads // 4)
         while True:
@@ -621,6 +710,8 @@ def run_reference(args, rank, world):
             sec, u = oracle_decode_sample(shape, units)
         elif args.workload == "flash_attend_decode":
             sec, u = oracle_attend_sample(synth.FLASH_DECODE, units)
+        elif args.workload == "flash_decode_compress":
+            sec, u = oracle_decode_compress_sample(units)
         elif args.workload == "hca_decode":
             sec, u = oracle_hca_sample(units)
         elif args.workload == "hca_compress":
@@ -632,7 +723,7 @@ def run_reference(args, rank, world):
     total = sum(times)
     value = units * len(times) / total
     wl = WORKLOADS_CONFIG_NAME.get(args.workload, args.workload)
-    unit = "tokens/s" if args.workload in ("hca_compress", "prefill") else "queries/s"
+    unit = "tokens/s" if args.workload in ("hca_compress", "prefill", "flash_decode_compress") else "queries/s"
     line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -650,6 +741,7 @@ WORKLOADS_CONFIG_NAME = {
     "hca_compress": "hca_compress_chunk131072_d4096",
     "prefill": synth.PREFILL.name,
     "flash_attend_decode": ATTEND_NAME,
+    "flash_decode_compress": COMPRESS_STEP_NAME,
 }
 
 

@@ -69,6 +69,10 @@ _SIGS = {
     "csa_prefill_workspace_size": (_SZ, [_I64, _I64, _I, _I, _I, _I, _I, _I, _I, _I]),
     "csa_prefill": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I, _I, _I, _I, _P, _P, _I64, _P, _P, _P,
                          _I, _I, _I, _F, _P, _P, _P, _P, _P, _SZ, _I, _P]),
+    "csa_compress_step": (_I, [_P, _P, _P, _P, _I, _I, _I, _I64, _P, _I, _P]),
+    "hca_compress_step": (_I, [_P, _P, _P, _P, _I, _I, _I, _I64, _P, _I, _P]),
+    "csa_decode_compress_workspace_size": (_SZ, [_I, _I, _I]),
+    "csa_decode_compress": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I64, _P, _SZ, _I, _P]),
     "csa_norm_rope": (_I, [_P, _P, _I64, _I, _I, _P, _F, _I, _F, _P, _I64, _I64, _I, _I, _P]),
     "csa_window_entries": (_I, [_P, _I, _P, _I64, _I, _I, _I64, _I64, _P, _P]),
     "csa_attend_decode_workspace_size": (_SZ, [_I, _I64, _I64, _I, _I, _I, _I, _I, _I, _I]),
@@ -213,6 +217,38 @@ def hca_compress_from_hidden(x, W, bias, mp: int, out=None, ws=None):
     _check(_lib.hca_compress_from_hidden(_ptr(x), _ptr(W), _ptr(bias), n, d, c, mp, _ptr(out), _ptr(ws),
                                          _nbytes(ws), mode, _stream()))
     return out
+
+
+# ---------------------------------------------------------------- decode-time compression
+def csa_compress_step(proj_new, state, bias, pos, cache, m: int):
+    """Store each sequence's newest projected row (proj_new [B, 4c] fp32) in its
+    state ring (state [B, 2m, 4c] fp32, updated in place) and write the entry
+    of every block the token at pos[b] closes into cache [B, Nmax, c]."""
+    B, c4 = proj_new.shape
+    _check(_lib.csa_compress_step(_ptr(proj_new), _ptr(state), _ptr(bias), _ptr(pos), B, c4 // 4, m, cache.shape[1],
+                                  _ptr(cache), _mode(cache), _stream()))
+    return cache
+
+
+def hca_compress_step(proj_new, state, bias, pos, cache, mp: int):
+    """HCA: proj_new [B, 2c] fp32, state [B, mp, 2c] fp32, cache [B, Nmax, c]."""
+    B, c2 = proj_new.shape
+    _check(_lib.hca_compress_step(_ptr(proj_new), _ptr(state), _ptr(bias), _ptr(pos), B, c2 // 2, mp, cache.shape[1],
+                                  _ptr(cache), _mode(cache), _stream()))
+    return cache
+
+
+def csa_decode_compress(x_new, W_kv, B_kv, W_idx, B_idx, pos, state_kv, state_idx, kv_cache, idx_cache, m: int = 4,
+                        ws=None):
+    """One decode step's compression of both CSA streams from the new tokens'
+    hidden states x_new [B, d]; states and caches are updated in place."""
+    B, d = x_new.shape
+    c = W_kv.shape[0] // 4
+    cI = W_idx.shape[0] // 4
+    ws = _ws(_lib.csa_decode_compress_workspace_size(B, c, cI), x_new.device, ws)
+    _check(_lib.csa_decode_compress(_ptr(x_new), _ptr(W_kv), _ptr(B_kv), _ptr(W_idx), _ptr(B_idx), _ptr(pos), B, d, m,
+                                    c, cI, _ptr(state_kv), _ptr(state_idx), _ptr(kv_cache), _ptr(idx_cache),
+                                    kv_cache.shape[1], _ptr(ws), _nbytes(ws), _mode(x_new), _stream()))
 
 
 # ---------------------------------------------------------------- a4 / a5

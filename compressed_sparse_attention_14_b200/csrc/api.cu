@@ -256,6 +256,74 @@ int hca_compress(const void* proj, const float* bias, int64_t n, int c, int mp, 
     return CSA_OK;
 }
 
+static int compress_step_common(const float* proj_new, float* state, const float* bias, const int32_t* pos, int B,
+                                int c, int m, int mmax, int64_t Nmax, void* cache, int dtype, bool overlap,
+                                void* stream, const char* who) {
+    ElemType t;
+    CSA_TRY(check_dtype(dtype, &t));
+    CSA_TRY(check_compress(0, c, m, mmax, who));
+    if (B < 0 || Nmax < 0) return fail(CSA_ERR_INVALID_ARG, "%s: bad B/Nmax", who);
+    if (B == 0) return CSA_OK;
+    CSA_TRY(check_ptr(proj_new, "proj_new"));
+    CSA_TRY(check_ptr(state, "state"));
+    CSA_TRY(check_ptr(bias, "bias"));
+    CSA_TRY(check_ptr(pos, "pos"));
+    CSA_TRY(check_ptr(cache, "cache", Nmax > 0));
+    CSA_CUDA(compress_step(proj_new, state, bias, pos, B, c, m, overlap, Nmax, cache, t, (cudaStream_t)stream), who);
+    return CSA_OK;
+}
+
+int csa_compress_step(const float* proj_new, float* state, const float* bias, const int32_t* pos, int B, int c, int m,
+                      int64_t Nmax, void* cache, int dtype, void* stream) {
+    return compress_step_common(proj_new, state, bias, pos, B, c, m, 64, Nmax, cache, dtype, true, stream,
+                                "csa_compress_step");
+}
+
+int hca_compress_step(const float* proj_new, float* state, const float* bias, const int32_t* pos, int B, int c,
+                      int mp, int64_t Nmax, void* cache, int dtype, void* stream) {
+    return compress_step_common(proj_new, state, bias, pos, B, c, mp, 1024, Nmax, cache, dtype, false, stream,
+                                "hca_compress_step");
+}
+
+size_t csa_decode_compress_workspace_size(int B, int c, int cI) {
+    if (B < 0 || c < 0 || cI < 0) return 0;
+    return align256((size_t)B * 4 * c * sizeof(float)) + align256((size_t)B * 4 * cI * sizeof(float));
+}
+
+int csa_decode_compress(const void* x_new, const void* W_kv, const float* B_kv, const void* W_idx, const float* B_idx,
+                        const int32_t* pos, int B, int d, int m, int c, int cI, float* state_kv, float* state_idx,
+                        void* kv_cache, void* idx_cache, int64_t Nmax, void* ws, size_t ws_bytes, int dtype,
+                        void* stream) {
+    ElemType t;
+    CSA_TRY(check_dtype(dtype, &t));
+    CSA_TRY(check_compress(0, c, m, 64, "csa_decode_compress"));
+    CSA_TRY(check_compress(0, cI, m, 64, "csa_decode_compress"));
+    if (d < 8 || d % 8) return fail(CSA_ERR_INVALID_ARG, "d=%d must be a positive multiple of 8", d);
+    if (B < 0 || Nmax < 0) return fail(CSA_ERR_INVALID_ARG, "csa_decode_compress: bad B/Nmax");
+    if (B == 0) return CSA_OK;
+    CSA_TRY(check_ptr(x_new, "x_new"));
+    CSA_TRY(check_ptr(W_kv, "W_kv"));
+    CSA_TRY(check_ptr(B_kv, "B_kv"));
+    CSA_TRY(check_ptr(W_idx, "W_idx"));
+    CSA_TRY(check_ptr(B_idx, "B_idx"));
+    CSA_TRY(check_ptr(pos, "pos"));
+    CSA_TRY(check_ptr(state_kv, "state_kv"));
+    CSA_TRY(check_ptr(state_idx, "state_idx"));
+    CSA_TRY(check_ptr(kv_cache, "kv_cache", Nmax > 0));
+    CSA_TRY(check_ptr(idx_cache, "idx_cache", Nmax > 0));
+    CSA_TRY(check_ws(ws, ws_bytes, csa_decode_compress_workspace_size(B, c, cI)));
+    cudaStream_t st = (cudaStream_t)stream;
+    Carve cv(ws);
+    float* pk = (float*)cv.take((size_t)B * 4 * c * sizeof(float));
+    float* pi = (float*)cv.take((size_t)B * 4 * cI * sizeof(float));
+    CSA_CUDA(project(x_new, W_kv, B, d, 4 * c, pk, t, st), "csa_decode_compress: KV projection");
+    CSA_CUDA(project(x_new, W_idx, B, d, 4 * cI, pi, t, st), "csa_decode_compress: index-key projection");
+    CSA_CUDA(compress_step(pk, state_kv, B_kv, pos, B, c, m, true, Nmax, kv_cache, t, st), "csa_decode_compress: KV");
+    CSA_CUDA(compress_step(pi, state_idx, B_idx, pos, B, cI, m, true, Nmax, idx_cache, t, st),
+             "csa_decode_compress: index keys");
+    return CSA_OK;
+}
+
 size_t csa_compress_from_hidden_workspace_size(int64_t n, int d, int c, int m, int dtype) {
     (void)d; (void)dtype;
     if (n < 0 || c < 0 || m < 1) return 0;

@@ -119,6 +119,130 @@ __global__ void __launch_bounds__(256) hca_compress_kernel(const TIn* __restrict
     else store8(reinterpret_cast<float*>(out + i * c + j), o);
 }
 
+// Decode-time compression through the per-sequence state cache [Walk §5
+// item 2: CSA keeps the tail tokens that have not yet formed a block; Notes
+// §2.6 Fig. 6]. Each sequence keeps the projected rows of its last 2m tokens
+// (m' for HCA) in a ring, token tau in slot tau mod 2m. A step stores the
+// newest token's row and, when that token closes a block, mixes the block
+// from the ring in exactly the order of the chunk kernels above (a-window,
+// then b-window), so a sequence compressed token by token gets the same
+// entries as one compressed in a chunk. A thread owns 8 channels of one
+// sequence: it reads back only ring values it wrote itself.
+template <typename TOut>
+__global__ void __launch_bounds__(256) csa_compress_step_kernel(const float* __restrict__ proj_new,
+                                                                float* __restrict__ state,
+                                                                const float* __restrict__ bias,
+                                                                const int32_t* __restrict__ pos, int B, int c,
+                                                                int m, int64_t Nmax, TOut* __restrict__ cache) {
+    pdl_wait();
+    pdl_launch_next();
+    const int groups = c / 8;
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= (int64_t)B * groups) return;
+    const int b = (int)(gid / groups);
+    const int j = (int)(gid % groups) * 8;
+    const int64_t p = pos[b];
+    if (p < 0) return;
+    const int64_t ld = 4 * (int64_t)c;
+    float* ring = state + (int64_t)b * 2 * m * ld;
+    {
+        const float* src = proj_new + (int64_t)b * ld;
+        float* dst = ring + (p % (2 * m)) * ld;
+        float v[8];
+#pragma unroll
+        for (int s4 = 0; s4 < 4; ++s4) {
+            load8(src + s4 * c + j, v);
+            store8(dst + s4 * c + j, v);
+        }
+    }
+    if ((p + 1) % m != 0) return;
+    const int64_t i = (p + 1) / m - 1;   // the block this token closes
+    if (i >= Nmax) return;
+
+    OnlineSoftmax8 sm;
+    sm.init();
+    float z[8], bb[8], v[8];
+    for (int r = 0; r < m; ++r) {
+        const float* row = ring + ((m * i + r) % (2 * m)) * ld;
+        load8(row + 2 * c + j, z);
+        load8(bias + (int64_t)r * c + j, bb);
+        load8(row + j, v);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) z[u] += bb[u];
+        sm.push(z, v);
+    }
+    if (i > 0) {
+        for (int r = 0; r < m; ++r) {
+            const float* row = ring + ((m * (i - 1) + r) % (2 * m)) * ld;
+            load8(row + 3 * c + j, z);
+            load8(bias + (int64_t)(m + r) * c + j, bb);
+            load8(row + c + j, v);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) z[u] += bb[u];
+            sm.push(z, v);
+        }
+    }
+    float o[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) o[u] = sm.acc[u] / sm.den[u];
+    TOut* out = cache + ((int64_t)b * Nmax + i) * c + j;
+    if constexpr (sizeof(TOut) == 2) store8(reinterpret_cast<bf16*>(out), o);
+    else store8(reinterpret_cast<float*>(out), o);
+}
+
+// HCA: a ring of m' rows (C | Z), slot tau mod m'; the token that closes a
+// block finds the block's rows in slots 0 .. m'-1 in token order.
+template <typename TOut>
+__global__ void __launch_bounds__(256) hca_compress_step_kernel(const float* __restrict__ proj_new,
+                                                                float* __restrict__ state,
+                                                                const float* __restrict__ bias,
+                                                                const int32_t* __restrict__ pos, int B, int c,
+                                                                int mp, int64_t Nmax, TOut* __restrict__ cache) {
+    pdl_wait();
+    pdl_launch_next();
+    const int groups = c / 8;
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= (int64_t)B * groups) return;
+    const int b = (int)(gid / groups);
+    const int j = (int)(gid % groups) * 8;
+    const int64_t p = pos[b];
+    if (p < 0) return;
+    const int64_t ld = 2 * (int64_t)c;
+    float* ring = state + (int64_t)b * mp * ld;
+    {
+        const float* src = proj_new + (int64_t)b * ld;
+        float* dst = ring + (p % mp) * ld;
+        float v[8];
+        load8(src + j, v);
+        store8(dst + j, v);
+        load8(src + c + j, v);
+        store8(dst + c + j, v);
+    }
+    if ((p + 1) % mp != 0) return;
+    const int64_t i = (p + 1) / mp - 1;
+    if (i >= Nmax) return;
+
+    OnlineSoftmax8 sm;
+    sm.init();
+    float z[8], bb[8], v[8];
+#pragma unroll 4
+    for (int r = 0; r < mp; ++r) {
+        const float* row = ring + (int64_t)r * ld;
+        load8(row + c + j, z);
+        load8(bias + (int64_t)r * c + j, bb);
+        load8(row + j, v);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) z[u] += bb[u];
+        sm.push(z, v);
+    }
+    float o[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) o[u] = sm.acc[u] / sm.den[u];
+    TOut* out = cache + ((int64_t)b * Nmax + i) * c + j;
+    if constexpr (sizeof(TOut) == 2) store8(reinterpret_cast<bf16*>(out), o);
+    else store8(reinterpret_cast<float*>(out), o);
+}
+
 template <typename TIn, typename TOut>
 cudaError_t launch_csa_compress(const void* proj, const void* left, const float* bias, int64_t n,
                                 int c, int m, void* out, cudaStream_t st) {
@@ -163,6 +287,35 @@ cudaError_t compress_hca(const void* proj, const float* bias, int64_t n, int c, 
     if (in_t == ElemType::F32 && out_t == ElemType::BF16)
         return launch_hca_compress<float, bf16>(proj, bias, n, c, mp, out, st);
     return launch_hca_compress<float, float>(proj, bias, n, c, mp, out, st);
+}
+
+cudaError_t compress_step(const float* proj_new, float* state, const float* bias, const int32_t* pos, int B, int c,
+                          int m, bool overlap, int64_t Nmax, void* cache, ElemType out_t, cudaStream_t st) {
+    const int64_t threads = (int64_t)B * (c / 8);
+    if (threads == 0) return cudaSuccess;
+    const dim3 grid((unsigned)((threads + 255) / 256));
+    cudaError_t e = cudaSuccess;
+    if (overlap) {
+        if (out_t == ElemType::BF16)
+            CSA_LAUNCH(st, "csa_compress_step",
+                       e = launch_pdl(csa_compress_step_kernel<bf16>, grid, dim3(256), 0, st, 0, proj_new, state, bias,
+                                      pos, B, c, m, Nmax, (bf16*)cache));
+        else
+            CSA_LAUNCH(st, "csa_compress_step",
+                       e = launch_pdl(csa_compress_step_kernel<float>, grid, dim3(256), 0, st, 0, proj_new, state,
+                                      bias, pos, B, c, m, Nmax, (float*)cache));
+    } else {
+        if (out_t == ElemType::BF16)
+            CSA_LAUNCH(st, "hca_compress_step",
+                       e = launch_pdl(hca_compress_step_kernel<bf16>, grid, dim3(256), 0, st, 0, proj_new, state, bias,
+                                      pos, B, c, m, Nmax, (bf16*)cache));
+        else
+            CSA_LAUNCH(st, "hca_compress_step",
+                       e = launch_pdl(hca_compress_step_kernel<float>, grid, dim3(256), 0, st, 0, proj_new, state,
+                                      bias, pos, B, c, m, Nmax, (float*)cache));
+    }
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
 }
 
 }  // namespace csa

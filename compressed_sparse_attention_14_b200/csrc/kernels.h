@@ -75,6 +75,12 @@ cudaError_t compress_csa(const void* proj, const void* left, const float* bias, 
 cudaError_t compress_hca(const void* proj, const float* bias, int64_t n, int c, int mp, void* out,
                          ElemType in_t, ElemType out_t, cudaStream_t st);
 
+// compress.cu, decode time: store the newest token's projected row of each
+// sequence in its state ring (2m rows of [C^a|C^b|Z^a|Z^b] when overlap, m
+// rows of [C|Z] otherwise) and write the entry of a block the token closes.
+cudaError_t compress_step(const float* proj_new, float* state, const float* bias, const int32_t* pos, int B, int c,
+                          int m, bool overlap, int64_t Nmax, void* cache, ElemType out_t, cudaStream_t st);
+
 // gemm.cu: out[n, M] (fp32) = x[n, d] . W[M, d]^T (bf16 -> gemm_tc.cu)
 cudaError_t project(const void* x, const void* W, int64_t n, int d, int M, float* out, ElemType t,
                     cudaStream_t st);

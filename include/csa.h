@@ -137,6 +137,48 @@ int hca_compress_from_hidden(const void* x, const void* W, const float* bias, in
                              void* stream);
 
 /* ------------------------------------------------------------------------
+ * Decode-time compression through the per-sequence state cache [Walk §5
+ * item 2: CSA keeps the "tail" tokens that have not yet formed a block, in a
+ * fixed-size per-request state; Notes §2.6 Fig. 6, state cache]. One new
+ * token per sequence per step; the entry of a block is written by the step
+ * whose token closes it, and equals what csa_compress gives for the same
+ * rows (the same operations in the same order).
+ *
+ * csa_compress_step:
+ *   proj_new [B, 4c] fp32: the newest token's projections (C^a|C^b|Z^a|Z^b,
+ *            as csa_project writes them) of sequence b;
+ *   state    [B, 2m, 4c] fp32, caller-owned and kept across steps: the ring
+ *            of the last 2m tokens' projections (token tau in slot
+ *            tau mod 2m); only slots of the last 2m tokens are ever read;
+ *   bias     [2m, c] fp32 (as csa_compress);
+ *   pos      [B] int32 (device): the newest token's position (= tokens
+ *            before it); a negative position skips the sequence;
+ *   cache    [B, Nmax, c] (dtype): when (pos+1) % m == 0, entry
+ *            i = (pos+1)/m - 1 (if i < Nmax) is written from the ring:
+ *            a-window tokens mi..mi+m-1, b-window m(i-1)..mi-1 (none for
+ *            i = 0); nothing else is written.
+ * c % 8 == 0, 1 <= m <= 64. */
+int csa_compress_step(const float* proj_new, float* state, const float* bias, const int32_t* pos, int B, int c, int m,
+                      int64_t Nmax, void* cache, int dtype, void* stream);
+
+/* hca_compress_step: the same for HCA: proj_new [B, 2c] (C|Z), state
+ * [B, mp, 2c] (token tau in slot tau mod mp), bias [mp, c]; entry
+ * (pos+1)/mp - 1 is written when (pos+1) % mp == 0. 1 <= mp <= 1024. */
+int hca_compress_step(const float* proj_new, float* state, const float* bias, const int32_t* pos, int B, int c,
+                      int mp, int64_t Nmax, void* cache, int dtype, void* stream);
+
+/* csa_decode_compress: a1 + csa_compress_step for both CSA streams of one
+ * decode step: x_new [B, d] (dtype) projected by W_kv [4c, d] and W_idx
+ * [4cI, d], then stepped through state_kv [B, 2m, 4c] and state_idx
+ * [B, 2m, 4cI] (fp32) into kv_cache [B, Nmax, c] and idx_cache [B, Nmax, cI]
+ * with B_kv [2m, c], B_idx [2m, cI]; pos as csa_compress_step. */
+size_t csa_decode_compress_workspace_size(int B, int c, int cI);
+int csa_decode_compress(const void* x_new, const void* W_kv, const float* B_kv, const void* W_idx, const float* B_idx,
+                        const int32_t* pos, int B, int d, int m, int c, int cI, float* state_kv, float* state_idx,
+                        void* kv_cache, void* idx_cache, int64_t Nmax, void* ws, size_t ws_bytes, int dtype,
+                        void* stream);
+
+/* ------------------------------------------------------------------------
  * a4. Lightning indexer [Notes §1.1, equation I_{t,s}; Walk §2.3.1]:
  *   scores[t][s] = sum_h w[t][h] * ReLU(qI[t][h] . K[seq_t][s]),
  *   for s < floor(pos[t] / m); columns s >= that are set to -inf.

@@ -163,6 +163,29 @@ def attend_decode_inputs(s: DecodeShape, device="cpu", batch: Optional[int] = No
     return inp
 
 
+def decode_compress_inputs(s: DecodeShape, d: int, device="cpu", batch: Optional[int] = None, caches: bool = True):
+    """One decode step's compression inputs: the new tokens' hidden states
+    x [B, d], the compressor weights and biases of both CSA streams, the new
+    tokens' positions (the context lengths), zeroed state rings and caches."""
+    B = s.batch if batch is None else batch
+    m, c, cI = s.m, s.c, s.idx_dim
+    inp = dict(
+        x=normal((B, d), s.seed, "step_x", device=device),
+        W_kv=normal((4 * c, d), s.seed, "step_W_kv", std=1.0 / math.sqrt(d), device=device),
+        B_kv=normal((2 * m, c), s.seed, "step_B_kv", std=math.sqrt(0.1), dtype=torch.float32, device=device),
+        W_idx=normal((4 * cI, d), s.seed, "step_W_idx", std=1.0 / math.sqrt(d), device=device),
+        B_idx=normal((2 * m, cI), s.seed, "step_B_idx", std=math.sqrt(0.1), dtype=torch.float32, device=device),
+        pos=uniform_int(s.batch, s.ctx_lo, s.ctx_hi, s.seed, "ctx_len", device)[:B].contiguous()
+        if B <= s.batch else uniform_int(B, s.ctx_lo, s.ctx_hi, s.seed, "step_pos", device),
+    )
+    if caches:
+        inp["state_kv"] = torch.zeros((B, 2 * m, 4 * c), dtype=torch.float32, device=device)
+        inp["state_idx"] = torch.zeros((B, 2 * m, 4 * cI), dtype=torch.float32, device=device)
+        inp["kv_cache"] = torch.zeros((B, s.n_max, c), dtype=torch.bfloat16, device=device)
+        inp["idx_cache"] = torch.zeros((B, s.n_max, cI), dtype=torch.bfloat16, device=device)
+    return inp
+
+
 def hca_decode_inputs(s: HcaShape, device="cpu", batch: Optional[int] = None, n_max: Optional[int] = None):
     B = s.batch if batch is None else batch
     N = s.n_max if n_max is None else n_max

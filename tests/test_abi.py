@@ -134,6 +134,26 @@ def test_attention_completion_arguments_are_checked_on_the_host():
                                None) == csa.CSA_ERR_WORKSPACE
 
 
+def test_compress_step_arguments_are_checked_on_the_host():
+    L = _lib()
+    fake = 0x10000
+    # compression rate outside the kernels' range, channels not a multiple of 8
+    assert L.csa_compress_step(fake, fake, fake, fake, 4, 64, 0, 16, fake, csa.CSA_BF16, None) == csa.CSA_ERR_INVALID_ARG
+    assert L.csa_compress_step(fake, fake, fake, fake, 4, 64, 65, 16, fake, csa.CSA_BF16, None) == csa.CSA_ERR_INVALID_ARG
+    assert L.hca_compress_step(fake, fake, fake, fake, 4, 60, 128, 16, fake, csa.CSA_BF16, None) == csa.CSA_ERR_INVALID_ARG
+    assert L.hca_compress_step(fake, fake, fake, fake, 4, 64, 2048, 16, fake, csa.CSA_BF16, None) == csa.CSA_ERR_INVALID_ARG
+    # the state ring is required; misaligned pointers are refused
+    assert L.csa_compress_step(fake, None, fake, fake, 4, 64, 4, 16, fake, csa.CSA_BF16, None) == csa.CSA_ERR_INVALID_ARG
+    assert b"state" in L.csa_last_error()
+    assert L.csa_compress_step(fake + 8, fake, fake, fake, 4, 64, 4, 16, fake, csa.CSA_BF16, None) == csa.CSA_ERR_INVALID_ARG
+    # the fused step: workspace for both projections
+    need = L.csa_decode_compress_workspace_size(64, 512, 128)
+    assert need >= 64 * 4 * (512 + 128) * 4
+    rc = L.csa_decode_compress(fake, fake, fake, fake, fake, fake, 64, 4096, 4, 512, 128, fake, fake, fake, fake,
+                               32768, None, 0, csa.CSA_BF16, None)
+    assert rc == csa.CSA_ERR_WORKSPACE
+
+
 def test_empty_inputs_are_no_ops():
     L = _lib()
     assert L.csa_compress(None, None, None, 0, 8, 4, None, csa.CSA_BF16, None) == csa.CSA_OK
@@ -144,6 +164,9 @@ def test_empty_inputs_are_no_ops():
     assert L.csa_norm_rope(None, None, 0, 1, 128, None, F(1e-6), 64, F(1e4), None, 0, 1, 0, csa.CSA_BF16,
                            None) == csa.CSA_OK
     assert L.csa_window_entries(None, 0, None, 0, 0, 128, 0, 128, None, None) == csa.CSA_OK
+    assert L.csa_compress_step(None, None, None, None, 0, 64, 4, 16, None, csa.CSA_BF16, None) == csa.CSA_OK
+    assert L.csa_decode_compress(None, None, None, None, None, None, 0, 256, 4, 64, 64, None, None, None, None, 16,
+                                 None, 0, csa.CSA_BF16, None) == csa.CSA_OK
     assert L.csa_attend_decode(None, None, None, None, None, None, 0, 16, 128, 128, 4, 8, 128, 4, 64, 16, F(0.0),
                                None, F(1e-6), 64, F(1e4), None, None, None, None, None, 0, csa.CSA_BF16,
                                None) == csa.CSA_OK

@@ -1,7 +1,9 @@
-"""GPU parity of the attention-output completion against the CPU oracle:
+"""GPU parity of the steps around the hot path against the CPU oracle:
 query / KV RMSNorm with partial rotary encoding and the output's
-back-rotation, the sliding-window entry lists, and the complete decode step
-(the window joined to the top-k selection in one softmax with a sink)."""
+back-rotation, the sliding-window entry lists, the complete decode step (the
+window joined to the top-k selection in one softmax with a sink), and
+decode-time compression through the per-sequence state cache (token by token
+it must give the chunk compressor's entries)."""
 import math
 
 import numpy as np
@@ -160,3 +162,89 @@ def test_attend_prefill_composed_from_the_entry_points(csa):
     ref_o = oracle.norm_rope(ref_o, pos, rope_dims=64, inverse=True)
     assert_close(out, ref_o, torch.bfloat16, "composed prefill out")
     assert_close(lse, ref_l, torch.bfloat16, "composed prefill lse")
+
+
+# ---------------------------------------------------------------- decode-time compression
+def _step_schedule(T_b):
+    """pos per step: sequence b takes token s at step s while s < T_b[b], then sits out (-1)."""
+    T = max(T_b)
+    return [torch.tensor([s if s < t else -1 for t in T_b], dtype=torch.int32) for s in range(T)]
+
+
+@pytest.mark.parametrize("dtype", MODES)
+def test_csa_compress_step_equals_chunk_compression(csa, dtype):
+    m, c, Nmax = 4, 136, 10                  # 17 channel groups; entry 10 of the longest sequence is out of range
+    T_b = [37, 4, 5, 44, 1, 0]
+    B = len(T_b)
+    rows = synth.normal((B, max(T_b), 4 * c), 15, "step_rows", dtype=torch.float32)
+    bias = synth.normal((2 * m, c), 15, "step_bias", std=math.sqrt(0.1), dtype=torch.float32)
+    state = torch.zeros((B, 2 * m, 4 * c), dtype=torch.float32, device=DEV)
+    sentinel = 7.0
+    cache = torch.full((B, Nmax, c), sentinel, dtype=dtype, device=DEV)
+    rows_d, bias_d = rows.to(DEV), bias.to(DEV)
+    for s, pos in enumerate(_step_schedule(T_b)):
+        csa.csa_compress_step(rows_d[:, s].contiguous(), state, bias_d, pos.to(DEV), cache, m)
+    got = host(cache)
+    for b, T in enumerate(T_b):
+        n = min((T // m), Nmax)
+        if n:
+            ref = oracle.csa_compress(rows[b, :n * m], bias, m)
+            assert_close(got[b, :n], ref, dtype, f"sequence {b}")
+        assert np.all(got[b, n:] == sentinel), f"sequence {b}: rows past its closed blocks were written"
+    if dtype == torch.float32:
+        # the chunk kernel on the same rows: the same operations in the same order
+        for b, T in enumerate(T_b):
+            n = min((T // m), Nmax)
+            if n:
+                chunk = csa.csa_compress(rows_d[b, :n * m].contiguous(), bias_d, m)
+                assert float((chunk - cache[b, :n]).abs().max()) <= 1e-6
+
+
+@pytest.mark.parametrize("dtype", MODES)
+@pytest.mark.parametrize("mp", [8, 128])
+def test_hca_compress_step_equals_chunk_compression(csa, dtype, mp):
+    c, Nmax = 64, 3
+    T_b = [3 * mp + 5, mp, mp - 1, 2 * mp + 1]
+    B = len(T_b)
+    rows = synth.normal((B, max(T_b), 2 * c), 16, f"hstep_rows{mp}", dtype=torch.float32)
+    bias = synth.normal((mp, c), 16, f"hstep_bias{mp}", std=math.sqrt(0.1), dtype=torch.float32)
+    state = torch.zeros((B, mp, 2 * c), dtype=torch.float32, device=DEV)
+    cache = torch.full((B, Nmax, c), 7.0, dtype=dtype, device=DEV)
+    rows_d, bias_d = rows.to(DEV), bias.to(DEV)
+    for s, pos in enumerate(_step_schedule(T_b)):
+        csa.hca_compress_step(rows_d[:, s].contiguous(), state, bias_d, pos.to(DEV), cache, mp)
+    got = host(cache)
+    for b, T in enumerate(T_b):
+        n = min(T // mp, Nmax)
+        if n:
+            assert_close(got[b, :n], oracle.hca_compress(rows[b, :n * mp], bias, mp), dtype, f"sequence {b}")
+        assert np.all(got[b, n:] == 7.0)
+
+
+@pytest.mark.parametrize("dtype", MODES)
+def test_decode_compress_from_hidden(csa, dtype):
+    # both CSA streams of a decode loop, projected from each step's hidden
+    # states, against the chunk definition over each sequence's history
+    m, d, c, cI, Nmax = 4, 256, 64, 64, 8
+    T_b = [13, 8, 3, 11]
+    B = len(T_b)
+    X = synth.normal((B, max(T_b), d), 17, "dc_x", dtype=dtype)
+    W_kv = synth.normal((4 * c, d), 17, "dc_Wkv", std=1 / math.sqrt(d), dtype=dtype)
+    W_idx = synth.normal((4 * cI, d), 17, "dc_Widx", std=1 / math.sqrt(d), dtype=dtype)
+    B_kv = synth.normal((2 * m, c), 17, "dc_Bkv", std=math.sqrt(0.1), dtype=torch.float32)
+    B_idx = synth.normal((2 * m, cI), 17, "dc_Bidx", std=math.sqrt(0.1), dtype=torch.float32)
+    st_kv = torch.zeros((B, 2 * m, 4 * c), dtype=torch.float32, device=DEV)
+    st_idx = torch.zeros((B, 2 * m, 4 * cI), dtype=torch.float32, device=DEV)
+    kv = torch.zeros((B, Nmax, c), dtype=dtype, device=DEV)
+    ik = torch.zeros((B, Nmax, cI), dtype=dtype, device=DEV)
+    dev = [t.to(DEV) for t in (X, W_kv, B_kv, W_idx, B_idx)]
+    for s, pos in enumerate(_step_schedule(T_b)):
+        csa.csa_decode_compress(dev[0][:, s].contiguous(), dev[1], dev[2], dev[3], dev[4], pos.to(DEV), st_kv, st_idx,
+                                kv, ik, m)
+    for b, T in enumerate(T_b):
+        n = T // m
+        if n:
+            ref_kv = oracle.csa_compress_from_hidden(X[b, :n * m], W_kv, B_kv, m)
+            ref_ik = oracle.csa_compress_from_hidden(X[b, :n * m], W_idx, B_idx, m)
+            assert_close(kv[b, :n], ref_kv, dtype, f"KV entries of sequence {b}")
+            assert_close(ik[b, :n], ref_ik, dtype, f"index keys of sequence {b}")
