@@ -63,6 +63,9 @@ def _load():
             lib.orc_topk.argtypes = [_D, _I32, i32, i64, i32, _I32]
             lib.orc_sparse_mqa.argtypes = [_D, _D, _I32, _I32, i32, i32, i32, i64, i32, dbl, _D, _D, _D]
             lib.orc_dense_mqa.argtypes = [_D, _D, _I32, _I32, i32, i32, i32, i64, i32, dbl, _D, _D, _D]
+            lib.orc_e4m3_round.restype = dbl
+            lib.orc_e4m3_round.argtypes = [dbl]
+            lib.orc_quantize_rows_e4m3.argtypes = [_D, i64, i64, _D, _D]
             lib.orc_norm_rope.argtypes = [_D, i64, i32, i32, _D, dbl, i32, dbl, _I32, i32, _D]
             lib.orc_window_entries.argtypes = [_I32, i32, i32, i64, i64, _I32]
             lib.orc_num_threads.restype = i32
@@ -109,6 +112,46 @@ def bf16_round(x) -> np.ndarray:
     y = np.empty_like(x)
     _load().orc_bf16_round_array(_p(x), x.size, _p(y))
     return y
+
+
+def e4m3_round(x) -> np.ndarray:
+    """Nearest e4m3 (FP8) value of each element, ties to even, saturating at
+    +-448, returned as float64."""
+    x = _f64(x)
+    f = _load().orc_e4m3_round
+    return np.vectorize(f, otypes=[np.float64])(x) if x.size else x.copy()
+
+
+def quantize_rows_e4m3(x):
+    """Row-wise e4m3 quantisation of x [..., n] with scale max|row| / 448.
+    Returns (dequantised values, scales [...])."""
+    x = _f64(x)
+    n = x.shape[-1]
+    rows = x.size // n if n else 0
+    y = np.empty_like(x)
+    s = np.empty(x.shape[:-1])
+    _load().orc_quantize_rows_e4m3(_p(x), rows, n, _p(y), _p(s))
+    return y, s
+
+
+def index_scores_fp8(qI, w, K, pos, m: int, seq=None) -> np.ndarray:
+    """The indexer with q^I and K stored in e4m3 (one scale per query head
+    row and per key row), the products and sums exact: the definition of
+    index_scores applied to the dequantised operands."""
+    q8, _ = quantize_rows_e4m3(qI)
+    k8, _ = quantize_rows_e4m3(K)
+    return index_scores(q8, w, k8, pos, m, seq=seq)
+
+
+def topk_recall(idx, ref_idx) -> float:
+    """Mean over rows of |idx ∩ ref_idx| / |ref_idx| (entries >= 0 only)."""
+    idx, ref_idx = _i32(idx), _i32(ref_idx)
+    rec = []
+    for a, b in zip(idx, ref_idx):
+        rb = set(b[b >= 0].tolist())
+        if rb:
+            rec.append(len(set(a[a >= 0].tolist()) & rb) / len(rb))
+    return float(np.mean(rec)) if rec else 1.0
 
 
 def project(X, W) -> np.ndarray:

@@ -75,6 +75,43 @@ void orc_bf16_round_array(const double* x, int64_t n, double* y) {
 }
 
 /* ------------------------------------------------------------------------ */
+/* FP8 (e4m3) storage rounding, for the low-precision indexer and KV storage */
+/* [Walk §2.3.4 and Notes §1.3 "mixed-precision storage": FP8 for the KV     */
+/* channels outside the rotary ones, low-precision indexer arithmetic].      */
+/* e4m3: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits, no          */
+/* infinities; normal numbers 2^-6 .. 448, subnormals in steps of 2^-9.     */
+/* Nearest value, ties to even; magnitudes beyond 448 saturate to 448 (the  */
+/* saturating conversion; the format has no infinity).                      */
+/* ------------------------------------------------------------------------ */
+double orc_e4m3_round(double x) {
+    if (x == 0.0 || isnan(x)) return x;
+    double a = fabs(x);
+    if (a >= 448.0) return x < 0 ? -448.0 : 448.0;
+    int e;
+    frexp(a, &e);              /* a = f * 2^e, f in [0.5, 1) */
+    int q = e - 4;             /* quantum exponent for 4 significant bits */
+    if (q < -9) q = -9;        /* subnormal quantum */
+    double r = ldexp(round_half_even(ldexp(a, -q)), q);
+    return x < 0 ? -r : r;
+}
+
+/* Row-wise e4m3 quantisation: each row of n values is divided by its scale  */
+/* s = max|x| / 448 (1 for an all-zero row), rounded to e4m3, and the        */
+/* dequantised value code * s is returned in y; scale[r] = s.               */
+void orc_quantize_rows_e4m3(const double* x, int64_t rows, int64_t n, double* y, double* scale) {
+    for (int64_t r = 0; r < rows; ++r) {
+        double amax = 0.0;
+        for (int64_t j = 0; j < n; ++j) {
+            double v = fabs(x[r * n + j]);
+            if (v > amax) amax = v;
+        }
+        double s = amax > 0.0 ? amax / 448.0 : 1.0;
+        scale[r] = s;
+        for (int64_t j = 0; j < n; ++j) y[r * n + j] = orc_e4m3_round(x[r * n + j] / s) * s;
+    }
+}
+
+/* ------------------------------------------------------------------------ */
 /* a1. Projections [Walk §2.3.1 "KV compression"; Notes §1.1]: each of the   */
 /* compressor streams is a learnable linear map of the hidden state.         */
 /* W is stored as [M][d] (one row per output feature).                      */

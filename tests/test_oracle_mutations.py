@@ -55,6 +55,14 @@ MUTATIONS = [
     ("window leaves out the query's own token", "int64_t tau = (int64_t)pos[t] - n_win + 1 + j;",
      "int64_t tau = (int64_t)pos[t] - n_win + j;"),
     ("window ring rows shifted by one", "ring_off + tau % ring_len", "ring_off + (tau + 1) % ring_len"),
+    ("e4m3 with four mantissa bits", "int q = e - 4;             /* quantum exponent for 4 significant bits */",
+     "int q = e - 5;"),
+    ("e4m3 subnormals in steps of 2^-10", "if (q < -9) q = -9;        /* subnormal quantum */",
+     "if (q < -10) q = -10;"),
+    ("e4m3 ties rounded away from zero",
+     "double r = ldexp(round_half_even(ldexp(a, -q)), q);\n    return x < 0 ? -r : r;\n}\n\n/* Row-wise",
+     "double r = ldexp(floor(ldexp(a, -q) + 0.5), q);\n    return x < 0 ? -r : r;\n}\n\n/* Row-wise"),
+    ("row scale maps the maximum to 240", "amax / 448.0 : 1.0", "amax / 240.0 : 1.0"),
 ]
 
 

@@ -607,3 +607,74 @@ def test_attend_decode_reduces_to_plain_decode():
     np.testing.assert_array_equal(idx, ref_idx)
     np.testing.assert_allclose(out, ref, rtol=1e-13, atol=1e-14)
     np.testing.assert_allclose(lse, ref_l, rtol=1e-13, atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# FP8 (e4m3) storage for the low-precision indexer and KV (walk-through
+# §2.3.4 and study notes §1.3, mixed-precision storage)
+# --------------------------------------------------------------------------
+
+def test_e4m3_round_matches_torch_on_every_bf16_value_in_range():
+    # torch's float8_e4m3fn conversion (nearest, ties to even) agrees with the
+    # oracle wherever torch does not overflow to NaN (|x| <= 464)
+    bits = torch.arange(0, 1 << 16, dtype=torch.int32).to(torch.int16).view(torch.bfloat16)
+    x = bits.float()
+    x = x[torch.isfinite(x) & (x.abs() <= 464)]
+    want = x.to(torch.float8_e4m3fn).float().double().numpy()
+    got = oracle.e4m3_round(x.double().numpy())
+    np.testing.assert_array_equal(got, want)
+    r = torch.from_numpy(rng.standard_normal(20000) * np.exp(rng.uniform(-12, 6, 20000))).float()
+    r = r[r.abs() <= 464]
+    np.testing.assert_array_equal(oracle.e4m3_round(r.double().numpy()), r.to(torch.float8_e4m3fn).double().numpy())
+
+
+def test_e4m3_round_by_hand():
+    cases = {1.0625: 1.0,           # tie between 1 and 1.125: even mantissa
+             1.1875: 1.25,          # tie between 1.125 and 1.25
+             448.0: 448.0, 464.0: 448.0, 500.0: 448.0, -1e9: -448.0,   # saturation, no infinity
+             2.0 ** -9: 2.0 ** -9,  # smallest subnormal
+             2.0 ** -10: 0.0,       # tie between 0 and 2^-9
+             3 * 2.0 ** -11: 2.0 ** -9,
+             0.0: 0.0}
+    for x, want in cases.items():
+        assert oracle.e4m3_round(np.array([x]))[0] == want, x
+
+
+def test_row_quantisation_bounds():
+    x = rng.standard_normal((50, 128)) * np.exp(rng.uniform(-3, 3, (50, 1)))
+    x[3] = 0.0
+    y, s = oracle.quantize_rows_e4m3(x)
+    amax = np.abs(x).max(1)
+    np.testing.assert_allclose(s[amax > 0], amax[amax > 0] / 448.0, rtol=1e-15)
+    assert s[3] == 1.0 and np.all(y[3] == 0.0)
+    # the largest element of a row is exact; every element is within half a
+    # quantum of 3 mantissa bits (normal range) or 2^-10 * s (subnormal range)
+    for r in range(50):
+        j = np.argmax(np.abs(x[r]))
+        assert abs(y[r, j] - x[r, j]) <= 1e-12 * abs(x[r, j])
+        u = np.abs(x[r]) / s[r]
+        bound = np.where(u >= 2.0 ** -6, u * 2.0 ** -4, 2.0 ** -10) * s[r]
+        assert np.all(np.abs(y[r] - x[r]) <= bound * (1 + 1e-12))
+
+
+def test_fp8_indexer_equals_exact_indexer_on_representable_inputs():
+    # rows whose values lie on the e4m3 grid with a largest magnitude of 448
+    # quantise exactly (scale 1), so the FP8 indexer is the exact one
+    grid = np.unique(oracle.e4m3_round(np.linspace(-448, 448, 4001)))
+    nq, HI, cI, N, m = 5, 3, 16, 40, 4
+    qI = rng.choice(grid, (nq, HI, cI))
+    K = rng.choice(grid, (N, cI))
+    qI[..., 0] = 448.0
+    K[:, 0] = -448.0
+    w = rng.random((nq, HI))
+    pos = rng.integers(0, N * m, nq)
+    np.testing.assert_array_equal(oracle.index_scores_fp8(qI, w, K, pos, m), oracle.index_scores(qI, w, K, pos, m))
+    # and a common factor on every row changes only the scale
+    a = oracle.index_scores_fp8(qI * 0.01, w, K * 3.0, pos, m)
+    b = oracle.index_scores(qI, w, K, pos, m) * 0.03
+    np.testing.assert_allclose(a, b, rtol=1e-12)
+
+
+def test_topk_recall_by_hand():
+    assert oracle.topk_recall([[1, 2, 3, -1]], [[3, 2, 9, -1]]) == pytest.approx(2 / 3)
+    assert oracle.topk_recall([[0, 1], [5, 4]], [[1, 0], [4, 6]]) == pytest.approx(0.75)
