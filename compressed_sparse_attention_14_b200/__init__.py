@@ -132,6 +132,13 @@ def _nbytes(t: Optional[torch.Tensor]) -> int:
     return 0 if t is None else t.numel() * t.element_size()
 
 
+def _shape(t: Optional[torch.Tensor], want: tuple, name: str) -> None:
+    """The C entry points take bare pointers: a buffer of the wrong shape would
+    be read or written out of bounds, so shapes are checked here."""
+    if t is not None and tuple(t.shape) != tuple(want):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(want)}")
+
+
 def abi_version() -> int:
     return _lib.csa_abi_version()
 
@@ -225,6 +232,12 @@ def csa_compress_step(proj_new, state, bias, pos, cache, m: int):
     state ring (state [B, 2m, 4c] fp32, updated in place) and write the entry
     of every block the token at pos[b] closes into cache [B, Nmax, c]."""
     B, c4 = proj_new.shape
+    c = c4 // 4
+    _shape(state, (B, 2 * m, c4), "state")
+    _shape(bias, (2 * m, c), "bias")
+    _shape(pos, (B,), "pos")
+    if cache.dim() != 3 or cache.shape[0] != B or cache.shape[2] != c:
+        raise ValueError(f"cache has shape {tuple(cache.shape)}, expected ({B}, Nmax, {c})")
     _check(_lib.csa_compress_step(_ptr(proj_new), _ptr(state), _ptr(bias), _ptr(pos), B, c4 // 4, m, cache.shape[1],
                                   _ptr(cache), _mode(cache), _stream()))
     return cache
@@ -233,6 +246,12 @@ def csa_compress_step(proj_new, state, bias, pos, cache, m: int):
 def hca_compress_step(proj_new, state, bias, pos, cache, mp: int):
     """HCA: proj_new [B, 2c] fp32, state [B, mp, 2c] fp32, cache [B, Nmax, c]."""
     B, c2 = proj_new.shape
+    c = c2 // 2
+    _shape(state, (B, mp, c2), "state")
+    _shape(bias, (mp, c), "bias")
+    _shape(pos, (B,), "pos")
+    if cache.dim() != 3 or cache.shape[0] != B or cache.shape[2] != c:
+        raise ValueError(f"cache has shape {tuple(cache.shape)}, expected ({B}, Nmax, {c})")
     _check(_lib.hca_compress_step(_ptr(proj_new), _ptr(state), _ptr(bias), _ptr(pos), B, c2 // 2, mp, cache.shape[1],
                                   _ptr(cache), _mode(cache), _stream()))
     return cache
@@ -245,6 +264,16 @@ def csa_decode_compress(x_new, W_kv, B_kv, W_idx, B_idx, pos, state_kv, state_id
     B, d = x_new.shape
     c = W_kv.shape[0] // 4
     cI = W_idx.shape[0] // 4
+    Nmax = kv_cache.shape[1]
+    _shape(W_kv, (4 * c, d), "W_kv")
+    _shape(W_idx, (4 * cI, d), "W_idx")
+    _shape(B_kv, (2 * m, c), "B_kv")
+    _shape(B_idx, (2 * m, cI), "B_idx")
+    _shape(pos, (B,), "pos")
+    _shape(state_kv, (B, 2 * m, 4 * c), "state_kv")
+    _shape(state_idx, (B, 2 * m, 4 * cI), "state_idx")
+    _shape(kv_cache, (B, Nmax, c), "kv_cache")
+    _shape(idx_cache, (B, Nmax, cI), "idx_cache")
     ws = _ws(_lib.csa_decode_compress_workspace_size(B, c, cI), x_new.device, ws)
     _check(_lib.csa_decode_compress(_ptr(x_new), _ptr(W_kv), _ptr(B_kv), _ptr(W_idx), _ptr(B_idx), _ptr(pos), B, d, m,
                                     c, cI, _ptr(state_kv), _ptr(state_idx), _ptr(kv_cache), _ptr(idx_cache),
@@ -398,6 +427,8 @@ def csa_norm_rope(x, pos=None, gamma=None, eps: float = 1e-6, rope_dims: int = 6
     sits at pos0 + g * pos_step. out may be x (in place)."""
     c = x.shape[-1]
     rows = x.numel() // c
+    _shape(gamma, (c,), "gamma")
+    _shape(out, tuple(x.shape), "out")
     if pos is not None:
         G = pos.numel()
         if G == 0 or rows % G:
@@ -444,6 +475,12 @@ def csa_attend_decode(qI, w, idx_cache, q, kv_cache, ctx_len, m: int, k: int, n_
         ring_len = kv_cache.shape[1] - Nmax
     if kv_cache.shape[1] != Nmax + ring_len:
         raise ValueError(f"kv_cache has {kv_cache.shape[1]} rows per sequence, Nmax + ring_len = {Nmax + ring_len}")
+    _shape(kv_cache, (B, Nmax + ring_len, c), "kv_cache")
+    _shape(idx_cache, (B, Nmax, cI), "idx_cache")
+    _shape(w, (B, HI), "w")
+    _shape(ctx_len, (B,), "ctx_len")
+    _shape(q_gamma, (c,), "q_gamma")
+    _shape(sink, (H,), "sink")
     mode = _mode(q)
     out = torch.empty_like(q) if out is None else out
     if lse is None:

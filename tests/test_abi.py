@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import compressed_sparse_attention_14_b200 as csa
 
@@ -189,3 +190,26 @@ def test_workspace_sizes():
     # the prefill score block is bounded (query chunking) at long context
     big = L.csa_prefill_workspace_size(65536, 65536, 4096, 4, 512, 128, 64, 64, 512, csa.CSA_BF16)
     assert big < 8 * (1 << 30)
+
+
+def test_bindings_check_buffer_shapes_before_the_call():
+    # buffers the C calls only see as pointers: a wrong shape is refused in
+    # the binding before anything reaches the library (CPU tensors suffice)
+    B, m, c = 4, 4, 64
+    f32 = dict(dtype=torch.float32)
+    with pytest.raises(ValueError, match="state"):
+        csa.csa_compress_step(torch.zeros(B, 4 * c, **f32), torch.zeros(B, m, 4 * c, **f32),
+                              torch.zeros(2 * m, c, **f32), torch.zeros(B, dtype=torch.int32),
+                              torch.zeros(B, 8, c, dtype=torch.bfloat16), m)
+    with pytest.raises(ValueError, match="cache"):
+        csa.hca_compress_step(torch.zeros(B, 2 * c, **f32), torch.zeros(B, 128, 2 * c, **f32),
+                              torch.zeros(128, c, **f32), torch.zeros(B, dtype=torch.int32),
+                              torch.zeros(B, 8, c + 8, dtype=torch.bfloat16), 128)
+    with pytest.raises(ValueError, match="gamma"):
+        csa.csa_norm_rope(torch.zeros(3, 2, c, dtype=torch.bfloat16), torch.zeros(3, dtype=torch.int32),
+                          gamma=torch.ones(c // 2, **f32))
+    with pytest.raises(ValueError, match="q_gamma"):
+        csa.csa_attend_decode(torch.zeros(B, 8, 64, dtype=torch.bfloat16), torch.zeros(B, 8, **f32),
+                              torch.zeros(B, 16, 64, dtype=torch.bfloat16), torch.zeros(B, 2, 128, dtype=torch.bfloat16),
+                              torch.zeros(B, 16 + 8, 128, dtype=torch.bfloat16), torch.zeros(B, dtype=torch.int32), 4, 4,
+                              n_win=8, q_gamma=torch.ones(64, **f32))
