@@ -1,14 +1,14 @@
 """Each plausible mistake in the oracle must fail at least one pin.
 
 A mutation is planted in a temporary copy of oracle/csa_oracle.c (CPU only),
-built with gcc, loaded in place of the real oracle, and the pin suite is run
-against it; the test passes when some pin fails. The real oracle is restored
-afterwards.
+built with gcc, loaded in place of the real oracle (which is never touched),
+and the pin suite is run against it; the test passes when some pin fails.
+The mutants run several at a time, each in its own process.
 """
+import concurrent.futures as cf
 import os
-import shutil
 import subprocess
-import tempfile
+import sys
 
 import pytest
 
@@ -39,8 +39,8 @@ MUTATIONS = [
     ("sink added to the numerator set twice", "if (sink) den += exp(sink[h] - mx);",
      "if (sink) den += 2.0 * exp(sink[h] - mx);"),
     ("dense MQA sees its own block", "int64_t vis = pos[t] / mp;", "int64_t vis = pos[t] / mp + 1;"),
-    ("bf16 rounding truncates", "double r = ldexp(round_half_even(ldexp(a, -q)), q);",
-     "double r = ldexp(floor(ldexp(a, -q)), q);"),
+    ("bf16 rounding truncates", "double r = ldexp(round_half_even(ldexp(a, -q)), q);\n    /* largest finite bf16",
+     "double r = ldexp(floor(ldexp(a, -q)), q);\n    /* largest finite bf16"),
     ("projection loops use a transposed W index", "X[t * d + k] * W[o * d + k]",
      "X[t * d + k] * W[(k * M + o) % (M * d)]"),
     ("RMSNorm over the sum of squares instead of the mean", "sqrt(ss / c + eps)", "sqrt(ss + eps)"),
@@ -66,17 +66,39 @@ MUTATIONS = [
 ]
 
 
-@pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
-def test_pins_catch_mutation(name, old, new, tmp_path):
+def _run_mutant(name, old, new, workdir):
+    """Build one mutant and run the pin suite against it; returns (anchor
+    found once, pin suite exit code, tail of its output)."""
     src = open(SRC).read()
-    assert src.count(old) == 1, f"mutation anchor not unique/present: {old!r}"
-    mutated = tmp_path / "mut.c"
-    mutated.write_text(src.replace(old, new))
-    lib = tmp_path / "libmut.so"
-    subprocess.check_call(["gcc", "-O1", "-fopenmp", "-std=c11", "-shared", "-fPIC", "-o", str(lib),
-                           str(mutated), "-lm"])
+    if src.count(old) != 1:
+        return False, None, ""
+    d = os.path.join(workdir, "m%d" % [m[0] for m in MUTATIONS].index(name))
+    os.makedirs(d, exist_ok=True)
+    mutated = os.path.join(d, "mut.c")
+    with open(mutated, "w") as f:
+        f.write(src.replace(old, new))
+    lib = os.path.join(d, "libmut.so")
+    subprocess.check_call(["gcc", "-O1", "-fopenmp", "-std=c11", "-shared", "-fPIC", "-o", lib, mutated, "-lm"])
     pins = os.path.join(os.path.dirname(__file__), "test_oracle_pins.py")
-    env = dict(os.environ, CSA_ORACLE_LIB=str(lib))
-    r = subprocess.run(["python", "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider", pins],
+    env = dict(os.environ, CSA_ORACLE_LIB=lib, OMP_NUM_THREADS="2")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider", pins],
                        env=env, capture_output=True, text=True, timeout=600)
-    assert r.returncode != 0, f"no pin failed for mutation '{name}'\n{r.stdout[-2000:]}"
+    return True, r.returncode, r.stdout[-2000:]
+
+
+@pytest.fixture(scope="module")
+def mutant_results(tmp_path_factory):
+    """Every mutant's pin-suite run, several at a time (each is an
+    independent process on its own copy of the oracle)."""
+    workdir = str(tmp_path_factory.mktemp("mutants"))
+    workers = max(1, min(8, (os.cpu_count() or 2) // 2))
+    with cf.ThreadPoolExecutor(workers) as ex:
+        futs = {m[0]: ex.submit(_run_mutant, *m, workdir) for m in MUTATIONS}
+        return {name: f.result() for name, f in futs.items()}
+
+
+@pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_pins_catch_mutation(name, old, new, mutant_results):
+    found, rc, tail = mutant_results[name]
+    assert found, f"mutation anchor not unique/present: {old!r}"
+    assert rc != 0, f"no pin failed for mutation '{name}'\n{tail}"
