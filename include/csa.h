@@ -7,11 +7,13 @@
  * Sources, cited by page title and section:
  *   [Notes] "DeepSeek-V4: 迈向高效百万级上下文智能" — study notes on the
  *           DeepSeek-V4 report (notes.kuangjux.top): §1.1 CSA (compressor and
- *           indexer equations), §1.2 HCA (comparison table), §1.3 (sink
- *           equation), model configuration table.
+ *           indexer equations), §1.2 HCA (comparison table), §1.3 (partial
+ *           RoPE, sliding window, sink equation, mixed-precision storage),
+ *           §2.6 Fig. 6 (state cache), model configuration table.
  *   [Walk]  mlpod.com walk-through of "DeepSeek-V4: Towards Highly Efficient
  *           Million-Token Context Intelligence": §2.3.1 CSA, §2.3.2 HCA and
- *           MQA, §2.3.3 attention details (causality, sink).
+ *           MQA, §2.3.3 attention details (query/KV RMSNorm, partial RoPE,
+ *           sliding window, sink; causality), §5 item 2 (state cache).
  *
  * Conventions shared by every call
  * --------------------------------
