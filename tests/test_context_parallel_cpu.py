@@ -128,3 +128,81 @@ def test_chunk_layout():
     sys.path.insert(0, ROOT)
     from compressed_sparse_attention_14_b200.context_parallel import chunk_layout
     assert chunk_layout(32, [24, 16, 8], 4) == [(32, 8), (56, 14), (72, 18)]
+
+
+def _subgroup_main(rank, world, port, out_dir, start, sizes):
+    # ranks 1 and 2 form the context-parallel group; rank 0 only takes part in
+    # creating it (every rank must call new_group)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import datetime
+    import torch.distributed as dist
+    from compressed_sparse_attention_14_b200 import context_parallel as cp
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    group = dist.new_group([1, 2])
+    if rank > 0:
+        inp = _inputs(start, sum(sizes))
+        r = rank - 1
+        lo = sum(sizes[:r])
+        hi = lo + sizes[r]
+        ops, _ = _oracle_ops()
+        out, lse = cp.csa_prefill_context_parallel(
+            inp["x"][lo:hi].contiguous(), inp["x_left"] if r == 0 else None, inp["W_kv"], inp["B_kv"], inp["W_idx"],
+            inp["B_idx"], start, inp["kv"], inp["ik"], inp["qI"][lo:hi].contiguous(), inp["w"][lo:hi].contiguous(),
+            inp["q"][lo:hi].contiguous(), K, m=M, scale=C ** -0.5, sink=inp["sink"], group=group, ops=ops)
+        torch.save(dict(out=out, lse=lse, kv=inp["kv"]), os.path.join(out_dir, f"rank{r}.pt"))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_context_parallel_on_a_subgroup(tmp_path):
+    start, sizes = 32, [16, 24]
+    mp.start_processes(_subgroup_main, args=(3, _free_port(), str(tmp_path), start, sizes), nprocs=3, join=True,
+                       start_method="spawn")
+    inp = _inputs(start, sum(sizes))
+    _, prefill = _oracle_ops()
+    ref_o, ref_l = prefill(inp["x"], inp["x_left"], inp["W_kv"], inp["B_kv"], inp["W_idx"], inp["B_idx"], start,
+                           inp["kv"], inp["ik"], inp["qI"], inp["w"], inp["q"], K, M, C ** -0.5, inp["sink"])
+    lo = 0
+    for r, n in enumerate(sizes):
+        got = torch.load(tmp_path / f"rank{r}.pt")
+        assert torch.equal(got["kv"], inp["kv"]) and torch.equal(got["out"], ref_o[lo:lo + n])
+        lo += n
+
+
+def _absent_peer_main(rank, world, port, out_dir):
+    # rank 1 leaves before the prefill; rank 0's first collective must end
+    # with an error (peer gone or the short group timeout), not wait forever
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import datetime
+    import time
+    import torch.distributed as dist
+    from compressed_sparse_attention_14_b200 import context_parallel as cp
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        os._exit(0)
+    inp = _inputs(0, 16)
+    ops, _ = _oracle_ops()
+    t0 = time.time()
+    res = {}
+    try:
+        cp.csa_prefill_context_parallel(inp["x"][:8].contiguous(), None, inp["W_kv"], inp["B_kv"], inp["W_idx"],
+                                        inp["B_idx"], 0, inp["kv"], inp["ik"], inp["qI"][:8].contiguous(),
+                                        inp["w"][:8].contiguous(), inp["q"][:8].contiguous(), K, m=M, ops=ops)
+        res["raised"] = False
+    except Exception as e:  # noqa: BLE001 - any error ends the wait; the test checks that one came
+        res["raised"] = True
+        res["error"] = type(e).__name__
+    res["seconds"] = time.time() - t0
+    with open(os.path.join(out_dir, "rank0.json"), "w") as f:
+        json.dump(res, f)
+    os._exit(0)
+
+
+def test_absent_peer_ends_with_an_error(tmp_path):
+    mp.start_processes(_absent_peer_main, args=(2, _free_port(), str(tmp_path)), nprocs=2, join=True,
+                       start_method="spawn")
+    res = json.load(open(tmp_path / "rank0.json"))
+    assert res["raised"], res
+    assert res["seconds"] < 60, res
