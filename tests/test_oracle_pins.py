@@ -678,3 +678,22 @@ def test_fp8_indexer_equals_exact_indexer_on_representable_inputs():
 def test_topk_recall_by_hand():
     assert oracle.topk_recall([[1, 2, 3, -1]], [[3, 2, 9, -1]]) == pytest.approx(2 / 3)
     assert oracle.topk_recall([[0, 1], [5, 4]], [[1, 0], [4, 6]]) == pytest.approx(0.75)
+
+
+def test_fp8_scales_factor_out_of_the_relu():
+    # positive row scales commute with the ReLU, so the FP8 indexer can run on
+    # raw e4m3 codes: I = s_k * sum_h (w_h s_q,h) ReLU(codes_q,h . codes_k)
+    nq, HI, cI, N, m = 4, 3, 32, 30, 4
+    qI = rng.standard_normal((nq, HI, cI)) * 3.0
+    K = rng.standard_normal((N, cI)) * 0.2
+    w = rng.random((nq, HI))
+    pos = rng.integers(m, N * m, nq)
+    q8, sq = oracle.quantize_rows_e4m3(qI)
+    k8, sk = oracle.quantize_rows_e4m3(K)
+    codes_q, codes_k = q8 / sq[..., None], k8 / sk[:, None]
+    assert np.all(np.abs(codes_q) <= 448) and np.all(oracle.e4m3_round(codes_k) == codes_k)
+    direct = oracle.index_scores_fp8(qI, w, K, pos, m)
+    factored = oracle.index_scores(codes_q, w * sq, codes_k, pos, m) * sk[None, :]
+    vis = np.isfinite(direct)
+    assert np.array_equal(vis, np.isfinite(factored))
+    np.testing.assert_allclose(factored[vis], direct[vis], rtol=1e-12, atol=1e-12)
