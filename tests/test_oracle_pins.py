@@ -690,8 +690,13 @@ def test_fp8_scales_factor_out_of_the_relu():
     pos = rng.integers(m, N * m, nq)
     q8, sq = oracle.quantize_rows_e4m3(qI)
     k8, sk = oracle.quantize_rows_e4m3(K)
-    codes_q, codes_k = q8 / sq[..., None], k8 / sk[:, None]
-    assert np.all(np.abs(codes_q) <= 448) and np.all(oracle.e4m3_round(codes_k) == codes_k)
+    # the codes: dequantised values over their scales, on the e4m3 grid up to
+    # the rounding of that division
+    codes_q = oracle.e4m3_round(q8 / sq[..., None])
+    codes_k = oracle.e4m3_round(k8 / sk[:, None])
+    np.testing.assert_allclose(codes_q, q8 / sq[..., None], rtol=1e-14)
+    np.testing.assert_allclose(codes_k, k8 / sk[:, None], rtol=1e-14)
+    assert np.abs(codes_q).max() == 448.0 and np.abs(codes_k).max() == 448.0
     direct = oracle.index_scores_fp8(qI, w, K, pos, m)
     factored = oracle.index_scores(codes_q, w * sq, codes_k, pos, m) * sk[None, :]
     vis = np.isfinite(direct)
