@@ -692,6 +692,22 @@ def oracle_measure(workload: str, budget_s: float = 15.0):
     return units / sec, desc, units, sec
 
 
+def cpu_baseline_for(workload: str, unit: str) -> dict:
+    """The oracle timed on the host at all its threads (the reported value)
+    and on one thread (single_core), each on a bounded sample."""
+    import oracle
+    threads = cpu_oracle_threads()
+    cps, desc, _, _ = oracle_measure(workload)
+    out = {"value": cps, "unit": unit, "cores": threads, "kind": "oracle", "sample": desc}
+    oracle.set_num_threads(1)
+    try:
+        cps1, desc1, _, _ = oracle_measure(workload, budget_s=6.0)
+    finally:
+        oracle.set_num_threads(threads)
+    out["single_core"] = {"value": cps1, "unit": unit, "cores": 1, "sample": desc1}
+    return out
+
+
 # ----------------------------------------------------------------------------
 # main
 # ----------------------------------------------------------------------------
@@ -851,9 +867,7 @@ def run_ours(args, rank, world, local):
     del wl
     torch.cuda.empty_cache()
     if rank == 0 and not args.no_cpu_baseline:
-        cps, desc, _, _ = oracle_measure(args.workload)
-        line["cpu_baseline"] = {"value": cps, "unit": line["unit"], "cores": cpu_oracle_threads(),
-                                "kind": "oracle", "sample": desc}
+        line["cpu_baseline"] = cpu_baseline_for(args.workload, line["unit"])
     if rank == 0:
         print(json.dumps(line), flush=True)
     dist_done(world)

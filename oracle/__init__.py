@@ -69,6 +69,7 @@ def _load():
             lib.orc_norm_rope.argtypes = [_D, i64, i32, i32, _D, dbl, i32, dbl, _I32, i32, _D]
             lib.orc_window_entries.argtypes = [_I32, i32, i32, i64, i64, _I32]
             lib.orc_num_threads.restype = i32
+            lib.orc_set_num_threads.argtypes = [i32]
             _lib = lib
     return _lib
 
@@ -104,6 +105,11 @@ def _p(a: np.ndarray | None):
 
 def num_threads() -> int:
     return int(_load().orc_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads for the oracle's parallel loops from now on (this thread)."""
+    _load().orc_set_num_threads(int(n))
 
 
 def bf16_round(x) -> np.ndarray:

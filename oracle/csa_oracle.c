@@ -441,3 +441,14 @@ int orc_num_threads(void) {
     return 1;
 #endif
 }
+
+/* Threads for the oracle's later parallel loops (the CPU baseline is timed
+   at all cores and at one). */
+void orc_set_num_threads(int n) {
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    omp_set_num_threads(n > 0 ? n : 1);
+#else
+    (void)n;
+#endif
+}
