@@ -18,7 +18,7 @@
  *            Million-Token Context Intelligence" (its inline formulas were
  *            stripped; the prose still fixes the semantics).
  *
- * Readings taken where the pages are silent (each is listed in the design doc):
+ * Readings taken where the pages are silent:
  *   - the four compressor maps are bias-free linear maps d -> c;
  *   - ONE softmax per (block, channel) over all 2m window logits (a-part and
  *     b-part together), so the weights sum to 1;
