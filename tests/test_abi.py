@@ -4,6 +4,7 @@ bad arguments before touching the device, and sizes its workspaces."""
 import ctypes
 import os
 import re
+import subprocess
 
 import pytest
 import torch
@@ -213,3 +214,22 @@ def test_bindings_check_buffer_shapes_before_the_call():
                               torch.zeros(B, 16, 64, dtype=torch.bfloat16), torch.zeros(B, 2, 128, dtype=torch.bfloat16),
                               torch.zeros(B, 16 + 8, 128, dtype=torch.bfloat16), torch.zeros(B, dtype=torch.int32), 4, 4,
                               n_win=8, q_gamma=torch.ones(64, **f32))
+
+
+def test_header_is_plain_c_and_the_library_links_from_c(tmp_path):
+    # the boundary is a C ABI: a C program includes csa.h, links libcsa.so
+    # and calls into it (host-only calls: no GPU is touched)
+    src = tmp_path / "use_csa.c"
+    src.write_text(
+        '#include <stdio.h>\n#include "csa.h"\n'
+        "int main(void) {\n"
+        "    int rc = csa_compress(NULL, NULL, NULL, 6, 8, 4, NULL, CSA_BF16, NULL);\n"
+        '    printf("%d %d %s\\n", csa_abi_version(), rc, csa_last_error());\n'
+        "    return rc == CSA_ERR_INVALID_ARG ? 0 : 1;\n}\n")
+    exe = tmp_path / "use_csa"
+    libdir = os.path.dirname(csa.LIB_PATH)
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
+                           "-o", str(exe), "-L", libdir, "-lcsa", "-Wl,-rpath," + libdir])
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stdout + out.stderr
+    assert out.stdout.startswith(f"{csa.abi_version()} {csa.CSA_ERR_INVALID_ARG} ")
