@@ -866,7 +866,7 @@ def run_ours(args, rank, world, local):
                                  "frac": sb / peaks["hbm_gbs"]}
     del wl
     torch.cuda.empty_cache()
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_for(args.workload, line["unit"])
     if rank == 0:
         print(json.dumps(line), flush=True)
