@@ -208,7 +208,7 @@ int csa_poll_status(void* stream, int reset) {
 // ---------------------------------------------------------------- a1
 int csa_project(const void* x, const void* W, int64_t n, int d, int M, float* out, int dtype,
                 void* stream) {
-    ElemType t;
+    ElemType t = ElemType::BF16;   // set by check_dtype
     CSA_TRY(check_dtype(dtype, &t));
     if (n < 0 || d < 8 || d % 8 || M < 8 || M % 8)
         return fail(CSA_ERR_INVALID_ARG, "csa_project: need n>=0, d and M multiples of 8 (n=%lld d=%d M=%d)",
@@ -231,7 +231,7 @@ static int check_compress(int64_t n, int c, int m, int mmax, const char* who) {
 
 int csa_compress(const void* proj, const void* left, const float* bias, int64_t n, int c, int m,
                  void* out, int dtype, void* stream) {
-    ElemType t;
+    ElemType t = ElemType::BF16;   // set by check_dtype
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_compress(n, c, m, 64, "csa_compress"));
     if (n == 0) return CSA_OK;
@@ -245,7 +245,7 @@ int csa_compress(const void* proj, const void* left, const float* bias, int64_t 
 
 int hca_compress(const void* proj, const float* bias, int64_t n, int c, int mp, void* out,
                  int dtype, void* stream) {
-    ElemType t;
+    ElemType t = ElemType::BF16;   // set by check_dtype
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_compress(n, c, mp, 1024, "hca_compress"));
     if (n == 0) return CSA_OK;
@@ -259,7 +259,7 @@ int hca_compress(const void* proj, const float* bias, int64_t n, int c, int mp, 
 static int compress_step_common(const float* proj_new, float* state, const float* bias, const int32_t* pos, int B,
                                 int c, int m, int mmax, int64_t Nmax, void* cache, int dtype, bool overlap,
                                 void* stream, const char* who) {
-    ElemType t;
+    ElemType t = ElemType::BF16;   // set by check_dtype
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_compress(0, c, m, mmax, who));
     if (B < 0 || Nmax < 0) return fail(CSA_ERR_INVALID_ARG, "%s: bad B/Nmax", who);
@@ -294,7 +294,7 @@ int csa_decode_compress(const void* x_new, const void* W_kv, const float* B_kv, 
                         const int32_t* pos, int B, int d, int m, int c, int cI, float* state_kv, float* state_idx,
                         void* kv_cache, void* idx_cache, int64_t Nmax, void* ws, size_t ws_bytes, int dtype,
                         void* stream) {
-    ElemType t;
+    ElemType t = ElemType::BF16;   // set by check_dtype
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_compress(0, c, m, 64, "csa_decode_compress"));
     CSA_TRY(check_compress(0, cI, m, 64, "csa_decode_compress"));
@@ -333,7 +333,7 @@ size_t csa_compress_from_hidden_workspace_size(int64_t n, int d, int c, int m, i
 int csa_compress_from_hidden(const void* x, const void* x_left, const void* W, const float* bias,
                              int64_t n, int d, int c, int m, void* out, void* ws, size_t ws_bytes,
                              int dtype, void* stream) {
-    ElemType t;
+    ElemType t = ElemType::BF16;   // set by check_dtype
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_compress(n, c, m, 64, "csa_compress_from_hidden"));
     if (d < 8 || d % 8) return fail(CSA_ERR_INVALID_ARG, "d=%d must be a positive multiple of 8", d);
@@ -364,7 +364,7 @@ size_t hca_compress_from_hidden_workspace_size(int64_t n, int d, int c, int mp, 
 int hca_compress_from_hidden(const void* x, const void* W, const float* bias, int64_t n, int d,
                              int c, int mp, void* out, void* ws, size_t ws_bytes, int dtype,
                              void* stream) {
-    ElemType t;
+    ElemType t = ElemType::BF16;   // set by check_dtype
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_compress(n, c, mp, 1024, "hca_compress_from_hidden"));
     if (d < 8 || d % 8) return fail(CSA_ERR_INVALID_ARG, "d=%d must be a positive multiple of 8", d);
@@ -385,7 +385,7 @@ int hca_compress_from_hidden(const void* x, const void* W, const float* bias, in
 int csa_index_scores(const void* qI, const float* w, const void* K, const int32_t* pos,
                      const int32_t* seq_of_q, int nq, int n_seq, int HI, int cI, int64_t Nmax, int m,
                      float* scores, int dtype, void* stream) {
-    ElemType t;
+    ElemType t = ElemType::BF16;   // set by check_dtype
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_index_shape(HI, cI));
     CSA_TRY(check_index_mode(HI, cI, t));
@@ -441,7 +441,7 @@ int csa_index_topk(const void* qI, const float* w, const void* K, const int32_t*
                    const int32_t* seq_of_q, int nq, int n_seq, int HI, int cI, int64_t Nmax, int m, int k,
                    int32_t* idx, float* top_scores, void* ws, size_t ws_bytes, int dtype,
                    void* stream) {
-    ElemType t;
+    ElemType t = ElemType::BF16;   // set by check_dtype
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_index_shape(HI, cI));
     CSA_TRY(check_index_mode(HI, cI, t));
@@ -479,7 +479,7 @@ size_t csa_sparse_mqa_workspace_size(int nq, int H, int c, int k, int dtype) {
 int csa_sparse_mqa(const void* q, const void* KV, const int32_t* idx, const int32_t* seq_of_q,
                    int nq, int n_seq, int H, int c, int64_t Nmax, int k, float scale, const float* sink,
                    void* out, float* lse, void* ws, size_t ws_bytes, int dtype, void* stream) {
-    ElemType t;
+    ElemType t = ElemType::BF16;   // set by check_dtype
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_attn_shape(H, c));
     CSA_TRY(check_attn_mode(H, c, t));
@@ -512,7 +512,7 @@ size_t hca_dense_mqa_workspace_size(int nq, int H, int c, int64_t Nmax, int dtyp
 int hca_dense_mqa(const void* q, const void* KV, const int32_t* pos, const int32_t* seq_of_q,
                   int nq, int n_seq, int H, int c, int64_t Nmax, int mp, float scale, const float* sink,
                   void* out, float* lse, void* ws, size_t ws_bytes, int dtype, void* stream) {
-    ElemType t;
+    ElemType t = ElemType::BF16;   // set by check_dtype
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_attn_shape(H, c));
     CSA_TRY(check_attn_mode(H, c, t));
@@ -549,7 +549,7 @@ int csa_decode(const void* qI, const float* w, const void* idx_cache, const void
                const void* kv_cache, const int32_t* ctx_len, int B, int64_t Nmax, int m, int H,
                int c, int HI, int cI, int k, float scale, const float* sink, void* out, float* lse,
                int32_t* topk_idx, void* ws, size_t ws_bytes, int dtype, void* stream) {
-    ElemType t;
+    ElemType t = ElemType::BF16;   // set by check_dtype
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_index_shape(HI, cI));
     CSA_TRY(check_index_mode(HI, cI, t));
@@ -617,7 +617,7 @@ int csa_prefill(const void* x, const void* x_left, const void* W_kv, const float
                 const float* w, const void* q, int H, int HI, int k, float scale,
                 const float* sink, void* out, float* lse, int32_t* topk_idx, void* ws,
                 size_t ws_bytes, int dtype, void* stream) {
-    ElemType t;
+    ElemType t = ElemType::BF16;   // set by check_dtype
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_index_shape(HI, cI));
     CSA_TRY(check_index_mode(HI, cI, t));
@@ -715,7 +715,7 @@ static int check_window(int n_win, int64_t ring_off, int64_t ring_len) {
 int csa_norm_rope(const void* x, void* y, int64_t rows, int group, int c, const float* gamma, float eps,
                   int rope_dims, float rope_base, const int32_t* pos, int64_t pos0, int64_t pos_step, int inverse,
                   int dtype, void* stream) {
-    ElemType t;
+    ElemType t = ElemType::BF16;   // set by check_dtype
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_norm_rope(c, rope_dims, rope_base, eps));
     if (rows < 0 || group < 1 || rows % group)
@@ -767,7 +767,7 @@ int csa_attend_decode(const void* qI, const float* w, const void* idx_cache, con
                       int HI, int cI, int k, float scale, const float* q_gamma, float eps, int rope_dims,
                       float rope_base, const float* sink, void* out, float* lse, int32_t* topk_idx, void* ws,
                       size_t ws_bytes, int dtype, void* stream) {
-    ElemType t;
+    ElemType t = ElemType::BF16;   // set by check_dtype
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_index_shape(HI, cI));
     CSA_TRY(check_index_mode(HI, cI, t));
