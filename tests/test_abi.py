@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 import subprocess
+import sys
 
 import pytest
 import torch
@@ -233,3 +234,20 @@ def test_header_is_plain_c_and_the_library_links_from_c(tmp_path):
     out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert out.returncode == 0, out.stdout + out.stderr
     assert out.stdout.startswith(f"{csa.abi_version()} {csa.CSA_ERR_INVALID_ARG} ")
+
+
+def test_no_cpu_path(tmp_path):
+    # without the built library the package refuses to import, and with it
+    # every compute call refuses host tensors: there is no CPU fallback
+    pkg = os.path.dirname(csa.__file__)
+    copy = tmp_path / "compressed_sparse_attention_14_b200"
+    copy.mkdir()
+    for name in ("__init__.py", "context_parallel.py"):
+        (copy / name).write_text(open(os.path.join(pkg, name)).read())
+    r = subprocess.run([sys.executable, "-c", "import compressed_sparse_attention_14_b200"], cwd=str(tmp_path),
+                       capture_output=True, text=True, timeout=120)
+    assert r.returncode != 0 and "ImportError" in r.stderr and "libcsa.so is missing" in r.stderr
+    x = torch.zeros(16, 64, dtype=torch.bfloat16)
+    W = torch.zeros(32, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensors only"):
+        csa.csa_project(x, W, out=torch.zeros(16, 32))
