@@ -251,3 +251,19 @@ def test_no_cpu_path(tmp_path):
     W = torch.zeros(32, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA tensors only"):
         csa.csa_project(x, W, out=torch.zeros(16, 32))
+
+
+def test_product_code_does_not_reach_the_oracle():
+    # the oracle is test infrastructure: the package and the CUDA sources
+    # neither import, include nor load it
+    pkg = os.path.dirname(csa.__file__)
+    offenders = []
+    for dirpath, _, files in os.walk(pkg):
+        if "_build" in dirpath:
+            continue
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".c")):
+                text = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                if re.search(r"^\s*(import oracle|from oracle)|csa_oracle|liboracle", text, flags=re.M):
+                    offenders.append(f)
+    assert not offenders, offenders
