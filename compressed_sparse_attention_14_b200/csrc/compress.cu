@@ -127,7 +127,9 @@ __global__ void __launch_bounds__(256) hca_compress_kernel(const TIn* __restrict
 // from the ring in exactly the order of the chunk kernels above (a-window,
 // then b-window), so a sequence compressed token by token gets the same
 // entries as one compressed in a chunk. A thread owns 8 channels of one
-// sequence: it reads back only ring values it wrote itself.
+// sequence and reads only the ring values of those channels, written by the
+// same thread slot in this step or an earlier one (an earlier launch has
+// completed before pdl_wait returns).
 template <typename TOut>
 __global__ void __launch_bounds__(256) csa_compress_step_kernel(const float* __restrict__ proj_new,
                                                                 float* __restrict__ state,
