@@ -18,6 +18,9 @@ query RMSNorm + partial rotary, the 128-token sliding window joined to the
 selection in one softmax with a sink, the output turned back by position),
 flash_decode_compress (one decode step's compression of both CSA streams
 through the per-sequence state cache, from the new tokens' hidden states).
+On one GPU the default line also carries "extra_workloads": Pro decode, the
+long prefill chunk, HCA decode and the HCA compressor, each measured the same
+way right after the Flash decode line (--no-extra skips them).
 
 Multi-GPU (under torchrun): every rank runs its own independent batch
 (decode queries are independent: no collective on the data path), the step
@@ -761,13 +764,17 @@ WORKLOADS_CONFIG_NAME = {
 }
 
 
-def run_ours(args, rank, world, local):
+def measure(name, args, rank, world, local, steps, warmup, batch=None):
+    """Time one workload: `warmup` untimed steps, then exactly `steps` steps
+    bracketed by barrier + synchronize, each step on the device with CUDA
+    events after an L2 flush; per-kernel times from a second, traced pass;
+    clocks sampled over the timed region; the end-to-end rate through the
+    public call with host buffers. Returns the workload's JSON fields."""
     import compressed_sparse_attention_14_b200 as csa
-    wl = WORKLOADS[args.workload](rank, args.batch)
+    wl = WORKLOADS[name](rank, batch)
     step, e2e_step = wl["step"], wl["e2e_step"]
 
-    # warm-up
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize()
 
@@ -779,7 +786,7 @@ def run_ours(args, rank, world, local):
     barrier(world)
     torch.cuda.synchronize()
     t_wall0 = time.perf_counter()
-    for _ in range(args.steps):
+    for _ in range(steps):
         timer.step(step)
     torch.cuda.synchronize()
     barrier(world)
@@ -792,7 +799,7 @@ def run_ours(args, rank, world, local):
     # library's kernel events on
     csa.trace_enable(True)
     ktimer = Timer()
-    for _ in range(args.steps):
+    for _ in range(steps):
         ktimer.step(step)
     ktimer.total_ms()
     trace = csa.trace_read()
@@ -808,7 +815,7 @@ def run_ours(args, rank, world, local):
     clk = clocks.stop()
     clk["window"] = f"timed region plus {soak_steps} untimed steps of the same work"
     ms_total_max = max_over_ranks(ms_total, world)
-    ms_step = ms_total_max / args.steps
+    ms_step = ms_total_max / steps
 
     # end to end: host buffers in, host result out, through the public call
     e2e_timer = Timer()
@@ -816,19 +823,18 @@ def run_ours(args, rank, world, local):
         e2e_step()
     torch.cuda.synchronize()
     barrier(world)
-    for _ in range(args.steps):
+    for _ in range(steps):
         e2e_timer.step(e2e_step)
-    e2e_ms = max_over_ranks(e2e_timer.total_ms(), world) / args.steps
+    e2e_ms = max_over_ranks(e2e_timer.total_ms(), world) / steps
 
     units = wl["units"]
-    value = job_rate(units, world, ms_step)
     peaks = measured_peaks()
 
-    def roofline_of(name):
-        info = wl["kernels"][name]
-        k_ms, k_n = trace.get(name, (float("nan"), 0))
+    def roofline_of(kname):
+        info = wl["kernels"][kname]
+        k_ms, k_n = trace.get(kname, (float("nan"), 0))
         avg_s = k_ms / max(k_n, 1) / 1e3
-        per_launch = info["work"] * args.steps / max(k_n, 1)   # the work is per step
+        per_launch = info["work"] * steps / max(k_n, 1)   # the work is per step
         if info["bound"] == "hbm":
             achieved = per_launch / avg_s / 1e9
             r = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -837,35 +843,57 @@ def run_ours(args, rank, world, local):
             achieved = per_launch / avg_s / 1e12
             r = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                  "frac": achieved / peaks["bf16_tflops"], "peak_source": peaks["source"] + " bf16_tflops (burst)"}
-        r["kernel"] = name
-        r["launches_per_step"] = k_n / args.steps
+        r["kernel"] = kname
+        r["launches_per_step"] = k_n / steps
         r["ms_per_launch"] = avg_s * 1e3
-        r["traffic"] = ncu_traffic(name, args.workload, info["files"])
+        r["traffic"] = ncu_traffic(kname, name, info["files"])
         return r
 
     timed = [n for n in wl["kernels"] if n in trace]
     dom = max(timed, key=lambda n: trace[n][0]) if timed else next(iter(wl["kernels"]))
-    roof = roofline_of(dom)
     others = {n: roofline_of(n) for n in timed if n != dom}
-
-    line = {"metric": METRIC, "value": value, "unit": wl["unit"], "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": wl["config"],
-            "roofline": roof,
-            "kernels_ms_per_step": {k: v[0] / args.steps for k, v in sorted(trace.items())},
-            "other_kernels_roofline": {n: {k: r[k] for k in ("bound", "achieved", "unit", "frac")}
-                                       for n, r in others.items()},
-            "e2e": {"value": job_rate(units, world, e2e_ms), "unit": wl["unit"], "h2d_bytes_per_step": wl["h2d"],
-                    "d2h_bytes_per_step": wl["d2h"]},
-            "gpu_launches": launches, "clocks": clk, "wall_s_timed": t_wall,
-            "kernel_times": "per-kernel CUDA events on the library's stream over a second pass of the same steps "
-                            "(the timed region itself runs without them)"}
+    out = {"value": job_rate(units, world, ms_step), "unit": wl["unit"], "ms_per_step": ms_step, "steps": steps,
+           "warmup": warmup, "config": wl["config"], "roofline": roofline_of(dom),
+           "kernels_ms_per_step": {k: v[0] / steps for k, v in sorted(trace.items())},
+           "other_kernels_roofline": {n: {k: r[k] for k in ("bound", "achieved", "unit", "frac")}
+                                      for n, r in others.items()},
+           "e2e": {"value": job_rate(units, world, e2e_ms), "unit": wl["unit"], "h2d_bytes_per_step": wl["h2d"],
+                   "d2h_bytes_per_step": wl["d2h"]},
+           "gpu_launches": launches, "clocks": clk, "wall_s_timed": t_wall}
     if wl.get("step_bytes"):
         sb = wl["step_bytes"] / (ms_step / 1e3) / 1e9
-        line["step_roofline"] = {"bound": "hbm", "achieved": sb, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                 "frac": sb / peaks["hbm_gbs"]}
-    del wl
+        out["step_roofline"] = {"bound": "hbm", "achieved": sb, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                "frac": sb / peaks["hbm_gbs"]}
+    del wl, step, e2e_step
+    torch.cuda.synchronize()
     torch.cuda.empty_cache()
+    return out
+
+
+# Measured after the default (Flash decode) line on one GPU and reported in
+# its "extra_workloads": the other workloads the metric names (Pro-shaped
+# 1M-context decode, the long prefill chunk, HCA decode, the HCA compressor).
+# Each keeps its own step count, at most the headline's.
+EXTRA_WORKLOADS = {"pro_decode": 20, "prefill": 5, "hca_decode": 20, "hca_compress": 10}
+
+
+def run_ours(args, rank, world, local):
+    m = measure(args.workload, args, rank, world, local, args.steps, args.warmup, args.batch)
+    line = {"metric": METRIC, "value": m["value"], "unit": m["unit"], "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": m["config"],
+            "roofline": m["roofline"]}
+    for k in ("kernels_ms_per_step", "other_kernels_roofline", "e2e", "gpu_launches", "clocks", "wall_s_timed",
+              "step_roofline"):
+        if k in m:
+            line[k] = m[k]
+    line["kernel_times"] = ("per-kernel CUDA events on the library's stream over a second pass of the same steps "
+                            "(the timed region itself runs without them)")
+    if world == 1 and args.workload == "flash_decode" and args.batch is None and not args.no_extra:
+        extra = {}
+        for name, cap in EXTRA_WORKLOADS.items():
+            extra[name] = measure(name, args, rank, world, local, min(args.steps, cap), min(args.warmup, 3))
+        line["extra_workloads"] = extra
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_for(args.workload, line["unit"])
     if rank == 0:
@@ -881,6 +909,8 @@ def main():
     ap.add_argument("--workload", default="flash_decode", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="default workload only: skip the extra_workloads (Pro decode, prefill, HCA) measured after it")
     ap.add_argument("--batch", type=int, default=None,
                     help="decode workloads: only the first N queries; prefill: only the last N tokens of the "
                          "chunk, a multiple of m (small profiling cases)")

@@ -67,8 +67,10 @@ _SIGS = {
     "hca_decode_workspace_size": (_SZ, [_I, _I64, _I, _I, _I]),
     "hca_decode": (_I, [_P, _P, _P, _I, _I64, _I, _I, _I, _F, _P, _P, _P, _P, _SZ, _I, _P]),
     "csa_prefill_workspace_size": (_SZ, [_I64, _I64, _I, _I, _I, _I, _I, _I, _I, _I]),
-    "csa_prefill": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I, _I, _I, _I, _P, _P, _I64, _P, _P, _P,
+    "csa_prefill": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I, _I, _I, _I, _P, _P, _I64, _P, _P, _P, _P, _P,
                          _I, _I, _I, _F, _P, _P, _P, _P, _P, _SZ, _I, _P]),
+    "csa_compress_chunk": (_I, [_P, _P, _P, _I64, _I64, _I, _I, _P, _I64, _I, _P]),
+    "hca_compress_chunk": (_I, [_P, _P, _P, _I64, _I64, _I, _I, _P, _I64, _I, _P]),
     "csa_compress_step": (_I, [_P, _P, _P, _P, _I, _I, _I, _I64, _P, _I, _P]),
     "hca_compress_step": (_I, [_P, _P, _P, _P, _I, _I, _I, _I64, _P, _I, _P]),
     "csa_decode_compress_workspace_size": (_SZ, [_I, _I, _I]),
@@ -137,6 +139,11 @@ def _shape(t: Optional[torch.Tensor], want: tuple, name: str) -> None:
     be read or written out of bounds, so shapes are checked here."""
     if t is not None and tuple(t.shape) != tuple(want):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(want)}")
+
+
+def _dtype(t: Optional[torch.Tensor], want: torch.dtype, name: str) -> None:
+    if t is not None and t.dtype != want:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {want}")
 
 
 def abi_version() -> int:
@@ -254,6 +261,39 @@ def hca_compress_step(proj_new, state, bias, pos, cache, mp: int):
         raise ValueError(f"cache has shape {tuple(cache.shape)}, expected ({B}, Nmax, {c})")
     _check(_lib.hca_compress_step(_ptr(proj_new), _ptr(state), _ptr(bias), _ptr(pos), B, c2 // 2, mp, cache.shape[1],
                                   _ptr(cache), _mode(cache), _stream()))
+    return cache
+
+
+def csa_compress_chunk(proj, state, bias, start: int, cache, m: int):
+    """Compress tokens start .. start+n-1 of one sequence (proj [n, 4c] fp32)
+    at any start and length: writes the entry of every block ending inside
+    the chunk into cache [Nmax, c], earlier window tokens from the state ring
+    (state [2m, 4c] fp32, updated in place to the last 2m tokens)."""
+    n, c4 = proj.shape
+    c = c4 // 4
+    _dtype(proj, torch.float32, "proj")
+    _dtype(state, torch.float32, "state")
+    _shape(state, (2 * m, c4), "state")
+    _shape(bias, (2 * m, c), "bias")
+    if cache.dim() != 2 or cache.shape[1] != c:
+        raise ValueError(f"cache has shape {tuple(cache.shape)}, expected (Nmax, {c})")
+    _check(_lib.csa_compress_chunk(_ptr(proj), _ptr(state), _ptr(bias), start, n, c, m, _ptr(cache), cache.shape[0],
+                                   _mode(cache), _stream()))
+    return cache
+
+
+def hca_compress_chunk(proj, state, bias, start: int, cache, mp: int):
+    """HCA: proj [n, 2c] fp32, state [mp, 2c] fp32, cache [Nmax, c]."""
+    n, c2 = proj.shape
+    c = c2 // 2
+    _dtype(proj, torch.float32, "proj")
+    _dtype(state, torch.float32, "state")
+    _shape(state, (mp, c2), "state")
+    _shape(bias, (mp, c), "bias")
+    if cache.dim() != 2 or cache.shape[1] != c:
+        raise ValueError(f"cache has shape {tuple(cache.shape)}, expected (Nmax, {c})")
+    _check(_lib.hca_compress_chunk(_ptr(proj), _ptr(state), _ptr(bias), start, n, c, mp, _ptr(cache), cache.shape[0],
+                                   _mode(cache), _stream()))
     return cache
 
 
@@ -397,7 +437,12 @@ def hca_decode(q, kv_cache, ctx_len, mp: int, scale: float = 0.0, sink=None, out
 
 
 def csa_prefill(x, x_left, W_kv, B_kv, W_idx, B_idx, start: int, kv_cache, idx_cache, qI, w, q, k: int,
-                m: int = 4, scale: float = 0.0, sink=None, out=None, ws=None, return_topk: bool = False):
+                m: int = 4, scale: float = 0.0, sink=None, out=None, ws=None, return_topk: bool = False,
+                state_kv=None, state_idx=None):
+    """One prefill chunk of one sequence. Without state rings the chunk starts
+    and ends on block boundaries (x_left: the m hidden rows before it). With
+    state_kv [2m, 4c] and state_idx [2m, 4cI] (fp32, updated in place) the
+    chunk may start and end anywhere; x_left is then ignored."""
     n, d = x.shape
     c = W_kv.shape[0] // 4
     cI = W_idx.shape[0] // 4
@@ -405,13 +450,20 @@ def csa_prefill(x, x_left, W_kv, B_kv, W_idx, B_idx, start: int, kv_cache, idx_c
     _, HI, _ = qI.shape
     Nmax = kv_cache.shape[0]
     mode = _mode(x)
+    if (state_kv is None) != (state_idx is None):
+        raise ValueError("state_kv and state_idx go together")
+    _shape(state_kv, (2 * m, 4 * c), "state_kv")
+    _shape(state_idx, (2 * m, 4 * cI), "state_idx")
+    _dtype(state_kv, torch.float32, "state_kv")
+    _dtype(state_idx, torch.float32, "state_idx")
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty((n, H), dtype=torch.float32, device=x.device)
     topk_idx = torch.empty((n, k), dtype=torch.int32, device=x.device) if return_topk else None
     nb = _lib.csa_prefill_workspace_size(n, Nmax, d, m, c, cI, H, HI, k, mode)
     ws = _ws(nb, x.device, ws)
     _check(_lib.csa_prefill(_ptr(x), _ptr(x_left), _ptr(W_kv), _ptr(B_kv), _ptr(W_idx), _ptr(B_idx), start, n, d,
-                            m, c, cI, _ptr(kv_cache), _ptr(idx_cache), Nmax, _ptr(qI), _ptr(w), _ptr(q), H, HI, k,
+                            m, c, cI, _ptr(kv_cache), _ptr(idx_cache), Nmax, _ptr(state_kv), _ptr(state_idx),
+                            _ptr(qI), _ptr(w), _ptr(q), H, HI, k,
                             scale, _ptr(sink), _ptr(out), _ptr(lse), _ptr(topk_idx), _ptr(ws), _nbytes(ws), mode,
                             _stream()))
     return (out, lse, topk_idx) if return_topk else (out, lse)

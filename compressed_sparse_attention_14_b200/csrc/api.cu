@@ -285,6 +285,37 @@ int hca_compress_step(const float* proj_new, float* state, const float* bias, co
                                 "hca_compress_step");
 }
 
+static int compress_chunk_common(const float* proj, float* state, const float* bias, int64_t start, int64_t n, int c,
+                                 int m, int mmax, void* cache, int64_t Nmax, int dtype, bool overlap, void* stream,
+                                 const char* who) {
+    ElemType t = ElemType::BF16;   // set by check_dtype
+    CSA_TRY(check_dtype(dtype, &t));
+    CSA_TRY(check_compress(0, c, m, mmax, who));
+    if (start < 0 || n < 0 || Nmax < 0) return fail(CSA_ERR_INVALID_ARG, "%s: bad start/n/Nmax", who);
+    if ((start + n) / m > Nmax)
+        return fail(CSA_ERR_INVALID_ARG, "%s: the cache holds %lld entries, %lld needed", who, (long long)Nmax,
+                    (long long)((start + n) / m));
+    if (n == 0) return CSA_OK;
+    CSA_TRY(check_ptr(proj, "proj"));
+    CSA_TRY(check_ptr(state, "state"));
+    CSA_TRY(check_ptr(bias, "bias"));
+    CSA_TRY(check_ptr(cache, "cache", (start + n) / m > start / m));
+    CSA_CUDA(compress_chunk_state(proj, state, bias, start, n, c, m, overlap, cache, t, (cudaStream_t)stream), who);
+    return CSA_OK;
+}
+
+int csa_compress_chunk(const float* proj, float* state, const float* bias, int64_t start, int64_t n, int c, int m,
+                       void* cache, int64_t Nmax, int dtype, void* stream) {
+    return compress_chunk_common(proj, state, bias, start, n, c, m, 64, cache, Nmax, dtype, true, stream,
+                                 "csa_compress_chunk");
+}
+
+int hca_compress_chunk(const float* proj, float* state, const float* bias, int64_t start, int64_t n, int c, int mp,
+                       void* cache, int64_t Nmax, int dtype, void* stream) {
+    return compress_chunk_common(proj, state, bias, start, n, c, mp, 1024, cache, Nmax, dtype, false, stream,
+                                 "hca_compress_chunk");
+}
+
 size_t csa_decode_compress_workspace_size(int B, int c, int cI) {
     if (B < 0 || c < 0 || cI < 0) return 0;
     return align256((size_t)B * 4 * c * sizeof(float)) + align256((size_t)B * 4 * cI * sizeof(float));
@@ -465,7 +496,8 @@ int csa_index_topk(const void* qI, const float* w, const void* K, const int32_t*
     void* tws = cv.take(topk_workspace_bytes(nq, Nmax, k));
     QuerySpec qs{seq_of_q, pos, 0, 0};
     CSA_CUDA(run_indexer(qI, w, K, qs, nq, n_seq, HI, cI, Nmax, m, sc, Nmax, 1, false, t, st), "csa_index_topk: scores");
-    CSA_CUDA(topk_select(sc, Nmax, pos, m, nq, Nmax, k, idx, top_scores, tws, st), "csa_index_topk: top-k");
+    CSA_CUDA(topk_select(sc, Nmax, pos, m, nq, Nmax, k, idx, top_scores, tws, st, seq_of_q, n_seq),
+             "csa_index_topk: top-k");
     return CSA_OK;
 }
 
@@ -613,9 +645,9 @@ size_t csa_prefill_workspace_size(int64_t n, int64_t Nmax, int d, int m, int c, 
 
 int csa_prefill(const void* x, const void* x_left, const void* W_kv, const float* B_kv,
                 const void* W_idx, const float* B_idx, int64_t start, int64_t n, int d, int m,
-                int c, int cI, void* kv_cache, void* idx_cache, int64_t Nmax, const void* qI,
-                const float* w, const void* q, int H, int HI, int k, float scale,
-                const float* sink, void* out, float* lse, int32_t* topk_idx, void* ws,
+                int c, int cI, void* kv_cache, void* idx_cache, int64_t Nmax, float* state_kv,
+                float* state_idx, const void* qI, const float* w, const void* q, int H, int HI, int k,
+                float scale, const float* sink, void* out, float* lse, int32_t* topk_idx, void* ws,
                 size_t ws_bytes, int dtype, void* stream) {
     ElemType t = ElemType::BF16;   // set by check_dtype
     CSA_TRY(check_dtype(dtype, &t));
@@ -624,10 +656,18 @@ int csa_prefill(const void* x, const void* x_left, const void* W_kv, const float
     CSA_TRY(check_attn_shape(H, c));
     CSA_TRY(check_attn_mode(H, c, t));
     CSA_TRY(check_k(k));
-    CSA_TRY(check_compress(n, c, m, 64, "csa_prefill"));
+    const bool stateful = state_kv || state_idx;
+    if (stateful && !(state_kv && state_idx))
+        return fail(CSA_ERR_INVALID_ARG, "state_kv and state_idx go together (both or neither)");
+    CSA_TRY(check_compress(stateful ? 0 : n, c, m, 64, "csa_prefill"));
+    if (n < 0) return fail(CSA_ERR_INVALID_ARG, "n=%lld is negative", (long long)n);
     if (d < 8 || d % 8) return fail(CSA_ERR_INVALID_ARG, "d=%d must be a positive multiple of 8", d);
-    if (start < 0 || start % m) return fail(CSA_ERR_INVALID_ARG, "start=%lld is not a non-negative multiple of m", (long long)start);
-    if (start > 0 && !x_left) return fail(CSA_ERR_INVALID_ARG, "x_left is required when start > 0");
+    if (start < 0) return fail(CSA_ERR_INVALID_ARG, "start=%lld is negative", (long long)start);
+    if (!stateful && start % m)
+        return fail(CSA_ERR_INVALID_ARG, "start=%lld is not a multiple of m (pass the state rings to start "
+                    "mid-block)", (long long)start);
+    if (!stateful && start > 0 && !x_left)
+        return fail(CSA_ERR_INVALID_ARG, "x_left is required when start > 0 (or pass the state rings)");
     if ((start + n) / m > Nmax) return fail(CSA_ERR_INVALID_ARG, "caches hold %lld entries, %lld needed",
                                             (long long)Nmax, (long long)((start + n) / m));
     if (Nmax > INT32_MAX || start + n > INT32_MAX) return fail(CSA_ERR_UNSUPPORTED, "positions beyond int32");
@@ -640,6 +680,8 @@ int csa_prefill(const void* x, const void* x_left, const void* W_kv, const float
     CSA_TRY(check_ptr(B_idx, "B_idx"));
     CSA_TRY(check_ptr(kv_cache, "kv_cache"));
     CSA_TRY(check_ptr(idx_cache, "idx_cache"));
+    CSA_TRY(check_ptr(state_kv, "state_kv", false));
+    CSA_TRY(check_ptr(state_idx, "state_idx", false));
     CSA_TRY(check_ptr(qI, "qI"));
     CSA_TRY(check_ptr(w, "w"));
     CSA_TRY(check_ptr(q, "q"));
@@ -660,26 +702,38 @@ int csa_prefill(const void* x, const void* x_left, const void* W_kv, const float
     int32_t* sel_ws = (int32_t*)cv.take((size_t)qc * k * sizeof(int32_t));
     void* mws = cv.take(mqa_workspace_bytes((int)qc, H, c, k, t));
 
-    // 1-2. compress the chunk into both caches (entries start/m ..)
+    // 1-2. compress the chunk into both caches: aligned chunks from their own
+    // rows and the m rows before (entries start/m ..); with the state rings,
+    // any chunk: every block that ends inside it, earlier window tokens from
+    // the ring, which then keeps the chunk's last 2m projected rows
     const int64_t e0 = start / m;
-    struct { const void* W; const float* B; int cc; void* cache; } streams[2] = {
-        {W_kv, B_kv, c, kv_cache}, {W_idx, B_idx, cI, idx_cache}};
+    struct { const void* W; const float* B; int cc; void* cache; float* state; } streams[2] = {
+        {W_kv, B_kv, c, kv_cache, state_kv}, {W_idx, B_idx, cI, idx_cache, state_idx}};
     for (auto& s : streams) {
         CSA_CUDA(project(x, s.W, n, d, 4 * s.cc, proj, t, st), "csa_prefill: projection");
+        if (stateful) {
+            CSA_CUDA(compress_chunk_state(proj, s.state, s.B, start, n, s.cc, m, true, s.cache, t, st),
+                     "csa_prefill: compress");
+            continue;
+        }
         if (start > 0) CSA_CUDA(project(x_left, s.W, m, d, 4 * s.cc, lproj, t, st), "csa_prefill: left projection");
         CSA_CUDA(compress_csa(proj, start > 0 ? lproj : nullptr, s.B, n, s.cc, m,
                               (char*)s.cache + (size_t)e0 * s.cc * es, ElemType::F32, t, st),
                  "csa_prefill: compress");
     }
-    // 3. indexer -> top-k -> sparse MQA per query chunk
+    // 3. indexer -> top-k -> sparse MQA per query chunk; a chunk that starts
+    // mid-block first takes the queries up to the next block boundary alone
     const float sc_scale = default_scale(scale, c);
-    for (int64_t q0 = 0; q0 < n; q0 += qc) {
-        const int nqc = (int)((n - q0) < qc ? (n - q0) : qc);
+    const int64_t head = (m - start % m) % m;
+    for (int64_t q0 = 0; q0 < n;) {
+        const int64_t span = (q0 == 0 && head > 0) ? head : qc;
+        const int nqc = (int)((n - q0) < span ? (n - q0) : span);
         QuerySpec qs{nullptr, nullptr, start + q0, 1};
         int32_t* sel = topk_idx ? topk_idx + q0 * k : sel_ws;
         // the m tokens of one compressed block see the same entries: score them
-        // together against each key tile when the group fits one MMA
-        const int group = (m <= 4 && index_tc_supported(HI, cI, m)) ? m : 1;
+        // together against each key tile when the group fits one MMA (the
+        // group starts on a block boundary)
+        const int group = (m <= 4 && (start + q0) % m == 0 && index_tc_supported(HI, cI, m)) ? m : 1;
         CSA_CUDA(run_indexer((const char*)qI + (size_t)q0 * HI * cI * es, w + q0 * HI, idx_cache, qs, nqc, 1, HI,
                              cI, Nmax, m, sc, Nmax, group, false, t, st), "csa_prefill: indexer");
         // visible count of query t is floor((start + q0 + t) / m); pass it through a
@@ -688,6 +742,7 @@ int csa_prefill(const void* x, const void* x_left, const void* W_kv, const float
         CSA_CUDA(mqa((const char*)q + (size_t)q0 * H * c * es, kv_cache, sel, k, qs, 1, nqc, 1, H, c, Nmax,
                      sc_scale, sink, (char*)out + (size_t)q0 * H * c * es, lse ? lse + q0 * H : nullptr, mws,
                      t, st), "csa_prefill: mqa");
+        q0 += nqc;
     }
     return CSA_OK;
 }

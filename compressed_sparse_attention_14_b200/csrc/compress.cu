@@ -245,6 +245,119 @@ __global__ void __launch_bounds__(256) hca_compress_step_kernel(const float* __r
     else store8(reinterpret_cast<float*>(out), o);
 }
 
+// Chunk compression at any start and length through the state ring [Walk §5
+// item 2; Notes §2.6 Fig. 6]: the chunk holds tokens start .. start+n-1 of
+// one sequence, projected (fp32, proj row tau - start). It writes the entry
+// of every block that ends inside the chunk, i in [i_lo, i_lo + nb), taking
+// each window token tau from the chunk when tau >= start and from the ring
+// (slot tau mod ring_rows) when the token came earlier: the ring holds the
+// projected rows of the sequence's last ring_rows tokens before the chunk
+// (2m for CSA, m' for HCA). One thread per (entry, 8 channels), the window
+// terms in the chunk kernels' order, so an entry is the same wherever its
+// tokens came from. The ring is refreshed afterwards by ring_store_kernel, a
+// separate launch, because a new token's slot may hold a row this one reads.
+template <typename TOut>
+__global__ void __launch_bounds__(256) compress_chunk_state_kernel(const float* __restrict__ proj,
+                                                                   const float* __restrict__ ring,
+                                                                   const float* __restrict__ bias, int64_t start,
+                                                                   int64_t i_lo, int64_t nb, int c, int m,
+                                                                   int overlap, TOut* __restrict__ cache) {
+    pdl_wait();
+    pdl_launch_next();
+    const int groups = c / 8;
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= nb * groups) return;
+    const int64_t i = i_lo + gid / groups;
+    const int j = (int)(gid % groups) * 8;
+    const int64_t ld = (overlap ? 4 : 2) * (int64_t)c;
+    const int ring_rows = overlap ? 2 * m : m;
+    auto row_of = [&](int64_t tau) -> const float* {
+        return tau >= start ? proj + (tau - start) * ld : ring + (tau % ring_rows) * ld;
+    };
+    OnlineSoftmax8 sm;
+    sm.init();
+    float z[8], b[8], v[8];
+    // a-window (CSA: C^a, Z^a, bias rows 0..m-1; HCA: C, Z, bias rows 0..m'-1)
+    for (int r = 0; r < m; ++r) {
+        const float* row = row_of(m * i + r);
+        load8(row + (overlap ? 2 * c : c) + j, z);
+        load8(bias + (int64_t)r * c + j, b);
+        load8(row + j, v);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) z[u] += b[u];
+        sm.push(z, v);
+    }
+    // CSA b-window: the previous block's tokens, C^b, Z^b, bias rows m..2m-1;
+    // none for the first block of the sequence
+    if (overlap && i > 0) {
+        for (int r = 0; r < m; ++r) {
+            const float* row = row_of(m * (i - 1) + r);
+            load8(row + 3 * c + j, z);
+            load8(bias + (int64_t)(m + r) * c + j, b);
+            load8(row + c + j, v);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) z[u] += b[u];
+            sm.push(z, v);
+        }
+    }
+    float o[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) o[u] = sm.acc[u] / sm.den[u];
+    TOut* out = cache + i * c + j;
+    if constexpr (sizeof(TOut) == 2) store8(reinterpret_cast<bf16*>(out), o);
+    else store8(reinterpret_cast<float*>(out), o);
+}
+
+// The ring after the chunk: the projected rows of the chunk's last
+// min(n, ring_rows) tokens go to their slots (tau mod ring_rows); the other
+// slots keep the earlier tokens that are still among the last ring_rows.
+__global__ void __launch_bounds__(256) ring_store_kernel(const float* __restrict__ proj, float* __restrict__ ring,
+                                                         int64_t start, int64_t n, int ring_rows, int64_t ld) {
+    pdl_wait();
+    pdl_launch_next();
+    const int64_t keep = n < ring_rows ? n : ring_rows;
+    const int64_t per_row = ld / 4;
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= keep * per_row) return;
+    const int64_t tau = start + n - keep + gid / per_row;
+    const int64_t col = (gid % per_row) * 4;
+    const float4 v = *reinterpret_cast<const float4*>(proj + (tau - start) * ld + col);
+    *reinterpret_cast<float4*>(ring + (tau % ring_rows) * ld + col) = v;
+}
+
+cudaError_t compress_chunk_state(const float* proj, float* state, const float* bias, int64_t start, int64_t n, int c,
+                                 int m, bool overlap, void* cache, ElemType out_t, cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    const int64_t i_lo = start / m;
+    const int64_t nb = (start + n) / m - i_lo;
+    const int64_t threads = nb * (c / 8);
+    cudaError_t e = cudaSuccess;
+    if (threads > 0) {
+        const dim3 grid((unsigned)((threads + 255) / 256));
+        if (out_t == ElemType::BF16)
+            CSA_LAUNCH(st, overlap ? "csa_compress_chunk" : "hca_compress_chunk",
+                       e = launch_pdl(compress_chunk_state_kernel<bf16>, grid, dim3(256), 0, st, 0, proj,
+                                      (const float*)state, bias, start, i_lo, nb, c, m, overlap ? 1 : 0, (bf16*)cache));
+        else
+            CSA_LAUNCH(st, overlap ? "csa_compress_chunk" : "hca_compress_chunk",
+                       e = launch_pdl(compress_chunk_state_kernel<float>, grid, dim3(256), 0, st, 0, proj,
+                                      (const float*)state, bias, start, i_lo, nb, c, m, overlap ? 1 : 0,
+                                      (float*)cache));
+        if (e != cudaSuccess) return e;
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    const int ring_rows = overlap ? 2 * m : m;
+    const int64_t ld = (overlap ? 4 : 2) * (int64_t)c;
+    const int64_t keep = n < ring_rows ? n : ring_rows;
+    const int64_t t2 = keep * (ld / 4);
+    CSA_LAUNCH(st, "ring_store",
+               e = launch_pdl(ring_store_kernel, dim3((unsigned)((t2 + 255) / 256)), dim3(256), 0, st, 0, proj, state,
+                              start, n, ring_rows, ld));
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
 template <typename TIn, typename TOut>
 cudaError_t launch_csa_compress(const void* proj, const void* left, const float* bias, int64_t n,
                                 int c, int m, void* out, cudaStream_t st) {

@@ -213,7 +213,7 @@ cudaError_t project_tc(const void* x, const void* W, int64_t n, int d, int M, fl
     if (!make_tmap_bf16_2d(&tmX, x, (uint64_t)n, d, d, kBM, kBK)) return cudaErrorInvalidValue;
     if (!make_tmap_bf16_2d(&tmW, W, (uint64_t)M, d, d, kBN, kBK)) return cudaErrorInvalidValue;
     const size_t smem = 1024 + (size_t)kStages * kStageBytes + 16 * sizeof(uint64_t);
-    cudaError_t e = cudaFuncSetAttribute(project_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = smem_ceiling(project_tc_kernel);
     if (e != cudaSuccess) return e;
     const int ntiles = a.tiles_m * a.tiles_n;
     const int grid = ntiles < sm_count() ? ntiles : sm_count();

@@ -91,13 +91,13 @@ cudaError_t index_scores(const void* qI, const float* w, const void* K, QuerySpe
     cudaError_t e;
     if (t == ElemType::BF16) {
         auto kern = index_scores_ffma_kernel<bf16>;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = smem_ceiling(kern);
         if (e != cudaSuccess) return e;
         CSA_LAUNCH(st, "index_scores_ffma", kern<<<grid, 256, smem, st>>>((const bf16*)qI, w, (const bf16*)K, qm, HI, cI, Nmax, m,
                                       scores, ld_scores));
     } else {
         auto kern = index_scores_ffma_kernel<float>;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = smem_ceiling(kern);
         if (e != cudaSuccess) return e;
         CSA_LAUNCH(st, "index_scores_ffma", kern<<<grid, 256, smem, st>>>((const float*)qI, w, (const float*)K, qm, HI, cI, Nmax, m,
                                       scores, ld_scores));

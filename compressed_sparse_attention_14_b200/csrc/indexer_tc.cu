@@ -483,7 +483,7 @@ cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, Query
         if (e == cudaSuccess) e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    e = cudaFuncSetAttribute(index_scores_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = smem_ceiling(index_scores_tc_kernel);
     if (e != cudaSuccess) return e;
     CSA_LAUNCH(st, "index_scores_tc",
                e = launch_pdl(index_scores_tc_kernel, dim3(num_sms()), dim3(kThreads), smem, st, 0, a, tmK, tmQ));

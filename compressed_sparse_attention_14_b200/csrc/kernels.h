@@ -54,6 +54,16 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+// launch.cu: raise `kern`'s dynamic shared-memory ceiling to the device's
+// opt-in maximum, once per (kernel, device); thread-safe. Every launcher calls
+// this instead of setting the attribute to its own size per call, which would
+// race with calls on other host threads.
+cudaError_t smem_ceiling(const void* kern);
+template <typename... KArgs>
+cudaError_t smem_ceiling(void (*kern)(KArgs...)) {
+    return smem_ceiling(reinterpret_cast<const void*>(kern));
+}
+
 inline size_t elem_size(ElemType t) { return t == ElemType::BF16 ? 2 : 4; }
 inline size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
 
@@ -81,6 +91,14 @@ cudaError_t compress_hca(const void* proj, const float* bias, int64_t n, int c, 
 cudaError_t compress_step(const float* proj_new, float* state, const float* bias, const int32_t* pos, int B, int c,
                           int m, bool overlap, int64_t Nmax, void* cache, ElemType out_t, cudaStream_t st);
 
+// compress.cu, chunks at any start and length: the entries of every block
+// that ends inside the chunk [start, start+n) (proj rows fp32, one sequence),
+// earlier window tokens read from the state ring (2m rows for CSA, m' for
+// HCA, slot tau mod ring rows), which is then refreshed with the chunk's last
+// tokens. cache is the sequence's [Nmax, c] cache; entry i at row i.
+cudaError_t compress_chunk_state(const float* proj, float* state, const float* bias, int64_t start, int64_t n, int c,
+                                 int m, bool overlap, void* cache, ElemType out_t, cudaStream_t st);
+
 // gemm.cu: out[n, M] (fp32) = x[n, d] . W[M, d]^T (bf16 -> gemm_tc.cu)
 cudaError_t project(const void* x, const void* W, int64_t n, int d, int M, float* out, ElemType t,
                     cudaStream_t st);
@@ -102,11 +120,12 @@ cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, Query
 // api.cu: device address of the status word on the current device
 int* device_status();
 
-// topk.cu
+// topk.cu. With seq given, a row whose sequence seq[t] is outside
+// [0, n_seq) has no candidate (its indexer row was never written).
 size_t topk_workspace_bytes(int nq, int64_t ncols, int k);
 cudaError_t topk_select(const float* scores, int64_t ld, const int32_t* valid, int valid_div,
                         int nq, int64_t ncols, int k, int32_t* idx, float* top_scores, void* ws,
-                        cudaStream_t st);
+                        cudaStream_t st, const int32_t* seq = nullptr, int n_seq = 0);
 // as topk_select with the candidate count of row t = (pos_base + t) / m
 cudaError_t topk_select_positions(const float* scores, int64_t ld, int64_t pos_base, int m, int nq,
                                   int64_t ncols, int k, int32_t* idx, void* ws, cudaStream_t st);

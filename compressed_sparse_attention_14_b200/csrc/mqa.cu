@@ -268,12 +268,12 @@ cudaError_t mqa(const void* q, const void* KV, const int32_t* idx, int k, QueryS
     cudaError_t e;
     if (t == ElemType::BF16) {
         auto kern = mqa_partial_ffma_kernel<bf16>;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = smem_ceiling(kern);
         if (e != cudaSuccess) return e;
         CSA_LAUNCH(st, "mqa_partial_ffma", kern<<<grid, 256, smem, st>>>(a));
     } else {
         auto kern = mqa_partial_ffma_kernel<float>;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = smem_ceiling(kern);
         if (e != cudaSuccess) return e;
         CSA_LAUNCH(st, "mqa_partial_ffma", kern<<<grid, 256, smem, st>>>(a));
     }

@@ -786,7 +786,7 @@ cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, Que
         kv_bytes = (size_t)ring * 2 * kE * 128;
     }
     const size_t smem = fixed + kv_bytes;
-    cudaError_t e = cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = smem_ceiling(mqa_tc_kernel);
     if (e != cudaSuccess) return e;
     cudaError_t le = cudaSuccess;
     CSA_LAUNCH(st, "mqa_tc",

@@ -79,7 +79,10 @@ struct RowSpec {
     int64_t pos_base;         // used when use_pos
     int use_pos;
     int64_t ncols;
+    const int32_t* seq;       // nullable: row t reads sequence seq[t]
+    int n_seq;                // a row whose sequence is outside [0, n_seq) has no candidate
     __device__ __forceinline__ int64_t count(int row) const {
+        if (seq && (seq[row] < 0 || seq[row] >= n_seq)) return 0;
         if (!valid && !use_pos) return ncols;
         int64_t v = (valid ? (int64_t)valid[row] : pos_base + row) / valid_div;
         return v < 0 ? 0 : (v < ncols ? v : ncols);
@@ -641,7 +644,7 @@ static cudaError_t topk_run(const RowSpec& R, int nq, int k, int32_t* idx, float
     const bool spread = (int64_t)nq * G <= sm_count();
     auto kern = topk_kernel;
     const size_t smem = spread ? kSmemSpread : kSmemBytes;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = smem_ceiling(kern);
     if (e != cudaSuccess) return e;
     cudaError_t le = cudaSuccess;
     CSA_LAUNCH(st, "topk_select",
@@ -651,16 +654,17 @@ static cudaError_t topk_run(const RowSpec& R, int nq, int k, int32_t* idx, float
 }
 
 cudaError_t topk_select(const float* scores, int64_t ld, const int32_t* valid, int valid_div, int nq, int64_t ncols,
-                        int k, int32_t* idx, float* top_scores, void* ws, cudaStream_t st) {
+                        int k, int32_t* idx, float* top_scores, void* ws, cudaStream_t st, const int32_t* seq,
+                        int n_seq) {
     (void)ws;
-    RowSpec R{scores, ld, valid, valid_div, 0, 0, ncols};
+    RowSpec R{scores, ld, valid, valid_div, 0, 0, ncols, seq, n_seq};
     return topk_run(R, nq, k, idx, top_scores, st);
 }
 
 cudaError_t topk_select_positions(const float* scores, int64_t ld, int64_t pos_base, int m, int nq, int64_t ncols,
                                   int k, int32_t* idx, void* ws, cudaStream_t st) {
     (void)ws;
-    RowSpec R{scores, ld, nullptr, m, pos_base, 1, ncols};
+    RowSpec R{scores, ld, nullptr, m, pos_base, 1, ncols, nullptr, 0};
     return topk_run(R, nq, k, idx, nullptr, st);
 }
 

@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define CSA_ABI_VERSION 1
+#define CSA_ABI_VERSION 2
 
 enum csa_status {
     CSA_OK = 0,
@@ -169,6 +169,28 @@ int csa_compress_step(const float* proj_new, float* state, const float* bias, co
 int hca_compress_step(const float* proj_new, float* state, const float* bias, const int32_t* pos, int B, int c,
                       int mp, int64_t Nmax, void* cache, int dtype, void* stream);
 
+/* csa_compress_chunk: a chunk of ONE sequence at ANY start and length
+ * through the same state ring, so prefill chunks and decode steps can split
+ * a sequence anywhere (a chunk that ends mid-block leaves its tail in the
+ * ring; the next chunk or step closes the block):
+ *   proj  [n, 4c] fp32: the projections of tokens start .. start+n-1;
+ *   state [2m, 4c] fp32: this sequence's ring (as csa_compress_step); on
+ *         entry it holds the tokens before start that are among the last
+ *         2m, on return the last 2m tokens up to start+n;
+ *   cache [Nmax, c] (dtype): the sequence's entries; every block that ends
+ *         inside the chunk, i = floor(start/m) .. floor((start+n)/m) - 1, is
+ *         written at row i, its window tokens before start read from the
+ *         ring. Nmax >= floor((start+n)/m). Entries equal csa_compress's for
+ *         the same rows (the same operations in the same order).
+ * c % 8 == 0, 1 <= m <= 64; n may be 0 (nothing happens). */
+int csa_compress_chunk(const float* proj, float* state, const float* bias, int64_t start, int64_t n, int c, int m,
+                       void* cache, int64_t Nmax, int dtype, void* stream);
+
+/* hca_compress_chunk: the same for HCA: proj [n, 2c] (C|Z), state [mp, 2c]
+ * (token tau in slot tau mod mp), bias [mp, c]; blocks of mp tokens. */
+int hca_compress_chunk(const float* proj, float* state, const float* bias, int64_t start, int64_t n, int c, int mp,
+                       void* cache, int64_t Nmax, int dtype, void* stream);
+
 /* csa_decode_compress: a1 + csa_compress_step for both CSA streams of one
  * decode step: x_new [B, d] (dtype) projected by W_kv [4c, d] and W_idx
  * [4cI, d], then stepped through state_kv [B, 2m, 4c] and state_idx
@@ -280,7 +302,12 @@ int hca_decode(const void* q, const void* kv_cache, const int32_t* ctx_len, int 
                void* ws, size_t ws_bytes, int dtype, void* stream);
 
 /* csa_prefill: one chunk of n new tokens of ONE sequence at positions
- * start .. start+n-1 (start % m == 0, n % m == 0):
+ * start .. start+n-1. Without state rings (state_kv = state_idx = NULL)
+ * start % m == 0 and n % m == 0, and x_left supplies the b-window of the
+ * first block. With both state rings ([2m, 4c] and [2m, 4cI] fp32, as
+ * csa_compress_chunk) start and n are free: the blocks that end inside the
+ * chunk are written (earlier window tokens from the rings), the rings then
+ * hold the chunk's last 2m projected rows, and x_left is not read. Steps:
  *   1. compress the chunk's KV entries (a1+a2 with W_kv [4c, d], B_kv
  *      [2m, c]) into kv_cache rows start/m .. (start+n)/m - 1;
  *   2. the same for the indexer keys (W_idx [4cI, d], B_idx [2m, cI]) into
@@ -297,9 +324,9 @@ size_t csa_prefill_workspace_size(int64_t n, int64_t Nmax, int d, int m, int c, 
                                   int HI, int k, int dtype);
 int csa_prefill(const void* x, const void* x_left, const void* W_kv, const float* B_kv,
                 const void* W_idx, const float* B_idx, int64_t start, int64_t n, int d, int m,
-                int c, int cI, void* kv_cache, void* idx_cache, int64_t Nmax, const void* qI,
-                const float* w, const void* q, int H, int HI, int k, float scale,
-                const float* sink, void* out, float* lse, int32_t* topk_idx, void* ws,
+                int c, int cI, void* kv_cache, void* idx_cache, int64_t Nmax, float* state_kv,
+                float* state_idx, const void* qI, const float* w, const void* q, int H, int HI, int k,
+                float scale, const float* sink, void* out, float* lse, int32_t* topk_idx, void* ws,
                 size_t ws_bytes, int dtype, void* stream);
 
 /* ------------------------------------------------------------------------

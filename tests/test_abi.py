@@ -32,7 +32,7 @@ def test_header_declarations_are_exported():
 
 
 def test_abi_version():
-    assert csa.abi_version() == 1
+    assert csa.abi_version() == 2
 
 
 def _lib():
@@ -84,15 +84,23 @@ def test_invalid_arguments_are_rejected_on_the_host():
     assert rc == csa.CSA_ERR_WORKSPACE
     # prefill: start not a multiple of m, cache too small, missing left rows
     args = dict(n=8, Nmax=4, start=4)
-    rc = L.csa_prefill(fake, fake, fake, fake, fake, fake, 2, 8, 64, 4, 128, 64, fake, fake, 16, fake, fake, fake,
+    rc = L.csa_prefill(fake, fake, fake, fake, fake, fake, 2, 8, 64, 4, 128, 64, fake, fake, 16, None, None, fake, fake, fake,
                        8, 4, 4, 0.0, None, fake, None, None, None, 0, csa.CSA_BF16, None)
     assert rc == csa.CSA_ERR_INVALID_ARG
-    rc = L.csa_prefill(fake, fake, fake, fake, fake, fake, 4, 8, 64, 4, 128, 64, fake, fake, 2, fake, fake, fake,
+    rc = L.csa_prefill(fake, fake, fake, fake, fake, fake, 4, 8, 64, 4, 128, 64, fake, fake, 2, None, None, fake, fake, fake,
                        8, 4, 4, 0.0, None, fake, None, None, None, 0, csa.CSA_BF16, None)
     assert rc == csa.CSA_ERR_INVALID_ARG
-    rc = L.csa_prefill(fake, None, fake, fake, fake, fake, 4, 8, 64, 4, 128, 64, fake, fake, 16, fake, fake, fake,
+    rc = L.csa_prefill(fake, None, fake, fake, fake, fake, 4, 8, 64, 4, 128, 64, fake, fake, 16, None, None, fake, fake, fake,
                        8, 4, 4, 0.0, None, fake, None, None, None, 0, csa.CSA_BF16, None)
     assert rc == csa.CSA_ERR_INVALID_ARG
+    # prefill with one state ring but not the other
+    rc = L.csa_prefill(fake, None, fake, fake, fake, fake, 6, 9, 64, 4, 128, 64, fake, fake, 16, fake, None, fake,
+                       fake, fake, 8, 4, 4, 0.0, None, fake, None, None, None, 0, csa.CSA_BF16, None)
+    assert rc == csa.CSA_ERR_INVALID_ARG and b"together" in L.csa_last_error()
+    # chunk compression: the cache must hold every block the chunk closes
+    assert L.csa_compress_chunk(fake, fake, fake, 6, 11, 64, 4, fake, 3, csa.CSA_BF16, None) == csa.CSA_ERR_INVALID_ARG
+    assert L.hca_compress_chunk(fake, None, fake, 0, 8, 64, 4, fake, 2, csa.CSA_BF16, None) == csa.CSA_ERR_INVALID_ARG
+    assert L.hca_compress_chunk(fake, fake, fake, -1, 8, 64, 4, fake, 2, csa.CSA_BF16, None) == csa.CSA_ERR_INVALID_ARG
     del args
 
 

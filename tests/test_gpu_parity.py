@@ -180,6 +180,22 @@ def test_index_topk(csa, dtype):
         assert np.all(s < pos_h[t].item() // m)
 
 
+@pytest.mark.parametrize("dtype", MODES)
+def test_index_topk_query_on_a_missing_sequence_selects_nothing(csa, dtype):
+    # a query whose sequence is outside [0, n_seq) sees no entry (csa.h): its
+    # indexer row is never written, so the selection must not read it
+    nq, HI, cI, B, Nmax, m, k = 6, 64, 128, 3, 2000, 4, 64
+    qI_h, qI, K_h, K, w_h, w, _, _ = _index_inputs(dtype, nq, HI, cI, B, Nmax, m, seed=12)
+    pos_h = torch.tensor([8000, 5000, 7999, 300, 8000, 64], dtype=torch.int32)
+    seq_h = torch.tensor([0, 2, 3, 1, -1, 2], dtype=torch.int32)
+    idx, _ = csa.csa_index_topk(qI, w, K, pos_h.to(DEV), m, k, seq_of_q=seq_h.to(DEV))
+    sel = host(idx)
+    assert np.all(sel[2] == -1) and np.all(sel[4] == -1)
+    ok = [0, 1, 3, 5]
+    ref_idx, S = oracle.index_topk(qI_h[ok], w_h[ok], K_h, pos_h[ok], m, k, seq=seq_h[ok])
+    assert_topk_sets(idx[ok], ref_idx, S, k)
+
+
 # ---------------------------------------------------------------- a6 / a7
 @pytest.mark.parametrize("dtype", MODES)
 @pytest.mark.parametrize("H,c,k", [(64, 512, 512), (8, 128, 16), (128, 512, 96)])
