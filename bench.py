@@ -229,7 +229,11 @@ class Timer:
 # workloads (ours)
 # ----------------------------------------------------------------------------
 
-def decode_workload(shape, rank, batch=None):
+def decode_workload(shape, rank, batch=None, fp8=False):
+    """One csa_decode step over the batch. fp8: the FP8 indexer
+    (csa_decode_fp8): the indexer keys are held as e4m3 codes with one fp32
+    scale per key (quantized once when the cache is built, outside the timed
+    region, as the compressor would store them), q^I is quantized in the call."""
     import dataclasses
     import compressed_sparse_attention_14_b200 as csa
     s = shape if batch is None else dataclasses.replace(shape, batch=batch)
@@ -238,19 +242,32 @@ def decode_workload(shape, rank, batch=None):
     mode = csa.CSA_BF16
     out = torch.empty_like(inp["q"])
     lse = torch.empty((B, s.heads), dtype=torch.float32, device="cuda")
-    ws = torch.empty(csa.csa_decode_workspace_size(B, s.n_max, s.heads, s.c, s.idx_heads, s.idx_dim, s.k, mode),
-                     dtype=torch.uint8, device="cuda")
+    if fp8:
+        k8, ks, _ = csa.csa_quantize_e4m3(inp["idx_cache"])
+        del inp["idx_cache"]
+        torch.cuda.synchronize()
+        ws = torch.empty(csa.workspace_size("csa_decode_fp8", B, s.n_max, s.heads, s.c, s.idx_heads, s.idx_dim, s.k),
+                         dtype=torch.uint8, device="cuda")
+
+        def call(qI, w, q, ctx):
+            csa.csa_decode_fp8(qI, w, k8, ks, q, inp["kv_cache"], ctx, s.m, s.k, out=out, lse=lse, ws=ws)
+    else:
+        ws = torch.empty(csa.csa_decode_workspace_size(B, s.n_max, s.heads, s.c, s.idx_heads, s.idx_dim, s.k, mode),
+                         dtype=torch.uint8, device="cuda")
+
+        def call(qI, w, q, ctx):
+            csa.csa_decode(qI, w, inp["idx_cache"], q, inp["kv_cache"], ctx, s.m, s.k, out=out, lse=lse, ws=ws)
 
     def step():
-        csa.csa_decode(inp["qI"], inp["w"], inp["idx_cache"], inp["q"], inp["kv_cache"], inp["ctx_len"], s.m, s.k,
-                       out=out, lse=lse, ws=ws)
+        call(inp["qI"], inp["w"], inp["q"], inp["ctx_len"])
 
     ctx = inp["ctx_len"].double()
     vis = torch.floor(ctx / s.m)
     v_sum = float(vis.sum())
-    # algorithmic bytes: indexer keys of the visible entries, q^I and w; the
-    # selected KV rows; q and out (bf16)
-    idx_bytes = v_sum * s.idx_dim * 2 + B * (s.idx_heads * s.idx_dim * 2 + s.idx_heads * 4)
+    # algorithmic bytes: indexer keys of the visible entries (bf16, or e4m3
+    # plus one fp32 scale), q^I and w; the selected KV rows; q and out (bf16)
+    key_bytes = (s.idx_dim + 4) if fp8 else s.idx_dim * 2
+    idx_bytes = v_sum * key_bytes + B * (s.idx_heads * s.idx_dim * (1 if fp8 else 2) + s.idx_heads * 4)
     step_bytes = idx_bytes + B * (s.k * s.c * 2 + 2 * s.heads * s.c * 2)
     # the indexer kernel also writes one fp32 score per visible entry
     idx_kernel_bytes = idx_bytes + v_sum * 4
@@ -262,24 +279,28 @@ def decode_workload(shape, rank, batch=None):
     def e2e_step():
         for k, v in pinned.items():
             dev_in[k].copy_(v, non_blocking=True)
-        csa.csa_decode(dev_in["qI"], dev_in["w"], inp["idx_cache"], dev_in["q"], inp["kv_cache"], dev_in["ctx_len"],
-                       s.m, s.k, out=out, lse=lse, ws=ws)
+        call(dev_in["qI"], dev_in["w"], dev_in["q"], dev_in["ctx_len"])
         out_h.copy_(out, non_blocking=True)
 
     h2d = sum(v.numel() * v.element_size() for v in pinned.values())
     d2h = out_h.numel() * out_h.element_size()
     mqa_bytes = B * (s.k * s.c * 2 + 2 * s.heads * s.c * 2)
+    idx_name = "index_scores_tc_fp8" if fp8 else "index_scores_tc"
     kernels = {
-        "index_scores_tc": dict(bound="hbm", work=idx_kernel_bytes, files=("indexer_tc.cu", "tc.cuh", "common.cuh")),
+        idx_name: dict(bound="hbm", work=idx_kernel_bytes, files=("indexer_tc.cu", "tc.cuh", "common.cuh")),
         "mqa_tc": dict(bound="hbm", work=mqa_bytes, files=("mqa_tc.cu", "tc.cuh", "common.cuh")),
         # one pass over each row's visible scores, k indices out
         "topk_select": dict(bound="hbm", work=v_sum * 4 + B * s.k * 4, files=("topk.cu",)),
     }
+    if fp8:
+        kernels["quantize_e4m3"] = dict(bound="hbm", work=B * s.idx_heads * (s.idx_dim * 3 + 12), files=("quant.cu",))
     return dict(step=step, e2e_step=e2e_step, units=B, unit="queries/s", h2d=h2d, d2h=d2h,
                 kernels=kernels, step_bytes=step_bytes,
-                config=dict(workload=s.name, batch=B, ctx_len=f"U[{s.ctx_lo},{s.ctx_hi}]", m=s.m,
+                config=dict(workload=s.name + ("_fp8_indexer" if fp8 else ""), batch=B,
+                            ctx_len=f"U[{s.ctx_lo},{s.ctx_hi}]", m=s.m,
                             entries_max=s.n_max, head_dim=s.c, heads=s.heads, index_heads=s.idx_heads,
                             index_dim=s.idx_dim, topk=s.k, visible_entries_total=int(v_sum),
+                            index_keys="e4m3 + fp32 scale per key" if fp8 else "bf16",
                             l2="flushed before every timed step (256 MiB write + 256 MiB read)"),
                 inputs=inp)
 
@@ -536,6 +557,8 @@ def prefill_workload(rank, tokens=None):
 WORKLOADS = {
     "flash_decode": lambda r, b=None: decode_workload(synth.FLASH_DECODE, r, b),
     "pro_decode": lambda r, b=None: decode_workload(synth.PRO_DECODE, r, b),
+    "flash_decode_fp8": lambda r, b=None: decode_workload(synth.FLASH_DECODE, r, b, fp8=True),
+    "pro_decode_fp8": lambda r, b=None: decode_workload(synth.PRO_DECODE, r, b, fp8=True),
     "hca_decode": lambda r, b=None: hca_decode_workload(r),
     "hca_compress": lambda r, b=None: hca_compress_workload(r),
     "prefill": lambda r, b=None: prefill_workload(r, b),
@@ -548,15 +571,21 @@ WORKLOADS = {
 # CPU oracle timing (the reference arm and the cpu_baseline object)
 # ----------------------------------------------------------------------------
 
-def oracle_decode_sample(shape, n_queries: int, seed_rank: int = 0):
-    """Time the oracle (indexer + top-k + sparse MQA, fp64) on the first
-    n_queries of the decode batch. Returns (seconds, queries)."""
+def oracle_decode_sample(shape, n_queries: int, seed_rank: int = 0, fp8: bool = False):
+    """Time the oracle (indexer + top-k + sparse MQA, fp64; fp8: the indexer
+    on e4m3-quantized q^I and keys) on the first n_queries of the decode
+    batch. Returns (seconds, queries)."""
     import oracle
     s = dataclass_seed(shape, seed_rank)
     inp = synth.decode_inputs(s, device="cpu", batch=n_queries)
     t0 = time.perf_counter()
-    idx, _ = oracle.index_topk(inp["qI"], inp["w"], inp["idx_cache"], inp["ctx_len"], s.m, s.k,
-                               seq=torch.arange(n_queries))
+    if fp8:
+        S = oracle.index_scores_fp8(inp["qI"], inp["w"], inp["idx_cache"], inp["ctx_len"], s.m,
+                                    seq=torch.arange(n_queries))
+        idx = oracle.topk(S, (inp["ctx_len"].numpy() // s.m).astype("int32"), s.k)
+    else:
+        idx, _ = oracle.index_topk(inp["qI"], inp["w"], inp["idx_cache"], inp["ctx_len"], s.m, s.k,
+                                   seq=torch.arange(n_queries))
     oracle.sparse_mqa(inp["q"], inp["kv_cache"], idx, 1 / math.sqrt(s.c), seq=torch.arange(n_queries))
     return time.perf_counter() - t0, n_queries
 
@@ -639,15 +668,16 @@ def oracle_measure(workload: str, budget_s: float = 15.0):
     """Grow the sample until it takes about budget_s seconds; return
     (units per second, description, units)."""
     threads = cpu_oracle_threads()
-    if workload in ("flash_decode", "pro_decode"):
-        shape = synth.FLASH_DECODE if workload == "flash_decode" else synth.PRO_DECODE
+    if workload in DECODE_SHAPES:
+        shape, fp8 = DECODE_SHAPES[workload]
         n = max(1, threads // 2)
         while True:
-            sec, units = oracle_decode_sample(shape, min(n, shape.batch))
+            sec, units = oracle_decode_sample(shape, min(n, shape.batch), fp8=fp8)
             if sec >= budget_s / 3 or n >= shape.batch:
                 break
             n *= 2
-        desc = f"first {units} of the {shape.batch} decode queries (indexer + top-k + sparse MQA, fp64)"
+        desc = (f"first {units} of the {shape.batch} decode queries (indexer{' on e4m3 operands' if fp8 else ''} "
+                f"+ top-k + sparse MQA, fp64)")
     elif workload == "flash_attend_decode":
         shape = synth.FLASH_DECODE
         n = max(1, threads // 2)
@@ -724,9 +754,9 @@ def run_reference(args, rank, world):
     # each step: a sample of about the size measured above
     times = []
     for i in range(args.warmup + args.steps):
-        if args.workload in ("flash_decode", "pro_decode"):
-            shape = synth.FLASH_DECODE if args.workload == "flash_decode" else synth.PRO_DECODE
-            sec, u = oracle_decode_sample(shape, units)
+        if args.workload in DECODE_SHAPES:
+            shape, fp8 = DECODE_SHAPES[args.workload]
+            sec, u = oracle_decode_sample(shape, units, fp8=fp8)
         elif args.workload == "flash_attend_decode":
             sec, u = oracle_attend_sample(synth.FLASH_DECODE, units)
         elif args.workload == "flash_decode_compress":
@@ -753,7 +783,12 @@ def run_reference(args, rank, world):
     dist_done(world)
 
 
+DECODE_SHAPES = {"flash_decode": (synth.FLASH_DECODE, False), "pro_decode": (synth.PRO_DECODE, False),
+                 "flash_decode_fp8": (synth.FLASH_DECODE, True), "pro_decode_fp8": (synth.PRO_DECODE, True)}
+
 WORKLOADS_CONFIG_NAME = {
+    "flash_decode_fp8": synth.FLASH_DECODE.name + "_fp8_indexer",
+    "pro_decode_fp8": synth.PRO_DECODE.name + "_fp8_indexer",
     "flash_decode": synth.FLASH_DECODE.name,
     "pro_decode": synth.PRO_DECODE.name,
     "hca_decode": synth.HCA.name.split("_plus")[0],
@@ -874,7 +909,8 @@ def measure(name, args, rank, world, local, steps, warmup, batch=None):
 # its "extra_workloads": the other workloads the metric names (Pro-shaped
 # 1M-context decode, the long prefill chunk, HCA decode, the HCA compressor).
 # Each keeps its own step count, at most the headline's.
-EXTRA_WORKLOADS = {"pro_decode": 20, "prefill": 5, "hca_decode": 20, "hca_compress": 10}
+EXTRA_WORKLOADS = {"pro_decode": 20, "prefill": 5, "hca_decode": 20, "hca_compress": 10, "flash_decode_fp8": 20,
+                   "pro_decode_fp8": 20}
 
 
 def run_ours(args, rank, world, local):

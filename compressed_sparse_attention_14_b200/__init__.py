@@ -23,6 +23,8 @@ LIB_PATH = os.path.join(_HERE, "libcsa.so")
 
 CSA_OK, CSA_ERR_INVALID_ARG, CSA_ERR_UNSUPPORTED, CSA_ERR_WORKSPACE, CSA_ERR_CUDA, CSA_ERR_TIMEOUT = range(6)
 CSA_BF16, CSA_FP32 = 0, 1
+CSA_SCORES_BF16 = 1
+CSA_DEBUG_SKIP_FIRST_TILE = 1
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
@@ -44,6 +46,7 @@ _SIGS = {
     "csa_trace_enable": (None, [_I]),
     "csa_trace_read": (_I, [_I, _P, _P, _P, _P]),
     "csa_poll_status": (_I, [_P, _I]),
+    "csa_debug_set": (_I, [ctypes.c_uint32, ctypes.c_uint32]),
     "csa_project": (_I, [_P, _P, _I64, _I, _I, _P, _I, _P]),
     "csa_compress": (_I, [_P, _P, _P, _I64, _I, _I, _P, _I, _P]),
     "hca_compress": (_I, [_P, _P, _I64, _I, _I, _P, _I, _P]),
@@ -57,6 +60,12 @@ _SIGS = {
     "csa_topk_from_scores_noalloc": (_I, [_P, _I64, _P, _I, _I, _I64, _I, _P, _P, _P]),
     "csa_index_topk_workspace_size": (_SZ, [_I, _I64, _I, _I]),
     "csa_index_topk": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I64, _I, _I, _P, _P, _P, _SZ, _I, _P]),
+    "csa_quantize_e4m3": (_I, [_P, _I64, _I, _P, _P, _P, _P, _I, _P]),
+    "csa_index_scores_fp8": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I64, _I, _P, _P]),
+    "csa_decode_fp8_workspace_size": (_SZ, [_I, _I64, _I, _I, _I, _I, _I]),
+    "csa_decode_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I64, _I, _I, _I, _I, _I, _I, _F, _P, _I, _P, _P, _P,
+                            _P, _SZ, _P]),
+    "csa_topk_from_scores_bf16": (_I, [_P, _I64, _P, _I, _I, _I64, _I, _P, _P, _P]),
     "csa_sparse_mqa_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "csa_sparse_mqa": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I64, _I, _F, _P, _P, _P, _P, _SZ, _I, _P]),
     "hca_dense_mqa_workspace_size": (_SZ, [_I, _I, _I, _I64, _I]),
@@ -177,6 +186,13 @@ def trace_read(max_kernels: int = 64) -> dict:
 
 def poll_status(reset: bool = True) -> None:
     _check(_lib.csa_poll_status(_stream(), int(reset)))
+
+
+def debug_set(wait_limit: int = 0, flags: int = 0) -> None:
+    """Failure-path test hooks (off by default): a shorter bound on the
+    indexer's device waits, and CSA_DEBUG_SKIP_FIRST_TILE to withhold its first
+    key tile so that a wait runs out."""
+    _check(_lib.csa_debug_set(wait_limit, flags))
 
 
 def workspace_size(name: str, *args) -> int:
@@ -358,6 +374,19 @@ def csa_topk_from_scores_noalloc(scores, k: int, valid=None, valid_div: int = 1,
     return idx, top_scores
 
 
+def csa_topk_from_scores_bf16(scores, k: int, valid=None, valid_div: int = 1):
+    """Top-k over bf16 scores [nq, ncols] (same rule as csa_topk_from_scores)."""
+    nq, ncols = scores.shape
+    _dtype(scores, torch.bfloat16, "scores")
+    _dtype(valid, torch.int32, "valid")
+    _shape(valid, (nq,), "valid")
+    idx = torch.empty((nq, k), dtype=torch.int32, device=scores.device)
+    top = torch.empty((nq, k), dtype=torch.float32, device=scores.device)
+    _check(_lib.csa_topk_from_scores_bf16(_ptr(scores), ncols, _ptr(valid), valid_div, nq, ncols, k, _ptr(idx),
+                                          _ptr(top), _stream()))
+    return idx, top
+
+
 def csa_index_topk(qI, w, K, pos, m: int, k: int, seq_of_q=None, ws=None):
     nq, HI, cI = qI.shape
     K = _kv3(K)
@@ -370,6 +399,69 @@ def csa_index_topk(qI, w, K, pos, m: int, k: int, seq_of_q=None, ws=None):
                                Nmax, m, k,
                                _ptr(idx), _ptr(top), _ptr(ws), _nbytes(ws), mode, _stream()))
     return idx, top
+
+
+# ---------------------------------------------------------------- FP8 indexer
+def csa_quantize_e4m3(x, w=None):
+    """Row-wise e4m3 storage of x [..., cols] (bf16 or fp32): returns (codes,
+    a uint8 tensor of x's shape holding the e4m3 bytes (view it as
+    torch.float8_e4m3fn to read values), scales [...] fp32, w * scales or
+    None). w, when given, has the shape of the scales."""
+    cols = x.shape[-1]
+    rows = x.numel() // cols if cols else 0
+    out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    scale = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    w_out = None
+    if w is not None:
+        _dtype(w, torch.float32, "w")
+        _shape(w, tuple(x.shape[:-1]), "w")
+        w_out = torch.empty_like(w)
+    _check(_lib.csa_quantize_e4m3(_ptr(x), rows, cols, _ptr(out), _ptr(scale), _ptr(w), _ptr(w_out), _mode(x),
+                                  _stream()))
+    return out, scale, w_out
+
+
+def csa_index_scores_fp8(qI8, wq, K8, k_scale, pos, m: int, seq_of_q=None):
+    """Indexer scores from e4m3 operands: qI8 [nq, HI, cI] and K8 [B, Nmax, cI]
+    uint8 codes, wq [nq, HI] (head weights times query scales), k_scale
+    [B, Nmax]. Returns fp32 [nq, Nmax] (-inf where invisible)."""
+    nq, HI, cI = qI8.shape
+    K8 = _kv3(K8)
+    n_seq, Nmax = K8.shape[0], K8.shape[1]
+    for t, nm in ((qI8, "qI8"), (K8, "K8")):
+        _dtype(t, torch.uint8, nm)
+    _shape(wq, (nq, HI), "wq")
+    _shape(k_scale, (n_seq, Nmax), "k_scale")
+    _shape(pos, (nq,), "pos")
+    scores = torch.empty((nq, Nmax), dtype=torch.float32, device=qI8.device)
+    _check(_lib.csa_index_scores_fp8(_ptr(qI8), _ptr(wq), _ptr(K8), _ptr(k_scale), _ptr(pos), _ptr(seq_of_q), nq,
+                                     n_seq, HI, cI, Nmax, m, _ptr(scores), _stream()))
+    return scores
+
+
+def csa_decode_fp8(qI, w, idx_cache8, idx_scale, q, kv_cache, ctx_len, m: int, k: int, scale: float = 0.0,
+                   sink=None, out=None, lse=None, ws=None, return_topk: bool = False, bf16_scores: bool = False):
+    """csa_decode with the FP8 indexer: idx_cache8 [B, Nmax, cI] e4m3 codes
+    (uint8) with idx_scale [B, Nmax]; qI [B, HI, cI] bf16 is quantized inside.
+    bf16_scores: the index scores are stored and selected as bf16."""
+    B, HI, cI = qI.shape
+    _, Nmax, _ = idx_cache8.shape
+    _, H, c = q.shape
+    _dtype(idx_cache8, torch.uint8, "idx_cache8")
+    _shape(idx_cache8, (B, Nmax, cI), "idx_cache8")
+    _shape(idx_scale, (B, Nmax), "idx_scale")
+    _shape(w, (B, HI), "w")
+    _shape(kv_cache, (B, Nmax, c), "kv_cache")
+    _shape(ctx_len, (B,), "ctx_len")
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H), dtype=torch.float32, device=q.device) if lse is None else lse
+    topk_idx = torch.empty((B, k), dtype=torch.int32, device=q.device) if return_topk else None
+    ws = _ws(_lib.csa_decode_fp8_workspace_size(B, Nmax, H, c, HI, cI, k), q.device, ws)
+    _check(_lib.csa_decode_fp8(_ptr(qI), _ptr(w), _ptr(idx_cache8), _ptr(idx_scale), _ptr(q), _ptr(kv_cache),
+                               _ptr(ctx_len), B, Nmax, m, H, c, HI, cI, k, scale, _ptr(sink),
+                               CSA_SCORES_BF16 if bf16_scores else 0, _ptr(out), _ptr(lse),
+                               _ptr(topk_idx), _ptr(ws), _nbytes(ws), _stream()))
+    return (out, lse, topk_idx) if return_topk else (out, lse)
 
 
 # ---------------------------------------------------------------- a6 / a7
@@ -442,10 +534,12 @@ def csa_prefill(x, x_left, W_kv, B_kv, W_idx, B_idx, start: int, kv_cache, idx_c
     """One prefill chunk of one sequence. Without state rings the chunk starts
     and ends on block boundaries (x_left: the m hidden rows before it). With
     state_kv [2m, 4c] and state_idx [2m, 4cI] (fp32, updated in place) the
-    chunk may start and end anywhere; x_left is then ignored."""
+    chunk may start and end anywhere; x_left is then ignored. With W_kv and
+    W_idx None the caches already hold the chunk's entries and only the
+    attention runs (x gives the chunk length)."""
     n, d = x.shape
-    c = W_kv.shape[0] // 4
-    cI = W_idx.shape[0] // 4
+    c = kv_cache.shape[1] if W_kv is None else W_kv.shape[0] // 4
+    cI = idx_cache.shape[1] if W_idx is None else W_idx.shape[0] // 4
     _, H, _ = q.shape
     _, HI, _ = qI.shape
     Nmax = kv_cache.shape[0]

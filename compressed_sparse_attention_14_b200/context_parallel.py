@@ -26,10 +26,9 @@ the caches; unequal n_r are padded to the longest, gathered, and the valid
 rows of each rank copied into place (the select-and-pad step).
 
 The compute steps are the library's kernels (`csa_compress_from_hidden`,
-`csa_prefill`); the exchange is torch.distributed (NCCL over NVLink on GPUs).
-`csa_prefill` recompresses the rank's own chunk into the caches before its
-queries attend: the entries it writes are the ones already gathered, computed
-again from the same inputs. Every rank takes the same collective steps in the
+then `csa_prefill` without weights: the gathered caches already hold the
+rank's own entries, so it only attends); the exchange is torch.distributed
+(NCCL over NVLink on GPUs). Every rank takes the same collective steps in the
 same order, and every argument check that can fail runs on every rank before
 the first data exchange, so a bad argument raises on all ranks together.
 """
@@ -62,7 +61,9 @@ def cuda_ops() -> PrefillOps:
         return csa_compress_from_hidden(x, W, bias, m, x_left=x_left)
 
     def prefill(x, x_left, W_kv, B_kv, W_idx, B_idx, start, kv_cache, idx_cache, qI, w, q, k, m, scale, sink):
-        return csa_prefill(x, x_left, W_kv, B_kv, W_idx, B_idx, start, kv_cache, idx_cache, qI, w, q, k, m=m,
+        # the all-gather has put this rank's entries into the caches already:
+        # no weights, so csa_prefill attends without compressing again
+        return csa_prefill(x, None, None, None, None, None, start, kv_cache, idx_cache, qI, w, q, k, m=m,
                            scale=scale, sink=sink)
 
     return PrefillOps(compress_from_hidden=compress, prefill=prefill)

@@ -462,6 +462,23 @@ int csa_topk_from_scores(const float* scores, int64_t ld, const int32_t* valid, 
     return CSA_OK;
 }
 
+int csa_topk_from_scores_bf16(const void* scores, int64_t ld, const int32_t* valid, int valid_div, int nq,
+                              int64_t ncols, int k, int32_t* idx, float* top_scores, void* stream) {
+    CSA_TRY(check_k(k));
+    if (nq < 0 || ncols < 0 || ld < ncols || valid_div < 1)
+        return fail(CSA_ERR_INVALID_ARG, "csa_topk_from_scores_bf16: bad nq/ncols/ld/valid_div");
+    if (ncols > INT32_MAX) return fail(CSA_ERR_UNSUPPORTED, "ncols beyond int32 indices");
+    CSA_TRY(check_rows(nq, "csa_topk_from_scores_bf16"));
+    if (nq == 0) return CSA_OK;
+    if (ncols > 0) CSA_TRY(check_ptr(scores, "scores"));
+    CSA_TRY(check_ptr(valid, "valid", false));
+    CSA_TRY(check_ptr(idx, "idx"));
+    CSA_TRY(check_ptr(top_scores, "top_scores", false));
+    CSA_CUDA(topk_select_bf16(scores, ld, valid, valid_div, nq, ncols, k, idx, top_scores, (cudaStream_t)stream),
+             "csa_topk_from_scores_bf16");
+    return CSA_OK;
+}
+
 size_t csa_index_topk_workspace_size(int nq, int64_t Nmax, int k, int dtype) {
     (void)dtype;
     if (nq < 0 || Nmax < 0 || k < 1) return 0;
@@ -498,6 +515,112 @@ int csa_index_topk(const void* qI, const float* w, const void* K, const int32_t*
     CSA_CUDA(run_indexer(qI, w, K, qs, nq, n_seq, HI, cI, Nmax, m, sc, Nmax, 1, false, t, st), "csa_index_topk: scores");
     CSA_CUDA(topk_select(sc, Nmax, pos, m, nq, Nmax, k, idx, top_scores, tws, st, seq_of_q, n_seq),
              "csa_index_topk: top-k");
+    return CSA_OK;
+}
+
+// ---------------------------------------------------------------- FP8 indexer
+int csa_quantize_e4m3(const void* x, int64_t rows, int cols, void* out, float* scale, const float* w, float* w_out,
+                      int dtype, void* stream) {
+    ElemType t = ElemType::BF16;   // set by check_dtype
+    CSA_TRY(check_dtype(dtype, &t));
+    if (rows < 0 || cols < 8 || cols % 8) return fail(CSA_ERR_INVALID_ARG, "rows=%lld cols=%d: cols must be a "
+                                                      "positive multiple of 8", (long long)rows, cols);
+    if ((rows + 7) / 8 > INT32_MAX) return fail(CSA_ERR_UNSUPPORTED, "rows beyond one launch");
+    if ((w == nullptr) != (w_out == nullptr)) return fail(CSA_ERR_INVALID_ARG, "w and w_out go together");
+    if (rows == 0) return CSA_OK;
+    CSA_TRY(check_ptr(x, "x"));
+    CSA_TRY(check_ptr(out, "out"));
+    CSA_TRY(check_ptr(scale, "scale"));
+    CSA_TRY(check_ptr(w, "w", false));
+    CSA_TRY(check_ptr(w_out, "w_out", false));
+    CSA_CUDA(quantize_e4m3(x, rows, cols, out, scale, w, w_out, t, (cudaStream_t)stream), "csa_quantize_e4m3");
+    return CSA_OK;
+}
+
+static int check_index_fp8(int HI, int cI) {
+    CSA_TRY(check_index_shape(HI, cI));
+    if (!index_tc_supported(HI, cI, 1, true))
+        return fail(CSA_ERR_UNSUPPORTED, "FP8 indexer needs cI a multiple of 128 (<= 256) (cI=%d)", cI);
+    return CSA_OK;
+}
+
+int csa_index_scores_fp8(const void* qI8, const float* wq, const void* K8, const float* k_scale, const int32_t* pos,
+                         const int32_t* seq_of_q, int nq, int n_seq, int HI, int cI, int64_t Nmax, int m,
+                         float* scores, void* stream) {
+    CSA_TRY(check_index_fp8(HI, cI));
+    CSA_TRY(check_rows(nq, "csa_index_scores_fp8"));
+    if (nq < 0 || Nmax < 0 || m < 1 || n_seq < 1) return fail(CSA_ERR_INVALID_ARG, "bad nq/n_seq/Nmax/m");
+    if (!seq_of_q && n_seq < nq) return fail(CSA_ERR_INVALID_ARG, "seq_of_q is NULL (query t reads sequence t) but n_seq < nq");
+    if (Nmax > INT32_MAX) return fail(CSA_ERR_UNSUPPORTED, "Nmax beyond int32 entry indices");
+    CSA_TRY(check_cache_rows(n_seq, Nmax));
+    if (nq == 0 || Nmax == 0) return CSA_OK;
+    CSA_TRY(check_ptr(qI8, "qI8"));
+    CSA_TRY(check_ptr(wq, "wq"));
+    CSA_TRY(check_ptr(K8, "K8"));
+    CSA_TRY(check_ptr(k_scale, "k_scale"));
+    CSA_TRY(check_ptr(pos, "pos"));
+    CSA_TRY(check_ptr(seq_of_q, "seq_of_q", false));
+    CSA_TRY(check_ptr(scores, "scores"));
+    QuerySpec qs{seq_of_q, pos, 0, 0};
+    CSA_CUDA(index_scores_tc(qI8, wq, K8, qs, nq, n_seq, HI, cI, Nmax, m, scores, Nmax, 1, true, device_status(),
+                             (cudaStream_t)stream, k_scale), "csa_index_scores_fp8");
+    return CSA_OK;
+}
+
+size_t csa_decode_fp8_workspace_size(int B, int64_t Nmax, int H, int c, int HI, int cI, int k) {
+    if (B < 0 || Nmax < 0 || k < 1 || H < 1 || c < 1 || HI < 1 || cI < 1) return 0;
+    return align256((size_t)B * HI * cI) + 2 * align256((size_t)B * HI * sizeof(float)) +
+           index_topk_bytes(B, Nmax, k) + align256((size_t)B * k * sizeof(int32_t)) +
+           mqa_workspace_bytes(B, H, c, k, ElemType::BF16);
+}
+
+int csa_decode_fp8(const void* qI, const float* w, const void* idx_cache8, const float* idx_scale, const void* q,
+                   const void* kv_cache, const int32_t* ctx_len, int B, int64_t Nmax, int m, int H, int c, int HI,
+                   int cI, int k, float scale, const float* sink, int flags, void* out, float* lse, int32_t* topk_idx,
+                   void* ws, size_t ws_bytes, void* stream) {
+    CSA_TRY(check_index_fp8(HI, cI));
+    if (flags & ~CSA_SCORES_BF16) return fail(CSA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+    const bool sbf = (flags & CSA_SCORES_BF16) != 0;
+    CSA_TRY(check_attn_shape(H, c));
+    CSA_TRY(check_attn_mode(H, c, ElemType::BF16));
+    CSA_TRY(check_cache_rows(B, Nmax));
+    CSA_TRY(check_k(k));
+    CSA_TRY(check_rows(B, "csa_decode_fp8"));
+    if (B < 0 || Nmax < 0 || m < 1) return fail(CSA_ERR_INVALID_ARG, "bad B/Nmax/m");
+    if (Nmax > INT32_MAX) return fail(CSA_ERR_UNSUPPORTED, "Nmax beyond int32 entry indices");
+    if (B == 0) return CSA_OK;
+    CSA_TRY(check_ptr(qI, "qI"));
+    CSA_TRY(check_ptr(w, "w"));
+    CSA_TRY(check_ptr(idx_cache8, "idx_cache8", Nmax > 0));
+    CSA_TRY(check_ptr(idx_scale, "idx_scale", Nmax > 0));
+    CSA_TRY(check_ptr(q, "q"));
+    CSA_TRY(check_ptr(kv_cache, "kv_cache", Nmax > 0));
+    CSA_TRY(check_ptr(ctx_len, "ctx_len"));
+    CSA_TRY(check_ptr(sink, "sink", false));
+    CSA_TRY(check_ptr(out, "out"));
+    CSA_TRY(check_ptr(lse, "lse", false));
+    CSA_TRY(check_ptr(topk_idx, "topk_idx", false));
+    CSA_TRY(check_ws(ws, ws_bytes, csa_decode_fp8_workspace_size(B, Nmax, H, c, HI, cI, k)));
+    cudaStream_t st = (cudaStream_t)stream;
+    Carve cv(ws);
+    void* q8 = cv.take((size_t)B * HI * cI);
+    float* qs8 = (float*)cv.take((size_t)B * HI * sizeof(float));
+    float* wq = (float*)cv.take((size_t)B * HI * sizeof(float));
+    float* sc = (float*)cv.take((size_t)B * Nmax * sizeof(float));
+    void* tws = cv.take(topk_workspace_bytes(B, Nmax, k));
+    int32_t* sel = (int32_t*)cv.take((size_t)B * k * sizeof(int32_t));
+    void* mws = cv.take(mqa_workspace_bytes(B, H, c, k, ElemType::BF16));
+    if (topk_idx) sel = topk_idx;
+    QuerySpec qs{nullptr, ctx_len, 0, 0};
+    CSA_CUDA(quantize_e4m3(qI, (int64_t)B * HI, cI, q8, qs8, w, wq, ElemType::BF16, st), "csa_decode_fp8: quantize q");
+    CSA_CUDA(index_scores_tc(q8, wq, idx_cache8, qs, B, B, HI, cI, Nmax, m, sc, Nmax, 1, false, device_status(), st,
+                             idx_scale, sbf), "csa_decode_fp8: indexer");
+    if (sbf)
+        CSA_CUDA(topk_select_bf16(sc, Nmax, ctx_len, m, B, Nmax, k, sel, nullptr, st), "csa_decode_fp8: top-k");
+    else
+        CSA_CUDA(topk_select(sc, Nmax, ctx_len, m, B, Nmax, k, sel, nullptr, tws, st), "csa_decode_fp8: top-k");
+    CSA_CUDA(mqa(q, kv_cache, sel, k, qs, 1, B, B, H, c, Nmax, default_scale(scale, c), sink, out, lse, mws,
+                 ElemType::BF16, st), "csa_decode_fp8: mqa");
     return CSA_OK;
 }
 
@@ -659,25 +782,32 @@ int csa_prefill(const void* x, const void* x_left, const void* W_kv, const float
     const bool stateful = state_kv || state_idx;
     if (stateful && !(state_kv && state_idx))
         return fail(CSA_ERR_INVALID_ARG, "state_kv and state_idx go together (both or neither)");
+    // no weights: the chunk's entries are already in the caches (compressed
+    // elsewhere, e.g. gathered from the ranks that own them); attend only
+    const bool attend_only = !W_kv && !W_idx;
+    if (attend_only && stateful)
+        return fail(CSA_ERR_INVALID_ARG, "state rings given without compressor weights");
     CSA_TRY(check_compress(stateful ? 0 : n, c, m, 64, "csa_prefill"));
     if (n < 0) return fail(CSA_ERR_INVALID_ARG, "n=%lld is negative", (long long)n);
     if (d < 8 || d % 8) return fail(CSA_ERR_INVALID_ARG, "d=%d must be a positive multiple of 8", d);
     if (start < 0) return fail(CSA_ERR_INVALID_ARG, "start=%lld is negative", (long long)start);
-    if (!stateful && start % m)
+    if (!stateful && !attend_only && start % m)
         return fail(CSA_ERR_INVALID_ARG, "start=%lld is not a multiple of m (pass the state rings to start "
                     "mid-block)", (long long)start);
-    if (!stateful && start > 0 && !x_left)
+    if (!stateful && !attend_only && start > 0 && !x_left)
         return fail(CSA_ERR_INVALID_ARG, "x_left is required when start > 0 (or pass the state rings)");
     if ((start + n) / m > Nmax) return fail(CSA_ERR_INVALID_ARG, "caches hold %lld entries, %lld needed",
                                             (long long)Nmax, (long long)((start + n) / m));
     if (Nmax > INT32_MAX || start + n > INT32_MAX) return fail(CSA_ERR_UNSUPPORTED, "positions beyond int32");
     if (n == 0) return CSA_OK;
-    CSA_TRY(check_ptr(x, "x"));
+    CSA_TRY(check_ptr(x, "x", !attend_only));
     CSA_TRY(check_ptr(x_left, "x_left", false));
-    CSA_TRY(check_ptr(W_kv, "W_kv"));
-    CSA_TRY(check_ptr(B_kv, "B_kv"));
-    CSA_TRY(check_ptr(W_idx, "W_idx"));
-    CSA_TRY(check_ptr(B_idx, "B_idx"));
+    CSA_TRY(check_ptr(W_kv, "W_kv", !attend_only));
+    CSA_TRY(check_ptr(B_kv, "B_kv", !attend_only));
+    CSA_TRY(check_ptr(W_idx, "W_idx", !attend_only));
+    CSA_TRY(check_ptr(B_idx, "B_idx", !attend_only));
+    if (attend_only != (!W_kv || !W_idx))
+        return fail(CSA_ERR_INVALID_ARG, "W_kv and W_idx go together (both, or neither to attend only)");
     CSA_TRY(check_ptr(kv_cache, "kv_cache"));
     CSA_TRY(check_ptr(idx_cache, "idx_cache"));
     CSA_TRY(check_ptr(state_kv, "state_kv", false));
@@ -710,6 +840,7 @@ int csa_prefill(const void* x, const void* x_left, const void* W_kv, const float
     struct { const void* W; const float* B; int cc; void* cache; float* state; } streams[2] = {
         {W_kv, B_kv, c, kv_cache, state_kv}, {W_idx, B_idx, cI, idx_cache, state_idx}};
     for (auto& s : streams) {
+        if (attend_only) break;
         CSA_CUDA(project(x, s.W, n, d, 4 * s.cc, proj, t, st), "csa_prefill: projection");
         if (stateful) {
             CSA_CUDA(compress_chunk_state(proj, s.state, s.B, start, n, s.cc, m, true, s.cache, t, st),

@@ -25,6 +25,14 @@
 //              coalesced fp32 score stores.
 // Every wait is bounded; a timeout records CSA_ERR_TIMEOUT in the status
 // word, stops all roles, drains the copies in flight and frees TMEM.
+//
+// FP8 variant [Notes §2.4 (low-precision indexer arithmetic) and §1.3
+// (FP8 storage)]: q^I and K stored as e4m3 with one fp32 scale per query-head
+// row and per key row; tcgen05.mma kind::f8f6f4 (K = 32 per instruction, so a
+// 128-byte shared-memory row holds 128 channels). The scales are positive, so
+// they leave the ReLU: sum_h w_h ReLU(sq_h sk x_h) = sk sum_h (w_h sq_h)
+// ReLU(x_h). The caller passes w_h sq_h as the head weights and the key
+// scales; the epilogue multiplies each key's sum by its scale.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -48,18 +56,23 @@ struct IdxArgs {
     int stages;
     int64_t Nmax;
     int m;
-    const float* w;     // [nq][HI]
-    float* scores;      // [nq][ld]
+    const float* w;     // [nq][HI] (FP8: w times the query-head scale)
+    const float* kscale;    // FP8: [n_seq * Nmax] key scales; nullptr for bf16
+    int blk_elems;      // elements per 128-byte row of a tile (64 bf16, 128 e4m3)
+    float* scores;      // [nq][ld] fp32, or bf16 values when score_bf16
+    int score_bf16;
     int64_t ld;
     int* status;
     uint32_t stage_bytes, q_bytes, tmem_cols;
+    uint32_t wait_limit;    // polls before a wait gives up (CSA_ERR_TIMEOUT)
+    int skip_first_tile;    // failure-path test hook: the first key tile is never loaded
     int nbuf;           // TMEM accumulator buffers (2..4)
 };
 
 struct Smem {
     uint8_t* stage0;    // stages x stage_bytes
     uint8_t* q;         // q_bytes
-    float* w;           // [2][256], one copy per epilogue set
+    float* w;           // [8][256], one copy per epilogue warp
     uint64_t* full;     // [stages]
     uint64_t* empty;    // [stages]
     uint64_t* tfull;    // [4]
@@ -74,7 +87,7 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const IdxArgs& a) {
     s.stage0 = base;
     s.q = base + (size_t)a.stages * a.stage_bytes;
     s.w = (float*)(s.q + a.q_bytes);
-    uint64_t* bars = (uint64_t*)(s.w + 512);
+    uint64_t* bars = (uint64_t*)(s.w + 8 * 256);
     s.full = bars;
     s.empty = bars + a.stages;
     s.tfull = bars + 2 * a.stages;
@@ -171,8 +184,8 @@ __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
 }
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                              int* status) {
-    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+                                              int* status, uint32_t limit) {
+    for (uint32_t i = 0; i < limit; ++i) {
         if (tc::mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 255u && *abort_flag) return false;
     }
@@ -183,6 +196,7 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 
 }  // namespace
 
+template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __grid_constant__ IdxArgs a,
                                                                       const __grid_constant__ CUtensorMap tmK,
                                                                       const __grid_constant__ CUtensorMap tmQ) {
@@ -239,27 +253,29 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
             int64_t it = 0;
             for (; it < my; ++it) {
                 if (wk.g != cur) {
-                    if (switches > 0 && !wait_or_abort(sm.qempty, (switches - 1) & 1, abort_flag, a.status)) break;
+                    if (switches > 0 && !wait_or_abort(sm.qempty, (switches - 1) & 1, abort_flag, a.status, a.wait_limit)) break;
                     tc::mbar_expect_tx(sm.qfull, a.q_bytes);
                     for (int kb = 0; kb < a.kblocks; ++kb)
-                        tc::tma_load_2d(sm.q + (size_t)kb * a.npad * 128, &tmQ, sm.qfull, kb * 64,
+                        tc::tma_load_2d(sm.q + (size_t)kb * a.npad * 128, &tmQ, sm.qfull, kb * a.blk_elems,
                                         wk.g * a.group * a.HI);
                     cur = wk.g;
                     ++switches;
                 }
                 const int s = (int)(it % a.stages);
-                if (it >= a.stages && !wait_or_abort(&sm.empty[s], ((it / a.stages) - 1) & 1, abort_flag, a.status))
+                if (it >= a.stages && !wait_or_abort(&sm.empty[s], ((it / a.stages) - 1) & 1, abort_flag, a.status, a.wait_limit))
                     break;
-                tc::mbar_expect_tx(&sm.full[s], a.stage_bytes);
-                const int row = (int)((int64_t)group_seq(a, wk.g) * a.Nmax + wk.t * kKeys);
-                uint8_t* dst = sm.stage0 + (size_t)s * a.stage_bytes;
-                for (int kb = 0; kb < a.kblocks; ++kb)
-                    tc::tma_load_2d(dst + (size_t)kb * kKeys * 128, &tmK, &sm.full[s], kb * 64, row);
+                if (!(a.skip_first_tile && it == 0)) {
+                    tc::mbar_expect_tx(&sm.full[s], a.stage_bytes);
+                    const int row = (int)((int64_t)group_seq(a, wk.g) * a.Nmax + wk.t * kKeys);
+                    uint8_t* dst = sm.stage0 + (size_t)s * a.stage_bytes;
+                    for (int kb = 0; kb < a.kblocks; ++kb)
+                        tc::tma_load_2d(dst + (size_t)kb * kKeys * 128, &tmK, &sm.full[s], kb * a.blk_elems, row);
+                }
                 wk.next(a, ngroups);
             }
             // drain: the copies of the last `stages` tiles (and the last Q) must land
             for (int64_t j = (it > a.stages ? it - a.stages : 0); j < it; ++j)
-                tc::mbar_wait(&sm.full[j % a.stages], (j / a.stages) & 1, kWaitLimit);
+                if (!(a.skip_first_tile && j == 0)) tc::mbar_wait(&sm.full[j % a.stages], (j / a.stages) & 1, kWaitLimit);
             if (switches > 0) tc::mbar_wait(sm.qfull, (switches - 1) & 1, kWaitLimit);
         }
     } else if (warp == 1) {
@@ -269,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
             wk.start(a, g0, t0);
             int cur = -1;
             uint32_t switches = 0;
-            const uint32_t idesc = tc::idesc_bf16_f32(128, a.npad, 0, 0);
+            const uint32_t idesc = kFp8 ? tc::idesc_e4m3_f32(128, a.npad, 0, 0) : tc::idesc_bf16_f32(128, a.npad, 0, 0);
             // descriptors built once; a K step or a stage only moves the start
             // address field (bits 0-13, in 16-byte units), so it is added in place
             const uint64_t a_desc0 = tc::sdesc_sw128(tc::smem_u32(sm.stage0), 16, 1024);
@@ -280,15 +296,15 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
             int64_t it = 0;
             for (; it < my; ++it) {
                 if (wk.g != cur) {
-                    if (!wait_or_abort(sm.qfull, switches & 1, abort_flag, a.status)) break;
+                    if (!wait_or_abort(sm.qfull, switches & 1, abort_flag, a.status, a.wait_limit)) break;
                     cur = wk.g;
                     ++switches;
                 }
                 const int s = (int)(it % a.stages);
                 const int buf = (int)(it % a.nbuf);
                 const int64_t use = it / a.nbuf;
-                if (!wait_or_abort(&sm.full[s], (it / a.stages) & 1, abort_flag, a.status)) break;
-                if (use >= 1 && !wait_or_abort(&sm.tempty[buf], (use - 1) & 1, abort_flag, a.status)) break;
+                if (!wait_or_abort(&sm.full[s], (it / a.stages) & 1, abort_flag, a.status, a.wait_limit)) break;
+                if (use >= 1 && !wait_or_abort(&sm.tempty[buf], (use - 1) & 1, abort_flag, a.status, a.wait_limit)) break;
                 tc::tc_fence_after();
                 const uint64_t a_s = a_desc0 + (uint64_t)(s * stage_step);
                 const uint32_t d = tmem + (uint32_t)(buf * a.npad);
@@ -296,8 +312,10 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
                     const uint64_t ad = a_s + (uint64_t)(kb * a_kb_step);
                     const uint64_t bd = b_desc0 + (uint64_t)(kb * b_kb_step);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)   // 16 bf16 = 32 bytes = 2 units per K step
-                        tc::umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) ? 1u : 0u);
+                    for (int kk = 0; kk < 4; ++kk) {   // 32 bytes = 2 units per K step
+                        if constexpr (kFp8) tc::umma_f8(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) ? 1u : 0u);
+                        else tc::umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) ? 1u : 0u);
+                    }
                 }
                 tc::umma_commit(&sm.empty[s]);
                 tc::umma_commit(&sm.tfull[buf]);
@@ -315,8 +333,10 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
         const int set = (warp - 2) >> 2;
         const int quad = warp & 3;
         const int row = quad * 32 + lane;          // key within the tile
-        const int ethread = (warp - 2 - 4 * set) * 32 + lane;   // 0..127 within the set
-        float* wv = sm.w + set * 256;
+        // each epilogue warp keeps its own copy of the group's head weights, so
+        // that no barrier ties the warps of a set together (a warp that stops
+        // on a timeout can never leave the others waiting)
+        float* wv = sm.w + (warp - 2) * 256;
         Walk wk;
         wk.start(a, g0, t0);
         int cur = -1;
@@ -324,20 +344,23 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
         for (int64_t it = 0; it < my; ++it, wk.next(a, ngroups)) {
             if ((int)(it & 1) != set) continue;
             if (wk.g != cur) {
-                if (set == 0) asm volatile("bar.sync 1, 128;" ::: "memory");
-                else asm volatile("bar.sync 2, 128;" ::: "memory");
-                for (int c = ethread; c < a.npad; c += 128) {
+                __syncwarp();
+                for (int c = lane; c < a.npad; c += 32) {
                     const int gq = c / a.HI, h = c % a.HI;
                     const int tq = wk.g * a.group + gq;
                     wv[c] = (gq < a.group && tq < a.nq) ? a.w[(int64_t)tq * a.HI + h] : 0.f;
                 }
-                if (set == 0) asm volatile("bar.sync 1, 128;" ::: "memory");
-                else asm volatile("bar.sync 2, 128;" ::: "memory");
+                __syncwarp();
                 cur = wk.g;
                 vis = group_visible(a, wk.g);
             }
             const int buf = (int)(it % a.nbuf);
-            if (!wait_or_abort(&sm.tfull[buf], (uint32_t)((it / a.nbuf) & 1), abort_flag, a.status)) break;
+            const int64_t key = wk.t * kKeys + row;
+            // FP8: the key's scale, loaded before the wait so its latency hides
+            float kscale = 1.f;
+            if constexpr (kFp8)
+                if (key < vis) kscale = __ldg(a.kscale + (int64_t)group_seq(a, wk.g) * a.Nmax + key);
+            if (!wait_or_abort(&sm.tfull[buf], (uint32_t)((it / a.nbuf) & 1), abort_flag, a.status, a.wait_limit)) break;
             tc::tc_fence_after();
             float sc[4] = {0.f, 0.f, 0.f, 0.f};
             const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * a.npad);
@@ -383,12 +406,17 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&sm.tempty[buf]);
-            const int64_t key = wk.t * kKeys + row;
             if (key < vis) {
 #pragma unroll
                 for (int gq = 0; gq < 4; ++gq) {
                     const int tq = wk.g * a.group + gq;
-                    if (gq < a.group && tq < a.nq) a.scores[(int64_t)tq * a.ld + key] = sc[gq];
+                    if (gq < a.group && tq < a.nq) {
+                        const float v = kFp8 ? sc[gq] * kscale : sc[gq];
+                        if (a.score_bf16)
+                            reinterpret_cast<bf16*>(a.scores)[(int64_t)tq * a.ld + key] = __float2bfloat16_rn(v);
+                        else
+                            a.scores[(int64_t)tq * a.ld + key] = v;
+                    }
                 }
             }
         }
@@ -425,8 +453,8 @@ static int num_sms() {
     return n;
 }
 
-bool index_tc_supported(int HI, int cI, int group) {
-    if (cI % 64 != 0 || cI > 256) return false;
+bool index_tc_supported(int HI, int cI, int group, bool fp8) {
+    if (cI % (fp8 ? 128 : 64) != 0 || cI > 256) return false;
     if (group < 1 || group > 4) return false;
     if (group > 1 && HI % 16 != 0) return false;
     int n = group * HI;
@@ -435,7 +463,10 @@ bool index_tc_supported(int HI, int cI, int group) {
 
 cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, QuerySpec qs, int nq, int n_seq, int HI,
                             int cI, int64_t Nmax, int m, float* scores, int64_t ld, int group, bool fill_invisible,
-                            int* status, cudaStream_t st) {
+                            int* status, cudaStream_t st, const float* kscale, bool score_bf16) {
+    if (score_bf16 && fill_invisible) return cudaErrorInvalidValue;
+    const bool fp8 = kscale != nullptr;
+    const int es = fp8 ? 1 : 2;
     if (nq == 0 || Nmax == 0) return cudaSuccess;
     IdxArgs a{};
     a.qm = QueryMap{qs.seq, qs.pos, qs.pos_base, qs.single_seq};
@@ -446,15 +477,20 @@ cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, Query
     a.cI = cI;
     int n = group * HI;
     a.npad = n < 16 ? 16 : ((n + 15) / 16) * 16;
-    a.kblocks = cI / 64;
+    a.kblocks = cI * es / 128;
+    a.blk_elems = 128 / es;
+    a.kscale = kscale;
     a.Nmax = Nmax;
     a.m = m;
     a.w = w;
     a.scores = scores;
+    a.score_bf16 = score_bf16 ? 1 : 0;
+    a.wait_limit = debug_wait_limit() ? debug_wait_limit() : kWaitLimit;
+    a.skip_first_tile = (debug_flags() & CSA_DEBUG_SKIP_FIRST_TILE) ? 1 : 0;
     a.ld = ld;
     a.status = status;
-    a.stage_bytes = (uint32_t)(kKeys * cI * 2);
-    a.q_bytes = (uint32_t)(a.npad * cI * 2);
+    a.stage_bytes = (uint32_t)(kKeys * cI * es);
+    a.q_bytes = (uint32_t)(a.npad * cI * es);
     // as many accumulator buffers (2..4) as fit 512 TMEM columns
     a.nbuf = 512 / a.npad;
     if (a.nbuf > 4) a.nbuf = 4;
@@ -462,17 +498,22 @@ cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, Query
     uint32_t cols = 32;
     while (cols < (uint32_t)(a.nbuf * a.npad)) cols <<= 1;
     a.tmem_cols = cols;
-    const size_t fixed = 1024 + a.q_bytes + 512 * sizeof(float) + 64 * sizeof(uint64_t);
+    const size_t fixed = 1024 + a.q_bytes + 8 * 256 * sizeof(float) + 64 * sizeof(uint64_t);
     const size_t budget = 226 * 1024;
     int stages = (int)((budget - fixed) / a.stage_bytes);
-    if (stages > 8) stages = 8;
+    if (stages > (fp8 ? 12 : 8)) stages = fp8 ? 12 : 8;
     if (stages < 2) return cudaErrorInvalidConfiguration;
     a.stages = stages;
     const size_t smem = fixed + (size_t)stages * a.stage_bytes;
 
     CUtensorMap tmK, tmQ;
-    if (!make_tmap_bf16_2d(&tmK, K, (uint64_t)n_seq * Nmax, cI, cI, kKeys, 64)) return cudaErrorInvalidValue;
-    if (!make_tmap_bf16_2d(&tmQ, qI, (uint64_t)nq * HI, cI, cI, a.npad, 64)) return cudaErrorInvalidValue;
+    if (fp8) {
+        if (!make_tmap_u8_2d(&tmK, K, (uint64_t)n_seq * Nmax, cI, cI, kKeys, 128)) return cudaErrorInvalidValue;
+        if (!make_tmap_u8_2d(&tmQ, qI, (uint64_t)nq * HI, cI, cI, a.npad, 128)) return cudaErrorInvalidValue;
+    } else {
+        if (!make_tmap_bf16_2d(&tmK, K, (uint64_t)n_seq * Nmax, cI, cI, kKeys, 64)) return cudaErrorInvalidValue;
+        if (!make_tmap_bf16_2d(&tmQ, qI, (uint64_t)nq * HI, cI, cI, a.npad, 64)) return cudaErrorInvalidValue;
+    }
 
     cudaError_t e;
     if (fill_invisible) {
@@ -483,10 +524,11 @@ cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, Query
         if (e == cudaSuccess) e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    e = smem_ceiling(index_scores_tc_kernel);
+    auto kern = fp8 ? index_scores_tc_kernel<true> : index_scores_tc_kernel<false>;
+    e = smem_ceiling(kern);
     if (e != cudaSuccess) return e;
-    CSA_LAUNCH(st, "index_scores_tc",
-               e = launch_pdl(index_scores_tc_kernel, dim3(num_sms()), dim3(kThreads), smem, st, 0, a, tmK, tmQ));
+    CSA_LAUNCH(st, fp8 ? "index_scores_tc_fp8" : "index_scores_tc",
+               e = launch_pdl(kern, dim3(num_sms()), dim3(kThreads), smem, st, 0, a, tmK, tmQ));
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

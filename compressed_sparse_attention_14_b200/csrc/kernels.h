@@ -64,6 +64,10 @@ cudaError_t smem_ceiling(void (*kern)(KArgs...)) {
     return smem_ceiling(reinterpret_cast<const void*>(kern));
 }
 
+// launch.cu: the failure-path test hooks set by csa_debug_set (0 = off).
+uint32_t debug_wait_limit();
+uint32_t debug_flags();
+
 inline size_t elem_size(ElemType t) { return t == ElemType::BF16 ? 2 : 4; }
 inline size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
 
@@ -112,10 +116,21 @@ cudaError_t index_scores(const void* qI, const float* w, const void* K, QuerySpe
                          ElemType t, cudaStream_t st);
 // indexer_tc.cu (tcgen05, bf16): groups of `group` consecutive queries share
 // one visible range; fill_invisible writes -inf past each visible range.
-bool index_tc_supported(int HI, int cI, int group);
+// With kscale (fp32 [n_seq * Nmax]) qI and K are e4m3 bytes, w holds the
+// head weights times the query-head scales, and each key's sum is scaled.
+// score_bf16: scores are stored as bf16 (nearest, ties to even), row stride
+// ld bf16 values (no fill_invisible).
+bool index_tc_supported(int HI, int cI, int group, bool fp8 = false);
 cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, QuerySpec qs, int nq, int n_seq, int HI,
                             int cI, int64_t Nmax, int m, float* scores, int64_t ld, int group, bool fill_invisible,
-                            int* status, cudaStream_t st);
+                            int* status, cudaStream_t st, const float* kscale = nullptr,
+                            bool score_bf16 = false);
+
+// quant.cu: row-wise e4m3 codes out [rows, cols] and fp32 scales
+// s = max|row| / 448 (1 for a zero row), decided in fp64; w_out = w * s when
+// w is given (one head weight per row).
+cudaError_t quantize_e4m3(const void* x, int64_t rows, int cols, void* out, float* scale, const float* w, float* w_out,
+                          ElemType t, cudaStream_t st);
 
 // api.cu: device address of the status word on the current device
 int* device_status();
@@ -126,6 +141,10 @@ size_t topk_workspace_bytes(int nq, int64_t ncols, int k);
 cudaError_t topk_select(const float* scores, int64_t ld, const int32_t* valid, int valid_div,
                         int nq, int64_t ncols, int k, int32_t* idx, float* top_scores, void* ws,
                         cudaStream_t st, const int32_t* seq = nullptr, int n_seq = 0);
+// as topk_select on bf16 scores (row stride ld bf16 values)
+cudaError_t topk_select_bf16(const void* scores, int64_t ld, const int32_t* valid, int valid_div, int nq,
+                             int64_t ncols, int k, int32_t* idx, float* top_scores, cudaStream_t st,
+                             const int32_t* seq = nullptr, int n_seq = 0);
 // as topk_select with the candidate count of row t = (pos_base + t) / m
 cudaError_t topk_select_positions(const float* scores, int64_t ld, int64_t pos_base, int m, int nq,
                                   int64_t ncols, int k, int32_t* idx, void* ws, cudaStream_t st);

@@ -15,4 +15,8 @@ namespace csa {
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t pitch_elems,
                        uint32_t box_rows, uint32_t box_cols);
 
+// The same for a byte matrix (e4m3 values): row pitch in bytes, box_cols <= 128.
+bool make_tmap_u8_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t pitch_bytes,
+                     uint32_t box_rows, uint32_t box_cols);
+
 }  // namespace csa

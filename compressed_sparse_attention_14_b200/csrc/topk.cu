@@ -10,6 +10,10 @@
 // +0.0). Composite keys are distinct and their descending order is exactly
 // the selection order, so the k largest composites ARE the answer.
 //
+// Scores are read as fp32, or as bf16 [Notes §2.4: index scores quantized
+// to BF16 halve the selector's reads]: a bf16 score widens exactly to fp32,
+// so the order is the same as on fp32 scores holding those values.
+//
 // One launch, no global scratch; a row is served by one CTA, or by a cluster
 // of G CTAs (G = 2, 4, 8 when there are few long rows, so that the row's
 // pass over its scores has G SMs' worth of loads in flight):
@@ -50,6 +54,25 @@ __device__ __forceinline__ float from_orderable(uint32_t k) {
 __device__ __forceinline__ uint64_t composite(float s, int64_t col) {
     return ((uint64_t)orderable(s) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)col);
 }
+// One score, widened to fp32 (L2-cached load: each is read once).
+__device__ __forceinline__ float ld_score(const float* p) { return __ldcg(p); }
+__device__ __forceinline__ float ld_score(const bf16* p) {
+    return __uint_as_float((uint32_t)__ldcg(reinterpret_cast<const unsigned short*>(p)) << 16);
+}
+// 16 bytes of scores, widened: 4 fp32 or 8 bf16.
+__device__ __forceinline__ void ld_vec(const float* p, float* f) {
+    const float4 q = __ldcg(reinterpret_cast<const float4*>(p));
+    f[0] = q.x; f[1] = q.y; f[2] = q.z; f[3] = q.w;
+}
+__device__ __forceinline__ void ld_vec(const bf16* p, float* f) {
+    const uint4 q = __ldcg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
 
 namespace cg = cooperative_groups;
 
@@ -72,7 +95,8 @@ constexpr size_t kSmemSpread = 160 * 1024;
 
 // The candidate columns of each row: 0 .. count(row) - 1.
 struct RowSpec {
-    const float* scores;
+    const void* scores;       // fp32, or bf16 when bf16 != 0
+    int bf16;
     int64_t ld;
     const int32_t* valid;     // nullable
     int valid_div;
@@ -101,9 +125,10 @@ struct SmemSrc {
     const uint64_t* e;
     __device__ __forceinline__ uint64_t operator()(int64_t i) const { return e[i]; }
 };
+template <typename TS>
 struct RowSrc {
-    const float* row;
-    __device__ __forceinline__ uint64_t operator()(int64_t i) const { return composite(row[i], i); }
+    const TS* row;
+    __device__ __forceinline__ uint64_t operator()(int64_t i) const { return composite(ld_score(row + i), i); }
 };
 
 // Largest T such that exactly min(k, n) elements are >= T (distinct keys).
@@ -364,7 +389,8 @@ __device__ __forceinline__ void bins_clear(BinShared& bs) {
 // Threshold estimate from the row's strided sample: the smallest key of the
 // bin that holds the sample's r-th largest score, so that at least r sample
 // scores reach it.
-__device__ uint32_t sample_threshold(const float* srow, int64_t n, int r, BinShared& bs) {
+template <typename TS>
+__device__ uint32_t sample_threshold(const TS* srow, int64_t n, int r, BinShared& bs) {
     constexpr int kPer = kSample / kThreads;
     const int tid = threadIdx.x;
     uint32_t key[kPer];
@@ -372,7 +398,7 @@ __device__ uint32_t sample_threshold(const float* srow, int64_t n, int r, BinSha
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
         const int t = u * kThreads + tid;
-        key[u] = orderable(__ldcg(srow + ((int64_t)t * n) / kSample));
+        key[u] = orderable(ld_score(srow + ((int64_t)t * n) / kSample));
         lo = min(lo, key[u]);
         hi = max(hi, key[u]);
     }
@@ -474,39 +500,40 @@ __device__ __forceinline__ void append_if(float s, int64_t i, bool in, uint32_t 
 }
 
 // Every score of srow[lo, hi) that reaches thr, appended to buf; kU 16-byte
-// loads in flight per thread.
-template <int kU>
-__device__ void filter_slice(const float* srow, int64_t lo, int64_t hi, uint32_t thr, uint64_t* buf, uint32_t cap,
+// loads (kV scores each) in flight per thread.
+template <int kU, typename TS>
+__device__ void filter_slice(const TS* srow, int64_t lo, int64_t hi, uint32_t thr, uint64_t* buf, uint32_t cap,
                              uint32_t* cnt) {
+    constexpr int kV = 16 / (int)sizeof(TS);
     const int tid = threadIdx.x, lane = tid & 31;
     // scalar head up to the first 16-byte boundary, 16-byte body, scalar
     // tail; the head and tail loads are issued first and used last
-    int64_t lo_v = lo + (int64_t)((4u - (((uint32_t)((uintptr_t)(srow + lo)) >> 2) & 3u)) & 3u);
+    int64_t lo_v = lo + (int64_t)(((16u - ((uint32_t)(uintptr_t)(srow + lo) & 15u)) & 15u) / sizeof(TS));
     if (lo_v > hi) lo_v = hi;
-    const int64_t nvec = (hi - lo_v) >> 2;
-    const int64_t hi_v = lo_v + 4 * nvec;
+    const int64_t nvec = (hi - lo_v) / kV;
+    const int64_t hi_v = lo_v + kV * nvec;
     const int64_t ih = lo + tid, it = hi_v + tid;
     const bool inh = ih < lo_v, intl = it < hi;
-    const float sh = inh ? __ldcg(srow + ih) : 0.f;
-    const float stl = intl ? __ldcg(srow + it) : 0.f;
-    const float4* v4 = reinterpret_cast<const float4*>(srow + lo_v);
-    static_assert(4 * kU <= 64, "one mask bit per value");
+    const float sh = inh ? ld_score(srow + ih) : 0.f;
+    const float stl = intl ? ld_score(srow + it) : 0.f;
+    static_assert(kV * kU <= 64, "one mask bit per value");
     for (int64_t b0 = 0; b0 < nvec; b0 += kU * kThreads) {
-        float f[4 * kU];
+        float f[kV * kU];
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
             const int64_t j = b0 + u * kThreads + tid;
-            const float4 q = j < nvec ? __ldcg(v4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-            f[4 * u] = q.x;
-            f[4 * u + 1] = q.y;
-            f[4 * u + 2] = q.z;
-            f[4 * u + 3] = q.w;
+            if (j < nvec) {
+                ld_vec(srow + lo_v + kV * j, f + kV * u);
+            } else {
+#pragma unroll
+                for (int v = 0; v < kV; ++v) f[kV * u + v] = 0.f;
+            }
         }
         // this thread's takers, then one reservation per warp
         uint64_t mask = 0;
 #pragma unroll
-        for (int e = 0; e < 4 * kU; ++e) {
-            const int64_t j = b0 + (e >> 2) * kThreads + tid;
+        for (int e = 0; e < kV * kU; ++e) {
+            const int64_t j = b0 + (e / kV) * kThreads + tid;
             if (j < nvec && orderable(f[e]) >= thr) mask |= 1ull << e;
         }
         const uint32_t mine = __popcll(mask);
@@ -522,9 +549,9 @@ __device__ void filter_slice(const float* srow, int64_t lo, int64_t hi, uint32_t
         if (lane == 31) base = atomicAdd(cnt, total);
         uint32_t slot = __shfl_sync(0xffffffffu, base, 31) + incl - mine;
 #pragma unroll
-        for (int e = 0; e < 4 * kU; ++e) {
+        for (int e = 0; e < kV * kU; ++e) {
             if (mask & (1ull << e)) {
-                const int64_t i = lo_v + 4 * (b0 + (e >> 2) * kThreads + tid) + (e & 3);
+                const int64_t i = lo_v + kV * (b0 + (e / kV) * kThreads + tid) + (e % kV);
                 if (slot < cap) buf[slot] = composite(f[e], i);
                 ++slot;
             }
@@ -543,6 +570,7 @@ __device__ __forceinline__ void cluster_wait_acquire() {
 
 constexpr int kFilterLoads = 4;   // 16-byte filter loads in flight per thread
 
+template <typename TS>
 __global__ void __launch_bounds__(kThreads, 2) topk_kernel(RowSpec R, int k, int32_t* idx, float* top) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     uint64_t* cand = reinterpret_cast<uint64_t*>(smem_raw);
@@ -558,14 +586,14 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(RowSpec R, int k, int
     const int row = blockIdx.x / G;
     const int tid = threadIdx.x;
     const int64_t n = R.count(row);
-    const float* srow = R.scores + (int64_t)row * R.ld;
+    const TS* srow = reinterpret_cast<const TS*>(R.scores) + (int64_t)row * R.ld;
     int32_t* idx_row = idx + (int64_t)row * k;
     float* score_row = top ? top + (int64_t)row * k : nullptr;
     const int kk = (int)(n < k ? n : k);
 
     if (n <= kCap) {   // the same branch for every CTA of the cluster
         if (g != 0) return;
-        for (int64_t i = tid; i < n; i += kThreads) cand[i] = composite(srow[i], i);
+        for (int64_t i = tid; i < n; i += kThreads) cand[i] = composite(ld_score(srow + i), i);
         __syncthreads();
         select_exact(SmemSrc{cand}, n, k, idx_row, score_row, scratch, sh, bs);
         return;
@@ -613,7 +641,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(RowSpec R, int k, int
     if (c >= (uint32_t)kk && c <= (uint32_t)kCap)
         select_exact(SmemSrc{cand}, (int64_t)c, k, idx_row, score_row, scratch, sh, bs);
     else
-        select_exact(RowSrc{srow}, n, k, idx_row, score_row, scratch, sh, bs);   // the estimate missed
+        select_exact(RowSrc<TS>{srow}, n, k, idx_row, score_row, scratch, sh, bs);   // the estimate missed
 }
 
 // ---------------------------------------------------------------- host side
@@ -642,7 +670,7 @@ static cudaError_t topk_run(const RowSpec& R, int nq, int k, int32_t* idx, float
     if (R.ncols > kCap)
         while (G < kMaxCluster && (int64_t)nq * G * 2 <= sm_count()) G <<= 1;
     const bool spread = (int64_t)nq * G <= sm_count();
-    auto kern = topk_kernel;
+    auto kern = R.bf16 ? topk_kernel<bf16> : topk_kernel<float>;
     const size_t smem = spread ? kSmemSpread : kSmemBytes;
     cudaError_t e = smem_ceiling(kern);
     if (e != cudaSuccess) return e;
@@ -657,15 +685,22 @@ cudaError_t topk_select(const float* scores, int64_t ld, const int32_t* valid, i
                         int k, int32_t* idx, float* top_scores, void* ws, cudaStream_t st, const int32_t* seq,
                         int n_seq) {
     (void)ws;
-    RowSpec R{scores, ld, valid, valid_div, 0, 0, ncols, seq, n_seq};
+    RowSpec R{scores, 0, ld, valid, valid_div, 0, 0, ncols, seq, n_seq};
     return topk_run(R, nq, k, idx, top_scores, st);
 }
 
 cudaError_t topk_select_positions(const float* scores, int64_t ld, int64_t pos_base, int m, int nq, int64_t ncols,
                                   int k, int32_t* idx, void* ws, cudaStream_t st) {
     (void)ws;
-    RowSpec R{scores, ld, nullptr, m, pos_base, 1, ncols, nullptr, 0};
+    RowSpec R{scores, 0, ld, nullptr, m, pos_base, 1, ncols, nullptr, 0};
     return topk_run(R, nq, k, idx, nullptr, st);
+}
+
+cudaError_t topk_select_bf16(const void* scores, int64_t ld, const int32_t* valid, int valid_div, int nq,
+                             int64_t ncols, int k, int32_t* idx, float* top_scores, cudaStream_t st,
+                             const int32_t* seq, int n_seq) {
+    RowSpec R{scores, 1, ld, valid, valid_div, 0, 0, ncols, seq, n_seq};
+    return topk_run(R, nq, k, idx, top_scores, st);
 }
 
 }  // namespace csa

@@ -89,6 +89,17 @@ int csa_trace_read(int max_kernels, char* names, double* total_ms, int* counts, 
  * CSA_OK when no kernel reported an error; resets the word when `reset`. */
 int csa_poll_status(void* stream, int reset);
 
+/* Failure-path test hooks (for the tests of the timeout path; leave off in
+ * production). csa_debug_set(wait_limit, flags): wait_limit > 0 bounds every
+ * device wait of the tensor-core indexer to that many polls (0 restores the
+ * built-in bound); flags CSA_DEBUG_SKIP_FIRST_TILE makes the indexer never
+ * load its first key tile, so the wait for it runs out: the kernel records
+ * CSA_ERR_TIMEOUT in the status word (csa_poll_status), stops every role,
+ * drains its copies, frees its tensor memory and returns. Process-wide;
+ * affects launches made after the call. */
+#define CSA_DEBUG_SKIP_FIRST_TILE 1u
+int csa_debug_set(uint32_t wait_limit, uint32_t flags);
+
 /* ------------------------------------------------------------------------
  * a1. Projection [Walk §2.3.1 "KV compression": the KV streams and their
  * compression weights are learnable linear maps of the hidden state H].
@@ -243,12 +254,59 @@ int csa_topk_from_scores(const float* scores, int64_t ld, const int32_t* valid, 
 int csa_topk_from_scores_noalloc(const float* scores, int64_t ld, const int32_t* valid, int valid_div, int nq,
                                  int64_t ncols, int k, int32_t* idx, float* top_scores, void* stream);
 
+/* a5 on bf16 scores [Notes §2.4]: as csa_topk_from_scores with scores
+ * [nq, ld] bf16 (row stride ld bf16 values); a bf16 score widens exactly to
+ * fp32, so the result is csa_topk_from_scores's on those values. No
+ * workspace. */
+int csa_topk_from_scores_bf16(const void* scores, int64_t ld, const int32_t* valid, int valid_div, int nq,
+                              int64_t ncols, int k, int32_t* idx, float* top_scores, void* stream);
+
 /* a4+a5: indexer then top-k over the visible entries of each query. */
 size_t csa_index_topk_workspace_size(int nq, int64_t Nmax, int k, int dtype);
 int csa_index_topk(const void* qI, const float* w, const void* K, const int32_t* pos,
                    const int32_t* seq_of_q, int nq, int n_seq, int HI, int cI, int64_t Nmax, int m, int k,
                    int32_t* idx, float* top_scores, void* ws, size_t ws_bytes, int dtype,
                    void* stream);
+
+/* ------------------------------------------------------------------------
+ * FP8 indexer [Notes §2.4: the indexer's query-key products run in low
+ * precision; Notes §1.3: FP8 storage; Walk §2.3.4]. q^I and the indexer keys
+ * are stored as e4m3 (OCP FP8: 4 exponent bits, 3 mantissa bits, largest
+ * magnitude 448, no infinity) with one fp32 scale per row.
+ *
+ * csa_quantize_e4m3: x [rows, cols] (dtype) -> out [rows, cols] e4m3 bytes
+ *   and scale [rows] fp32, s = max|row| / 448 (1 for an all-zero row);
+ *   out = the e4m3 value nearest x / s (ties to even, saturating at 448),
+ *   with s and x / s taken in fp64. With w [rows] fp32 given, w_out [rows]
+ *   = w * s: for q^I rows (one per query head) this folds the query scale into
+ *   the head weight, since ReLU(s x) = s ReLU(x) for s > 0.
+ *   cols % 8 == 0.
+ * csa_index_scores_fp8: as csa_index_scores on e4m3 operands, on tensor cores
+ *   (kind::f8f6f4, fp32 accumulation):
+ *     scores[t][s] = k_scale[seq_t][s] * sum_h wq[t][h] * ReLU(qI8[t][h] . K8[seq_t][s])
+ *   qI8 [nq, HI, cI] e4m3, wq [nq, HI] fp32 (w times the query-head scale, as
+ *   csa_quantize_e4m3 writes it), K8 [B, Nmax, cI] e4m3, k_scale [B, Nmax]
+ *   fp32; invisible columns -inf. cI % 128 == 0, cI <= 256.
+ * csa_decode_fp8: csa_decode with the FP8 indexer: qI [B, HI, cI] bf16 is
+ *   quantized per head row inside the call, the indexer reads idx_cache8
+ *   [B, Nmax, cI] e4m3 with idx_scale [B, Nmax] fp32 (the keys quantized once
+ *   when their entries were written, csa_quantize_e4m3), top-k over the
+ *   scores, sparse MQA over kv_cache [B, Nmax, c] bf16. flags: 0, or
+ *   CSA_SCORES_BF16 to store the index scores as bf16 (nearest, ties to even)
+ *   and select on those [Notes §2.4: BF16 index scores halve the selector's
+ *   reads]; ties among rounded scores go to the lower entry index.
+ * ------------------------------------------------------------------------ */
+#define CSA_SCORES_BF16 1
+int csa_quantize_e4m3(const void* x, int64_t rows, int cols, void* out, float* scale, const float* w, float* w_out,
+                      int dtype, void* stream);
+int csa_index_scores_fp8(const void* qI8, const float* wq, const void* K8, const float* k_scale, const int32_t* pos,
+                         const int32_t* seq_of_q, int nq, int n_seq, int HI, int cI, int64_t Nmax, int m,
+                         float* scores, void* stream);
+size_t csa_decode_fp8_workspace_size(int B, int64_t Nmax, int H, int c, int HI, int cI, int k);
+int csa_decode_fp8(const void* qI, const float* w, const void* idx_cache8, const float* idx_scale, const void* q,
+                   const void* kv_cache, const int32_t* ctx_len, int B, int64_t Nmax, int m, int H, int c, int HI,
+                   int cI, int k, float scale, const float* sink, int flags, void* out, float* lse, int32_t* topk_idx,
+                   void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * a6. Sparse shared-KV MQA [Notes §1.1 last paragraph: every compressed
@@ -307,7 +365,10 @@ int hca_decode(const void* q, const void* kv_cache, const int32_t* ctx_len, int 
  * first block. With both state rings ([2m, 4c] and [2m, 4cI] fp32, as
  * csa_compress_chunk) start and n are free: the blocks that end inside the
  * chunk are written (earlier window tokens from the rings), the rings then
- * hold the chunk's last 2m projected rows, and x_left is not read. Steps:
+ * hold the chunk's last 2m projected rows, and x_left is not read. With
+ * W_kv = W_idx = NULL the chunk's entries are already in the caches
+ * (compressed elsewhere, e.g. gathered from other ranks): steps 1-2 are
+ * skipped and x, x_left, B_kv, B_idx are not read. Steps:
  *   1. compress the chunk's KV entries (a1+a2 with W_kv [4c, d], B_kv
  *      [2m, c]) into kv_cache rows start/m .. (start+n)/m - 1;
  *   2. the same for the indexer keys (W_idx [4cI, d], B_idx [2m, cI]) into

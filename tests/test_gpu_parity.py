@@ -407,3 +407,26 @@ def test_errors_surface_as_exceptions(csa):
         csa.csa_compress(x, torch.zeros(8, 8, device=DEV), 4)
     assert e.value.code == csa.CSA_ERR_INVALID_ARG
     csa.poll_status()
+
+
+def test_indexer_wait_timeout_is_reported_and_the_next_call_is_correct(csa):
+    # the failure path of the bounded device waits [failure detection without
+    # a fault]: the indexer is made to wait for a key tile that is never
+    # loaded, with a short wait bound; the kernel must return, the status word
+    # must say CSA_ERR_TIMEOUT, and the context must stay usable
+    nq, HI, cI, B, Nmax, m = 8, 64, 128, 8, 4000, 4
+    qI_h, qI, K_h, K, w_h, w, pos_h, pos = _index_inputs(torch.bfloat16, nq, HI, cI, B, Nmax, m, seed=13)
+    csa.poll_status()                                   # start from a clean word
+    csa.debug_set(4096, csa.CSA_DEBUG_SKIP_FIRST_TILE)
+    try:
+        csa.csa_index_scores(qI, w, K, pos, m)
+        torch.cuda.synchronize()                        # the kernel returned
+    finally:
+        csa.debug_set(0, 0)
+    with pytest.raises(csa.CsaError) as e:
+        csa.poll_status()
+    assert e.value.code == csa.CSA_ERR_TIMEOUT
+    csa.poll_status()                                   # the word was reset
+    got = csa.csa_index_scores(qI, w, K, pos, m)
+    ref = oracle.index_scores(qI_h, w_h, K_h, pos_h, m, seq=torch.arange(nq))
+    assert_scores_close(got, ref, score_bound(qI_h, w_h, K_h, pos_h, m, seq=torch.arange(nq)))
