@@ -5,8 +5,9 @@
 // every host thread. Setting it per call to the call's own size would let a
 // call on another thread lower it between this call's set and its launch,
 // and that launch would then fail. So each kernel's ceiling is raised once
-// per device to the device's opt-in maximum; a launch still asks for exactly
-// the shared memory it uses (the ceiling is only an upper bound).
+// per device to the device's opt-in maximum (less the kernel's static shared
+// memory); a launch still asks for exactly the shared memory it uses (the
+// ceiling is only an upper bound).
 #include <atomic>
 #include <mutex>
 #include <set>
@@ -27,7 +28,11 @@ cudaError_t smem_ceiling(const void* kern) {
     int optin = 0;
     e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+    // the kernel's static shared memory counts against the same per-block limit
+    cudaFuncAttributes fa{};
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin - (int)fa.sharedSizeBytes);
     if (e != cudaSuccess) return e;
     done.insert({kern, dev});
     return cudaSuccess;
