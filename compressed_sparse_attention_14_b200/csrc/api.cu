@@ -140,7 +140,7 @@ static cudaError_t run_indexer(const void* qI, const float* w, const void* K, Qu
     if (t == ElemType::BF16)
         return index_scores_tc(qI, w, K, qs, nq, n_seq, HI, cI, Nmax, m, scores, ld, group, fill_invisible,
                                device_status(), st);
-    return index_scores(qI, w, K, qs, nq, HI, cI, Nmax, m, scores, ld, t, st);
+    return index_scores(qI, w, K, qs, nq, n_seq, HI, cI, Nmax, m, scores, ld, t, st);
 }
 
 static int check_index_mode(int HI, int cI, ElemType t) {

@@ -18,7 +18,7 @@ constexpr int kIdxTile = 64;
 template <typename T>
 __global__ void __launch_bounds__(256) index_scores_ffma_kernel(
     const T* __restrict__ qI, const float* __restrict__ w, const T* __restrict__ K, QueryMap qm,
-    int HI, int cI, int64_t Nmax, int m, float* __restrict__ scores, int64_t ld) {
+    int n_seq, int HI, int cI, int64_t Nmax, int m, float* __restrict__ scores, int64_t ld) {
     extern __shared__ float smem[];
     const int kstride = cI + 1;
     float* q_s = smem;                       // [HI][cI]
@@ -30,14 +30,16 @@ __global__ void __launch_bounds__(256) index_scores_ffma_kernel(
     const int64_t s0 = (int64_t)blockIdx.x * kIdxTile;
     const int tid = threadIdx.x;
     if (s0 >= Nmax) return;
-    const int64_t vis = visible_entries(qm.pos_of(t), m, Nmax);
+    // a query whose sequence is outside [0, n_seq) sees no entry
+    const int seq = qm.seq_of(t);
+    const int64_t vis = (seq >= 0 && seq < n_seq) ? visible_entries(qm.pos_of(t), m, Nmax) : 0;
     float* srow = scores + (int64_t)t * ld;
     if (s0 >= vis) {
         for (int i = tid; i < kIdxTile; i += 256)
             if (s0 + i < Nmax) srow[s0 + i] = -INFINITY;
         return;
     }
-    const T* Kb = K + (int64_t)qm.seq_of(t) * Nmax * cI;
+    const T* Kb = K + (int64_t)seq * Nmax * cI;
     for (int i = tid * 8; i < HI * cI; i += 256 * 8) {
         float v[8];
         load8(qI + (int64_t)t * HI * cI + i, v);
@@ -81,7 +83,7 @@ __global__ void __launch_bounds__(256) index_scores_ffma_kernel(
     }
 }
 
-cudaError_t index_scores(const void* qI, const float* w, const void* K, QuerySpec qs, int nq,
+cudaError_t index_scores(const void* qI, const float* w, const void* K, QuerySpec qs, int nq, int n_seq,
                          int HI, int cI, int64_t Nmax, int m, float* scores, int64_t ld_scores,
                          ElemType t, cudaStream_t st) {
     if (nq == 0 || Nmax == 0) return cudaSuccess;
@@ -93,13 +95,13 @@ cudaError_t index_scores(const void* qI, const float* w, const void* K, QuerySpe
         auto kern = index_scores_ffma_kernel<bf16>;
         e = smem_ceiling(kern);
         if (e != cudaSuccess) return e;
-        CSA_LAUNCH(st, "index_scores_ffma", kern<<<grid, 256, smem, st>>>((const bf16*)qI, w, (const bf16*)K, qm, HI, cI, Nmax, m,
+        CSA_LAUNCH(st, "index_scores_ffma", kern<<<grid, 256, smem, st>>>((const bf16*)qI, w, (const bf16*)K, qm, n_seq, HI, cI, Nmax, m,
                                       scores, ld_scores));
     } else {
         auto kern = index_scores_ffma_kernel<float>;
         e = smem_ceiling(kern);
         if (e != cudaSuccess) return e;
-        CSA_LAUNCH(st, "index_scores_ffma", kern<<<grid, 256, smem, st>>>((const float*)qI, w, (const float*)K, qm, HI, cI, Nmax, m,
+        CSA_LAUNCH(st, "index_scores_ffma", kern<<<grid, 256, smem, st>>>((const float*)qI, w, (const float*)K, qm, n_seq, HI, cI, Nmax, m,
                                       scores, ld_scores));
     }
     return cudaGetLastError();

@@ -183,6 +183,59 @@ __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
     return d;
 }
 
+// The head reduction of one key's accumulator row: sc[q] += sum over the
+// heads h of query q of w[q][h] * max(x[q][h], 0), 64 columns per round (four
+// TMEM loads in flight, one wait), four independent partial sums per 16
+// columns in paired fp32 FMAs (each lane rounds as a separate fmaf would).
+// kN > 0: the row has kN columns and each query kHI heads, known at compile
+// time (the loop unrolls and each 16-column block's query is a constant);
+// kN == 0: npad and HI at run time.
+template <int kN, int kHI>
+__device__ __forceinline__ void head_reduce(uint32_t taddr, const float* wv, int npad, int HI, int group,
+                                            float (&sc)[4]) {
+    const int n = kN > 0 ? kN : npad;
+#pragma unroll(kN > 0 ? 4 : 1)
+    for (int c0 = 0; c0 < n; c0 += 64) {
+        float v[64];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (kN > 0 || c0 + 16 * u < n) {
+                float* vv = v + 16 * u;
+                tc::tmem_ld16(taddr + c0 + 16 * u, *reinterpret_cast<float(*)[16]>(vv));
+            }
+        }
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int cc = c0 + 16 * u;
+            if (kN > 0 || cc < n) {
+                uint64_t p01 = 0, p23 = 0;
+#pragma unroll
+                for (int i = 0; i < 16; i += 4) {
+                    const float4 w4 = *reinterpret_cast<const float4*>(wv + cc + i);
+                    p01 = fma2(pack2(w4.x, w4.y),
+                               pack2(fmaxf(v[16 * u + i], 0.f), fmaxf(v[16 * u + i + 1], 0.f)), p01);
+                    p23 = fma2(pack2(w4.z, w4.w),
+                               pack2(fmaxf(v[16 * u + i + 2], 0.f), fmaxf(v[16 * u + i + 3], 0.f)), p23);
+                }
+                float p4[4];
+                unpack2(p01, p4[0], p4[1]);
+                unpack2(p23, p4[2], p4[3]);
+                const float part = (p4[0] + p4[1]) + (p4[2] + p4[3]);
+                if constexpr (kN > 0) {
+                    sc[cc / kHI] += part;
+                } else {
+                    const int gq = (group > 1) ? cc / HI : 0;
+                    if (gq == 0) sc[0] += part;
+                    else if (gq == 1) sc[1] += part;
+                    else if (gq == 2) sc[2] += part;
+                    else sc[3] += part;
+                }
+            }
+        }
+    }
+}
+
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                               int* status, uint32_t limit) {
     for (uint32_t i = 0; i < limit; ++i) {
@@ -196,7 +249,7 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 
 }  // namespace
 
-template <bool kFp8>
+template <bool kFp8, int kN, int kHI>
 __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __grid_constant__ IdxArgs a,
                                                                       const __grid_constant__ CUtensorMap tmK,
                                                                       const __grid_constant__ CUtensorMap tmQ) {
@@ -364,45 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
             tc::tc_fence_after();
             float sc[4] = {0.f, 0.f, 0.f, 0.f};
             const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * a.npad);
-            // 64 columns per round: four loads in flight, one wait; four
-            // independent partial sums per 16 columns
-            for (int c0 = 0; c0 < a.npad; c0 += 64) {
-                float v[64];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    if (c0 + 16 * u < a.npad) {
-                        float* vv = v + 16 * u;
-                        tc::tmem_ld16(taddr + c0 + 16 * u, *reinterpret_cast<float(*)[16]>(vv));
-                    }
-                }
-                tc::tmem_ld_wait();
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int cc = c0 + 16 * u;
-                    if (cc < a.npad) {
-                        // four independent partial sums, two per paired fp32
-                        // FMA (each lane rounds as a separate fmaf would)
-                        uint64_t p01 = 0, p23 = 0;
-#pragma unroll
-                        for (int i = 0; i < 16; i += 4) {
-                            const float4 w4 = *reinterpret_cast<const float4*>(wv + cc + i);
-                            p01 = fma2(pack2(w4.x, w4.y),
-                                       pack2(fmaxf(v[16 * u + i], 0.f), fmaxf(v[16 * u + i + 1], 0.f)), p01);
-                            p23 = fma2(pack2(w4.z, w4.w),
-                                       pack2(fmaxf(v[16 * u + i + 2], 0.f), fmaxf(v[16 * u + i + 3], 0.f)), p23);
-                        }
-                        float p4[4];
-                        unpack2(p01, p4[0], p4[1]);
-                        unpack2(p23, p4[2], p4[3]);
-                        const float part = (p4[0] + p4[1]) + (p4[2] + p4[3]);
-                        const int gq = (a.group > 1) ? cc / a.HI : 0;
-                        if (gq == 0) sc[0] += part;
-                        else if (gq == 1) sc[1] += part;
-                        else if (gq == 2) sc[2] += part;
-                        else sc[3] += part;
-                    }
-                }
-            }
+            head_reduce<kN, kHI>(taddr, wv, a.npad, a.HI, a.group, sc);
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&sm.tempty[buf]);
@@ -524,7 +539,13 @@ cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, Query
         if (e == cudaSuccess) e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    auto kern = fp8 ? index_scores_tc_kernel<true> : index_scores_tc_kernel<false>;
+    // the two shapes of the workloads get a fully unrolled epilogue: decode
+    // (one query of 64 heads per MMA) and grouped prefill (4 queries of 64)
+    auto kern = fp8 ? index_scores_tc_kernel<true, 0, 0> : index_scores_tc_kernel<false, 0, 0>;
+    if (a.npad == 64 && HI == 64 && group == 1)
+        kern = fp8 ? index_scores_tc_kernel<true, 64, 64> : index_scores_tc_kernel<false, 64, 64>;
+    else if (a.npad == 256 && HI == 64 && group == 4)
+        kern = fp8 ? index_scores_tc_kernel<true, 256, 64> : index_scores_tc_kernel<false, 256, 64>;
     e = smem_ceiling(kern);
     if (e != cudaSuccess) return e;
     CSA_LAUNCH(st, fp8 ? "index_scores_tc_fp8" : "index_scores_tc",

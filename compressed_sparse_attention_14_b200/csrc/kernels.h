@@ -110,8 +110,9 @@ cudaError_t project_tc(const void* x, const void* W, int64_t n, int d, int M, fl
                        cudaStream_t st);
 
 // indexer.cu (FFMA, fp32 mode): scores[t, 0..Nmax) with ld = ld_scores;
-// -inf past the visible range
-cudaError_t index_scores(const void* qI, const float* w, const void* K, QuerySpec qs, int nq,
+// -inf past the visible range (the whole row for a query whose sequence is
+// outside [0, n_seq))
+cudaError_t index_scores(const void* qI, const float* w, const void* K, QuerySpec qs, int nq, int n_seq,
                          int HI, int cI, int64_t Nmax, int m, float* scores, int64_t ld_scores,
                          ElemType t, cudaStream_t st);
 // indexer_tc.cu (tcgen05, bf16): groups of `group` consecutive queries share

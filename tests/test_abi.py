@@ -93,6 +93,16 @@ def test_invalid_arguments_are_rejected_on_the_host():
     rc = L.csa_prefill(fake, None, fake, fake, fake, fake, 4, 8, 64, 4, 128, 64, fake, fake, 16, None, None, fake, fake, fake,
                        8, 4, 4, 0.0, None, fake, None, None, None, 0, csa.CSA_BF16, None)
     assert rc == csa.CSA_ERR_INVALID_ARG
+    # FP8 indexer: cI must fill whole 128-byte rows; w and w_out go together
+    assert L.csa_index_scores_fp8(fake, fake, fake, fake, fake, None, 2, 2, 4, 64, 16, 4, fake,
+                                  None) == csa.CSA_ERR_UNSUPPORTED
+    assert L.csa_quantize_e4m3(fake, 4, 12, fake, fake, None, None, csa.CSA_BF16, None) == csa.CSA_ERR_INVALID_ARG
+    assert L.csa_quantize_e4m3(fake, 4, 16, fake, fake, fake, None, csa.CSA_BF16, None) == csa.CSA_ERR_INVALID_ARG
+    assert L.csa_decode_fp8(fake, fake, fake, fake, fake, fake, fake, 2, 1024, 4, 8, 128, 4, 128, 16, 0.0, None, 2,
+                            fake, None, None, fake * 16, 1 << 30, None) == csa.CSA_ERR_INVALID_ARG
+    assert b"flags" in L.csa_last_error()
+    assert L.csa_topk_from_scores_bf16(fake, 16, None, 1, 1, 16, 0, fake, None, None) == csa.CSA_ERR_UNSUPPORTED
+    assert L.csa_debug_set(0, 2) == csa.CSA_ERR_INVALID_ARG
     # prefill with one state ring but not the other
     rc = L.csa_prefill(fake, None, fake, fake, fake, fake, 6, 9, 64, 4, 128, 64, fake, fake, 16, fake, None, fake,
                        fake, fake, 8, 4, 4, 0.0, None, fake, None, None, None, 0, csa.CSA_BF16, None)
