@@ -57,9 +57,9 @@ _SIGS = {
     "csa_index_scores": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I64, _I, _P, _I, _P]),
     "csa_topk_workspace_size": (_SZ, [_I, _I64, _I]),
     "csa_topk_from_scores": (_I, [_P, _I64, _P, _I, _I, _I64, _I, _P, _P, _P, _SZ, _P]),
-    "csa_topk_from_scores_noalloc": (_I, [_P, _I64, _P, _I, _I, _I64, _I, _P, _P, _P]),
     "csa_index_topk_workspace_size": (_SZ, [_I, _I64, _I, _I]),
     "csa_index_topk": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I64, _I, _I, _P, _P, _P, _SZ, _I, _P]),
+    "csa_index_topk_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I64, _I, _I, _P, _P, _I, _P]),
     "csa_quantize_e4m3": (_I, [_P, _I64, _I, _P, _P, _P, _P, _I, _P]),
     "csa_index_scores_fp8": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I64, _I, _P, _P]),
     "csa_decode_fp8_workspace_size": (_SZ, [_I, _I64, _I, _I, _I, _I, _I]),
@@ -361,19 +361,6 @@ def csa_topk_from_scores(scores, k: int, valid=None, valid_div: int = 1, ws=None
     return idx, top
 
 
-def csa_topk_from_scores_noalloc(scores, k: int, valid=None, valid_div: int = 1, idx=None, top_scores=None):
-    """csa_topk_from_scores without a workspace (for callers that cannot
-    allocate device memory when they select): the selection keeps its
-    scratch in on-chip shared memory. Pass preallocated idx / top_scores to
-    make the call itself allocation-free."""
-    nq, ncols = scores.shape
-    if idx is None:
-        idx = torch.empty((nq, k), dtype=torch.int32, device=scores.device)
-    _check(_lib.csa_topk_from_scores_noalloc(_ptr(scores), ncols, _ptr(valid), valid_div, nq, ncols, k, _ptr(idx),
-                                             _ptr(top_scores), _stream()))
-    return idx, top_scores
-
-
 def csa_topk_from_scores_bf16(scores, k: int, valid=None, valid_div: int = 1):
     """Top-k over bf16 scores [nq, ncols] (same rule as csa_topk_from_scores)."""
     nq, ncols = scores.shape
@@ -399,6 +386,36 @@ def csa_index_topk(qI, w, K, pos, m: int, k: int, seq_of_q=None, ws=None):
                                Nmax, m, k,
                                _ptr(idx), _ptr(top), _ptr(ws), _nbytes(ws), mode, _stream()))
     return idx, top
+
+
+def csa_index_topk_noalloc(qI, w, K, pos, m: int, k: int, seq_of_q=None, idx=None, top_scores=None):
+    """csa_index_topk without a workspace, for callers that cannot allocate
+    device memory when they select: the score block between the indexer and
+    the selection lives in a fixed 16 MiB array inside the library
+    (nq * Nmax <= CSA_NOALLOC_MAX_SCORES). Pass preallocated idx [nq, k]
+    int32 and top_scores [nq, k] fp32 (or None) to make the call itself
+    allocation-free. Calls that overlap on the GPU share that array and race."""
+    nq, HI, cI = qI.shape
+    K = _kv3(K)
+    n_seq, Nmax = K.shape[0], K.shape[1]
+    mode = _mode(qI)
+    _dtype(K, qI.dtype, "K")
+    _shape(K, (n_seq, Nmax, cI), "K")
+    _dtype(w, torch.float32, "w")
+    _shape(w, (nq, HI), "w")
+    _dtype(pos, torch.int32, "pos")
+    _shape(pos, (nq,), "pos")
+    _dtype(seq_of_q, torch.int32, "seq_of_q")
+    _shape(seq_of_q, (nq,), "seq_of_q")
+    if idx is None:
+        idx = torch.empty((nq, k), dtype=torch.int32, device=qI.device)
+    _dtype(idx, torch.int32, "idx")
+    _shape(idx, (nq, k), "idx")
+    _dtype(top_scores, torch.float32, "top_scores")
+    _shape(top_scores, (nq, k), "top_scores")
+    _check(_lib.csa_index_topk_noalloc(_ptr(qI), _ptr(w), _ptr(K), _ptr(pos), _ptr(seq_of_q), nq, n_seq, HI, cI,
+                                       Nmax, m, k, _ptr(idx), _ptr(top_scores), mode, _stream()))
+    return idx, top_scores
 
 
 # ---------------------------------------------------------------- FP8 indexer

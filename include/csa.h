@@ -242,18 +242,6 @@ int csa_topk_from_scores(const float* scores, int64_t ld, const int32_t* valid, 
                          int nq, int64_t ncols, int k, int32_t* idx, float* top_scores, void* ws,
                          size_t ws_bytes, void* stream);
 
-/* a5 without a workspace, for callers that cannot allocate device memory at
- * the point of the call (a plug-in whose host framework owns every device
- * allocation and gives it no workspace, a serving loop that forbids
- * allocation after start-up). The pages have no counterpart: this is a
- * library convenience. Same arguments and exactly the same result as
- * csa_topk_from_scores, minus ws/ws_bytes; nq <= 65535. The selection keeps
- * all of its scratch in on-chip shared memory: no cudaMalloc, cudaFree or
- * other allocating call is made, no device memory is held between calls, and
- * calls on different streams share no state. */
-int csa_topk_from_scores_noalloc(const float* scores, int64_t ld, const int32_t* valid, int valid_div, int nq,
-                                 int64_t ncols, int k, int32_t* idx, float* top_scores, void* stream);
-
 /* a5 on bf16 scores [Notes §2.4]: as csa_topk_from_scores with scores
  * [nq, ld] bf16 (row stride ld bf16 values); a bf16 score widens exactly to
  * fp32, so the result is csa_topk_from_scores's on those values. No
@@ -267,6 +255,31 @@ int csa_index_topk(const void* qI, const float* w, const void* K, const int32_t*
                    const int32_t* seq_of_q, int nq, int n_seq, int HI, int cI, int64_t Nmax, int m, int k,
                    int32_t* idx, float* top_scores, void* ws, size_t ws_bytes, int dtype,
                    void* stream);
+
+/* a4+a5 without a workspace, for callers that cannot allocate device memory
+ * at the point of the call: a plug-in whose host framework owns every device
+ * allocation and gives it no scratch, a serving loop whose memory footprint
+ * is fixed after start-up, a latency-critical path that cannot afford
+ * cudaMalloc (which may synchronise the device). The pages have no
+ * counterpart: this is a library convenience. Same arguments and exactly the
+ * same result as csa_index_topk, minus ws/ws_bytes.
+ *
+ * The score block between the indexer and the selection lives in a fixed
+ * array of device memory inside the library, CSA_NOALLOC_MAX_SCORES fp32
+ * scores (16 MiB), held by every GPU that loads the library until the
+ * process exits. nq * Nmax above CSA_NOALLOC_MAX_SCORES returns
+ * CSA_ERR_UNSUPPORTED (use csa_index_topk). The call makes no cudaMalloc,
+ * cudaFree or other allocating call.
+ *  - The first call on a device (with that device current) looks up the
+ *    array's device address; make it before any stream capture.
+ *  - All calls on a device share the array, which keeps the last call's
+ *    scores; nothing in it must start at zero (each call writes every score
+ *    it reads). Calls that overlap on the GPU (other streams, other host
+ *    threads) race on it: serialise them. */
+#define CSA_NOALLOC_MAX_SCORES (4 * 1024 * 1024)
+int csa_index_topk_noalloc(const void* qI, const float* w, const void* K, const int32_t* pos,
+                           const int32_t* seq_of_q, int nq, int n_seq, int HI, int cI, int64_t Nmax, int m, int k,
+                           int32_t* idx, float* top_scores, int dtype, void* stream);
 
 /* ------------------------------------------------------------------------
  * FP8 indexer [Notes §2.4: the indexer's query-key products run in low

@@ -71,8 +71,15 @@ def test_invalid_arguments_are_rejected_on_the_host():
                               None) == csa.CSA_ERR_UNSUPPORTED
     # more rows than one launch grid holds
     assert L.csa_topk_from_scores(fake, 16, None, 1, 70000, 16, 4, fake, None, None, 0, None) == csa.CSA_ERR_UNSUPPORTED
-    assert L.csa_topk_from_scores_noalloc(fake, 16, None, 1, 70000, 16, 4, fake, None, None) == csa.CSA_ERR_UNSUPPORTED
     assert b"65535" in L.csa_last_error()
+    # the allocation-free indexer + top-k: more scores than its fixed array
+    assert L.csa_index_topk_noalloc(fake, fake, fake, fake, None, 64, 64, 64, 128, 65537, 4, 16, fake, None,
+                                    csa.CSA_BF16, None) == csa.CSA_ERR_UNSUPPORTED
+    assert b"fixed" in L.csa_last_error()
+    assert L.csa_index_topk_noalloc(fake, fake, fake, fake, None, 70000, 70000, 64, 128, 8, 4, 16, fake, None,
+                                    csa.CSA_BF16, None) == csa.CSA_ERR_UNSUPPORTED
+    assert L.csa_index_topk_noalloc(fake, fake, fake, fake + 4, None, 4, 4, 64, 128, 8, 4, 16, fake, None,
+                                    csa.CSA_BF16, None) == csa.CSA_ERR_INVALID_ARG
     # missing / short workspace
     need = L.csa_decode_workspace_size(2, 1024, 8, 128, 4, 64, 16, csa.CSA_BF16)
     assert need > 0
