@@ -18,8 +18,13 @@
 // read on the device). Warp roles:
 //   warp 0     TMA producer: the group's Q rows once per group, then the key
 //              tiles through a ring of `stages` shared-memory buffers;
-//   warp 1     allocates TMEM; one lane issues the MMAs of each tile into one
-//              of 2-4 accumulator buffers and commits their completion;
+//   warps 1,10 one lane of each issues the MMAs of alternate tiles into one
+//              of 2-4 accumulator buffers and commits their completion
+//              (warp 1 also allocates TMEM). A single issuing thread was the
+//              bottleneck: each tcgen05.mma costs its thread ~70 ns to issue,
+//              so one thread issuing 8 per 32 KB key tile capped the stream
+//              near 4 TB/s; two threads issuing alternate tiles bring it to
+//              the memory rate;
 //   warps 2-9  epilogue, two sets of four warps taking alternate tiles:
 //              tcgen05.ld of the accumulator, ReLU/weight/head reduction,
 //              coalesced fp32 score stores.
@@ -42,7 +47,10 @@ namespace csa {
 
 namespace {
 
-constexpr int kThreads = 320;   // producer, MMA, two epilogue sets of 4 warps
+// warp 0 producer, warp 1 MMA issuer 0 (and TMEM owner), warps 2-9 two
+// epilogue sets of 4, warp 10 MMA issuer 1
+constexpr int kThreads = 352;
+constexpr int kIssuers = 2;
 constexpr int kKeys = 128;
 constexpr uint32_t kWaitLimit = 1u << 24;
 
@@ -266,8 +274,8 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
         for (int i = 0; i < a.stages; ++i) { tc::mbar_init(&sm.full[i], 1); tc::mbar_init(&sm.empty[i], 1); }
         for (int i = 0; i < 4; ++i) { tc::mbar_init(&sm.tfull[i], 1); tc::mbar_init(&sm.tempty[i], 4); }
         tc::mbar_init(sm.qfull, 1);
-        tc::mbar_init(sm.qempty, 1);
-        tc::mbar_init(sm.fin, 1);
+        tc::mbar_init(sm.qempty, kIssuers);   // every issuer releases each group's q
+        tc::mbar_init(sm.fin, kIssuers);
         tc::fence_mbar_init();
         s_abort = 0;
     }
@@ -331,8 +339,11 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
                 if (!(a.skip_first_tile && j == 0)) tc::mbar_wait(&sm.full[j % a.stages], (j / a.stages) & 1, kWaitLimit);
             if (switches > 0) tc::mbar_wait(sm.qfull, (switches - 1) & 1, kWaitLimit);
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == 1 || warp == 10) {
+        // ------------------------------------------------------------ MMA issuers
+        // issuer mi takes the tiles with it % kIssuers == mi; both walk the
+        // whole list, wait for each group's q and release it at the group's end
+        const int mi = warp == 10 ? 1 : 0;
         if (lane == 0 && my > 0) {
             Walk wk;
             wk.start(a, g0, t0);
@@ -352,6 +363,11 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
                     if (!wait_or_abort(sm.qfull, switches & 1, abort_flag, a.status, a.wait_limit)) break;
                     cur = wk.g;
                     ++switches;
+                }
+                if ((int)(it % kIssuers) != mi) {
+                    if (wk.last_of_group() || it + 1 == my) tc::umma_commit(sm.qempty);
+                    wk.next(a, ngroups);
+                    continue;
                 }
                 const int s = (int)(it % a.stages);
                 const int buf = (int)(it % a.nbuf);
