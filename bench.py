@@ -230,12 +230,11 @@ class Timer:
 # ----------------------------------------------------------------------------
 
 def decode_workload(shape, rank, batch=None, fp8=False):
-    """One csa_decode step over the batch. fp8: the pages' low-precision
-    indexer path (csa_decode_fp8 with bf16 index scores): the indexer keys are
-    held as e4m3 codes with one fp32 scale per key (quantized once when the
-    cache is built, outside the timed region, as the compressor would store
-    them), q^I is quantized in the call, the scores are stored as bf16 and the
-    top-k selects on those."""
+    """One csa_decode step over the batch. fp8: the FP8 indexer
+    (csa_decode_fp8): the indexer keys are held as e4m3 codes with one fp32
+    scale per key (quantized once when the cache is built, outside the timed
+    region, as the compressor would store them), q^I is quantized in the call;
+    fp32 index scores (bf16 scores tie more often and made this top-k slower)."""
     import dataclasses
     import compressed_sparse_attention_14_b200 as csa
     s = shape if batch is None else dataclasses.replace(shape, batch=batch)
@@ -252,8 +251,7 @@ def decode_workload(shape, rank, batch=None, fp8=False):
                          dtype=torch.uint8, device="cuda")
 
         def call(qI, w, q, ctx, o=out):
-            csa.csa_decode_fp8(qI, w, k8, ks, q, inp["kv_cache"], ctx, s.m, s.k, out=o, lse=lse, ws=ws,
-                               bf16_scores=True)
+            csa.csa_decode_fp8(qI, w, k8, ks, q, inp["kv_cache"], ctx, s.m, s.k, out=o, lse=lse, ws=ws)
     else:
         ws = torch.empty(csa.csa_decode_workspace_size(B, s.n_max, s.heads, s.c, s.idx_heads, s.idx_dim, s.k, mode),
                          dtype=torch.uint8, device="cuda")
@@ -274,7 +272,7 @@ def decode_workload(shape, rank, batch=None, fp8=False):
     step_bytes = idx_bytes + B * (s.k * s.c * 2 + 2 * s.heads * s.c * 2)
     # the indexer kernel also writes one score per visible entry (fp32, or
     # bf16 on the low-precision path)
-    score_bytes = 2 if fp8 else 4
+    score_bytes = 4
     idx_kernel_bytes = idx_bytes + v_sum * score_bytes
 
     pinned = {k: inp[k].cpu().pin_memory() for k in ("q", "qI", "w", "ctx_len")}
@@ -307,7 +305,7 @@ def decode_workload(shape, rank, batch=None, fp8=False):
                             entries_max=s.n_max, head_dim=s.c, heads=s.heads, index_heads=s.idx_heads,
                             index_dim=s.idx_dim, topk=s.k, visible_entries_total=int(v_sum),
                             index_keys="e4m3 + fp32 scale per key" if fp8 else "bf16",
-                            index_scores="bf16" if fp8 else "fp32",
+                            index_scores="fp32",
                             l2="flushed before every timed step (256 MiB write + 256 MiB read)"),
                 inputs=inp)
 

@@ -51,7 +51,7 @@ namespace {
 // epilogue sets of 4, warp 10 MMA issuer 1
 constexpr int kThreads = 352;
 constexpr int kIssuers = 2;
-constexpr int kKeys = 128;
+constexpr int kKeys = 128;      // keys per MMA (M) and per TMA box
 constexpr uint32_t kWaitLimit = 1u << 24;
 
 struct IdxArgs {
@@ -75,6 +75,8 @@ struct IdxArgs {
     uint32_t wait_limit;    // polls before a wait gives up (CSA_ERR_TIMEOUT)
     int skip_first_tile;    // failure-path test hook: the first key tile is never loaded
     int nbuf;           // TMEM accumulator buffers (2..4)
+    int kpt;            // keys per tile: kKeys, or 2 * kKeys (FP8 decode: a
+                        // 32 KB stage, so per-tile costs spread over 256 keys)
 };
 
 struct Smem {
@@ -115,7 +117,7 @@ __device__ __forceinline__ int64_t group_visible(const IdxArgs& a, int g) {
     return visible_entries(a.qm.pos_of(g * a.group), a.m, a.Nmax);
 }
 __device__ __forceinline__ int64_t group_tiles(const IdxArgs& a, int g) {
-    return (group_visible(a, g) + kKeys - 1) / kKeys;
+    return (group_visible(a, g) + a.kpt - 1) / a.kpt;
 }
 
 // Warp-cooperative: total tiles, and the (group, tile) at flat index `target`.
@@ -257,7 +259,7 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 
 }  // namespace
 
-template <bool kFp8, int kN, int kHI>
+template <bool kFp8, int kN, int kHI, int kH>
 __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __grid_constant__ IdxArgs a,
                                                                       const __grid_constant__ CUtensorMap tmK,
                                                                       const __grid_constant__ CUtensorMap tmQ) {
@@ -327,10 +329,15 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
                     break;
                 if (!(a.skip_first_tile && it == 0)) {
                     tc::mbar_expect_tx(&sm.full[s], a.stage_bytes);
-                    const int row = (int)((int64_t)group_seq(a, wk.g) * a.Nmax + wk.t * kKeys);
+                    const int row = (int)((int64_t)group_seq(a, wk.g) * a.Nmax + wk.t * a.kpt);
                     uint8_t* dst = sm.stage0 + (size_t)s * a.stage_bytes;
-                    for (int kb = 0; kb < a.kblocks; ++kb)
-                        tc::tma_load_2d(dst + (size_t)kb * kKeys * 128, &tmK, &sm.full[s], kb * a.blk_elems, row);
+                    // the stage holds kH halves of 128 keys, each kblocks
+                    // 128-byte column blocks of 128 rows
+#pragma unroll
+                    for (int hh = 0; hh < kH; ++hh)
+                        for (int kb = 0; kb < a.kblocks; ++kb)
+                            tc::tma_load_2d(dst + (size_t)(hh * a.kblocks + kb) * kKeys * 128, &tmK, &sm.full[s],
+                                            kb * a.blk_elems, row + hh * kKeys);
                 }
                 wk.next(a, ngroups);
             }
@@ -376,14 +383,18 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
                 if (use >= 1 && !wait_or_abort(&sm.tempty[buf], (use - 1) & 1, abort_flag, a.status, a.wait_limit)) break;
                 tc::tc_fence_after();
                 const uint64_t a_s = a_desc0 + (uint64_t)(s * stage_step);
-                const uint32_t d = tmem + (uint32_t)(buf * a.npad);
-                for (int kb = 0; kb < a.kblocks; ++kb) {
-                    const uint64_t ad = a_s + (uint64_t)(kb * a_kb_step);
-                    const uint64_t bd = b_desc0 + (uint64_t)(kb * b_kb_step);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {   // 32 bytes = 2 units per K step
-                        if constexpr (kFp8) tc::umma_f8(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) ? 1u : 0u);
-                        else tc::umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) ? 1u : 0u);
+                for (int hh = 0; hh < kH; ++hh) {
+                    // half hh: keys hh*128 .. +127 into accumulator columns hh*npad
+                    const uint32_t d = tmem + (uint32_t)((buf * kH + hh) * a.npad);
+                    for (int kb = 0; kb < a.kblocks; ++kb) {
+                        const uint64_t ad = a_s + (uint64_t)((hh * a.kblocks + kb) * a_kb_step);
+                        const uint64_t bd = b_desc0 + (uint64_t)(kb * b_kb_step);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {   // 32 bytes = 2 units per K step
+                            if constexpr (kFp8) tc::umma_f8(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) ? 1u : 0u);
+                            else tc::umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) ? 1u : 0u);
+                        }
                     }
                 }
                 tc::umma_commit(&sm.empty[s]);
@@ -424,29 +435,42 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
                 vis = group_visible(a, wk.g);
             }
             const int buf = (int)(it % a.nbuf);
-            const int64_t key = wk.t * kKeys + row;
-            // FP8: the key's scale, loaded before the wait so its latency hides
-            float kscale = 1.f;
-            if constexpr (kFp8)
-                if (key < vis) kscale = __ldg(a.kscale + (int64_t)group_seq(a, wk.g) * a.Nmax + key);
+            // this thread's keys: row of each 128-key half of the tile
+            int64_t key[kH];
+            float kscale[kH];
+#pragma unroll
+            for (int hh = 0; hh < kH; ++hh) {
+                key[hh] = wk.t * a.kpt + hh * kKeys + row;
+                // FP8: the key's scale, loaded before the wait so its latency hides
+                kscale[hh] = 1.f;
+                if constexpr (kFp8)
+                    if (key[hh] < vis) kscale[hh] = __ldg(a.kscale + (int64_t)group_seq(a, wk.g) * a.Nmax + key[hh]);
+            }
             if (!wait_or_abort(&sm.tfull[buf], (uint32_t)((it / a.nbuf) & 1), abort_flag, a.status, a.wait_limit)) break;
             tc::tc_fence_after();
-            float sc[4] = {0.f, 0.f, 0.f, 0.f};
-            const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * a.npad);
-            head_reduce<kN, kHI>(taddr, wv, a.npad, a.HI, a.group, sc);
+            float sc[kH][4];
+#pragma unroll
+            for (int hh = 0; hh < kH; ++hh) {
+                sc[hh][0] = sc[hh][1] = sc[hh][2] = sc[hh][3] = 0.f;
+                const uint32_t taddr =
+                    tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)((buf * kH + hh) * a.npad);
+                head_reduce<kN, kHI>(taddr, wv, a.npad, a.HI, a.group, sc[hh]);
+            }
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&sm.tempty[buf]);
-            if (key < vis) {
+#pragma unroll
+            for (int hh = 0; hh < kH; ++hh) {
+                if (key[hh] >= vis) continue;
 #pragma unroll
                 for (int gq = 0; gq < 4; ++gq) {
                     const int tq = wk.g * a.group + gq;
                     if (gq < a.group && tq < a.nq) {
-                        const float v = kFp8 ? sc[gq] * kscale : sc[gq];
+                        const float v = kFp8 ? sc[hh][gq] * kscale[hh] : sc[hh][gq];
                         if (a.score_bf16)
-                            reinterpret_cast<bf16*>(a.scores)[(int64_t)tq * a.ld + key] = __float2bfloat16_rn(v);
+                            reinterpret_cast<bf16*>(a.scores)[(int64_t)tq * a.ld + key[hh]] = __float2bfloat16_rn(v);
                         else
-                            a.scores[(int64_t)tq * a.ld + key] = v;
+                            a.scores[(int64_t)tq * a.ld + key[hh]] = v;
                     }
                 }
             }
@@ -520,14 +544,17 @@ cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, Query
     a.skip_first_tile = (debug_flags() & CSA_DEBUG_SKIP_FIRST_TILE) ? 1 : 0;
     a.ld = ld;
     a.status = status;
-    a.stage_bytes = (uint32_t)(kKeys * cI * es);
+    // FP8 decode (one query of at most 128 heads per MMA): tiles of 256 keys
+    const int kh = (fp8 && group == 1 && n <= 128) ? 2 : 1;
+    a.kpt = kh * kKeys;
+    a.stage_bytes = (uint32_t)(a.kpt * cI * es);
     a.q_bytes = (uint32_t)(a.npad * cI * es);
     // as many accumulator buffers (2..4) as fit 512 TMEM columns
-    a.nbuf = 512 / a.npad;
+    a.nbuf = 512 / (kh * a.npad);
     if (a.nbuf > 4) a.nbuf = 4;
     if (a.nbuf < 2) a.nbuf = 2;
     uint32_t cols = 32;
-    while (cols < (uint32_t)(a.nbuf * a.npad)) cols <<= 1;
+    while (cols < (uint32_t)(a.nbuf * kh * a.npad)) cols <<= 1;
     a.tmem_cols = cols;
     const size_t fixed = 1024 + a.q_bytes + 8 * 256 * sizeof(float) + 64 * sizeof(uint64_t);
     const size_t budget = 226 * 1024;
@@ -557,11 +584,12 @@ cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, Query
     }
     // the two shapes of the workloads get a fully unrolled epilogue: decode
     // (one query of 64 heads per MMA) and grouped prefill (4 queries of 64)
-    auto kern = fp8 ? index_scores_tc_kernel<true, 0, 0> : index_scores_tc_kernel<false, 0, 0>;
+    auto kern = fp8 ? (kh == 2 ? index_scores_tc_kernel<true, 0, 0, 2> : index_scores_tc_kernel<true, 0, 0, 1>)
+                    : index_scores_tc_kernel<false, 0, 0, 1>;
     if (a.npad == 64 && HI == 64 && group == 1)
-        kern = fp8 ? index_scores_tc_kernel<true, 64, 64> : index_scores_tc_kernel<false, 64, 64>;
+        kern = fp8 ? index_scores_tc_kernel<true, 64, 64, 2> : index_scores_tc_kernel<false, 64, 64, 1>;
     else if (a.npad == 256 && HI == 64 && group == 4)
-        kern = fp8 ? index_scores_tc_kernel<true, 256, 64> : index_scores_tc_kernel<false, 256, 64>;
+        kern = fp8 ? index_scores_tc_kernel<true, 256, 64, 1> : index_scores_tc_kernel<false, 256, 64, 1>;
     e = smem_ceiling(kern);
     if (e != cudaSuccess) return e;
     CSA_LAUNCH(st, fp8 ? "index_scores_tc_fp8" : "index_scores_tc",

@@ -59,19 +59,15 @@ __device__ __forceinline__ float ld_score(const float* p) { return __ldcg(p); }
 __device__ __forceinline__ float ld_score(const bf16* p) {
     return __uint_as_float((uint32_t)__ldcg(reinterpret_cast<const unsigned short*>(p)) << 16);
 }
-// 16 bytes of scores, widened: 4 fp32 or 8 bf16.
-__device__ __forceinline__ void ld_vec(const float* p, float* f) {
-    const float4 q = __ldcg(reinterpret_cast<const float4*>(p));
-    f[0] = q.x; f[1] = q.y; f[2] = q.z; f[3] = q.w;
-}
-__device__ __forceinline__ void ld_vec(const bf16* p, float* f) {
-    const uint4 q = __ldcg(reinterpret_cast<const uint4*>(p));
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
+// Score e of a 16-byte vector of scores kept as raw words (4 fp32 or 8 bf16),
+// widened to fp32 where it is used, so the vectors in flight take 4
+// registers each whatever the score type.
+template <typename TS>
+__device__ __forceinline__ float vec_score(const uint4& q, int e) {
+    const uint32_t w = (e & (16 / (int)sizeof(TS) / 2)) ? ((e & (16 / (int)sizeof(TS) / 4)) ? q.w : q.z)
+                                                         : ((e & (16 / (int)sizeof(TS) / 4)) ? q.y : q.x);
+    if constexpr (sizeof(TS) == 4) return __uint_as_float(w);
+    else return __uint_as_float((e & 1) ? (w & 0xFFFF0000u) : (w << 16));
 }
 
 namespace cg = cooperative_groups;
@@ -518,23 +514,18 @@ __device__ void filter_slice(const TS* srow, int64_t lo, int64_t hi, uint32_t th
     const float stl = intl ? ld_score(srow + it) : 0.f;
     static_assert(kV * kU <= 64, "one mask bit per value");
     for (int64_t b0 = 0; b0 < nvec; b0 += kU * kThreads) {
-        float f[kV * kU];
+        uint4 raw[kU];
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
             const int64_t j = b0 + u * kThreads + tid;
-            if (j < nvec) {
-                ld_vec(srow + lo_v + kV * j, f + kV * u);
-            } else {
-#pragma unroll
-                for (int v = 0; v < kV; ++v) f[kV * u + v] = 0.f;
-            }
+            raw[u] = j < nvec ? __ldcg(reinterpret_cast<const uint4*>(srow + lo_v + kV * j)) : make_uint4(0, 0, 0, 0);
         }
         // this thread's takers, then one reservation per warp
         uint64_t mask = 0;
 #pragma unroll
         for (int e = 0; e < kV * kU; ++e) {
             const int64_t j = b0 + (e / kV) * kThreads + tid;
-            if (j < nvec && orderable(f[e]) >= thr) mask |= 1ull << e;
+            if (j < nvec && orderable(vec_score<TS>(raw[e / kV], e % kV)) >= thr) mask |= 1ull << e;
         }
         const uint32_t mine = __popcll(mask);
         uint32_t incl = mine;
@@ -552,7 +543,7 @@ __device__ void filter_slice(const TS* srow, int64_t lo, int64_t hi, uint32_t th
         for (int e = 0; e < kV * kU; ++e) {
             if (mask & (1ull << e)) {
                 const int64_t i = lo_v + kV * (b0 + (e / kV) * kThreads + tid) + (e % kV);
-                if (slot < cap) buf[slot] = composite(f[e], i);
+                if (slot < cap) buf[slot] = composite(vec_score<TS>(raw[e / kV], e % kV), i);
                 ++slot;
             }
         }
