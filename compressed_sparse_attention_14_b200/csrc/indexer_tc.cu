@@ -274,7 +274,8 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < a.stages; ++i) { tc::mbar_init(&sm.full[i], 1); tc::mbar_init(&sm.empty[i], 1); }
-        for (int i = 0; i < 4; ++i) { tc::mbar_init(&sm.tfull[i], 1); tc::mbar_init(&sm.tempty[i], 4); }
+        // prefill (kN == 256): both epilogue sets reduce every tile, so all 8 warps release it
+        for (int i = 0; i < 4; ++i) { tc::mbar_init(&sm.tfull[i], 1); tc::mbar_init(&sm.tempty[i], kN == 256 ? 8 : 4); }
         tc::mbar_init(sm.qfull, 1);
         tc::mbar_init(sm.qempty, kIssuers);   // every issuer releases each group's q
         tc::mbar_init(sm.fin, kIssuers);
@@ -408,8 +409,11 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        // two sets of four warps take alternate tiles; within a set, warp w
-        // reads TMEM lane quadrant w % 4
+        // two sets of four warps take alternate tiles (prefill, kN == 256:
+        // both sets take every tile, set s reducing the columns of queries
+        // 2s and 2s+1, which halves the per-tile latency of the epilogue that
+        // paces the two accumulator buffers); within a set, warp w reads TMEM
+        // lane quadrant w % 4
         const int set = (warp - 2) >> 2;
         const int quad = warp & 3;
         const int row = quad * 32 + lane;          // key within the tile
@@ -422,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
         int cur = -1;
         int64_t vis = 0;
         for (int64_t it = 0; it < my; ++it, wk.next(a, ngroups)) {
-            if ((int)(it & 1) != set) continue;
+            if (kN != 256 && (int)(it & 1) != set) continue;
             if (wk.g != cur) {
                 __syncwarp();
                 for (int c = lane; c < a.npad; c += 32) {
@@ -454,7 +458,14 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
                 sc[hh][0] = sc[hh][1] = sc[hh][2] = sc[hh][3] = 0.f;
                 const uint32_t taddr =
                     tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)((buf * kH + hh) * a.npad);
-                head_reduce<kN, kHI>(taddr, wv, a.npad, a.HI, a.group, sc[hh]);
+                if constexpr (kN == 256) {
+                    float s2[4] = {0.f, 0.f, 0.f, 0.f};
+                    head_reduce<128, kHI>(taddr + set * 128, wv + set * 128, a.npad, a.HI, a.group, s2);
+                    sc[hh][2 * set] = s2[0];
+                    sc[hh][2 * set + 1] = s2[1];
+                } else {
+                    head_reduce<kN, kHI>(taddr, wv, a.npad, a.HI, a.group, sc[hh]);
+                }
             }
             tc::tc_fence_before();
             __syncwarp();
@@ -465,6 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
 #pragma unroll
                 for (int gq = 0; gq < 4; ++gq) {
                     const int tq = wk.g * a.group + gq;
+                    if (kN == 256 && (gq >> 1) != set) continue;
                     if (gq < a.group && tq < a.nq) {
                         const float v = kFp8 ? sc[hh][gq] * kscale[hh] : sc[hh][gq];
                         if (a.score_bf16)

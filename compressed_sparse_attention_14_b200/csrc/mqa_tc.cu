@@ -50,7 +50,9 @@ namespace cg = cooperative_groups;
 
 namespace {
 
-constexpr int kThreads = 192;
+// warp 0 loads, warps 1 and 6 issue MMAs (warp 1 also owns TMEM), warps 2-5
+// run the softmax and the epilogue
+constexpr int kThreads = 224;
 constexpr int kE = 128;                 // entries per tile
 constexpr int kMaxDBlocks = 8;          // c <= 512
 constexpr uint32_t kWaitLimit = 1u << 24;
@@ -266,11 +268,13 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kMaxDBlocks; ++i) { tc::mbar_init(&kv_full[i], 1); tc::mbar_init(&kv_empty[i], 1); }
-        for (int i = 0; i < 2; ++i) { tc::mbar_init(&s_full[i], 1); tc::mbar_init(&s_empty[i], 4); }
+        // sparse: two issuers each commit their half of S and of O
+        const uint32_t nis = a.idx ? 2u : 1u;
+        for (int i = 0; i < 2; ++i) { tc::mbar_init(&s_full[i], nis); tc::mbar_init(&s_empty[i], 4); }
         tc::mbar_init(q_full, 1);
         tc::mbar_init(p_full, 4);
-        tc::mbar_init(o_done, 1);
-        tc::mbar_init(fin, 1);
+        tc::mbar_init(o_done, nis);
+        tc::mbar_init(fin, nis);
         tc::fence_mbar_init();
         s_abort = 0;
     }
@@ -282,8 +286,11 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = s_tmem;
-    const uint32_t tmem_S = tmem;                              // 2 x hg columns
-    const uint32_t tmem_O = tmem + 2 * (uint32_t)a.hg;         // mtiles x hg columns
+    // S^T (double-buffered); sparse: the second issuer's half of S^T beside
+    // it; then O^T (mtiles x hg columns)
+    const uint32_t tmem_S = tmem;                                      // 2 x hg columns
+    const uint32_t tmem_SB = tmem + 2 * (uint32_t)a.hg;                // 2 x hg columns (sparse)
+    const uint32_t tmem_O = tmem + (a.idx ? 4u : 2u) * (uint32_t)a.hg; // mtiles x hg columns
     volatile int* abort_flag = &s_abort;
 
     if (warp == 0) {
@@ -379,9 +386,18 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
                 for (int b = 0; b < a.dblocks; ++b) tc::mbar_wait(&kv_full[b], (j - 1) & 1, kWaitLimit);
             if (lane == 0) tc::mbar_wait(q_full, 0, kWaitLimit);
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp == 6) {
         // ---------------------------------------------------------------- MMA
-        if (lane == 0 && ntiles > 0) {
+        // Sparse: two issuing threads (each tcgen05.mma costs its issuer
+        // tens of ns, and a tile takes 32 for S and 32 for O). Issuer mi
+        // accumulates S^T over its half of the 64-dim blocks into its own
+        // accumulator (the softmax adds the two) and O^T for the dim tiles
+        // mt with mt % 2 == mi; both wait for the same phases of every
+        // barrier they share, in the same order. Dense: warp 1 alone (two
+        // consumers of one ring would wait on different phases of a slot's
+        // barrier, which a parity wait cannot tell apart).
+        const int mi = warp == 6 ? 1 : 0;
+        if (lane == 0 && ntiles > 0 && (mi == 0 || a.idx)) {
             const uint32_t idesc1 = tc::idesc_bf16_f32(128, a.hg, 0, 0);
             const uint32_t idesc2 = tc::idesc_bf16_f32(128, a.hg, 1, 1);
             const uint32_t kv_addr = tc::smem_u32(kv_s);
@@ -435,17 +451,19 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
                 }
                 j = ntiles;   // skip the sparse loop below
             }
+            const int b_lo = mi * (a.dblocks / 2), b_hi = b_lo + a.dblocks / 2;
+            const uint32_t my_S = mi ? tmem_SB : tmem_S;
             for (; ok && j < ntiles; ++j) {
                 const int sb = j & 1;
                 if (j >= 2 && !(ok = wait_or_abort(&s_empty[sb], ((j >> 1) - 1) & 1, abort_flag, a.status))) break;
-                // S^T = KV . q^T
-                for (int b = 0; b < a.dblocks && ok; ++b) {
+                // this issuer's part of S^T = KV . q^T (its 64-dim blocks)
+                for (int b = b_lo; b < b_hi && ok; ++b) {
                     if (!(ok = wait_or_abort(&kv_full[b], j & 1, abort_flag, a.status))) break;
                     tc::tc_fence_after();
                     for (int kk = 0; kk < 4; ++kk) {
                         uint64_t ad = tc::sdesc_sw128(kv_addr + b * (kE * 128) + kk * 32, 16, 1024);
                         uint64_t bd = tc::sdesc_sw128(q_addr + b * (a.hg * 128) + kk * 32, 16, 1024);
-                        tc::umma_bf16(tmem_S + sb * a.hg, ad, bd, idesc1, (b | kk) ? 1u : 0u);
+                        tc::umma_bf16(my_S + sb * a.hg, ad, bd, idesc1, (b > b_lo || kk) ? 1u : 0u);
                     }
                 }
                 if (!ok) break;
@@ -453,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
                 // O^T += KV^T . P^T once the softmax has written P
                 if (!(ok = wait_or_abort(p_full, j & 1, abort_flag, a.status))) break;
                 tc::tc_fence_after();
-                for (int mt = 0; mt < a.mtiles; ++mt) {
+                for (int mt = mi; mt < a.mtiles; mt += 2) {
                     for (int ke = 0; ke < kE / 16; ++ke) {
                         uint64_t ad = tc::sdesc_sw128(kv_addr + (2 * mt) * (kE * 128) + ke * 2048, kE * 128, 1024);
                         uint64_t bd = tc::sdesc_sw128(p_addr + ke * 2048, kE * 128, 1024);
@@ -468,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
             tc::umma_commit(fin);
             tc::mbar_wait(fin, 0, kWaitLimit);
         }
-    } else {
+    } else if (warp < 6) {
         // ---------------------------------------------------------------- softmax + epilogue
         const int quad = warp & 3;
         const int row = quad * 32 + lane;            // entry within the tile / dim within an M tile
@@ -495,11 +513,20 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
             tc::tc_fence_after();
             float z[64];
             const uint32_t taddr = tmem_S + ((uint32_t)(quad * 32) << 16) + sb * hg;
+            const uint32_t taddr_b = tmem_SB + ((uint32_t)(quad * 32) << 16) + sb * hg;
 #pragma unroll
             for (int cc = 0; cc < 64; cc += 16) {
                 if (cc < hg) {
                     float v[16];
                     tc::tmem_ld16(taddr + cc, v);
+                    if (a.idx) {
+                        // sparse: S^T is the sum of the two issuers' halves
+                        float v2[16];
+                        tc::tmem_ld16(taddr_b + cc, v2);
+                        tc::tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] += v2[i];
+                    }
 #pragma unroll
                     for (int i = 0; i < 16; ++i) z[cc + i] = v[i];
                 } else {
@@ -765,7 +792,7 @@ cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, Que
     a.dblocks = c / 64;
     a.mtiles = c / 128;
     a.q_bytes = (uint32_t)(a.hg * c * 2);
-    uint32_t need = 2 * a.hg + a.mtiles * a.hg, cols = 32;
+    uint32_t need = (idx ? 4 : 2) * a.hg + a.mtiles * a.hg, cols = 32;
     while (cols < need) cols <<= 1;
     a.tmem_cols = cols;
 
