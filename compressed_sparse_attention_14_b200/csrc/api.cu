@@ -318,7 +318,11 @@ int hca_compress_chunk(const float* proj, float* state, const float* bias, int64
 
 size_t csa_decode_compress_workspace_size(int B, int c, int cI) {
     if (B < 0 || c < 0 || cI < 0) return 0;
-    return align256((size_t)B * 4 * c * sizeof(float)) + align256((size_t)B * 4 * cI * sizeof(float));
+    // decode-time projections run split over K (a few rows, a 21 MB weight
+    // stream at d = 4096) and the workspace holds every slice's partial sums;
+    // the split count depends on d, which this query does not take: size for
+    // the largest split project_ksplit2 can choose (64 slices)
+    return align256((size_t)64 * B * 4 * c * sizeof(float)) + align256((size_t)64 * B * 4 * cI * sizeof(float));
 }
 
 int csa_decode_compress(const void* x_new, const void* W_kv, const float* B_kv, const void* W_idx, const float* B_idx,
@@ -345,13 +349,23 @@ int csa_decode_compress(const void* x_new, const void* W_kv, const float* B_kv, 
     CSA_TRY(check_ws(ws, ws_bytes, csa_decode_compress_workspace_size(B, c, cI)));
     cudaStream_t st = (cudaStream_t)stream;
     Carve cv(ws);
-    float* pk = (float*)cv.take((size_t)B * 4 * c * sizeof(float));
-    float* pi = (float*)cv.take((size_t)B * 4 * cI * sizeof(float));
-    CSA_CUDA(project(x_new, W_kv, B, d, 4 * c, pk, t, st), "csa_decode_compress: KV projection");
-    CSA_CUDA(project(x_new, W_idx, B, d, 4 * cI, pi, t, st), "csa_decode_compress: index-key projection");
-    CSA_CUDA(compress_step(pk, state_kv, B_kv, pos, B, c, m, true, Nmax, kv_cache, t, st), "csa_decode_compress: KV");
-    CSA_CUDA(compress_step(pi, state_idx, B_idx, pos, B, cI, m, true, Nmax, idx_cache, t, st),
-             "csa_decode_compress: index keys");
+    float* pk = (float*)cv.take((size_t)64 * B * 4 * c * sizeof(float));
+    float* pi = (float*)cv.take((size_t)64 * B * 4 * cI * sizeof(float));
+    // bf16: both split-K tensor-core projections in one launch (every SM
+    // streams a slice of the weights); then one launch of the step kernel
+    // adds the slices' partial sums in order and compresses both streams
+    int ks_kv = 1, ks_idx = 1;
+    if (t == ElemType::BF16) {
+        project_ksplit2(B, d, 4 * c, 4 * cI, &ks_kv, &ks_idx);
+        CSA_CUDA(project_tc2(x_new, B, d, W_kv, 4 * c, pk, ks_kv, W_idx, 4 * cI, pi, ks_idx, device_status(), st),
+                 "csa_decode_compress: projections");
+    } else {
+        CSA_CUDA(project(x_new, W_kv, B, d, 4 * c, pk, t, st), "csa_decode_compress: KV projection");
+        CSA_CUDA(project(x_new, W_idx, B, d, 4 * cI, pi, t, st), "csa_decode_compress: index-key projection");
+    }
+    const StepStream skv{pk, state_kv, B_kv, kv_cache, c, ks_kv, (int64_t)B * 4 * c};
+    const StepStream sidx{pi, state_idx, B_idx, idx_cache, cI, ks_idx, (int64_t)B * 4 * cI};
+    CSA_CUDA(compress_step_csa2(skv, sidx, pos, B, m, Nmax, t, st), "csa_decode_compress: compressors");
     return CSA_OK;
 }
 

@@ -119,6 +119,24 @@ __global__ void __launch_bounds__(256) hca_compress_kernel(const TIn* __restrict
     else store8(reinterpret_cast<float*>(out + i * c + j), o);
 }
 
+// The sum of nsplit fp32 slices of 8 channels, slice s at src + s * pstride,
+// added in slice order. The loads of 16 slices issue before their adds (a
+// batch past the last slice re-reads the last one and adds nothing).
+__device__ __forceinline__ void sum_slices(const float* src, int nsplit, int64_t pstride, float (&v)[8]) {
+    load8(src, v);
+    for (int k0 = 1; k0 < nsplit; k0 += 16) {
+        float u[16][8];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) load8(src + (int64_t)min(k0 + q, nsplit - 1) * pstride, u[q]);
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+            if (k0 + q < nsplit) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[e] += u[q][e];
+            }
+    }
+}
+
 // Decode-time compression through the per-sequence state cache [Walk §5
 // item 2: CSA keeps the tail tokens that have not yet formed a block; Notes
 // §2.6 Fig. 6]. Each sequence keeps the projected rows of its last 2m tokens
@@ -130,40 +148,57 @@ __global__ void __launch_bounds__(256) hca_compress_kernel(const TIn* __restrict
 // sequence and reads only the ring values of those channels, written by the
 // same thread slot in this step or an earlier one (an earlier launch has
 // completed before pdl_wait returns).
-template <typename TOut>
-__global__ void __launch_bounds__(256) csa_compress_step_kernel(const float* __restrict__ proj_new,
-                                                                float* __restrict__ state,
-                                                                const float* __restrict__ bias,
-                                                                const int32_t* __restrict__ pos, int B, int c,
-                                                                int m, int64_t Nmax, TOut* __restrict__ cache) {
+// proj may hold nsplit partial sums of the projection (a split-K GEMM),
+// slice s at proj + s * pstride; they are added in slice order. One launch
+// serves up to two streams with the same m and positions (the KV and
+// index-key compressors of a decode step): blocks [0, blocks0) take stream 0,
+// the rest stream 1. A block takes 32 (sequence, 8-channel) pairs; warp w
+// sums and stores group w of the four (a-values, b-values, a-logits,
+// b-logits), and after a block barrier warp 0 mixes the blocks that close.
+// kM > 0: the compression rate is the compile-time kM, so the window loops
+// unroll and their loads issue together.
+template <typename TOut, int kM>
+__global__ void __launch_bounds__(128) csa_compress_step_kernel(const StepStream s0, const StepStream s1,
+                                                                const int32_t* __restrict__ pos, int B, int m_rt,
+                                                                int64_t Nmax, int blocks0) {
+    const int m = kM > 0 ? kM : m_rt;
     pdl_wait();
     pdl_launch_next();
+    const bool second = (int)blockIdx.x >= blocks0;
+    const int blk = second ? (int)blockIdx.x - blocks0 : (int)blockIdx.x;
+    const int c = second ? s1.c : s0.c;
+    const float* __restrict__ proj_new = second ? s1.proj : s0.proj;
+    float* state = second ? s1.state : s0.state;
+    const float* __restrict__ bias = second ? s1.bias : s0.bias;
+    const int nsplit = second ? s1.nsplit : s0.nsplit;
+    const int64_t pstride = second ? s1.pstride : s0.pstride;
     const int groups = c / 8;
-    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (gid >= (int64_t)B * groups) return;
-    const int b = (int)(gid / groups);
-    const int j = (int)(gid % groups) * 8;
-    const int64_t p = pos[b];
-    if (p < 0) return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t pair = (int64_t)blk * 32 + lane;
+    const bool live = groups > 0 && pair < (int64_t)B * groups;
+    int b = 0, j = 0;
+    int64_t p = -1;
+    if (live) {
+        b = (int)(pair / groups);
+        j = (int)(pair % groups) * 8;
+        p = pos[b];
+    }
     const int64_t ld = 4 * (int64_t)c;
     float* ring = state + (int64_t)b * 2 * m * ld;
-    {
-        const float* src = proj_new + (int64_t)b * ld;
-        float* dst = ring + (p % (2 * m)) * ld;
+    if (live && p >= 0) {
         float v[8];
-#pragma unroll
-        for (int s4 = 0; s4 < 4; ++s4) {
-            load8(src + s4 * c + j, v);
-            store8(dst + s4 * c + j, v);
-        }
+        sum_slices(proj_new + (int64_t)b * ld + warp * c + j, nsplit, pstride, v);
+        store8(ring + (p % (2 * m)) * ld + warp * c + j, v);
     }
-    if ((p + 1) % m != 0) return;
+    __syncthreads();   // the block's ring stores are visible to its warp 0
+    if (warp != 0 || !live || p < 0 || (p + 1) % m != 0) return;
     const int64_t i = (p + 1) / m - 1;   // the block this token closes
     if (i >= Nmax) return;
 
     OnlineSoftmax8 sm;
     sm.init();
     float z[8], bb[8], v[8];
+#pragma unroll(kM > 0 ? kM : 1)
     for (int r = 0; r < m; ++r) {
         const float* row = ring + ((m * i + r) % (2 * m)) * ld;
         load8(row + 2 * c + j, z);
@@ -174,6 +209,7 @@ __global__ void __launch_bounds__(256) csa_compress_step_kernel(const float* __r
         sm.push(z, v);
     }
     if (i > 0) {
+#pragma unroll(kM > 0 ? kM : 1)
         for (int r = 0; r < m; ++r) {
             const float* row = ring + ((m * (i - 1) + r) % (2 * m)) * ld;
             load8(row + 3 * c + j, z);
@@ -187,7 +223,7 @@ __global__ void __launch_bounds__(256) csa_compress_step_kernel(const float* __r
     float o[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) o[u] = sm.acc[u] / sm.den[u];
-    TOut* out = cache + ((int64_t)b * Nmax + i) * c + j;
+    TOut* out = reinterpret_cast<TOut*>(second ? s1.cache : s0.cache) + ((int64_t)b * Nmax + i) * c + j;
     if constexpr (sizeof(TOut) == 2) store8(reinterpret_cast<bf16*>(out), o);
     else store8(reinterpret_cast<float*>(out), o);
 }
@@ -199,7 +235,8 @@ __global__ void __launch_bounds__(256) hca_compress_step_kernel(const float* __r
                                                                 float* __restrict__ state,
                                                                 const float* __restrict__ bias,
                                                                 const int32_t* __restrict__ pos, int B, int c,
-                                                                int mp, int64_t Nmax, TOut* __restrict__ cache) {
+                                                                int mp, int64_t Nmax, TOut* __restrict__ cache,
+                                                                int nsplit, int64_t pstride) {
     pdl_wait();
     pdl_launch_next();
     const int groups = c / 8;
@@ -214,11 +251,12 @@ __global__ void __launch_bounds__(256) hca_compress_step_kernel(const float* __r
     {
         const float* src = proj_new + (int64_t)b * ld;
         float* dst = ring + (p % mp) * ld;
-        float v[8];
-        load8(src + j, v);
-        store8(dst + j, v);
-        load8(src + c + j, v);
-        store8(dst + c + j, v);
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+            float v[8];
+            sum_slices(src + h * c + j, nsplit, pstride, v);
+            store8(dst + h * c + j, v);
+        }
     }
     if ((p + 1) % mp != 0) return;
     const int64_t i = (p + 1) / mp - 1;
@@ -405,30 +443,45 @@ cudaError_t compress_hca(const void* proj, const float* bias, int64_t n, int c, 
 }
 
 cudaError_t compress_step(const float* proj_new, float* state, const float* bias, const int32_t* pos, int B, int c,
-                          int m, bool overlap, int64_t Nmax, void* cache, ElemType out_t, cudaStream_t st) {
+                          int m, bool overlap, int64_t Nmax, void* cache, ElemType out_t, cudaStream_t st, int nsplit) {
+    if (overlap) {
+        StepStream s{proj_new, state, bias, cache, c, nsplit, (int64_t)B * 4 * c};
+        StepStream none{};
+        return compress_step_csa2(s, none, pos, B, m, Nmax, out_t, st);
+    }
+    const int64_t pstride = (int64_t)B * 2 * c;
     const int64_t threads = (int64_t)B * (c / 8);
     if (threads == 0) return cudaSuccess;
     const dim3 grid((unsigned)((threads + 255) / 256));
     cudaError_t e = cudaSuccess;
-    if (overlap) {
-        if (out_t == ElemType::BF16)
-            CSA_LAUNCH(st, "csa_compress_step",
-                       e = launch_pdl(csa_compress_step_kernel<bf16>, grid, dim3(256), 0, st, 0, proj_new, state, bias,
-                                      pos, B, c, m, Nmax, (bf16*)cache));
-        else
-            CSA_LAUNCH(st, "csa_compress_step",
-                       e = launch_pdl(csa_compress_step_kernel<float>, grid, dim3(256), 0, st, 0, proj_new, state,
-                                      bias, pos, B, c, m, Nmax, (float*)cache));
-    } else {
-        if (out_t == ElemType::BF16)
-            CSA_LAUNCH(st, "hca_compress_step",
-                       e = launch_pdl(hca_compress_step_kernel<bf16>, grid, dim3(256), 0, st, 0, proj_new, state, bias,
-                                      pos, B, c, m, Nmax, (bf16*)cache));
-        else
-            CSA_LAUNCH(st, "hca_compress_step",
-                       e = launch_pdl(hca_compress_step_kernel<float>, grid, dim3(256), 0, st, 0, proj_new, state,
-                                      bias, pos, B, c, m, Nmax, (float*)cache));
-    }
+    if (out_t == ElemType::BF16)
+        CSA_LAUNCH(st, "hca_compress_step",
+                   e = launch_pdl(hca_compress_step_kernel<bf16>, grid, dim3(256), 0, st, 0, proj_new, state, bias,
+                                  pos, B, c, m, Nmax, (bf16*)cache, nsplit, pstride));
+    else
+        CSA_LAUNCH(st, "hca_compress_step",
+                   e = launch_pdl(hca_compress_step_kernel<float>, grid, dim3(256), 0, st, 0, proj_new, state, bias,
+                                  pos, B, c, m, Nmax, (float*)cache, nsplit, pstride));
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+cudaError_t compress_step_csa2(const StepStream& s0, const StepStream& s1, const int32_t* pos, int B, int m,
+                               int64_t Nmax, ElemType out_t, cudaStream_t st) {
+    const int64_t pairs0 = (int64_t)B * (s0.c / 8), pairs1 = (int64_t)B * (s1.c / 8);
+    const int blocks0 = (int)((pairs0 + 31) / 32);
+    const int64_t blocks = blocks0 + (pairs1 + 31) / 32;
+    if (blocks == 0) return cudaSuccess;
+    const dim3 grid((unsigned)blocks);
+    cudaError_t e = cudaSuccess;
+    if (out_t == ElemType::BF16)
+        CSA_LAUNCH(st, "csa_compress_step",
+                   e = launch_pdl(m == 4 ? csa_compress_step_kernel<bf16, 4> : csa_compress_step_kernel<bf16, 0>, grid,
+                                  dim3(128), 0, st, 0, s0, s1, pos, B, m, Nmax, blocks0));
+    else
+        CSA_LAUNCH(st, "csa_compress_step",
+                   e = launch_pdl(m == 4 ? csa_compress_step_kernel<float, 4> : csa_compress_step_kernel<float, 0>,
+                                  grid, dim3(128), 0, st, 0, s0, s1, pos, B, m, Nmax, blocks0));
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

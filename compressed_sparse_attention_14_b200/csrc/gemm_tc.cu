@@ -16,6 +16,13 @@
 //              thread), 16-byte fp32 stores, masked at the matrix edges.
 // The two accumulators let the epilogue of one tile overlap the main loop of
 // the next. Waits are bounded (CSA_ERR_TIMEOUT in the status word).
+//
+// Split K (project_tc_splitk): for a few rows (one decode step's new tokens)
+// the 128 x 256 tiles are too few to stream the weights from every SM, so
+// the contraction is also cut into ksplit slices: a work item is (row tile,
+// column tile, K slice), and slice s writes its fp32 partial sums to
+// out + s * n * M. The consumer adds the ksplit partials in slice order
+// (deterministic).
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -38,7 +45,34 @@ struct GemmArgs {
     float* out;
     int* status;
     int tiles_m, tiles_n;
+    int ksplit;     // K slices (1: no split); slice s covers 64-deep blocks [s*kbs, (s+1)*kbs)
+    int kbs;        // 64-deep K blocks per slice
+    int items0;     // work items of this problem; items past it belong to the second problem
+    // second problem (same x): W2 [M2, d] into out2
+    int M2;
+    float* out2;
+    int tiles_n2, ksplit2, kbs2, items2;
 };
+
+// A work item: problem, K slice, row tile, column tile and its K blocks.
+struct Item {
+    int prob, ks, tm, tn, kb0, kb1;
+};
+
+__device__ __forceinline__ Item item_of(const GemmArgs& a, int tile, int kblocks_all) {
+    Item it;
+    it.prob = tile >= a.items0;
+    if (it.prob) tile -= a.items0;
+    const int ksplit = it.prob ? a.ksplit2 : a.ksplit, tiles_n = it.prob ? a.tiles_n2 : a.tiles_n;
+    const int kbs = it.prob ? a.kbs2 : a.kbs;
+    it.ks = tile % ksplit;
+    const int mn = tile / ksplit;
+    it.tm = mn / tiles_n;
+    it.tn = mn % tiles_n;
+    it.kb0 = it.ks * kbs;
+    it.kb1 = min(kblocks_all, it.kb0 + kbs);
+    return it;
+}
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                               int* status) {
@@ -55,7 +89,8 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 
 __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_constant__ GemmArgs a,
                                                                  const __grid_constant__ CUtensorMap tmX,
-                                                                 const __grid_constant__ CUtensorMap tmW) {
+                                                                 const __grid_constant__ CUtensorMap tmW,
+                                                                 const __grid_constant__ CUtensorMap tmW2) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint64_t* full = (uint64_t*)(base + kStages * kStageBytes);
@@ -67,8 +102,8 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
     __shared__ int s_abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int ntiles = a.tiles_m * a.tiles_n;
-    const int kblocks = (a.d + kBK - 1) / kBK;
+    const int ntiles = a.items0 + a.items2;
+    const int kblocks_all = (a.d + kBK - 1) / kBK;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) { tc::mbar_init(&full[i], 1); tc::mbar_init(&empty[i], 1); }
@@ -85,6 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
     if (warp == 0 && lane == 0) {
         tc::tma_prefetch_desc(&tmX);
         tc::tma_prefetch_desc(&tmW);
+        if (a.items2) tc::tma_prefetch_desc(&tmW2);
     }
     __syncthreads();
     tc::tc_fence_after();
@@ -98,16 +134,17 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
             uint32_t it = 0;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
-                const int tm = tile / a.tiles_n, tn = tile % a.tiles_n;
-                for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                const Item w = item_of(a, tile, kblocks_all);
+                const CUtensorMap* tw = w.prob ? &tmW2 : &tmW;
+                for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
                     const int s = (int)(it % kStages);
                     if (it >= kStages && !(ok = wait_or_abort(&empty[s], ((it / kStages) - 1) & 1, abort_flag,
                                                               a.status)))
                         break;
                     uint8_t* st = base + (size_t)s * kStageBytes;
                     tc::mbar_expect_tx(&full[s], kStageBytes);
-                    tc::tma_load_2d(st, &tmX, &full[s], kb * kBK, tm * kBM);
-                    tc::tma_load_2d(st + kBM * 128, &tmW, &full[s], kb * kBK, tn * kBN);
+                    tc::tma_load_2d(st, &tmX, &full[s], kb * kBK, w.tm * kBM);
+                    tc::tma_load_2d(st + kBM * 128, tw, &full[s], kb * kBK, w.tn * kBN);
                 }
             }
             // drain the copies of the last stages
@@ -128,7 +165,9 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
                     break;
                 tc::tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)(buf * kBN);
-                for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                const Item w = item_of(a, tile, kblocks_all);
+                const int kb0 = w.kb0;
+                for (int kb = kb0; kb < w.kb1; ++kb, ++it) {
                     const int s = (int)(it % kStages);
                     if (!(ok = wait_or_abort(&full[s], (it / kStages) & 1, abort_flag, a.status))) break;
                     tc::tc_fence_after();
@@ -136,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
                     const uint64_t bd = b0 + (uint64_t)(s * stage_step);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        tc::umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) ? 1u : 0u);
+                        tc::umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb > kb0 || kk) ? 1u : 0u);
                     tc::umma_commit(&empty[s]);
                 }
                 if (ok) tc::umma_commit(&tfull[buf]);
@@ -152,11 +191,12 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
             const int buf = (int)(tcount & 1);
             if (!wait_or_abort(&tfull[buf], (tcount >> 1) & 1, abort_flag, a.status)) break;
             tc::tc_fence_after();
-            const int tm = tile / a.tiles_n, tn = tile % a.tiles_n;
-            const int64_t row = (int64_t)tm * kBM + row_in_tile;
-            const int col0 = tn * kBN;
+            const Item w = item_of(a, tile, kblocks_all);
+            const int M = w.prob ? a.M2 : a.M;
+            const int64_t row = (int64_t)w.tm * kBM + row_in_tile;
+            const int col0 = w.tn * kBN;
             const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * kBN);
-            float* orow = a.out + row * a.M;
+            float* orow = (w.prob ? a.out2 : a.out) + (int64_t)w.ks * a.n * M + row * M;
             for (int c0 = 0; c0 < kBN; c0 += 64) {
                 float v[64];
 #pragma unroll
@@ -166,11 +206,11 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
 #pragma unroll
                     for (int j = 0; j < 64; j += 4) {
                         const int col = col0 + c0 + j;
-                        if (col + 3 < a.M) {
+                        if (col + 3 < M) {
                             *reinterpret_cast<float4*>(orow + col) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
                         } else {
                             for (int u = 0; u < 4; ++u)
-                                if (col + u < a.M) orow[col + u] = v[j + u];
+                                if (col + u < M) orow[col + u] = v[j + u];
                         }
                     }
                 }
@@ -198,28 +238,68 @@ static int sm_count() {
     return n;
 }
 
-cudaError_t project_tc(const void* x, const void* W, int64_t n, int d, int M, float* out, int* status,
-                       cudaStream_t st) {
-    if (n == 0 || M == 0) return cudaSuccess;
+static int clamp_ksplit(int ks, int kblocks_all) { return ks < 1 ? 1 : ks > kblocks_all ? kblocks_all : ks; }
+
+cudaError_t project_tc2(const void* x, int64_t n, int d, const void* W0, int M0, float* out0, int ks0, const void* W1,
+                        int M1, float* out1, int ks1, int* status, cudaStream_t st) {
+    if (n == 0 || (M0 == 0 && M1 == 0)) return cudaSuccess;
+    const int kblocks_all = (d + kBK - 1) / kBK;
     GemmArgs a{};
     a.n = n;
     a.d = d;
-    a.M = M;
-    a.out = out;
     a.status = status;
     a.tiles_m = (int)((n + kBM - 1) / kBM);
-    a.tiles_n = (M + kBN - 1) / kBN;
-    CUtensorMap tmX, tmW;
+    a.M = M0;
+    a.out = out0;
+    a.ksplit = clamp_ksplit(ks0, kblocks_all);
+    a.kbs = (kblocks_all + a.ksplit - 1) / a.ksplit;
+    a.tiles_n = (M0 + kBN - 1) / kBN;
+    a.items0 = a.tiles_m * a.tiles_n * a.ksplit;
+    a.M2 = W1 ? M1 : 0;
+    a.out2 = out1;
+    a.ksplit2 = clamp_ksplit(ks1, kblocks_all);
+    a.kbs2 = (kblocks_all + a.ksplit2 - 1) / a.ksplit2;
+    a.tiles_n2 = (a.M2 + kBN - 1) / kBN;
+    a.items2 = a.tiles_m * a.tiles_n2 * a.ksplit2;
+    CUtensorMap tmX, tmW, tmW2;
     if (!make_tmap_bf16_2d(&tmX, x, (uint64_t)n, d, d, kBM, kBK)) return cudaErrorInvalidValue;
-    if (!make_tmap_bf16_2d(&tmW, W, (uint64_t)M, d, d, kBN, kBK)) return cudaErrorInvalidValue;
+    if (M0 > 0 && !make_tmap_bf16_2d(&tmW, W0, (uint64_t)M0, d, d, kBN, kBK)) return cudaErrorInvalidValue;
+    if (a.items2 > 0 && !make_tmap_bf16_2d(&tmW2, W1, (uint64_t)a.M2, d, d, kBN, kBK)) return cudaErrorInvalidValue;
+    if (M0 == 0) tmW = tmW2;
+    if (a.items2 == 0) tmW2 = tmW;
     const size_t smem = 1024 + (size_t)kStages * kStageBytes + 16 * sizeof(uint64_t);
     cudaError_t e = smem_ceiling(project_tc_kernel);
     if (e != cudaSuccess) return e;
-    const int ntiles = a.tiles_m * a.tiles_n;
+    const int ntiles = a.items0 + a.items2;
     const int grid = ntiles < sm_count() ? ntiles : sm_count();
-    CSA_LAUNCH(st, "project_tc", e = launch_pdl(project_tc_kernel, dim3(grid), dim3(kThreads), smem, st, 0, a, tmX, tmW));
+    CSA_LAUNCH(st, "project_tc",
+               e = launch_pdl(project_tc_kernel, dim3(grid), dim3(kThreads), smem, st, 0, a, tmX, tmW, tmW2));
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
+}
+
+cudaError_t project_tc(const void* x, const void* W, int64_t n, int d, int M, float* out, int* status,
+                       cudaStream_t st, int ksplit) {
+    if (M == 0) return cudaSuccess;
+    return project_tc2(x, n, d, W, M, out, ksplit, nullptr, 0, nullptr, 1, status, st);
+}
+
+void project_ksplit2(int64_t n, int d, int M0, int M1, int* ks0, int* ks1) {
+    const int64_t rows = (n + kBM - 1) / kBM;
+    const int64_t t0 = rows * ((M0 + kBN - 1) / kBN), t1 = rows * ((M1 + kBN - 1) / kBN);
+    const int kblocks = (d + kBK - 1) / kBK;
+    int k0 = 1, k1 = 1;
+    for (;;) {
+        // the problem whose items stream the most weight blocks splits next
+        const int64_t w0 = t0 ? (kblocks + k0 - 1) / k0 : 0, w1 = t1 ? (kblocks + k1 - 1) / k1 : 0;
+        const bool first = w0 >= w1;
+        const int kn = 2 * (first ? k0 : k1);
+        const int64_t items = first ? t0 * kn + t1 * k1 : t0 * k0 + t1 * kn;
+        if (kn > 64 || kblocks / kn < 4 || items > sm_count()) break;
+        (first ? k0 : k1) = kn;
+    }
+    *ks0 = k0;
+    *ks1 = k1;
 }
 
 }  // namespace csa

@@ -92,8 +92,26 @@ cudaError_t compress_hca(const void* proj, const float* bias, int64_t n, int c, 
 // compress.cu, decode time: store the newest token's projected row of each
 // sequence in its state ring (2m rows of [C^a|C^b|Z^a|Z^b] when overlap, m
 // rows of [C|Z] otherwise) and write the entry of a block the token closes.
+// proj_new may hold nsplit partial sums (slice s at proj_new + s * B * row
+// width), added in slice order.
 cudaError_t compress_step(const float* proj_new, float* state, const float* bias, const int32_t* pos, int B, int c,
-                          int m, bool overlap, int64_t Nmax, void* cache, ElemType out_t, cudaStream_t st);
+                          int m, bool overlap, int64_t Nmax, void* cache, ElemType out_t, cudaStream_t st,
+                          int nsplit = 1);
+// One CSA compressor stream of a decode step: proj holds nsplit partial sums
+// [B, 4c] fp32, slice s at proj + s * pstride; state [B, 2m, 4c]; bias [2m, c];
+// cache [B, Nmax, c] of the output type.
+struct StepStream {
+    const float* proj;
+    float* state;
+    const float* bias;
+    void* cache;
+    int c, nsplit;
+    int64_t pstride;
+};
+// both CSA streams of a decode step (same m, positions and output type) in
+// one launch; s1.c == 0 leaves the second out
+cudaError_t compress_step_csa2(const StepStream& s0, const StepStream& s1, const int32_t* pos, int B, int m,
+                               int64_t Nmax, ElemType out_t, cudaStream_t st);
 
 // compress.cu, chunks at any start and length: the entries of every block
 // that ends inside the chunk [start, start+n) (proj rows fp32, one sequence),
@@ -106,8 +124,19 @@ cudaError_t compress_chunk_state(const float* proj, float* state, const float* b
 // gemm.cu: out[n, M] (fp32) = x[n, d] . W[M, d]^T (bf16 -> gemm_tc.cu)
 cudaError_t project(const void* x, const void* W, int64_t n, int d, int M, float* out, ElemType t,
                     cudaStream_t st);
+// ksplit > 1: the contraction is cut into ksplit slices whose fp32 partial
+// sums go to out + s * n * M (out holds ksplit * n * M floats).
 cudaError_t project_tc(const void* x, const void* W, int64_t n, int d, int M, float* out, int* status,
-                       cudaStream_t st);
+                       cudaStream_t st, int ksplit = 1);
+// Two projections of the same rows in one launch: x [n, d] times W0 [M0, d]
+// into out0 (ks0 K slices) and times W1 [M1, d] into out1 (ks1 slices), each
+// laid out as project_tc lays out its output.
+cudaError_t project_tc2(const void* x, int64_t n, int d, const void* W0, int M0, float* out0, int ks0, const void* W1,
+                        int M1, float* out1, int ks1, int* status, cudaStream_t st);
+// K slices for two projections of n rows sharing one launch: the slices of
+// the one with the longer weight stream per work item double while the work
+// items fit on the SMs and a slice keeps at least 4 blocks of 64
+void project_ksplit2(int64_t n, int d, int M0, int M1, int* ks0, int* ks1);
 
 // indexer.cu (FFMA, fp32 mode): scores[t, 0..Nmax) with ld = ld_scores;
 // -inf past the visible range (the whole row for a query whose sequence is
@@ -154,7 +183,7 @@ cudaError_t topk_select_positions(const float* scores, int64_t ld, int64_t pos_b
 bool mqa_tc_supported(int H, int c);
 int mqa_tc_nsplit(int nq, int H, int64_t max_entries, int num_sms);
 // splits merged inside one thread-block cluster (no workspace, no combine launch)
-bool mqa_tc_cluster(int nsplit);
+bool mqa_tc_cluster(int nsplit, int nq, int H);
 cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, QuerySpec qs, int mp, int nq, int n_seq,
                    int H, int c, int64_t Nmax, float scale, const float* sink, void* out, float* lse, void* ws,
                    int nsplit, int* status, cudaStream_t st);

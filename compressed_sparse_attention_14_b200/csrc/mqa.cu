@@ -230,7 +230,7 @@ static int plan_nsplit(int nq, int H, int64_t max_entries, ElemType t) {
 size_t mqa_workspace_bytes(int nq, int H, int c, int64_t max_entries, ElemType t) {
     int ns = plan_nsplit(nq, H, max_entries, t);
     // a single split writes the output directly; clustered splits merge on chip
-    if (t == ElemType::BF16 && (ns == 1 || mqa_tc_cluster(ns))) return 0;
+    if (t == ElemType::BF16 && (ns == 1 || mqa_tc_cluster(ns, nq, H))) return 0;
     return align256((size_t)nq * ns * H * c * sizeof(float)) +
            align256((size_t)nq * ns * H * 2 * sizeof(float));
 }
@@ -244,7 +244,7 @@ cudaError_t mqa(const void* q, const void* KV, const int32_t* idx, int k, QueryS
         const int ns = plan_nsplit(nq, H, max_entries, t);
         cudaError_t e = mqa_tc(q, KV, idx, k, qs, mp, nq, n_seq, H, c, Nmax, scale, sink, out, lse, ws, ns,
                                device_status(), st);
-        if (e != cudaSuccess || ns == 1 || mqa_tc_cluster(ns)) return e;
+        if (e != cudaSuccess || ns == 1 || mqa_tc_cluster(ns, nq, H)) return e;
         float* part_o = (float*)ws;
         float* part_ml = (float*)((char*)ws + align256((size_t)nq * ns * H * c * sizeof(float)));
         CSA_LAUNCH(st, "mqa_combine",

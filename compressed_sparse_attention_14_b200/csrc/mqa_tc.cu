@@ -21,23 +21,27 @@
 // gathered with 16-byte cp.async (the producer warp moves four rows'
 // 128-byte block per instruction), and the tile's 64-dim blocks are released
 // one by one as the second product finishes with them, so the next tile's
-// gather overlaps it. HCA (dense): consecutive rows stream through a ring of
-// 32 KB slots (a pair of 64-dim blocks per slot, one TMA box per block);
-// every tile passes through twice, for S and again (from L2) for O, in the
-// order S(0), S(1), O(0), S(2), O(1), ..., O(n-1), so the HBM read of tile
-// j+1 overlaps the softmax of tile j.
+// gather overlaps it. HCA (dense): consecutive rows stream through two rings
+// of 32 KB slots (a pair of 64-dim blocks per slot, one TMA box per block):
+// every tile passes through twice, once through the S ring for the first
+// product and again (mostly from L2) through the O ring for the second, each
+// ring with its own loading thread and its own MMA-issuing thread, so the
+// HBM read of the next tiles runs while tile j waits for its softmax.
 //
-// Warp roles: warp 0 loads (all lanes issue gathers), warp 1 allocates TMEM
-// and one lane issues the MMAs, warps 2-5 run the softmax and the epilogue.
+// Warp roles: warp 0 loads (sparse: all lanes issue gathers; dense: the S
+// ring), warp 1 allocates TMEM, one lane each of warps 1 and 6 issues MMAs,
+// warps 2-5 run the softmax and the epilogue, warp 7 loads the dense O ring.
 // A single split writes the normalised output directly. Up to
 // kMaxClusterSplits splits of one query run as one thread-block cluster and
 // merge on chip: each CTA stages its unnormalised O (fp32) in the shared
 // memory its KV tile used, and after a cluster barrier CTA g combines the
 // g-th slice of the head dimension from every split's O over distributed
-// shared memory (fixed order: deterministic). More splits write partials
-// (O, max, sum) to the workspace for mqa_combine. Waits are bounded
+// shared memory (fixed order: deterministic). Otherwise the splits write
+// partials (O, max, sum) to the workspace for mqa_combine. Waits are bounded
 // (CSA_ERR_TIMEOUT).
 #include <cooperative_groups.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -50,16 +54,18 @@ namespace cg = cooperative_groups;
 
 namespace {
 
-// warp 0 loads, warps 1 and 6 issue MMAs (warp 1 also owns TMEM), warps 2-5
-// run the softmax and the epilogue
-constexpr int kThreads = 224;
+// warp 0 loads (dense: the S-pass ring), warps 1 and 6 issue MMAs (warp 1
+// also owns TMEM), warps 2-5 run the softmax and the epilogue, warp 7 loads
+// the O-pass ring of the dense path
+constexpr int kThreads = 256;
 constexpr int kE = 128;                 // entries per tile
 constexpr int kMaxDBlocks = 8;          // c <= 512
 constexpr uint32_t kWaitLimit = 1u << 24;
 constexpr float kRescaleLog2 = 8.0f;    // move the reference max past 2^8
-// Splits merged in one cluster: at most 4, since clusters of one-CTA-per-SM
-// blocks larger than that fit fewer at a time than the SMs allow.
-constexpr int kMaxClusterSplits = 4;
+// Splits merged in one cluster: at most 8 (the portable cluster size); the
+// host takes a cluster only when all of the launch's clusters can be resident
+// at once.
+constexpr int kMaxClusterSplits = 8;
 
 struct MqaArgs {
     QueryMap qm;
@@ -134,93 +140,124 @@ __device__ __forceinline__ void bar_sync_128() { asm volatile("bar.sync 1, 128;"
 // The splits of query t (one cluster, rank = split) merge on chip: after a
 // cluster barrier, CTA `split` combines its slice of the head dimension for
 // every head from all splits' staged O (fp32, [head][dim] where the KV tile
-// was), their reference maxima and sums (log2 domain) and the sink.
+// was), their reference maxima and sums (log2 domain) and the sink. kG is the
+// largest cluster the instance handles (G <= kG splits take part).
 // (The launch parameters come in by value: read through a pointer to the
 // kernel's parameter block inside this out-of-line function, every access
 // would be a slow generic load.)
+template <int kG>
 __device__ __noinline__ void cluster_merge(int G, int c, int H, const float* sink, float* lse_out, bf16* out, int t,
-                                           int h0, int split, float* obuf, float* mref_s, float* lsum_s) {
-    __shared__ float coef_s[kMaxClusterSplits][64];
+                                           int h0, int split, float* obuf, float* mref_s, float* lsum_s,
+                                           float (*coef_s)[64]) {
     cg::cluster_group cl = cg::this_cluster();
     cl.sync();   // every split's obuf, reference max and sum are final
     const int tid = threadIdx.x;
     if (tid < 64) {
         const int h = h0 + tid;
-        // every split's max and sum loaded at once (fully unrolled over the
-        // largest cluster, so the arrays stay in registers)
+        // every split's max and sum loaded at once (fully unrolled, so the
+        // arrays stay in registers)
         const float sk = (sink && h < H) ? sink[h] * 1.4426950408889634f : -INFINITY;
-        float mq[kMaxClusterSplits], lq[kMaxClusterSplits];
+        float mq[kG], lq[kG];
 #pragma unroll
-        for (int q = 0; q < kMaxClusterSplits; ++q) {
+        for (int q = 0; q < kG; ++q) {
             mq[q] = q < G ? cl.map_shared_rank(mref_s, q)[tid] : -INFINITY;
             lq[q] = q < G ? cl.map_shared_rank(lsum_s, q)[tid] : 0.f;
         }
         float M = sk;
 #pragma unroll
-        for (int q = 0; q < kMaxClusterSplits; ++q) M = fmaxf(M, mq[q]);
+        for (int q = 0; q < kG; ++q) M = fmaxf(M, mq[q]);
         float L = (sk == -INFINITY) ? 0.f : exp2f(sk - M);
 #pragma unroll
-        for (int q = 0; q < kMaxClusterSplits; ++q)
+        for (int q = 0; q < kG; ++q)
             if (mq[q] != -INFINITY) L += lq[q] * exp2f(mq[q] - M);
         const float inv = L > 0.f ? 1.f / L : 0.f;
 #pragma unroll
-        for (int q = 0; q < kMaxClusterSplits; ++q)
+        for (int q = 0; q < kG; ++q)
             if (q < G) coef_s[q][tid] = (mq[q] == -INFINITY) ? 0.f : exp2f(mq[q] - M) * inv;
         if (split == 0 && lse_out && h < H)
             lse_out[(int64_t)t * H + h] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
     }
     __syncthreads();
     // this CTA's slice of the head dimension, every head, in units of 4
-    // dims (16-byte aligned, whatever G): sum over the splits in rank order
+    // dims (16-byte aligned, whatever G): sum over the splits in rank order.
+    // The (head, 4-dim chunk) items of the slice are spread over all threads,
+    // consecutive threads on consecutive chunks of one head; kR items per
+    // thread per round, every load of the round issued before any is used
+    // (the rounds are bound by the latency of the distributed-shared-memory
+    // reads)
     const int n4 = c / 4;
     const int lo4 = split * n4 / G, dn4 = (split + 1) * n4 / G - lo4;
-    // warp w takes heads w, w + 6, ...; its lanes walk the slice's 4-dim
-    // chunks (no division in the loop)
     const int nh = H - h0 < 64 ? H - h0 : 64;
-    for (int i = tid >> 5; i < nh; i += kThreads / 32) {
-        const int h = h0 + i;
-        float w[kMaxClusterSplits];
+    const int total = nh * dn4;
+    constexpr int kR = 16 / kG;
+    const float* src[kG];
 #pragma unroll
-        for (int q = 0; q < kMaxClusterSplits; ++q) w[q] = q < G ? coef_s[q][i] : 0.f;
-        // two 4-dim chunks per lane per round, all their loads issued
-        // before any is used
-        for (int j0 = tid & 31; j0 < dn4; j0 += 64) {
-            float4 v[kMaxClusterSplits][2];
+    for (int q = 0; q < kG; ++q)   // this CTA's own split straight from its shared memory
+        src[q] = q < G ? (q == split ? obuf : cl.map_shared_rank(obuf, q)) : obuf;
+    for (int base = tid; base < total; base += kR * kThreads) {
+        float4 v[kR][kG];
+        float w[kR][kG];
+        int hi[kR], ji[kR];
 #pragma unroll
-            for (int q = 0; q < kMaxClusterSplits; ++q) {
-                // this CTA's own split is read from its shared memory
-                // directly, the others' over distributed shared memory
-                const float* src = q == split ? obuf : cl.map_shared_rank(obuf, q);
+        for (int u = 0; u < kR; ++u) {
+            const int item = base + u * kThreads;
+            const bool ok = item < total;
+            hi[u] = ok ? item / dn4 : 0;
+            ji[u] = ok ? item - hi[u] * dn4 : 0;
 #pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    const int j = j0 + 32 * r;
-                    v[q][r] = (w[q] != 0.f && j < dn4)   // also every q >= G
-                                  ? *reinterpret_cast<const float4*>(src + i * c + 4 * (lo4 + j))
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
+            for (int q = 0; q < kG; ++q) {
+                w[u][q] = (ok && q < G) ? coef_s[q][hi[u]] : 0.f;
+                v[u][q] = w[u][q] != 0.f   // an empty split staged no O
+                              ? *reinterpret_cast<const float4*>(src[q] + hi[u] * c + 4 * (lo4 + ji[u]))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
             }
+        }
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int j = j0 + 32 * r;
-                if (j >= dn4) continue;
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int u = 0; u < kR; ++u) {
+            if (base + u * kThreads >= total) continue;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                for (int q = 0; q < kMaxClusterSplits; ++q) {
-                    if (w[q] == 0.f) continue;   // an empty split staged no O
-                    acc.x = fmaf(w[q], v[q][r].x, acc.x);
-                    acc.y = fmaf(w[q], v[q][r].y, acc.y);
-                    acc.z = fmaf(w[q], v[q][r].z, acc.z);
-                    acc.w = fmaf(w[q], v[q][r].w, acc.w);
-                }
-                __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x, acc.y), hi2 = __floats2bfloat162_rn(acc.z, acc.w);
-                uint2 pk;
-                pk.x = *reinterpret_cast<uint32_t*>(&lo2);
-                pk.y = *reinterpret_cast<uint32_t*>(&hi2);
-                *reinterpret_cast<uint2*>(out + ((int64_t)t * H + h) * c + 4 * (lo4 + j)) = pk;
+            for (int q = 0; q < kG; ++q) {
+                if (w[u][q] == 0.f) continue;
+                acc.x = fmaf(w[u][q], v[u][q].x, acc.x);
+                acc.y = fmaf(w[u][q], v[u][q].y, acc.y);
+                acc.z = fmaf(w[u][q], v[u][q].z, acc.z);
+                acc.w = fmaf(w[u][q], v[u][q].w, acc.w);
             }
+            __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x, acc.y), hi2 = __floats2bfloat162_rn(acc.z, acc.w);
+            uint2 pk;
+            pk.x = *reinterpret_cast<uint32_t*>(&lo2);
+            pk.y = *reinterpret_cast<uint32_t*>(&hi2);
+            *reinterpret_cast<uint2*>(out + ((int64_t)t * H + h0 + hi[u]) * c + 4 * (lo4 + ji[u])) = pk;
         }
     }
     cl.sync();   // the other CTAs' shared memory stays alive until read
+}
+
+// Dense path: one ring of 32 KB slots (a pair of 64-dim blocks each),
+// slots [r_lo, r_lo + r_n), filled with every tile of the split pair by pair,
+// in order; one producer and one consumer per ring.
+__device__ __noinline__ void dense_ring_load(const MqaArgs& a, uint8_t* kv_s, const CUtensorMap* tm, uint64_t* kv_full,
+                                             uint64_t* kv_empty, int r_lo, int r_n, int ntiles, int64_t row_base,
+                                             volatile int* abort_flag) {
+    uint32_t cnt = 0;
+    bool ok = true;
+    for (int jt = 0; ok && jt < ntiles; ++jt) {
+        const int row = (int)(row_base + (int64_t)jt * kE);
+        for (int mt = 0; mt < a.mtiles; ++mt, ++cnt) {
+            const int slot = r_lo + (int)(cnt % (uint32_t)r_n);
+            if (cnt >= (uint32_t)r_n &&
+                !(ok = wait_or_abort(&kv_empty[slot], ((cnt / r_n) - 1) & 1, abort_flag, a.status)))
+                break;
+            uint8_t* dst = kv_s + (size_t)slot * 2 * kE * 128;
+            tc::mbar_expect_tx(&kv_full[slot], 2 * kE * 128);
+            tc::tma_load_2d(dst, tm, &kv_full[slot], 2 * mt * 64, row);
+            tc::tma_load_2d(dst + kE * 128, tm, &kv_full[slot], (2 * mt + 1) * 64, row);
+        }
+    }
+    // drain: the copies still in flight must land
+    for (uint32_t i = cnt > (uint32_t)r_n ? cnt - r_n : 0; i < cnt; ++i)
+        tc::mbar_wait(&kv_full[r_lo + i % r_n], (i / r_n) & 1, kWaitLimit);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_constant__ MqaArgs a,
@@ -249,6 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
     uint64_t* fin = o_done + 1;
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
+    __shared__ float merge_coef[kMaxClusterSplits][64];   // cluster merge: each split's weight per head
 
     pdl_wait();
     pdl_launch_next();
@@ -268,13 +306,14 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kMaxDBlocks; ++i) { tc::mbar_init(&kv_full[i], 1); tc::mbar_init(&kv_empty[i], 1); }
-        // sparse: two issuers each commit their half of S and of O
+        // sparse: both issuers commit their half of S and of O; dense: the
+        // first issuer makes S, the second O
         const uint32_t nis = a.idx ? 2u : 1u;
         for (int i = 0; i < 2; ++i) { tc::mbar_init(&s_full[i], nis); tc::mbar_init(&s_empty[i], 4); }
         tc::mbar_init(q_full, 1);
         tc::mbar_init(p_full, 4);
         tc::mbar_init(o_done, nis);
-        tc::mbar_init(fin, nis);
+        tc::mbar_init(fin, 2);
         tc::fence_mbar_init();
         s_abort = 0;
     }
@@ -352,33 +391,11 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
                     }
                 }
             } else if (lane == 0) {
-                // Dense rows stream through the ring twice per tile, pair
-                // by pair of 64-dim blocks: for the first product (S) and
-                // again, from L2, for the second (O). Order S(0), then
-                // S(j), O(j-1) for j >= 1, then O(n-1): the HBM read of
-                // tile j+1 overlaps the softmax of tile j.
-                uint32_t cnt = 0;
-                bool ok = true;
-                for (int step = 0; ok && step <= ntiles; ++step) {
-                    for (int pass = 0; ok && pass < 2; ++pass) {
-                        const int jt = pass == 0 ? step : step - 1;   // S pass of tile step, O pass of step-1
-                        if (jt < 0 || jt >= ntiles) continue;
-                        const int row = (int)(row0 + e_beg + (int64_t)jt * kE);
-                        for (int mt = 0; mt < a.mtiles; ++mt, ++cnt) {
-                            const int slot = (int)(cnt % (uint32_t)a.ring);
-                            if (cnt >= (uint32_t)a.ring &&
-                                !(ok = wait_or_abort(&kv_empty[slot], ((cnt / a.ring) - 1) & 1, abort_flag, a.status)))
-                                break;
-                            uint8_t* dst = kv_s + (size_t)slot * 2 * kE * 128;
-                            tc::mbar_expect_tx(&kv_full[slot], 2 * kE * 128);
-                            tc::tma_load_2d(dst, &tmTile, &kv_full[slot], 2 * mt * 64, row);
-                            tc::tma_load_2d(dst + kE * 128, &tmTile, &kv_full[slot], (2 * mt + 1) * 64, row);
-                        }
-                    }
-                }
-                // drain: the copies still in flight must land
-                for (uint32_t i = cnt > (uint32_t)a.ring ? cnt - a.ring : 0; i < cnt; ++i)
-                    tc::mbar_wait(&kv_full[i % a.ring], (i / a.ring) & 1, kWaitLimit);
+                // Dense rows stream through the ring twice per tile, pair by
+                // pair of 64-dim blocks: for the first product (S) through
+                // this thread's ring, and again (mostly from L2) for the
+                // second (O) through warp 7's ring
+                dense_ring_load(a, kv_s, &tmTile, kv_full, kv_empty, 0, a.ring / 2, ntiles, row0 + e_beg, abort_flag);
                 j = 0;
             }
             // drain (sparse): the last issued tile and q must have landed
@@ -386,18 +403,24 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
                 for (int b = 0; b < a.dblocks; ++b) tc::mbar_wait(&kv_full[b], (j - 1) & 1, kWaitLimit);
             if (lane == 0) tc::mbar_wait(q_full, 0, kWaitLimit);
         }
+    } else if (warp == 7) {
+        // ---------------------------------------------------------------- dense: O-pass ring
+        if (!a.idx && lane == 0 && ntiles > 0)
+            dense_ring_load(a, kv_s, &tmTile, kv_full, kv_empty, a.ring / 2, a.ring - a.ring / 2, ntiles,
+                            row0 + e_beg, abort_flag);
     } else if (warp == 1 || warp == 6) {
         // ---------------------------------------------------------------- MMA
-        // Sparse: two issuing threads (each tcgen05.mma costs its issuer
-        // tens of ns, and a tile takes 32 for S and 32 for O). Issuer mi
+        // Two issuing threads (each tcgen05.mma costs its issuer tens of
+        // ns, and a tile takes 32 for S and 32 for O). Sparse: issuer mi
         // accumulates S^T over its half of the 64-dim blocks into its own
         // accumulator (the softmax adds the two) and O^T for the dim tiles
         // mt with mt % 2 == mi; both wait for the same phases of every
-        // barrier they share, in the same order. Dense: warp 1 alone (two
-        // consumers of one ring would wait on different phases of a slot's
-        // barrier, which a parity wait cannot tell apart).
+        // barrier they share, in the same order. Dense: issuer 0 makes S from
+        // the S-pass ring, issuer 1 makes O from the O-pass ring; each ring
+        // has one producer and one consumer, which take its slots' phases in
+        // order (a parity wait can only tell consecutive phases apart).
         const int mi = warp == 6 ? 1 : 0;
-        if (lane == 0 && ntiles > 0 && (mi == 0 || a.idx)) {
+        if (lane == 0 && ntiles > 0) {
             const uint32_t idesc1 = tc::idesc_bf16_f32(128, a.hg, 0, 0);
             const uint32_t idesc2 = tc::idesc_bf16_f32(128, a.hg, 1, 1);
             const uint32_t kv_addr = tc::smem_u32(kv_s);
@@ -406,48 +429,44 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
             bool ok = wait_or_abort(q_full, 0, abort_flag, a.status);
             int j = 0;
             if (!a.idx) {
-                // dense: the ring order of the producer, pair by pair
+                // dense: this issuer's ring, in the order its producer fills it
+                const int r_lo = mi ? a.ring / 2 : 0, r_n = mi ? a.ring - a.ring / 2 : a.ring / 2;
                 uint32_t cnt = 0;
-                for (int step = 0; ok && step <= ntiles; ++step) {
-                    for (int pass = 0; ok && pass < 2; ++pass) {
-                        const int jt = pass == 0 ? step : step - 1;
-                        if (jt < 0 || jt >= ntiles) continue;
-                        const int sb = jt & 1;
-                        if (pass == 0) {
-                            if (jt >= 2 && !(ok = wait_or_abort(&s_empty[sb], ((jt >> 1) - 1) & 1, abort_flag,
-                                                               a.status)))
-                                break;
-                        } else {
-                            if (!(ok = wait_or_abort(p_full, jt & 1, abort_flag, a.status))) break;
-                            tc::tc_fence_after();
-                        }
-                        for (int mt = 0; mt < a.mtiles; ++mt, ++cnt) {
-                            const int slot = (int)(cnt % (uint32_t)a.ring);
-                            if (!(ok = wait_or_abort(&kv_full[slot], (cnt / a.ring) & 1, abort_flag, a.status))) break;
-                            tc::tc_fence_after();
-                            const uint32_t sa = kv_addr + (uint32_t)slot * 2 * kE * 128;
-                            if (pass == 0) {
-                                // S^T += KV[:, blocks 2mt, 2mt+1] . q[:, same]^T
-                                for (int bb = 0; bb < 2; ++bb)
-                                    for (int kk = 0; kk < 4; ++kk) {
-                                        uint64_t ad = tc::sdesc_sw128(sa + bb * (kE * 128) + kk * 32, 16, 1024);
-                                        uint64_t bd = tc::sdesc_sw128(q_addr + (2 * mt + bb) * (a.hg * 128) + kk * 32,
-                                                                      16, 1024);
-                                        tc::umma_bf16(tmem_S + sb * a.hg, ad, bd, idesc1, (mt | bb | kk) ? 1u : 0u);
-                                    }
-                            } else {
-                                // O^T[dims of mt] += KV^T . P^T
-                                for (int ke = 0; ke < kE / 16; ++ke) {
-                                    uint64_t ad = tc::sdesc_sw128(sa + ke * 2048, kE * 128, 1024);
-                                    uint64_t bd = tc::sdesc_sw128(p_addr + ke * 2048, kE * 128, 1024);
-                                    tc::umma_bf16(tmem_O + mt * a.hg, ad, bd, idesc2, (jt > 0 || ke > 0) ? 1u : 0u);
-                                }
-                            }
-                            tc::umma_commit(&kv_empty[slot]);
-                        }
-                        if (!ok) break;
-                        tc::umma_commit(pass == 0 ? &s_full[sb] : o_done);
+                for (int jt = 0; ok && jt < ntiles; ++jt) {
+                    const int sb = jt & 1;
+                    if (mi == 0) {
+                        if (jt >= 2 && !(ok = wait_or_abort(&s_empty[sb], ((jt >> 1) - 1) & 1, abort_flag, a.status)))
+                            break;
+                    } else {
+                        if (!(ok = wait_or_abort(p_full, jt & 1, abort_flag, a.status))) break;
+                        tc::tc_fence_after();
                     }
+                    for (int mt = 0; mt < a.mtiles; ++mt, ++cnt) {
+                        const int slot = r_lo + (int)(cnt % (uint32_t)r_n);
+                        if (!(ok = wait_or_abort(&kv_full[slot], (cnt / r_n) & 1, abort_flag, a.status))) break;
+                        tc::tc_fence_after();
+                        const uint32_t sa = kv_addr + (uint32_t)slot * 2 * kE * 128;
+                        if (mi == 0) {
+                            // S^T += KV[:, blocks 2mt, 2mt+1] . q[:, same]^T
+                            for (int bb = 0; bb < 2; ++bb)
+                                for (int kk = 0; kk < 4; ++kk) {
+                                    uint64_t ad = tc::sdesc_sw128(sa + bb * (kE * 128) + kk * 32, 16, 1024);
+                                    uint64_t bd = tc::sdesc_sw128(q_addr + (2 * mt + bb) * (a.hg * 128) + kk * 32,
+                                                                  16, 1024);
+                                    tc::umma_bf16(tmem_S + sb * a.hg, ad, bd, idesc1, (mt | bb | kk) ? 1u : 0u);
+                                }
+                        } else {
+                            // O^T[dims of mt] += KV^T . P^T
+                            for (int ke = 0; ke < kE / 16; ++ke) {
+                                uint64_t ad = tc::sdesc_sw128(sa + ke * 2048, kE * 128, 1024);
+                                uint64_t bd = tc::sdesc_sw128(p_addr + ke * 2048, kE * 128, 1024);
+                                tc::umma_bf16(tmem_O + mt * a.hg, ad, bd, idesc2, (jt > 0 || ke > 0) ? 1u : 0u);
+                            }
+                        }
+                        tc::umma_commit(&kv_empty[slot]);
+                    }
+                    if (!ok) break;
+                    tc::umma_commit(mi == 0 ? &s_full[sb] : o_done);
                 }
                 j = ntiles;   // skip the sparse loop below
             }
@@ -623,26 +642,32 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
         // ------------------------------------------------------------ epilogue
         if (ok && ntiles > 0) ok = wait_or_abort(o_done, (ntiles - 1) & 1, abort_flag, a.status);
         tc::tc_fence_after();
-        // per-head sums: fixed-order reduction of the 128 per-entry partials
-        // [128][65] floats (padded: no bank conflicts) over the KV tile and, for
-        // c = 128, the start of q: neither is read any more
-        float* lred = (float*)kv_s;
-        bar_sync_128();
+        // per-head sums of the 128 per-entry partials (fixed order): a
+        // butterfly reduce-scatter within each warp leaves lane l with the
+        // warp's sums of heads 2l and 2l+1 (62 shuffles), then the four warps'
+        // sums are added through shared memory
+        {
 #pragma unroll
-        for (int h = 0; h < 64; ++h) lred[eth * 65 + h] = lpart[h];
-        bar_sync_128();
-        if (eth < 64) {
-            // eight interleaved partial sums (fixed order), so the loads
-            // are not one dependent chain of 128
-            float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-            for (int i = 0; i < 128; i += 8) {
+            for (int r = 0; r < 5; ++r) {
+                const int o = 16 >> r, nh = 32 >> r;
+                const bool upper = (lane & o) != 0;
 #pragma unroll
-                for (int u = 0; u < 8; ++u) ps[u] += lred[(i + u) * 65 + eth];
+                for (int i = 0; i < 32; ++i) {
+                    if (i < nh) {
+                        const float send = upper ? lpart[i] : lpart[i + nh];
+                        const float keep = upper ? lpart[i + nh] : lpart[i];
+                        lpart[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                    }
+                }
             }
-            lsum_s[eth] = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+            bar_sync_128();   // red_s may still be read by the last max update
+            red_s[quad * 64 + 2 * lane] = lpart[0];
+            red_s[quad * 64 + 2 * lane + 1] = lpart[1];
+            bar_sync_128();
+            if (eth < 64)
+                lsum_s[eth] = (red_s[eth] + red_s[64 + eth]) + (red_s[128 + eth] + red_s[192 + eth]);
+            bar_sync_128();
         }
-        bar_sync_128();
         const bool have_o = ok && ntiles > 0;
         if (a.cluster) {
             // stage this split's O^T as obuf[head][dim] (fp32) where the KV
@@ -741,8 +766,17 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, a.tmem_cols);
     }
-    if (a.cluster)
-        cluster_merge(a.nsplit, a.c, a.H, a.sink, a.lse, a.out, t, h0, split, (float*)kv_s, mref_s, lsum_s);
+    if (a.cluster) {
+        if (a.nsplit <= 2)
+            cluster_merge<2>(a.nsplit, a.c, a.H, a.sink, a.lse, a.out, t, h0, split, (float*)kv_s, mref_s, lsum_s,
+                             merge_coef);
+        else if (a.nsplit <= 4)
+            cluster_merge<4>(a.nsplit, a.c, a.H, a.sink, a.lse, a.out, t, h0, split, (float*)kv_s, mref_s, lsum_s,
+                             merge_coef);
+        else
+            cluster_merge<8>(a.nsplit, a.c, a.H, a.sink, a.lse, a.out, t, h0, split, (float*)kv_s, mref_s, lsum_s,
+                             merge_coef);
+    }
 }
 
 bool mqa_tc_supported(int H, int c) { return c % 128 == 0 && c <= 512 && H >= 1; }
@@ -755,10 +789,49 @@ int mqa_tc_nsplit(int nq, int H, int64_t max_entries, int num_sms) {
     if (ns > tiles) ns = tiles;
     if (ns < 1) ns = 1;
     if (ns > 64) ns = 64;
+    // splits are whole tiles: as many as the tiles per split need (9 splits
+    // of 64 tiles take 8 tiles each, so 8 splits do the same work)
+    if (tiles > 0) ns = (tiles + (tiles + ns - 1) / ns - 1) / ((tiles + ns - 1) / ns);
     return (int)ns;
 }
 
-bool mqa_tc_cluster(int nsplit) { return nsplit >= 2 && nsplit <= kMaxClusterSplits; }
+// Whether the nsplit splits of every (query, head group) run as one cluster
+// and merge on chip: clusters of up to 4 one-CTA-per-SM blocks always; of 5
+// to 8 only when every cluster of the launch can be resident at once (the
+// device's count of such clusters, asked once per cluster size).
+bool mqa_tc_cluster(int nsplit, int nq, int H) {
+    if (nsplit < 2 || nsplit > kMaxClusterSplits) return false;
+    if (nsplit <= 4) return true;
+    static std::mutex mu;
+    static int dev_seen[kMaxClusterSplits + 1][64];   // per (cluster size, device): 0 unknown, else count + 1
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    std::lock_guard<std::mutex> lock(mu);
+    int& cached = dev_seen[nsplit][dev];
+    if (cached == 0) {
+        int n = 0;
+        if (smem_ceiling(mqa_tc_kernel) == cudaSuccess) {
+            cudaLaunchConfig_t cfg = {};
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = (unsigned)nsplit;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.gridDim = dim3((unsigned)nsplit, 1, 1);
+            cfg.blockDim = dim3(kThreads);
+            cfg.dynamicSmemBytes = 200 * 1024;   // one CTA per SM, as every launch of this kernel
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if (cudaOccupancyMaxActiveClusters(&n, mqa_tc_kernel, &cfg) != cudaSuccess) {
+                (void)cudaGetLastError();
+                n = 0;
+            }
+        }
+        cached = n + 1;
+    }
+    const int64_t clusters = (int64_t)nq * ((H + 63) / 64);
+    return clusters <= (int64_t)(cached - 1);
+}
 
 cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, QuerySpec qs, int mp, int nq, int n_seq,
                    int H, int c, int64_t Nmax, float scale, const float* sink, void* out, float* lse, void* ws,
@@ -779,7 +852,7 @@ cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, Que
     a.scale_log2 = scale * 1.4426950408889634f;
     a.sink = sink;
     a.nsplit = nsplit;
-    a.cluster = mqa_tc_cluster(nsplit) ? 1 : 0;
+    a.cluster = mqa_tc_cluster(nsplit, nq, H) ? 1 : 0;
     const int64_t max_entries = idx ? k : Nmax;
     int64_t per = (max_entries + nsplit - 1) / nsplit;
     a.split_len = ((per + kE - 1) / kE) * kE;
@@ -804,11 +877,13 @@ cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, Que
     size_t kv_bytes = (size_t)a.dblocks * kE * 128;
     if (!idx) {
         // dense ring: as many 32 KB slots as fit (at most 8, at least the
-        // KV tile's size so the staging areas that reuse it still fit)
+        // KV tile's size so the staging areas that reuse it still fit, and
+        // at least 2: half the slots carry the S pass, half the O pass)
         // (4 KB left for the kernel's static shared memory)
         int ring = (int)((223 * 1024 - fixed) / (2 * kE * 128));
         if (ring > kMaxDBlocks) ring = kMaxDBlocks;
         if (ring < a.mtiles) ring = a.mtiles;
+        if (ring < 2) ring = 2;
         a.ring = ring;
         kv_bytes = (size_t)ring * 2 * kE * 128;
     }
