@@ -36,6 +36,18 @@ template <> __device__ __forceinline__ bf16 from_f32<bf16>(float v) { return __f
 
 // Load 8 consecutive elements (16-byte aligned for bf16, 32-byte for fp32)
 // as fp32.
+// four consecutive values, one 16-byte (fp32) or 8-byte (bf16) store
+__device__ __forceinline__ void store4(float* p, float a, float b, float c, float d) {
+    *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
+}
+__device__ __forceinline__ void store4(bf16* p, float a, float b, float c, float d) {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&lo);
+    u.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(p) = u;
+}
+
 __device__ __forceinline__ void load8(const bf16* p, float (&v)[8]) {
     uint4 u = *reinterpret_cast<const uint4*>(p);
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);

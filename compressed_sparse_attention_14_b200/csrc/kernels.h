@@ -182,8 +182,8 @@ cudaError_t topk_select_positions(const float* scores, int64_t ld, int64_t pos_b
 // mqa_tc.cu: tensor-core shared-KV MQA (bf16); ws holds split partials when nsplit > 1
 bool mqa_tc_supported(int H, int c);
 int mqa_tc_nsplit(int nq, int H, int64_t max_entries, int num_sms);
-// splits merged inside one thread-block cluster (no workspace, no combine launch)
-bool mqa_tc_cluster(int nsplit, int nq, int H);
+// two splits run as a cluster of two and merge on chip (no workspace, no combine launch)
+bool mqa_tc_pair(int nsplit);
 cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, QuerySpec qs, int mp, int nq, int n_seq,
                    int H, int c, int64_t Nmax, float scale, const float* sink, void* out, float* lse, void* ws,
                    int nsplit, int* status, cudaStream_t st);

@@ -147,57 +147,84 @@ __global__ void __launch_bounds__(256) mqa_partial_ffma_kernel(MqaPartialArgs a)
     }
 }
 
-// Merge of split-KV partials for one (query, head): split s holds O_s (fp32,
-// scaled by exp(-m_s)), m_s and l_s; the result is
+// Merge of split-KV partials: split s holds O_s (fp32, scaled by exp(-m_s)),
+// m_s and l_s for every (query, head); the result is
 //   out = sum_s e^{m_s - M} O_s / (sum_s e^{m_s - M} l_s + [sink] e^{z' - M})
 // with M the largest of the m_s and the sink logit, and lse = M + log(...).
-// The split weights are computed once into shared memory; each thread then
-// combines 4 consecutive dims with 16-byte loads.
+// A block takes kCombineHeads heads of one query and kCombineDims of their
+// dims: warp w works out head w's split weights (lanes over the splits), then
+// every thread combines 4 consecutive dims of one head at a time, the 16-byte
+// loads of up to 8 splits issued before their adds (in split order), one
+// store per 4 results.
+constexpr int kCombineHeads = 8;
+constexpr int kCombineDims = 128;
 template <typename T>
-__global__ void __launch_bounds__(128) mqa_combine_kernel(const float* __restrict__ part_o,
-                                                          const float* __restrict__ part_ml,
-                                                          int nsplit, int H, int c,
-                                                          const float* __restrict__ sink,
-                                                          T* __restrict__ out, float* __restrict__ lse) {
+__global__ void __launch_bounds__(kCombineHeads * 32) mqa_combine_kernel(const float* __restrict__ part_o,
+                                                                         const float* __restrict__ part_ml,
+                                                                         int nsplit, int H, int c,
+                                                                         const float* __restrict__ sink,
+                                                                         T* __restrict__ out, float* __restrict__ lse) {
     pdl_wait();
     pdl_launch_next();
-    __shared__ float s_w[64];
-    __shared__ float s_inv;
-    const int t = blockIdx.y, h = blockIdx.x;
-    const float* ml = part_ml + ((int64_t)t * nsplit * H + h) * 2;
-    if (threadIdx.x < 32) {
+    __shared__ float s_w[kCombineHeads][64];
+    __shared__ float s_inv[kCombineHeads];
+    const int t = blockIdx.y, h0 = blockIdx.x * kCombineHeads;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nh = H - h0 < kCombineHeads ? H - h0 : kCombineHeads;
+    if (warp < nh) {
+        const int h = h0 + warp;
+        const float* ml = part_ml + ((int64_t)t * nsplit * H + h) * 2;
         float M = sink ? sink[h] : -INFINITY;
-        for (int s = threadIdx.x; s < nsplit; s += 32) M = fmaxf(M, ml[(int64_t)s * H * 2]);
+        float mv[2], lv[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int sp = lane + 32 * u;
+            mv[u] = sp < nsplit ? ml[(int64_t)sp * H * 2] : -INFINITY;
+            lv[u] = sp < nsplit ? ml[(int64_t)sp * H * 2 + 1] : 0.f;
+            M = fmaxf(M, mv[u]);
+        }
         M = warp_max(M);
         float L = 0.f;
-        for (int s = threadIdx.x; s < nsplit; s += 32) {
-            float ms = ml[(int64_t)s * H * 2];
-            float wgt = (ms == -INFINITY || M == -INFINITY) ? 0.f : expf(ms - M);
-            s_w[s] = wgt;
-            L += wgt * ml[(int64_t)s * H * 2 + 1];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int sp = lane + 32 * u;
+            const float wgt = (mv[u] == -INFINITY || M == -INFINITY) ? 0.f : expf(mv[u] - M);
+            if (sp < nsplit) s_w[warp][sp] = wgt;
+            L += wgt * lv[u];
         }
         L = warp_sum(L);
-        if (threadIdx.x == 0) {
+        if (lane == 0) {
             if (sink && M != -INFINITY) L += expf(sink[h] - M);
-            s_inv = (L > 0.f) ? 1.f / L : 0.f;
-            if (lse) lse[(int64_t)t * H + h] = (L > 0.f) ? M + logf(L) : -INFINITY;
+            s_inv[warp] = (L > 0.f) ? 1.f / L : 0.f;
+            if (lse && blockIdx.z == 0) lse[(int64_t)t * H + h] = (L > 0.f) ? M + logf(L) : -INFINITY;
         }
     }
     __syncthreads();
-    const float inv = s_inv;
-    T* o = out + ((int64_t)t * H + h) * c;
-    for (int d = threadIdx.x * 4; d < c; d += blockDim.x * 4) {
+    const int d0 = blockIdx.z * kCombineDims;
+    const int c4 = (c - d0 < kCombineDims ? c - d0 : kCombineDims) / 4;
+    const int64_t sstride = (int64_t)H * c;   // one split to the next
+    for (int e = threadIdx.x; e < nh * c4; e += blockDim.x) {
+        const int i = e / c4, d = d0 + (e - i * c4) * 4;
+        const float* po = part_o + ((int64_t)t * nsplit * H + h0 + i) * c + d;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s = 0; s < nsplit; ++s) {
-            const float wgt = s_w[s];
-            if (wgt == 0.f) continue;
-            const float4 v = *reinterpret_cast<const float4*>(part_o + (((int64_t)t * nsplit + s) * H + h) * c + d);
-            acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
+        for (int s0 = 0; s0 < nsplit; s0 += 8) {
+            float4 v[8];
+            float wv[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                wv[u] = s0 + u < nsplit ? s_w[i][s0 + u] : 0.f;
+                // a split with weight 0 staged no O (its rows may be stale)
+                v[u] = wv[u] != 0.f ? *reinterpret_cast<const float4*>(po + (s0 + u) * sstride)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (wv[u] == 0.f) continue;
+                acc.x += wv[u] * v[u].x; acc.y += wv[u] * v[u].y; acc.z += wv[u] * v[u].z; acc.w += wv[u] * v[u].w;
+            }
         }
-        o[d] = from_f32<T>(acc.x * inv);
-        o[d + 1] = from_f32<T>(acc.y * inv);
-        o[d + 2] = from_f32<T>(acc.z * inv);
-        o[d + 3] = from_f32<T>(acc.w * inv);
+        const float inv = s_inv[i];
+        store4(out + ((int64_t)t * H + h0 + i) * c + d, acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
     }
 }
 
@@ -229,8 +256,8 @@ static int plan_nsplit(int nq, int H, int64_t max_entries, ElemType t) {
 
 size_t mqa_workspace_bytes(int nq, int H, int c, int64_t max_entries, ElemType t) {
     int ns = plan_nsplit(nq, H, max_entries, t);
-    // a single split writes the output directly; clustered splits merge on chip
-    if (t == ElemType::BF16 && (ns == 1 || mqa_tc_cluster(ns, nq, H))) return 0;
+    // a single split writes the output directly; two merge on chip
+    if (t == ElemType::BF16 && (ns == 1 || mqa_tc_pair(ns))) return 0;
     return align256((size_t)nq * ns * H * c * sizeof(float)) +
            align256((size_t)nq * ns * H * 2 * sizeof(float));
 }
@@ -244,11 +271,13 @@ cudaError_t mqa(const void* q, const void* KV, const int32_t* idx, int k, QueryS
         const int ns = plan_nsplit(nq, H, max_entries, t);
         cudaError_t e = mqa_tc(q, KV, idx, k, qs, mp, nq, n_seq, H, c, Nmax, scale, sink, out, lse, ws, ns,
                                device_status(), st);
-        if (e != cudaSuccess || ns == 1 || mqa_tc_cluster(ns, nq, H)) return e;
+        if (e != cudaSuccess || ns == 1 || mqa_tc_pair(ns)) return e;
         float* part_o = (float*)ws;
         float* part_ml = (float*)((char*)ws + align256((size_t)nq * ns * H * c * sizeof(float)));
         CSA_LAUNCH(st, "mqa_combine",
-                   e = launch_pdl(mqa_combine_kernel<bf16>, dim3(H, nq), dim3(128), 0, st, 0, (const float*)part_o,
+                   e = launch_pdl(mqa_combine_kernel<bf16>,
+                                  dim3((H + kCombineHeads - 1) / kCombineHeads, nq, (c + kCombineDims - 1) / kCombineDims),
+                                  dim3(kCombineHeads * 32), 0, st, 0, (const float*)part_o,
                                   (const float*)part_ml, ns, H, c, sink, (bf16*)out, lse));
         if (e != cudaSuccess) return e;
         return cudaGetLastError();
@@ -279,11 +308,13 @@ cudaError_t mqa(const void* q, const void* KV, const int32_t* idx, int k, QueryS
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    dim3 g2(H, nq);
+    dim3 g2((H + kCombineHeads - 1) / kCombineHeads, nq, (c + kCombineDims - 1) / kCombineDims);
     if (t == ElemType::BF16)
-        CSA_LAUNCH(st, "mqa_combine", mqa_combine_kernel<bf16><<<g2, 128, 0, st>>>(a.part_o, a.part_ml, ns, H, c, sink, (bf16*)out, lse));
+        CSA_LAUNCH(st, "mqa_combine", mqa_combine_kernel<bf16><<<g2, kCombineHeads * 32, 0, st>>>(
+                                          a.part_o, a.part_ml, ns, H, c, sink, (bf16*)out, lse));
     else
-        CSA_LAUNCH(st, "mqa_combine", mqa_combine_kernel<float><<<g2, 128, 0, st>>>(a.part_o, a.part_ml, ns, H, c, sink, (float*)out, lse));
+        CSA_LAUNCH(st, "mqa_combine", mqa_combine_kernel<float><<<g2, kCombineHeads * 32, 0, st>>>(
+                                          a.part_o, a.part_ml, ns, H, c, sink, (float*)out, lse));
     return cudaGetLastError();
 }
 

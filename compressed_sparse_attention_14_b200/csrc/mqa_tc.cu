@@ -18,8 +18,9 @@
 // reference, and cheap, since it rarely moves after the first tile.
 //
 // Entry sources. CSA (sparse): one tile buffer; the selected rows are
-// gathered with 16-byte cp.async (the producer warp moves four rows'
-// 128-byte block per instruction), and the tile's 64-dim blocks are released
+// gathered with 16-byte cp.async (two producer warps, half the rows each; a
+// warp moves four rows' 128-byte block per instruction), and the tile's
+// 64-dim blocks are released
 // one by one as the second product finishes with them, so the next tile's
 // gather overlaps it. HCA (dense): consecutive rows stream through two rings
 // of 32 KB slots (a pair of 64-dim blocks per slot, one TMA box per block):
@@ -28,21 +29,15 @@
 // ring with its own loading thread and its own MMA-issuing thread, so the
 // HBM read of the next tiles runs while tile j waits for its softmax.
 //
-// Warp roles: warp 0 loads (sparse: all lanes issue gathers; dense: the S
-// ring), warp 1 allocates TMEM, one lane each of warps 1 and 6 issues MMAs,
-// warps 2-5 run the softmax and the epilogue, warp 7 loads the dense O ring.
-// A single split writes the normalised output directly. Up to
-// kMaxClusterSplits splits of one query run as one thread-block cluster and
-// merge on chip: each CTA stages its unnormalised O (fp32) in the shared
-// memory its KV tile used, and after a cluster barrier CTA g combines the
-// g-th slice of the head dimension from every split's O over distributed
-// shared memory (fixed order: deterministic). Otherwise the splits write
-// partials (O, max, sum) to the workspace for mqa_combine. Waits are bounded
-// (CSA_ERR_TIMEOUT).
-#include <cooperative_groups.h>
-
-#include <mutex>
-
+// Warp roles: warps 0 and 7 load (sparse: all their lanes gather, half a
+// tile each; dense: one lane each fills the S ring and the O ring), warp 1
+// allocates TMEM, one lane each of warps 1 and 6 issues MMAs, warps 2-5 run
+// the softmax and the epilogue.
+// A single split writes the normalised output directly. More splits stage
+// their unnormalised O^T (fp32, [head][dim]) in the shared memory the KV
+// tile used, and one thread writes it to the workspace with bulk copies,
+// beside the split's reference maxima and sums; mqa_combine then merges the
+// splits in split order (deterministic). Waits are bounded (CSA_ERR_TIMEOUT).
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -50,22 +45,15 @@
 
 namespace csa {
 
-namespace cg = cooperative_groups;
-
 namespace {
 
-// warp 0 loads (dense: the S-pass ring), warps 1 and 6 issue MMAs (warp 1
-// also owns TMEM), warps 2-5 run the softmax and the epilogue, warp 7 loads
-// the O-pass ring of the dense path
+// warps 0 and 7 load, warps 1 and 6 issue MMAs (warp 1 also owns TMEM),
+// warps 2-5 run the softmax and the epilogue
 constexpr int kThreads = 256;
 constexpr int kE = 128;                 // entries per tile
 constexpr int kMaxDBlocks = 8;          // c <= 512
 constexpr uint32_t kWaitLimit = 1u << 24;
 constexpr float kRescaleLog2 = 8.0f;    // move the reference max past 2^8
-// Splits merged in one cluster: at most 8 (the portable cluster size); the
-// host takes a cluster only when all of the launch's clusters can be resident
-// at once.
-constexpr int kMaxClusterSplits = 8;
 
 struct MqaArgs {
     QueryMap qm;
@@ -79,7 +67,7 @@ struct MqaArgs {
     float scale_log2;
     const float* sink;
     int nsplit;
-    int cluster;              // the splits of a query form one cluster
+    int pair;                 // nsplit == 2: the query's two splits form a cluster and merge on chip
     int64_t split_len;
     bf16* out;
     float* lse;
@@ -137,101 +125,62 @@ __device__ __forceinline__ void bar_sync_128() { asm volatile("bar.sync 1, 128;"
 
 }  // namespace
 
-// The splits of query t (one cluster, rank = split) merge on chip: after a
-// cluster barrier, CTA `split` combines its slice of the head dimension for
-// every head from all splits' staged O (fp32, [head][dim] where the KV tile
-// was), their reference maxima and sums (log2 domain) and the sink. kG is the
-// largest cluster the instance handles (G <= kG splits take part).
-// (The launch parameters come in by value: read through a pointer to the
-// kernel's parameter block inside this out-of-line function, every access
-// would be a slow generic load.)
-template <int kG>
-__device__ __noinline__ void cluster_merge(int G, int c, int H, const float* sink, float* lse_out, bf16* out, int t,
-                                           int h0, int split, float* obuf, float* mref_s, float* lsum_s,
-                                           float (*coef_s)[64]) {
-    cg::cluster_group cl = cg::this_cluster();
-    cl.sync();   // every split's obuf, reference max and sum are final
-    const int tid = threadIdx.x;
-    if (tid < 64) {
-        const int h = h0 + tid;
-        // every split's max and sum loaded at once (fully unrolled, so the
-        // arrays stay in registers)
-        const float sk = (sink && h < H) ? sink[h] * 1.4426950408889634f : -INFINITY;
-        float mq[kG], lq[kG];
+// Sparse rows: 16-byte cp.async by whole warps, kGatherWarps of them, warp
+// `part` taking rows [part, part + 1) * kE / kGatherWarps of every tile. One
+// warp instruction moves one 64-dim block (128 B) of four rows, so every
+// access is a full, aligned 128-byte line; the chunk lands at its
+// 128-byte-swizzle position. (A TMA gather4 moves the same 512 B per
+// instruction but its issue rate, not DRAM, bounded the tile load.) Each
+// warp arrives on block b's barrier once its copies of it have completed.
+// Returns the tiles handed over.
+constexpr int kGatherWarps = 2;
+__device__ __forceinline__ int sparse_gather(const MqaArgs& a, uint8_t* kv_s, uint64_t* kv_full, uint64_t* kv_empty,
+                                             int part, int lane, int t, int ntiles, int64_t e_beg, int64_t e_end,
+                                             int64_t row0, volatile int* abort_flag) {
+    constexpr int kRows = kE / kGatherWarps;   // rows per warp per tile
+    const int chunk = lane & 7, rsub = lane >> 3;
+    const char* kv_g = (const char*)a.KV;
+    const int64_t row_bytes = (int64_t)a.c * 2;
+    int j = 0;
+    for (; j < ntiles; ++j) {
+        const int64_t e0 = e_beg + (int64_t)j * kE + part * kRows;
+        int rows[kRows / 4];
 #pragma unroll
-        for (int q = 0; q < kG; ++q) {
-            mq[q] = q < G ? cl.map_shared_rank(mref_s, q)[tid] : -INFINITY;
-            lq[q] = q < G ? cl.map_shared_rank(lsum_s, q)[tid] : 0.f;
+        for (int i = 0; i < kRows / 4; ++i) {
+            const int64_t e = e0 + 4 * i + rsub;
+            int s = -1;
+            if (e < e_end) s = a.idx[(int64_t)t * a.k + e];
+            if (s < 0 || s >= a.Nmax) s = 0;   // masked in the softmax
+            rows[i] = (int)(row0 + s);
         }
-        float M = sk;
+        bool ok = true;
+        for (int b = 0; b < a.dblocks; ++b) {
+            if (j > 0 && lane == 0) ok = wait_or_abort(&kv_empty[b], (j - 1) & 1, abort_flag, a.status);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            uint8_t* dst = kv_s + (size_t)b * kE * 128;
 #pragma unroll
-        for (int q = 0; q < kG; ++q) M = fmaxf(M, mq[q]);
-        float L = (sk == -INFINITY) ? 0.f : exp2f(sk - M);
-#pragma unroll
-        for (int q = 0; q < kG; ++q)
-            if (mq[q] != -INFINITY) L += lq[q] * exp2f(mq[q] - M);
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-#pragma unroll
-        for (int q = 0; q < kG; ++q)
-            if (q < G) coef_s[q][tid] = (mq[q] == -INFINITY) ? 0.f : exp2f(mq[q] - M) * inv;
-        if (split == 0 && lse_out && h < H)
-            lse_out[(int64_t)t * H + h] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
-    }
-    __syncthreads();
-    // this CTA's slice of the head dimension, every head, in units of 4
-    // dims (16-byte aligned, whatever G): sum over the splits in rank order.
-    // The (head, 4-dim chunk) items of the slice are spread over all threads,
-    // consecutive threads on consecutive chunks of one head; kR items per
-    // thread per round, every load of the round issued before any is used
-    // (the rounds are bound by the latency of the distributed-shared-memory
-    // reads)
-    const int n4 = c / 4;
-    const int lo4 = split * n4 / G, dn4 = (split + 1) * n4 / G - lo4;
-    const int nh = H - h0 < 64 ? H - h0 : 64;
-    const int total = nh * dn4;
-    constexpr int kR = 16 / kG;
-    const float* src[kG];
-#pragma unroll
-    for (int q = 0; q < kG; ++q)   // this CTA's own split straight from its shared memory
-        src[q] = q < G ? (q == split ? obuf : cl.map_shared_rank(obuf, q)) : obuf;
-    for (int base = tid; base < total; base += kR * kThreads) {
-        float4 v[kR][kG];
-        float w[kR][kG];
-        int hi[kR], ji[kR];
-#pragma unroll
-        for (int u = 0; u < kR; ++u) {
-            const int item = base + u * kThreads;
-            const bool ok = item < total;
-            hi[u] = ok ? item / dn4 : 0;
-            ji[u] = ok ? item - hi[u] * dn4 : 0;
-#pragma unroll
-            for (int q = 0; q < kG; ++q) {
-                w[u][q] = (ok && q < G) ? coef_s[q][hi[u]] : 0.f;
-                v[u][q] = w[u][q] != 0.f   // an empty split staged no O
-                              ? *reinterpret_cast<const float4*>(src[q] + hi[u] * c + 4 * (lo4 + ji[u]))
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int i = 0; i < kRows / 4; ++i) {
+                const int r = part * kRows + 4 * i + rsub;
+                cp_async16(dst + r * 128 + ((chunk ^ (r & 7)) << 4),
+                           kv_g + (int64_t)rows[i] * row_bytes + b * 128 + chunk * 16);
             }
+            cp_async_commit();
         }
-#pragma unroll
-        for (int u = 0; u < kR; ++u) {
-            if (base + u * kThreads >= total) continue;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int q = 0; q < kG; ++q) {
-                if (w[u][q] == 0.f) continue;
-                acc.x = fmaf(w[u][q], v[u][q].x, acc.x);
-                acc.y = fmaf(w[u][q], v[u][q].y, acc.y);
-                acc.z = fmaf(w[u][q], v[u][q].z, acc.z);
-                acc.w = fmaf(w[u][q], v[u][q].w, acc.w);
-            }
-            __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x, acc.y), hi2 = __floats2bfloat162_rn(acc.z, acc.w);
-            uint2 pk;
-            pk.x = *reinterpret_cast<uint32_t*>(&lo2);
-            pk.y = *reinterpret_cast<uint32_t*>(&hi2);
-            *reinterpret_cast<uint2*>(out + ((int64_t)t * H + h0 + hi[u]) * c + 4 * (lo4 + ji[u])) = pk;
+        // hand the blocks over in order as they complete
+        const int issued = ok ? a.dblocks : 0;
+        for (int b = 0; b < issued; ++b) {
+            cp_async_wait_pending(issued - 1 - b);
+            tc::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&kv_full[b]);
+        }
+        if (!ok) {
+            cp_async_wait_pending(0);
+            break;
         }
     }
-    cl.sync();   // the other CTAs' shared memory stays alive until read
+    return j;
 }
 
 // Dense path: one ring of 32 KB slots (a pair of 64-dim blocks each),
@@ -260,6 +209,73 @@ __device__ __noinline__ void dense_ring_load(const MqaArgs& a, uint8_t* kv_s, co
         tc::mbar_wait(&kv_full[r_lo + i % r_n], (i / r_n) & 1, kWaitLimit);
 }
 
+// The two splits of query t (a cluster of two, rank = split) merge on chip.
+// Each has staged its unnormalised O^T as [half][head][dim in half] fp32; after
+// a cluster barrier (both staged, maxima and sums final, receive areas free)
+// one thread of each sends the other split's half to it with one bulk copy
+// over distributed shared memory (into the peer's q area), counted on the
+// peer's mbarrier. Both work out the two weights per head from both splits'
+// reference maxima and sums and the sink (the same arithmetic on each side),
+// then split g writes half g of every head: w0 O_0 + w1 O_1, in split order,
+// 4 dims per 8-byte store. A last cluster barrier keeps each CTA's shared
+// memory alive until the peer's copy of it has landed.
+__device__ __noinline__ void pair_merge(int c, int H, const float* sink, float* lse_out, bf16* out, int t, int h0,
+                                        uint32_t split, bool have_o, const float* obuf, float* recv, float* mref_s,
+                                        float* lsum_s, uint64_t* xbar, float (*coef_s)[64], volatile int* abort_flag,
+                                        int* status) {
+    const int tid = threadIdx.x;
+    const uint32_t peer = split ^ 1u;
+    const int half = c / 2;
+    const uint32_t bytes = 64u * (uint32_t)half * 4u;
+    if (tid == 0) tc::mbar_expect_tx(xbar, bytes);
+    if (tid < 64 && !have_o) { mref_s[tid] = -INFINITY; lsum_s[tid] = 0.f; }
+    tc::cluster_sync();
+    if (tid == 0)
+        tc::bulk_copy_to_peer(tc::mapa(tc::smem_u32(recv), peer), obuf + (size_t)peer * 64 * half, bytes,
+                              tc::mapa(tc::smem_u32(xbar), peer));
+    if (tid < 64) {
+        const int h = h0 + tid;
+        const float sk = (sink && h < H) ? sink[h] * 1.4426950408889634f : -INFINITY;
+        const float m_own = mref_s[tid], l_own = lsum_s[tid];
+        const float m_peer = tc::ld_cluster_f32(tc::mapa(tc::smem_u32(mref_s + tid), peer));
+        const float l_peer = tc::ld_cluster_f32(tc::mapa(tc::smem_u32(lsum_s + tid), peer));
+        const float mq[2] = {split == 0 ? m_own : m_peer, split == 0 ? m_peer : m_own};
+        const float lq[2] = {split == 0 ? l_own : l_peer, split == 0 ? l_peer : l_own};
+        const float M = fmaxf(sk, fmaxf(mq[0], mq[1]));
+        float L = (sk == -INFINITY) ? 0.f : exp2f(sk - M);
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+            if (mq[q] != -INFINITY) L += lq[q] * exp2f(mq[q] - M);
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) coef_s[q][tid] = (mq[q] == -INFINITY) ? 0.f : exp2f(mq[q] - M) * inv;
+        if (split == 0 && lse_out && h < H)
+            lse_out[(int64_t)t * H + h] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+    }
+    // every thread waits for the peer's half (a bounded wait: on a timeout the
+    // status word says so and the half read below is stale)
+    wait_or_abort(xbar, 0, abort_flag, status);
+    __syncthreads();   // coef_s
+    const float* mine = obuf + (size_t)split * 64 * half;
+    const int nh = H - h0 < 64 ? H - h0 : 64;
+    const int h4 = half / 4;
+    for (int e = tid; e < nh * h4; e += kThreads) {
+        const int i = e / h4, j = e - i * h4;
+        const float4 va = *reinterpret_cast<const float4*>(mine + i * half + 4 * j);
+        const float4 vb = *reinterpret_cast<const float4*>(recv + i * half + 4 * j);
+        const float4 o0 = split == 0 ? va : vb, o1 = split == 0 ? vb : va;
+        const float w0 = coef_s[0][i], w1 = coef_s[1][i];
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (w0 != 0.f) { acc.x = w0 * o0.x; acc.y = w0 * o0.y; acc.z = w0 * o0.z; acc.w = w0 * o0.w; }
+        if (w1 != 0.f) {
+            acc.x = fmaf(w1, o1.x, acc.x); acc.y = fmaf(w1, o1.y, acc.y);
+            acc.z = fmaf(w1, o1.z, acc.z); acc.w = fmaf(w1, o1.w, acc.w);
+        }
+        store4(out + ((int64_t)t * H + h0 + i) * c + (int)split * half + 4 * j, acc.x, acc.y, acc.z, acc.w);
+    }
+    tc::cluster_sync();
+}
+
 __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_constant__ MqaArgs a,
                                                              const __grid_constant__ CUtensorMap tmQ,
                                                              const __grid_constant__ CUtensorMap tmTile) {
@@ -284,9 +300,10 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
     uint64_t* p_full = q_full + 1;
     uint64_t* o_done = p_full + 1;
     uint64_t* fin = o_done + 1;
+    uint64_t* xbar = fin + 1;   // pair merge: the peer's slice has arrived
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
-    __shared__ float merge_coef[kMaxClusterSplits][64];   // cluster merge: each split's weight per head
+    __shared__ float pair_coef[2][64];   // pair merge: each split's weight per head
 
     pdl_wait();
     pdl_launch_next();
@@ -305,7 +322,11 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
     const int64_t row0 = (int64_t)(seq_ok ? seq : 0) * a.Nmax;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kMaxDBlocks; ++i) { tc::mbar_init(&kv_full[i], 1); tc::mbar_init(&kv_empty[i], 1); }
+        // sparse: every gathering warp arrives on a block's full barrier
+        for (int i = 0; i < kMaxDBlocks; ++i) {
+            tc::mbar_init(&kv_full[i], a.idx ? (uint32_t)kGatherWarps : 1u);
+            tc::mbar_init(&kv_empty[i], 1);
+        }
         // sparse: both issuers commit their half of S and of O; dense: the
         // first issuer makes S, the second O
         const uint32_t nis = a.idx ? 2u : 1u;
@@ -314,6 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
         tc::mbar_init(p_full, 4);
         tc::mbar_init(o_done, nis);
         tc::mbar_init(fin, 2);
+        tc::mbar_init(xbar, 1);
         tc::fence_mbar_init();
         s_abort = 0;
     }
@@ -342,54 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
             }
             int j = 0;
             if (a.idx) {
-                // Sparse rows: 16-byte cp.async by the whole warp. One warp
-                // instruction moves one 64-dim block (128 B) of four rows, so
-                // every access is a full, aligned 128-byte line; the chunk
-                // lands at its 128-byte-swizzle position. (A TMA gather4 moves
-                // the same 512 B per instruction but its issue rate, not DRAM,
-                // bounded the tile load.) Block b is handed to the MMA once
-                // this warp's copies of it have completed.
-                const int chunk = lane & 7, rsub = lane >> 3;
-                const char* kv_g = (const char*)a.KV;
-                const int64_t row_bytes = (int64_t)a.c * 2;
-                for (; j < ntiles; ++j) {
-                    const int64_t e0 = e_beg + (int64_t)j * kE;
-                    int rows[kE / 4];
-#pragma unroll
-                    for (int i = 0; i < kE / 4; ++i) {
-                        const int64_t e = e0 + 4 * i + rsub;
-                        int s = -1;
-                        if (e < e_end) s = a.idx[(int64_t)t * a.k + e];
-                        if (s < 0 || s >= a.Nmax) s = 0;   // masked in the softmax
-                        rows[i] = (int)(row0 + s);
-                    }
-                    bool ok = true;
-                    for (int b = 0; b < a.dblocks; ++b) {
-                        if (j > 0 && lane == 0) ok = wait_or_abort(&kv_empty[b], (j - 1) & 1, abort_flag, a.status);
-                        ok = __shfl_sync(0xffffffffu, ok, 0);
-                        if (!ok) break;
-                        uint8_t* dst = kv_s + (size_t)b * kE * 128;
-#pragma unroll
-                        for (int i = 0; i < kE / 4; ++i) {
-                            const int r = 4 * i + rsub;
-                            cp_async16(dst + r * 128 + ((chunk ^ (r & 7)) << 4),
-                                       kv_g + (int64_t)rows[i] * row_bytes + b * 128 + chunk * 16);
-                        }
-                        cp_async_commit();
-                    }
-                    // hand the blocks over in order as they complete
-                    const int issued = ok ? a.dblocks : 0;
-                    for (int b = 0; b < issued; ++b) {
-                        cp_async_wait_pending(issued - 1 - b);
-                        tc::fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) tc::mbar_arrive(&kv_full[b]);
-                    }
-                    if (!ok) {
-                        cp_async_wait_pending(0);
-                        break;
-                    }
-                }
+                j = sparse_gather(a, kv_s, kv_full, kv_empty, 0, lane, t, ntiles, e_beg, e_end, row0, abort_flag);
             } else if (lane == 0) {
                 // Dense rows stream through the ring twice per tile, pair by
                 // pair of 64-dim blocks: for the first product (S) through
@@ -404,10 +379,14 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
             if (lane == 0) tc::mbar_wait(q_full, 0, kWaitLimit);
         }
     } else if (warp == 7) {
-        // ---------------------------------------------------------------- dense: O-pass ring
-        if (!a.idx && lane == 0 && ntiles > 0)
+        // ---------------------------------------------------------------- loads: sparse second half, dense O ring
+        if (a.idx) {
+            if (ntiles > 0)
+                sparse_gather(a, kv_s, kv_full, kv_empty, 1, lane, t, ntiles, e_beg, e_end, row0, abort_flag);
+        } else if (lane == 0 && ntiles > 0) {
             dense_ring_load(a, kv_s, &tmTile, kv_full, kv_empty, a.ring / 2, a.ring - a.ring / 2, ntiles,
                             row0 + e_beg, abort_flag);
+        }
     } else if (warp == 1 || warp == 6) {
         // ---------------------------------------------------------------- MMA
         // Two issuing threads (each tcgen05.mma costs its issuer tens of
@@ -669,25 +648,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
             bar_sync_128();
         }
         const bool have_o = ok && ntiles > 0;
-        if (a.cluster) {
-            // stage this split's O^T as obuf[head][dim] (fp32) where the KV
-            // tile was; the combine after the role branches reads it
-            float* obuf = (float*)kv_s;
-            if (eth < 64 && !have_o) { mref_s[eth] = -INFINITY; lsum_s[eth] = 0.f; }
-            if (have_o) {
-                for (int mt = 0; mt < a.mtiles; ++mt) {
-                    const int dim = mt * 128 + row;
-                    float v[64];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        tc::tmem_ld16(tmem_O + ((uint32_t)(quad * 32) << 16) + mt * hg + 16 * u,
-                                      *reinterpret_cast<float(*)[16]>(v + 16 * u));
-                    tc::tmem_ld_wait();
-#pragma unroll
-                    for (int i = 0; i < 64; ++i) obuf[i * a.c + dim] = v[i];
-                }
-            }
-        } else if (a.nsplit == 1) {
+        if (a.nsplit == 1) {
             // normalise: denominator = sum + sink term (same reference max)
             if (eth < 64) {
                 const int h = h0 + eth;
@@ -735,26 +696,59 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
                 *reinterpret_cast<uint4*>(a.out + ((int64_t)t * a.H + h0 + i) * a.c + ch * 8) =
                     *reinterpret_cast<const uint4*>(stage + i * a.c + ch * 8);
             }
+        } else if (a.pair) {
+            // stage O^T as [slice][head][dim in slice] fp32 where the KV tile
+            // was (slice g = the half of the head dimension split g writes
+            // out); the merge after the role branches sends the peer's half
+            if (ntiles > 0) {
+                float* obuf = (float*)kv_s;
+                const int half = a.c / 2;
+                // (a short loop body of 16 columns: code run once per block
+                // is fetched cold, so a compact loop beats a long unrolled one)
+#pragma unroll 1
+                for (int k = 0; k < a.mtiles * 4; ++k) {
+                    const int mt = k >> 2, u = k & 3;
+                    const int dim = mt * 128 + row;
+                    float* dst = obuf + (size_t)(dim / half) * 64 * half + dim % half + (size_t)(16 * u) * half;
+                    float v[16];
+                    tc::tmem_ld16(tmem_O + ((uint32_t)(quad * 32) << 16) + mt * hg + 16 * u, v);
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) dst[i * half] = v[i];
+                }
+                tc::fence_proxy_async_smem();
+            }
         } else {
             if (eth < 64 && h0 + eth < a.H) {
                 float* pm = a.part_ml + (((int64_t)t * a.nsplit + split) * a.H + h0 + eth) * 2;
                 pm[0] = (have_o && mref_s[eth] != -INFINITY) ? mref_s[eth] * 0.6931471805599453f : -INFINITY;
                 pm[1] = have_o ? lsum_s[eth] : 0.f;
             }
-            if (have_o) {
-                for (int mt = 0; mt < a.mtiles; ++mt) {
-                    const int dim = mt * 128 + row;
-                    float v[64];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        tc::tmem_ld16(tmem_O + ((uint32_t)(quad * 32) << 16) + mt * hg + 16 * u,
-                                      *reinterpret_cast<float(*)[16]>(v + 16 * u));
+            if (ntiles > 0) {   // (a block-uniform test: the barrier below takes all four warps)
+                // O^T staged as [head][dim] fp32 where the KV tile was: this
+                // split's heads h0.. are one contiguous block of part_o,
+                // which one thread then writes with bulk copies
+                float* obuf = (float*)kv_s;
+#pragma unroll 1
+                for (int k = 0; k < a.mtiles * 4; ++k) {
+                    const int mt = k >> 2, u = k & 3;
+                    float* dst = obuf + (size_t)(16 * u) * a.c + mt * 128 + row;
+                    float v[16];
+                    tc::tmem_ld16(tmem_O + ((uint32_t)(quad * 32) << 16) + mt * hg + 16 * u, v);
                     tc::tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) {
-                        const int h = h0 + i;
-                        if (h < a.H) a.part_o[(((int64_t)t * a.nsplit + split) * a.H + h) * a.c + dim] = v[i];
-                    }
+                    for (int i = 0; i < 16; ++i) dst[i * a.c] = v[i];
+                }
+                tc::fence_proxy_async_smem();
+                bar_sync_128();
+                if (eth == 0 && have_o) {
+                    const int nh = a.H - h0 < 64 ? a.H - h0 : 64;
+                    const uint32_t bytes = (uint32_t)nh * a.c * 4, chunk = 32768;
+                    char* dst = (char*)(a.part_o + (((int64_t)t * a.nsplit + split) * a.H + h0) * a.c);
+                    for (uint32_t off = 0; off < bytes; off += chunk)
+                        tc::bulk_store(dst + off, (const char*)obuf + off, bytes - off < chunk ? bytes - off : chunk);
+                    tc::bulk_commit();
+                    tc::bulk_wait_all();
                 }
             }
         }
@@ -762,24 +756,18 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
     }
 
     __syncthreads();
+    if (a.pair)
+        pair_merge(a.c, a.H, a.sink, a.lse, a.out, t, h0, (uint32_t)split, ntiles > 0 && !s_abort, (const float*)kv_s,
+                   (float*)q_s, mref_s, lsum_s, xbar, pair_coef, abort_flag, a.status);
     if (warp == 1) {
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, a.tmem_cols);
     }
-    if (a.cluster) {
-        if (a.nsplit <= 2)
-            cluster_merge<2>(a.nsplit, a.c, a.H, a.sink, a.lse, a.out, t, h0, split, (float*)kv_s, mref_s, lsum_s,
-                             merge_coef);
-        else if (a.nsplit <= 4)
-            cluster_merge<4>(a.nsplit, a.c, a.H, a.sink, a.lse, a.out, t, h0, split, (float*)kv_s, mref_s, lsum_s,
-                             merge_coef);
-        else
-            cluster_merge<8>(a.nsplit, a.c, a.H, a.sink, a.lse, a.out, t, h0, split, (float*)kv_s, mref_s, lsum_s,
-                             merge_coef);
-    }
 }
 
 bool mqa_tc_supported(int H, int c) { return c % 128 == 0 && c <= 512 && H >= 1; }
+
+bool mqa_tc_pair(int nsplit) { return nsplit == 2; }
 
 int mqa_tc_nsplit(int nq, int H, int64_t max_entries, int num_sms) {
     const int hgroups = (H + 63) / 64;
@@ -793,44 +781,6 @@ int mqa_tc_nsplit(int nq, int H, int64_t max_entries, int num_sms) {
     // of 64 tiles take 8 tiles each, so 8 splits do the same work)
     if (tiles > 0) ns = (tiles + (tiles + ns - 1) / ns - 1) / ((tiles + ns - 1) / ns);
     return (int)ns;
-}
-
-// Whether the nsplit splits of every (query, head group) run as one cluster
-// and merge on chip: clusters of up to 4 one-CTA-per-SM blocks always; of 5
-// to 8 only when every cluster of the launch can be resident at once (the
-// device's count of such clusters, asked once per cluster size).
-bool mqa_tc_cluster(int nsplit, int nq, int H) {
-    if (nsplit < 2 || nsplit > kMaxClusterSplits) return false;
-    if (nsplit <= 4) return true;
-    static std::mutex mu;
-    static int dev_seen[kMaxClusterSplits + 1][64];   // per (cluster size, device): 0 unknown, else count + 1
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-    std::lock_guard<std::mutex> lock(mu);
-    int& cached = dev_seen[nsplit][dev];
-    if (cached == 0) {
-        int n = 0;
-        if (smem_ceiling(mqa_tc_kernel) == cudaSuccess) {
-            cudaLaunchConfig_t cfg = {};
-            cudaLaunchAttribute attr[1];
-            attr[0].id = cudaLaunchAttributeClusterDimension;
-            attr[0].val.clusterDim.x = (unsigned)nsplit;
-            attr[0].val.clusterDim.y = 1;
-            attr[0].val.clusterDim.z = 1;
-            cfg.gridDim = dim3((unsigned)nsplit, 1, 1);
-            cfg.blockDim = dim3(kThreads);
-            cfg.dynamicSmemBytes = 200 * 1024;   // one CTA per SM, as every launch of this kernel
-            cfg.attrs = attr;
-            cfg.numAttrs = 1;
-            if (cudaOccupancyMaxActiveClusters(&n, mqa_tc_kernel, &cfg) != cudaSuccess) {
-                (void)cudaGetLastError();
-                n = 0;
-            }
-        }
-        cached = n + 1;
-    }
-    const int64_t clusters = (int64_t)nq * ((H + 63) / 64);
-    return clusters <= (int64_t)(cached - 1);
 }
 
 cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, QuerySpec qs, int mp, int nq, int n_seq,
@@ -852,7 +802,7 @@ cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, Que
     a.scale_log2 = scale * 1.4426950408889634f;
     a.sink = sink;
     a.nsplit = nsplit;
-    a.cluster = mqa_tc_cluster(nsplit, nq, H) ? 1 : 0;
+    a.pair = mqa_tc_pair(nsplit) ? 1 : 0;
     const int64_t max_entries = idx ? k : Nmax;
     int64_t per = (max_entries + nsplit - 1) / nsplit;
     a.split_len = ((per + kE - 1) / kE) * kE;
@@ -893,7 +843,7 @@ cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, Que
     cudaError_t le = cudaSuccess;
     CSA_LAUNCH(st, "mqa_tc",
                le = launch_pdl(mqa_tc_kernel, dim3(nsplit, (H + a.hg - 1) / a.hg, nq), dim3(kThreads), smem, st,
-                               a.cluster ? (unsigned)nsplit : 0u, a, tmQ, tmTile));
+                               a.pair ? 2u : 0u, a, tmQ, tmTile));
     if (le != cudaSuccess) return le;
     return cudaGetLastError();
 }

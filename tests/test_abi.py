@@ -205,12 +205,16 @@ def test_workspace_sizes():
     # the selection keeps its scratch in shared memory at every row length
     assert L.csa_topk_workspace_size(64, 16384, 512) == 0
     assert L.csa_topk_workspace_size(32, 262144, 1024) == 0
-    # bf16 MQA: a single split or up to four splits merged in a cluster need
-    # no workspace; more splits keep fp32 partials (O, max, sum) per split
-    assert L.csa_sparse_mqa_workspace_size(64, 64, 512, 512, csa.CSA_BF16) == 0        # 2 splits
+    # bf16 MQA: a single split, or two merged on chip, need no workspace;
+    # more splits keep fp32 partials (O, max, sum) per split for the combine
     assert L.csa_sparse_mqa_workspace_size(4096, 64, 512, 512, csa.CSA_BF16) == 0      # 1 split
-    hca = L.hca_dense_mqa_workspace_size(16, 64, 512, 8192, csa.CSA_BF16)              # 9 splits
-    assert hca >= 16 * 9 * 64 * 512 * 4
+    assert L.csa_sparse_mqa_workspace_size(64, 64, 512, 512, csa.CSA_BF16) == 0        # 2 splits
+    three = L.csa_sparse_mqa_workspace_size(40, 64, 512, 384, csa.CSA_BF16)            # 3 splits
+    assert three >= 40 * 3 * 64 * 512 * 4 + 40 * 3 * 64 * 2 * 4
+    # 148 SMs over 16 queries allow 9 splits; 64 tiles of 128 entries need
+    # only 8 splits of 8 tiles
+    hca = L.hca_dense_mqa_workspace_size(16, 64, 512, 8192, csa.CSA_BF16)
+    assert hca >= 16 * 8 * 64 * 512 * 4
     assert L.csa_decode_workspace_size(64, 32768, 64, 512, 64, 128, 512, csa.CSA_BF16) >= 64 * 32768 * 4
     small = L.csa_prefill_workspace_size(1024, 256, 512, 4, 128, 64, 8, 4, 16, csa.CSA_BF16)
     assert small >= 1024 * 4 * 128 * 4

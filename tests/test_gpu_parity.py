@@ -218,14 +218,13 @@ def test_sparse_mqa(csa, dtype, H, c, k, with_sink):
 
 
 # (kind, queries, head dim, heads, k or visible entries): query counts chosen
-# so that the KV of one query is split 3 ways (merged in a thread-block
-# cluster; 3 does not divide c/4, so the merge slices are uneven), 4, 5, 6 or
-# 8 ways (clusters of up to 8 blocks, merged on chip when all the launch's
-# clusters fit on the device at once, else by the combine launch), or 10 ways
-# (partials merged by the separate combine launch), with one and two head
-# groups. The split count of a launch is the SM count over the (query, head
-# group) blocks, capped by the 128-entry tiles and then reduced to the count
-# the tiles per split need.
+# so that the KV of one query is split 2 ways (the two splits form a cluster
+# and merge on chip) or 3, 4, 5, 6, 8 or 10 ways (every split writes fp32
+# partials, merged in split order by the combine launch), some splits seeing
+# no entry at all, with one and two head groups and head
+# dims of 128 to 512. The split count of a launch is the SM count over the
+# (query, head group) blocks, capped by the 128-entry tiles and then reduced
+# to the count the tiles per split need.
 SPLIT_CASES = [
     ("sparse", 40, 512, 64, 512),
     ("sparse", 40, 128, 64, 384),
@@ -233,13 +232,15 @@ SPLIT_CASES = [
     ("sparse", 20, 256, 64, 1024),     # 4 ways
     ("dense", 40, 512, 64, 700),
     ("dense", 20, 128, 64, 1100),      # 5 ways
-    ("dense", 24, 512, 128, 700),      # two head groups, 3-way cluster
+    ("dense", 24, 512, 128, 700),      # two head groups, 3 ways
     ("dense", 40, 384, 64, 900),       # three 128-dim M tiles through the two rings
     ("sparse", 40, 384, 64, 512),
     ("sparse", 12, 512, 64, 1024),     # 8 ways
     ("sparse", 24, 512, 64, 768),      # 6 ways
     ("dense", 16, 256, 64, 1100),      # 5 ways, one head group
-    ("dense", 8, 512, 64, 1100),       # 10 ways: combine launch
+    ("dense", 8, 512, 64, 1100),       # 10 ways
+    ("dense", 64, 512, 64, 700),       # 2 ways
+    ("dense", 32, 256, 128, 1100),     # two head groups, 2 ways
 ]
 
 
