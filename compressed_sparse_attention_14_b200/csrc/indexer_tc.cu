@@ -452,20 +452,20 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
             }
             if (!wait_or_abort(&sm.tfull[buf], (uint32_t)((it / a.nbuf) & 1), abort_flag, a.status, a.wait_limit)) break;
             tc::tc_fence_after();
+            // sc[hh][q]: the scores of query q of the group; with kN == 256
+            // this set's two queries (2 set, 2 set + 1) sit in sc[hh][0..1]
+            // (the set is a run-time value: indexing by it would put the
+            // array in local memory)
             float sc[kH][4];
 #pragma unroll
             for (int hh = 0; hh < kH; ++hh) {
                 sc[hh][0] = sc[hh][1] = sc[hh][2] = sc[hh][3] = 0.f;
                 const uint32_t taddr =
                     tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)((buf * kH + hh) * a.npad);
-                if constexpr (kN == 256) {
-                    float s2[4] = {0.f, 0.f, 0.f, 0.f};
-                    head_reduce<128, kHI>(taddr + set * 128, wv + set * 128, a.npad, a.HI, a.group, s2);
-                    sc[hh][2 * set] = s2[0];
-                    sc[hh][2 * set + 1] = s2[1];
-                } else {
+                if constexpr (kN == 256)
+                    head_reduce<128, kHI>(taddr + set * 128, wv + set * 128, a.npad, a.HI, a.group, sc[hh]);
+                else
                     head_reduce<kN, kHI>(taddr, wv, a.npad, a.HI, a.group, sc[hh]);
-                }
             }
             tc::tc_fence_before();
             __syncwarp();
@@ -474,11 +474,11 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
             for (int hh = 0; hh < kH; ++hh) {
                 if (key[hh] >= vis) continue;
 #pragma unroll
-                for (int gq = 0; gq < 4; ++gq) {
+                for (int gs = 0; gs < (kN == 256 ? 2 : 4); ++gs) {
+                    const int gq = kN == 256 ? 2 * set + gs : gs;   // query within the group
                     const int tq = wk.g * a.group + gq;
-                    if (kN == 256 && (gq >> 1) != set) continue;
                     if (gq < a.group && tq < a.nq) {
-                        const float v = kFp8 ? sc[hh][gq] * kscale[hh] : sc[hh][gq];
+                        const float v = kFp8 ? sc[hh][gs] * kscale[hh] : sc[hh][gs];
                         if (a.score_bf16)
                             reinterpret_cast<bf16*>(a.scores)[(int64_t)tq * a.ld + key[hh]] = __float2bfloat16_rn(v);
                         else
