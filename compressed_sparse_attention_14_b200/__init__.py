@@ -84,6 +84,13 @@ _SIGS = {
     "hca_compress_step": (_I, [_P, _P, _P, _P, _I, _I, _I, _I64, _P, _I, _P]),
     "csa_decode_compress_workspace_size": (_SZ, [_I, _I, _I]),
     "csa_decode_compress": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I64, _P, _SZ, _I, _P]),
+    "csa_cache_block_layout": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "csa_decode_blocked": (_I, [_P, _P, _P, _P, _P, _P, _I, _I64, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P,
+                                _I, _I64, _P, _SZ, _I, _P]),
+    "hca_decode_blocked": (_I, [_P, _P, _P, _I, _I64, _I, _I, _I, _F, _P, _P, _P, _I, _I64, _P, _SZ, _I, _P]),
+    "csa_decode_compress_blocked": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I64, _I, _I64,
+                                         _P, _SZ, _I, _P]),
+    "hca_compress_step_blocked": (_I, [_P, _P, _P, _P, _I, _I, _I, _I64, _P, _I, _I64, _I, _P]),
     "csa_norm_rope": (_I, [_P, _P, _I64, _I, _I, _P, _F, _I, _F, _P, _I64, _I64, _I, _I, _P]),
     "csa_window_entries": (_I, [_P, _I, _P, _I64, _I, _I, _I64, _I64, _P, _P]),
     "csa_attend_decode_workspace_size": (_SZ, [_I, _I64, _I64, _I, _I, _I, _I, _I, _I, _I]),
@@ -657,3 +664,102 @@ def csa_attend_decode(qI, w, idx_cache, q, kv_cache, ctx_len, m: int, k: int, n_
                                   rope_base, _ptr(sink), _ptr(out), _ptr(lse), _ptr(topk_idx), _ptr(ws), _nbytes(ws),
                                   mode, _stream()))
     return (out, lse, topk_idx) if return_topk else (out, lse)
+
+
+# ---------------------------------------------------------------- cache blocks
+def csa_cache_block_layout(m: int, mp: int, c: int, cI: int, dtype: int = CSA_BF16) -> dict:
+    """The lcm(m, m')-token cache block: rows of each part per block, bytes
+    per block and each part's byte offset within a block."""
+    r1, r2 = ctypes.c_int(0), ctypes.c_int(0)
+    bb, o_kv, o_idx, o_hca = ctypes.c_int64(0), ctypes.c_int64(0), ctypes.c_int64(0), ctypes.c_int64(0)
+    _check(_lib.csa_cache_block_layout(m, mp, c, cI, dtype, ctypes.byref(r1), ctypes.byref(r2), ctypes.byref(bb),
+                                       ctypes.byref(o_kv), ctypes.byref(o_idx), ctypes.byref(o_hca)))
+    return {"csa_rows": r1.value, "hca_rows": r2.value, "block_bytes": bb.value, "kv_offset": o_kv.value,
+            "idx_offset": o_idx.value, "hca_offset": o_hca.value, "m": m, "mp": mp, "c": c, "cI": cI}
+
+
+def _blocks_check(blocks, layout, B):
+    if blocks.dtype != torch.uint8 or blocks.dim() != 3 or blocks.shape[0] != B or \
+            blocks.shape[2] != layout["block_bytes"] or not blocks.is_contiguous():
+        raise ValueError(f"blocks must be a contiguous uint8 tensor [B={B}, nblocks, {layout['block_bytes']}], "
+                         f"got {tuple(blocks.shape)} {blocks.dtype}")
+    return blocks.shape[1]
+
+
+def csa_decode_blocked(qI, w, q, blocks, layout, ctx_len, k: int, scale: float = 0.0, sink=None, out=None, lse=None,
+                       topk_idx=None, ws=None, return_topk: bool = False):
+    """csa_decode over block caches: blocks [B, nblocks, block_bytes] uint8
+    in the layout of csa_cache_block_layout (bf16 entries)."""
+    B, HI, cI = qI.shape
+    _, H, c = q.shape
+    nblk = _blocks_check(blocks, layout, B)
+    if c != layout["c"] or cI != layout["cI"]:
+        raise ValueError(f"layout is for c={layout['c']}, cI={layout['cI']}; q has c={c}, qI has cI={cI}")
+    rpb, m = layout["csa_rows"], layout["m"]
+    Nmax = nblk * rpb
+    out = torch.empty_like(q) if out is None else out
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    if return_topk and topk_idx is None:
+        topk_idx = torch.empty((B, k), dtype=torch.int32, device=q.device)
+    mode = _mode(q)
+    ws = _ws(csa_decode_workspace_size(B, Nmax, H, c, HI, cI, k, mode), q.device, ws)
+    base = blocks.data_ptr()
+    _check(_lib.csa_decode_blocked(_ptr(qI), _ptr(w), base + layout["idx_offset"], _ptr(q), base + layout["kv_offset"],
+                                   _ptr(ctx_len), B, Nmax, m, H, c, HI, cI, k, scale, _ptr(sink), _ptr(out),
+                                   _ptr(lse), _ptr(topk_idx), rpb, layout["block_bytes"], _ptr(ws), _nbytes(ws), mode,
+                                   _stream()))
+    return (out, lse, topk_idx) if return_topk else (out, lse)
+
+
+def hca_decode_blocked(q, blocks, layout, ctx_len, scale: float = 0.0, sink=None, out=None, lse=None, ws=None):
+    """hca_decode over the HCA part of block caches (one entry per block)."""
+    B, H, c = q.shape
+    nblk = _blocks_check(blocks, layout, B)
+    rpb = layout["hca_rows"]
+    Nmax = nblk * rpb
+    out = torch.empty_like(q) if out is None else out
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    mode = _mode(q)
+    ws = _ws(_lib.hca_decode_workspace_size(B, Nmax, H, c, mode), q.device, ws)
+    _check(_lib.hca_decode_blocked(_ptr(q), blocks.data_ptr() + layout["hca_offset"], _ptr(ctx_len), B, Nmax,
+                                   layout["mp"], H, c, scale, _ptr(sink), _ptr(out), _ptr(lse), rpb,
+                                   layout["block_bytes"], _ptr(ws), _nbytes(ws), mode, _stream()))
+    return out, lse
+
+
+def csa_decode_compress_blocked(x_new, W_kv, B_kv, W_idx, B_idx, pos, state_kv, state_idx, blocks, layout, ws=None):
+    """csa_decode_compress writing the entries into block caches."""
+    B, d = x_new.shape
+    c, cI, m = layout["c"], layout["cI"], layout["m"]
+    nblk = _blocks_check(blocks, layout, B)
+    rpb = layout["csa_rows"]
+    _shape(W_kv, (4 * c, d), "W_kv")
+    _shape(W_idx, (4 * cI, d), "W_idx")
+    _shape(B_kv, (2 * m, c), "B_kv")
+    _shape(B_idx, (2 * m, cI), "B_idx")
+    _shape(pos, (B,), "pos")
+    _shape(state_kv, (B, 2 * m, 4 * c), "state_kv")
+    _shape(state_idx, (B, 2 * m, 4 * cI), "state_idx")
+    ws = _ws(_lib.csa_decode_compress_workspace_size(B, c, cI), x_new.device, ws)
+    base = blocks.data_ptr()
+    _check(_lib.csa_decode_compress_blocked(_ptr(x_new), _ptr(W_kv), _ptr(B_kv), _ptr(W_idx), _ptr(B_idx), _ptr(pos),
+                                            B, d, m, c, cI, _ptr(state_kv), _ptr(state_idx),
+                                            base + layout["kv_offset"], base + layout["idx_offset"], nblk * rpb, rpb,
+                                            layout["block_bytes"], _ptr(ws), _nbytes(ws), _mode(x_new), _stream()))
+
+
+def hca_compress_step_blocked(proj_new, state, bias, pos, blocks, layout):
+    """hca_compress_step writing the entries into the HCA part of block caches."""
+    B, c2 = proj_new.shape
+    c, mp = layout["c"], layout["mp"]
+    nblk = _blocks_check(blocks, layout, B)
+    _shape(proj_new, (B, 2 * c), "proj_new")
+    _shape(state, (B, mp, 2 * c), "state")
+    _shape(bias, (mp, c), "bias")
+    _shape(pos, (B,), "pos")
+    rpb = layout["hca_rows"]
+    _check(_lib.hca_compress_step_blocked(_ptr(proj_new), _ptr(state), _ptr(bias), _ptr(pos), B, c, mp, nblk * rpb,
+                                          blocks.data_ptr() + layout["hca_offset"], rpb, layout["block_bytes"],
+                                          CSA_BF16, _stream()))

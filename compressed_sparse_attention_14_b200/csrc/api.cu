@@ -136,10 +136,10 @@ static int check_k(int k) {
 // Indexer of the mode: tcgen05 kernel for bf16, FFMA kernel for fp32.
 static cudaError_t run_indexer(const void* qI, const float* w, const void* K, QuerySpec qs, int nq, int n_seq,
                                int HI, int cI, int64_t Nmax, int m, float* scores, int64_t ld, int group,
-                               bool fill_invisible, ElemType t, cudaStream_t st) {
+                               bool fill_invisible, ElemType t, cudaStream_t st, RowBlocks kb = RowBlocks{0, 0}) {
     if (t == ElemType::BF16)
         return index_scores_tc(qI, w, K, qs, nq, n_seq, HI, cI, Nmax, m, scores, ld, group, fill_invisible,
-                               device_status(), st);
+                               device_status(), st, nullptr, false, kb);
     return index_scores(qI, w, K, qs, nq, n_seq, HI, cI, Nmax, m, scores, ld, t, st);
 }
 
@@ -258,7 +258,7 @@ int hca_compress(const void* proj, const float* bias, int64_t n, int c, int mp, 
 
 static int compress_step_common(const float* proj_new, float* state, const float* bias, const int32_t* pos, int B,
                                 int c, int m, int mmax, int64_t Nmax, void* cache, int dtype, bool overlap,
-                                void* stream, const char* who) {
+                                void* stream, const char* who, RowBlocks cb = RowBlocks{0, 0}) {
     ElemType t = ElemType::BF16;   // set by check_dtype
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_compress(0, c, m, mmax, who));
@@ -269,7 +269,8 @@ static int compress_step_common(const float* proj_new, float* state, const float
     CSA_TRY(check_ptr(bias, "bias"));
     CSA_TRY(check_ptr(pos, "pos"));
     CSA_TRY(check_ptr(cache, "cache", Nmax > 0));
-    CSA_CUDA(compress_step(proj_new, state, bias, pos, B, c, m, overlap, Nmax, cache, t, (cudaStream_t)stream), who);
+    CSA_CUDA(compress_step(proj_new, state, bias, pos, B, c, m, overlap, Nmax, cache, t, (cudaStream_t)stream, 1, cb),
+             who);
     return CSA_OK;
 }
 
@@ -283,6 +284,54 @@ int hca_compress_step(const float* proj_new, float* state, const float* bias, co
                       int mp, int64_t Nmax, void* cache, int dtype, void* stream) {
     return compress_step_common(proj_new, state, bias, pos, B, c, mp, 1024, Nmax, cache, dtype, false, stream,
                                 "hca_compress_step");
+}
+
+// ---------------------------------------------------------------- cache blocks
+static int64_t gcd64(int64_t a, int64_t b) { return b ? gcd64(b, a % b) : a; }
+
+int csa_cache_block_layout(int m, int mp, int c, int cI, int dtype, int* csa_rows, int* hca_rows,
+                           int64_t* block_bytes, int64_t* kv_offset, int64_t* idx_offset, int64_t* hca_offset) {
+    ElemType t = ElemType::BF16;   // set by check_dtype
+    CSA_TRY(check_dtype(dtype, &t));
+    if (m < 1 || mp < 1 || c < 8 || cI < 8 || c % 8 || cI % 8)
+        return fail(CSA_ERR_INVALID_ARG, "csa_cache_block_layout: m=%d mp=%d c=%d cI=%d", m, mp, c, cI);
+    CSA_TRY(check_ptr(csa_rows, "csa_rows"));
+    CSA_TRY(check_ptr(hca_rows, "hca_rows"));
+    CSA_TRY(check_ptr(block_bytes, "block_bytes"));
+    const int64_t L = (int64_t)m / gcd64(m, mp) * mp;   // lcm(m, m')
+    if (L > (1 << 20)) return fail(CSA_ERR_UNSUPPORTED, "csa_cache_block_layout: lcm(m, m') = %lld", (long long)L);
+    const int64_t es = t == ElemType::BF16 ? 2 : 4;
+    const int64_t r1 = L / m, r2 = L / mp;
+    *csa_rows = (int)r1;
+    *hca_rows = (int)r2;
+    const int64_t kv = 0, idx = kv + r1 * c * es, hca = idx + r1 * cI * es;
+    *block_bytes = hca + r2 * c * es;   // a multiple of 16: c and cI are multiples of 8
+    if (kv_offset) *kv_offset = kv;
+    if (idx_offset) *idx_offset = idx;
+    if (hca_offset) *hca_offset = hca;
+    return CSA_OK;
+}
+
+// the blocked calls: bf16 caches, rows in blocks of rpb (dividing Nmax),
+// blocks 16-byte aligned and at least rpb rows of `width` long
+static int check_blocks(int rpb, int64_t block_bytes, int64_t Nmax, int width, const void* base, int dtype,
+                        const char* who) {
+    if (dtype != CSA_BF16) return fail(CSA_ERR_UNSUPPORTED, "%s: bf16 caches only", who);
+    if (rpb < 1 || block_bytes % 16 || block_bytes < (int64_t)rpb * width * 2)
+        return fail(CSA_ERR_INVALID_ARG, "%s: rows_per_block=%d block_bytes=%lld (a multiple of 16 holding %d rows of "
+                    "%d bf16)", who, rpb, (long long)block_bytes, rpb, width);
+    if (Nmax % rpb) return fail(CSA_ERR_INVALID_ARG, "%s: Nmax=%lld is not a multiple of rows_per_block=%d", who,
+                                (long long)Nmax, rpb);
+    if (base && ((uintptr_t)base & 15)) return fail(CSA_ERR_INVALID_ARG, "%s: cache pointer not 16-byte aligned", who);
+    return CSA_OK;
+}
+
+int hca_compress_step_blocked(const float* proj_new, float* state, const float* bias, const int32_t* pos, int B,
+                              int c, int mp, int64_t Nmax, void* cache, int rows_per_block, int64_t block_bytes,
+                              int dtype, void* stream) {
+    CSA_TRY(check_blocks(rows_per_block, block_bytes, Nmax, c, cache, dtype, "hca_compress_step_blocked"));
+    return compress_step_common(proj_new, state, bias, pos, B, c, mp, 1024, Nmax, cache, dtype, false, stream,
+                                "hca_compress_step_blocked", RowBlocks{rows_per_block, block_bytes});
 }
 
 static int compress_chunk_common(const float* proj, float* state, const float* bias, int64_t start, int64_t n, int c,
@@ -325,10 +374,10 @@ size_t csa_decode_compress_workspace_size(int B, int c, int cI) {
     return align256((size_t)64 * B * 4 * c * sizeof(float)) + align256((size_t)64 * B * 4 * cI * sizeof(float));
 }
 
-int csa_decode_compress(const void* x_new, const void* W_kv, const float* B_kv, const void* W_idx, const float* B_idx,
-                        const int32_t* pos, int B, int d, int m, int c, int cI, float* state_kv, float* state_idx,
-                        void* kv_cache, void* idx_cache, int64_t Nmax, void* ws, size_t ws_bytes, int dtype,
-                        void* stream) {
+static int decode_compress_impl(const void* x_new, const void* W_kv, const float* B_kv, const void* W_idx,
+                                const float* B_idx, const int32_t* pos, int B, int d, int m, int c, int cI,
+                                float* state_kv, float* state_idx, void* kv_cache, void* idx_cache, int64_t Nmax,
+                                void* ws, size_t ws_bytes, int dtype, void* stream, RowBlocks cb) {
     ElemType t = ElemType::BF16;   // set by check_dtype
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_compress(0, c, m, 64, "csa_decode_compress"));
@@ -363,10 +412,29 @@ int csa_decode_compress(const void* x_new, const void* W_kv, const float* B_kv, 
         CSA_CUDA(project(x_new, W_kv, B, d, 4 * c, pk, t, st), "csa_decode_compress: KV projection");
         CSA_CUDA(project(x_new, W_idx, B, d, 4 * cI, pi, t, st), "csa_decode_compress: index-key projection");
     }
-    const StepStream skv{pk, state_kv, B_kv, kv_cache, c, ks_kv, (int64_t)B * 4 * c};
-    const StepStream sidx{pi, state_idx, B_idx, idx_cache, cI, ks_idx, (int64_t)B * 4 * cI};
+    const StepStream skv{pk, state_kv, B_kv, kv_cache, c, ks_kv, (int64_t)B * 4 * c, cb};
+    const StepStream sidx{pi, state_idx, B_idx, idx_cache, cI, ks_idx, (int64_t)B * 4 * cI, cb};
     CSA_CUDA(compress_step_csa2(skv, sidx, pos, B, m, Nmax, t, st), "csa_decode_compress: compressors");
     return CSA_OK;
+}
+
+int csa_decode_compress(const void* x_new, const void* W_kv, const float* B_kv, const void* W_idx, const float* B_idx,
+                        const int32_t* pos, int B, int d, int m, int c, int cI, float* state_kv, float* state_idx,
+                        void* kv_cache, void* idx_cache, int64_t Nmax, void* ws, size_t ws_bytes, int dtype,
+                        void* stream) {
+    return decode_compress_impl(x_new, W_kv, B_kv, W_idx, B_idx, pos, B, d, m, c, cI, state_kv, state_idx, kv_cache,
+                                idx_cache, Nmax, ws, ws_bytes, dtype, stream, RowBlocks{0, 0});
+}
+
+int csa_decode_compress_blocked(const void* x_new, const void* W_kv, const float* B_kv, const void* W_idx,
+                                const float* B_idx, const int32_t* pos, int B, int d, int m, int c, int cI,
+                                float* state_kv, float* state_idx, void* kv_cache, void* idx_cache, int64_t Nmax,
+                                int rows_per_block, int64_t block_bytes, void* ws, size_t ws_bytes, int dtype,
+                                void* stream) {
+    CSA_TRY(check_blocks(rows_per_block, block_bytes, Nmax, c, kv_cache, dtype, "csa_decode_compress_blocked"));
+    CSA_TRY(check_blocks(rows_per_block, block_bytes, Nmax, cI, idx_cache, dtype, "csa_decode_compress_blocked"));
+    return decode_compress_impl(x_new, W_kv, B_kv, W_idx, B_idx, pos, B, d, m, c, cI, state_kv, state_idx, kv_cache,
+                                idx_cache, Nmax, ws, ws_bytes, dtype, stream, RowBlocks{rows_per_block, block_bytes});
 }
 
 size_t csa_compress_from_hidden_workspace_size(int64_t n, int d, int c, int m, int dtype) {
@@ -678,9 +746,10 @@ size_t hca_dense_mqa_workspace_size(int nq, int H, int c, int64_t Nmax, int dtyp
     return mqa_workspace_bytes(nq, H, c, Nmax, t);
 }
 
-int hca_dense_mqa(const void* q, const void* KV, const int32_t* pos, const int32_t* seq_of_q,
-                  int nq, int n_seq, int H, int c, int64_t Nmax, int mp, float scale, const float* sink,
-                  void* out, float* lse, void* ws, size_t ws_bytes, int dtype, void* stream) {
+static int hca_dense_mqa_impl(const void* q, const void* KV, const int32_t* pos, const int32_t* seq_of_q,
+                              int nq, int n_seq, int H, int c, int64_t Nmax, int mp, float scale, const float* sink,
+                              void* out, float* lse, void* ws, size_t ws_bytes, int dtype, void* stream,
+                              RowBlocks kvb) {
     ElemType t = ElemType::BF16;   // set by check_dtype
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_attn_shape(H, c));
@@ -701,8 +770,15 @@ int hca_dense_mqa(const void* q, const void* KV, const int32_t* pos, const int32
     CSA_TRY(check_ws(ws, ws_bytes, mqa_workspace_bytes(nq, H, c, Nmax, t)));
     QuerySpec qs{seq_of_q, pos, 0, 0};
     CSA_CUDA(mqa(q, KV, nullptr, 0, qs, mp, nq, n_seq, H, c, Nmax, default_scale(scale, c), sink, out, lse, ws,
-                 t, (cudaStream_t)stream), "hca_dense_mqa");
+                 t, (cudaStream_t)stream, kvb), "hca_dense_mqa");
     return CSA_OK;
+}
+
+int hca_dense_mqa(const void* q, const void* KV, const int32_t* pos, const int32_t* seq_of_q,
+                  int nq, int n_seq, int H, int c, int64_t Nmax, int mp, float scale, const float* sink,
+                  void* out, float* lse, void* ws, size_t ws_bytes, int dtype, void* stream) {
+    return hca_dense_mqa_impl(q, KV, pos, seq_of_q, nq, n_seq, H, c, Nmax, mp, scale, sink, out, lse, ws, ws_bytes,
+                              dtype, stream, RowBlocks{0, 0});
 }
 
 // ---------------------------------------------------------------- fused
@@ -714,10 +790,10 @@ size_t csa_decode_workspace_size(int B, int64_t Nmax, int H, int c, int HI, int 
            mqa_workspace_bytes(B, H, c, k, t);
 }
 
-int csa_decode(const void* qI, const float* w, const void* idx_cache, const void* q,
-               const void* kv_cache, const int32_t* ctx_len, int B, int64_t Nmax, int m, int H,
-               int c, int HI, int cI, int k, float scale, const float* sink, void* out, float* lse,
-               int32_t* topk_idx, void* ws, size_t ws_bytes, int dtype, void* stream) {
+static int csa_decode_impl(const void* qI, const float* w, const void* idx_cache, const void* q,
+                           const void* kv_cache, const int32_t* ctx_len, int B, int64_t Nmax, int m, int H,
+                           int c, int HI, int cI, int k, float scale, const float* sink, void* out, float* lse,
+                           int32_t* topk_idx, void* ws, size_t ws_bytes, int dtype, void* stream, RowBlocks cb) {
     ElemType t = ElemType::BF16;   // set by check_dtype
     CSA_TRY(check_dtype(dtype, &t));
     CSA_TRY(check_index_shape(HI, cI));
@@ -749,11 +825,34 @@ int csa_decode(const void* qI, const float* w, const void* idx_cache, const void
     void* mws = cv.take(mqa_workspace_bytes(B, H, c, k, t));
     if (topk_idx) sel = topk_idx;
     QuerySpec qs{nullptr, ctx_len, 0, 0};
-    CSA_CUDA(run_indexer(qI, w, idx_cache, qs, B, B, HI, cI, Nmax, m, sc, Nmax, 1, false, t, st), "csa_decode: indexer");
+    CSA_CUDA(run_indexer(qI, w, idx_cache, qs, B, B, HI, cI, Nmax, m, sc, Nmax, 1, false, t, st, cb),
+             "csa_decode: indexer");
     CSA_CUDA(topk_select(sc, Nmax, ctx_len, m, B, Nmax, k, sel, nullptr, tws, st), "csa_decode: top-k");
-    CSA_CUDA(mqa(q, kv_cache, sel, k, qs, 1, B, B, H, c, Nmax, default_scale(scale, c), sink, out, lse, mws, t, st),
+    CSA_CUDA(mqa(q, kv_cache, sel, k, qs, 1, B, B, H, c, Nmax, default_scale(scale, c), sink, out, lse, mws, t, st,
+                 cb),
              "csa_decode: mqa");
     return CSA_OK;
+}
+
+int csa_decode(const void* qI, const float* w, const void* idx_cache, const void* q,
+               const void* kv_cache, const int32_t* ctx_len, int B, int64_t Nmax, int m, int H,
+               int c, int HI, int cI, int k, float scale, const float* sink, void* out, float* lse,
+               int32_t* topk_idx, void* ws, size_t ws_bytes, int dtype, void* stream) {
+    return csa_decode_impl(qI, w, idx_cache, q, kv_cache, ctx_len, B, Nmax, m, H, c, HI, cI, k, scale, sink, out, lse,
+                           topk_idx, ws, ws_bytes, dtype, stream, RowBlocks{0, 0});
+}
+
+int csa_decode_blocked(const void* qI, const float* w, const void* idx_cache, const void* q, const void* kv_cache,
+                       const int32_t* ctx_len, int B, int64_t Nmax, int m, int H, int c, int HI, int cI, int k,
+                       float scale, const float* sink, void* out, float* lse, int32_t* topk_idx, int rows_per_block,
+                       int64_t block_bytes, void* ws, size_t ws_bytes, int dtype, void* stream) {
+    CSA_TRY(check_blocks(rows_per_block, block_bytes, Nmax, c, kv_cache, dtype, "csa_decode_blocked"));
+    CSA_TRY(check_blocks(rows_per_block, block_bytes, Nmax, cI, idx_cache, dtype, "csa_decode_blocked"));
+    if (128 % rows_per_block)
+        return fail(CSA_ERR_UNSUPPORTED, "csa_decode_blocked: rows_per_block=%d must divide the indexer's 128-key tile",
+                    rows_per_block);
+    return csa_decode_impl(qI, w, idx_cache, q, kv_cache, ctx_len, B, Nmax, m, H, c, HI, cI, k, scale, sink, out, lse,
+                           topk_idx, ws, ws_bytes, dtype, stream, RowBlocks{rows_per_block, block_bytes});
 }
 
 size_t hca_decode_workspace_size(int B, int64_t Nmax, int H, int c, int dtype) {
@@ -765,6 +864,17 @@ int hca_decode(const void* q, const void* kv_cache, const int32_t* ctx_len, int 
                void* ws, size_t ws_bytes, int dtype, void* stream) {
     return hca_dense_mqa(q, kv_cache, ctx_len, nullptr, B, B, H, c, Nmax, mp, scale, sink, out, lse, ws,
                          ws_bytes, dtype, stream);
+}
+
+int hca_decode_blocked(const void* q, const void* kv_cache, const int32_t* ctx_len, int B, int64_t Nmax, int mp,
+                       int H, int c, float scale, const float* sink, void* out, float* lse, int rows_per_block,
+                       int64_t block_bytes, void* ws, size_t ws_bytes, int dtype, void* stream) {
+    CSA_TRY(check_blocks(rows_per_block, block_bytes, Nmax, c, kv_cache, dtype, "hca_decode_blocked"));
+    if (rows_per_block != 1)
+        return fail(CSA_ERR_UNSUPPORTED, "hca_decode_blocked: one HCA entry per block (rows_per_block=%d)",
+                    rows_per_block);
+    return hca_dense_mqa_impl(q, kv_cache, ctx_len, nullptr, B, B, H, c, Nmax, mp, scale, sink, out, lse, ws, ws_bytes,
+                              dtype, stream, RowBlocks{rows_per_block, block_bytes});
 }
 
 size_t csa_prefill_workspace_size(int64_t n, int64_t Nmax, int d, int m, int c, int cI, int H,

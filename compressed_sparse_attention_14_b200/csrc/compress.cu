@@ -223,7 +223,9 @@ __global__ void __launch_bounds__(128) csa_compress_step_kernel(const StepStream
     float o[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) o[u] = sm.acc[u] / sm.den[u];
-    TOut* out = reinterpret_cast<TOut*>(second ? s1.cache : s0.cache) + ((int64_t)b * Nmax + i) * c + j;
+    TOut* out = reinterpret_cast<TOut*>(static_cast<char*>(second ? s1.cache : s0.cache) +
+                                        row_byte_offset((int64_t)b * Nmax + i, (int64_t)c * sizeof(TOut),
+                                                        second ? s1.cb : s0.cb)) + j;
     if constexpr (sizeof(TOut) == 2) store8(reinterpret_cast<bf16*>(out), o);
     else store8(reinterpret_cast<float*>(out), o);
 }
@@ -236,7 +238,7 @@ __global__ void __launch_bounds__(256) hca_compress_step_kernel(const float* __r
                                                                 const float* __restrict__ bias,
                                                                 const int32_t* __restrict__ pos, int B, int c,
                                                                 int mp, int64_t Nmax, TOut* __restrict__ cache,
-                                                                int nsplit, int64_t pstride) {
+                                                                int nsplit, int64_t pstride, RowBlocks cb) {
     pdl_wait();
     pdl_launch_next();
     const int groups = c / 8;
@@ -278,7 +280,8 @@ __global__ void __launch_bounds__(256) hca_compress_step_kernel(const float* __r
     float o[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) o[u] = sm.acc[u] / sm.den[u];
-    TOut* out = cache + ((int64_t)b * Nmax + i) * c + j;
+    TOut* out = reinterpret_cast<TOut*>(reinterpret_cast<char*>(cache) +
+                                        row_byte_offset((int64_t)b * Nmax + i, (int64_t)c * sizeof(TOut), cb)) + j;
     if constexpr (sizeof(TOut) == 2) store8(reinterpret_cast<bf16*>(out), o);
     else store8(reinterpret_cast<float*>(out), o);
 }
@@ -443,9 +446,10 @@ cudaError_t compress_hca(const void* proj, const float* bias, int64_t n, int c, 
 }
 
 cudaError_t compress_step(const float* proj_new, float* state, const float* bias, const int32_t* pos, int B, int c,
-                          int m, bool overlap, int64_t Nmax, void* cache, ElemType out_t, cudaStream_t st, int nsplit) {
+                          int m, bool overlap, int64_t Nmax, void* cache, ElemType out_t, cudaStream_t st, int nsplit,
+                          RowBlocks cb) {
     if (overlap) {
-        StepStream s{proj_new, state, bias, cache, c, nsplit, (int64_t)B * 4 * c};
+        StepStream s{proj_new, state, bias, cache, c, nsplit, (int64_t)B * 4 * c, cb};
         StepStream none{};
         return compress_step_csa2(s, none, pos, B, m, Nmax, out_t, st);
     }
@@ -457,11 +461,11 @@ cudaError_t compress_step(const float* proj_new, float* state, const float* bias
     if (out_t == ElemType::BF16)
         CSA_LAUNCH(st, "hca_compress_step",
                    e = launch_pdl(hca_compress_step_kernel<bf16>, grid, dim3(256), 0, st, 0, proj_new, state, bias,
-                                  pos, B, c, m, Nmax, (bf16*)cache, nsplit, pstride));
+                                  pos, B, c, m, Nmax, (bf16*)cache, nsplit, pstride, cb));
     else
         CSA_LAUNCH(st, "hca_compress_step",
                    e = launch_pdl(hca_compress_step_kernel<float>, grid, dim3(256), 0, st, 0, proj_new, state, bias,
-                                  pos, B, c, m, Nmax, (float*)cache, nsplit, pstride));
+                                  pos, B, c, m, Nmax, (float*)cache, nsplit, pstride, cb));
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

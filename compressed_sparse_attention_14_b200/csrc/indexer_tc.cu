@@ -67,6 +67,7 @@ struct IdxArgs {
     const float* w;     // [nq][HI] (FP8: w times the query-head scale)
     const float* kscale;    // FP8: [n_seq * Nmax] key scales; nullptr for bf16
     int blk_elems;      // elements per 128-byte row of a tile (64 bf16, 128 e4m3)
+    int key_rpb;        // keys in blocks of key_rpb rows (a 3D key map); 0: contiguous rows
     float* scores;      // [nq][ld] fp32, or bf16 values when score_bf16
     int score_bf16;
     int64_t ld;
@@ -337,8 +338,12 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
 #pragma unroll
                     for (int hh = 0; hh < kH; ++hh)
                         for (int kb = 0; kb < a.kblocks; ++kb)
-                            tc::tma_load_2d(dst + (size_t)(hh * a.kblocks + kb) * kKeys * 128, &tmK, &sm.full[s],
-                                            kb * a.blk_elems, row + hh * kKeys);
+                            if (a.key_rpb)   // kKeys / key_rpb blocks of key_rpb rows
+                                tc::tma_load_3d(dst + (size_t)(hh * a.kblocks + kb) * kKeys * 128, &tmK, &sm.full[s],
+                                                kb * a.blk_elems, 0, (row + hh * kKeys) / a.key_rpb);
+                            else
+                                tc::tma_load_2d(dst + (size_t)(hh * a.kblocks + kb) * kKeys * 128, &tmK, &sm.full[s],
+                                                kb * a.blk_elems, row + hh * kKeys);
                 }
                 wk.next(a, ngroups);
             }
@@ -530,9 +535,11 @@ bool index_tc_supported(int HI, int cI, int group, bool fp8) {
 
 cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, QuerySpec qs, int nq, int n_seq, int HI,
                             int cI, int64_t Nmax, int m, float* scores, int64_t ld, int group, bool fill_invisible,
-                            int* status, cudaStream_t st, const float* kscale, bool score_bf16) {
+                            int* status, cudaStream_t st, const float* kscale, bool score_bf16, RowBlocks kb) {
     if (score_bf16 && fill_invisible) return cudaErrorInvalidValue;
     const bool fp8 = kscale != nullptr;
+    // keys in blocks: bf16 only, whole blocks per 128-key tile and per sequence
+    if (kb.rpb > 0 && (fp8 || kKeys % kb.rpb || Nmax % kb.rpb || kb.block_bytes % 16)) return cudaErrorInvalidValue;
     const int es = fp8 ? 1 : 2;
     if (nq == 0 || Nmax == 0) return cudaSuccess;
     IdxArgs a{};
@@ -581,7 +588,14 @@ cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, Query
         if (!make_tmap_u8_2d(&tmK, K, (uint64_t)n_seq * Nmax, cI, cI, kKeys, 128)) return cudaErrorInvalidValue;
         if (!make_tmap_u8_2d(&tmQ, qI, (uint64_t)nq * HI, cI, cI, a.npad, 128)) return cudaErrorInvalidValue;
     } else {
-        if (!make_tmap_bf16_2d(&tmK, K, (uint64_t)n_seq * Nmax, cI, cI, kKeys, 64)) return cudaErrorInvalidValue;
+        if (kb.rpb > 0) {
+            a.key_rpb = kb.rpb;
+            if (!make_tmap_bf16_blocks(&tmK, K, (uint64_t)n_seq * Nmax / kb.rpb, (uint32_t)kb.rpb, cI,
+                                       (uint64_t)kb.block_bytes, (uint32_t)(kKeys / kb.rpb), 64))
+                return cudaErrorInvalidValue;
+        } else if (!make_tmap_bf16_2d(&tmK, K, (uint64_t)n_seq * Nmax, cI, cI, kKeys, 64)) {
+            return cudaErrorInvalidValue;
+        }
         if (!make_tmap_bf16_2d(&tmQ, qI, (uint64_t)nq * HI, cI, cI, a.npad, 64)) return cudaErrorInvalidValue;
     }
 

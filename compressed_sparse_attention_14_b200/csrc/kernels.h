@@ -79,6 +79,18 @@ struct QuerySpec {
     int single_seq;
 };
 
+// Where row R of a cache lives (R = sequence * Nmax + entry). rpb == 0: a
+// contiguous [rows, width] matrix. rpb > 0: rows come in blocks of rpb, block
+// j at j * block_bytes from the cache pointer (the other parts of a block,
+// such as the other cache types of the same raw tokens, lie between them).
+struct RowBlocks {
+    int rpb;
+    int64_t block_bytes;
+};
+__host__ __device__ __forceinline__ int64_t row_byte_offset(int64_t R, int64_t row_bytes, RowBlocks L) {
+    return L.rpb ? (R / L.rpb) * L.block_bytes + (R % L.rpb) * row_bytes : R * row_bytes;
+}
+
 // api.cu: record the thread's last error message (csa_last_error) and
 // return `code`.
 int set_last_error(int code, const char* fmt, ...);
@@ -96,7 +108,7 @@ cudaError_t compress_hca(const void* proj, const float* bias, int64_t n, int c, 
 // width), added in slice order.
 cudaError_t compress_step(const float* proj_new, float* state, const float* bias, const int32_t* pos, int B, int c,
                           int m, bool overlap, int64_t Nmax, void* cache, ElemType out_t, cudaStream_t st,
-                          int nsplit = 1);
+                          int nsplit = 1, RowBlocks cb = RowBlocks{0, 0});
 // One CSA compressor stream of a decode step: proj holds nsplit partial sums
 // [B, 4c] fp32, slice s at proj + s * pstride; state [B, 2m, 4c]; bias [2m, c];
 // cache [B, Nmax, c] of the output type.
@@ -107,6 +119,7 @@ struct StepStream {
     void* cache;
     int c, nsplit;
     int64_t pstride;
+    RowBlocks cb;   // where the cache's entry rows live
 };
 // both CSA streams of a decode step (same m, positions and output type) in
 // one launch; s1.c == 0 leaves the second out
@@ -151,10 +164,12 @@ cudaError_t index_scores(const void* qI, const float* w, const void* K, QuerySpe
 // score_bf16: scores are stored as bf16 (nearest, ties to even), row stride
 // ld bf16 values (no fill_invisible).
 bool index_tc_supported(int HI, int cI, int group, bool fp8 = false);
+// K in blocks (kb.rpb > 0; bf16 keys only): rpb must divide the 128-key tile
+// and Nmax.
 cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, QuerySpec qs, int nq, int n_seq, int HI,
                             int cI, int64_t Nmax, int m, float* scores, int64_t ld, int group, bool fill_invisible,
                             int* status, cudaStream_t st, const float* kscale = nullptr,
-                            bool score_bf16 = false);
+                            bool score_bf16 = false, RowBlocks kb = RowBlocks{0, 0});
 
 // quant.cu: row-wise e4m3 codes out [rows, cols] and fp32 scales
 // s = max|row| / 448 (1 for a zero row), decided in fp64; w_out = w * s when
@@ -184,15 +199,18 @@ bool mqa_tc_supported(int H, int c);
 int mqa_tc_nsplit(int nq, int H, int64_t max_entries, int num_sms);
 // two splits run as a cluster of two and merge on chip (no workspace, no combine launch)
 bool mqa_tc_pair(int nsplit);
+// KV in blocks (kvb.rpb > 0): any rpb dividing Nmax for the sparse path, rpb
+// == 1 for the dense one (its rows are read by TMA with the block as the row
+// pitch).
 cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, QuerySpec qs, int mp, int nq, int n_seq,
                    int H, int c, int64_t Nmax, float scale, const float* sink, void* out, float* lse, void* ws,
-                   int nsplit, int* status, cudaStream_t st);
+                   int nsplit, int* status, cudaStream_t st, RowBlocks kvb = RowBlocks{0, 0});
 
 // mqa.cu: sparse (idx != nullptr) or dense (entries s < pos/mp) shared-KV MQA
 size_t mqa_workspace_bytes(int nq, int H, int c, int64_t max_entries, ElemType t);
 cudaError_t mqa(const void* q, const void* KV, const int32_t* idx, int k, QuerySpec qs, int mp,
                 int nq, int n_seq, int H, int c, int64_t Nmax, float scale, const float* sink, void* out,
-                float* lse, void* ws, ElemType t, cudaStream_t st);
+                float* lse, void* ws, ElemType t, cudaStream_t st, RowBlocks kvb = RowBlocks{0, 0});
 
 // norm_rope.cu: RMSNorm (gamma != nullptr) then rotary encoding of the last R
 // channels of every row of c channels; row r takes the position of group

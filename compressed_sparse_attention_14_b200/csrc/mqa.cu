@@ -264,13 +264,13 @@ size_t mqa_workspace_bytes(int nq, int H, int c, int64_t max_entries, ElemType t
 
 cudaError_t mqa(const void* q, const void* KV, const int32_t* idx, int k, QuerySpec qs, int mp,
                 int nq, int n_seq, int H, int c, int64_t Nmax, float scale, const float* sink, void* out,
-                float* lse, void* ws, ElemType t, cudaStream_t st) {
+                float* lse, void* ws, ElemType t, cudaStream_t st, RowBlocks kvb) {
     if (nq == 0) return cudaSuccess;
     const int64_t max_entries = idx ? k : Nmax;
     if (t == ElemType::BF16) {
         const int ns = plan_nsplit(nq, H, max_entries, t);
         cudaError_t e = mqa_tc(q, KV, idx, k, qs, mp, nq, n_seq, H, c, Nmax, scale, sink, out, lse, ws, ns,
-                               device_status(), st);
+                               device_status(), st, kvb);
         if (e != cudaSuccess || ns == 1 || mqa_tc_pair(ns)) return e;
         float* part_o = (float*)ws;
         float* part_ml = (float*)((char*)ws + align256((size_t)nq * ns * H * c * sizeof(float)));

@@ -68,6 +68,7 @@ struct MqaArgs {
     const float* sink;
     int nsplit;
     int pair;                 // nsplit == 2: the query's two splits form a cluster and merge on chip
+    RowBlocks kvb;            // where the cache rows live (sparse gather)
     int64_t split_len;
     bf16* out;
     float* lse;
@@ -144,14 +145,14 @@ __device__ __forceinline__ int sparse_gather(const MqaArgs& a, uint8_t* kv_s, ui
     int j = 0;
     for (; j < ntiles; ++j) {
         const int64_t e0 = e_beg + (int64_t)j * kE + part * kRows;
-        int rows[kRows / 4];
+        int64_t rows[kRows / 4];   // byte offsets of the rows
 #pragma unroll
         for (int i = 0; i < kRows / 4; ++i) {
             const int64_t e = e0 + 4 * i + rsub;
             int s = -1;
             if (e < e_end) s = a.idx[(int64_t)t * a.k + e];
             if (s < 0 || s >= a.Nmax) s = 0;   // masked in the softmax
-            rows[i] = (int)(row0 + s);
+            rows[i] = row_byte_offset(row0 + s, row_bytes, a.kvb);
         }
         bool ok = true;
         for (int b = 0; b < a.dblocks; ++b) {
@@ -162,8 +163,7 @@ __device__ __forceinline__ int sparse_gather(const MqaArgs& a, uint8_t* kv_s, ui
 #pragma unroll
             for (int i = 0; i < kRows / 4; ++i) {
                 const int r = part * kRows + 4 * i + rsub;
-                cp_async16(dst + r * 128 + ((chunk ^ (r & 7)) << 4),
-                           kv_g + (int64_t)rows[i] * row_bytes + b * 128 + chunk * 16);
+                cp_async16(dst + r * 128 + ((chunk ^ (r & 7)) << 4), kv_g + rows[i] + b * 128 + chunk * 16);
             }
             cp_async_commit();
         }
@@ -785,9 +785,12 @@ int mqa_tc_nsplit(int nq, int H, int64_t max_entries, int num_sms) {
 
 cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, QuerySpec qs, int mp, int nq, int n_seq,
                    int H, int c, int64_t Nmax, float scale, const float* sink, void* out, float* lse, void* ws,
-                   int nsplit, int* status, cudaStream_t st) {
+                   int nsplit, int* status, cudaStream_t st, RowBlocks kvb) {
     if (nq == 0) return cudaSuccess;
+    if (kvb.rpb > 0 && (Nmax % kvb.rpb || (!idx && kvb.rpb != 1) || kvb.block_bytes % 16))
+        return cudaErrorInvalidValue;
     MqaArgs a{};
+    a.kvb = kvb;
     a.qm = QueryMap{qs.seq, qs.pos, qs.pos_base, qs.single_seq};
     a.n_seq = n_seq;
     a.mp = mp;
@@ -821,7 +824,9 @@ cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, Que
 
     CUtensorMap tmQ, tmTile;
     if (!make_tmap_bf16_2d(&tmQ, q, (uint64_t)nq * H, c, c, a.hg, 64)) return cudaErrorInvalidValue;
-    if (!make_tmap_bf16_2d(&tmTile, KV, (uint64_t)n_seq * Nmax, c, c, kE, 64)) return cudaErrorInvalidValue;
+    // dense rows in blocks (one per block): the block is the row pitch
+    const uint64_t kv_pitch = kvb.rpb ? (uint64_t)kvb.block_bytes / 2 : (uint64_t)c;
+    if (!make_tmap_bf16_2d(&tmTile, KV, (uint64_t)n_seq * Nmax, c, kv_pitch, kE, 64)) return cudaErrorInvalidValue;
 
     const size_t fixed = 1024 + a.q_bytes + kE * 128 + (64 * 4 + 256) * sizeof(float) + 32 * sizeof(uint64_t);
     size_t kv_bytes = (size_t)a.dblocks * kE * 128;

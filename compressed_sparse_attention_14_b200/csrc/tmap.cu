@@ -48,4 +48,18 @@ bool make_tmap_u8_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t
     return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_bf16_blocks(CUtensorMap* map, const void* base, uint64_t nblocks, uint32_t rows_per_block,
+                           uint64_t cols, uint64_t block_bytes, uint32_t box_blocks, uint32_t box_cols) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {cols, rows_per_block, nblocks};
+    cuuint64_t strides[2] = {cols * 2, block_bytes};
+    cuuint32_t box[3] = {box_cols, rows_per_block, box_blocks};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 }  // namespace csa

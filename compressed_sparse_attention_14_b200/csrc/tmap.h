@@ -19,4 +19,12 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64
 bool make_tmap_u8_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t pitch_bytes,
                      uint32_t box_rows, uint32_t box_cols);
 
+// Rows of a bf16 matrix that come in blocks: rows_per_block rows of `cols`
+// elements (row pitch cols, 16-byte multiple), block j at j * block_bytes;
+// viewed as 3D tiles of box_blocks x rows_per_block x box_cols with 128-byte
+// swizzle (the tile lands in shared memory exactly as box_blocks *
+// rows_per_block consecutive rows of a 2D tile would).
+bool make_tmap_bf16_blocks(CUtensorMap* map, const void* base, uint64_t nblocks, uint32_t rows_per_block,
+                           uint64_t cols, uint64_t block_bytes, uint32_t box_blocks, uint32_t box_cols);
+
 }  // namespace csa

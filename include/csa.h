@@ -463,6 +463,67 @@ int csa_attend_decode(const void* qI, const float* w, const void* idx_cache, con
                       float rope_base, const float* sink, void* out, float* lse, int32_t* topk_idx, void* ws,
                       size_t ws_bytes, int dtype, void* stream);
 
+/* ------------------------------------------------------------------------
+ * The lcm(m, m')-token cache block [Notes §2.6, the compressed KV cache: one
+ * block covers lcm(m, m') raw tokens and holds their lcm/m CSA entries and
+ * lcm/m' HCA entries; Walk §5 item 2]. The entries of one sequence live in
+ * consecutive blocks; block j (raw tokens j*L .. j*L+L-1, L = lcm(m, m'))
+ * holds, in this order:
+ *   CSA KV entries   [L/m][c]   (entries j*L/m ..),
+ *   CSA index keys   [L/m][cI],
+ *   HCA entries      [L/m'][c]  (entries j*L/m' ..),
+ * each row in the cache dtype. The compressor state rings of the tail tokens
+ * (csa_compress_step, hca_compress_step) stay per sequence, outside the
+ * blocks. Sequence b's blocks start Nmax/(L/m) blocks after sequence b-1's,
+ * Nmax being the CSA entry capacity per sequence (a multiple of L/m); the HCA
+ * capacity is then Nmax*m/m'.
+ *
+ * csa_cache_block_layout: the block for (m, m', c, cI, dtype): rows of each
+ * part per block, bytes per block (a multiple of 16: c and cI multiples of
+ * 8) and the byte offset of each part in a block (offset pointers may be
+ * NULL). The *_blocked calls below take a cache as (pointer to the part in
+ * block 0 = block base + its offset, rows_per_block, block_bytes); they
+ * compute exactly what the contiguous calls compute (same kernels, same
+ * arithmetic), bf16 caches only. CSA_ERR_INVALID_ARG for an inconsistent
+ * layout (rows_per_block < 1, block_bytes not a multiple of 16 or too short
+ * for its rows, Nmax not a multiple of rows_per_block, a cache pointer not
+ * 16-byte aligned); CSA_ERR_UNSUPPORTED for fp32 caches, a CSA rows_per_block
+ * that does not divide 128 (the indexer's key tile), or more than one HCA row
+ * per block. Nothing is allocated.
+ * ------------------------------------------------------------------------ */
+int csa_cache_block_layout(int m, int mp, int c, int cI, int dtype, int* csa_rows, int* hca_rows,
+                           int64_t* block_bytes, int64_t* kv_offset, int64_t* idx_offset, int64_t* hca_offset);
+
+/* csa_decode over block caches: kv_cache -> block 0's CSA KV part,
+ * idx_cache -> block 0's index-key part, rows_per_block = L/m. Workspace as
+ * csa_decode_workspace_size. */
+int csa_decode_blocked(const void* qI, const float* w, const void* idx_cache, const void* q, const void* kv_cache,
+                       const int32_t* ctx_len, int B, int64_t Nmax, int m, int H, int c, int HI, int cI, int k,
+                       float scale, const float* sink, void* out, float* lse, int32_t* topk_idx, int rows_per_block,
+                       int64_t block_bytes, void* ws, size_t ws_bytes, int dtype, void* stream);
+
+/* hca_decode over block caches: kv_cache -> block 0's HCA part,
+ * rows_per_block = L/m' = 1, Nmax = the HCA capacity per sequence. Workspace
+ * as hca_decode_workspace_size. */
+int hca_decode_blocked(const void* q, const void* kv_cache, const int32_t* ctx_len, int B, int64_t Nmax, int mp,
+                       int H, int c, float scale, const float* sink, void* out, float* lse, int rows_per_block,
+                       int64_t block_bytes, void* ws, size_t ws_bytes, int dtype, void* stream);
+
+/* csa_decode_compress writing the closed blocks' entries into block caches
+ * (kv_cache, idx_cache as for csa_decode_blocked). Workspace as
+ * csa_decode_compress_workspace_size. */
+int csa_decode_compress_blocked(const void* x_new, const void* W_kv, const float* B_kv, const void* W_idx,
+                                const float* B_idx, const int32_t* pos, int B, int d, int m, int c, int cI,
+                                float* state_kv, float* state_idx, void* kv_cache, void* idx_cache, int64_t Nmax,
+                                int rows_per_block, int64_t block_bytes, void* ws, size_t ws_bytes, int dtype,
+                                void* stream);
+
+/* hca_compress_step writing into block caches (cache -> block 0's HCA part,
+ * rows_per_block = 1, Nmax = the HCA capacity per sequence). */
+int hca_compress_step_blocked(const float* proj_new, float* state, const float* bias, const int32_t* pos, int B,
+                              int c, int mp, int64_t Nmax, void* cache, int rows_per_block, int64_t block_bytes,
+                              int dtype, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -182,6 +182,53 @@ def test_compress_step_arguments_are_checked_on_the_host():
     assert rc == csa.CSA_ERR_WORKSPACE
 
 
+def test_cache_block_layout_is_the_lcm_block():
+    # [Notes §2.6: one block covers lcm(m, m') raw tokens, i.e. lcm/m CSA
+    # entries and lcm/m' HCA entries]; parts in the order KV, index keys, HCA
+    for m, mp, c, cI in [(4, 128, 512, 128), (4, 6, 64, 32), (3, 5, 16, 8), (8, 8, 128, 64)]:
+        lcm = next(L for L in range(max(m, mp), m * mp + 1) if L % m == 0 and L % mp == 0)   # brute force
+        lay = csa.csa_cache_block_layout(m, mp, c, cI)
+        assert (lay["csa_rows"], lay["hca_rows"]) == (lcm // m, lcm // mp)
+        assert lay["kv_offset"] == 0
+        assert lay["idx_offset"] == lcm // m * c * 2
+        assert lay["hca_offset"] == lay["idx_offset"] + lcm // m * cI * 2
+        assert lay["block_bytes"] == lay["hca_offset"] + lcm // mp * c * 2
+        assert lay["block_bytes"] % 16 == 0
+    assert csa.csa_cache_block_layout(4, 128, 512, 128, csa.CSA_FP32)["block_bytes"] == 4 * (32 * 512 + 32 * 128 + 512)
+    L = _lib()
+    out = [ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int64(0)]
+    assert L.csa_cache_block_layout(0, 128, 512, 128, csa.CSA_BF16, *[ctypes.byref(o) for o in out], None, None,
+                                    None) == csa.CSA_ERR_INVALID_ARG
+    assert L.csa_cache_block_layout(4, 128, 60, 128, csa.CSA_BF16, *[ctypes.byref(o) for o in out], None, None,
+                                    None) == csa.CSA_ERR_INVALID_ARG
+
+
+def test_blocked_calls_check_the_layout_on_the_host():
+    L = _lib()
+    fake = 0x10000
+    bb = 41984   # lcm block of m = 4, m' = 128, c = 512, cI = 128 (bf16)
+
+    def dec(rpb, block_bytes, Nmax=1024, dtype=csa.CSA_BF16, kv=fake):
+        return L.csa_decode_blocked(fake, fake, fake, fake, kv, fake, 4, Nmax, 4, 64, 512, 64, 128, 512, 0.0, None,
+                                    fake, None, None, rpb, block_bytes, None, 0, dtype, None)
+    assert dec(0, bb) == csa.CSA_ERR_INVALID_ARG                 # no rows per block
+    assert dec(32, bb + 8) == csa.CSA_ERR_INVALID_ARG            # block not a multiple of 16 bytes
+    assert dec(32, 16 * 1024) == csa.CSA_ERR_INVALID_ARG         # too short for 32 rows of 512 bf16
+    assert dec(32, bb, Nmax=1000) == csa.CSA_ERR_INVALID_ARG     # Nmax not a multiple of the block's rows
+    assert dec(32, bb, kv=fake + 8) == csa.CSA_ERR_INVALID_ARG   # misaligned cache pointer
+    assert dec(32, bb, dtype=csa.CSA_FP32) == csa.CSA_ERR_UNSUPPORTED
+    assert dec(24, 24 * 1024 * 2, Nmax=960) == csa.CSA_ERR_UNSUPPORTED   # 24 does not divide the 128-key tile
+    assert dec(32, bb) == csa.CSA_ERR_WORKSPACE                  # a consistent layout reaches the workspace check
+    rc = L.hca_decode_blocked(fake, fake, fake, 4, 256, 128, 64, 512, 0.0, None, fake, None, 2, bb, None, 0,
+                              csa.CSA_BF16, None)
+    assert rc == csa.CSA_ERR_UNSUPPORTED                         # one HCA entry per block
+    rc = L.csa_decode_compress_blocked(fake, fake, fake, fake, fake, fake, 4, 4096, 4, 512, 128, fake, fake, fake,
+                                       fake, 1000, 32, bb, None, 0, csa.CSA_BF16, None)
+    assert rc == csa.CSA_ERR_INVALID_ARG
+    rc = L.hca_compress_step_blocked(fake, fake, fake, fake, 4, 512, 128, 256, fake, 1, bb + 4, csa.CSA_BF16, None)
+    assert rc == csa.CSA_ERR_INVALID_ARG
+
+
 def test_empty_inputs_are_no_ops():
     L = _lib()
     assert L.csa_compress(None, None, None, 0, 8, 4, None, csa.CSA_BF16, None) == csa.CSA_OK
