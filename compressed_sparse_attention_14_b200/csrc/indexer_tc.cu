@@ -260,7 +260,9 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 
 }  // namespace
 
-template <bool kFp8, int kN, int kHI, int kH>
+// kBlk: the keys come in blocks (a 3D key map); a separate instantiation, so
+// that the contiguous path's producer loop stays as it was
+template <bool kFp8, int kN, int kHI, int kH, bool kBlk = false>
 __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __grid_constant__ IdxArgs a,
                                                                       const __grid_constant__ CUtensorMap tmK,
                                                                       const __grid_constant__ CUtensorMap tmQ) {
@@ -338,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
 #pragma unroll
                     for (int hh = 0; hh < kH; ++hh)
                         for (int kb = 0; kb < a.kblocks; ++kb)
-                            if (a.key_rpb)   // kKeys / key_rpb blocks of key_rpb rows
+                            if constexpr (kBlk)   // kKeys / key_rpb blocks of key_rpb rows
                                 tc::tma_load_3d(dst + (size_t)(hh * a.kblocks + kb) * kKeys * 128, &tmK, &sm.full[s],
                                                 kb * a.blk_elems, 0, (row + hh * kKeys) / a.key_rpb);
                             else
@@ -616,6 +618,9 @@ cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, Query
         kern = fp8 ? index_scores_tc_kernel<true, 64, 64, 2> : index_scores_tc_kernel<false, 64, 64, 1>;
     else if (a.npad == 256 && HI == 64 && group == 4)
         kern = fp8 ? index_scores_tc_kernel<true, 256, 64, 1> : index_scores_tc_kernel<false, 256, 64, 1>;
+    if (a.key_rpb)   // bf16 keys in blocks (decode shape, or any other)
+        kern = (a.npad == 64 && HI == 64 && group == 1) ? index_scores_tc_kernel<false, 64, 64, 1, true>
+                                                          : index_scores_tc_kernel<false, 0, 0, 1, true>;
     e = smem_ceiling(kern);
     if (e != cudaSuccess) return e;
     CSA_LAUNCH(st, fp8 ? "index_scores_tc_fp8" : "index_scores_tc",

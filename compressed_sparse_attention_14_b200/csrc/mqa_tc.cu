@@ -38,6 +38,8 @@
 // tile used, and one thread writes it to the workspace with bulk copies,
 // beside the split's reference maxima and sums; mqa_combine then merges the
 // splits in split order (deterministic). Waits are bounded (CSA_ERR_TIMEOUT).
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -135,6 +137,7 @@ __device__ __forceinline__ void bar_sync_128() { asm volatile("bar.sync 1, 128;"
 // warp arrives on block b's barrier once its copies of it have completed.
 // Returns the tiles handed over.
 constexpr int kGatherWarps = 2;
+template <bool kBlk>
 __device__ __forceinline__ int sparse_gather(const MqaArgs& a, uint8_t* kv_s, uint64_t* kv_full, uint64_t* kv_empty,
                                              int part, int lane, int t, int ntiles, int64_t e_beg, int64_t e_end,
                                              int64_t row0, volatile int* abort_flag) {
@@ -145,14 +148,17 @@ __device__ __forceinline__ int sparse_gather(const MqaArgs& a, uint8_t* kv_s, ui
     int j = 0;
     for (; j < ntiles; ++j) {
         const int64_t e0 = e_beg + (int64_t)j * kE + part * kRows;
-        int64_t rows[kRows / 4];   // byte offsets of the rows
+        // rows: the row indices (contiguous cache), or their byte offsets
+        // (rows in blocks)
+        std::conditional_t<kBlk, int64_t, int> rows[kRows / 4];
 #pragma unroll
         for (int i = 0; i < kRows / 4; ++i) {
             const int64_t e = e0 + 4 * i + rsub;
             int s = -1;
             if (e < e_end) s = a.idx[(int64_t)t * a.k + e];
             if (s < 0 || s >= a.Nmax) s = 0;   // masked in the softmax
-            rows[i] = row_byte_offset(row0 + s, row_bytes, a.kvb);
+            if constexpr (kBlk) rows[i] = row_byte_offset(row0 + s, row_bytes, a.kvb);
+            else rows[i] = (int)(row0 + s);
         }
         bool ok = true;
         for (int b = 0; b < a.dblocks; ++b) {
@@ -163,7 +169,8 @@ __device__ __forceinline__ int sparse_gather(const MqaArgs& a, uint8_t* kv_s, ui
 #pragma unroll
             for (int i = 0; i < kRows / 4; ++i) {
                 const int r = part * kRows + 4 * i + rsub;
-                cp_async16(dst + r * 128 + ((chunk ^ (r & 7)) << 4), kv_g + rows[i] + b * 128 + chunk * 16);
+                const int64_t off = kBlk ? (int64_t)rows[i] : (int64_t)rows[i] * row_bytes;
+                cp_async16(dst + r * 128 + ((chunk ^ (r & 7)) << 4), kv_g + off + b * 128 + chunk * 16);
             }
             cp_async_commit();
         }
@@ -276,6 +283,9 @@ __device__ __noinline__ void pair_merge(int c, int H, const float* sink, float* 
     tc::cluster_sync();
 }
 
+// kBlk: the cache rows come in blocks (a separate instantiation, so that the
+// contiguous path's gather stays as it was)
+template <bool kBlk>
 __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_constant__ MqaArgs a,
                                                              const __grid_constant__ CUtensorMap tmQ,
                                                              const __grid_constant__ CUtensorMap tmTile) {
@@ -364,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
             }
             int j = 0;
             if (a.idx) {
-                j = sparse_gather(a, kv_s, kv_full, kv_empty, 0, lane, t, ntiles, e_beg, e_end, row0, abort_flag);
+                j = sparse_gather<kBlk>(a, kv_s, kv_full, kv_empty, 0, lane, t, ntiles, e_beg, e_end, row0, abort_flag);
             } else if (lane == 0) {
                 // Dense rows stream through the ring twice per tile, pair by
                 // pair of 64-dim blocks: for the first product (S) through
@@ -382,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
         // ---------------------------------------------------------------- loads: sparse second half, dense O ring
         if (a.idx) {
             if (ntiles > 0)
-                sparse_gather(a, kv_s, kv_full, kv_empty, 1, lane, t, ntiles, e_beg, e_end, row0, abort_flag);
+                sparse_gather<kBlk>(a, kv_s, kv_full, kv_empty, 1, lane, t, ntiles, e_beg, e_end, row0, abort_flag);
         } else if (lane == 0 && ntiles > 0) {
             dense_ring_load(a, kv_s, &tmTile, kv_full, kv_empty, a.ring / 2, a.ring - a.ring / 2, ntiles,
                             row0 + e_beg, abort_flag);
@@ -843,11 +853,12 @@ cudaError_t mqa_tc(const void* q, const void* KV, const int32_t* idx, int k, Que
         kv_bytes = (size_t)ring * 2 * kE * 128;
     }
     const size_t smem = fixed + kv_bytes;
-    cudaError_t e = smem_ceiling(mqa_tc_kernel);
+    auto kern = kvb.rpb ? mqa_tc_kernel<true> : mqa_tc_kernel<false>;
+    cudaError_t e = smem_ceiling(kern);
     if (e != cudaSuccess) return e;
     cudaError_t le = cudaSuccess;
     CSA_LAUNCH(st, "mqa_tc",
-               le = launch_pdl(mqa_tc_kernel, dim3(nsplit, (H + a.hg - 1) / a.hg, nq), dim3(kThreads), smem, st,
+               le = launch_pdl(kern, dim3(nsplit, (H + a.hg - 1) / a.hg, nq), dim3(kThreads), smem, st,
                                a.pair ? 2u : 0u, a, tmQ, tmTile));
     if (le != cudaSuccess) return le;
     return cudaGetLastError();
