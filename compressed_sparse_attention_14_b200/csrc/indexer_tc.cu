@@ -178,6 +178,23 @@ struct Walk {
     __device__ bool last_of_group() const { return t + 1 == tiles_g; }
 };
 
+// Position in a ring of n slots as the tile counter advances: slot, the
+// parity of the slot's current use, and whether the ring has wrapped (the
+// counter's quotient and remainder without a 64-bit division per tile).
+struct RingPos {
+    int n, slot = 0;
+    uint32_t phase = 0;
+    bool wrapped = false;
+    __device__ explicit RingPos(int n_) : n(n_) {}
+    __device__ void advance() {
+        if (++slot == n) {
+            slot = 0;
+            phase ^= 1u;
+            wrapped = true;
+        }
+    }
+};
+
 // Paired fp32: two values in one 64-bit register; d = a * b + c lane by
 // lane, round to nearest (sm_100 packed FMA).
 __device__ __forceinline__ uint64_t pack2(float lo, float hi) {
@@ -318,7 +335,8 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
             int cur = -1;
             uint32_t switches = 0;
             int64_t it = 0;
-            for (; it < my; ++it) {
+            RingPos st(a.stages);
+            for (; it < my; ++it, st.advance()) {
                 if (wk.g != cur) {
                     if (switches > 0 && !wait_or_abort(sm.qempty, (switches - 1) & 1, abort_flag, a.status, a.wait_limit)) break;
                     tc::mbar_expect_tx(sm.qfull, a.q_bytes);
@@ -328,8 +346,8 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
                     cur = wk.g;
                     ++switches;
                 }
-                const int s = (int)(it % a.stages);
-                if (it >= a.stages && !wait_or_abort(&sm.empty[s], ((it / a.stages) - 1) & 1, abort_flag, a.status, a.wait_limit))
+                const int s = st.slot;
+                if (st.wrapped && !wait_or_abort(&sm.empty[s], st.phase ^ 1u, abort_flag, a.status, a.wait_limit))
                     break;
                 if (!(a.skip_first_tile && it == 0)) {
                     tc::mbar_expect_tx(&sm.full[s], a.stage_bytes);
@@ -373,7 +391,8 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
             const uint32_t a_kb_step = (kKeys * 128) >> 4;
             const uint32_t b_kb_step = (uint32_t)(a.npad * 128) >> 4;
             int64_t it = 0;
-            for (; it < my; ++it) {
+            RingPos st(a.stages), bf(a.nbuf);
+            for (; it < my; ++it, st.advance(), bf.advance()) {
                 if (wk.g != cur) {
                     if (!wait_or_abort(sm.qfull, switches & 1, abort_flag, a.status, a.wait_limit)) break;
                     cur = wk.g;
@@ -384,11 +403,11 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
                     wk.next(a, ngroups);
                     continue;
                 }
-                const int s = (int)(it % a.stages);
-                const int buf = (int)(it % a.nbuf);
-                const int64_t use = it / a.nbuf;
-                if (!wait_or_abort(&sm.full[s], (it / a.stages) & 1, abort_flag, a.status, a.wait_limit)) break;
-                if (use >= 1 && !wait_or_abort(&sm.tempty[buf], (use - 1) & 1, abort_flag, a.status, a.wait_limit)) break;
+                const int s = st.slot;
+                const int buf = bf.slot;
+                if (!wait_or_abort(&sm.full[s], st.phase, abort_flag, a.status, a.wait_limit)) break;
+                if (bf.wrapped && !wait_or_abort(&sm.tempty[buf], bf.phase ^ 1u, abort_flag, a.status, a.wait_limit))
+                    break;
                 tc::tc_fence_after();
                 const uint64_t a_s = a_desc0 + (uint64_t)(s * stage_step);
 #pragma unroll
@@ -432,7 +451,8 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
         wk.start(a, g0, t0);
         int cur = -1;
         int64_t vis = 0;
-        for (int64_t it = 0; it < my; ++it, wk.next(a, ngroups)) {
+        RingPos bf(a.nbuf);
+        for (int64_t it = 0; it < my; ++it, wk.next(a, ngroups), bf.advance()) {
             if (kN != 256 && (int)(it & 1) != set) continue;
             if (wk.g != cur) {
                 __syncwarp();
@@ -445,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
                 cur = wk.g;
                 vis = group_visible(a, wk.g);
             }
-            const int buf = (int)(it % a.nbuf);
+            const int buf = bf.slot;
             // this thread's keys: row of each 128-key half of the tile
             int64_t key[kH];
             float kscale[kH];
@@ -457,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
                 if constexpr (kFp8)
                     if (key[hh] < vis) kscale[hh] = __ldg(a.kscale + (int64_t)group_seq(a, wk.g) * a.Nmax + key[hh]);
             }
-            if (!wait_or_abort(&sm.tfull[buf], (uint32_t)((it / a.nbuf) & 1), abort_flag, a.status, a.wait_limit)) break;
+            if (!wait_or_abort(&sm.tfull[buf], bf.phase, abort_flag, a.status, a.wait_limit)) break;
             tc::tc_fence_after();
             // sc[hh][q]: the scores of query q of the group; with kN == 256
             // this set's two queries (2 set, 2 set + 1) sit in sc[hh][0..1]

@@ -198,13 +198,20 @@ __device__ __noinline__ void dense_ring_load(const MqaArgs& a, uint8_t* kv_s, co
                                              volatile int* abort_flag) {
     uint32_t cnt = 0;
     bool ok = true;
+    // ring position without a division per slot: index, use parity, wrapped
+    int pos = 0;
+    uint32_t phase = 0;
+    bool wrapped = false;
     for (int jt = 0; ok && jt < ntiles; ++jt) {
         const int row = (int)(row_base + (int64_t)jt * kE);
         for (int mt = 0; mt < a.mtiles; ++mt, ++cnt) {
-            const int slot = r_lo + (int)(cnt % (uint32_t)r_n);
-            if (cnt >= (uint32_t)r_n &&
-                !(ok = wait_or_abort(&kv_empty[slot], ((cnt / r_n) - 1) & 1, abort_flag, a.status)))
-                break;
+            const int slot = r_lo + pos;
+            if (wrapped && !(ok = wait_or_abort(&kv_empty[slot], phase ^ 1u, abort_flag, a.status))) break;
+            if (++pos == r_n) {
+                pos = 0;
+                phase ^= 1u;
+                wrapped = true;
+            }
             uint8_t* dst = kv_s + (size_t)slot * 2 * kE * 128;
             tc::mbar_expect_tx(&kv_full[slot], 2 * kE * 128);
             tc::tma_load_2d(dst, tm, &kv_full[slot], 2 * mt * 64, row);
@@ -420,7 +427,8 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
             if (!a.idx) {
                 // dense: this issuer's ring, in the order its producer fills it
                 const int r_lo = mi ? a.ring / 2 : 0, r_n = mi ? a.ring - a.ring / 2 : a.ring / 2;
-                uint32_t cnt = 0;
+                int pos = 0;          // ring position (no division per slot)
+                uint32_t phase = 0;
                 for (int jt = 0; ok && jt < ntiles; ++jt) {
                     const int sb = jt & 1;
                     if (mi == 0) {
@@ -430,9 +438,13 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
                         if (!(ok = wait_or_abort(p_full, jt & 1, abort_flag, a.status))) break;
                         tc::tc_fence_after();
                     }
-                    for (int mt = 0; mt < a.mtiles; ++mt, ++cnt) {
-                        const int slot = r_lo + (int)(cnt % (uint32_t)r_n);
-                        if (!(ok = wait_or_abort(&kv_full[slot], (cnt / r_n) & 1, abort_flag, a.status))) break;
+                    for (int mt = 0; mt < a.mtiles; ++mt) {
+                        const int slot = r_lo + pos;
+                        if (!(ok = wait_or_abort(&kv_full[slot], phase, abort_flag, a.status))) break;
+                        if (++pos == r_n) {
+                            pos = 0;
+                            phase ^= 1u;
+                        }
                         tc::tc_fence_after();
                         const uint32_t sa = kv_addr + (uint32_t)slot * 2 * kE * 128;
                         if (mi == 0) {
