@@ -165,6 +165,35 @@ def test_topk_rows_against_a_strided_sample(csa):
     np.testing.assert_array_equal(host(idx), ref)
 
 
+@pytest.mark.parametrize("score_dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("ncols,k", [(20003, 512), (9000, 128)])
+def test_topk_many_long_rows(csa, score_dtype, ncols, k):
+    """More rows than SMs (one CTA per row), every row past the in-shared-
+    memory limit, so every row goes through the sampled estimate and the
+    filter pass; rows that mislead the estimate (too many or too few
+    candidates) and heavy ties fall back to the exact selection on the whole
+    row."""
+    nq = 200
+    g = torch.Generator().manual_seed(77)
+    S = torch.randn(nq, ncols, generator=g)
+    S[0] = torch.round(S[0] * 2) / 2              # heavy ties
+    S[1, 1::2] = 0.0                              # signed zeros
+    S[1, ::2] = -0.0
+    pos = (torch.arange(4096, dtype=torch.int64) * ncols) // 4096
+    S[2, pos] += 10.0                             # the sample sees only the largest
+    S[3, pos] -= 10.0                             # the sample sees only the smallest
+    S[4, 7::3] = 2.0                              # many equal scores above the k-th
+    S = S.to(score_dtype)
+    if score_dtype == torch.bfloat16:
+        idx, top = csa.csa_topk_from_scores_bf16(S.to(DEV), k)
+    else:
+        idx, top = csa.csa_topk_from_scores(S.to(DEV), k)
+    ref = oracle.topk(S.float().double().numpy(), np.full(nq, ncols, dtype=np.int32), k)
+    np.testing.assert_array_equal(host(idx), ref)
+    want = np.take_along_axis(S.float().numpy(), np.maximum(ref, 0), 1)
+    np.testing.assert_array_equal(top.cpu().numpy(), want.astype(np.float32))
+
+
 # ---------------------------------------------------------------- a4 + a5
 @pytest.mark.parametrize("dtype", MODES)
 def test_index_topk(csa, dtype):
