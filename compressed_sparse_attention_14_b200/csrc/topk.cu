@@ -561,6 +561,18 @@ __device__ __forceinline__ void cluster_wait_acquire() {
 
 constexpr int kFilterLoads = 4;   // 16-byte filter loads in flight per thread
 
+// Bulk prefetch of the bytes [b, e) into L2 (the 16-byte-aligned part, in
+// 32 KB pieces); a hint only.
+template <typename TS>
+__device__ __forceinline__ void prefetch_l2(const TS* b, const TS* e) {
+    uintptr_t p = ((uintptr_t)b + 15) & ~(uintptr_t)15;
+    const uintptr_t end = (uintptr_t)e & ~(uintptr_t)15;
+    for (; p + 16 <= end; p += 32768) {
+        const uint32_t bytes = (uint32_t)(end - p < 32768 ? end - p : 32768);
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+    }
+}
+
 template <typename TS>
 __global__ void __launch_bounds__(kThreads, 2) topk_kernel(RowSpec R, int k, int32_t* idx, float* top) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -590,6 +602,11 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(RowSpec R, int k, int
         return;
     }
 
+    // ---- this CTA's slice starts on its way to L2 while the threshold is
+    // worked out (bulk prefetches: no registers or shared memory held)
+    const int64_t lo = n * g / G, hi = n * (g + 1) / G;
+    if (tid == 0) prefetch_l2(srow + lo, srow + hi);
+
     // ---- threshold from the sample (identical in every CTA of the cluster)
     if (tid == 0) { s_cnt = 0; s_total = 0; }
     // CTA 0's total must be zero before any CTA of the cluster adds to it:
@@ -601,7 +618,6 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(RowSpec R, int k, int
     const uint32_t thr = sample_threshold(srow, n, r, bs);
 
     // ---- this CTA's slice: keep every score that reaches it
-    const int64_t lo = n * g / G, hi = n * (g + 1) / G;
     if (G == 1) {
         filter_slice<kFilterLoads>(srow, lo, hi, thr, cand, kCap, &s_cnt);
         __syncthreads();
