@@ -229,12 +229,14 @@ class Timer:
 # workloads (ours)
 # ----------------------------------------------------------------------------
 
-def decode_workload(shape, rank, batch=None, fp8=False):
+def decode_workload(shape, rank, batch=None, fp8=False, fp8kv=False):
     """One csa_decode step over the batch. fp8: the FP8 indexer
     (csa_decode_fp8): the indexer keys are held as e4m3 codes with one fp32
     scale per key (quantized once when the cache is built, outside the timed
     region, as the compressor would store them), q^I is quantized in the call;
-    fp32 index scores (bf16 scores tie more often and made this top-k slower)."""
+    fp32 index scores (bf16 scores tie more often and made this top-k slower).
+    fp8kv: the KV entries held in FP8 storage with bf16 rotary dims
+    (csa_decode_fp8kv; quantized once outside the timed region)."""
     import dataclasses
     import compressed_sparse_attention_14_b200 as csa
     s = shape if batch is None else dataclasses.replace(shape, batch=batch)
@@ -243,7 +245,16 @@ def decode_workload(shape, rank, batch=None, fp8=False):
     mode = csa.CSA_BF16
     out = torch.empty_like(inp["q"])
     lse = torch.empty((B, s.heads), dtype=torch.float32, device="cuda")
-    if fp8:
+    if fp8kv:
+        kv8, kvs, kvr = csa.csa_quantize_kv_fp8(inp["kv_cache"], rope_dims=ATTEND_ROPE)
+        del inp["kv_cache"]
+        torch.cuda.synchronize()
+        ws = torch.empty(csa._lib.csa_decode_fp8kv_workspace_size(B, s.n_max, s.heads, s.c, s.idx_heads, s.idx_dim,
+                                                                  s.k), dtype=torch.uint8, device="cuda")
+
+        def call(qI, w, q, ctx, o=out):
+            csa.csa_decode_fp8kv(qI, w, inp["idx_cache"], q, kv8, kvs, kvr, ctx, s.m, s.k, out=o, lse=lse, ws=ws)
+    elif fp8:
         k8, ks, _ = csa.csa_quantize_e4m3(inp["idx_cache"])
         del inp["idx_cache"]
         torch.cuda.synchronize()
@@ -269,7 +280,9 @@ def decode_workload(shape, rank, batch=None, fp8=False):
     # plus one fp32 scale), q^I and w; the selected KV rows; q and out (bf16)
     key_bytes = (s.idx_dim + 4) if fp8 else s.idx_dim * 2
     idx_bytes = v_sum * key_bytes + B * (s.idx_heads * s.idx_dim * (1 if fp8 else 2) + s.idx_heads * 4)
-    step_bytes = idx_bytes + B * (s.k * s.c * 2 + 2 * s.heads * s.c * 2)
+    # a selected KV row: bf16, or e4m3 codes + fp32 scale + bf16 rotary dims
+    row_bytes = (s.c - ATTEND_ROPE) + 4 + 2 * ATTEND_ROPE if fp8kv else s.c * 2
+    step_bytes = idx_bytes + B * (s.k * row_bytes + 2 * s.heads * s.c * 2)
     # the indexer kernel also writes one score per visible entry (fp32, or
     # bf16 on the low-precision path)
     score_bytes = 4
@@ -297,15 +310,19 @@ def decode_workload(shape, rank, batch=None, fp8=False):
     }
     if fp8:
         kernels["quantize_e4m3"] = dict(bound="hbm", work=B * s.idx_heads * (s.idx_dim * 3 + 12), files=("quant.cu",))
+    if fp8kv:
+        # the selection's FP8 rows in, bf16 rows out (then read by the MQA)
+        kernels["gather_kv_fp8"] = dict(bound="hbm", work=B * s.k * (row_bytes + s.c * 2 + 8), files=("quant.cu",))
     pipe = dict(pinned=pinned, out=out, run=lambda d, o: call(d["qI"], d["w"], d["q"], d["ctx_len"], o))
     return dict(step=step, e2e_step=e2e_step, pipe=pipe, units=B, unit="queries/s", h2d=h2d, d2h=d2h,
                 kernels=kernels, step_bytes=step_bytes,
-                config=dict(workload=s.name + ("_fp8_indexer" if fp8 else ""), batch=B,
+                config=dict(workload=s.name + ("_fp8_indexer" if fp8 else "_fp8_kv" if fp8kv else ""), batch=B,
                             ctx_len=f"U[{s.ctx_lo},{s.ctx_hi}]", m=s.m,
                             entries_max=s.n_max, head_dim=s.c, heads=s.heads, index_heads=s.idx_heads,
                             index_dim=s.idx_dim, topk=s.k, visible_entries_total=int(v_sum),
                             index_keys="e4m3 + fp32 scale per key" if fp8 else "bf16",
                             index_scores="fp32",
+                            kv_entries="e4m3 + fp32 scale per entry, bf16 rotary dims" if fp8kv else "bf16",
                             l2="flushed before every timed step (256 MiB write + 256 MiB read)"),
                 inputs=inp)
 
@@ -567,6 +584,7 @@ WORKLOADS = {
     "pro_decode": lambda r, b=None: decode_workload(synth.PRO_DECODE, r, b),
     "flash_decode_fp8": lambda r, b=None: decode_workload(synth.FLASH_DECODE, r, b, fp8=True),
     "pro_decode_fp8": lambda r, b=None: decode_workload(synth.PRO_DECODE, r, b, fp8=True),
+    "flash_decode_fp8kv": lambda r, b=None: decode_workload(synth.FLASH_DECODE, r, b, fp8kv=True),
     "hca_decode": lambda r, b=None: hca_decode_workload(r),
     "hca_compress": lambda r, b=None: hca_compress_workload(r),
     "prefill": lambda r, b=None: prefill_workload(r, b),
@@ -579,22 +597,30 @@ WORKLOADS = {
 # CPU oracle timing (the reference arm and the cpu_baseline object)
 # ----------------------------------------------------------------------------
 
-def oracle_decode_sample(shape, n_queries: int, seed_rank: int = 0, fp8: bool = False):
-    """Time the oracle (indexer + top-k + sparse MQA, fp64; fp8: the indexer
-    on e4m3-quantized q^I and keys) on the first n_queries of the decode
-    batch. Returns (seconds, queries)."""
+def oracle_decode_sample(shape, n_queries: int, seed_rank: int = 0, fp8=False):
+    """Time the oracle (indexer + top-k + sparse MQA, fp64; fp8 True: the
+    indexer on e4m3-quantized q^I and keys; fp8 "kv": the attention over the
+    selected entries in FP8 storage, quantized and dequantized per selected
+    row) on the first n_queries of the decode batch. Returns (seconds,
+    queries)."""
     import oracle
     s = dataclass_seed(shape, seed_rank)
     inp = synth.decode_inputs(s, device="cpu", batch=n_queries)
     t0 = time.perf_counter()
-    if fp8:
+    if fp8 is True:
         S = oracle.index_scores_fp8(inp["qI"], inp["w"], inp["idx_cache"], inp["ctx_len"], s.m,
                                     seq=torch.arange(n_queries))
         idx = oracle.topk(S, (inp["ctx_len"].numpy() // s.m).astype("int32"), s.k)
     else:
         idx, _ = oracle.index_topk(inp["qI"], inp["w"], inp["idx_cache"], inp["ctx_len"], s.m, s.k,
                                    seq=torch.arange(n_queries))
-    oracle.sparse_mqa(inp["q"], inp["kv_cache"], idx, 1 / math.sqrt(s.c), seq=torch.arange(n_queries))
+    if fp8 == "kv":
+        rows = np.stack([inp["kv_cache"][t].double().numpy()[np.maximum(idx[t], 0)] for t in range(n_queries)])
+        kv_sel = oracle.dequantize_kv_fp8(*oracle.quantize_kv_fp8(rows, ATTEND_ROPE))
+        sel = np.where(idx >= 0, np.arange(idx.shape[1])[None, :], -1).astype("int32")
+        oracle.sparse_mqa(inp["q"], kv_sel, sel, 1 / math.sqrt(s.c), seq=np.arange(n_queries))
+    else:
+        oracle.sparse_mqa(inp["q"], inp["kv_cache"], idx, 1 / math.sqrt(s.c), seq=torch.arange(n_queries))
     return time.perf_counter() - t0, n_queries
 
 
@@ -792,10 +818,12 @@ def run_reference(args, rank, world):
 
 
 DECODE_SHAPES = {"flash_decode": (synth.FLASH_DECODE, False), "pro_decode": (synth.PRO_DECODE, False),
-                 "flash_decode_fp8": (synth.FLASH_DECODE, True), "pro_decode_fp8": (synth.PRO_DECODE, True)}
+                 "flash_decode_fp8": (synth.FLASH_DECODE, True), "pro_decode_fp8": (synth.PRO_DECODE, True),
+                 "flash_decode_fp8kv": (synth.FLASH_DECODE, "kv")}
 
 WORKLOADS_CONFIG_NAME = {
     "flash_decode_fp8": synth.FLASH_DECODE.name + "_fp8_indexer",
+    "flash_decode_fp8kv": synth.FLASH_DECODE.name + "_fp8_kv",
     "pro_decode_fp8": synth.PRO_DECODE.name + "_fp8_indexer",
     "flash_decode": synth.FLASH_DECODE.name,
     "pro_decode": synth.PRO_DECODE.name,
@@ -978,6 +1006,7 @@ def measure(name, args, rank, world, local, steps, warmup, batch=None):
 # 1M-context decode, the long prefill chunk, HCA decode, the HCA compressor).
 # Each keeps its own step count, at most the headline's.
 EXTRA_WORKLOADS = {"pro_decode": 20, "prefill": 5, "hca_decode": 20, "hca_compress": 10, "flash_decode_fp8": 20,
+                   "flash_decode_fp8kv": 20,
                    "pro_decode_fp8": 20}
 
 

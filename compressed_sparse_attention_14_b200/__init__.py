@@ -84,6 +84,10 @@ _SIGS = {
     "hca_compress_step": (_I, [_P, _P, _P, _P, _I, _I, _I, _I64, _P, _I, _P]),
     "csa_decode_compress_workspace_size": (_SZ, [_I, _I, _I]),
     "csa_decode_compress": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I64, _P, _SZ, _I, _P]),
+    "csa_quantize_kv_fp8": (_I, [_P, _I64, _I, _I, _P, _P, _P, _P]),
+    "csa_decode_fp8kv_workspace_size": (_SZ, [_I, _I64, _I, _I, _I, _I, _I]),
+    "csa_decode_fp8kv": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I64, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P,
+                              _P, _P, _SZ, _P]),
     "csa_cache_block_layout": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "csa_decode_blocked": (_I, [_P, _P, _P, _P, _P, _P, _I, _I64, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P,
                                 _I, _I64, _P, _SZ, _I, _P]),
@@ -763,3 +767,43 @@ def hca_compress_step_blocked(proj_new, state, bias, pos, blocks, layout):
     _check(_lib.hca_compress_step_blocked(_ptr(proj_new), _ptr(state), _ptr(bias), _ptr(pos), B, c, mp, nblk * rpb,
                                           blocks.data_ptr() + layout["hca_offset"], rpb, layout["block_bytes"],
                                           CSA_BF16, _stream()))
+
+
+# ---------------------------------------------------------------- FP8 KV
+def csa_quantize_kv_fp8(kv, rope_dims: int = 64):
+    """KV entries [..., c] bf16 into FP8 storage: (codes [..., c-R] uint8,
+    scales [...] fp32, rope [..., R] bf16)."""
+    _dtype(kv, torch.bfloat16, "kv")
+    c = kv.shape[-1]
+    rows = kv.numel() // c if c else 0
+    lead = tuple(kv.shape[:-1])
+    codes = torch.empty(lead + (c - rope_dims,), dtype=torch.uint8, device=kv.device)
+    scales = torch.empty(lead, dtype=torch.float32, device=kv.device)
+    rope = torch.empty(lead + (rope_dims,), dtype=torch.bfloat16, device=kv.device)
+    _check(_lib.csa_quantize_kv_fp8(_ptr(kv.contiguous()), rows, c, rope_dims, _ptr(codes), _ptr(scales),
+                                    _ptr(rope) if rope_dims else None, _stream()))
+    return codes, scales, rope
+
+
+def csa_decode_fp8kv(qI, w, idx_cache, q, kv_codes, kv_scales, kv_rope, ctx_len, m: int, k: int, scale: float = 0.0,
+                     sink=None, out=None, lse=None, topk_idx=None, ws=None, return_topk: bool = False):
+    """csa_decode with the KV entries in FP8 storage (csa_quantize_kv_fp8)."""
+    B, HI, cI = qI.shape
+    _, H, c = q.shape
+    Nmax = idx_cache.shape[1]
+    R = kv_rope.shape[-1]
+    _shape(kv_codes, (B, Nmax, c - R), "kv_codes")
+    _shape(kv_scales, (B, Nmax), "kv_scales")
+    _shape(kv_rope, (B, Nmax, R), "kv_rope")
+    _dtype(kv_codes, torch.uint8, "kv_codes")
+    _dtype(kv_scales, torch.float32, "kv_scales")
+    out = torch.empty_like(q) if out is None else out
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    if return_topk and topk_idx is None:
+        topk_idx = torch.empty((B, k), dtype=torch.int32, device=q.device)
+    ws = _ws(_lib.csa_decode_fp8kv_workspace_size(B, Nmax, H, c, HI, cI, k), q.device, ws)
+    _check(_lib.csa_decode_fp8kv(_ptr(qI), _ptr(w), _ptr(idx_cache), _ptr(q), _ptr(kv_codes), _ptr(kv_scales),
+                                 _ptr(kv_rope), _ptr(ctx_len), B, Nmax, m, H, c, R, HI, cI, k, scale, _ptr(sink),
+                                 _ptr(out), _ptr(lse), _ptr(topk_idx), _ptr(ws), _nbytes(ws), _stream()))
+    return (out, lse, topk_idx) if return_topk else (out, lse)

@@ -619,6 +619,30 @@ int csa_quantize_e4m3(const void* x, int64_t rows, int cols, void* out, float* s
     return CSA_OK;
 }
 
+// ---------------------------------------------------------------- FP8 KV
+static int check_kv_fp8(int c, int rope_dims, const char* who) {
+    if (rope_dims < 0 || rope_dims % 16 || c % 16 || c - rope_dims < 16 || c > CSA_MAX_HEAD_DIM)
+        return fail(CSA_ERR_INVALID_ARG, "%s: c=%d rope_dims=%d (c and rope_dims multiples of 16, at least 16 "
+                    "quantised dims, c <= %d)", who, c, rope_dims, CSA_MAX_HEAD_DIM);
+    return CSA_OK;
+}
+
+int csa_quantize_kv_fp8(const void* kv, int64_t rows, int c, int rope_dims, uint8_t* codes, float* scales,
+                        void* rope, void* stream) {
+    CSA_TRY(check_kv_fp8(c, rope_dims, "csa_quantize_kv_fp8"));
+    if (rows < 0) return fail(CSA_ERR_INVALID_ARG, "csa_quantize_kv_fp8: rows=%lld", (long long)rows);
+    if ((rows + 7) / 8 > INT32_MAX) return fail(CSA_ERR_UNSUPPORTED, "rows beyond one launch");
+    if (rows == 0) return CSA_OK;
+    CSA_TRY(check_ptr(kv, "kv"));
+    CSA_TRY(check_ptr(codes, "codes"));
+    CSA_TRY(check_ptr(scales, "scales"));
+    CSA_TRY(check_ptr(rope, "rope", rope_dims > 0));
+    CSA_CUDA(quantize_e4m3(kv, rows, c - rope_dims, codes, scales, nullptr, nullptr, ElemType::BF16,
+                           (cudaStream_t)stream, c, rope_dims ? rope : nullptr, rope_dims),
+             "csa_quantize_kv_fp8");
+    return CSA_OK;
+}
+
 static int check_index_fp8(int HI, int cI) {
     CSA_TRY(check_index_shape(HI, cI));
     if (!index_tc_supported(HI, cI, 1, true))
@@ -857,6 +881,66 @@ int csa_decode_blocked(const void* qI, const float* w, const void* idx_cache, co
 
 size_t hca_decode_workspace_size(int B, int64_t Nmax, int H, int c, int dtype) {
     return hca_dense_mqa_workspace_size(B, H, c, Nmax, dtype);
+}
+
+size_t csa_decode_fp8kv_workspace_size(int B, int64_t Nmax, int H, int c, int HI, int cI, int k) {
+    (void)HI; (void)cI;
+    if (B < 0 || Nmax < 0 || k < 1 || H < 1 || c < 1) return 0;
+    return index_topk_bytes(B, Nmax, k) + align256((size_t)B * k * sizeof(int32_t)) +
+           align256((size_t)B * k * c * sizeof(uint16_t)) + align256((size_t)B * k * sizeof(int32_t)) +
+           mqa_workspace_bytes(B, H, c, k, ElemType::BF16);
+}
+
+int csa_decode_fp8kv(const void* qI, const float* w, const void* idx_cache, const void* q, const uint8_t* kv_codes,
+                     const float* kv_scales, const void* kv_rope, const int32_t* ctx_len, int B, int64_t Nmax, int m,
+                     int H, int c, int rope_dims, int HI, int cI, int k, float scale, const float* sink, void* out,
+                     float* lse, int32_t* topk_idx, void* ws, size_t ws_bytes, void* stream) {
+    CSA_TRY(check_kv_fp8(c, rope_dims, "csa_decode_fp8kv"));
+    CSA_TRY(check_index_shape(HI, cI));
+    CSA_TRY(check_index_mode(HI, cI, ElemType::BF16));
+    CSA_TRY(check_attn_shape(H, c));
+    CSA_TRY(check_attn_mode(H, c, ElemType::BF16));
+    CSA_TRY(check_cache_rows(B, Nmax));
+    CSA_TRY(check_k(k));
+    CSA_TRY(check_rows(B, "csa_decode_fp8kv"));
+    if (B < 0 || Nmax < 0 || m < 1) return fail(CSA_ERR_INVALID_ARG, "bad B/Nmax/m");
+    if (Nmax > INT32_MAX) return fail(CSA_ERR_UNSUPPORTED, "Nmax beyond int32 entry indices");
+    if (B == 0) return CSA_OK;
+    CSA_TRY(check_ptr(qI, "qI"));
+    CSA_TRY(check_ptr(w, "w"));
+    CSA_TRY(check_ptr(idx_cache, "idx_cache", Nmax > 0));
+    CSA_TRY(check_ptr(q, "q"));
+    CSA_TRY(check_ptr(kv_codes, "kv_codes", Nmax > 0));
+    CSA_TRY(check_ptr(kv_scales, "kv_scales", Nmax > 0));
+    CSA_TRY(check_ptr(kv_rope, "kv_rope", Nmax > 0 && rope_dims > 0));
+    CSA_TRY(check_ptr(ctx_len, "ctx_len"));
+    CSA_TRY(check_ptr(sink, "sink", false));
+    CSA_TRY(check_ptr(out, "out"));
+    CSA_TRY(check_ptr(lse, "lse", false));
+    CSA_TRY(check_ptr(topk_idx, "topk_idx", false));
+    CSA_TRY(check_ws(ws, ws_bytes, csa_decode_fp8kv_workspace_size(B, Nmax, H, c, HI, cI, k)));
+    cudaStream_t st = (cudaStream_t)stream;
+    const ElemType t = ElemType::BF16;
+    Carve cv(ws);
+    float* sc = (float*)cv.take((size_t)B * Nmax * sizeof(float));
+    void* tws = cv.take(topk_workspace_bytes(B, Nmax, k));
+    int32_t* sel = (int32_t*)cv.take((size_t)B * k * sizeof(int32_t));
+    void* rows = cv.take((size_t)B * k * c * sizeof(uint16_t));
+    int32_t* slots = (int32_t*)cv.take((size_t)B * k * sizeof(int32_t));
+    void* mws = cv.take(mqa_workspace_bytes(B, H, c, k, t));
+    if (topk_idx) sel = topk_idx;
+    QuerySpec qs{nullptr, ctx_len, 0, 0};
+    CSA_CUDA(run_indexer(qI, w, idx_cache, qs, B, B, HI, cI, Nmax, m, sc, Nmax, 1, false, t, st),
+             "csa_decode_fp8kv: indexer");
+    CSA_CUDA(topk_select(sc, Nmax, ctx_len, m, B, Nmax, k, sel, nullptr, tws, st), "csa_decode_fp8kv: top-k");
+    // the selected entries, dequantised into one row list per query; the
+    // attention then runs on those rows (query t over "sequence" t of k rows)
+    CSA_CUDA(gather_kv_fp8(kv_codes, kv_scales, kv_rope, sel, B, k, Nmax, c, rope_dims, rows, slots, st),
+             "csa_decode_fp8kv: dequantise the selection");
+    QuerySpec qs_rows{nullptr, ctx_len, 0, 0};
+    CSA_CUDA(mqa(q, rows, slots, k, qs_rows, 1, B, B, H, c, k, default_scale(scale, c), sink, out, lse, mws, t, st),
+             "csa_decode_fp8kv: mqa");
+    return CSA_OK;
 }
 
 int hca_decode(const void* q, const void* kv_cache, const int32_t* ctx_len, int B, int64_t Nmax,

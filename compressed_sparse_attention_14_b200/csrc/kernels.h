@@ -175,7 +175,13 @@ cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, Query
 // s = max|row| / 448 (1 for a zero row), decided in fp64; w_out = w * s when
 // w is given (one head weight per row).
 cudaError_t quantize_e4m3(const void* x, int64_t rows, int cols, void* out, float* scale, const float* w, float* w_out,
-                          ElemType t, cudaStream_t st);
+                          ElemType t, cudaStream_t st, int64_t ld = 0, void* rope = nullptr, int rope_dims = 0);
+// FP8 KV entries of a selection dequantised into bf16 rows out [nq, k, c]
+// (codes [n_seq*Nmax, c-R] e4m3, scales [n_seq*Nmax], rope [n_seq*Nmax, R]
+// bf16; query t reads sequence t); idx_out [nq, k]: i for a selected slot,
+// -1 for an empty one.
+cudaError_t gather_kv_fp8(const uint8_t* codes, const float* scales, const void* rope, const int32_t* idx, int nq,
+                          int k, int64_t Nmax, int c, int rope_dims, void* out, int32_t* idx_out, cudaStream_t st);
 
 // api.cu: device address of the status word on the current device
 int* device_status();

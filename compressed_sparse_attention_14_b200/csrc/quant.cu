@@ -49,16 +49,21 @@ __device__ __forceinline__ uint8_t e4m3_code(double v) {
     return (uint8_t)(sign | code);
 }
 
+// x rows of `ld` values; the first `cols` are quantised. rope (rows of
+// rope_dims, the cache dtype) gets the row's values cols .. cols+rope_dims-1
+// unchanged when given (the rotary dims of an FP8 KV entry).
 template <typename TIn>
 __global__ void __launch_bounds__(256) quantize_e4m3_kernel(const TIn* __restrict__ x, int64_t rows, int cols,
-                                                            uint8_t* __restrict__ out, float* __restrict__ scale,
-                                                            const float* __restrict__ w, float* __restrict__ w_out) {
+                                                            int64_t ld, uint8_t* __restrict__ out,
+                                                            float* __restrict__ scale, const float* __restrict__ w,
+                                                            float* __restrict__ w_out, TIn* __restrict__ rope,
+                                                            int rope_dims) {
     pdl_wait();
     pdl_launch_next();
     const int lane = threadIdx.x & 31;
     const int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
     if (r >= rows) return;
-    const TIn* row = x + r * cols;
+    const TIn* row = x + r * ld;
     double amax = 0.0;
     for (int j = lane * 8; j < cols; j += 256) {
         float v[8];
@@ -83,23 +88,101 @@ __global__ void __launch_bounds__(256) quantize_e4m3_kernel(const TIn* __restric
         scale[r] = (float)s;
         if (w) w_out[r] = w[r] * (float)s;
     }
+    if (rope)
+        for (int j = lane * 8; j < rope_dims; j += 256) {
+            float v[8];
+            load8(row + cols + j, v);
+            if constexpr (sizeof(TIn) == 2) store8(reinterpret_cast<bf16*>(rope + r * rope_dims + j), v);
+            else store8(reinterpret_cast<float*>(rope + r * rope_dims + j), v);
+        }
+}
+
+// The value of an e4m3 code, from the format's definition (sign, 4 exponent
+// bits with bias 7, 3 mantissa bits; exponent field 0: subnormal).
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+    const uint32_t ef = (code >> 3) & 15u, mf = code & 7u;
+    const float mag = ef ? ldexpf(1.f + (float)mf * 0.125f, (int)ef - 7) : ldexpf((float)mf * 0.125f, -6);
+    return (code & 0x80u) ? -mag : mag;
+}
+
+// FP8 KV entries of the selection, dequantised to bf16 rows: out[t][i] =
+// entry idx[t][i] of sequence t (bf16(code * scale) for the first c - R
+// dims, the bf16 rotary dims after them), idx_out[t][i] = i for a selected
+// entry, -1 for an empty slot (its row is zero). A warp per slot, 16 dims
+// per lane.
+__global__ void __launch_bounds__(256) gather_kv_fp8_kernel(const uint8_t* __restrict__ codes,
+                                                            const float* __restrict__ scales,
+                                                            const bf16* __restrict__ rope, const int32_t* __restrict__ idx,
+                                                            int nq, int k, int64_t Nmax, int c, int rope_dims,
+                                                            bf16* __restrict__ out, int32_t* __restrict__ idx_out) {
+    pdl_wait();
+    pdl_launch_next();
+    const int lane = threadIdx.x & 31;
+    const int64_t slot = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    if (slot >= (int64_t)nq * k) return;
+    const int64_t t = slot / k;
+    const int i = (int)(slot - t * k);
+    const int e = idx[slot];
+    const bool ok = e >= 0 && e < Nmax;
+    if (lane == 0) idx_out[slot] = ok ? i : -1;
+    const int cq = c - rope_dims;
+    const int64_t R = t * Nmax + (ok ? e : 0);
+    const float s = ok ? scales[R] : 0.f;
+    bf16* orow = out + slot * c;
+    for (int j = lane * 16; j < c; j += 512) {
+        float v[16];
+        if (!ok) {
+#pragma unroll
+            for (int u = 0; u < 16; ++u) v[u] = 0.f;
+        } else if (j < cq) {
+            const uint4 q = *reinterpret_cast<const uint4*>(codes + R * cq + j);
+            const uint32_t wd[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int u = 0; u < 16; ++u) v[u] = e4m3_value((wd[u >> 2] >> (8 * (u & 3))) & 255u) * s;
+        } else {
+            float a[8], b[8];
+            load8(rope + R * rope_dims + (j - cq), a);
+            load8(rope + R * rope_dims + (j - cq) + 8, b);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) { v[u] = a[u]; v[8 + u] = b[u]; }
+        }
+        float lo[8], hi[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) { lo[u] = v[u]; hi[u] = v[8 + u]; }
+        store8(orow + j, lo);
+        store8(orow + j + 8, hi);
+    }
 }
 
 }  // namespace
 
 cudaError_t quantize_e4m3(const void* x, int64_t rows, int cols, void* out, float* scale, const float* w, float* w_out,
-                          ElemType t, cudaStream_t st) {
+                          ElemType t, cudaStream_t st, int64_t ld, void* rope, int rope_dims) {
     if (rows == 0) return cudaSuccess;
+    if (ld == 0) ld = cols;
     const dim3 grid((unsigned)((rows + 7) / 8));
     cudaError_t e = cudaSuccess;
     if (t == ElemType::BF16)
         CSA_LAUNCH(st, "quantize_e4m3",
-                   e = launch_pdl(quantize_e4m3_kernel<bf16>, grid, dim3(256), 0, st, 0, (const bf16*)x, rows, cols,
-                                  (uint8_t*)out, scale, w, w_out));
+                   e = launch_pdl(quantize_e4m3_kernel<bf16>, grid, dim3(256), 0, st, 0, (const bf16*)x, rows, cols, ld,
+                                  (uint8_t*)out, scale, w, w_out, (bf16*)rope, rope_dims));
     else
         CSA_LAUNCH(st, "quantize_e4m3",
                    e = launch_pdl(quantize_e4m3_kernel<float>, grid, dim3(256), 0, st, 0, (const float*)x, rows, cols,
-                                  (uint8_t*)out, scale, w, w_out));
+                                  ld, (uint8_t*)out, scale, w, w_out, (float*)rope, rope_dims));
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+cudaError_t gather_kv_fp8(const uint8_t* codes, const float* scales, const void* rope, const int32_t* idx, int nq,
+                          int k, int64_t Nmax, int c, int rope_dims, void* out, int32_t* idx_out, cudaStream_t st) {
+    const int64_t slots = (int64_t)nq * k;
+    if (slots == 0) return cudaSuccess;
+    const dim3 grid((unsigned)((slots + 7) / 8));
+    cudaError_t e = cudaSuccess;
+    CSA_LAUNCH(st, "gather_kv_fp8",
+               e = launch_pdl(gather_kv_fp8_kernel, grid, dim3(256), 0, st, 0, codes, scales, (const bf16*)rope, idx,
+                              nq, k, Nmax, c, rope_dims, (bf16*)out, idx_out));
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -321,6 +321,31 @@ int csa_decode_fp8(const void* qI, const float* w, const void* idx_cache8, const
                    int cI, int k, float scale, const float* sink, int flags, void* out, float* lse, int32_t* topk_idx,
                    void* ws, size_t ws_bytes, void* stream);
 
+/* FP8 KV storage with bf16 rotary dims [Notes §1.3 and §2.4: compressed
+ * entries stored in FP8 except the rotary dims, which stay BF16]. An entry
+ * row x of c values (bf16) becomes: codes [c - R] e4m3 with one fp32 scale
+ * s = max|x[0 .. c-R)| / 448 (1 for an all-zero part), decided in fp64 as
+ * csa_quantize_e4m3 does, and its last R = rope_dims values unchanged (bf16).
+ * In attention the entry is bf16(code * s) for the first c - R dims (the
+ * product in fp32) and the stored rotary values after them.
+ *
+ * csa_quantize_kv_fp8: kv [rows, c] bf16 -> codes [rows, c-R] u8, scales
+ * [rows] fp32, rope [rows, R] bf16 (may be NULL when R == 0). c and R
+ * multiples of 16, c - R >= 16. */
+int csa_quantize_kv_fp8(const void* kv, int64_t rows, int c, int rope_dims, uint8_t* codes, float* scales,
+                        void* rope, void* stream);
+
+/* csa_decode_fp8kv: csa_decode (bf16 index keys, bf16 out) with the KV
+ * entries in FP8 storage: kv_codes [B, Nmax, c-R], kv_scales [B, Nmax],
+ * kv_rope [B, Nmax, R] as csa_quantize_kv_fp8 writes them. The selected
+ * entries are dequantised into the workspace (k rows per query) and the
+ * sparse MQA runs on those rows; the selection equals csa_decode's. */
+size_t csa_decode_fp8kv_workspace_size(int B, int64_t Nmax, int H, int c, int HI, int cI, int k);
+int csa_decode_fp8kv(const void* qI, const float* w, const void* idx_cache, const void* q, const uint8_t* kv_codes,
+                     const float* kv_scales, const void* kv_rope, const int32_t* ctx_len, int B, int64_t Nmax, int m,
+                     int H, int c, int rope_dims, int HI, int cI, int k, float scale, const float* sink, void* out,
+                     float* lse, int32_t* topk_idx, void* ws, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * a6. Sparse shared-KV MQA [Notes §1.1 last paragraph: every compressed
  * entry is both key and value, all query heads share it; Walk §2.3.2; sink

@@ -149,6 +149,26 @@ def index_scores_fp8(qI, w, K, pos, m: int, seq=None) -> np.ndarray:
     return index_scores(q8, w, k8, pos, m, seq=seq)
 
 
+def quantize_kv_fp8(KV, rope_dims: int):
+    """FP8 KV storage with bf16 rotary dims [Notes §1.3 and §2.4]: each entry
+    row's first c - R values get one scale s = max|x| / 448 (1 for an
+    all-zero part) and are stored as the e4m3 values nearest x / s; the last
+    R values are kept as they are. Returns (codes [..., c-R] as the e4m3
+    values, float64; scales [...]; rope [..., R])."""
+    KV = _f64(KV)
+    c = KV.shape[-1]
+    q = KV[..., :c - rope_dims]
+    amax = np.abs(q).max(axis=-1) if q.shape[-1] else np.zeros(q.shape[:-1])
+    s = np.where(amax > 0, amax / 448.0, 1.0)
+    codes = e4m3_round(q / s[..., None])
+    return codes, s, KV[..., c - rope_dims:].copy()
+
+
+def dequantize_kv_fp8(codes, scales, rope):
+    """The entries attention sees: code * s (exact), then the rotary values."""
+    return np.concatenate([_f64(codes) * _f64(scales)[..., None], _f64(rope)], axis=-1)
+
+
 def topk_recall(idx, ref_idx) -> float:
     """Mean over rows of |idx ∩ ref_idx| / |ref_idx| (entries >= 0 only)."""
     idx, ref_idx = _i32(idx), _i32(ref_idx)

@@ -11,6 +11,10 @@
   rule, and its attention output matches the oracle on the GPU's selection.
 * Recall of the FP8 selection against the exact (bf16-operand) top-k is
   reported and held to >= 0.9 on these inputs (N(0,1) keys and queries).
+* FP8 KV storage (bf16 rotary dims): codes bit-exact and scales equal as for
+  the indexer operands, rotary dims copied; the FP8-KV decode selects exactly
+  what csa_decode selects (same indexer and top-k) and its output matches the
+  oracle's attention over the dequantised entries within the bf16 tolerance.
 """
 import math
 
@@ -162,3 +166,43 @@ def test_decode_fp8_with_bf16_scores(csa):
     rec_bf = oracle.topk_recall(oracle.topk(_bf16_round(S), (ctx.numpy() // m).astype(np.int32), k), exact)
     print(f"FP8 indexer + bf16 scores recall@{k} vs exact: {rec:.4f} (exact scores rounded to bf16: {rec_bf:.4f})")
     assert rec >= 0.9
+
+
+@pytest.mark.parametrize("c,R", [(512, 64), (128, 32)])
+def test_quantize_kv_fp8_matches_the_oracle(csa, c, R):
+    g = torch.Generator().manual_seed(61)
+    KV = (torch.randn(3, 70, c, generator=g) * torch.exp(torch.randn(3, 70, 1, generator=g) * 2)).to(torch.bfloat16)
+    KV[1, 5, :c - R] = 0.0
+    codes, scales, rope = csa.csa_quantize_kv_fp8(KV.to(DEV), rope_dims=R)
+    ref_codes, ref_s, ref_rope = oracle.quantize_kv_fp8(KV.float().double().numpy(), R)
+    np.testing.assert_array_equal(_codes_to_f64(codes), ref_codes)
+    np.testing.assert_array_equal(scales.cpu().numpy(), ref_s.astype(np.float32))
+    assert torch.equal(rope.cpu(), KV[..., c - R:])
+
+
+@pytest.mark.parametrize("B,Nmax,H,c,R,HI,cI,k", [(4, 1024, 64, 512, 64, 64, 128, 256), (3, 512, 128, 256, 32, 32, 64, 96)])
+def test_decode_fp8kv_selection_and_output(csa, B, Nmax, H, c, R, HI, cI, k):
+    m = 4
+    g = torch.Generator().manual_seed(62)
+    KV = torch.randn(B, Nmax, c, generator=g).to(torch.bfloat16)
+    K = torch.randn(B, Nmax, cI, generator=g).to(torch.bfloat16)
+    qI = torch.randn(B, HI, cI, generator=g).to(torch.bfloat16)
+    w = torch.softmax(torch.randn(B, HI, generator=g), -1)
+    q = torch.randn(B, H, c, generator=g).to(torch.bfloat16)
+    sink = torch.randn(H, generator=g)
+    ctx = torch.randint(m, Nmax * m + 1, (B,), generator=g, dtype=torch.int32)
+    ctx[0] = Nmax * m
+    ctx[-1] = 2 * m + 1          # fewer entries than k
+    dev = dict(KV=KV.to(DEV), K=K.to(DEV), qI=qI.to(DEV), w=w.to(DEV), q=q.to(DEV), sink=sink.to(DEV), ctx=ctx.to(DEV))
+    codes, scales, rope = csa.csa_quantize_kv_fp8(dev["KV"], rope_dims=R)
+    out, lse, sel = csa.csa_decode_fp8kv(dev["qI"], dev["w"], dev["K"], dev["q"], codes, scales, rope, dev["ctx"], m, k,
+                                         sink=dev["sink"], return_topk=True)
+    _, _, sel_bf16 = csa.csa_decode(dev["qI"], dev["w"], dev["K"], dev["q"], dev["KV"], dev["ctx"], m, k,
+                                    sink=dev["sink"], return_topk=True)
+    assert torch.equal(sel, sel_bf16), "the FP8-KV decode selects what csa_decode selects"
+    rc, rs, rr = oracle.quantize_kv_fp8(KV.float().double().numpy(), R)
+    KVd = oracle.dequantize_kv_fp8(rc, rs, rr)
+    ref_o, ref_l = oracle.sparse_mqa(q.float().double().numpy(), KVd, host(sel), 1 / math.sqrt(c),
+                                     sink=sink.double().numpy(), seq=np.arange(B))
+    assert_close(out, ref_o, torch.bfloat16, "fp8-kv decode out")
+    assert_close(lse, ref_l, torch.bfloat16, "fp8-kv decode lse")

@@ -628,6 +628,31 @@ def test_e4m3_round_matches_torch_on_every_bf16_value_in_range():
     np.testing.assert_array_equal(oracle.e4m3_round(r.double().numpy()), r.to(torch.float8_e4m3fn).double().numpy())
 
 
+def test_fp8_kv_storage_pins():
+    # rotary dims untouched; each entry's largest quantised magnitude exact;
+    # every other value within half an e4m3 step (2^-4 relative for normal
+    # codes, 2^-10 * s for subnormal ones); an all-zero part gets s = 1
+    R, c = 16, 64
+    KV = rng.standard_normal((5, 7, c)) * np.exp(rng.uniform(-6, 6, (5, 7, 1)))
+    KV[0, 0, :c - R] = 0.0
+    codes, s, rope = oracle.quantize_kv_fp8(KV, R)
+    np.testing.assert_array_equal(rope, KV[..., c - R:])
+    assert s[0, 0] == 1.0 and not codes[0, 0].any()
+    x = KV[..., :c - R]
+    deq = oracle.dequantize_kv_fp8(codes, s, rope)
+    np.testing.assert_array_equal(deq[..., c - R:], KV[..., c - R:])
+    amax = np.abs(x).max(-1)
+    got_max = np.abs(deq[..., :c - R]).max(-1)
+    np.testing.assert_allclose(got_max, amax, rtol=1e-15, atol=0)
+    err = np.abs(deq[..., :c - R] - x)
+    normal = np.abs(codes) >= 2.0 ** -6
+    bound = np.where(normal, 2.0 ** -4 * np.abs(x) * (1 + 1e-12), 2.0 ** -10 * s[..., None] * (1 + 1e-12))
+    assert (err <= bound).all()
+    # the codes are e4m3 values (what torch's conversion gives on x / s)
+    want = torch.from_numpy((x / s[..., None]).astype(np.float32)).to(torch.float8_e4m3fn).double().numpy()
+    np.testing.assert_array_equal(codes, want)
+
+
 def test_e4m3_round_by_hand():
     cases = {1.0625: 1.0,           # tie between 1 and 1.125: even mantissa
              1.1875: 1.25,          # tie between 1.125 and 1.25
