@@ -46,6 +46,7 @@ import sys
 import tempfile
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -710,8 +711,8 @@ def oracle_measure(workload: str, budget_s: float = 15.0):
             if sec >= budget_s / 3 or n >= shape.batch:
                 break
             n *= 2
-        desc = (f"first {units} of the {shape.batch} decode queries (indexer{' on e4m3 operands' if fp8 else ''} "
-                f"+ top-k + sparse MQA, fp64)")
+        desc = (f"first {units} of the {shape.batch} decode queries (indexer{' on e4m3 operands' if fp8 is True else ''} "
+                f"+ top-k + sparse MQA{' on FP8-stored entries' if fp8 == 'kv' else ''}, fp64)")
     elif workload == "flash_attend_decode":
         shape = synth.FLASH_DECODE
         n = max(1, threads // 2)

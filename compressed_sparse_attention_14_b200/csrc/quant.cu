@@ -100,16 +100,23 @@ __global__ void __launch_bounds__(256) quantize_e4m3_kernel(const TIn* __restric
 // The value of an e4m3 code, from the format's definition (sign, 4 exponent
 // bits with bias 7, 3 mantissa bits; exponent field 0: subnormal).
 __device__ __forceinline__ float e4m3_value(uint32_t code) {
+    // normal codes (exponent field 1..15): 2^(e-7) * (1 + m/8), assembled
+    // as fp32 bits (exponent e - 7 + 127, the 3 mantissa bits on top);
+    // subnormals (field 0): m * 2^-9
     const uint32_t ef = (code >> 3) & 15u, mf = code & 7u;
-    const float mag = ef ? ldexpf(1.f + (float)mf * 0.125f, (int)ef - 7) : ldexpf((float)mf * 0.125f, -6);
+    const float mag = ef ? __uint_as_float(((ef + 120u) << 23) | (mf << 20)) : (float)mf * 0.001953125f;
     return (code & 0x80u) ? -mag : mag;
 }
 
 // FP8 KV entries of the selection, dequantised to bf16 rows: out[t][i] =
 // entry idx[t][i] of sequence t (bf16(code * scale) for the first c - R
 // dims, the bf16 rotary dims after them), idx_out[t][i] = i for a selected
-// entry, -1 for an empty slot (its row is zero). A warp per slot, 16 dims
-// per lane.
+// entry, -1 for an empty slot (its row is zero). A warp takes kGatherSlots
+// consecutive slots, 16 dims per lane: all the slots' indices are loaded,
+// then all their scales and 16-byte pieces, then converted and stored, so
+// that each lane has several loads in flight instead of one.
+constexpr int kGatherSlots = 1;
+
 __global__ void __launch_bounds__(256) gather_kv_fp8_kernel(const uint8_t* __restrict__ codes,
                                                             const float* __restrict__ scales,
                                                             const bf16* __restrict__ rope, const int32_t* __restrict__ idx,
@@ -118,39 +125,61 @@ __global__ void __launch_bounds__(256) gather_kv_fp8_kernel(const uint8_t* __res
     pdl_wait();
     pdl_launch_next();
     const int lane = threadIdx.x & 31;
-    const int64_t slot = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-    if (slot >= (int64_t)nq * k) return;
-    const int64_t t = slot / k;
-    const int i = (int)(slot - t * k);
-    const int e = idx[slot];
-    const bool ok = e >= 0 && e < Nmax;
-    if (lane == 0) idx_out[slot] = ok ? i : -1;
+    const int64_t nslots = (int64_t)nq * k;
+    const int64_t slot0 = ((int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5)) * kGatherSlots;
+    if (slot0 >= nslots) return;
     const int cq = c - rope_dims;
-    const int64_t R = t * Nmax + (ok ? e : 0);
-    const float s = ok ? scales[R] : 0.f;
-    bf16* orow = out + slot * c;
+    int64_t R[kGatherSlots];
+    bool ok[kGatherSlots];
+#pragma unroll
+    for (int u = 0; u < kGatherSlots; ++u) {
+        const int64_t slot = slot0 + u;
+        const bool in = slot < nslots;
+        const int e = in ? __ldg(idx + slot) : -1;
+        const int64_t t = in ? slot / k : 0;
+        ok[u] = e >= 0 && e < Nmax;
+        R[u] = t * Nmax + (ok[u] ? e : 0);
+        if (in && lane == 0) idx_out[slot] = ok[u] ? (int)(slot - t * k) : -1;
+    }
     for (int j = lane * 16; j < c; j += 512) {
-        float v[16];
-        if (!ok) {
+        uint4 lo[kGatherSlots], hi[kGatherSlots];
+        float s[kGatherSlots];
 #pragma unroll
-            for (int u = 0; u < 16; ++u) v[u] = 0.f;
-        } else if (j < cq) {
-            const uint4 q = *reinterpret_cast<const uint4*>(codes + R * cq + j);
-            const uint32_t wd[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-            for (int u = 0; u < 16; ++u) v[u] = e4m3_value((wd[u >> 2] >> (8 * (u & 3))) & 255u) * s;
-        } else {
-            float a[8], b[8];
-            load8(rope + R * rope_dims + (j - cq), a);
-            load8(rope + R * rope_dims + (j - cq) + 8, b);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) { v[u] = a[u]; v[8 + u] = b[u]; }
+        for (int u = 0; u < kGatherSlots; ++u) {
+            lo[u] = hi[u] = make_uint4(0, 0, 0, 0);
+            s[u] = 0.f;
+            if (!ok[u]) continue;
+            if (j < cq) {
+                s[u] = __ldg(scales + R[u]);
+                lo[u] = __ldg(reinterpret_cast<const uint4*>(codes + R[u] * cq + j));
+            } else {
+                const uint4* p = reinterpret_cast<const uint4*>(rope + R[u] * rope_dims + (j - cq));
+                lo[u] = __ldg(p);
+                hi[u] = __ldg(p + 1);
+            }
         }
-        float lo[8], hi[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) { lo[u] = v[u]; hi[u] = v[8 + u]; }
-        store8(orow + j, lo);
-        store8(orow + j + 8, hi);
+        for (int u = 0; u < kGatherSlots; ++u) {
+            const int64_t slot = slot0 + u;
+            if (slot >= nslots) break;
+            bf16* orow = out + slot * c + j;
+            if (j < cq) {
+                // 16 codes -> 16 bf16 values, written as two 16-byte stores
+                const uint32_t wd[4] = {lo[u].x, lo[u].y, lo[u].z, lo[u].w};
+                float v[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) v[q] = e4m3_value((wd[q >> 2] >> (8 * (q & 3))) & 255u) * s[u];
+                float a[8], b[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) { a[q] = v[q]; b[q] = v[8 + q]; }
+                store8(orow, a);
+                store8(orow + 8, b);
+            } else {
+                // the rotary dims are bf16 already (zeros for an empty slot)
+                reinterpret_cast<uint4*>(orow)[0] = lo[u];
+                reinterpret_cast<uint4*>(orow)[1] = hi[u];
+            }
+        }
     }
 }
 
@@ -178,7 +207,7 @@ cudaError_t gather_kv_fp8(const uint8_t* codes, const float* scales, const void*
                           int k, int64_t Nmax, int c, int rope_dims, void* out, int32_t* idx_out, cudaStream_t st) {
     const int64_t slots = (int64_t)nq * k;
     if (slots == 0) return cudaSuccess;
-    const dim3 grid((unsigned)((slots + 7) / 8));
+    const dim3 grid((unsigned)((slots + 8 * kGatherSlots - 1) / (8 * kGatherSlots)));
     cudaError_t e = cudaSuccess;
     CSA_LAUNCH(st, "gather_kv_fp8",
                e = launch_pdl(gather_kv_fp8_kernel, grid, dim3(256), 0, st, 0, codes, scales, (const bf16*)rope, idx,
