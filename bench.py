@@ -305,6 +305,9 @@ def decode_workload(shape, rank, batch=None, fp8=False, fp8kv=False):
     idx_name = "index_scores_tc_fp8" if fp8 else "index_scores_tc"
     kernels = {
         idx_name: dict(bound="hbm", work=idx_kernel_bytes, files=("indexer_tc.cu", "tc.cuh", "common.cuh")),
+        # the indexer with the top-k filter on its epilogue: the same reads, no
+        # score block (its candidate lists are a few percent of the scores)
+        "index_topk_filter_tc": dict(bound="hbm", work=idx_bytes, files=("indexer_tc.cu", "tc.cuh", "common.cuh")),
         "mqa_tc": dict(bound="hbm", work=mqa_bytes, files=("mqa_tc.cu", "tc.cuh", "common.cuh")),
         # one pass over each row's visible scores, k indices out
         "topk_select": dict(bound="hbm", work=v_sum * score_bytes + B * s.k * 4, files=("topk.cu",)),
@@ -380,6 +383,8 @@ def attend_decode_workload(shape, rank, batch=None):
     d2h = out_h.numel() * out_h.element_size()
     kernels = {
         "index_scores_tc": dict(bound="hbm", work=idx_kernel_bytes, files=("indexer_tc.cu", "tc.cuh", "common.cuh")),
+        "index_topk_filter_tc": dict(bound="hbm", work=idx_kernel_bytes - v_sum * 4,
+                                     files=("indexer_tc.cu", "tc.cuh", "common.cuh")),
         "mqa_tc": dict(bound="hbm", work=B * ke * s.c * 2 + 2 * qo, files=("mqa_tc.cu", "tc.cuh", "common.cuh")),
         "topk_select": dict(bound="hbm", work=v_sum * 4 + B * s.k * 4, files=("topk.cu",)),
         # two launches per step (query in, output back): each one read and one write of [B, H, c]
@@ -570,6 +575,8 @@ def prefill_workload(rank, tokens=None):
     mqa_flops = 4.0 * n * s.heads * s.k * s.c
     proj_flops = 2.0 * (n + s.m) * s.d * 4 * (s.c + s.idx_dim)
     kernels = {"index_scores_tc": dict(bound="tensor", work=idx_flops, files=("indexer_tc.cu", "tc.cuh", "common.cuh")),
+               "index_topk_filter_tc": dict(bound="tensor", work=idx_flops,
+                                            files=("indexer_tc.cu", "tc.cuh", "common.cuh")),
                "mqa_tc": dict(bound="tensor", work=mqa_flops, files=("mqa_tc.cu", "tc.cuh", "common.cuh")),
                "project_tc": dict(bound="tensor", work=proj_flops, files=("gemm_tc.cu", "tc.cuh", "common.cuh"))}
     return dict(step=step, e2e_step=e2e_step, units=n, unit="tokens/s",
@@ -980,6 +987,9 @@ def measure(name, args, rank, world, local, steps, warmup, batch=None):
         r["traffic"] = ncu_traffic(kname, name, info["files"])
         return r
 
+    if "index_topk_filter_tc" in wl["kernels"]:
+        wl["config"]["selection"] = ("top-k filter on the indexer epilogue, exact selection over its candidates"
+                                     if "index_topk_filter_tc" in trace else "fp32 score block, then top-k")
     timed = [n for n in wl["kernels"] if n in trace]
     dom = max(timed, key=lambda n: trace[n][0]) if timed else next(iter(wl["kernels"]))
     others = {n: roofline_of(n) for n in timed if n != dom}
@@ -1012,6 +1022,9 @@ EXTRA_WORKLOADS = {"pro_decode": 20, "prefill": 5, "hca_decode": 20, "hca_compre
 
 
 def run_ours(args, rank, world, local):
+    import compressed_sparse_attention_14_b200 as csa
+    if args.topk_filter:
+        csa.debug_set(0, csa.CSA_DEBUG_TOPK_FILTER)
     m = measure(args.workload, args, rank, world, local, args.steps, args.warmup, args.batch)
     line = {"metric": METRIC, "value": m["value"], "unit": m["unit"], "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True, "scaling": "weak",
@@ -1045,6 +1058,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
     ap.add_argument("--no-extra", action="store_true",
                     help="default workload only: skip the extra_workloads (Pro decode, prefill, HCA) measured after it")
+    ap.add_argument("--topk-filter", action="store_true",
+                    help="select through the top-k filter on the indexer epilogue instead of the fp32 score block "
+                         "(comparison runs)")
     ap.add_argument("--batch", type=int, default=None,
                     help="decode workloads: only the first N queries; prefill: only the last N tokens of the "
                          "chunk, a multiple of m (small profiling cases)")

@@ -25,6 +25,8 @@ CSA_OK, CSA_ERR_INVALID_ARG, CSA_ERR_UNSUPPORTED, CSA_ERR_WORKSPACE, CSA_ERR_CUD
 CSA_BF16, CSA_FP32 = 0, 1
 CSA_SCORES_BF16 = 1
 CSA_DEBUG_SKIP_FIRST_TILE = 1
+CSA_DEBUG_SCORE_BLOCK = 2
+CSA_DEBUG_TOPK_FILTER = 4
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "

@@ -161,6 +161,52 @@ static size_t index_topk_bytes(int nq, int64_t Nmax, int k) {
     return align256((size_t)nq * (size_t)Nmax * sizeof(float)) + topk_workspace_bytes(nq, Nmax, k);
 }
 
+// The selection stage of csa_decode / csa_prefill: the indexer's top-k filter
+// (candidate lists [nq][Nmax] of 64-bit keys + their lengths) where it
+// applies, else the fp32 score block; the workspace holds either.
+static size_t select_bytes(int nq, int64_t Nmax, int k) {
+    const size_t cand = align256((size_t)nq * (size_t)Nmax * sizeof(uint64_t)) + align256((size_t)nq * sizeof(uint32_t));
+    const size_t block = index_topk_bytes(nq, Nmax, k);
+    return cand > block ? cand : block;
+}
+
+// The filter is opt-in (CSA_DEBUG_TOPK_FILTER): measured on B200 it makes the
+// selection cheaper (long prefill: 7.1 -> 2.5 ms of top-k, 3.9 K candidates
+// per 50 K-score row) but the indexer slower (59 -> 74-82 ms), because the
+// prefill indexer is paced by its epilogue and every per-tile instruction
+// there adds to the tile time; decode rows are split over several CTAs,
+// whose bounds stay weak.
+static bool use_topk_filter(ElemType t, int HI, int cI, int group, int k) {
+    const uint32_t f = debug_flags();
+    return t == ElemType::BF16 && (f & CSA_DEBUG_TOPK_FILTER) && !(f & CSA_DEBUG_SCORE_BLOCK) &&
+           index_cand_supported(HI, cI, group, k);
+}
+
+// indexer -> top-k for nq queries into sel, through the filter (blk holds
+// select_bytes) or the score block
+static cudaError_t index_then_select(const void* qI, const float* w, const void* K, QuerySpec qs, int nq, int n_seq,
+                                     int HI, int cI, int64_t Nmax, int m, int group, int k, int32_t* sel, void* blk,
+                                     ElemType t, cudaStream_t st, RowBlocks kb, const char*& step) {
+    if (kb.rpb == 0 && use_topk_filter(t, HI, cI, group, k)) {
+        uint64_t* cand = (uint64_t*)blk;
+        uint32_t* cnt = (uint32_t*)((char*)blk + align256((size_t)nq * (size_t)Nmax * sizeof(uint64_t)));
+        step = "indexer with top-k filter";
+        cudaError_t e = index_scores_tc(qI, w, K, qs, nq, n_seq, HI, cI, Nmax, m, nullptr, Nmax, group, false,
+                                        device_status(), st, nullptr, false, RowBlocks{0, 0},
+                                        CandOut{cand, cnt, Nmax, k});
+        if (e != cudaSuccess) return e;
+        step = "top-k of the candidates";
+        return topk_from_candidates(cand, cnt, Nmax, nq, k, sel, nullptr, st);
+    }
+    float* sc = (float*)blk;
+    step = "indexer";
+    cudaError_t e = run_indexer(qI, w, K, qs, nq, n_seq, HI, cI, Nmax, m, sc, Nmax, group, false, t, st, kb);
+    if (e != cudaSuccess) return e;
+    step = "top-k";
+    if (qs.pos) return topk_select(sc, Nmax, qs.pos, m, nq, Nmax, k, sel, nullptr, nullptr, st);
+    return topk_select_positions(sc, Nmax, qs.pos_base, m, nq, Nmax, k, sel, nullptr, st);
+}
+
 static int64_t prefill_query_chunk(int64_t n, int64_t Nmax, int m) {
     // bound the fp32 score block of one query chunk to 1 GiB; whole
     // compressed blocks (multiples of m tokens) and at most 65535 queries
@@ -810,8 +856,7 @@ size_t csa_decode_workspace_size(int B, int64_t Nmax, int H, int c, int HI, int 
     (void)HI; (void)cI;
     ElemType t = dtype == CSA_FP32 ? ElemType::F32 : ElemType::BF16;
     if (B < 0 || Nmax < 0 || k < 1 || H < 1 || c < 1) return 0;
-    return index_topk_bytes(B, Nmax, k) + align256((size_t)B * k * sizeof(int32_t)) +
-           mqa_workspace_bytes(B, H, c, k, t);
+    return select_bytes(B, Nmax, k) + align256((size_t)B * k * sizeof(int32_t)) + mqa_workspace_bytes(B, H, c, k, t);
 }
 
 static int csa_decode_impl(const void* qI, const float* w, const void* idx_cache, const void* q,
@@ -843,15 +888,15 @@ static int csa_decode_impl(const void* qI, const float* w, const void* idx_cache
     CSA_TRY(check_ws(ws, ws_bytes, csa_decode_workspace_size(B, Nmax, H, c, HI, cI, k, dtype)));
     cudaStream_t st = (cudaStream_t)stream;
     Carve cv(ws);
-    float* sc = (float*)cv.take((size_t)B * Nmax * sizeof(float));
-    void* tws = cv.take(topk_workspace_bytes(B, Nmax, k));
+    void* blk = cv.take(select_bytes(B, Nmax, k));
     int32_t* sel = (int32_t*)cv.take((size_t)B * k * sizeof(int32_t));
     void* mws = cv.take(mqa_workspace_bytes(B, H, c, k, t));
     if (topk_idx) sel = topk_idx;
     QuerySpec qs{nullptr, ctx_len, 0, 0};
-    CSA_CUDA(run_indexer(qI, w, idx_cache, qs, B, B, HI, cI, Nmax, m, sc, Nmax, 1, false, t, st, cb),
-             "csa_decode: indexer");
-    CSA_CUDA(topk_select(sc, Nmax, ctx_len, m, B, Nmax, k, sel, nullptr, tws, st), "csa_decode: top-k");
+    const char* step = "indexer";
+    const cudaError_t se = index_then_select(qI, w, idx_cache, qs, B, B, HI, cI, Nmax, m, 1, k, sel, blk, t, st, cb,
+                                             step);
+    if (se != cudaSuccess) return fail(CSA_ERR_CUDA, "csa_decode: %s: %s", step, cudaGetErrorString(se));
     CSA_CUDA(mqa(q, kv_cache, sel, k, qs, 1, B, B, H, c, Nmax, default_scale(scale, c), sink, out, lse, mws, t, st,
                  cb),
              "csa_decode: mqa");
@@ -886,7 +931,7 @@ size_t hca_decode_workspace_size(int B, int64_t Nmax, int H, int c, int dtype) {
 size_t csa_decode_fp8kv_workspace_size(int B, int64_t Nmax, int H, int c, int HI, int cI, int k) {
     (void)HI; (void)cI;
     if (B < 0 || Nmax < 0 || k < 1 || H < 1 || c < 1) return 0;
-    return index_topk_bytes(B, Nmax, k) + align256((size_t)B * k * sizeof(int32_t)) +
+    return select_bytes(B, Nmax, k) + align256((size_t)B * k * sizeof(int32_t)) +
            align256((size_t)B * k * c * sizeof(uint16_t)) + align256((size_t)B * k * sizeof(int32_t)) +
            mqa_workspace_bytes(B, H, c, k, ElemType::BF16);
 }
@@ -922,17 +967,17 @@ int csa_decode_fp8kv(const void* qI, const float* w, const void* idx_cache, cons
     cudaStream_t st = (cudaStream_t)stream;
     const ElemType t = ElemType::BF16;
     Carve cv(ws);
-    float* sc = (float*)cv.take((size_t)B * Nmax * sizeof(float));
-    void* tws = cv.take(topk_workspace_bytes(B, Nmax, k));
+    void* blk = cv.take(select_bytes(B, Nmax, k));
     int32_t* sel = (int32_t*)cv.take((size_t)B * k * sizeof(int32_t));
     void* rows = cv.take((size_t)B * k * c * sizeof(uint16_t));
     int32_t* slots = (int32_t*)cv.take((size_t)B * k * sizeof(int32_t));
     void* mws = cv.take(mqa_workspace_bytes(B, H, c, k, t));
     if (topk_idx) sel = topk_idx;
     QuerySpec qs{nullptr, ctx_len, 0, 0};
-    CSA_CUDA(run_indexer(qI, w, idx_cache, qs, B, B, HI, cI, Nmax, m, sc, Nmax, 1, false, t, st),
-             "csa_decode_fp8kv: indexer");
-    CSA_CUDA(topk_select(sc, Nmax, ctx_len, m, B, Nmax, k, sel, nullptr, tws, st), "csa_decode_fp8kv: top-k");
+    const char* step = "indexer";
+    const cudaError_t se = index_then_select(qI, w, idx_cache, qs, B, B, HI, cI, Nmax, m, 1, k, sel, blk, t, st,
+                                             RowBlocks{0, 0}, step);
+    if (se != cudaSuccess) return fail(CSA_ERR_CUDA, "csa_decode_fp8kv: %s: %s", step, cudaGetErrorString(se));
     // the selected entries, dequantised into one row list per query; the
     // attention then runs on those rows (query t over "sequence" t of k rows)
     CSA_CUDA(gather_kv_fp8(kv_codes, kv_scales, kv_rope, sel, B, k, Nmax, c, rope_dims, rows, slots, st),
@@ -969,7 +1014,7 @@ size_t csa_prefill_workspace_size(int64_t n, int64_t Nmax, int d, int m, int c, 
     const int cw = c > cI ? c : cI;
     int64_t qc = prefill_query_chunk(n, Nmax, m);
     size_t b = align256((size_t)n * 4 * cw * sizeof(float)) + align256((size_t)m * 4 * cw * sizeof(float));
-    b += index_topk_bytes((int)qc, Nmax, k) + align256((size_t)qc * k * sizeof(int32_t));
+    b += select_bytes((int)qc, Nmax, k) + align256((size_t)qc * k * sizeof(int32_t));
     b += mqa_workspace_bytes((int)qc, H, c, k, t);
     return b;
 }
@@ -1035,8 +1080,7 @@ int csa_prefill(const void* x, const void* x_left, const void* W_kv, const float
     Carve cv(ws);
     float* proj = (float*)cv.take((size_t)n * 4 * cw * sizeof(float));
     float* lproj = (float*)cv.take((size_t)m * 4 * cw * sizeof(float));
-    float* sc = (float*)cv.take((size_t)qc * Nmax * sizeof(float));
-    void* tws = cv.take(topk_workspace_bytes((int)qc, Nmax, k));
+    void* blk = cv.take(select_bytes((int)qc, Nmax, k));
     int32_t* sel_ws = (int32_t*)cv.take((size_t)qc * k * sizeof(int32_t));
     void* mws = cv.take(mqa_workspace_bytes((int)qc, H, c, k, t));
 
@@ -1073,11 +1117,12 @@ int csa_prefill(const void* x, const void* x_left, const void* W_kv, const float
         // together against each key tile when the group fits one MMA (the
         // group starts on a block boundary)
         const int group = (m <= 4 && (start + q0) % m == 0 && index_tc_supported(HI, cI, m)) ? m : 1;
-        CSA_CUDA(run_indexer((const char*)qI + (size_t)q0 * HI * cI * es, w + q0 * HI, idx_cache, qs, nqc, 1, HI,
-                             cI, Nmax, m, sc, Nmax, group, false, t, st), "csa_prefill: indexer");
-        // visible count of query t is floor((start + q0 + t) / m); pass it through a
-        // position-based valid rule: the top-k kernel reads valid[] = positions
-        CSA_CUDA(topk_select_positions(sc, Nmax, start + q0, m, nqc, Nmax, k, sel, tws, st), "csa_prefill: top-k");
+        // the visible count of query t is floor((start + q0 + t) / m)
+        const char* step = "indexer";
+        const cudaError_t se = index_then_select((const char*)qI + (size_t)q0 * HI * cI * es, w + q0 * HI, idx_cache,
+                                                 qs, nqc, 1, HI, cI, Nmax, m, group, k, sel, blk, t, st,
+                                                 RowBlocks{0, 0}, step);
+        if (se != cudaSuccess) return fail(CSA_ERR_CUDA, "csa_prefill: %s: %s", step, cudaGetErrorString(se));
         CSA_CUDA(mqa((const char*)q + (size_t)q0 * H * c * es, kv_cache, sel, k, qs, 1, nqc, 1, H, c, Nmax,
                      sc_scale, sink, (char*)out + (size_t)q0 * H * c * es, lse ? lse + q0 * H : nullptr, mws,
                      t, st), "csa_prefill: mqa");
@@ -1151,7 +1196,7 @@ size_t csa_attend_decode_workspace_size(int B, int64_t Nmax, int64_t ring_len, i
     ElemType t = dtype == CSA_FP32 ? ElemType::F32 : ElemType::BF16;
     if (B < 0 || Nmax < 0 || k < 1 || n_win < 0 || H < 1 || c < 1) return 0;
     const int ke = k + n_win;
-    return index_topk_bytes(B, Nmax, k) + align256((size_t)B * k * sizeof(int32_t)) +
+    return select_bytes(B, Nmax, k) + align256((size_t)B * k * sizeof(int32_t)) +
            align256((size_t)B * ke * sizeof(int32_t)) + align256((size_t)B * H * c * elem_size(t)) +
            mqa_workspace_bytes(B, H, c, ke, t);
 }
@@ -1193,8 +1238,7 @@ int csa_attend_decode(const void* qI, const float* w, const void* idx_cache, con
     cudaStream_t st = (cudaStream_t)stream;
     const int ke = k + n_win;
     Carve cv(ws);
-    float* sc = (float*)cv.take((size_t)B * Nmax * sizeof(float));
-    void* tws = cv.take(topk_workspace_bytes(B, Nmax, k));
+    void* blk = cv.take(select_bytes(B, Nmax, k));
     int32_t* sel = (int32_t*)cv.take((size_t)B * k * sizeof(int32_t));
     int32_t* ent = (int32_t*)cv.take((size_t)B * ke * sizeof(int32_t));
     void* qn = cv.take((size_t)B * H * c * elem_size(t));
@@ -1205,9 +1249,10 @@ int csa_attend_decode(const void* qI, const float* w, const void* idx_cache, con
     if (prep_q)
         CSA_CUDA(norm_rope(q, qn, (int64_t)B * H, H, c, q_gamma, eps, rope_dims, (double)rope_base, ctx_len, 0, 0, 0,
                            t, st), "csa_attend_decode: query norm/rotary");
-    CSA_CUDA(run_indexer(qI, w, idx_cache, qs, B, B, HI, cI, Nmax, m, sc, Nmax, 1, false, t, st),
-             "csa_attend_decode: indexer");
-    CSA_CUDA(topk_select(sc, Nmax, ctx_len, m, B, Nmax, k, sel, nullptr, tws, st), "csa_attend_decode: top-k");
+    const char* step = "indexer";
+    const cudaError_t se = index_then_select(qI, w, idx_cache, qs, B, B, HI, cI, Nmax, m, 1, k, sel, blk, t, st,
+                                             RowBlocks{0, 0}, step);
+    if (se != cudaSuccess) return fail(CSA_ERR_CUDA, "csa_attend_decode: %s: %s", step, cudaGetErrorString(se));
     CSA_CUDA(window_entries(sel, k, ctx_len, 0, B, n_win, Nmax, ring_len > 0 ? ring_len : 1, ent, st),
              "csa_attend_decode: window entries");
     CSA_CUDA(mqa(prep_q ? qn : q, kv_cache, ent, ke, qs, 1, B, B, H, c, rows, default_scale(scale, c), sink, out,

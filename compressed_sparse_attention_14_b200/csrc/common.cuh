@@ -26,6 +26,23 @@ __device__ __forceinline__ void report_device_error(int* status, int code) {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_next() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// ---- selection order (top-k): score descending, then column ascending
+// orderable() maps fp32 to uint32 monotonically (-0.0 folded into +0.0);
+// the composite key (orderable(score) << 32) | (0xFFFFFFFF - column) is
+// distinct per column and its descending order is the selection order.
+__device__ __forceinline__ uint32_t orderable(float f) {
+    uint32_t u = __float_as_uint(f);
+    if (u == 0x80000000u) u = 0u;  // -0.0 == +0.0
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float from_orderable(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+__device__ __forceinline__ uint64_t composite_key(uint32_t key, int64_t col) {
+    return ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)col);
+}
+__device__ __forceinline__ uint64_t composite(float s, int64_t col) { return composite_key(orderable(s), col); }
+
 // ---- element conversion -------------------------------------------------
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(bf16 v) { return __bfloat162float(v); }

@@ -38,6 +38,29 @@
 // they leave the ReLU: sum_h w_h ReLU(sq_h sk x_h) = sk sum_h (w_h sq_h)
 // ReLU(x_h). The caller passes w_h sq_h as the head weights and the key
 // scales; the epilogue multiplies each key's sum by its scale.
+//
+// Top-k filter on the epilogue [Notes §1.1: the indexer's scores choose each
+// query's k entries] (bf16, contiguous keys): instead of storing every
+// score, the epilogue appends to the query's candidate list only the scores
+// that can still be among its k largest, as 64-bit composite keys (order
+// key << 32 | ~column); a small selection over the lists finishes the top-k.
+// Per query it scores, each epilogue warp queues the scores that reach the
+// current bound in shared memory (a ballot and one 8-byte store per taker:
+// no global atomics in the per-tile path). Every 32 queued entries make a
+// batch, one entry per lane: each lane inserts its entry's order key into a
+// list of the kCandR largest keys it has been handed, the batch is reserved
+// in the row's global list with one addition (whose result is first needed
+// at the next batch, so its latency hides) and stored as 256 contiguous
+// bytes. The warp then finds p_w, a lower bound of the kk-th largest key in
+// its lanes' lists (kk = ceil(k / warps scoring the query)), and publishes
+// it in shared memory: the listed keys belong to distinct columns, so at
+// least k scores of the row reach min_w p_w over the warps scoring the
+// query, which is therefore at most the row's k-th largest score. A score
+// below the bound can never be selected; every other one is kept. The bound
+// only rises, it is local to the CTA (a row split over two CTAs gets two
+// valid bounds), and a row's list never holds more entries than it has
+// visible columns. The bound is only tight when a CTA scores long stretches
+// of a row (many rows per launch).
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -78,6 +101,10 @@ struct IdxArgs {
     int nbuf;           // TMEM accumulator buffers (2..4)
     int kpt;            // keys per tile: kKeys, or 2 * kKeys (FP8 decode: a
                         // 32 KB stage, so per-tile costs spread over 256 keys)
+    uint64_t* cand;     // candidate lists [nq][cand_ld] (top-k filter), else nullptr
+    uint32_t* cand_cnt; // [nq] entries appended to each list (zeroed before the launch)
+    int64_t cand_ld;
+    uint32_t cand_kk;   // keys each publishing warp vouches for: ceil(k / warps per query)
 };
 
 struct Smem {
@@ -91,6 +118,7 @@ struct Smem {
     uint64_t* qfull;
     uint64_t* qempty;
     uint64_t* fin;
+    uint8_t* cq;        // top-k filter: [8 warps][1-2 query slots] queue and lists (kCandSlotBytes each)
 };
 
 __device__ __forceinline__ Smem carve(uint8_t* base, const IdxArgs& a) {
@@ -106,6 +134,7 @@ __device__ __forceinline__ Smem carve(uint8_t* base, const IdxArgs& a) {
     s.qfull = s.tempty + 4;
     s.qempty = s.qfull + 1;
     s.fin = s.qempty + 1;
+    s.cq = (uint8_t*)(bars + 64);
     return s;
 }
 
@@ -264,6 +293,101 @@ __device__ __forceinline__ void head_reduce(uint32_t taddr, const float* wv, int
     }
 }
 
+// ---- top-k filter helpers
+constexpr int kCandR = 8;                  // order keys each thread keeps per query
+constexpr uint32_t kTagNone = 0xFFFFFFFFu; // no bound published yet
+
+// Insert order key u into the descending list t (u = 0 leaves it as it is).
+__device__ __forceinline__ void cand_insert(uint32_t (&t)[kCandR], uint32_t u) {
+#pragma unroll
+    for (int i = 0; i < kCandR; ++i) {
+        const uint32_t hi = max(t[i], u);
+        u = min(t[i], u);
+        t[i] = hi;
+    }
+}
+// A lane's list lives in shared memory ([i][lane]: conflict-free), loaded
+// into registers only while a batch is handled.
+__device__ __forceinline__ void list_load(const uint32_t* l, int lane, uint32_t (&t)[kCandR]) {
+#pragma unroll
+    for (int i = 0; i < kCandR; ++i) t[i] = l[i * 32 + lane];
+}
+__device__ __forceinline__ void list_store(uint32_t* l, int lane, const uint32_t (&t)[kCandR]) {
+#pragma unroll
+    for (int i = 0; i < kCandR; ++i) l[i * 32 + lane] = t[i];
+}
+
+// The largest multiple of 2^16 that at least kk keys of the warp's lists
+// reach (0 when fewer are listed): a lower bound of the warp's kk-th largest
+// listed key, digit by digit from the top bit (16 rounds, one warp sum each).
+__device__ __forceinline__ uint32_t warp_kth_bound(const uint32_t (&t)[kCandR], uint32_t kk) {
+    uint32_t p = 0;
+#pragma unroll 1
+    for (int b = 31; b >= 16; --b) {
+        const uint32_t c = p | (1u << b);
+        uint32_t n = 0;
+#pragma unroll
+        for (int i = 0; i < kCandR; ++i) n += t[i] >= c ? 1u : 0u;
+        if (__reduce_add_sync(0xffffffffu, n) >= kk) p = c;
+    }
+    return p;
+}
+
+constexpr int kCandQueue = 64;              // queued entries per (warp, query): a batch + one tile
+// per (epilogue warp, query slot): the queue, then the lanes' lists
+constexpr uint32_t kCandSlotBytes = kCandQueue * sizeof(uint64_t) + kCandR * 32 * sizeof(uint32_t);
+
+// One warp's filter state for one query (qn, nb, pend_n and pend_row are
+// the same in every lane; pend_base lives in lane 0).
+struct CandState {
+    uint32_t tau;           // the bound in force
+    int qn;                 // entries in the queue
+    int nb;                 // batches handled for the current row
+    int pend_n;             // entries of the last batch still to store
+    uint32_t pend_base;     // their reservation (lane 0)
+    uint64_t pend_x;        // this lane's entry of that batch
+    uint64_t* pend_row;
+};
+
+__device__ __forceinline__ void cand_reset(CandState& st, uint32_t* list, int lane) {
+#pragma unroll
+    for (int i = 0; i < kCandR; ++i) list[i * 32 + lane] = 0u;
+    st.tau = 0u;
+    st.qn = 0;
+    st.nb = 0;
+}
+
+// The stores of the last batch (its reservation was issued a batch earlier).
+__device__ __forceinline__ void cand_complete(CandState& st, int64_t cap, int lane) {
+    if (st.pend_n == 0) return;
+    const uint32_t b = __shfl_sync(0xffffffffu, st.pend_base, 0);
+    if (lane < st.pend_n && (int64_t)b + lane < cap) st.pend_row[b + lane] = st.pend_x;
+    st.pend_n = 0;
+}
+
+// The first n (<= 32) queued entries as a batch: into the lanes' lists
+// (left in t), the previous batch stored, this one reserved in the row's
+// list, the rest of the queue moved to its front.
+__device__ __forceinline__ void cand_batch(CandState& st, uint64_t* qb, uint32_t* list, int n, uint64_t* row,
+                                           uint32_t* cnt, int64_t cap, int lane, uint32_t (&t)[kCandR]) {
+    __syncwarp();
+    const uint64_t x = lane < n ? qb[lane] : 0ull;
+    list_load(list, lane, t);
+    cand_insert(t, (uint32_t)(x >> 32));
+    list_store(list, lane, t);
+    ++st.nb;
+    cand_complete(st, cap, lane);
+    if (lane == 0) st.pend_base = atomicAdd(cnt, (uint32_t)n);
+    st.pend_x = x;
+    st.pend_n = n;
+    st.pend_row = row;
+    const int rest = st.qn - n;
+    const uint64_t y = lane < rest ? qb[n + lane] : 0ull;
+    __syncwarp();
+    if (lane < rest) qb[lane] = y;
+    st.qn = rest;
+}
+
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                               int* status, uint32_t limit) {
     for (uint32_t i = 0; i < limit; ++i) {
@@ -278,8 +402,9 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 }  // namespace
 
 // kBlk: the keys come in blocks (a 3D key map); a separate instantiation, so
-// that the contiguous path's producer loop stays as it was
-template <bool kFp8, int kN, int kHI, int kH, bool kBlk = false>
+// that the contiguous path's producer loop stays as it was. kCand: the top-k
+// filter replaces the score stores (bf16, one 128-key half per tile).
+template <bool kFp8, int kN, int kHI, int kH, bool kBlk = false, bool kCand = false>
 __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __grid_constant__ IdxArgs a,
                                                                       const __grid_constant__ CUtensorMap tmK,
                                                                       const __grid_constant__ CUtensorMap tmQ) {
@@ -288,6 +413,9 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
     Smem sm = carve(base, a);
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
+    // top-k filter: [query of the group][epilogue warp] = (group << 32) | bound
+    __shared__ uint64_t s_pub[4 * 8];
+    static_assert(!kCand || (!kFp8 && kH == 1), "the top-k filter runs on bf16 tiles of 128 keys");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ngroups = (a.nq + a.group - 1) / a.group;
@@ -301,6 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
         tc::mbar_init(sm.fin, kIssuers);
         tc::fence_mbar_init();
         s_abort = 0;
+        for (int i = 0; i < 4 * 8; ++i) s_pub[i] = (uint64_t)kTagNone << 32;
     }
     if (warp == 1) {
         tc::tmem_alloc(&s_tmem, a.tmem_cols);
@@ -452,6 +581,34 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
         int cur = -1;
         int64_t vis = 0;
         RingPos bf(a.nbuf);
+        // top-k filter: this warp's queries (the grouped prefill: its set's
+        // two; otherwise one) and their queues
+        constexpr int kQ = kN == 256 ? 2 : 1;
+        CandState cst[kQ];
+        uint8_t* cslot = sm.cq + (size_t)(warp - 2) * kQ * kCandSlotBytes;
+        auto cq_of = [&](int q) { return reinterpret_cast<uint64_t*>(cslot + q * kCandSlotBytes); };
+        auto cl_of = [&](int q) {
+            return reinterpret_cast<uint32_t*>(cslot + q * kCandSlotBytes + kCandQueue * sizeof(uint64_t));
+        };
+        uint32_t ctop[kCandR];
+        if constexpr (kCand) {
+#pragma unroll
+            for (int q = 0; q < kQ; ++q) {
+                cand_reset(cst[q], cl_of(q), lane);
+                cst[q].pend_n = 0;
+                cst[q].pend_base = 0;
+                cst[q].pend_x = 0;
+                cst[q].pend_row = nullptr;
+            }
+        }
+        // the row of this warp's query slot gs in group g (nullptr: none)
+        auto cand_row = [&](int g, int gs, uint32_t*& cnt) -> uint64_t* {
+            const int gq = kN == 256 ? 2 * set + gs : gs;
+            const int tq = g * a.group + gq;
+            if (g < 0 || gq >= a.group || tq >= a.nq) return nullptr;
+            cnt = a.cand_cnt + tq;
+            return a.cand + (int64_t)tq * a.cand_ld;
+        };
         for (int64_t it = 0; it < my; ++it, wk.next(a, ngroups), bf.advance()) {
             if (kN != 256 && (int)(it & 1) != set) continue;
             if (wk.g != cur) {
@@ -462,6 +619,17 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
                     wv[c] = (gq < a.group && tq < a.nq) ? a.w[(int64_t)tq * a.HI + h] : 0.f;
                 }
                 __syncwarp();
+                if constexpr (kCand) {
+                    // the previous group's queued entries go out before its state is reset
+#pragma unroll
+                    for (int q = 0; q < kQ; ++q) {
+                        uint32_t* cnt = nullptr;
+                        uint64_t* rowp = cand_row(cur, q, cnt);
+                        if (rowp && cst[q].qn > 0)
+                            cand_batch(cst[q], cq_of(q), cl_of(q), cst[q].qn, rowp, cnt, a.cand_ld, lane, ctop);
+                        cand_reset(cst[q], cl_of(q), lane);
+                    }
+                }
                 cur = wk.g;
                 vis = group_visible(a, wk.g);
             }
@@ -497,6 +665,47 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&sm.tempty[buf]);
+            if constexpr (kCand) {
+                const bool in = key[0] < vis;
+                const int c0 = kN == 256 ? 4 * set : 0;          // warps scoring this warp's queries
+                constexpr int nc = kN == 256 ? 4 : 8;
+#pragma unroll
+                for (int gs = 0; gs < kQ; ++gs) {
+                    uint32_t* cnt = nullptr;
+                    uint64_t* rowp = cand_row(wk.g, gs, cnt);
+                    if (!rowp) continue;                            // the same for the whole warp
+                    CandState& st = cst[gs];
+                    uint64_t* qb = cq_of(gs);
+                    const uint32_t u = in ? orderable(sc[0][gs]) : 0u;
+                    const bool take = in && u >= st.tau;
+                    const unsigned mk = __ballot_sync(0xffffffffu, take);
+                    if (!mk) continue;
+                    if (take) qb[st.qn + __popc(mk & ((1u << lane) - 1u))] = composite_key(u, key[0]);
+                    st.qn += __popc(mk);
+                    if (st.qn < 32) continue;
+                    cand_batch(st, qb, cl_of(gs), 32, rowp, cnt, a.cand_ld, lane, ctop);
+                    // publish this warp's bound (after batches 1, 2, 4, then
+                    // every fourth: it rises fastest early in the row) and take
+                    // the minimum over the warps scoring the query once all of
+                    // them have published for it
+                    if ((st.nb & (st.nb - 1)) != 0 && (st.nb & 3) != 0) continue;
+                    const int gq = kN == 256 ? 2 * set + gs : gs;
+                    const uint32_t p = warp_kth_bound(ctop, a.cand_kk);
+                    volatile uint64_t* slots = s_pub + gq * 8;
+                    if (lane == 0) slots[warp - 2] = ((uint64_t)(uint32_t)wk.g << 32) | p;
+                    __syncwarp();
+                    uint32_t lo = 0xFFFFFFFFu;
+                    bool all = true;
+#pragma unroll
+                    for (int j = 0; j < nc; ++j) {
+                        const uint64_t v = slots[c0 + j];
+                        all = all && (uint32_t)(v >> 32) == (uint32_t)wk.g;
+                        lo = min(lo, (uint32_t)v);
+                    }
+                    if (all) st.tau = max(st.tau, lo);
+                }
+                continue;
+            }
 #pragma unroll
             for (int hh = 0; hh < kH; ++hh) {
                 if (key[hh] >= vis) continue;
@@ -512,6 +721,17 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
                             a.scores[(int64_t)tq * a.ld + key[hh]] = v;
                     }
                 }
+            }
+        }
+        if constexpr (kCand) {
+            // the last group's queued entries, then every pending store
+#pragma unroll
+            for (int q = 0; q < kQ; ++q) {
+                uint32_t* cnt = nullptr;
+                uint64_t* rowp = cand_row(cur, q, cnt);
+                if (rowp && cst[q].qn > 0)
+                    cand_batch(cst[q], cq_of(q), cl_of(q), cst[q].qn, rowp, cnt, a.cand_ld, lane, ctop);
+                cand_complete(cst[q], a.cand_ld, lane);
             }
         }
     }
@@ -547,6 +767,18 @@ static int num_sms() {
     return n;
 }
 
+// warps whose lanes score one query: the 4 of its set in the grouped
+// prefill instantiation, all 8 elsewhere (the sets alternate tiles)
+static int cand_warps(int HI, int group) { return (HI == 64 && group == 4) ? 4 : 8; }
+
+bool index_cand_supported(int HI, int cI, int group, int k) {
+    // one query per epilogue warp, or the grouped prefill's two
+    if (!index_tc_supported(HI, cI, group, false) || k < 1 || !(group == 1 || (HI == 64 && group == 4)))
+        return false;
+    const int w = cand_warps(HI, group);
+    return (k + w - 1) / w <= 32 * kCandR;
+}
+
 bool index_tc_supported(int HI, int cI, int group, bool fp8) {
     if (cI % (fp8 ? 128 : 64) != 0 || cI > 256) return false;
     if (group < 1 || group > 4) return false;
@@ -557,12 +789,21 @@ bool index_tc_supported(int HI, int cI, int group, bool fp8) {
 
 cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, QuerySpec qs, int nq, int n_seq, int HI,
                             int cI, int64_t Nmax, int m, float* scores, int64_t ld, int group, bool fill_invisible,
-                            int* status, cudaStream_t st, const float* kscale, bool score_bf16, RowBlocks kb) {
+                            int* status, cudaStream_t st, const float* kscale, bool score_bf16, RowBlocks kb,
+                            CandOut co) {
     if (score_bf16 && fill_invisible) return cudaErrorInvalidValue;
     const bool fp8 = kscale != nullptr;
+    const bool cand = co.cand != nullptr;
+    if (cand && (fp8 || score_bf16 || fill_invisible || kb.rpb > 0 || !co.cnt || co.ld < Nmax ||
+                 !index_cand_supported(HI, cI, group, co.k)))
+        return cudaErrorInvalidValue;
     // keys in blocks: bf16 only, whole blocks per 128-key tile and per sequence
     if (kb.rpb > 0 && (fp8 || kKeys % kb.rpb || Nmax % kb.rpb || kb.block_bytes % 16)) return cudaErrorInvalidValue;
     const int es = fp8 ? 1 : 2;
+    if (cand && nq > 0) {
+        const cudaError_t ze = cudaMemsetAsync(co.cnt, 0, (size_t)nq * sizeof(uint32_t), st);
+        if (ze != cudaSuccess) return ze;
+    }
     if (nq == 0 || Nmax == 0) return cudaSuccess;
     IdxArgs a{};
     a.qm = QueryMap{qs.seq, qs.pos, qs.pos_base, qs.single_seq};
@@ -585,6 +826,13 @@ cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, Query
     a.skip_first_tile = (debug_flags() & CSA_DEBUG_SKIP_FIRST_TILE) ? 1 : 0;
     a.ld = ld;
     a.status = status;
+    if (cand) {
+        a.cand = co.cand;
+        a.cand_cnt = co.cnt;
+        a.cand_ld = co.ld;
+        const int cw = cand_warps(HI, group);
+        a.cand_kk = (uint32_t)((co.k + cw - 1) / cw);
+    }
     // FP8 decode (one query of at most 128 heads per MMA): tiles of 256 keys
     const int kh = (fp8 && group == 1 && n <= 128) ? 2 : 1;
     a.kpt = kh * kKeys;
@@ -597,7 +845,8 @@ cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, Query
     uint32_t cols = 32;
     while (cols < (uint32_t)(a.nbuf * kh * a.npad)) cols <<= 1;
     a.tmem_cols = cols;
-    const size_t fixed = 1024 + a.q_bytes + 8 * 256 * sizeof(float) + 64 * sizeof(uint64_t);
+    const size_t fixed = 1024 + a.q_bytes + 8 * 256 * sizeof(float) + 64 * sizeof(uint64_t) +
+                         (cand ? (size_t)8 * (group == 4 ? 2 : 1) * kCandSlotBytes : 0);
     const size_t budget = 226 * 1024;
     int stages = (int)((budget - fixed) / a.stage_bytes);
     if (stages > (fp8 ? 12 : 8)) stages = fp8 ? 12 : 8;
@@ -641,9 +890,14 @@ cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, Query
     if (a.key_rpb)   // bf16 keys in blocks (decode shape, or any other)
         kern = (a.npad == 64 && HI == 64 && group == 1) ? index_scores_tc_kernel<false, 64, 64, 1, true>
                                                           : index_scores_tc_kernel<false, 0, 0, 1, true>;
+    if (cand) {
+        if (a.npad == 64 && HI == 64 && group == 1) kern = index_scores_tc_kernel<false, 64, 64, 1, false, true>;
+        else if (a.npad == 256 && HI == 64 && group == 4) kern = index_scores_tc_kernel<false, 256, 64, 1, false, true>;
+        else kern = index_scores_tc_kernel<false, 0, 0, 1, false, true>;
+    }
     e = smem_ceiling(kern);
     if (e != cudaSuccess) return e;
-    CSA_LAUNCH(st, fp8 ? "index_scores_tc_fp8" : "index_scores_tc",
+    CSA_LAUNCH(st, fp8 ? "index_scores_tc_fp8" : (cand ? "index_topk_filter_tc" : "index_scores_tc"),
                e = launch_pdl(kern, dim3(num_sms()), dim3(kThreads), smem, st, 0, a, tmK, tmQ));
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

@@ -164,12 +164,24 @@ cudaError_t index_scores(const void* qI, const float* w, const void* K, QuerySpe
 // score_bf16: scores are stored as bf16 (nearest, ties to even), row stride
 // ld bf16 values (no fill_invisible).
 bool index_tc_supported(int HI, int cI, int group, bool fp8 = false);
+// Top-k filter on the indexer epilogue: instead of the score block, each
+// query's scores that can still be among its k largest are appended to
+// cand[t * ld ...] as 64-bit composite keys (order key << 32 | ~column),
+// cnt[t] counting them (at most the row's visible columns; ld >= Nmax). The
+// kernel zeroes cnt first. bf16 operands, contiguous keys.
+struct CandOut {
+    uint64_t* cand = nullptr;
+    uint32_t* cnt = nullptr;
+    int64_t ld = 0;
+    int k = 0;
+};
+bool index_cand_supported(int HI, int cI, int group, int k);
 // K in blocks (kb.rpb > 0; bf16 keys only): rpb must divide the 128-key tile
 // and Nmax.
 cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, QuerySpec qs, int nq, int n_seq, int HI,
                             int cI, int64_t Nmax, int m, float* scores, int64_t ld, int group, bool fill_invisible,
                             int* status, cudaStream_t st, const float* kscale = nullptr,
-                            bool score_bf16 = false, RowBlocks kb = RowBlocks{0, 0});
+                            bool score_bf16 = false, RowBlocks kb = RowBlocks{0, 0}, CandOut co = CandOut{});
 
 // quant.cu: row-wise e4m3 codes out [rows, cols] and fp32 scales
 // s = max|row| / 448 (1 for a zero row), decided in fp64; w_out = w * s when
@@ -199,6 +211,10 @@ cudaError_t topk_select_bf16(const void* scores, int64_t ld, const int32_t* vali
 // as topk_select with the candidate count of row t = (pos_base + t) / m
 cudaError_t topk_select_positions(const float* scores, int64_t ld, int64_t pos_base, int m, int nq,
                                   int64_t ncols, int k, int32_t* idx, void* ws, cudaStream_t st);
+// exact top-k of the candidate lists the indexer's filter wrote (row t:
+// cand[t * ld ...], cnt[t] entries); the same order and padding as topk_select
+cudaError_t topk_from_candidates(const uint64_t* cand, const uint32_t* cnt, int64_t ld, int nq, int k, int32_t* idx,
+                                 float* top_scores, cudaStream_t st);
 
 // mqa_tc.cu: tensor-core shared-KV MQA (bf16); ws holds split partials when nsplit > 1
 bool mqa_tc_supported(int H, int c);

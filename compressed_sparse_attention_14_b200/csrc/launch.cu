@@ -50,7 +50,7 @@ uint32_t debug_flags() { return g_debug_flags.load(std::memory_order_relaxed); }
 }  // namespace csa
 
 extern "C" int csa_debug_set(uint32_t wait_limit, uint32_t flags) {
-    if (flags & ~(uint32_t)CSA_DEBUG_SKIP_FIRST_TILE)
+    if (flags & ~(uint32_t)(CSA_DEBUG_SKIP_FIRST_TILE | CSA_DEBUG_SCORE_BLOCK | CSA_DEBUG_TOPK_FILTER))
         return csa::set_last_error(CSA_ERR_INVALID_ARG, "csa_debug_set: unknown flags 0x%x", flags);
     csa::g_wait_limit.store(wait_limit, std::memory_order_relaxed);
     csa::g_debug_flags.store(flags, std::memory_order_relaxed);

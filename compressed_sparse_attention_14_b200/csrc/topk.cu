@@ -43,17 +43,6 @@
 
 namespace csa {
 
-__device__ __forceinline__ uint32_t orderable(float f) {
-    uint32_t u = __float_as_uint(f);
-    if (u == 0x80000000u) u = 0u;  // -0.0 == +0.0
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-__device__ __forceinline__ float from_orderable(uint32_t k) {
-    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
-}
-__device__ __forceinline__ uint64_t composite(float s, int64_t col) {
-    return ((uint64_t)orderable(s) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)col);
-}
 // One score, widened to fp32 (L2-cached load: each is read once).
 __device__ __forceinline__ float ld_score(const float* p) { return __ldcg(p); }
 __device__ __forceinline__ float ld_score(const bf16* p) {
@@ -651,6 +640,41 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(RowSpec R, int k, int
         select_exact(RowSrc<TS>{srow}, n, k, idx_row, score_row, scratch, sh, bs);   // the estimate missed
 }
 
+// ---------------------------------------------------------------- candidate lists
+// Exact top-k of the lists the indexer's top-k filter wrote (composite keys
+// of distinct columns, in arbitrary order): a list of at most kCap entries is
+// read into shared memory and selected there like a short score row
+// (counting, sorting or radix select); a longer one is selected in place,
+// the radix passes streaming it from global memory.
+struct GmemKeySrc {
+    const uint64_t* e;
+    __device__ __forceinline__ uint64_t operator()(int64_t i) const { return __ldcg(e + i); }
+};
+
+__global__ void __launch_bounds__(kThreads, 2) topk_cand_kernel(const uint64_t* cand, const uint32_t* cnt, int64_t ld,
+                                                                int k, int32_t* idx, float* top) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    uint64_t* c = reinterpret_cast<uint64_t*>(smem_raw);
+    uint64_t* scratch = reinterpret_cast<uint64_t*>(smem_raw + kCandBytes);
+    __shared__ SelShared sh;
+    __shared__ BinShared bs;
+    pdl_wait();
+    pdl_launch_next();
+    const int row = blockIdx.x;
+    const int64_t n = (int64_t)cnt[row] < ld ? (int64_t)cnt[row] : ld;
+    const uint64_t* src = cand + (int64_t)row * ld;
+    int32_t* idx_row = idx + (int64_t)row * k;
+    float* score_row = top ? top + (int64_t)row * k : nullptr;
+    if (n <= kCap) {
+#pragma unroll 4
+        for (int64_t i = threadIdx.x; i < n; i += kThreads) c[i] = __ldcg(src + i);
+        __syncthreads();
+        select_exact(SmemSrc{c}, n, k, idx_row, score_row, scratch, sh, bs);
+    } else {
+        select_exact(GmemKeySrc{src}, n, k, idx_row, score_row, scratch, sh, bs);
+    }
+}
+
 // ---------------------------------------------------------------- host side
 
 size_t topk_workspace_bytes(int nq, int64_t ncols, int k) {
@@ -684,6 +708,20 @@ static cudaError_t topk_run(const RowSpec& R, int nq, int k, int32_t* idx, float
     cudaError_t le = cudaSuccess;
     CSA_LAUNCH(st, "topk_select",
                le = launch_pdl(kern, dim3((unsigned)nq * G), dim3(kThreads), smem, st, (unsigned)G, R, k, idx, top));
+    if (le != cudaSuccess) return le;
+    return cudaGetLastError();
+}
+
+cudaError_t topk_from_candidates(const uint64_t* cand, const uint32_t* cnt, int64_t ld, int nq, int k, int32_t* idx,
+                                 float* top_scores, cudaStream_t st) {
+    if (nq == 0) return cudaSuccess;
+    cudaError_t e = smem_ceiling(topk_cand_kernel);
+    if (e != cudaSuccess) return e;
+    const size_t smem = nq <= sm_count() ? kSmemSpread : kSmemBytes;
+    cudaError_t le = cudaSuccess;
+    CSA_LAUNCH(st, "topk_candidates",
+               le = launch_pdl(topk_cand_kernel, dim3((unsigned)nq), dim3(kThreads), smem, st, 0, cand, cnt, ld, k,
+                               idx, top_scores));
     if (le != cudaSuccess) return le;
     return cudaGetLastError();
 }

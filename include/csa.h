@@ -98,6 +98,19 @@ int csa_poll_status(void* stream, int reset);
  * drains its copies, frees its tensor memory and returns. Process-wide;
  * affects launches made after the call. */
 #define CSA_DEBUG_SKIP_FIRST_TILE 1u
+/* Selection paths of csa_decode, csa_prefill, csa_decode_fp8kv and
+ * csa_attend_decode (bf16, contiguous caches). By default the indexer stores
+ * every score (the fp32 score block) and a top-k kernel selects on it.
+ * CSA_DEBUG_TOPK_FILTER switches to the top-k filter on the indexer's
+ * epilogue: it writes only the scores that can still be among each query's
+ * k best (a running lower bound of the k-th score) and an exact selection
+ * runs over those (for k up to 1024 in the grouped prefill of 64 index
+ * heads, up to 2048 otherwise). Both give the same selection. The filter
+ * cuts the selection's reads but slows the indexer, whose epilogue paces it,
+ * so it is not the default. CSA_DEBUG_SCORE_BLOCK forces the score block
+ * (it wins when both are set). */
+#define CSA_DEBUG_SCORE_BLOCK 2u
+#define CSA_DEBUG_TOPK_FILTER 4u
 int csa_debug_set(uint32_t wait_limit, uint32_t flags);
 
 /* ------------------------------------------------------------------------

@@ -109,7 +109,7 @@ def test_invalid_arguments_are_rejected_on_the_host():
                             fake, None, None, fake * 16, 1 << 30, None) == csa.CSA_ERR_INVALID_ARG
     assert b"flags" in L.csa_last_error()
     assert L.csa_topk_from_scores_bf16(fake, 16, None, 1, 1, 16, 0, fake, None, None) == csa.CSA_ERR_UNSUPPORTED
-    assert L.csa_debug_set(0, 2) == csa.CSA_ERR_INVALID_ARG
+    assert L.csa_debug_set(0, 8) == csa.CSA_ERR_INVALID_ARG
     # prefill with one state ring but not the other
     rc = L.csa_prefill(fake, None, fake, fake, fake, fake, 6, 9, 64, 4, 128, 64, fake, fake, 16, fake, None, fake,
                        fake, fake, 8, 4, 4, 0.0, None, fake, None, None, None, 0, csa.CSA_BF16, None)
