@@ -70,10 +70,15 @@ namespace csa {
 
 namespace {
 
-// warp 0 producer, warp 1 MMA issuer 0 (and TMEM owner), warps 2-9 two
-// epilogue sets of 4, warp 10 MMA issuer 1
-constexpr int kThreads = 352;
+// warp 0 producer, warp 1 MMA issuer 0 (and TMEM owner), then the epilogue
+// sets of 4 warps, then MMA issuer 1. The grouped prefill (N = 256: four
+// queries of 64 heads) has four sets, each reducing one query's 64 columns
+// of every tile, so that four epilogue warps share each SM sub-partition to
+// hide the TMEM-read and arithmetic latency the tile time waits on; every
+// other shape has two sets taking alternate tiles.
 constexpr int kIssuers = 2;
+__host__ __device__ constexpr int epi_warps(int kN) { return kN == 256 ? 16 : 8; }
+__host__ __device__ constexpr int kernel_threads(int kN) { return (epi_warps(kN) + 3) * 32; }
 constexpr int kKeys = 128;      // keys per MMA (M) and per TMA box
 constexpr uint32_t kWaitLimit = 1u << 24;
 
@@ -241,21 +246,22 @@ __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
 }
 
 // The head reduction of one key's accumulator row: sc[q] += sum over the
-// heads h of query q of w[q][h] * max(x[q][h], 0), 64 columns per round (four
-// TMEM loads in flight, one wait), four independent partial sums per 16
-// columns in paired fp32 FMAs (each lane rounds as a separate fmaf would).
+// heads h of query q of w[q][h] * max(x[q][h], 0), kRound columns per round
+// (kRound / 16 TMEM loads in flight, one wait), four independent partial sums
+// per 16 columns in paired fp32 FMAs (each lane rounds as a separate fmaf
+// would).
 // kN > 0: the row has kN columns and each query kHI heads, known at compile
 // time (the loop unrolls and each 16-column block's query is a constant);
 // kN == 0: npad and HI at run time.
-template <int kN, int kHI>
+template <int kN, int kHI, int kRound = 64>
 __device__ __forceinline__ void head_reduce(uint32_t taddr, const float* wv, int npad, int HI, int group,
                                             float (&sc)[4]) {
     const int n = kN > 0 ? kN : npad;
 #pragma unroll(kN > 0 ? 4 : 1)
-    for (int c0 = 0; c0 < n; c0 += 64) {
-        float v[64];
+    for (int c0 = 0; c0 < n; c0 += kRound) {
+        float v[kRound];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kRound / 16; ++u) {
             if (kN > 0 || c0 + 16 * u < n) {
                 float* vv = v + 16 * u;
                 tc::tmem_ld16(taddr + c0 + 16 * u, *reinterpret_cast<float(*)[16]>(vv));
@@ -263,7 +269,7 @@ __device__ __forceinline__ void head_reduce(uint32_t taddr, const float* wv, int
         }
         tc::tmem_ld_wait();
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kRound / 16; ++u) {
             const int cc = c0 + 16 * u;
             if (kN > 0 || cc < n) {
                 uint64_t p01 = 0, p23 = 0;
@@ -405,7 +411,7 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 // that the contiguous path's producer loop stays as it was. kCand: the top-k
 // filter replaces the score stores (bf16, one 128-key half per tile).
 template <bool kFp8, int kN, int kHI, int kH, bool kBlk = false, bool kCand = false>
-__global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __grid_constant__ IdxArgs a,
+__global__ void __launch_bounds__(kernel_threads(kN), 1) index_scores_tc_kernel(const __grid_constant__ IdxArgs a,
                                                                       const __grid_constant__ CUtensorMap tmK,
                                                                       const __grid_constant__ CUtensorMap tmQ) {
     extern __shared__ uint8_t smem_raw[];
@@ -414,7 +420,9 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     // top-k filter: [query of the group][epilogue warp] = (group << 32) | bound
-    __shared__ uint64_t s_pub[4 * 8];
+    constexpr int kEpi = epi_warps(kN);
+    constexpr int kIssuer1 = kEpi + 2;   // warp of MMA issuer 1
+    __shared__ uint64_t s_pub[4 * kEpi];
     static_assert(!kCand || (!kFp8 && kH == 1), "the top-k filter runs on bf16 tiles of 128 keys");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -422,14 +430,14 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < a.stages; ++i) { tc::mbar_init(&sm.full[i], 1); tc::mbar_init(&sm.empty[i], 1); }
-        // prefill (kN == 256): both epilogue sets reduce every tile, so all 8 warps release it
-        for (int i = 0; i < 4; ++i) { tc::mbar_init(&sm.tfull[i], 1); tc::mbar_init(&sm.tempty[i], kN == 256 ? 8 : 4); }
+        // prefill (kN == 256): every epilogue set reduces every tile, so all its warps release it
+        for (int i = 0; i < 4; ++i) { tc::mbar_init(&sm.tfull[i], 1); tc::mbar_init(&sm.tempty[i], kN == 256 ? kEpi : 4); }
         tc::mbar_init(sm.qfull, 1);
         tc::mbar_init(sm.qempty, kIssuers);   // every issuer releases each group's q
         tc::mbar_init(sm.fin, kIssuers);
         tc::fence_mbar_init();
         s_abort = 0;
-        for (int i = 0; i < 4 * 8; ++i) s_pub[i] = (uint64_t)kTagNone << 32;
+        for (int i = 0; i < 4 * kEpi; ++i) s_pub[i] = (uint64_t)kTagNone << 32;
     }
     if (warp == 1) {
         tc::tmem_alloc(&s_tmem, a.tmem_cols);
@@ -501,11 +509,11 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
                 if (!(a.skip_first_tile && j == 0)) tc::mbar_wait(&sm.full[j % a.stages], (j / a.stages) & 1, kWaitLimit);
             if (switches > 0) tc::mbar_wait(sm.qfull, (switches - 1) & 1, kWaitLimit);
         }
-    } else if (warp == 1 || warp == 10) {
+    } else if (warp == 1 || warp == kIssuer1) {
         // ------------------------------------------------------------ MMA issuers
         // issuer mi takes the tiles with it % kIssuers == mi; both walk the
         // whole list, wait for each group's q and release it at the group's end
-        const int mi = warp == 10 ? 1 : 0;
+        const int mi = warp == kIssuer1 ? 1 : 0;
         if (lane == 0 && my > 0) {
             Walk wk;
             wk.start(a, g0, t0);
@@ -565,25 +573,27 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
     } else {
         // ------------------------------------------------------------ epilogue
         // two sets of four warps take alternate tiles (prefill, kN == 256:
-        // both sets take every tile, set s reducing the columns of queries
-        // 2s and 2s+1, which halves the per-tile latency of the epilogue that
-        // paces the two accumulator buffers); within a set, warp w reads TMEM
-        // lane quadrant w % 4
+        // every set takes every tile, set s reducing the kSetCols columns of
+        // its kQS queries, which shortens the per-tile latency of the
+        // epilogue that paces the two accumulator buffers); within a set,
+        // warp w reads TMEM lane quadrant w % 4
         const int set = (warp - 2) >> 2;
         const int quad = warp & 3;
         const int row = quad * 32 + lane;          // key within the tile
-        // each epilogue warp keeps its own copy of the group's head weights, so
+        constexpr int kQS = kN == 256 ? 4 / (kEpi / 4) : 4;   // queries a set reduces per tile (at most)
+        constexpr int kSetCols = kN == 256 ? kN / (kEpi / 4) : 256;
+        // each epilogue warp keeps its own copy of its set's head weights, so
         // that no barrier ties the warps of a set together (a warp that stops
         // on a timeout can never leave the others waiting)
-        float* wv = sm.w + (warp - 2) * 256;
+        float* wv = sm.w + (warp - 2) * (kN == 256 ? kSetCols : 256);
         Walk wk;
         wk.start(a, g0, t0);
         int cur = -1;
         int64_t vis = 0;
         RingPos bf(a.nbuf);
-        // top-k filter: this warp's queries (the grouped prefill: its set's
-        // two; otherwise one) and their queues
-        constexpr int kQ = kN == 256 ? 2 : 1;
+        // top-k filter: this warp's queries (the grouped prefill: its set's;
+        // otherwise one) and their queues
+        constexpr int kQ = kN == 256 ? kQS : 1;
         CandState cst[kQ];
         uint8_t* cslot = sm.cq + (size_t)(warp - 2) * kQ * kCandSlotBytes;
         auto cq_of = [&](int q) { return reinterpret_cast<uint64_t*>(cslot + q * kCandSlotBytes); };
@@ -603,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
         }
         // the row of this warp's query slot gs in group g (nullptr: none)
         auto cand_row = [&](int g, int gs, uint32_t*& cnt) -> uint64_t* {
-            const int gq = kN == 256 ? 2 * set + gs : gs;
+            const int gq = kN == 256 ? kQS * set + gs : gs;
             const int tq = g * a.group + gq;
             if (g < 0 || gq >= a.group || tq >= a.nq) return nullptr;
             cnt = a.cand_cnt + tq;
@@ -613,8 +623,9 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
             if (kN != 256 && (int)(it & 1) != set) continue;
             if (wk.g != cur) {
                 __syncwarp();
-                for (int c = lane; c < a.npad; c += 32) {
-                    const int gq = c / a.HI, h = c % a.HI;
+                const int c0w = kN == 256 ? set * kSetCols : 0;   // first column of this warp's copy
+                for (int c = lane; c < (kN == 256 ? kSetCols : a.npad); c += 32) {
+                    const int gq = (c0w + c) / a.HI, h = (c0w + c) % a.HI;
                     const int tq = wk.g * a.group + gq;
                     wv[c] = (gq < a.group && tq < a.nq) ? a.w[(int64_t)tq * a.HI + h] : 0.f;
                 }
@@ -648,9 +659,9 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
             if (!wait_or_abort(&sm.tfull[buf], bf.phase, abort_flag, a.status, a.wait_limit)) break;
             tc::tc_fence_after();
             // sc[hh][q]: the scores of query q of the group; with kN == 256
-            // this set's two queries (2 set, 2 set + 1) sit in sc[hh][0..1]
-            // (the set is a run-time value: indexing by it would put the
-            // array in local memory)
+            // this set's queries (kQS set + q) sit in sc[hh][0..kQS) (the set
+            // is a run-time value: indexing by it would put the array in
+            // local memory)
             float sc[kH][4];
 #pragma unroll
             for (int hh = 0; hh < kH; ++hh) {
@@ -658,7 +669,9 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
                 const uint32_t taddr =
                     tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)((buf * kH + hh) * a.npad);
                 if constexpr (kN == 256)
-                    head_reduce<128, kHI>(taddr + set * 128, wv + set * 128, a.npad, a.HI, a.group, sc[hh]);
+                    // (the wide layout's warps get fewer registers: 32-column rounds)
+                    head_reduce<kSetCols, kHI, (kEpi > 8 ? 32 : 64)>(taddr + set * kSetCols, wv, a.npad, a.HI,
+                                                                     a.group, sc[hh]);
                 else
                     head_reduce<kN, kHI>(taddr, wv, a.npad, a.HI, a.group, sc[hh]);
             }
@@ -668,7 +681,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
             if constexpr (kCand) {
                 const bool in = key[0] < vis;
                 const int c0 = kN == 256 ? 4 * set : 0;          // warps scoring this warp's queries
-                constexpr int nc = kN == 256 ? 4 : 8;
+                constexpr int nc = kN == 256 ? 4 : kEpi;
 #pragma unroll
                 for (int gs = 0; gs < kQ; ++gs) {
                     uint32_t* cnt = nullptr;
@@ -689,9 +702,9 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
                     // the minimum over the warps scoring the query once all of
                     // them have published for it
                     if ((st.nb & (st.nb - 1)) != 0 && (st.nb & 3) != 0) continue;
-                    const int gq = kN == 256 ? 2 * set + gs : gs;
+                    const int gq = kN == 256 ? kQS * set + gs : gs;
                     const uint32_t p = warp_kth_bound(ctop, a.cand_kk);
-                    volatile uint64_t* slots = s_pub + gq * 8;
+                    volatile uint64_t* slots = s_pub + gq * kEpi;
                     if (lane == 0) slots[warp - 2] = ((uint64_t)(uint32_t)wk.g << 32) | p;
                     __syncwarp();
                     uint32_t lo = 0xFFFFFFFFu;
@@ -710,8 +723,8 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(const __gr
             for (int hh = 0; hh < kH; ++hh) {
                 if (key[hh] >= vis) continue;
 #pragma unroll
-                for (int gs = 0; gs < (kN == 256 ? 2 : 4); ++gs) {
-                    const int gq = kN == 256 ? 2 * set + gs : gs;   // query within the group
+                for (int gs = 0; gs < kQS; ++gs) {
+                    const int gq = kN == 256 ? kQS * set + gs : gs;   // query within the group
                     const int tq = wk.g * a.group + gq;
                     if (gq < a.group && tq < a.nq) {
                         const float v = kFp8 ? sc[hh][gs] * kscale[hh] : sc[hh][gs];
@@ -846,7 +859,8 @@ cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, Query
     while (cols < (uint32_t)(a.nbuf * kh * a.npad)) cols <<= 1;
     a.tmem_cols = cols;
     const size_t fixed = 1024 + a.q_bytes + 8 * 256 * sizeof(float) + 64 * sizeof(uint64_t) +
-                         (cand ? (size_t)8 * (group == 4 ? 2 : 1) * kCandSlotBytes : 0);
+                         (cand ? (size_t)(group == 4 ? epi_warps(256) * (4 / (epi_warps(256) / 4))
+                                                     : epi_warps(0)) * kCandSlotBytes : 0);
     const size_t budget = 226 * 1024;
     int stages = (int)((budget - fixed) / a.stage_bytes);
     if (stages > (fp8 ? 12 : 8)) stages = fp8 ? 12 : 8;
@@ -898,7 +912,9 @@ cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, Query
     e = smem_ceiling(kern);
     if (e != cudaSuccess) return e;
     CSA_LAUNCH(st, fp8 ? "index_scores_tc_fp8" : (cand ? "index_topk_filter_tc" : "index_scores_tc"),
-               e = launch_pdl(kern, dim3(num_sms()), dim3(kThreads), smem, st, 0, a, tmK, tmQ));
+               e = launch_pdl(kern, dim3(num_sms()), dim3(kernel_threads(a.npad == 256 && HI == 64 && group == 4 && !a.key_rpb
+                                                                             ? 256 : 0)),
+                              smem, st, 0, a, tmK, tmQ));
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
