@@ -302,9 +302,17 @@ __device__ void sort_and_write(const uint64_t* src, int cnt, int kk, int k, int3
 // bins; bin order is value order. Exact integer arithmetic, so the smallest
 // key of bin B is kmin + (B << shift).
 constexpr int kBins = 2 * kThreads;     // two per thread in the scans
-constexpr int kBucketMax = 4096;        // candidates placed by counting (the scratch area)
+constexpr int kBucketMax = 4096;        // candidates placed by counting in the smaller scratch area
 constexpr uint32_t kMaxBinLoad = 64;    // larger bins (heavy ties): bitonic path
 static_assert(kScratchBytes >= (size_t)kBucketMax * sizeof(uint64_t), "buckets must fit the scratch area");
+
+// Entries the scratch area holds: the dynamic shared memory past the
+// candidates (a CTA launched with an SM to itself gets a larger one).
+__device__ __forceinline__ int scratch_entries() {
+    uint32_t dyn;
+    asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));
+    return (int)((dyn - (uint32_t)kCandBytes) / sizeof(uint64_t));
+}
 
 struct BinShared {
     uint32_t cnt[kBins];
@@ -373,7 +381,9 @@ __device__ __forceinline__ void bins_clear(BinShared& bs) {
 
 // Threshold estimate from the row's strided sample: the smallest key of the
 // bin that holds the sample's r-th largest score, so that at least r sample
-// scores reach it.
+// scores reach it. (Ranking the samples inside that bin to return the exact
+// r-th key was measured: the bins near the sample's top are narrow, the
+// candidates did not shrink and the two extra barriers cost 0.3 us.)
 template <typename TS>
 __device__ uint32_t sample_threshold(const TS* srow, int64_t n, int r, BinShared& bs) {
     constexpr int kPer = kSample / kThreads;
@@ -455,7 +465,7 @@ __device__ void select_exact(const Src& src, int64_t n, int k, int32_t* idx_row,
                              uint64_t* scratch, SelShared& sh, BinShared& bs) {
     const int kk = (int)(n < k ? n : k);
     if constexpr (std::is_same<Src, SmemSrc>::value) {
-        if (n <= kBucketMax && select_by_bins(src.e, (int)n, k, idx_row, score_row, scratch, bs)) return;
+        if (n <= scratch_entries() && select_by_bins(src.e, (int)n, k, idx_row, score_row, scratch, bs)) return;
         __syncthreads();   // the scratch area may hold buckets
         if (n <= kSortMax) {
             sort_and_write(src.e, (int)n, kk, k, idx_row, score_row, scratch);
@@ -615,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(RowSpec R, int k, int
         // range of CTA 0's candidate array with one remote addition and
         // stores its candidates there over distributed shared memory
         uint64_t* buf = g == 0 ? scratch : cand;
-        const uint32_t cap = g == 0 ? (uint32_t)kBucketMax : (uint32_t)kCap;
+        const uint32_t cap = g == 0 ? (uint32_t)scratch_entries() : (uint32_t)kCap;
         filter_slice<kFilterLoads>(srow, lo, hi, thr, buf, cap, &s_cnt);
         __syncthreads();
         const uint32_t mine = s_cnt;
