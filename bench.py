@@ -845,47 +845,57 @@ WORKLOADS_CONFIG_NAME = {
 
 def pipelined_e2e_ms(pipe, steps: int) -> float:
     """Device time per step of `steps` steps run through the public call from
-    pinned host buffers: inputs of step i+1 go host -> device on a copy stream
-    while step i computes on the current stream; step i's output goes back on
-    the copy stream once it is done. Two device input sets and outputs."""
+    pinned host buffers, as a serving loop runs them: the inputs of step i+1
+    go host -> device on one copy stream while step i computes on the current
+    stream, and step i's output goes device -> host on a second copy stream
+    once it is done (PCIe carries both directions at once, on separate copy
+    engines). Two device input sets and outputs: step i+2 overwrites step i's
+    inputs only after step i has computed, and its output only after that
+    output has been copied out."""
     pinned, run, out0 = pipe["pinned"], pipe["run"], pipe["out"]
     ms = torch.cuda.current_stream()
-    cs = torch.cuda.Stream()
+    hs, ds = torch.cuda.Stream(), torch.cuda.Stream()
     dev = [{k: torch.empty(v.shape, dtype=v.dtype, device="cuda") for k, v in pinned.items()} for _ in range(2)]
     outs = [out0, torch.empty_like(out0)]
     out_h = [torch.empty(out0.shape, dtype=out0.dtype).pin_memory() for _ in range(2)]
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
     def h2d(i):
         b = i % 2
-        with torch.cuda.stream(cs):
+        with torch.cuda.stream(hs):
             if i >= 2:
-                cs.wait_event(ev_comp[b])          # step i-2 no longer reads this buffer
+                hs.wait_event(ev_comp[b])          # step i-2 no longer reads this buffer
             for k, v in pinned.items():
                 dev[b][k].copy_(v, non_blocking=True)
-            ev_in[b].record(cs)
+            ev_in[b].record(hs)
 
     def loop(n):
         h2d(0)
         for i in range(n):
             b = i % 2
             ms.wait_event(ev_in[b])
+            if i >= 2:
+                ms.wait_event(ev_out[b])            # step i-2's output has left this buffer
             run(dev[b], outs[b])
             ev_comp[b].record(ms)
             if i + 1 < n:
                 h2d(i + 1)
-            with torch.cuda.stream(cs):
-                cs.wait_event(ev_comp[b])
+            with torch.cuda.stream(ds):
+                ds.wait_event(ev_comp[b])
                 out_h[b].copy_(outs[b], non_blocking=True)
-        ms.wait_stream(cs)
+                ev_out[b].record(ds)
+        ms.wait_stream(hs)
+        ms.wait_stream(ds)
 
     loop(4)                                          # warm-up
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
     z = torch.cuda.Event(enable_timing=True)
     a.record(ms)
-    cs.wait_event(a)
+    hs.wait_event(a)
+    ds.wait_event(a)
     loop(steps)
     z.record(ms)
     torch.cuda.synchronize()
@@ -962,8 +972,9 @@ def measure(name, args, rank, world, local, steps, warmup, batch=None):
     e2e_ms, e2e_mode = e2e_serial_ms, "serial: copy in, call, copy out, per step"
     if wl.get("pipe"):
         e2e_ms = max_over_ranks(pipelined_e2e_ms(wl["pipe"], steps), world)
-        e2e_mode = ("pipelined: step i+1's host inputs copied on a second stream while step i computes; "
-                    "every step's inputs and result cross PCIe inside the timed region")
+        e2e_mode = ("pipelined: step i+1's host inputs copied in on one copy stream and step i-1's result "
+                    "copied out on another while step i computes; every step's inputs and result cross PCIe "
+                    "inside the timed region")
 
     units = wl["units"]
     peaks = measured_peaks()
