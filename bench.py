@@ -1028,8 +1028,8 @@ def measure(name, args, rank, world, local, steps, warmup, batch=None):
 # 1M-context decode, the long prefill chunk, HCA decode, the HCA compressor).
 # Each keeps its own step count, at most the headline's.
 EXTRA_WORKLOADS = {"pro_decode": 20, "prefill": 5, "hca_decode": 20, "hca_compress": 10, "flash_decode_fp8": 20,
-                   "flash_decode_fp8kv": 20,
-                   "pro_decode_fp8": 20}
+                   "flash_decode_fp8kv": 20, "pro_decode_fp8": 20, "flash_attend_decode": 20,
+                   "flash_decode_compress": 20}
 
 
 def run_ours(args, rank, world, local):

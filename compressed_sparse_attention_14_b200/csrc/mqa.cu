@@ -152,10 +152,13 @@ __global__ void __launch_bounds__(256) mqa_partial_ffma_kernel(MqaPartialArgs a)
 //   out = sum_s e^{m_s - M} O_s / (sum_s e^{m_s - M} l_s + [sink] e^{z' - M})
 // with M the largest of the m_s and the sink logit, and lse = M + log(...).
 // A block takes kCombineHeads heads of one query and kCombineDims of their
-// dims: warp w works out head w's split weights (lanes over the splits), then
-// every thread combines 4 consecutive dims of one head at a time, the 16-byte
-// loads of up to 8 splits issued before their adds (in split order), one
-// store per 4 results.
+// dims; every thread combines 4 consecutive dims of one head on its own: the
+// splits' (m, l) pairs and 16-byte O loads of up to 8 splits are issued
+// together, then weighted in split order (one L2 round trip per 8 splits, no
+// block barrier); with more than 8 splits the running maximum moves from
+// group to group and the sums so far are rescaled (an online merge). A split
+// with m = -inf (it saw no entry) staged no O and gets weight 0 by selection,
+// never by multiplying its stale rows. One store per 4 results.
 constexpr int kCombineHeads = 8;
 constexpr int kCombineDims = 128;
 template <typename T>
@@ -166,65 +169,49 @@ __global__ void __launch_bounds__(kCombineHeads * 32) mqa_combine_kernel(const f
                                                                          T* __restrict__ out, float* __restrict__ lse) {
     pdl_wait();
     pdl_launch_next();
-    __shared__ float s_w[kCombineHeads][64];
-    __shared__ float s_inv[kCombineHeads];
     const int t = blockIdx.y, h0 = blockIdx.x * kCombineHeads;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nh = H - h0 < kCombineHeads ? H - h0 : kCombineHeads;
-    if (warp < nh) {
-        const int h = h0 + warp;
-        const float* ml = part_ml + ((int64_t)t * nsplit * H + h) * 2;
-        float M = sink ? sink[h] : -INFINITY;
-        float mv[2], lv[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int sp = lane + 32 * u;
-            mv[u] = sp < nsplit ? ml[(int64_t)sp * H * 2] : -INFINITY;
-            lv[u] = sp < nsplit ? ml[(int64_t)sp * H * 2 + 1] : 0.f;
-            M = fmaxf(M, mv[u]);
-        }
-        M = warp_max(M);
-        float L = 0.f;
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int sp = lane + 32 * u;
-            const float wgt = (mv[u] == -INFINITY || M == -INFINITY) ? 0.f : expf(mv[u] - M);
-            if (sp < nsplit) s_w[warp][sp] = wgt;
-            L += wgt * lv[u];
-        }
-        L = warp_sum(L);
-        if (lane == 0) {
-            if (sink && M != -INFINITY) L += expf(sink[h] - M);
-            s_inv[warp] = (L > 0.f) ? 1.f / L : 0.f;
-            if (lse && blockIdx.z == 0) lse[(int64_t)t * H + h] = (L > 0.f) ? M + logf(L) : -INFINITY;
-        }
-    }
-    __syncthreads();
     const int d0 = blockIdx.z * kCombineDims;
     const int c4 = (c - d0 < kCombineDims ? c - d0 : kCombineDims) / 4;
     const int64_t sstride = (int64_t)H * c;   // one split to the next
     for (int e = threadIdx.x; e < nh * c4; e += blockDim.x) {
-        const int i = e / c4, d = d0 + (e - i * c4) * 4;
-        const float* po = part_o + ((int64_t)t * nsplit * H + h0 + i) * c + d;
+        const int i = e / c4, j4 = e - i * c4, d = d0 + j4 * 4;
+        const int h = h0 + i;
+        const float* po = part_o + ((int64_t)t * nsplit * H + h) * c + d;
+        const float* ml = part_ml + ((int64_t)t * nsplit * H + h) * 2;
+        const float z = sink ? __ldg(sink + h) : -INFINITY;
+        float M = z, L = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int s0 = 0; s0 < nsplit; s0 += 8) {
+            float mv[8], lv[8];
             float4 v[8];
-            float wv[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                wv[u] = s0 + u < nsplit ? s_w[i][s0 + u] : 0.f;
-                // a split with weight 0 staged no O (its rows may be stale)
-                v[u] = wv[u] != 0.f ? *reinterpret_cast<const float4*>(po + (s0 + u) * sstride)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                const bool in = s0 + u < nsplit;
+                mv[u] = in ? ml[(int64_t)(s0 + u) * H * 2] : -INFINITY;
+                lv[u] = in ? ml[(int64_t)(s0 + u) * H * 2 + 1] : 0.f;
+                v[u] = in ? *reinterpret_cast<const float4*>(po + (s0 + u) * sstride) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
+            float Mn = M;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) Mn = fmaxf(Mn, mv[u]);
+            if (Mn == -INFINITY) continue;                 // nothing seen yet
+            const float r = M == -INFINITY ? 0.f : expf(M - Mn);
+            L *= r;
+            acc.x *= r; acc.y *= r; acc.z *= r; acc.w *= r;
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                if (wv[u] == 0.f) continue;
-                acc.x += wv[u] * v[u].x; acc.y += wv[u] * v[u].y; acc.z += wv[u] * v[u].z; acc.w += wv[u] * v[u].w;
+                if (mv[u] == -INFINITY) continue;
+                const float wgt = expf(mv[u] - Mn);
+                L += wgt * lv[u];
+                acc.x += wgt * v[u].x; acc.y += wgt * v[u].y; acc.z += wgt * v[u].z; acc.w += wgt * v[u].w;
             }
+            M = Mn;
         }
-        const float inv = s_inv[i];
-        store4(out + ((int64_t)t * H + h0 + i) * c + d, acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        if (sink && M != -INFINITY) L += expf(z - M);
+        const float inv = (L > 0.f) ? 1.f / L : 0.f;
+        store4(out + ((int64_t)t * H + h) * c + d, acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        if (lse && blockIdx.z == 0 && j4 == 0) lse[(int64_t)t * H + h] = (L > 0.f) ? M + logf(L) : -INFINITY;
     }
 }
 
