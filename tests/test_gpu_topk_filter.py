@@ -158,3 +158,32 @@ def _kv_after(inp, s):
     kv[s.start // s.m:(s.start + s.n) // s.m] = oracle.bf16_round(
         oracle.csa_compress_from_hidden(inp["x"], inp["W_kv"], inp["B_kv"], s.m, X_left=inp["x_left"]))
     return kv
+
+
+def test_attend_and_fp8kv_decode_filter_equals_score_block(csa):
+    # the complete-output decode and the FP8-KV decode select through the same
+    # step: the filter gives them the same entries and the same bits
+    B, Nmax, HI, cI, H, c, k, n_win = 5, 3000, 64, 128, 8, 128, 512, 128
+    inp = _decode_inputs(B, Nmax, HI, cI, H, c, [12000, 4 * 2200 + 1, 4 * 700, 4 * 1999, 11000], seed=34)
+    ring = synth.normal((B, n_win, c), 34, "f_ring")
+    dev = {kk: v.to(DEV) for kk, v in inp.items()}
+    kv_ext = torch.cat([inp["kv_cache"], ring], dim=1).contiguous().to(DEV)
+    gamma = (1.0 + synth.normal((c,), 34, "f_gamma", std=0.1, dtype=torch.float32)).to(DEV)
+    sink = synth.normal((H,), 34, "f_sink", dtype=torch.float32).to(DEV)
+
+    def attend():
+        return csa.csa_attend_decode(dev["qI"], dev["w"], dev["idx_cache"], dev["q"], kv_ext, dev["ctx_len"], 4, k,
+                                     n_win=n_win, ring_len=n_win, q_gamma=gamma, rope_dims=64, sink=sink,
+                                     return_topk=True)
+
+    (o1, l1, s1), (o2, l2, s2) = _both_paths(csa, attend)
+    assert torch.equal(s1, s2) and torch.equal(o1, o2) and torch.equal(l1, l2)
+
+    codes, scales, rope = csa.csa_quantize_kv_fp8(dev["kv_cache"], rope_dims=64)
+
+    def fp8kv():
+        return csa.csa_decode_fp8kv(dev["qI"], dev["w"], dev["idx_cache"], dev["q"], codes, scales, rope,
+                                    dev["ctx_len"], 4, k, return_topk=True)
+
+    (o1, l1, s1), (o2, l2, s2) = _both_paths(csa, fp8kv)
+    assert torch.equal(s1, s2) and torch.equal(o1, o2) and torch.equal(l1, l2)
