@@ -73,12 +73,14 @@ namespace {
 // warp 0 producer, warp 1 MMA issuer 0 (and TMEM owner), then the epilogue
 // sets of 4 warps, then MMA issuer 1. The grouped prefill (N = 256: four
 // queries of 64 heads) has four sets, each reducing one query's 64 columns
-// of every tile, so that four epilogue warps share each SM sub-partition to
-// hide the TMEM-read and arithmetic latency the tile time waits on; every
-// other shape has two sets taking alternate tiles.
+// of every tile, and the FP8 decode (256-key tiles: twice the epilogue work
+// per byte) four sets taking every fourth tile, so that four epilogue warps
+// share each SM sub-partition to hide the TMEM-read and arithmetic latency
+// the tile time waits on; every other shape has two sets taking alternate
+// tiles.
 constexpr int kIssuers = 2;
-__host__ __device__ constexpr int epi_warps(int kN) { return kN == 256 ? 16 : 8; }
-__host__ __device__ constexpr int kernel_threads(int kN) { return (epi_warps(kN) + 3) * 32; }
+__host__ __device__ constexpr int epi_warps(int kN, int kH = 1) { return (kN == 256 || (kN == 64 && kH == 2)) ? 16 : 8; }
+__host__ __device__ constexpr int kernel_threads(int kN, int kH = 1) { return (epi_warps(kN, kH) + 3) * 32; }
 constexpr int kKeys = 128;      // keys per MMA (M) and per TMA box
 constexpr uint32_t kWaitLimit = 1u << 24;
 
@@ -411,7 +413,7 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 // that the contiguous path's producer loop stays as it was. kCand: the top-k
 // filter replaces the score stores (bf16, one 128-key half per tile).
 template <bool kFp8, int kN, int kHI, int kH, bool kBlk = false, bool kCand = false>
-__global__ void __launch_bounds__(kernel_threads(kN), 1) index_scores_tc_kernel(const __grid_constant__ IdxArgs a,
+__global__ void __launch_bounds__(kernel_threads(kN, kH), 1) index_scores_tc_kernel(const __grid_constant__ IdxArgs a,
                                                                       const __grid_constant__ CUtensorMap tmK,
                                                                       const __grid_constant__ CUtensorMap tmQ) {
     extern __shared__ uint8_t smem_raw[];
@@ -420,7 +422,7 @@ __global__ void __launch_bounds__(kernel_threads(kN), 1) index_scores_tc_kernel(
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     // top-k filter: [query of the group][epilogue warp] = (group << 32) | bound
-    constexpr int kEpi = epi_warps(kN);
+    constexpr int kEpi = epi_warps(kN, kH);
     constexpr int kIssuer1 = kEpi + 2;   // warp of MMA issuer 1
     __shared__ uint64_t s_pub[4 * kEpi];
     static_assert(!kCand || (!kFp8 && kH == 1), "the top-k filter runs on bf16 tiles of 128 keys");
@@ -582,10 +584,11 @@ __global__ void __launch_bounds__(kernel_threads(kN), 1) index_scores_tc_kernel(
         const int row = quad * 32 + lane;          // key within the tile
         constexpr int kQS = kN == 256 ? 4 / (kEpi / 4) : 4;   // queries a set reduces per tile (at most)
         constexpr int kSetCols = kN == 256 ? kN / (kEpi / 4) : 256;
+        constexpr int kSets = kEpi / 4;                        // sets taking turns (kN != 256)
         // each epilogue warp keeps its own copy of its set's head weights, so
         // that no barrier ties the warps of a set together (a warp that stops
         // on a timeout can never leave the others waiting)
-        float* wv = sm.w + (warp - 2) * (kN == 256 ? kSetCols : 256);
+        float* wv = sm.w + (warp - 2) * (kN == 256 ? kSetCols : (kEpi > 8 ? 64 : 256));
         Walk wk;
         wk.start(a, g0, t0);
         int cur = -1;
@@ -620,7 +623,7 @@ __global__ void __launch_bounds__(kernel_threads(kN), 1) index_scores_tc_kernel(
             return a.cand + (int64_t)tq * a.cand_ld;
         };
         for (int64_t it = 0; it < my; ++it, wk.next(a, ngroups), bf.advance()) {
-            if (kN != 256 && (int)(it & 1) != set) continue;
+            if (kN != 256 && (int)(it & (kSets - 1)) != set) continue;
             if (wk.g != cur) {
                 __syncwarp();
                 const int c0w = kN == 256 ? set * kSetCols : 0;   // first column of this warp's copy
@@ -673,7 +676,7 @@ __global__ void __launch_bounds__(kernel_threads(kN), 1) index_scores_tc_kernel(
                     head_reduce<kSetCols, kHI, (kEpi > 8 ? 32 : 64)>(taddr + set * kSetCols, wv, a.npad, a.HI,
                                                                      a.group, sc[hh]);
                 else
-                    head_reduce<kN, kHI>(taddr, wv, a.npad, a.HI, a.group, sc[hh]);
+                    head_reduce<kN, kHI, (kEpi > 8 ? 32 : 64)>(taddr, wv, a.npad, a.HI, a.group, sc[hh]);
             }
             tc::tc_fence_before();
             __syncwarp();
@@ -909,12 +912,14 @@ cudaError_t index_scores_tc(const void* qI, const float* w, const void* K, Query
         else if (a.npad == 256 && HI == 64 && group == 4) kern = index_scores_tc_kernel<false, 256, 64, 1, false, true>;
         else kern = index_scores_tc_kernel<false, 0, 0, 1, false, true>;
     }
+    // the block size of the instantiation chosen above
+    int threads = kernel_threads(0);
+    if (!a.key_rpb && a.npad == 256 && HI == 64 && group == 4) threads = kernel_threads(256);
+    else if (fp8 && a.npad == 64 && HI == 64 && group == 1) threads = kernel_threads(64, kh);
     e = smem_ceiling(kern);
     if (e != cudaSuccess) return e;
     CSA_LAUNCH(st, fp8 ? "index_scores_tc_fp8" : (cand ? "index_topk_filter_tc" : "index_scores_tc"),
-               e = launch_pdl(kern, dim3(num_sms()), dim3(kernel_threads(a.npad == 256 && HI == 64 && group == 4 && !a.key_rpb
-                                                                             ? 256 : 0)),
-                              smem, st, 0, a, tmK, tmQ));
+               e = launch_pdl(kern, dim3(num_sms()), dim3(threads), smem, st, 0, a, tmK, tmQ));
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
