@@ -691,8 +691,16 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
             bar_sync_128();
             // the normalised O goes through shared memory (the KV area,
             // [head][dim] bf16) so that the output rows leave in 16-byte
-            // stores: a thread holds one dim of every head, and 2-byte
-            // stores at a head stride are slow
+            // stores (a thread holds one dim of every head). The heads'
+            // factors are read into registers once (0 for a head without
+            // entries): with them read from shared memory inside the staging
+            // loop, every load waited behind the staging stores before it
+            // and the loop took 15 us per query; storing each head's row
+            // straight from registers (64 contiguous bytes per warp store)
+            // measured 8.7 us, this 7.4 us.
+            float al[64];
+#pragma unroll
+            for (int i = 0; i < 64; ++i) al[i] = (have_o && mref_s[i] != -INFINITY) ? alpha_s[i] : 0.f;
             bf16* stage = reinterpret_cast<bf16*>(kv_s);
             for (int mt = 0; mt < a.mtiles; ++mt) {
                 const int dim = mt * 128 + row;
@@ -705,10 +713,8 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
                     tc::tmem_ld_wait();
                 }
 #pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    const float o = (have_o && mref_s[i] != -INFINITY) ? v[i] * alpha_s[i] : 0.f;
-                    stage[i * a.c + dim] = __float2bfloat16_rn(o);
-                }
+                for (int i = 0; i < 64; ++i)
+                    stage[i * a.c + dim] = __float2bfloat16_rn(al[i] != 0.f ? v[i] * al[i] : 0.f);
             }
             bar_sync_128();
             const int nh = a.H - h0 < 64 ? a.H - h0 : 64;
