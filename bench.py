@@ -449,7 +449,8 @@ def decode_compress_workload(rank, batch=None):
     h2d = sum(v.numel() * v.element_size() for v in pinned.values())
     kernels = {
         # two launches per step (KV: M = 4c, index keys: M = 4cI); work per step
-        "project_tc": dict(bound="hbm", work=w_bytes + 2 * B * d * 2 + proj_bytes, files=("gemm_tc.cu", "tc.cuh")),
+        "project_tc": dict(bound="hbm", work=w_bytes + 2 * B * d * 2 + proj_bytes,
+                           files=("gemm_tc.cu", "tc.cuh", "common.cuh")),
         "csa_compress_step": dict(bound="hbm", work=2 * proj_bytes, files=("compress.cu",)),
     }
     d2h = flag_h.numel() * flag_h.element_size()
