@@ -23,6 +23,19 @@ namespace csa {
 
 namespace {
 
+// 4 consecutive values as fp32 (an 8-byte bf16 load or a 16-byte fp32 one).
+__device__ __forceinline__ void load4(const bf16* p, float (&v)[4]) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    v[0] = __uint_as_float(u.x << 16);
+    v[1] = __uint_as_float(u.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(u.y << 16);
+    v[3] = __uint_as_float(u.y & 0xFFFF0000u);
+}
+__device__ __forceinline__ void load4(const float* p, float (&v)[4]) {
+    const float4 f = *reinterpret_cast<const float4*>(p);
+    v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+}
+
 // The e4m3 code of the value nearest to v (|v| <= 448 assumed after the
 // saturation test), written from the format's definition.
 __device__ __forceinline__ uint8_t e4m3_code(double v) {
@@ -30,10 +43,14 @@ __device__ __forceinline__ uint8_t e4m3_code(double v) {
     const double a = fabs(v);
     if (!(a > 0.0)) return (uint8_t)sign;                 // zero (NaN never reaches here)
     if (a >= 448.0) return (uint8_t)(sign | 0x7Eu);       // saturate: 1.75 * 2^8
-    int e = ilogb(a);                                     // a in [2^e, 2^(e+1))
+    // a in [2^e, 2^(e+1)), read from the exponent field: a is a normal double
+    // (a quotient of fp32 / bf16 values by their row's max / 448)
+    const int e = (int)((__double_as_longlong(a) >> 52) & 0x7ff) - 1023;
     int q = e - 3;                                        // spacing of 4 significant bits
     if (q < -9) q = -9;                                   // subnormal spacing
-    double r = rint(ldexp(a, -q));                        // nearest, ties to even
+    // a * 2^-q is exact (a power-of-two scale within range); then nearest,
+    // ties to even
+    double r = rint(a * __longlong_as_double((long long)(1023 - q) << 52));
     uint32_t code;
     if (q == -9 && r < 8.0) {
         code = (uint32_t)r;                               // subnormal (or zero)
@@ -64,25 +81,24 @@ __global__ void __launch_bounds__(256) quantize_e4m3_kernel(const TIn* __restric
     const int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
     if (r >= rows) return;
     const TIn* row = x + r * ld;
-    double amax = 0.0;
-    for (int j = lane * 8; j < cols; j += 256) {
-        float v[8];
-        load8(row + j, v);
+    // 4 values per lane per step, so that a row of 128 keeps all 32 lanes busy
+    float amax = 0.f;
+    for (int j = lane * 4; j < cols; j += 128) {
+        float v[4];
+        load4(row + j, v);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) amax = fmax(amax, (double)fabsf(v[u]));
+        for (int u = 0; u < 4; ++u) amax = fmaxf(amax, fabsf(v[u]));
     }
+    // non-negative floats order like their bits
+    amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax)));
+    const double s = amax > 0.f ? (double)amax / 448.0 : 1.0;
+    for (int j = lane * 4; j < cols; j += 128) {
+        float v[4];
+        load4(row + j, v);
+        uint32_t c4 = 0;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmax(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const double s = amax > 0.0 ? amax / 448.0 : 1.0;
-    for (int j = lane * 8; j < cols; j += 256) {
-        float v[8];
-        load8(row + j, v);
-        uint32_t lo = 0, hi = 0;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) lo |= (uint32_t)e4m3_code((double)v[u] / s) << (8 * u);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) hi |= (uint32_t)e4m3_code((double)v[4 + u] / s) << (8 * u);
-        *reinterpret_cast<uint2*>(out + r * cols + j) = make_uint2(lo, hi);
+        for (int u = 0; u < 4; ++u) c4 |= (uint32_t)e4m3_code((double)v[u] / s) << (8 * u);
+        *reinterpret_cast<uint32_t*>(out + r * cols + j) = c4;
     }
     if (lane == 0) {
         scale[r] = (float)s;
