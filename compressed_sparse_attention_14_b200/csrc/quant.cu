@@ -15,7 +15,7 @@
 //
 // e4m3: sign, 4 exponent bits (bias 7), 3 mantissa bits. Normal values
 // 2^-6 .. 448 (exponent field 1..15; the code 0x7F is NaN), subnormals in
-// steps of 2^-9 (exponent field 0). One warp per row, 16-byte loads.
+// steps of 2^-9 (exponent field 0). One warp per row, four values per lane.
 #include "common.cuh"
 #include "kernels.h"
 
