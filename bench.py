@@ -454,7 +454,10 @@ def decode_compress_workload(rank, batch=None):
         "csa_compress_step": dict(bound="hbm", work=2 * proj_bytes, files=("compress.cu",)),
     }
     d2h = flag_h.numel() * flag_h.element_size()
-    return dict(step=step, e2e_step=e2e_step, units=B, unit="tokens/s", h2d=h2d, d2h=d2h,
+    # pipelined: the step's result read back is the same cache element
+    flag_d = inp["kv_cache"].view(-1)[:1]
+    pipe = dict(pinned=pinned, out=flag_d, outs=[flag_d, flag_d], run=lambda dd, o: call(dd["x"], dd["pos"]))
+    return dict(step=step, e2e_step=e2e_step, pipe=pipe, units=B, unit="tokens/s", h2d=h2d, d2h=d2h,
                 kernels=kernels, step_bytes=step_bytes,
                 config=dict(workload=COMPRESS_STEP_NAME, batch=B, d=d, m=m, head_dim=c, index_dim=cI,
                             positions=f"U[{s.ctx_lo},{s.ctx_hi}]", blocks_closed_per_step=closing,
@@ -939,7 +942,7 @@ def pipelined_e2e_ms(pipe, steps: int, graphs: bool = False) -> float:
     dev_all = [torch.empty(nbytes, dtype=torch.uint8, device="cuda") for _ in range(2)]
     dev = [{k: dev_all[b][offs[k]:offs[k] + v.numel() * v.element_size()].view(v.dtype).view(v.shape)
             for k, v in pinned.items()} for b in range(2)]
-    outs = [out0, torch.empty_like(out0)]
+    outs = pipe.get("outs") or [out0, torch.empty_like(out0)]
     out_h = [torch.empty(out0.shape, dtype=out0.dtype).pin_memory() for _ in range(2)]
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_comp = [torch.cuda.Event() for _ in range(2)]
